@@ -1,0 +1,196 @@
+"""CPU oracle for tree speculative decoding verification -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  It never imports the CUDA package and
+the CUDA package never imports it; both read their inputs from the seeded
+generator in ``workloads``.
+
+The arithmetic lives in ``tsd_oracle.c`` (plain C, fp64, one loop per step
+of each definition); this module only marshals arguments through ctypes and
+allocates outputs.  Every output array is pre-filled with a sentinel so that
+callers can check which entries a function leaves untouched.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+from typing import Dict, Optional, Sequence
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "tsd_oracle.c")
+_LIB_DIR = os.path.join(_HERE, "_build")
+_LIB = os.path.join(_LIB_DIR, "libtsd_oracle.so")
+_lock = threading.Lock()
+_lib: Optional[ctypes.CDLL] = None
+
+SENTINEL = -7
+BAD_TREE, BAD_TOKEN, BAD_QROW = 1, 2, 4
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (IEEE semantics: no fast-math, no FMA
+    contraction) into ``oracle/_build/libtsd_oracle.so``."""
+    os.makedirs(_LIB_DIR, exist_ok=True)
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off",
+                               "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load() -> ctypes.CDLL:
+    global _lib
+    with _lock:
+        if _lib is None:
+            _lib = ctypes.CDLL(build())
+            _lib.oracle_num_threads.restype = ctypes.c_int
+        return _lib
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def _np(t, dtype=None) -> np.ndarray:
+    """Contiguous numpy view of a CPU tensor/array (bf16 as raw uint16 bits)."""
+    if isinstance(t, torch.Tensor):
+        t = t.detach().cpu().contiguous()
+        if t.dtype == torch.bfloat16:
+            return t.view(torch.int16).numpy().view(np.uint16)
+        a = t.numpy()
+    else:
+        a = np.ascontiguousarray(t)
+    if dtype is not None:
+        a = np.ascontiguousarray(a, dtype=dtype)
+    return a
+
+
+def _p(a: np.ndarray) -> ctypes.c_void_p:
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def _dtype_code(t) -> int:
+    if isinstance(t, torch.Tensor):
+        if t.dtype == torch.float32:
+            return 0
+        if t.dtype == torch.bfloat16:
+            return 1
+    elif isinstance(t, np.ndarray) and t.dtype == np.float32:
+        return 0
+    raise TypeError("oracle attention inputs must be float32 or bfloat16")
+
+
+def tree_mask(parent, n_nodes, Tmax: int) -> Dict[str, np.ndarray]:
+    """Ancestor-or-self bitmask [B][Tmax][ceil(Tmax/32)] u32, depth (path
+    length), first_child [B][Tmax+1] (slot 0 = root), next_sibling, status."""
+    lib = _load()
+    par = _np(parent, np.int32)
+    nn = _np(n_nodes, np.int32)
+    B = nn.shape[0]
+    W = (Tmax + 31) // 32
+    mask = np.zeros((B, Tmax, W), dtype=np.uint32)
+    depth = np.zeros((B, Tmax), dtype=np.int32)
+    fc = np.zeros((B, Tmax + 1), dtype=np.int32)
+    ns = np.zeros((B, Tmax), dtype=np.int32)
+    st = np.zeros(B, dtype=np.int32)
+    lib.oracle_tree_mask(_p(par), _p(nn), B, Tmax, _p(mask), _p(depth), _p(fc), _p(ns), _p(st))
+    return dict(mask=mask, depth=depth, first_child=fc, next_sibling=ns, status=st)
+
+
+def tree_attention(q, k_cache, v_cache, prefix_len, n_nodes, parent, scale: float) -> np.ndarray:
+    """All rows: float64 [B][Tmax][Hq][D]; padding rows are NaN."""
+    lib = _load()
+    dt = _dtype_code(q)
+    qa, ka, va = _np(q), _np(k_cache), _np(v_cache)
+    B, Tmax, Hq, D = qa.shape
+    Hkv, Lmax = ka.shape[1], ka.shape[2]
+    pl = _np(prefix_len, np.int32)
+    nn = _np(n_nodes, np.int32)
+    par = _np(parent, np.int32)
+    out = np.full((B, Tmax, Hq, D), np.nan, dtype=np.float64)
+    rc = lib.oracle_tree_attention(_p(qa), _p(ka), _p(va), dt, _p(pl), _p(nn), _p(par), B, Tmax,
+                                   Hq, Hkv, D, Lmax, ctypes.c_double(scale), _p(out))
+    if rc:
+        raise ValueError(f"oracle_tree_attention: malformed input (status {rc})")
+    return out
+
+
+def tree_attention_rows(q, k_cache, v_cache, prefix_len, n_nodes, parent, scale: float,
+                        rows: Sequence[Sequence[int]]) -> np.ndarray:
+    """Selected rows (b, u, h) -> float64 [len(rows)][D]."""
+    lib = _load()
+    dt = _dtype_code(q)
+    qa, ka, va = _np(q), _np(k_cache), _np(v_cache)
+    B, Tmax, Hq, D = qa.shape
+    Hkv, Lmax = ka.shape[1], ka.shape[2]
+    pl, nn, par = _np(prefix_len, np.int32), _np(n_nodes, np.int32), _np(parent, np.int32)
+    sel = np.ascontiguousarray(np.asarray(rows, dtype=np.int32).reshape(-1, 3))
+    out = np.full((sel.shape[0], D), np.nan, dtype=np.float64)
+    rc = lib.oracle_tree_attention_rows(_p(qa), _p(ka), _p(va), dt, _p(pl), _p(nn), _p(par),
+                                        B, Tmax, Hq, Hkv, D, Lmax, ctypes.c_double(scale),
+                                        sel.shape[0], _p(sel), _p(out))
+    if rc:
+        raise ValueError(f"oracle_tree_attention_rows: malformed input (status {rc})")
+    return out
+
+
+def verify_greedy(logits, tokens, parent, n_nodes) -> Dict[str, np.ndarray]:
+    lib = _load()
+    lg = _np(logits, np.float32)
+    B, R, V = lg.shape
+    Tmax = R - 1
+    tk, par, nn = _np(tokens, np.int32), _np(parent, np.int32), _np(n_nodes, np.int32)
+    out_tokens = np.full((B, Tmax + 1), SENTINEL, dtype=np.int32)
+    out_path = np.full((B, Tmax), SENTINEL, dtype=np.int32)
+    n_acc = np.full(B, SENTINEL, dtype=np.int32)
+    st = np.zeros(B, dtype=np.int32)
+    lib.oracle_verify_greedy(_p(lg), _p(tk), _p(par), _p(nn), B, Tmax, V, _p(out_tokens),
+                             _p(out_path), _p(n_acc), _p(st))
+    return dict(out_tokens=out_tokens, out_path=out_path, n_accepted=n_acc, status=st)
+
+
+def verify_stochastic(logits, temperature: float, q_probs, q_row, tokens, parent, n_nodes,
+                      u_accept, u_sample) -> Dict[str, np.ndarray]:
+    lib = _load()
+    lg = _np(logits, np.float32)
+    B, R, V = lg.shape
+    Tmax = R - 1
+    qp = _np(q_probs, np.float32)
+    Rq = qp.shape[1]
+    qr, tk = _np(q_row, np.int32), _np(tokens, np.int32)
+    par, nn = _np(parent, np.int32), _np(n_nodes, np.int32)
+    ua, us = _np(u_accept, np.float64), _np(u_sample, np.float64)
+    out_tokens = np.full((B, Tmax + 1), SENTINEL, dtype=np.int32)
+    out_path = np.full((B, Tmax), SENTINEL, dtype=np.int32)
+    n_acc = np.full(B, SENTINEL, dtype=np.int32)
+    nflag = np.zeros(B, dtype=np.int32)
+    ndec = np.zeros(B, dtype=np.int32)
+    st = np.zeros(B, dtype=np.int32)
+    lib.oracle_verify_stochastic(_p(lg), ctypes.c_double(temperature), _p(qp), _p(qr), Rq,
+                                 _p(tk), _p(par), _p(nn), _p(ua), _p(us), B, Tmax, V,
+                                 _p(out_tokens), _p(out_path), _p(n_acc), _p(nflag), _p(ndec),
+                                 _p(st))
+    return dict(out_tokens=out_tokens, out_path=out_path, n_accepted=n_acc, n_flagged=nflag,
+                n_decisions=ndec, status=st)
+
+
+# Convenience wrappers over a workloads.Workload -----------------------------
+
+def workload_attention(w) -> np.ndarray:
+    return tree_attention(w.q, w.k_cache, w.v_cache, w.prefix_len, w.n_nodes, w.parent, w.scale)
+
+
+def workload_greedy(w) -> Dict[str, np.ndarray]:
+    return verify_greedy(w.logits, w.tokens, w.parent, w.n_nodes)
+
+
+def workload_stochastic(w) -> Dict[str, np.ndarray]:
+    return verify_stochastic(w.logits, w.temperature, w.q_probs, w.q_row, w.tokens, w.parent,
+                             w.n_nodes, w.u_accept, w.u_sample)
