@@ -1,0 +1,434 @@
+"""Benchmark of the tree speculative decoding verification hot path.
+
+One step = one pass of the whole path over one batch of synthetic input:
+ancestor-mask build, tree attention (one attention layer), and tree
+verification (greedy and/or stochastic, as the workload states).  The metric
+is verified tree tokens/s = sum_b n_nodes[b] / step time, whole-job over all
+ranks (each rank verifies its own batch: weak scaling, no collective on the
+data path).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Workloads: tiny, llama7b, merge, gqa70b (default), long32k.
+
+Prints ONE JSON line (rank 0).  `--impl reference` times the CPU oracle on a
+bounded sample of the same workload instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from workloads import gen  # noqa: E402
+
+METRIC = "verified tree tokens/s (attn+verify) and KV-cache GB/s as % of B200 HBM peak"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "gqa70b"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ----------------------------------------------------------------- work
+def attn_flops(w) -> int:
+    """4*D flops per (query row, attended key): prefix + ancestors-or-self."""
+    total = 0
+    for b in range(w.B):
+        T, P = int(w.n_nodes[b]), int(w.prefix_len[b])
+        par = w.parent[b, :T].tolist()
+        depth = []
+        for u in range(T):
+            depth.append(1 if par[u] < 0 else depth[par[u]] + 1)
+        total += w.Hq * sum(P + d for d in depth) * 4 * w.D
+    return total
+
+
+def attn_bytes(w) -> int:
+    """K+V of the attended positions, once per (b, KV head), + Q read + O write."""
+    es = 4 if w.dtype == "f32" else 2
+    qo = 2 * int(w.n_nodes.sum()) * w.Hq * w.D * es
+    return w.kv_bytes() + qo
+
+
+def verify_bytes(w) -> int:
+    """Logits rows of the internal nodes (+ the root) once, plus the q rows read
+    by the first acceptance pass; a lower bound used for the report only."""
+    rows = 0
+    for b in range(w.B):
+        T = int(w.n_nodes[b])
+        par = set(w.parent[b, :T].tolist())
+        rows += len(par)   # includes -1 (root) when T > 0
+    return rows * w.V * 4
+
+
+class Step:
+    """Device buffers + one call sequence of the public API."""
+
+    def __init__(self, w, dev, tsd):
+        self.w, self.dev, self.tsd = w, dev, tsd
+        self.d = {f: getattr(w, f).to(dev) for f in
+                  ("parent", "n_nodes", "prefix_len", "tokens", "q_row", "q", "k_cache",
+                   "v_cache", "logits", "q_probs", "u_accept", "u_sample")}
+        d = self.d
+        self.tree = tsd.tree_mask_build(d["parent"], d["n_nodes"])
+        self.out = torch.empty_like(d["q"])
+        B, Tmax = w.B, w.Tmax
+        self.g = tsd.VerifyResult(torch.empty((B, Tmax + 1), dtype=torch.int32, device=dev),
+                                  torch.empty((B, Tmax), dtype=torch.int32, device=dev),
+                                  torch.empty((B,), dtype=torch.int32, device=dev))
+        self.s = tsd.VerifyResult(torch.empty((B, Tmax + 1), dtype=torch.int32, device=dev),
+                                  torch.empty((B, Tmax), dtype=torch.int32, device=dev),
+                                  torch.empty((B,), dtype=torch.int32, device=dev))
+        self.ws_attn = torch.empty(max(256, tsd.attention_workspace_size(
+            B, Tmax, w.Hq, w.Hkv, w.D, w.Lmax, d["q"].dtype)), dtype=torch.uint8, device=dev)
+        self.ws_ver = torch.empty(max(256, tsd.verify_workspace_size(B, Tmax, w.V)),
+                                  dtype=torch.uint8, device=dev)
+        self.ev = None
+
+    def run(self, attn_events=None):
+        w, d, tsd = self.w, self.d, self.tsd
+        tsd.tree_mask_build(d["parent"], d["n_nodes"], out=self.tree)
+        if attn_events is not None:
+            attn_events[0].record()
+        tsd.tree_attention(d["q"], d["k_cache"], d["v_cache"], d["prefix_len"], d["n_nodes"],
+                           self.tree.mask, out=self.out, workspace=self.ws_attn)
+        if attn_events is not None:
+            attn_events[1].record()
+        if "greedy" in w.verify:
+            tsd.tree_verify_greedy(d["logits"], d["tokens"], d["parent"], d["n_nodes"],
+                                   self.tree, out=self.g, workspace=self.ws_ver)
+        if "stochastic" in w.verify:
+            tsd.tree_verify_stochastic(d["logits"], w.temperature, d["q_probs"], d["q_row"],
+                                       d["tokens"], d["n_nodes"], self.tree, d["u_accept"],
+                                       d["u_sample"], out=self.s, workspace=self.ws_ver)
+
+
+def _clock_sampler(index):
+    try:
+        return subprocess.Popen(
+            ["nvidia-smi", f"--id={index}",
+             "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+             "--format=csv,noheader,nounits", "-lms", "100"],
+            stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+    except OSError:
+        return None
+
+
+def _clock_summary(proc):
+    if proc is None:
+        return None
+    proc.terminate()
+    try:
+        out, _ = proc.communicate(timeout=5)
+    except subprocess.TimeoutExpired:
+        proc.kill()
+        out, _ = proc.communicate()
+    sm, smax, reasons = [], None, set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for line in out.strip().splitlines():
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) < 8:
+            continue
+        try:
+            sm.append(float(parts[0]))
+            smax = float(parts[1])
+        except ValueError:
+            continue
+        for n, v in zip(names, parts[4:8]):
+            if v.lower() == "active":
+                reasons.add(n)
+    if not sm:
+        return None
+    return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+            "samples": len(sm)}
+
+
+def _traffic_record(kernel_src: str, workload: str):
+    """DRAM traffic of the dominant kernel from the committed ncu summary, if
+    the summary was taken on the current source of that kernel."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        rec = json.load(open(p)).get(workload)
+    except (ValueError, OSError):
+        return None
+    if not rec:
+        return None
+    h = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()[:16]
+    return rec.get("bytes_per_launch") if rec.get("source_sha") == h else None
+
+
+# ------------------------------------------------------------ CPU oracle
+def cpu_baseline(w, budget_s: float = 15.0):
+    """Time the oracle (as it stands) on a bounded sample of the workload:
+    whole sequences (attention over all heads + the verify call(s)), added
+    one at a time until ~budget_s of CPU work."""
+    import oracle
+    oracle.build()
+    done_nodes, elapsed, seqs = 0, 0.0, 0
+    for b in range(w.B):
+        T = int(w.n_nodes[b])
+        sub = _subset(w, b)
+        t0 = time.perf_counter()
+        if T:
+            rows = [(0, u, h) for u in range(T) for h in range(w.Hq)]
+            oracle.tree_attention_rows(sub.q, sub.k_cache, sub.v_cache, sub.prefix_len,
+                                       sub.n_nodes, sub.parent, sub.scale, rows)
+        if "greedy" in w.verify:
+            oracle.workload_greedy(sub)
+        if "stochastic" in w.verify:
+            oracle.workload_stochastic(sub)
+        elapsed += time.perf_counter() - t0
+        done_nodes += T
+        seqs += 1
+        if elapsed >= budget_s:
+            break
+    return {"value": done_nodes / elapsed, "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{seqs} of {w.B} sequences ({done_nodes} nodes), full attention layer "
+                      f"over all {w.Hq} heads + {'/'.join(w.verify)} verify, {elapsed:.1f} s"}
+
+
+def _subset(w, b):
+    import dataclasses
+    sl = slice(b, b + 1)
+    return dataclasses.replace(
+        w, B=1, parent=w.parent[sl], n_nodes=w.n_nodes[sl], prefix_len=w.prefix_len[sl],
+        tokens=w.tokens[sl], q_row=w.q_row[sl], q=w.q[sl], k_cache=w.k_cache[sl],
+        v_cache=w.v_cache[sl], logits=w.logits[sl], q_probs=w.q_probs[sl],
+        u_accept=w.u_accept[sl], u_sample=w.u_sample[sl])
+
+
+# ------------------------------------------------------------------ main
+def _workload_name(w):
+    return w.name
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(gen.WORKLOAD_NAMES))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    ws, rank, local = _dist()
+    cfg = gen.WORKLOAD_NAMES[args.workload]
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        w = gen.config_workload(cfg)
+        times = []
+        cb = None
+        for i in range(args.warmup + args.steps):
+            cb = cpu_baseline(w, budget_s=2.0 if i < args.warmup else 6.0)
+            if i >= args.warmup:
+                times.append(cb["value"])
+        val = statistics.median(times)
+        cb["value"] = val
+        line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT,
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": _workload_name(w)},
+                "cpu_baseline": cb,
+                "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import tree_speculative_decoding_ancestor_b200 as tsd
+
+    torch.cuda.set_device(local)
+    dev = torch.device(f"cuda:{local}")
+    pg = None
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    # weak scaling: every rank verifies its own batch (a different seed per rank)
+    w = gen.config_workload(cfg, seed=gen.SEED_BASE + cfg + 1000 * rank)
+    step = Step(w, dev, tsd)
+    tokens_per_step = int(w.n_nodes.sum())
+
+    for _ in range(max(3, args.warmup)):
+        step.run()
+    torch.cuda.synchronize(dev)
+    if int(tsd.device_status(dev).item()) != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    flush = None
+    working = w.kv_bytes() + w.logits.numel() * 4 + w.q_probs.numel() * 4
+    if working < 3 * L2_BYTES:
+        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+
+    n_att = args.steps
+    att_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n_att)]
+    st_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(args.steps)]
+    clocks = _clock_sampler(local)
+    time.sleep(0.3)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = tsd.launch_count()
+    for i in range(args.steps):
+        if flush is not None:
+            flush.fill_(float(i))
+        st_ev[i][0].record()
+        step.run(att_ev[i])
+        st_ev[i][1].record()
+    torch.cuda.synchronize(dev)
+    launches = tsd.launch_count() - launches0
+    if pg:
+        pg.barrier()
+    clk = _clock_summary(clocks)
+    step_ms = [a.elapsed_time(b) for a, b in st_ev]
+    att_ms = [a.elapsed_time(b) for a, b in att_ev]
+    total_ms = float(sum(step_ms))
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if pg:
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = ws * tokens_per_step / (ms_per_step / 1e3)
+    if int(tsd.device_status(dev).item()) != 0:
+        raise RuntimeError("device status set during the timed steps")
+
+    peaks, peak_kind = _peaks()
+    att_s = statistics.mean(att_ms) / 1e3
+    flops = attn_flops(w)
+    abytes = attn_bytes(w)
+    t_hbm = abytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    if t_tc > t_hbm:
+        roof = {"bound": "tensor", "achieved": flops / att_s / 1e12,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": abytes / att_s / 1e9, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json burst)" if peak_kind == \
+        "measured" else "fallback"
+    kernel_src = os.path.join(ROOT, "tree_speculative_decoding_ancestor_b200", "csrc",
+                              "attention_umma.cu")
+    roof["traffic"] = _traffic_record(kernel_src, args.workload)
+    roof["kernel"] = "tree attention (mask-aware split-KV), one layer"
+    roof["attn_us"] = att_s * 1e6
+    roof["algorithmic_bytes"] = abytes
+    roof["algorithmic_flops"] = flops
+    kv_gbs = w.kv_bytes() / att_s / 1e9
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": _workload_name(w), "batch_per_gpu": w.B,
+                       "tree_nodes_per_step_per_gpu": tokens_per_step, "Hq": w.Hq,
+                       "Hkv": w.Hkv, "head_dim": w.D, "prefix": int(w.prefix_len[0]),
+                       "vocab": w.V, "verify": list(w.verify),
+                       "l2": "flushed between steps (2x L2 write)" if flush is not None
+                       else f"inputs larger than L2 ({working / 1e6:.0f} MB read per step)",
+                       "parallelism": f"batch-sharded x{ws} (independent sequences)"},
+            "kv_cache_gbs": kv_gbs, "kv_cache_frac_of_hbm": kv_gbs / peaks["hbm_gbs"],
+            "roofline": roof, "gpu_launches": launches, "clocks": clk}
+
+    if not args.no_e2e:
+        line["e2e"] = e2e(w, dev, tsd, args, pg, ws)
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.destroy_process_group()
+
+
+def e2e(w, dev, tsd, args, pg, ws):
+    """Same metric through the public API with the inputs in pinned host
+    memory: every step copies its inputs host->device and the results back."""
+    fields = ("parent", "n_nodes", "prefix_len", "tokens", "q_row", "q", "k_cache", "v_cache",
+              "logits", "q_probs", "u_accept", "u_sample")
+    host = {f: getattr(w, f).pin_memory() for f in fields}
+    devb = {f: torch.empty_like(host[f], device=dev) for f in fields}
+    step = Step(w, dev, tsd)
+    step.d = devb
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    outs = [step.out, step.g.out_tokens, step.g.out_path, step.g.n_accepted,
+            step.s.out_tokens, step.s.out_path, step.s.n_accepted]
+    if "greedy" not in w.verify:
+        outs = [o for o in outs if o is not step.g.out_tokens and o is not step.g.out_path
+                and o is not step.g.n_accepted]
+    if "stochastic" not in w.verify:
+        outs = [o for o in outs if o is not step.s.out_tokens and o is not step.s.out_path
+                and o is not step.s.n_accepted]
+    host_out = [torch.empty_like(o, device="cpu").pin_memory() for o in outs]
+    d2h = sum(o.numel() * o.element_size() for o in outs)
+    steps = max(3, min(args.steps, 10))
+
+    def one():
+        for f in fields:
+            devb[f].copy_(host[f], non_blocking=True)
+        step.run()
+        for o, h in zip(outs, host_out):
+            h.copy_(o, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize(dev)
+    if pg:
+        pg.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if pg:
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    ms = float(t.item())
+    return {"value": ws * int(w.n_nodes.sum()) / (ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
+            "ms_per_step": ms}
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,210 @@
+/*
+ * tsd.h -- C ABI of the B200 (sm_100a) tree speculative decoding verification
+ * library (libtsd.so).
+ *
+ * The operations follow the SpecInfer explainer page "論文解説: SpecInfer -
+ * 投機的推論とトークンツリー検証によるLLMサービング高速化" (0h-n0.github.io,
+ * arXiv:2305.09781):
+ *   - a token tree of speculated tokens, one node per token, each root-to-node
+ *     path a candidate sequence S_u  (section "トークンツリー構造の仕組み");
+ *   - topology-aware tree attention, softmax(Q_u K_{S_u}^T / sqrt(d_k)) V_{S_u},
+ *     where a node sees only its ancestors (same section, and "Tree Attention
+ *     のカーネル融合", item 1);
+ *   - greedy and stochastic (multi-step speculative sampling) verification of
+ *     the tree from the target model's logits (section "ツリー検証アルゴリズム").
+ *
+ * Common conventions
+ * ------------------
+ *  - Every pointer is a DEVICE pointer owned by the caller unless stated
+ *    otherwise; tensors are dense and row-major in the stated shape.  The
+ *    library never allocates device memory: scratch comes from a caller
+ *    workspace whose size the matching *_workspace_size() call returns.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream) and never synchronizes.  Calls are reentrant across
+ *    streams; a workspace must not be shared by calls that may overlap.
+ *  - A tree has n_nodes[b] = T_b <= Tmax nodes (Tmax <= TSD_MAX_TREE).  Node u
+ *    has parent[b][u] in [-1, u-1]; -1 means "child of the root".  The root is
+ *    the last committed token: it is part of the prefix, not a tree node.
+ *    Slots u >= T_b are padding; outputs for them are not written unless a
+ *    function says so.
+ *  - The KV cache is [B][Hkv][Lmax][D]: the committed prefix of sequence b at
+ *    positions 0..prefix_len[b]-1 and tree node u at position prefix_len[b]+u
+ *    (the depth-first KV-cache layout of "Tree Attention のカーネル融合",
+ *    item 2, generalised to any parent-before-child numbering).
+ *  - Target logits are [B][Tmax+1][V] fp32: row 0 belongs to the root, row
+ *    1+u to node u.
+ *  - Return value: TSD_OK or a negative TSD_ERR_* code for errors found on the
+ *    host before any launch (nothing is launched then).  Errors found in the
+ *    data on the device are OR-ed into *dev_status (TSD_DEV_* bits; pass NULL
+ *    to ignore them); the caller reads that int32 when convenient.
+ */
+#ifndef TSD_H
+#define TSD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st *tsd_stream_t;
+
+#define TSD_MAX_TREE 128 /* largest Tmax (ancestor masks are 4 x u32) */
+
+enum tsd_status {
+    TSD_OK = 0,
+    TSD_ERR_NULL = -1,        /* a required pointer is NULL                 */
+    TSD_ERR_SHAPE = -2,       /* a size is out of range or inconsistent     */
+    TSD_ERR_DTYPE = -3,       /* unsupported dtype / head_dim combination   */
+    TSD_ERR_WORKSPACE = -4,   /* workspace smaller than *_workspace_size()  */
+    TSD_ERR_CUDA = -5,        /* a CUDA runtime/driver call failed          */
+    TSD_ERR_ALIGN = -6        /* a pointer is not 16-byte aligned           */
+};
+
+/* Bits OR-ed into *dev_status by the kernels. */
+enum tsd_dev_status {
+    TSD_DEV_BAD_TREE = 1,     /* n_nodes out of [0,Tmax] or parent[u] not in [-1,u-1] */
+    TSD_DEV_BAD_TOKEN = 2,    /* a token id outside [0, V)                  */
+    TSD_DEV_BAD_QROW = 4,     /* a q_row index outside [0, Rq)              */
+    TSD_DEV_BAD_PREFIX = 8,   /* prefix_len[b] + n_nodes[b] > Lmax or < 0   */
+    TSD_DEV_TIMEOUT = 16      /* a bounded pipeline wait expired (kernel bailed out) */
+};
+
+/* Element types of Q / K / V / attention output. */
+enum tsd_dtype { TSD_F32 = 0, TSD_BF16 = 1 };
+
+/* Marker written to first_child[b][0] by tsd_tree_mask_build for a malformed
+ * tree; the verify calls then report n_accepted[b] = -1 for that sequence. */
+#define TSD_TREE_INVALID (-2)
+
+/* Human-readable name of a tsd_status value. */
+const char *tsd_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int tsd_version(void);
+
+/* Number of kernels this library has launched in this process so far (all
+ * devices, all streams).  Instrumentation for benchmarks. */
+unsigned long long tsd_launch_count(void);
+
+/*
+ * Ancestor mask of each token tree (the topology-aware causal mask:
+ * "トークンツリー構造の仕組み", last paragraph; "Tree Attention のカーネル融合",
+ * item 1).
+ *   parent       [B][Tmax] int32        node -> parent (-1 = root)
+ *   n_nodes      [B] int32              T_b
+ *   mask         [B][Tmax][W] uint32    out, W = ceil(Tmax/32): bit v of row u is
+ *                                       set iff v is on the root->u path (u included)
+ *   depth        [B][Tmax] int32        out, number of nodes on the root->u path
+ *   first_child  [B][Tmax+1] int32      out, slot 0 = root, slot 1+c = node c:
+ *                                       smallest child index or -1
+ *   next_sibling [B][Tmax] int32        out, next larger index with the same parent, or -1
+ * Every output slot is written: padding rows get mask 0, depth 0, links -1.
+ * A malformed tree sets TSD_DEV_BAD_TREE, writes those padding values for the
+ * whole sequence and first_child[b][0] = TSD_TREE_INVALID.
+ * Host errors: TSD_ERR_NULL, TSD_ERR_SHAPE (B < 0, Tmax < 1 or > TSD_MAX_TREE).
+ */
+int tsd_tree_mask_build(const int32_t *parent, const int32_t *n_nodes, int B, int Tmax,
+                        uint32_t *mask, int32_t *depth, int32_t *first_child,
+                        int32_t *next_sibling, int32_t *dev_status, tsd_stream_t stream);
+
+/*
+ * Bytes of workspace tsd_tree_attention needs for these sizes (split-KV
+ * partial results).  Depends only on the arguments and the current device.
+ */
+size_t tsd_tree_attention_workspace_size(int B, int Tmax, int Hq, int Hkv, int D, int Lmax,
+                                         int dtype);
+
+/*
+ * Tree attention ("トークンツリー構造の仕組み", equation
+ * Attention(Q_u, K_{S_u}, V_{S_u})): for every node u < T_b and query head h,
+ *   out[b][u][h] = sum_{j in S_u} softmax_j(scale * q[b][u][h] . k_j) v_j
+ * where S_u = prefix positions 0..prefix_len[b]-1 plus the cache positions
+ * prefix_len[b]+v of the nodes v whose bit is set in mask[b][u], and k_j, v_j
+ * come from KV head h / (Hq / Hkv) (grouped-query attention).
+ *   q            [B][Tmax][Hq][D]   dtype
+ *   k_cache      [B][Hkv][Lmax][D]  dtype
+ *   v_cache      [B][Hkv][Lmax][D]  dtype
+ *   prefix_len   [B] int32          committed prefix length P_b
+ *   n_nodes      [B] int32          T_b (prefix_len[b] + T_b <= Lmax)
+ *   mask         [B][Tmax][W] uint32 from tsd_tree_mask_build
+ *   out          [B][Tmax][Hq][D]   dtype; rows u >= T_b are not written
+ * dtype TSD_BF16 (D = 64 or 128; fp32 accumulation and softmax) or TSD_F32.
+ * Cache positions at or beyond prefix_len[b] + T_b are never read into the
+ * result, whatever they hold.  q, k_cache, v_cache, out must be 16-byte
+ * aligned.  Host errors: TSD_ERR_NULL, TSD_ERR_SHAPE (Hq % Hkv != 0, sizes
+ * out of range), TSD_ERR_DTYPE, TSD_ERR_ALIGN, TSD_ERR_WORKSPACE, TSD_ERR_CUDA.
+ * Device: TSD_DEV_BAD_PREFIX (that sequence's rows are not written),
+ * TSD_DEV_TIMEOUT.
+ */
+int tsd_tree_attention(const void *q, const void *k_cache, const void *v_cache,
+                       const int32_t *prefix_len, const int32_t *n_nodes, const uint32_t *mask,
+                       int B, int Tmax, int Hq, int Hkv, int D, int Lmax, float scale,
+                       int dtype, void *out, void *workspace, size_t workspace_bytes,
+                       int32_t *dev_status, tsd_stream_t stream);
+
+/* Bytes of workspace either verify call needs (per-row statistics). */
+size_t tsd_tree_verify_workspace_size(int B, int Tmax, int V);
+
+/*
+ * Greedy verification ("ツリー検証アルゴリズム", greedy variant): accept the
+ * longest root path whose every token equals the argmax of its parent's
+ * logits row (lowest token id on argmax ties; lowest terminal node index when
+ * two paths are equally long), then append the argmax of the terminal's row
+ * (row 0 when nothing is accepted).
+ *   logits      [B][Tmax+1][V] fp32
+ *   tokens      [B][Tmax] int32     speculated token of each node
+ *   parent, n_nodes, mask, first_child   as produced / consumed above
+ *   out_tokens  [B][Tmax+1] int32   out: accepted tokens, then the bonus token
+ *   out_path    [B][Tmax] int32     out: accepted node indices, root-first
+ *   n_accepted  [B] int32           out: number of accepted nodes (-1 if the
+ *                                   sequence is malformed; nothing else written)
+ * Entries beyond n_accepted (+1 for out_tokens) are not written.
+ * Device: TSD_DEV_BAD_TOKEN.
+ */
+int tsd_tree_verify_greedy(const float *logits, const int32_t *tokens, const int32_t *parent,
+                           const int32_t *n_nodes, const uint32_t *mask,
+                           const int32_t *first_child, int B, int Tmax, int V,
+                           int32_t *out_tokens, int32_t *out_path, int32_t *n_accepted,
+                           void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                           tsd_stream_t stream);
+
+/*
+ * Stochastic verification by multi-step speculative sampling ("ツリー検証アル
+ * ゴリズム": P_accept = min(1, P_LLM(x)/P_SSM(x)); on rejection
+ * norm(max(0, P_LLM - P_SSM))).  Starting at the root, with p = softmax(l/T)
+ * of the current node's row (fp64): the children are tried in ascending
+ * index; child c with token x is accepted iff p(x) > 0 and
+ * u_accept[b][c] * q(x) <= p(x), where q = q_probs[b][q_row[b][c]]; after a
+ * rejection p becomes max(0, p - q) / sum(max(0, p - q)) (unchanged if that
+ * sum is 0).  An accepted child becomes the current node.  When no child is
+ * accepted (or there is none) the final token is drawn from p by inverse CDF:
+ * the smallest token i whose ascending cumulative sum exceeds
+ * u_sample[b][row], row being the current node's logits row (if rounding
+ * leaves none: the largest i with p_i > 0).
+ *   logits        [B][Tmax+1][V] fp32
+ *   temperature   T > 0
+ *   q_probs       [B][Rq][V] fp32   SSM distributions
+ *   q_row         [B][Tmax] int32   row of q_probs that proposed node u
+ *   tokens        [B][Tmax] int32
+ *   n_nodes, first_child, next_sibling   from tsd_tree_mask_build
+ *   u_accept      [B][Tmax] fp64, u_sample [B][Tmax+1] fp64: uniforms in (0,1)
+ *   out_tokens, out_path, n_accepted      as for the greedy call
+ * Device: TSD_DEV_BAD_TOKEN, TSD_DEV_BAD_QROW.
+ */
+int tsd_tree_verify_stochastic(const float *logits, double temperature, const float *q_probs,
+                               int Rq, const int32_t *q_row, const int32_t *tokens,
+                               const int32_t *n_nodes, const int32_t *first_child,
+                               const int32_t *next_sibling, const double *u_accept,
+                               const double *u_sample, int B, int Tmax, int V,
+                               int32_t *out_tokens, int32_t *out_path, int32_t *n_accepted,
+                               void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                               tsd_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TSD_H */

@@ -1,0 +1,27 @@
+"""B200-native verification hot path of tree speculative decoding (SpecInfer).
+
+Four calls, each a thin wrapper over the C ABI of ``lib/libtsd.so``
+(``include/tsd.h``):
+
+* :func:`tree_mask_build`     -- ancestor bitmask / depth / child lists from ``parent[]``;
+* :func:`tree_attention`      -- topology-aware tree attention over prefix KV + ancestors;
+* :func:`tree_verify_greedy`  -- longest argmax-matching root path + one bonus token;
+* :func:`tree_verify_stochastic` -- multi-step speculative sampling (exact target distribution).
+"""
+
+from .binding import (  # noqa: F401
+    LIB_PATH,
+    TsdError,
+    TreeMask,
+    VerifyResult,
+    attention_workspace_size,
+    device_status,
+    exported_symbols,
+    launch_count,
+    load_library,
+    tree_attention,
+    tree_mask_build,
+    tree_verify_greedy,
+    tree_verify_stochastic,
+    verify_workspace_size,
+)

@@ -1,0 +1,280 @@
+"""ctypes binding of libtsd.so (the C ABI declared in include/tsd.h).
+
+Argument marshalling only: shape/dtype/device checks, output and workspace
+allocation through PyTorch's caching allocator, and the caller's current
+CUDA stream.  Every step of the computation runs in the library's kernels;
+there is no CPU or PyTorch fallback -- if the library is missing, every call
+raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Dict, NamedTuple, Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "lib", "libtsd.so")
+
+TSD_OK = 0
+TSD_F32, TSD_BF16 = 0, 1
+TSD_MAX_TREE = 128
+TSD_TREE_INVALID = -2
+DEV_BAD_TREE, DEV_BAD_TOKEN, DEV_BAD_QROW, DEV_BAD_PREFIX, DEV_TIMEOUT = 1, 2, 4, 8, 16
+
+_lock = threading.Lock()
+_lib: Optional[ctypes.CDLL] = None
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_SZ = ctypes.c_size_t
+
+# name -> (restype, argtypes), mirroring include/tsd.h
+_SIGNATURES: Dict[str, Tuple[object, list]] = {
+    "tsd_status_string": (ctypes.c_char_p, [_I]),
+    "tsd_version": (_I, []),
+    "tsd_launch_count": (ctypes.c_ulonglong, []),
+    "tsd_tree_mask_build": (_I, [_P, _P, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "tsd_tree_attention_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
+    "tsd_tree_attention": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float,
+                                _I, _P, _P, _SZ, _P, _P]),
+    "tsd_tree_verify_workspace_size": (_SZ, [_I, _I, _I]),
+    "tsd_tree_verify_greedy": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _SZ, _P,
+                                    _P]),
+    "tsd_tree_verify_stochastic": (_I, [_P, ctypes.c_double, _P, _I, _P, _P, _P, _P, _P, _P, _P,
+                                        _I, _I, _I, _P, _P, _P, _P, _SZ, _P, _P]),
+}
+
+
+class TsdError(RuntimeError):
+    pass
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libtsd.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(path):
+                raise TsdError(f"{path} not found: build it with "
+                               "`python -m tree_speculative_decoding_ancestor_b200.build`")
+            lib = ctypes.CDLL(path)
+            for name, (res, args) in _SIGNATURES.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+        return _lib
+
+
+def exported_symbols() -> Tuple[str, ...]:
+    return tuple(_SIGNATURES)
+
+
+def launch_count() -> int:
+    """Kernels libtsd has launched in this process."""
+    return int(load_library().tsd_launch_count())
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != TSD_OK:
+        msg = load_library().tsd_status_string(rc).decode()
+        raise TsdError(f"{what} failed: {msg} ({rc})")
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape: Tuple[int, ...],
+          device: torch.device) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+# Per-device status word and workspace cache ---------------------------------
+_status: Dict[int, torch.Tensor] = {}
+_workspace: Dict[Tuple[int, str], torch.Tensor] = {}
+
+
+def device_status(device=None) -> torch.Tensor:
+    """The int32 word that the kernels OR their TSD_DEV_* bits into."""
+    device = torch.device(device or torch.cuda.current_device())
+    idx = device.index if device.index is not None else torch.cuda.current_device()
+    if idx not in _status:
+        _status[idx] = torch.zeros(1, dtype=torch.int32, device=f"cuda:{idx}")
+    return _status[idx]
+
+
+def _get_workspace(device: torch.device, kind: str, nbytes: int) -> torch.Tensor:
+    key = (device.index, kind)
+    ws = _workspace.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        _workspace[key] = ws
+    return ws
+
+
+class TreeMask(NamedTuple):
+    mask: torch.Tensor          # [B][Tmax][W] int32 (bit pattern of uint32)
+    depth: torch.Tensor         # [B][Tmax] int32
+    first_child: torch.Tensor   # [B][Tmax+1] int32
+    next_sibling: torch.Tensor  # [B][Tmax] int32
+
+
+class VerifyResult(NamedTuple):
+    out_tokens: torch.Tensor    # [B][Tmax+1] int32
+    out_path: torch.Tensor      # [B][Tmax] int32
+    n_accepted: torch.Tensor    # [B] int32
+
+
+def tree_mask_build(parent: torch.Tensor, n_nodes: torch.Tensor,
+                    out: Optional[TreeMask] = None, status: Optional[torch.Tensor] = None
+                    ) -> TreeMask:
+    """Ancestor mask, depth and child lists of each token tree."""
+    lib = load_library()
+    dev = parent.device
+    B, Tmax = parent.shape
+    W = (Tmax + 31) // 32
+    _need(parent, "parent", torch.int32, (B, Tmax), dev)
+    _need(n_nodes, "n_nodes", torch.int32, (B,), dev)
+    if out is None:
+        out = TreeMask(torch.empty((B, Tmax, W), dtype=torch.int32, device=dev),
+                       torch.empty((B, Tmax), dtype=torch.int32, device=dev),
+                       torch.empty((B, Tmax + 1), dtype=torch.int32, device=dev),
+                       torch.empty((B, Tmax), dtype=torch.int32, device=dev))
+    st = device_status(dev) if status is None else status
+    rc = lib.tsd_tree_mask_build(_ptr(parent), _ptr(n_nodes), B, Tmax, _ptr(out.mask),
+                                 _ptr(out.depth), _ptr(out.first_child), _ptr(out.next_sibling),
+                                 _ptr(st), _stream(dev))
+    _check(rc, "tsd_tree_mask_build")
+    return out
+
+
+def attention_workspace_size(B: int, Tmax: int, Hq: int, Hkv: int, D: int, Lmax: int,
+                             dtype: torch.dtype) -> int:
+    code = TSD_BF16 if dtype == torch.bfloat16 else TSD_F32
+    return int(load_library().tsd_tree_attention_workspace_size(B, Tmax, Hq, Hkv, D, Lmax, code))
+
+
+def tree_attention(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                   prefix_len: torch.Tensor, n_nodes: torch.Tensor, mask: torch.Tensor,
+                   scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                   workspace: Optional[torch.Tensor] = None,
+                   status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Topology-aware tree attention over prefix KV + ancestors (out[B][Tmax][Hq][D])."""
+    lib = load_library()
+    dev = q.device
+    B, Tmax, Hq, D = q.shape
+    Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
+    if q.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("q/k/v must be float32 or bfloat16")
+    _need(q, "q", q.dtype, (B, Tmax, Hq, D), dev)
+    _need(k_cache, "k_cache", q.dtype, (B, Hkv, Lmax, D), dev)
+    _need(v_cache, "v_cache", q.dtype, (B, Hkv, Lmax, D), dev)
+    _need(prefix_len, "prefix_len", torch.int32, (B,), dev)
+    _need(n_nodes, "n_nodes", torch.int32, (B,), dev)
+    _need(mask, "mask", torch.int32, (B, Tmax, (Tmax + 31) // 32), dev)
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", q.dtype, (B, Tmax, Hq, D), dev)
+    if scale is None:
+        scale = D ** -0.5
+    code = TSD_BF16 if q.dtype == torch.bfloat16 else TSD_F32
+    need = int(lib.tsd_tree_attention_workspace_size(B, Tmax, Hq, Hkv, D, Lmax, code))
+    ws = _get_workspace(dev, "attn", need) if workspace is None else workspace
+    st = device_status(dev) if status is None else status
+    rc = lib.tsd_tree_attention(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(prefix_len),
+                                _ptr(n_nodes), _ptr(mask), B, Tmax, Hq, Hkv, D, Lmax,
+                                float(scale), code, _ptr(out), _ptr(ws), ws.numel(), _ptr(st),
+                                _stream(dev))
+    _check(rc, "tsd_tree_attention")
+    return out
+
+
+def verify_workspace_size(B: int, Tmax: int, V: int) -> int:
+    return int(load_library().tsd_tree_verify_workspace_size(B, Tmax, V))
+
+
+def _verify_outputs(B, Tmax, dev, out):
+    if out is None:
+        out = VerifyResult(torch.empty((B, Tmax + 1), dtype=torch.int32, device=dev),
+                           torch.empty((B, Tmax), dtype=torch.int32, device=dev),
+                           torch.empty((B,), dtype=torch.int32, device=dev))
+    return out
+
+
+def tree_verify_greedy(logits: torch.Tensor, tokens: torch.Tensor, parent: torch.Tensor,
+                       n_nodes: torch.Tensor, tree: TreeMask,
+                       out: Optional[VerifyResult] = None,
+                       workspace: Optional[torch.Tensor] = None,
+                       status: Optional[torch.Tensor] = None) -> VerifyResult:
+    """Longest root path matching the target argmax, plus one bonus token."""
+    lib = load_library()
+    dev = logits.device
+    B, R, V = logits.shape
+    Tmax = R - 1
+    _need(logits, "logits", torch.float32, (B, Tmax + 1, V), dev)
+    _need(tokens, "tokens", torch.int32, (B, Tmax), dev)
+    _need(parent, "parent", torch.int32, (B, Tmax), dev)
+    _need(n_nodes, "n_nodes", torch.int32, (B,), dev)
+    out = _verify_outputs(B, Tmax, dev, out)
+    need = int(lib.tsd_tree_verify_workspace_size(B, Tmax, V))
+    ws = _get_workspace(dev, "verify", need) if workspace is None else workspace
+    st = device_status(dev) if status is None else status
+    rc = lib.tsd_tree_verify_greedy(_ptr(logits), _ptr(tokens), _ptr(parent), _ptr(n_nodes),
+                                    _ptr(tree.mask), _ptr(tree.first_child), B, Tmax, V,
+                                    _ptr(out.out_tokens), _ptr(out.out_path),
+                                    _ptr(out.n_accepted), _ptr(ws), ws.numel(), _ptr(st),
+                                    _stream(dev))
+    _check(rc, "tsd_tree_verify_greedy")
+    return out
+
+
+def tree_verify_stochastic(logits: torch.Tensor, temperature: float, q_probs: torch.Tensor,
+                           q_row: torch.Tensor, tokens: torch.Tensor, n_nodes: torch.Tensor,
+                           tree: TreeMask, u_accept: torch.Tensor, u_sample: torch.Tensor,
+                           out: Optional[VerifyResult] = None,
+                           workspace: Optional[torch.Tensor] = None,
+                           status: Optional[torch.Tensor] = None) -> VerifyResult:
+    """Multi-step speculative sampling over the tree (exact target distribution)."""
+    lib = load_library()
+    dev = logits.device
+    B, R, V = logits.shape
+    Tmax = R - 1
+    Rq = q_probs.shape[1]
+    _need(logits, "logits", torch.float32, (B, Tmax + 1, V), dev)
+    _need(q_probs, "q_probs", torch.float32, (B, Rq, V), dev)
+    _need(q_row, "q_row", torch.int32, (B, Tmax), dev)
+    _need(tokens, "tokens", torch.int32, (B, Tmax), dev)
+    _need(n_nodes, "n_nodes", torch.int32, (B,), dev)
+    _need(u_accept, "u_accept", torch.float64, (B, Tmax), dev)
+    _need(u_sample, "u_sample", torch.float64, (B, Tmax + 1), dev)
+    out = _verify_outputs(B, Tmax, dev, out)
+    need = int(lib.tsd_tree_verify_workspace_size(B, Tmax, V))
+    ws = _get_workspace(dev, "verify", need) if workspace is None else workspace
+    st = device_status(dev) if status is None else status
+    rc = lib.tsd_tree_verify_stochastic(_ptr(logits), float(temperature), _ptr(q_probs), Rq,
+                                        _ptr(q_row), _ptr(tokens), _ptr(n_nodes),
+                                        _ptr(tree.first_child), _ptr(tree.next_sibling),
+                                        _ptr(u_accept), _ptr(u_sample), B, Tmax, V,
+                                        _ptr(out.out_tokens), _ptr(out.out_path),
+                                        _ptr(out.n_accepted), _ptr(ws), ws.numel(), _ptr(st),
+                                        _stream(dev))
+    _check(rc, "tsd_tree_verify_stochastic")
+    return out

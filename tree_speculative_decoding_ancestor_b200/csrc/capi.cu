@@ -1,0 +1,190 @@
+// extern "C" entry points of libtsd: argument checks on the host, then the
+// launches.  Nothing here allocates device memory or synchronizes.
+#include <atomic>
+#include <cstdint>
+#include <cstdlib>
+
+#include "tsd_common.cuh"
+
+namespace tsd {
+static std::atomic<unsigned long long> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+}  // namespace tsd
+
+namespace {
+
+int device_sms()
+{
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return sms;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        sms = 148;
+    return sms;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Path selection for tree attention: the tensor-core kernel when the packed
+// query block is large enough and the layout fits it, otherwise CUDA cores.
+// TSD_FORCE_PATH=simt|umma overrides (for A/B measurement).
+int choose_umma(const tsd::AttnArgs &a)
+{
+    const char *force = std::getenv("TSD_FORCE_PATH");
+    const bool ok = tsd::umma_attention_supported(a);
+    if (force && force[0] == 's')
+        return 0;
+    if (force && force[0] == 'u')
+        return ok ? 1 : 0;
+    return ok ? 1 : 0;
+}
+
+int check_attn(const tsd::AttnArgs &a)
+{
+    if (!a.q || !a.k || !a.v || !a.prefix_len || !a.n_nodes || !a.mask || !a.out)
+        return TSD_ERR_NULL;
+    if (a.B < 0 || a.Tmax < 1 || a.Tmax > TSD_MAX_TREE || a.Hq < 1 || a.Hkv < 1 ||
+        a.Hq % a.Hkv != 0 || a.Lmax < a.Tmax)
+        return TSD_ERR_SHAPE;
+    if (a.dtype != TSD_F32 && a.dtype != TSD_BF16)
+        return TSD_ERR_DTYPE;
+    if (a.D != 64 && a.D != 128)
+        return TSD_ERR_DTYPE;
+    if (!aligned16(a.q) || !aligned16(a.k) || !aligned16(a.v) || !aligned16(a.out))
+        return TSD_ERR_ALIGN;
+    return TSD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *tsd_status_string(int status)
+{
+    switch (status) {
+    case TSD_OK: return "ok";
+    case TSD_ERR_NULL: return "a required pointer is NULL";
+    case TSD_ERR_SHAPE: return "size out of range or inconsistent";
+    case TSD_ERR_DTYPE: return "unsupported dtype / head_dim";
+    case TSD_ERR_WORKSPACE: return "workspace too small";
+    case TSD_ERR_CUDA: return "CUDA call failed";
+    case TSD_ERR_ALIGN: return "pointer not 16-byte aligned";
+    default: return "unknown status";
+    }
+}
+
+int tsd_version(void) { return 100; }
+
+unsigned long long tsd_launch_count(void) { return tsd::g_launches.load(); }
+
+int tsd_tree_mask_build(const int32_t *parent, const int32_t *n_nodes, int B, int Tmax,
+                        uint32_t *mask, int32_t *depth, int32_t *first_child,
+                        int32_t *next_sibling, int32_t *dev_status, tsd_stream_t stream)
+{
+    if (B < 0 || Tmax < 1 || Tmax > TSD_MAX_TREE)
+        return TSD_ERR_SHAPE;
+    if (B == 0)
+        return TSD_OK;
+    if (!parent || !n_nodes || !mask || !depth || !first_child || !next_sibling)
+        return TSD_ERR_NULL;
+    return tsd::launch_tree_mask(parent, n_nodes, B, Tmax, mask, depth, first_child, next_sibling,
+                                 dev_status, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t tsd_tree_attention_workspace_size(int B, int Tmax, int Hq, int Hkv, int D, int Lmax,
+                                         int dtype)
+{
+    tsd::AttnArgs a{};
+    a.B = B; a.Tmax = Tmax; a.Hq = Hq; a.Hkv = Hkv; a.D = D; a.Lmax = Lmax; a.dtype = dtype;
+    if (B <= 0 || Tmax < 1 || Tmax > TSD_MAX_TREE || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 ||
+        (D != 64 && D != 128) || Lmax < Tmax)
+        return 0;
+    const int sms = device_sms();
+    return choose_umma(a) ? tsd::umma_attention_workspace(a, sms)
+                          : tsd::simt_attention_workspace(a, sms);
+}
+
+int tsd_tree_attention(const void *q, const void *k_cache, const void *v_cache,
+                       const int32_t *prefix_len, const int32_t *n_nodes, const uint32_t *mask,
+                       int B, int Tmax, int Hq, int Hkv, int D, int Lmax, float scale,
+                       int dtype, void *out, void *workspace, size_t workspace_bytes,
+                       int32_t *dev_status, tsd_stream_t stream)
+{
+    tsd::AttnArgs a;
+    a.q = q; a.k = k_cache; a.v = v_cache; a.prefix_len = prefix_len; a.n_nodes = n_nodes;
+    a.mask = mask; a.B = B; a.Tmax = Tmax; a.Hq = Hq; a.Hkv = Hkv; a.D = D; a.Lmax = Lmax;
+    a.dtype = dtype; a.scale = scale; a.out = out; a.dev_status = dev_status;
+    if (B == 0)
+        return TSD_OK;
+    const int rc = check_attn(a);
+    if (rc != TSD_OK)
+        return rc;
+    const int sms = device_sms();
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (choose_umma(a)) {
+        if (workspace_bytes < tsd::umma_attention_workspace(a, sms))
+            return TSD_ERR_WORKSPACE;
+        return tsd::launch_umma_attention(a, workspace, workspace_bytes, sms, s);
+    }
+    if (workspace_bytes < tsd::simt_attention_workspace(a, sms))
+        return TSD_ERR_WORKSPACE;
+    return tsd::launch_simt_attention(a, workspace, workspace_bytes, sms, s);
+}
+
+size_t tsd_tree_verify_workspace_size(int B, int Tmax, int V)
+{
+    if (B <= 0 || Tmax < 1 || Tmax > TSD_MAX_TREE || V < 1)
+        return 0;
+    return tsd::verify_workspace(B, Tmax, V);
+}
+
+int tsd_tree_verify_greedy(const float *logits, const int32_t *tokens, const int32_t *parent,
+                           const int32_t *n_nodes, const uint32_t *mask,
+                           const int32_t *first_child, int B, int Tmax, int V,
+                           int32_t *out_tokens, int32_t *out_path, int32_t *n_accepted,
+                           void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                           tsd_stream_t stream)
+{
+    if (B < 0 || Tmax < 1 || Tmax > TSD_MAX_TREE || V < 1)
+        return TSD_ERR_SHAPE;
+    if (B == 0)
+        return TSD_OK;
+    if (!logits || !tokens || !parent || !n_nodes || !mask || !first_child || !out_tokens ||
+        !out_path || !n_accepted || !workspace)
+        return TSD_ERR_NULL;
+    if (!aligned16(logits))
+        return TSD_ERR_ALIGN;
+    if (workspace_bytes < tsd::verify_workspace(B, Tmax, V))
+        return TSD_ERR_WORKSPACE;
+    return tsd::launch_verify_greedy(logits, tokens, parent, n_nodes, mask, first_child, B, Tmax,
+                                     V, out_tokens, out_path, n_accepted, workspace, dev_status,
+                                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+int tsd_tree_verify_stochastic(const float *logits, double temperature, const float *q_probs,
+                               int Rq, const int32_t *q_row, const int32_t *tokens,
+                               const int32_t *n_nodes, const int32_t *first_child,
+                               const int32_t *next_sibling, const double *u_accept,
+                               const double *u_sample, int B, int Tmax, int V,
+                               int32_t *out_tokens, int32_t *out_path, int32_t *n_accepted,
+                               void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                               tsd_stream_t stream)
+{
+    if (B < 0 || Tmax < 1 || Tmax > TSD_MAX_TREE || V < 1 || Rq < 1 || !(temperature > 0.0))
+        return TSD_ERR_SHAPE;
+    if (B == 0)
+        return TSD_OK;
+    if (!logits || !q_probs || !q_row || !tokens || !n_nodes || !first_child || !next_sibling ||
+        !u_accept || !u_sample || !out_tokens || !out_path || !n_accepted || !workspace)
+        return TSD_ERR_NULL;
+    if (!aligned16(logits) || !aligned16(q_probs))
+        return TSD_ERR_ALIGN;
+    if (workspace_bytes < tsd::verify_workspace(B, Tmax, V))
+        return TSD_ERR_WORKSPACE;
+    return tsd::launch_verify_stochastic(logits, temperature, q_probs, Rq, q_row, tokens, n_nodes,
+                                         first_child, next_sibling, u_accept, u_sample, B, Tmax,
+                                         V, out_tokens, out_path, n_accepted, workspace,
+                                         dev_status, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

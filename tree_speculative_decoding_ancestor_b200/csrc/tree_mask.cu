@@ -1,0 +1,84 @@
+// Ancestor-mask builder: the topology-aware causal mask of SpecInfer's tree
+// attention ("トークンツリー構造の仕組み": node u attends only to the nodes on
+// its root path S_u; "Tree Attention のカーネル融合", item 1: the mask is
+// precomputed from the tree topology).
+//
+// One CTA of 128 threads per sequence, one thread per node slot.  The parent
+// array (<= 512 B) is staged in shared memory; every node walks its own root
+// path there (<= 128 steps, bounded because parent[v] < v is validated
+// first), so the whole build is a handful of shared-memory passes.
+#include <climits>
+
+#include "tsd_common.cuh"
+
+namespace tsd {
+
+__global__ void __launch_bounds__(kMaxTree)
+    tree_mask_kernel(const int32_t *__restrict__ parent, const int32_t *__restrict__ n_nodes,
+                     int Tmax, int W, uint32_t *__restrict__ mask, int32_t *__restrict__ depth,
+                     int32_t *__restrict__ first_child, int32_t *__restrict__ next_sibling,
+                     int32_t *dev_status)
+{
+    __shared__ int32_t par[kMaxTree];
+    __shared__ int32_t fc[kMaxTree + 1];
+    const int b = blockIdx.x;
+    const int u = threadIdx.x;
+    const int T = n_nodes[b];
+    const bool bad_T = !tree_header_ok(T, Tmax);
+    int p = -1;
+    if (u < Tmax && !bad_T && u < T)
+        p = parent[(size_t)b * Tmax + u];
+    par[u] = p;
+    fc[u] = INT_MAX;
+    if (u == 0)
+        fc[kMaxTree] = INT_MAX;
+    const bool bad_u = !bad_T && u < T && (p < -1 || p >= u);
+    const bool bad = __syncthreads_or(bad_T || bad_u);
+
+    uint32_t m[kMaskWords] = {0u, 0u, 0u, 0u};
+    int d = 0;
+    if (!bad && u < T) {
+        for (int v = u; v >= 0; v = par[v]) {
+            m[v >> 5] |= 1u << (v & 31);
+            ++d;
+        }
+        atomicMin(&fc[p + 1], u);
+    }
+    __syncthreads();
+    int ns = -1;
+    if (!bad && u < T)
+        for (int v = u + 1; v < T; ++v)
+            if (par[v] == p) {
+                ns = v;
+                break;
+            }
+    if (u < Tmax) {
+        for (int w = 0; w < W; ++w)
+            mask[((size_t)b * Tmax + u) * W + w] = m[w];
+        depth[(size_t)b * Tmax + u] = d;
+        next_sibling[(size_t)b * Tmax + u] = ns;
+    }
+    for (int s = u; s <= Tmax; s += blockDim.x) {
+        int v = (bad || fc[s] == INT_MAX) ? -1 : fc[s];
+        if (bad && s == 0)
+            v = TSD_TREE_INVALID;
+        first_child[(size_t)b * (Tmax + 1) + s] = v;
+    }
+    if (bad && u == 0)
+        flag(dev_status, TSD_DEV_BAD_TREE);
+}
+
+int launch_tree_mask(const int32_t *parent, const int32_t *n_nodes, int B, int Tmax,
+                     uint32_t *mask, int32_t *depth, int32_t *first_child, int32_t *next_sibling,
+                     int32_t *dev_status, cudaStream_t stream)
+{
+    if (B == 0)
+        return TSD_OK;
+    const int W = (Tmax + 31) / 32;
+    tree_mask_kernel<<<B, kMaxTree, 0, stream>>>(parent, n_nodes, Tmax, W, mask, depth,
+                                                 first_child, next_sibling, dev_status);
+    TSD_LAUNCH_CHECK();
+    return TSD_OK;
+}
+
+}  // namespace tsd

@@ -1,0 +1,115 @@
+// Device helpers shared by the libtsd kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "tsd.h"
+
+namespace tsd {
+
+constexpr int kMaxTree = TSD_MAX_TREE;
+constexpr int kMaskWords = (TSD_MAX_TREE + 31) / 32;
+
+__device__ __forceinline__ void flag(int32_t *dev_status, int bits)
+{
+    if (dev_status)
+        atomicOr(dev_status, bits);
+}
+
+__device__ __forceinline__ float to_float(float x) { return x; }
+__device__ __forceinline__ float to_float(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_float(float x);
+template <> __device__ __forceinline__ float from_float<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_float<__nv_bfloat16>(float x)
+{
+    return __float2bfloat16_rn(x);
+}
+
+__device__ __forceinline__ float warp_max(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ double warp_sum(double v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Sequence-level validity shared by the attention and verify kernels.
+__device__ __forceinline__ bool tree_header_ok(int T, int Tmax) { return T >= 0 && T <= Tmax; }
+
+}  // namespace tsd
+
+// Host-side launch helpers.
+#define TSD_CUDA_TRY(expr)                                                                    \
+    do {                                                                                      \
+        cudaError_t e_ = (expr);                                                              \
+        if (e_ != cudaSuccess)                                                                \
+            return TSD_ERR_CUDA;                                                              \
+    } while (0)
+
+// Checks the launch just made and counts it.
+#define TSD_LAUNCH_CHECK()                                                                    \
+    do {                                                                                      \
+        if (cudaPeekAtLastError() != cudaSuccess) {                                           \
+            (void)cudaGetLastError();                                                         \
+            return TSD_ERR_CUDA;                                                              \
+        }                                                                                     \
+        tsd::count_launch();                                                                  \
+    } while (0)
+
+// Internal launchers (defined in the kernel files, called by capi.cu).
+namespace tsd {
+void count_launch();
+int launch_tree_mask(const int32_t *parent, const int32_t *n_nodes, int B, int Tmax,
+                     uint32_t *mask, int32_t *depth, int32_t *first_child, int32_t *next_sibling,
+                     int32_t *dev_status, cudaStream_t stream);
+
+struct AttnArgs {
+    const void *q, *k, *v;
+    const int32_t *prefix_len, *n_nodes;
+    const uint32_t *mask;
+    int B, Tmax, Hq, Hkv, D, Lmax, dtype;
+    float scale;
+    void *out;
+    int32_t *dev_status;
+};
+size_t simt_attention_workspace(const AttnArgs &a, int num_sms);
+int launch_simt_attention(const AttnArgs &a, void *ws, size_t ws_bytes, int num_sms,
+                          cudaStream_t stream);
+bool umma_attention_supported(const AttnArgs &a);
+size_t umma_attention_workspace(const AttnArgs &a, int num_sms);
+int launch_umma_attention(const AttnArgs &a, void *ws, size_t ws_bytes, int num_sms,
+                          cudaStream_t stream);
+
+size_t verify_workspace(int B, int Tmax, int V);
+int launch_verify_greedy(const float *logits, const int32_t *tokens, const int32_t *parent,
+                         const int32_t *n_nodes, const uint32_t *mask,
+                         const int32_t *first_child, int B, int Tmax, int V,
+                         int32_t *out_tokens, int32_t *out_path, int32_t *n_accepted, void *ws,
+                         int32_t *dev_status, cudaStream_t stream);
+int launch_verify_stochastic(const float *logits, double temperature, const float *q_probs,
+                             int Rq, const int32_t *q_row, const int32_t *tokens,
+                             const int32_t *n_nodes, const int32_t *first_child,
+                             const int32_t *next_sibling, const double *u_accept,
+                             const double *u_sample, int B, int Tmax, int V,
+                             int32_t *out_tokens, int32_t *out_path, int32_t *n_accepted,
+                             void *ws, int32_t *dev_status, cudaStream_t stream);
+}  // namespace tsd

@@ -10,6 +10,7 @@ draw their inputs from it without sharing any of the method's code.
 
 from .gen import (  # noqa: F401
     CONFIGS,
+    WORKLOAD_NAMES,
     Workload,
     config_workload,
     random_workload,

@@ -377,6 +377,9 @@ CONFIGS: Dict[int, Dict] = {
 
 SEED_BASE = 20261202
 
+# Short names of the five workloads.
+WORKLOAD_NAMES = {"tiny": 0, "llama7b": 1, "merge": 2, "gqa70b": 3, "long32k": 4}
+
 
 def config_workload(index: int, seed: Optional[int] = None, B: Optional[int] = None,
                     with_attention: bool = True) -> Workload:
