@@ -266,7 +266,8 @@ def test_config_full_size(cuda_device, cfg):
         got = out.float().cpu().numpy()
         err = max(float(np.abs(got[b, u, h] - ref[i]).max()) for i, (b, u, h) in enumerate(rows))
         assert err <= 2e-2, err
-        assert torch.isfinite(out.float()).all().item()
+        for b in range(w.B):   # rows of padding slots are never written
+            assert torch.isfinite(out[b, :int(w.n_nodes[b])].float()).all().item()
     if "greedy" in w.verify:
         check_greedy(w, tsd.tree_verify_greedy(d["logits"], d["tokens"], d["parent"],
                                                d["n_nodes"], tree))
