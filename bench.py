@@ -243,6 +243,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(gen.WORKLOAD_NAMES))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--batch", type=int, default=None,
+                    help="sequences per GPU (default: the workload's batch)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
@@ -252,7 +254,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        w = gen.config_workload(cfg)
+        w = gen.config_workload(cfg, B=args.batch)
         times = []
         cb = None
         for i in range(args.warmup + args.steps):
@@ -283,7 +285,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         pg = dist
     # weak scaling: every rank verifies its own batch (a different seed per rank)
-    w = gen.config_workload(cfg, seed=gen.SEED_BASE + cfg + 1000 * rank)
+    w = gen.config_workload(cfg, seed=gen.SEED_BASE + cfg + 1000 * rank, B=args.batch)
     step = Step(w, dev, tsd)
     tokens_per_step = int(w.n_nodes.sum())
 
