@@ -203,6 +203,39 @@ int tsd_tree_verify_stochastic(const float *logits, double temperature, const fl
                                void *workspace, size_t workspace_bytes, int32_t *dev_status,
                                tsd_stream_t stream);
 
+/*
+ * Stochastic verification without a workspace, for callers that cannot
+ * allocate device memory (for example a serving engine whose KV-cache pool
+ * already owns nearly all of the GPU's memory, or a caller reaching the
+ * library through a plain C interface with no device allocator).  The paper
+ * has no counterpart to this call; it is the same operation as
+ * tsd_tree_verify_stochastic, with the same arguments minus the workspace.
+ *
+ * The scratch it needs lives in a fixed array of TSD_NOALLOC_SCRATCH_BYTES
+ * inside the library's device code; every GPU that loads the library holds
+ * that array until the process exits.  Nothing is allocated: no cudaMalloc,
+ * no cudaFree, no allocating library routine.
+ *   - Sizes whose scratch exceeds the array (about 28 bytes per logits row,
+ *     i.e. B * (Tmax + 1) up to roughly 37000 rows) return TSD_ERR_WORKSPACE
+ *     and launch nothing; use tsd_tree_verify_stochastic for those.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the one array, which keeps the last call's
+ *     contents.  Calls whose kernels may overlap on the GPU (different
+ *     streams, or concurrent host threads) race on it: serialise them.
+ */
+#define TSD_NOALLOC_SCRATCH_BYTES (1u << 20)
+
+int tsd_tree_verify_stochastic_noalloc(const float *logits, double temperature,
+                                       const float *q_probs, int Rq, const int32_t *q_row,
+                                       const int32_t *tokens, const int32_t *n_nodes,
+                                       const int32_t *first_child, const int32_t *next_sibling,
+                                       const double *u_accept, const double *u_sample, int B,
+                                       int Tmax, int V, int32_t *out_tokens, int32_t *out_path,
+                                       int32_t *n_accepted, int32_t *dev_status,
+                                       tsd_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -23,5 +23,6 @@ from .binding import (  # noqa: F401
     tree_mask_build,
     tree_verify_greedy,
     tree_verify_stochastic,
+    tree_verify_stochastic_noalloc,
     verify_workspace_size,
 )

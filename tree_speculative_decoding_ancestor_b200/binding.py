@@ -46,6 +46,8 @@ _SIGNATURES: Dict[str, Tuple[object, list]] = {
                                     _P]),
     "tsd_tree_verify_stochastic": (_I, [_P, ctypes.c_double, _P, _I, _P, _P, _P, _P, _P, _P, _P,
                                         _I, _I, _I, _P, _P, _P, _P, _SZ, _P, _P]),
+    "tsd_tree_verify_stochastic_noalloc": (_I, [_P, ctypes.c_double, _P, _I, _P, _P, _P, _P, _P,
+                                                _P, _P, _I, _I, _I, _P, _P, _P, _P, _P]),
 }
 
 
@@ -277,4 +279,37 @@ def tree_verify_stochastic(logits: torch.Tensor, temperature: float, q_probs: to
                                         _ptr(out.n_accepted), _ptr(ws), ws.numel(), _ptr(st),
                                         _stream(dev))
     _check(rc, "tsd_tree_verify_stochastic")
+    return out
+
+
+def tree_verify_stochastic_noalloc(logits: torch.Tensor, temperature: float,
+                                   q_probs: torch.Tensor, q_row: torch.Tensor,
+                                   tokens: torch.Tensor, n_nodes: torch.Tensor, tree: TreeMask,
+                                   u_accept: torch.Tensor, u_sample: torch.Tensor,
+                                   out: VerifyResult, status: Optional[torch.Tensor] = None
+                                   ) -> VerifyResult:
+    """tree_verify_stochastic for callers that cannot allocate device memory:
+    the scratch lives in a fixed array inside the library, so the caller
+    passes preallocated outputs and nothing is allocated here (see
+    tsd_tree_verify_stochastic_noalloc in include/tsd.h for the size limit,
+    the first-call set-up and why overlapping calls race)."""
+    lib = load_library()
+    dev = logits.device
+    B, R, V = logits.shape
+    Tmax = R - 1
+    Rq = q_probs.shape[1]
+    _need(logits, "logits", torch.float32, (B, Tmax + 1, V), dev)
+    _need(q_probs, "q_probs", torch.float32, (B, Rq, V), dev)
+    _need(q_row, "q_row", torch.int32, (B, Tmax), dev)
+    _need(tokens, "tokens", torch.int32, (B, Tmax), dev)
+    _need(n_nodes, "n_nodes", torch.int32, (B,), dev)
+    _need(u_accept, "u_accept", torch.float64, (B, Tmax), dev)
+    _need(u_sample, "u_sample", torch.float64, (B, Tmax + 1), dev)
+    st = device_status(dev) if status is None else status
+    rc = lib.tsd_tree_verify_stochastic_noalloc(
+        _ptr(logits), float(temperature), _ptr(q_probs), Rq, _ptr(q_row), _ptr(tokens),
+        _ptr(n_nodes), _ptr(tree.first_child), _ptr(tree.next_sibling), _ptr(u_accept),
+        _ptr(u_sample), B, Tmax, V, _ptr(out.out_tokens), _ptr(out.out_path),
+        _ptr(out.n_accepted), _ptr(st), _stream(dev))
+    _check(rc, "tsd_tree_verify_stochastic_noalloc")
     return out
