@@ -276,3 +276,20 @@ def test_config_full_size(cuda_device, cfg):
                                                        d["q_row"], d["tokens"], d["n_nodes"],
                                                        tree, d["u_accept"], d["u_sample"]))
     assert _status(cuda_device) == 0
+
+
+# ------------------------------------------------- table-driven fp64 exp
+def test_table_exp_accuracy(cuda_device, tmp_path):
+    """The verifier's bulk fp64 exp (Tang's table-driven method) stays within
+    4e-15 relative (a few ulp) of CUDA's exp() on [-60, 0] and at special
+    points down to -708, and flushes x < -708 to 0."""
+    import os
+    import subprocess
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    exe = str(tmp_path / "table_exp_check")
+    subprocess.run(["/usr/local/cuda/bin/nvcc", "-O3", "-gencode", "arch=compute_100a,code=sm_100a",
+                    "-I", os.path.join(root, "tree_speculative_decoding_ancestor_b200", "csrc"),
+                    os.path.join(root, "tests", "cuda", "table_exp_check.cu"), "-o", exe],
+                   check=True)
+    r = subprocess.run([exe, "4e-15"], capture_output=True, text=True)
+    assert r.returncode == 0, r.stdout + r.stderr

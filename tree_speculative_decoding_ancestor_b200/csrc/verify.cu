@@ -1,28 +1,38 @@
 // Tree verification from the target model's logits (SpecInfer explainer,
 // section "ツリー検証アルゴリズム").
 //
-// Both verifiers run in two launches:
-//   1. a row kernel, one CTA per (logits row, sequence), for the rows whose
-//      node has children (the root included).  Greedy: argmax of the row.
-//      Stochastic: max, Z = sum exp((l-m)/T) in fp64, then multi-step
-//      speculative sampling over the node's children in ascending index --
-//      acceptance test u*q(x) <= p(x) with p(x) > 0, and after each rejection
-//      the residual normaliser S = sum max(0, p - q) of the updated
-//      distribution p <- max(0, p - q)/S.  Every internal node is decided in
-//      parallel, whether or not the final path reaches it.
-//   2. a finalize kernel, one CTA per sequence, that walks from the root
-//      through the accepted children and emits the path, then the last token:
-//      greedy -> argmax of the terminal row; stochastic -> inverse-CDF draw
-//      from the terminal's (residual) distribution with a block-wide fp64
-//      prefix scan.  A terminal that is a leaf gets its row statistics here.
+// Both verifiers decide every logits row in parallel, then walk:
+//   greedy
+//     greedy_rows_kernel      one CTA per row whose node has children: argmax
+//                             (lowest index on ties), float4 loads, several in
+//                             flight per thread;
+//     greedy_finalize_kernel  one CTA per sequence: nodes whose whole root path
+//                             matches, the deepest (lowest index on ties), and
+//                             the argmax of its row (computed here for a leaf).
+//   stochastic (multi-step speculative sampling)
+//     mss_rows_kernel         one CTA per row (every node and the root):
+//                             m = max l, Z = sum exp((l-m)/T) in fp64; then the
+//                             children in ascending index: child c with token x
+//                             is accepted iff p(x) > 0 and u_c * q_c(x) <= p(x)
+//                             (evaluated by one thread with the exact fp64
+//                             formula); after a rejection the block computes
+//                             S = sum max(0, p - q_c) and p becomes
+//                             max(0, p - q_c)/S.  A row that accepts no child
+//                             (a leaf included) draws its token by inverse CDF
+//                             at u_sample[row], with a tiled fp64 block scan.
+//     mss_finalize_kernel     one CTA per sequence: follows the accepted
+//                             children from the root and emits the path and the
+//                             draw of the row where it stops.
 //
-// Residual distributions are never materialised: p^(i)(x) is recomputed per
+// Residual distributions are never materialised: p^(n)(x) is recomputed per
 // element from the logits row, the rejected siblings' q rows and their
-// normalisers, with the same element-wise formula as the definition, so the
-// only difference from a sequential fp64 evaluation is the summation order
-// of Z, S and the cumulative sums.
+// normalisers.  The bulk sums (Z, S, the CDF) use a table-driven fp64 exp and
+// reciprocals; the acceptance tests use the exact formula.  Both agree with a
+// sequential fp64 evaluation to ~1e-15 relative, so a decision can only differ
+// when its uniform lies within that distance of the boundary.
 #include <climits>
 
+#include "fp64_exp.cuh"
 #include "tsd_common.cuh"
 
 namespace tsd {
@@ -31,31 +41,26 @@ namespace {
 
 constexpr int kRowThreads = 512;
 constexpr int kWarps = kRowThreads / 32;
+constexpr int kFinThreads = 1024;
 
 struct VerifyWs {
-    int32_t *argmax;   // [B][Tmax+1]
-    int32_t *accepted; // [B][Tmax+1]  accepted child per row, -1 none
-    float *rmax;       // [B][Tmax+1]
-    double *Z;         // [B][Tmax+1]
-    double *S;         // [B][Tmax]    residual normaliser after rejecting child c
+    int32_t *argmax;    // [B][Tmax+1]  greedy: argmax of rows with children
+    int32_t *accepted;  // [B][Tmax+1]  stochastic: accepted child per row, -1 none
+    int32_t *draw;      // [B][Tmax+1]  stochastic: token drawn where no child is accepted
 };
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 VerifyWs carve(void *ws, int B, int Tmax)
 {
-    const size_t R = (size_t)B * (Tmax + 1), N = (size_t)B * Tmax;
+    const size_t R = (size_t)B * (Tmax + 1);
     char *p = static_cast<char *>(ws);
     VerifyWs w;
-    w.Z = reinterpret_cast<double *>(p);
-    p += align256(R * sizeof(double));
-    w.S = reinterpret_cast<double *>(p);
-    p += align256(N * sizeof(double));
     w.argmax = reinterpret_cast<int32_t *>(p);
     p += align256(R * sizeof(int32_t));
     w.accepted = reinterpret_cast<int32_t *>(p);
     p += align256(R * sizeof(int32_t));
-    w.rmax = reinterpret_cast<float *>(p);
+    w.draw = reinterpret_cast<int32_t *>(p);
     return w;
 }
 
@@ -65,8 +70,10 @@ __device__ __forceinline__ bool better(float v, int i, float bv, int bi)
     return v > bv || (v == bv && i < bi);
 }
 
+template <int NT>
 __device__ void block_argmax(float &v, int &i, float *shv, int *shi)
 {
+    constexpr int NW = NT / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -83,8 +90,8 @@ __device__ void block_argmax(float &v, int &i, float *shv, int *shi)
     }
     __syncthreads();
     if (warp == 0) {
-        v = lane < kWarps ? shv[lane] : -INFINITY;
-        i = lane < kWarps ? shi[lane] : INT_MAX;
+        v = lane < NW ? shv[lane] : -INFINITY;
+        i = lane < NW ? shi[lane] : INT_MAX;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             const float ov = __shfl_xor_sync(0xffffffffu, v, o);
@@ -143,8 +150,10 @@ __device__ double block_sum(double v, double *sh)
     return v;
 }
 
+template <int NT>
 __device__ int block_min_int(int v, int *sh)
 {
+    constexpr int NW = NT / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1)
@@ -153,7 +162,7 @@ __device__ int block_min_int(int v, int *sh)
         sh[warp] = v;
     __syncthreads();
     if (warp == 0) {
-        v = lane < kWarps ? sh[lane] : INT_MAX;
+        v = lane < NW ? sh[lane] : INT_MAX;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1)
             v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -166,19 +175,37 @@ __device__ int block_min_int(int v, int *sh)
     return v;
 }
 
+template <int NT>
 __device__ int block_max_int(int v, int *sh)
 {
-    return -block_min_int(-v, sh);
+    return -block_min_int<NT>(-v, sh);
 }
 
-// Row argmax (lowest index among the maxima), float4 loads when V % 4 == 0.
+// Row argmax (lowest index among the maxima); four float4 loads in flight.
+template <int NT>
 __device__ int row_argmax(const float *__restrict__ row, int V, float *shv, int *shi)
 {
     float bv = -INFINITY;
     int bi = INT_MAX;
     if ((V & 3) == 0) {
         const float4 *r4 = reinterpret_cast<const float4 *>(row);
-        for (int j = threadIdx.x; j < V / 4; j += kRowThreads) {
+        const int n4 = V >> 2;
+        int j = threadIdx.x;
+        for (; j + 3 * NT < n4; j += 4 * NT) {
+            float4 x[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                x[k] = __ldg(r4 + j + k * NT);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int i0 = 4 * (j + k * NT);
+                if (better(x[k].x, i0, bv, bi)) { bv = x[k].x; bi = i0; }
+                if (better(x[k].y, i0 + 1, bv, bi)) { bv = x[k].y; bi = i0 + 1; }
+                if (better(x[k].z, i0 + 2, bv, bi)) { bv = x[k].z; bi = i0 + 2; }
+                if (better(x[k].w, i0 + 3, bv, bi)) { bv = x[k].w; bi = i0 + 3; }
+            }
+        }
+        for (; j < n4; j += NT) {
             const float4 x = __ldg(r4 + j);
             const int i0 = 4 * j;
             if (better(x.x, i0, bv, bi)) { bv = x.x; bi = i0; }
@@ -187,12 +214,12 @@ __device__ int row_argmax(const float *__restrict__ row, int V, float *shv, int 
             if (better(x.w, i0 + 3, bv, bi)) { bv = x.w; bi = i0 + 3; }
         }
     } else {
-        for (int j = threadIdx.x; j < V; j += kRowThreads) {
+        for (int j = threadIdx.x; j < V; j += NT) {
             const float x = __ldg(row + j);
             if (better(x, j, bv, bi)) { bv = x; bi = j; }
         }
     }
-    block_argmax(bv, bi, shv, shi);
+    block_argmax<NT>(bv, bi, shv, shi);
     return bi == INT_MAX ? 0 : bi;
 }
 
@@ -201,9 +228,20 @@ __device__ float row_max(const float *__restrict__ row, int V, float *sh)
     float m = -INFINITY;
     if ((V & 3) == 0) {
         const float4 *r4 = reinterpret_cast<const float4 *>(row);
-        for (int j = threadIdx.x; j < V / 4; j += kRowThreads) {
+        const int n4 = V >> 2;
+        int j = threadIdx.x;
+        for (; j + 3 * kRowThreads < n4; j += 4 * kRowThreads) {
+            float4 x[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                x[k] = __ldg(r4 + j + k * kRowThreads);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                m = fmaxf(m, fmaxf(fmaxf(x[k].x, x[k].y), fmaxf(x[k].z, x[k].w)));
+        }
+        for (; j < n4; j += kRowThreads) {
             const float4 x = __ldg(r4 + j);
-            m = fmaxf(fmaxf(m, x.x), fmaxf(fmaxf(x.y, x.z), x.w));
+            m = fmaxf(m, fmaxf(fmaxf(x.x, x.y), fmaxf(x.z, x.w)));
         }
     } else {
         for (int j = threadIdx.x; j < V; j += kRowThreads)
@@ -212,47 +250,154 @@ __device__ float row_max(const float *__restrict__ row, int V, float *sh)
     return block_max(m, sh);
 }
 
-// exp((l - m) / T) summed in fp64.
-__device__ double row_Z(const float *__restrict__ row, int V, double m, double temp, double *sh)
-{
-    double z = 0.0;
-    for (int j = threadIdx.x; j < V; j += kRowThreads)
-        z += exp(((double)__ldg(row + j) - m) / temp);
-    return block_sum(z, sh);
-}
-
-// Rejected siblings so far: their q rows and residual normalisers.
-struct Residual {
-    const float *q[kMaxTree];
-    double S[kMaxTree];
-    int n;
+// Per-row state of multi-step speculative sampling.
+struct RowState {
+    double m, inv_temp, temp, Z, inv_Z;
+    int n;                         // siblings rejected so far
+    const float *q[kMaxTree];      // their SSM rows
+    double S[kMaxTree];            // their residual normalisers
+    double inv_S[kMaxTree];        // 1/S (0 when S == 0: p unchanged)
 };
 
-// p^(n)(x): the target distribution after the first n rejections.
-__device__ __forceinline__ double residual_p(float lx, double m, double temp, double Z,
-                                             const Residual &res, int x)
+// Four consecutive fp32 values starting at x0 (0 beyond V); one float4 load
+// when the row is 16-byte aligned and V % 4 == 0 (VEC).
+template <bool VEC>
+__device__ __forceinline__ void load4(const float *__restrict__ p, int x0, int V, float (&v)[4])
 {
-    double p = exp(((double)lx - m) / temp) / Z;
-    for (int j = 0; j < res.n; ++j) {
-        if (res.S[j] > 0.0) {
-            const double r = p - (double)__ldg(res.q[j] + x);
-            p = (r > 0.0 ? r : 0.0) / res.S[j];
+    if (VEC) {
+        if (x0 < V) {
+            const float4 t = __ldg(reinterpret_cast<const float4 *>(p + x0));
+            v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+        } else {
+            v[0] = v[1] = v[2] = v[3] = 0.f;
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            v[k] = x0 + k < V ? __ldg(p + x0 + k) : 0.f;
+    }
+}
+
+// p^(n)(x) for x in [x0, x0+4) (0 beyond V) for the bulk sums: table exp and
+// reciprocals; the loads of each rejected sibling's row are issued together.
+template <bool VEC>
+__device__ __forceinline__ void p_bulk4(const float *__restrict__ row, int x0, int V,
+                                        const RowState &st, const double *table, double (&p)[4])
+{
+    float l[4];
+    load4<VEC>(row, x0, V, l);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+        p[k] = x0 + k < V ? table_exp(((double)l[k] - st.m) * st.inv_temp, table) * st.inv_Z
+                          : 0.0;
+    for (int j = 0; j < st.n; ++j) {
+        if (st.S[j] > 0.0) {
+            float q[4];
+            load4<VEC>(st.q[j], x0, V, q);
+            const double is = st.inv_S[j];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const double r = p[k] - (double)q[k];
+                p[k] = (r > 0.0 ? r : 0.0) * is;
+            }
+        }
+    }
+}
+
+// sum_x max(0, p^(n)(x) - q(x)) (q == nullptr: sum_x p^(n)(x)), 8 tokens per
+// thread per iteration as two groups of four.
+template <bool VEC>
+__device__ double bulk_mass(const float *__restrict__ row, const float *__restrict__ q, int V,
+                            const RowState &st, const double *table, double *sh)
+{
+    double s = 0.0;
+    for (int x0 = 4 * threadIdx.x; x0 < V; x0 += 8 * kRowThreads) {
+        const int x1 = x0 + 4 * kRowThreads;
+        double p0[4], p1[4];
+        p_bulk4<VEC>(row, x0, V, st, table, p0);
+        p_bulk4<VEC>(row, x1, V, st, table, p1);
+        if (q) {
+            float q0[4], q1[4];
+            load4<VEC>(q, x0, V, q0);
+            load4<VEC>(q, x1, V, q1);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const double d0 = p0[k] - (double)q0[k], d1 = p1[k] - (double)q1[k];
+                s += (d0 > 0.0 ? d0 : 0.0) + (d1 > 0.0 ? d1 : 0.0);
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                s += p0[k] + p1[k];
+        }
+    }
+    return block_sum(s, sh);
+}
+
+// p^(n)(x) for one acceptance test: the exact fp64 formula of the definition.
+__device__ __forceinline__ double p_exact(float lx, int x, const RowState &st)
+{
+    double p = exp(((double)lx - st.m) / st.temp) / st.Z;
+    for (int j = 0; j < st.n; ++j) {
+        if (st.S[j] > 0.0) {
+            const double r = p - (double)st.q[j][x];
+            p = (r > 0.0 ? r : 0.0) / st.S[j];
         }
     }
     return p;
 }
 
-// sum_x max(0, p^(n)(x) - q(x))
-__device__ double residual_mass(const float *__restrict__ row, const float *__restrict__ q, int V,
-                                double m, double temp, double Z, const Residual &res,
-                                double *sh)
+// Inverse-CDF draw from p^(n): the smallest x whose ascending cumulative sum
+// exceeds u (fp64 block scan in tiles of 4 * kRowThreads tokens); if rounding
+// leaves none, the largest x with p(x) > 0.
+template <bool VEC>
+__device__ int residual_draw(const float *__restrict__ row, int V, const RowState &st,
+                             const double *table, double u, int *shi)
 {
-    double s = 0.0;
-    for (int x = threadIdx.x; x < V; x += kRowThreads) {
-        const double r = residual_p(__ldg(row + x), m, temp, Z, res, x) - (double)__ldg(q + x);
-        s += r > 0.0 ? r : 0.0;
+    __shared__ double warp_tot[kWarps];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    double carry = 0.0;
+    int last_pos = -1;
+    for (int base = 0; base < V; base += 4 * kRowThreads) {
+        const int x0 = base + 4 * threadIdx.x;
+        double p[4];
+        p_bulk4<VEC>(row, x0, V, st, table, p);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            if (p[k] > 0.0)
+                last_pos = x0 + k;
+        const double mine = ((p[0] + p[1]) + p[2]) + p[3];
+        double incl = mine;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const double y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o)
+                incl += y;
+        }
+        if (lane == 31)
+            warp_tot[warp] = incl;
+        __syncthreads();
+        double wbase = 0.0, tile = 0.0;
+        for (int w2 = 0; w2 < kWarps; ++w2) {
+            const double t = warp_tot[w2];
+            if (w2 < warp)
+                wbase += t;
+            tile += t;
+        }
+        double C = carry + wbase + (incl - mine);
+        int found = INT_MAX;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            C += p[k];
+            if (found == INT_MAX && x0 + k < V && C > u)
+                found = x0 + k;
+        }
+        found = block_min_int<kRowThreads>(found, shi);
+        if (found != INT_MAX)
+            return found;
+        carry += tile;
     }
-    return block_sum(s, sh);
+    return block_max_int<kRowThreads>(last_pos, shi);
 }
 
 __device__ __forceinline__ bool sequence_ok(const int32_t *n_nodes, const int32_t *first_child,
@@ -276,12 +421,13 @@ __global__ void __launch_bounds__(kRowThreads)
         return;
     if (first_child[(size_t)b * (Tmax + 1) + r] < 0)
         return;   // leaf: its argmax is needed only if it ends the path
-    const int a = row_argmax(logits + ((size_t)b * (Tmax + 1) + r) * V, V, shv, shi);
+    const int a =
+        row_argmax<kRowThreads>(logits + ((size_t)b * (Tmax + 1) + r) * V, V, shv, shi);
     if (threadIdx.x == 0)
         argmax_ws[(size_t)b * (Tmax + 1) + r] = a;
 }
 
-__global__ void __launch_bounds__(kRowThreads)
+__global__ void __launch_bounds__(kFinThreads)
     greedy_finalize_kernel(const float *__restrict__ logits, const int32_t *__restrict__ tokens,
                            const int32_t *__restrict__ parent,
                            const int32_t *__restrict__ n_nodes,
@@ -291,9 +437,10 @@ __global__ void __launch_bounds__(kRowThreads)
                            int32_t *__restrict__ out_path, int32_t *__restrict__ n_accepted,
                            int32_t *dev_status)
 {
+    constexpr int NW = kFinThreads / 32;
     __shared__ uint32_t matched[kMaskWords];
-    __shared__ float shv[kWarps];
-    __shared__ int shi[kWarps];
+    __shared__ float shv[NW];
+    __shared__ int shi[NW];
     const int b = blockIdx.x, u = threadIdx.x;
     const int W = (Tmax + 31) / 32;
     int T;
@@ -336,7 +483,7 @@ __global__ void __launch_bounds__(kRowThreads)
         if (full)
             key = (len << 8) | (255 - u);
     }
-    key = block_max_int(key, shi);
+    key = block_max_int<kFinThreads>(key, shi);
     const int t = key >= 0 ? 255 - (key & 255) : -1;
     const int n = key >= 0 ? key >> 8 : 0;
     if (t >= 0 && u < T) {
@@ -355,7 +502,8 @@ __global__ void __launch_bounds__(kRowThreads)
     if (first_child[(size_t)b * (Tmax + 1) + row] >= 0)
         bonus = argmax_ws[(size_t)b * (Tmax + 1) + row];
     else
-        bonus = row_argmax(logits + ((size_t)b * (Tmax + 1) + row) * V, V, shv, shi);
+        bonus = row_argmax<kFinThreads>(logits + ((size_t)b * (Tmax + 1) + row) * V, V, shv,
+                                        shi);
     if (u == 0) {
         out_tokens[(size_t)b * (Tmax + 1) + n] = bonus;
         n_accepted[b] = n;
@@ -363,33 +511,47 @@ __global__ void __launch_bounds__(kRowThreads)
 }
 
 // -------------------------------------------------------------- stochastic
+// VEC: V % 4 == 0, so every logits / q row is 16-byte aligned (the entry
+// point checks the base pointers) and the bulk passes use float4 loads.
+template <bool VEC>
 __global__ void __launch_bounds__(kRowThreads)
     mss_rows_kernel(const float *__restrict__ logits, double temp,
                     const float *__restrict__ q_probs, int Rq, const int32_t *__restrict__ q_row,
                     const int32_t *__restrict__ tokens, const int32_t *__restrict__ n_nodes,
                     const int32_t *__restrict__ first_child,
                     const int32_t *__restrict__ next_sibling,
-                    const double *__restrict__ u_accept, int Tmax, int V, VerifyWs ws)
+                    const double *__restrict__ u_accept, const double *__restrict__ u_sample,
+                    int Tmax, int V, VerifyWs ws)
 {
+    __shared__ double table[64];
     __shared__ float shf[kWarps];
     __shared__ double shd[kWarps];
-    __shared__ Residual res;
+    __shared__ int shi[kWarps];
+    __shared__ RowState st;
     __shared__ int decision;
     const int r = blockIdx.x, b = blockIdx.y;
     int T;
     if (!sequence_ok(n_nodes, first_child, b, Tmax, T) || r > T)
         return;
-    int c = first_child[(size_t)b * (Tmax + 1) + r];
-    if (c < 0)
-        return;
+    fill_exp_table(table);
     const float *row = logits + ((size_t)b * (Tmax + 1) + r) * V;
-    const float mf = row_max(row, V, shf);
-    const double m = (double)mf;
-    const double Z = row_Z(row, V, m, temp, shd);
-    if (threadIdx.x == 0)
-        res.n = 0;
+    const float mf = row_max(row, V, shf);   // also publishes the table
+    if (threadIdx.x == 0) {
+        st.m = (double)mf;
+        st.inv_temp = 1.0 / temp;
+        st.temp = temp;
+        st.inv_Z = 1.0;   // the first pass sums the unnormalised terms
+        st.n = 0;
+    }
+    __syncthreads();
+    const double Z = bulk_mass<VEC>(row, nullptr, V, st, table, shd);
+    if (threadIdx.x == 0) {
+        st.Z = Z;
+        st.inv_Z = 1.0 / Z;
+    }
     __syncthreads();
     int accepted = -1;
+    int c = first_child[(size_t)b * (Tmax + 1) + r];
     while (c >= 0) {
         const int x = tokens[(size_t)b * Tmax + c];
         const int qr = q_row[(size_t)b * Tmax + c];
@@ -397,7 +559,7 @@ __global__ void __launch_bounds__(kRowThreads)
             break;   // malformed; the finalize kernel reports it
         const float *qc = q_probs + ((size_t)b * Rq + qr) * V;
         if (threadIdx.x == 0) {
-            const double px = residual_p(row[x], m, temp, Z, res, x);
+            const double px = p_exact(row[x], x, st);
             const double qx = (double)qc[x];
             const double u = u_accept[(size_t)b * Tmax + c];
             decision = (px > 0.0 && u * qx <= px) ? 1 : 0;
@@ -407,93 +569,34 @@ __global__ void __launch_bounds__(kRowThreads)
             accepted = c;
             break;
         }
-        const double S = residual_mass(row, qc, V, m, temp, Z, res, shd);
+        const double S = bulk_mass<VEC>(row, qc, V, st, table, shd);
         if (threadIdx.x == 0) {
-            res.q[res.n] = qc;
-            res.S[res.n] = S;
-            res.n += 1;
-            ws.S[(size_t)b * Tmax + c] = S;
+            st.q[st.n] = qc;
+            st.S[st.n] = S;
+            st.inv_S[st.n] = S > 0.0 ? 1.0 / S : 0.0;
+            st.n += 1;
         }
         __syncthreads();
         c = next_sibling[(size_t)b * Tmax + c];
     }
+    int draw = -1;
+    if (accepted < 0)
+        draw = residual_draw<VEC>(row, V, st, table, u_sample[(size_t)b * (Tmax + 1) + r], shi);
     if (threadIdx.x == 0) {
         const size_t i = (size_t)b * (Tmax + 1) + r;
         ws.accepted[i] = accepted;
-        ws.rmax[i] = mf;
-        ws.Z[i] = Z;
+        ws.draw[i] = draw;
     }
 }
 
-// Inverse-CDF draw from p^(n) over the row, fp64 block scan in tiles of
-// 4 * kRowThreads consecutive tokens.
-__device__ int residual_draw(const float *__restrict__ row, int V, double m, double temp, double Z,
-                             const Residual &res, double u, double *shd, int *shi)
-{
-    __shared__ double warp_tot[kWarps];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    double carry = 0.0;
-    int last_pos = -1;
-    for (int base = 0; base < V; base += 4 * kRowThreads) {
-        const int x0 = base + 4 * threadIdx.x;
-        double p[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int x = x0 + k;
-            p[k] = x < V ? residual_p(__ldg(row + x), m, temp, Z, res, x) : 0.0;
-            if (p[k] > 0.0)
-                last_pos = x;
-        }
-        const double mine = ((p[0] + p[1]) + p[2]) + p[3];
-        // inclusive warp scan of the per-thread sums
-        double incl = mine;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const double y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o)
-                incl += y;
-        }
-        if (lane == 31)
-            warp_tot[warp] = incl;
-        __syncthreads();
-        double wbase = 0.0, tile = 0.0;
-        for (int w2 = 0; w2 < kWarps; ++w2) {
-            if (w2 < warp)
-                wbase += warp_tot[w2];
-            tile += warp_tot[w2];
-        }
-        double C = carry + wbase + (incl - mine);
-        int found = INT_MAX;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            C += p[k];
-            if (found == INT_MAX && x0 + k < V && C > u)
-                found = x0 + k;
-        }
-        found = block_min_int(found, shi);
-        if (found != INT_MAX)
-            return found;
-        carry += tile;
-    }
-    return block_max_int(last_pos, shi);
-}
-
-__global__ void __launch_bounds__(kRowThreads)
-    mss_finalize_kernel(const float *__restrict__ logits, double temp,
-                        const float *__restrict__ q_probs, int Rq,
-                        const int32_t *__restrict__ q_row, const int32_t *__restrict__ tokens,
+__global__ void __launch_bounds__(128)
+    mss_finalize_kernel(const int32_t *__restrict__ tokens, const int32_t *__restrict__ q_row,
                         const int32_t *__restrict__ n_nodes,
-                        const int32_t *__restrict__ first_child,
-                        const int32_t *__restrict__ next_sibling,
-                        const double *__restrict__ u_sample, int Tmax, int V, VerifyWs ws,
-                        int32_t *__restrict__ out_tokens, int32_t *__restrict__ out_path,
-                        int32_t *__restrict__ n_accepted, int32_t *dev_status)
+                        const int32_t *__restrict__ first_child, int Rq, int Tmax, int V,
+                        VerifyWs ws, int32_t *__restrict__ out_tokens,
+                        int32_t *__restrict__ out_path, int32_t *__restrict__ n_accepted,
+                        int32_t *dev_status)
 {
-    __shared__ float shf[kWarps];
-    __shared__ double shd[kWarps];
-    __shared__ int shi[kWarps];
-    __shared__ Residual res;
-    __shared__ int term_row, n_path;
     const int b = blockIdx.x, u = threadIdx.x;
     int T;
     if (!sequence_ok(n_nodes, first_child, b, Tmax, T)) {
@@ -519,45 +622,15 @@ __global__ void __launch_bounds__(kRowThreads)
         int row = 0, n = 0;
         while (n < T) {
             const int c = ws.accepted[(size_t)b * (Tmax + 1) + row];
-            if (first_child[(size_t)b * (Tmax + 1) + row] < 0 || c < 0)
+            if (c < 0)
                 break;
             out_path[(size_t)b * Tmax + n] = c;
             out_tokens[(size_t)b * (Tmax + 1) + n] = tokens[(size_t)b * Tmax + c];
             ++n;
             row = c + 1;
         }
-        term_row = row;
-        n_path = n;
-        res.n = 0;
-    }
-    __syncthreads();
-    const int row = term_row;
-    const float *lrow = logits + ((size_t)b * (Tmax + 1) + row) * V;
-    double m, Z;
-    int c = first_child[(size_t)b * (Tmax + 1) + row];
-    if (c >= 0) {
-        // every child was rejected: statistics and normalisers from the row kernel
-        m = (double)ws.rmax[(size_t)b * (Tmax + 1) + row];
-        Z = ws.Z[(size_t)b * (Tmax + 1) + row];
-        if (u == 0) {
-            int n = 0;
-            for (; c >= 0; c = next_sibling[(size_t)b * Tmax + c]) {
-                res.q[n] = q_probs + ((size_t)b * Rq + q_row[(size_t)b * Tmax + c]) * V;
-                res.S[n] = ws.S[(size_t)b * Tmax + c];
-                ++n;
-            }
-            res.n = n;
-        }
-        __syncthreads();
-    } else {
-        m = (double)row_max(lrow, V, shf);
-        Z = row_Z(lrow, V, m, temp, shd);
-    }
-    const double us = u_sample[(size_t)b * (Tmax + 1) + row];
-    const int pick = residual_draw(lrow, V, m, temp, Z, res, us, shd, shi);
-    if (u == 0) {
-        out_tokens[(size_t)b * (Tmax + 1) + n_path] = pick;
-        n_accepted[b] = n_path;
+        out_tokens[(size_t)b * (Tmax + 1) + n] = ws.draw[(size_t)b * (Tmax + 1) + row];
+        n_accepted[b] = n;
     }
 }
 
@@ -566,9 +639,8 @@ __global__ void __launch_bounds__(kRowThreads)
 size_t verify_workspace(int B, int Tmax, int V)
 {
     (void)V;
-    const size_t R = (size_t)B * (Tmax + 1), N = (size_t)B * Tmax;
-    return align256(R * sizeof(double)) + align256(N * sizeof(double)) +
-           align256(R * sizeof(int32_t)) * 2 + align256(R * sizeof(float));
+    const size_t R = (size_t)B * (Tmax + 1);
+    return 3 * align256(R * sizeof(int32_t));
 }
 
 int launch_verify_greedy(const float *logits, const int32_t *tokens, const int32_t *parent,
@@ -584,7 +656,7 @@ int launch_verify_greedy(const float *logits, const int32_t *tokens, const int32
                                                                       first_child, Tmax, V,
                                                                       w.argmax);
     TSD_LAUNCH_CHECK();
-    greedy_finalize_kernel<<<B, kRowThreads, 0, stream>>>(
+    greedy_finalize_kernel<<<B, kFinThreads, 0, stream>>>(
         logits, tokens, parent, n_nodes, mask, first_child, Tmax, V, w.argmax, out_tokens,
         out_path, n_accepted, dev_status);
     TSD_LAUNCH_CHECK();
@@ -602,13 +674,17 @@ int launch_verify_stochastic(const float *logits, double temperature, const floa
     if (B == 0)
         return TSD_OK;
     const VerifyWs w = carve(ws, B, Tmax);
-    mss_rows_kernel<<<dim3(Tmax + 1, B), kRowThreads, 0, stream>>>(
-        logits, temperature, q_probs, Rq, q_row, tokens, n_nodes, first_child, next_sibling,
-        u_accept, Tmax, V, w);
+    if ((V & 3) == 0)
+        mss_rows_kernel<true><<<dim3(Tmax + 1, B), kRowThreads, 0, stream>>>(
+            logits, temperature, q_probs, Rq, q_row, tokens, n_nodes, first_child, next_sibling,
+            u_accept, u_sample, Tmax, V, w);
+    else
+        mss_rows_kernel<false><<<dim3(Tmax + 1, B), kRowThreads, 0, stream>>>(
+            logits, temperature, q_probs, Rq, q_row, tokens, n_nodes, first_child, next_sibling,
+            u_accept, u_sample, Tmax, V, w);
     TSD_LAUNCH_CHECK();
-    mss_finalize_kernel<<<B, kRowThreads, 0, stream>>>(
-        logits, temperature, q_probs, Rq, q_row, tokens, n_nodes, first_child, next_sibling,
-        u_sample, Tmax, V, w, out_tokens, out_path, n_accepted, dev_status);
+    mss_finalize_kernel<<<B, 128, 0, stream>>>(tokens, q_row, n_nodes, first_child, Rq, Tmax, V,
+                                               w, out_tokens, out_path, n_accepted, dev_status);
     TSD_LAUNCH_CHECK();
     return TSD_OK;
 }
