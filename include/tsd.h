@@ -215,9 +215,11 @@ int tsd_tree_verify_stochastic(const float *logits, double temperature, const fl
  * inside the library's device code; every GPU that loads the library holds
  * that array until the process exits.  Nothing is allocated: no cudaMalloc,
  * no cudaFree, no allocating library routine.
- *   - Sizes whose scratch exceeds the array (12 bytes per logits row, i.e.
- *     B * (Tmax + 1) up to about 87000 rows) return TSD_ERR_WORKSPACE and
- *     launch nothing; use tsd_tree_verify_stochastic for those.
+ *   - Sizes whose scratch exceeds the array (tsd_tree_verify_workspace_size:
+ *     about 28 bytes per logits row plus 12 bytes per 4096 vocabulary entries
+ *     per sequence, i.e. B * (Tmax + 1) up to roughly 37000 rows) return
+ *     TSD_ERR_WORKSPACE and launch nothing; use tsd_tree_verify_stochastic
+ *     for those.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call
  *     before any stream capture.

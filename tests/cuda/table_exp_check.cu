@@ -10,8 +10,8 @@
 
 __global__ void eval(const double *x, double *y, double *ref, int n)
 {
-    __shared__ double table[64];
-    tsd::fill_exp_table(table);
+    __shared__ double table[tsd::kExpTable];
+    tsd::fill_exp_table(table, 1.0);
     __syncthreads();
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
         y[i] = tsd::table_exp(x[i], table);

@@ -307,12 +307,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::tmem_ld32(tmem + lane_off + scol + c * 32, sr[c]);
             ptx::tmem_wait_ld();
 
+            // Raw scores (masked ones -inf); the softmax scale (> 0) is applied
+            // inside the exponent's FMA, and to the max once.
             const int pos0 = kb + j * BN;
             float s[BN];
             if (pos0 + BN <= min(P, ke)) {
 #pragma unroll
                 for (int k = 0; k < BN; ++k)
-                    s[k] = __uint_as_float(sr[k >> 5][k & 31]) * scale_log2;
+                    s[k] = __uint_as_float(sr[k >> 5][k & 31]);
             } else {
 #pragma unroll
                 for (int k = 0; k < BN; ++k) {
@@ -322,13 +324,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int v = pos - P;
                         valid = (mask_word(mw, v) >> (v & 31)) & 1u;
                     }
-                    s[k] = valid ? __uint_as_float(sr[k >> 5][k & 31]) * scale_log2 : -INFINITY;
+                    s[k] = valid ? __uint_as_float(sr[k >> 5][k & 31]) : -INFINITY;
                 }
             }
-            float mt = -INFINITY;
+            // Tile max with 8 independent partial maxima (short dependency chains).
+            float mx[8];
 #pragma unroll
-            for (int k = 0; k < BN; ++k)
-                mt = fmaxf(mt, s[k]);
+            for (int i = 0; i < 8; ++i)
+                mx[i] = s[i];
+#pragma unroll
+            for (int k = 8; k < BN; ++k)
+                mx[k & 7] = fmaxf(mx[k & 7], s[k]);
+            const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
+                             scale_log2;
             const bool need = mt > m_run + kRescaleThreshold;   // false if mt is -inf
             const float m_new = need ? mt : m_run;
             const float alpha = need ? ptx::ex2(m_run - m_new) : 1.f;   // 0 when m_run = -inf
@@ -353,22 +362,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             l_run *= alpha;
             m_run = m_new;
-            const float m_use = m_run == -INFINITY ? 0.f : m_run;
-            float lsum = 0.f;
+            const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
+            float lsum[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 uint32_t pk[32];
 #pragma unroll
                 for (int k = 0; k < 32; ++k) {
-                    const float p0 = ptx::ex2(s[c * 64 + 2 * k] - m_use);
-                    const float p1 = ptx::ex2(s[c * 64 + 2 * k + 1] - m_use);
-                    lsum += p0 + p1;
+                    const float p0 = ptx::ex2(fmaf(s[c * 64 + 2 * k], scale_log2, neg_m));
+                    const float p1 = ptx::ex2(fmaf(s[c * 64 + 2 * k + 1], scale_log2, neg_m));
+                    lsum[k & 3] += p0 + p1;
                     pk[k] = ptx::pack_bf16(p0, p1);
                 }
                 ptx::tmem_st32(tmem + lane_off + scol + c * 32, pk);
             }
             ptx::tmem_wait_st();
-            l_run += lsum;
+            l_run += (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
             ptx::tc_fence_before();
             ptx::mbar_arrive(bars.p_full(sb));
         }

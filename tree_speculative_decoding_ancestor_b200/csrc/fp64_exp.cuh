@@ -2,47 +2,50 @@
 //
 // Method: P. T. P. Tang, "Table-driven implementation of the exponential
 // function in IEEE floating-point arithmetic", ACM TOMS 15(2), 1989:
-//   x = n * ln2/64 + r,  |r| <= ln2/128,
-//   e^x = 2^(n >> 6) * 2^((n & 63)/64) * e^r,
-// with 2^(j/64) from a 64-entry table (filled by the caller with CUDA's exp2)
-// and e^r - 1 from its Taylor series to degree 5 (truncation below 4e-17).
-// ln2/64 is split as C_HI + C_LO (C_HI has a 24-bit significand, so n*C_HI
-// is exact for |n| < 2^29; C_LO is the remainder to ~1e-27, computed offline
-// in 80-digit decimal arithmetic), which keeps the reduction error negligible
-// over the whole range.  The relative error stays within a few ulp, far
-// inside what the sums of probabilities need (the tokens are decided by the
-// exact fp64 formula; these sums only set the normalisers and the CDF).
+//   x = n * ln2/128 + r,  |r| <= ln2/256,
+//   e^x = 2^(n >> 7) * 2^((n & 127)/128) * e^r,
+// with 2^(j/128) from a 128-entry table (filled with CUDA's exp2 and
+// pre-multiplied by a per-row factor, so a normalising 1/Z costs nothing)
+// and e^r - 1 from its Taylor series to degree 4 (truncation below 1.3e-15).
+// The reduction is Cody-Waite with ln2/128 split as C_HI + C_LO (C_HI has a
+// 24-bit significand, so n*C_HI is exact for |n| < 2^29; C_LO is the
+// remainder to ~1e-27, computed offline in 80-digit decimal arithmetic), so
+// r is exact to rounding over the whole range.  The relative error stays
+// within a few ulp -- far inside what the sums of probabilities need (tokens
+// are decided by the exact fp64 formula; these sums only set the normalisers
+// and the CDF).
 #pragma once
 
 namespace tsd {
 
-constexpr double kLn2Over64Hi = 0x1.62e43p-7;              // 0.010830424726009369
-constexpr double kLn2Over64Lo = -0x1.05c610ca86c39p-35;     // -2.9760223436840126e-11
-constexpr double kSixtyFourOverLn2 = 92.33248261689366;
+constexpr int kExpTable = 128;
+constexpr double kLn2Over128Hi = 0x1.62e43p-8;              // 0.0054152123630046844
+constexpr double kLn2Over128Lo = -0x1.05c610ca86c39p-36;    // -1.4880111718420063e-11
+constexpr double kOneTwentyEightOverLn2 = 184.66496523378731;
 
-// table[j] = 2^(j/64), j = 0..63.
-__device__ __forceinline__ void fill_exp_table(double *table)
+// table[j] = scale * 2^(j/128), j = 0..127 (all threads of the block help).
+__device__ __forceinline__ void fill_exp_table(double *table, double scale)
 {
-    for (int j = threadIdx.x; j < 64; j += blockDim.x)
-        table[j] = exp2((double)j / 64.0);
+    for (int j = threadIdx.x; j < kExpTable; j += blockDim.x)
+        table[j] = scale * exp2((double)j / (double)kExpTable);
 }
 
+// scale * e^x for x <= 0; 0 for x < -708 (where e^x leaves the normal range).
 __device__ __forceinline__ double table_exp(double x, const double *table)
 {
     if (x < -708.0)
         return 0.0;
-    const double n = rint(x * kSixtyFourOverLn2);
-    const double r = fma(n, -kLn2Over64Lo, fma(n, -kLn2Over64Hi, x));
+    const double n = rint(x * kOneTwentyEightOverLn2);
+    const double r = fma(n, -kLn2Over128Lo, fma(n, -kLn2Over128Hi, x));
     const int ni = (int)n;
-    double p = 1.0 / 120.0;
-    p = fma(p, r, 1.0 / 24.0);
+    double p = 1.0 / 24.0;
     p = fma(p, r, 1.0 / 6.0);
     p = fma(p, r, 0.5);
     p = fma(p, r, 1.0);
     p = p * r;                               // e^r - 1
-    const double t = table[ni & 63];
-    const double y = fma(t, p, t);           // 2^(j/64) * e^r, in [0.99, 2.02]
-    const long long bits = __double_as_longlong(y) + ((long long)(ni >> 6) << 52);
+    const double t = table[ni & (kExpTable - 1)];
+    const double y = fma(t, p, t);           // scale * 2^(j/128) * e^r
+    const long long bits = __double_as_longlong(y) + ((long long)(ni >> 7) << 52);
     return __longlong_as_double(bits);
 }
 

@@ -1,35 +1,38 @@
 // Tree verification from the target model's logits (SpecInfer explainer,
 // section "ツリー検証アルゴリズム").
 //
-// Both verifiers decide every logits row in parallel, then walk:
-//   greedy
-//     greedy_rows_kernel      one CTA per row whose node has children: argmax
-//                             (lowest index on ties), float4 loads, several in
-//                             flight per thread;
-//     greedy_finalize_kernel  one CTA per sequence: nodes whose whole root path
-//                             matches, the deepest (lowest index on ties), and
-//                             the argmax of its row (computed here for a leaf).
-//   stochastic (multi-step speculative sampling)
-//     mss_rows_kernel         one CTA per row (every node and the root):
-//                             m = max l, Z = sum exp((l-m)/T) in fp64; then the
-//                             children in ascending index: child c with token x
-//                             is accepted iff p(x) > 0 and u_c * q_c(x) <= p(x)
-//                             (evaluated by one thread with the exact fp64
-//                             formula); after a rejection the block computes
-//                             S = sum max(0, p - q_c) and p becomes
-//                             max(0, p - q_c)/S.  A row that accepts no child
-//                             (a leaf included) draws its token by inverse CDF
-//                             at u_sample[row], with a tiled fp64 block scan.
-//     mss_finalize_kernel     one CTA per sequence: follows the accepted
-//                             children from the root and emits the path and the
-//                             draw of the row where it stops.
+// greedy
+//   greedy_rows_kernel      one CTA per logits row whose node has children:
+//                           argmax (lowest index on ties), float4 loads, several
+//                           in flight per thread;
+//   greedy_finalize_kernel  one CTA per sequence: the nodes whose whole root
+//                           path matches, the deepest (lowest index on ties),
+//                           and the argmax of its row (computed here for a leaf).
+// stochastic (multi-step speculative sampling)
+//   mss_rows_kernel         one CTA per logits row (every node and the root):
+//                           m = max l and Z = sum exp((l-m)/T) in fp64; for a
+//                           row with children, the children in ascending index:
+//                           child c with token x is accepted iff p(x) > 0 and
+//                           u_c * q_c(x) <= p(x) (one thread, exact fp64
+//                           formula); after a rejection the block computes
+//                           S = sum max(0, p - q_c), and p becomes
+//                           max(0, p - q_c) / S.
+//   mss_chunks_kernel       one CTA per (vocabulary chunk, sequence): follows
+//                           the accepted children from the root to the row where
+//                           the sequence stops and sums that row's final
+//                           distribution over its chunk;
+//   mss_finalize_kernel     one CTA per sequence: emits the path, then draws the
+//                           last token by inverse CDF at u_sample[row] -- the
+//                           chunk whose running sum passes u, then an fp64
+//                           block scan inside that chunk.
 //
 // Residual distributions are never materialised: p^(n)(x) is recomputed per
 // element from the logits row, the rejected siblings' q rows and their
-// normalisers.  The bulk sums (Z, S, the CDF) use a table-driven fp64 exp and
-// reciprocals; the acceptance tests use the exact formula.  Both agree with a
-// sequential fp64 evaluation to ~1e-15 relative, so a decision can only differ
-// when its uniform lies within that distance of the boundary.
+// normalisers.  The bulk sums (Z, S, the CDF) use a table-driven fp64 exp
+// (its table pre-scaled by 1/Z) and reciprocals; the acceptance tests use the
+// exact formula.  Both agree with a sequential fp64 evaluation to ~1e-15
+// relative, so a decision can only differ when its uniform lies within that
+// distance of the boundary.
 #include <climits>
 
 #include "fp64_exp.cuh"
@@ -42,25 +45,44 @@ namespace {
 constexpr int kRowThreads = 512;
 constexpr int kWarps = kRowThreads / 32;
 constexpr int kFinThreads = 1024;
+constexpr int kDrawThreads = 256;
+constexpr int kChunk = 4096;   // vocabulary chunk of the deferred draw (multiple of 4)
 
 struct VerifyWs {
-    int32_t *argmax;    // [B][Tmax+1]  greedy: argmax of rows with children
-    int32_t *accepted;  // [B][Tmax+1]  stochastic: accepted child per row, -1 none
-    int32_t *draw;      // [B][Tmax+1]  stochastic: token drawn where no child is accepted
+    double *Z;            // [B][Tmax+1]  sum exp((l - m)/T)
+    double *S;            // [B][Tmax]    residual normaliser after rejecting child c
+    double *chunk_sum;    // [B][nch]     final distribution summed over a chunk
+    int32_t *argmax;      // [B][Tmax+1]  greedy: argmax of rows with children
+    int32_t *accepted;    // [B][Tmax+1]  accepted child per row, -1 none
+    float *rmax;          // [B][Tmax+1]  row max
+    int32_t *chunk_last;  // [B][nch]     largest token of the chunk with p > 0, or -1
+    int nch;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-VerifyWs carve(void *ws, int B, int Tmax)
+int num_chunks(int V) { return (V + kChunk - 1) / kChunk; }
+
+VerifyWs carve(void *ws, int B, int Tmax, int V)
 {
-    const size_t R = (size_t)B * (Tmax + 1);
+    const size_t R = (size_t)B * (Tmax + 1), N = (size_t)B * Tmax;
+    const size_t C = (size_t)B * num_chunks(V);
     char *p = static_cast<char *>(ws);
     VerifyWs w;
+    w.nch = num_chunks(V);
+    w.Z = reinterpret_cast<double *>(p);
+    p += align256(R * sizeof(double));
+    w.S = reinterpret_cast<double *>(p);
+    p += align256(N * sizeof(double));
+    w.chunk_sum = reinterpret_cast<double *>(p);
+    p += align256(C * sizeof(double));
     w.argmax = reinterpret_cast<int32_t *>(p);
     p += align256(R * sizeof(int32_t));
     w.accepted = reinterpret_cast<int32_t *>(p);
     p += align256(R * sizeof(int32_t));
-    w.draw = reinterpret_cast<int32_t *>(p);
+    w.rmax = reinterpret_cast<float *>(p);
+    p += align256(R * sizeof(float));
+    w.chunk_last = reinterpret_cast<int32_t *>(p);
     return w;
 }
 
@@ -252,8 +274,8 @@ __device__ float row_max(const float *__restrict__ row, int V, float *sh)
 
 // Per-row state of multi-step speculative sampling.
 struct RowState {
-    double m, inv_temp, temp, Z, inv_Z;
-    int n;                         // siblings rejected so far
+    double m, inv_temp, temp, Z;
+    int n;                         // siblings rejected so far (-1: malformed input)
     const float *q[kMaxTree];      // their SSM rows
     double S[kMaxTree];            // their residual normalisers
     double inv_S[kMaxTree];        // 1/S (0 when S == 0: p unchanged)
@@ -278,8 +300,9 @@ __device__ __forceinline__ void load4(const float *__restrict__ p, int x0, int V
     }
 }
 
-// p^(n)(x) for x in [x0, x0+4) (0 beyond V) for the bulk sums: table exp and
-// reciprocals; the loads of each rejected sibling's row are issued together.
+// p^(n)(x) for x in [x0, x0+4) (0 beyond V) for the bulk sums.  `table` is
+// the exp table pre-scaled by 1/Z (by 1 while Z itself is being summed); the
+// loads of each rejected sibling's row are issued together.
 template <bool VEC>
 __device__ __forceinline__ void p_bulk4(const float *__restrict__ row, int x0, int V,
                                         const RowState &st, const double *table, double (&p)[4])
@@ -288,8 +311,7 @@ __device__ __forceinline__ void p_bulk4(const float *__restrict__ row, int x0, i
     load4<VEC>(row, x0, V, l);
 #pragma unroll
     for (int k = 0; k < 4; ++k)
-        p[k] = x0 + k < V ? table_exp(((double)l[k] - st.m) * st.inv_temp, table) * st.inv_Z
-                          : 0.0;
+        p[k] = x0 + k < V ? table_exp(((double)l[k] - st.m) * st.inv_temp, table) : 0.0;
     for (int j = 0; j < st.n; ++j) {
         if (st.S[j] > 0.0) {
             float q[4];
@@ -304,8 +326,8 @@ __device__ __forceinline__ void p_bulk4(const float *__restrict__ row, int x0, i
     }
 }
 
-// sum_x max(0, p^(n)(x) - q(x)) (q == nullptr: sum_x p^(n)(x)), 8 tokens per
-// thread per iteration as two groups of four.
+// sum_x max(0, p^(n)(x) - q(x)) (q == nullptr: sum_x p^(n)(x)), eight tokens
+// per thread per iteration as two groups of four.
 template <bool VEC>
 __device__ double bulk_mass(const float *__restrict__ row, const float *__restrict__ q, int V,
                             const RowState &st, const double *table, double *sh)
@@ -345,59 +367,6 @@ __device__ __forceinline__ double p_exact(float lx, int x, const RowState &st)
         }
     }
     return p;
-}
-
-// Inverse-CDF draw from p^(n): the smallest x whose ascending cumulative sum
-// exceeds u (fp64 block scan in tiles of 4 * kRowThreads tokens); if rounding
-// leaves none, the largest x with p(x) > 0.
-template <bool VEC>
-__device__ int residual_draw(const float *__restrict__ row, int V, const RowState &st,
-                             const double *table, double u, int *shi)
-{
-    __shared__ double warp_tot[kWarps];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    double carry = 0.0;
-    int last_pos = -1;
-    for (int base = 0; base < V; base += 4 * kRowThreads) {
-        const int x0 = base + 4 * threadIdx.x;
-        double p[4];
-        p_bulk4<VEC>(row, x0, V, st, table, p);
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-            if (p[k] > 0.0)
-                last_pos = x0 + k;
-        const double mine = ((p[0] + p[1]) + p[2]) + p[3];
-        double incl = mine;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const double y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o)
-                incl += y;
-        }
-        if (lane == 31)
-            warp_tot[warp] = incl;
-        __syncthreads();
-        double wbase = 0.0, tile = 0.0;
-        for (int w2 = 0; w2 < kWarps; ++w2) {
-            const double t = warp_tot[w2];
-            if (w2 < warp)
-                wbase += t;
-            tile += t;
-        }
-        double C = carry + wbase + (incl - mine);
-        int found = INT_MAX;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            C += p[k];
-            if (found == INT_MAX && x0 + k < V && C > u)
-                found = x0 + k;
-        }
-        found = block_min_int<kRowThreads>(found, shi);
-        if (found != INT_MAX)
-            return found;
-        carry += tile;
-    }
-    return block_max_int<kRowThreads>(last_pos, shi);
 }
 
 __device__ __forceinline__ bool sequence_ok(const int32_t *n_nodes, const int32_t *first_child,
@@ -520,38 +489,43 @@ __global__ void __launch_bounds__(kRowThreads)
                     const int32_t *__restrict__ tokens, const int32_t *__restrict__ n_nodes,
                     const int32_t *__restrict__ first_child,
                     const int32_t *__restrict__ next_sibling,
-                    const double *__restrict__ u_accept, const double *__restrict__ u_sample,
-                    int Tmax, int V, VerifyWs ws)
+                    const double *__restrict__ u_accept, int Tmax, int V, VerifyWs ws)
 {
-    __shared__ double table[64];
+    __shared__ double table[kExpTable];
     __shared__ float shf[kWarps];
     __shared__ double shd[kWarps];
-    __shared__ int shi[kWarps];
     __shared__ RowState st;
     __shared__ int decision;
     const int r = blockIdx.x, b = blockIdx.y;
     int T;
     if (!sequence_ok(n_nodes, first_child, b, Tmax, T) || r > T)
         return;
-    fill_exp_table(table);
+    fill_exp_table(table, 1.0);
     const float *row = logits + ((size_t)b * (Tmax + 1) + r) * V;
-    const float mf = row_max(row, V, shf);   // also publishes the table
+    const float mf = row_max(row, V, shf);   // its barriers also publish the table
     if (threadIdx.x == 0) {
         st.m = (double)mf;
         st.inv_temp = 1.0 / temp;
         st.temp = temp;
-        st.inv_Z = 1.0;   // the first pass sums the unnormalised terms
         st.n = 0;
     }
     __syncthreads();
     const double Z = bulk_mass<VEC>(row, nullptr, V, st, table, shd);
+    const size_t ri = (size_t)b * (Tmax + 1) + r;
     if (threadIdx.x == 0) {
         st.Z = Z;
-        st.inv_Z = 1.0 / Z;
+        ws.rmax[ri] = mf;
+        ws.Z[ri] = Z;
     }
+    int c = first_child[ri];
+    if (c < 0) {
+        if (threadIdx.x == 0)
+            ws.accepted[ri] = -1;
+        return;   // a leaf (or an empty tree's root): it only needs m and Z
+    }
+    fill_exp_table(table, 1.0 / Z);   // bulk_mass ended with a barrier: table is free
     __syncthreads();
     int accepted = -1;
-    int c = first_child[(size_t)b * (Tmax + 1) + r];
     while (c >= 0) {
         const int x = tokens[(size_t)b * Tmax + c];
         const int qr = q_row[(size_t)b * Tmax + c];
@@ -575,62 +549,254 @@ __global__ void __launch_bounds__(kRowThreads)
             st.S[st.n] = S;
             st.inv_S[st.n] = S > 0.0 ? 1.0 / S : 0.0;
             st.n += 1;
+            ws.S[(size_t)b * Tmax + c] = S;
         }
         __syncthreads();
         c = next_sibling[(size_t)b * Tmax + c];
     }
-    int draw = -1;
-    if (accepted < 0)
-        draw = residual_draw<VEC>(row, V, st, table, u_sample[(size_t)b * (Tmax + 1) + r], shi);
+    if (threadIdx.x == 0)
+        ws.accepted[ri] = accepted;
+}
+
+// Thread 0: walk the accepted children from the root (accepted row in shared
+// memory), fill `st` with the final distribution's state at the row where the
+// sequence stops, and return that row; n_out = accepted nodes.  Optionally
+// writes the path.  st.n = -1 if a q row index is malformed.
+__device__ int walk_to_terminal(int b, int T, int Tmax, int Rq, int V, double temp,
+                                const float *__restrict__ q_probs,
+                                const int32_t *__restrict__ q_row,
+                                const int32_t *__restrict__ tokens,
+                                const int32_t *__restrict__ first_child,
+                                const int32_t *__restrict__ next_sibling, const VerifyWs &ws,
+                                const int *acc, RowState &st, int &n_out,
+                                int32_t *__restrict__ out_path, int32_t *__restrict__ out_tokens)
+{
+    int row = 0, n = 0;
+    while (n < T && acc[row] >= 0) {
+        const int c = acc[row];
+        if (out_path) {
+            out_path[(size_t)b * Tmax + n] = c;
+            out_tokens[(size_t)b * (Tmax + 1) + n] = tokens[(size_t)b * Tmax + c];
+        }
+        row = c + 1;
+        ++n;
+    }
+    const size_t ri = (size_t)b * (Tmax + 1) + row;
+    st.m = (double)ws.rmax[ri];
+    st.Z = ws.Z[ri];
+    st.temp = temp;
+    st.inv_temp = 1.0 / temp;
+    st.n = 0;
+    for (int c = first_child[ri]; c >= 0; c = next_sibling[(size_t)b * Tmax + c]) {
+        const int qr = q_row[(size_t)b * Tmax + c];
+        if (qr < 0 || qr >= Rq) {
+            st.n = -1;
+            break;
+        }
+        const double S = ws.S[(size_t)b * Tmax + c];
+        st.q[st.n] = q_probs + ((size_t)b * Rq + qr) * V;
+        st.S[st.n] = S;
+        st.inv_S[st.n] = S > 0.0 ? 1.0 / S : 0.0;
+        st.n += 1;
+    }
+    n_out = n;
+    return row;
+}
+
+template <bool VEC>
+__global__ void __launch_bounds__(kDrawThreads)
+    mss_chunks_kernel(const float *__restrict__ logits, double temp,
+                      const float *__restrict__ q_probs, int Rq,
+                      const int32_t *__restrict__ q_row, const int32_t *__restrict__ tokens,
+                      const int32_t *__restrict__ n_nodes,
+                      const int32_t *__restrict__ first_child,
+                      const int32_t *__restrict__ next_sibling, int Tmax, int V, VerifyWs ws)
+{
+    __shared__ double table[kExpTable];
+    __shared__ double shd[kDrawThreads / 32];
+    __shared__ int shi[kDrawThreads / 32];
+    __shared__ int acc[kMaxTree + 1];
+    __shared__ RowState st;
+    __shared__ int term;
+    const int ch = blockIdx.x, b = blockIdx.y;
+    int T;
+    if (!sequence_ok(n_nodes, first_child, b, Tmax, T))
+        return;
+    for (int i = threadIdx.x; i <= T; i += kDrawThreads)
+        acc[i] = ws.accepted[(size_t)b * (Tmax + 1) + i];
+    __syncthreads();
     if (threadIdx.x == 0) {
-        const size_t i = (size_t)b * (Tmax + 1) + r;
-        ws.accepted[i] = accepted;
-        ws.draw[i] = draw;
+        int n;
+        term = walk_to_terminal(b, T, Tmax, Rq, V, temp, q_probs, q_row, tokens, first_child,
+                                next_sibling, ws, acc, st, n, nullptr, nullptr);
+    }
+    __syncthreads();
+    if (st.n < 0)
+        return;   // malformed; the finalize kernel reports it
+    fill_exp_table(table, 1.0 / st.Z);
+    __syncthreads();
+    const float *row = logits + ((size_t)b * (Tmax + 1) + term) * V;
+    const int x_begin = ch * kChunk, x_end = min(x_begin + kChunk, V);
+    double s = 0.0;
+    int last = -1;
+    for (int x0 = x_begin + 4 * threadIdx.x; x0 < x_end; x0 += 4 * kDrawThreads) {
+        double p[4];
+        p_bulk4<VEC>(row, x0, V, st, table, p);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            s += p[k];
+            if (p[k] > 0.0)
+                last = x0 + k;
+        }
+    }
+    // block reductions over kDrawThreads threads
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    s = warp_sum(s);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
+    if (lane == 0) {
+        shd[warp] = s;
+        shi[warp] = last;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double tot = 0.0;
+        int lst = -1;
+        for (int w2 = 0; w2 < kDrawThreads / 32; ++w2) {
+            tot += shd[w2];
+            lst = max(lst, shi[w2]);
+        }
+        ws.chunk_sum[(size_t)b * ws.nch + ch] = tot;
+        ws.chunk_last[(size_t)b * ws.nch + ch] = lst;
     }
 }
 
-__global__ void __launch_bounds__(128)
-    mss_finalize_kernel(const int32_t *__restrict__ tokens, const int32_t *__restrict__ q_row,
+template <bool VEC>
+__global__ void __launch_bounds__(kDrawThreads)
+    mss_finalize_kernel(const float *__restrict__ logits, double temp,
+                        const float *__restrict__ q_probs, int Rq,
+                        const int32_t *__restrict__ q_row, const int32_t *__restrict__ tokens,
                         const int32_t *__restrict__ n_nodes,
-                        const int32_t *__restrict__ first_child, int Rq, int Tmax, int V,
-                        VerifyWs ws, int32_t *__restrict__ out_tokens,
-                        int32_t *__restrict__ out_path, int32_t *__restrict__ n_accepted,
-                        int32_t *dev_status)
+                        const int32_t *__restrict__ first_child,
+                        const int32_t *__restrict__ next_sibling,
+                        const double *__restrict__ u_sample, int Tmax, int V, VerifyWs ws,
+                        int32_t *__restrict__ out_tokens, int32_t *__restrict__ out_path,
+                        int32_t *__restrict__ n_accepted, int32_t *dev_status)
 {
-    const int b = blockIdx.x, u = threadIdx.x;
+    constexpr int NW = kDrawThreads / 32;
+    __shared__ double table[kExpTable];
+    __shared__ double warp_tot[NW];
+    __shared__ int shi[NW];
+    __shared__ int acc[kMaxTree + 1];
+    __shared__ RowState st;
+    __shared__ int term, n_path, chosen;
+    __shared__ double carry0;
+    const int b = blockIdx.x, tid = threadIdx.x;
+    const int lane = tid & 31, warp = tid >> 5;
     int T;
     if (!sequence_ok(n_nodes, first_child, b, Tmax, T)) {
-        if (u == 0)
+        if (tid == 0)
             n_accepted[b] = -1;
         return;
     }
     int bad = 0;
-    if (u < T) {
-        const int x = tokens[(size_t)b * Tmax + u];
-        const int qr = q_row[(size_t)b * Tmax + u];
+    if (tid < T) {
+        const int x = tokens[(size_t)b * Tmax + tid];
+        const int qr = q_row[(size_t)b * Tmax + tid];
         bad = (x < 0 || x >= V) ? TSD_DEV_BAD_TOKEN : 0;
         bad |= (qr < 0 || qr >= Rq) ? TSD_DEV_BAD_QROW : 0;
     }
     if (__syncthreads_or(bad)) {
         if (bad)
             flag(dev_status, bad);
-        if (u == 0)
+        if (tid == 0)
             n_accepted[b] = -1;
         return;
     }
-    if (u == 0) {
-        int row = 0, n = 0;
-        while (n < T) {
-            const int c = ws.accepted[(size_t)b * (Tmax + 1) + row];
-            if (c < 0)
+    for (int i = tid; i <= T; i += kDrawThreads)
+        acc[i] = ws.accepted[(size_t)b * (Tmax + 1) + i];
+    __syncthreads();
+    if (tid == 0) {
+        int n;
+        term = walk_to_terminal(b, T, Tmax, Rq, V, temp, q_probs, q_row, tokens, first_child,
+                                next_sibling, ws, acc, st, n, out_path, out_tokens);
+        n_path = n;
+        // The chunk whose running sum passes u.
+        const double u = u_sample[(size_t)b * (Tmax + 1) + term];
+        double C = 0.0;
+        int pick = -1;
+        for (int c = 0; c < ws.nch; ++c) {
+            const double s = ws.chunk_sum[(size_t)b * ws.nch + c];
+            if (C + s > u) {
+                pick = c;
                 break;
-            out_path[(size_t)b * Tmax + n] = c;
-            out_tokens[(size_t)b * (Tmax + 1) + n] = tokens[(size_t)b * Tmax + c];
-            ++n;
-            row = c + 1;
+            }
+            C += s;
         }
-        out_tokens[(size_t)b * (Tmax + 1) + n] = ws.draw[(size_t)b * (Tmax + 1) + row];
-        n_accepted[b] = n;
+        chosen = pick;
+        carry0 = C;
+    }
+    __syncthreads();
+    const double u = u_sample[(size_t)b * (Tmax + 1) + term];
+    int token;
+    if (chosen < 0) {
+        // Rounding left the total at or below u: the largest token with p > 0.
+        int last = -1;
+        for (int c = tid; c < ws.nch; c += kDrawThreads)
+            last = max(last, ws.chunk_last[(size_t)b * ws.nch + c]);
+        token = block_max_int<kDrawThreads>(last, shi);
+    } else {
+        fill_exp_table(table, 1.0 / st.Z);
+        __syncthreads();
+        const float *row = logits + ((size_t)b * (Tmax + 1) + term) * V;
+        const int x_begin = chosen * kChunk, x_end = min(x_begin + kChunk, V);
+        double carry = carry0;
+        token = INT_MAX;
+        for (int base = x_begin; base < x_end; base += 4 * kDrawThreads) {
+            const int x0 = base + 4 * tid;
+            double p[4] = {0.0, 0.0, 0.0, 0.0};
+            if (x0 < x_end)
+                p_bulk4<VEC>(row, x0, V, st, table, p);
+            const double mine = ((p[0] + p[1]) + p[2]) + p[3];
+            double incl = mine;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const double y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o)
+                    incl += y;
+            }
+            if (lane == 31)
+                warp_tot[warp] = incl;
+            __syncthreads();
+            double wbase = 0.0, tile = 0.0;
+            for (int w2 = 0; w2 < NW; ++w2) {
+                const double t = warp_tot[w2];
+                if (w2 < warp)
+                    wbase += t;
+                tile += t;
+            }
+            double C = carry + wbase + (incl - mine);
+            int found = INT_MAX;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                C += p[k];
+                if (found == INT_MAX && x0 + k < x_end && C > u)
+                    found = x0 + k;
+            }
+            found = block_min_int<kDrawThreads>(found, shi);
+            if (found != INT_MAX) {
+                token = found;
+                break;
+            }
+            carry += tile;
+        }
+        if (token == INT_MAX)   // the chunk's own total fell short by rounding
+            token = ws.chunk_last[(size_t)b * ws.nch + chosen];
+    }
+    if (tid == 0) {
+        out_tokens[(size_t)b * (Tmax + 1) + n_path] = token;
+        n_accepted[b] = n_path;
     }
 }
 
@@ -638,9 +804,11 @@ __global__ void __launch_bounds__(128)
 
 size_t verify_workspace(int B, int Tmax, int V)
 {
-    (void)V;
-    const size_t R = (size_t)B * (Tmax + 1);
-    return 3 * align256(R * sizeof(int32_t));
+    const size_t R = (size_t)B * (Tmax + 1), N = (size_t)B * Tmax;
+    const size_t C = (size_t)B * num_chunks(V);
+    return align256(R * sizeof(double)) + align256(N * sizeof(double)) +
+           align256(C * sizeof(double)) + 3 * align256(R * sizeof(int32_t)) +
+           align256(C * sizeof(int32_t));
 }
 
 int launch_verify_greedy(const float *logits, const int32_t *tokens, const int32_t *parent,
@@ -651,7 +819,7 @@ int launch_verify_greedy(const float *logits, const int32_t *tokens, const int32
 {
     if (B == 0)
         return TSD_OK;
-    const VerifyWs w = carve(ws, B, Tmax);
+    const VerifyWs w = carve(ws, B, Tmax, V);
     greedy_rows_kernel<<<dim3(Tmax + 1, B), kRowThreads, 0, stream>>>(logits, n_nodes,
                                                                       first_child, Tmax, V,
                                                                       w.argmax);
@@ -673,18 +841,35 @@ int launch_verify_stochastic(const float *logits, double temperature, const floa
 {
     if (B == 0)
         return TSD_OK;
-    const VerifyWs w = carve(ws, B, Tmax);
-    if ((V & 3) == 0)
-        mss_rows_kernel<true><<<dim3(Tmax + 1, B), kRowThreads, 0, stream>>>(
+    const VerifyWs w = carve(ws, B, Tmax, V);
+    const bool vec = (V & 3) == 0;
+    const dim3 rows(Tmax + 1, B), chunks(w.nch, B);
+    if (vec)
+        mss_rows_kernel<true><<<rows, kRowThreads, 0, stream>>>(
             logits, temperature, q_probs, Rq, q_row, tokens, n_nodes, first_child, next_sibling,
-            u_accept, u_sample, Tmax, V, w);
+            u_accept, Tmax, V, w);
     else
-        mss_rows_kernel<false><<<dim3(Tmax + 1, B), kRowThreads, 0, stream>>>(
+        mss_rows_kernel<false><<<rows, kRowThreads, 0, stream>>>(
             logits, temperature, q_probs, Rq, q_row, tokens, n_nodes, first_child, next_sibling,
-            u_accept, u_sample, Tmax, V, w);
+            u_accept, Tmax, V, w);
     TSD_LAUNCH_CHECK();
-    mss_finalize_kernel<<<B, 128, 0, stream>>>(tokens, q_row, n_nodes, first_child, Rq, Tmax, V,
-                                               w, out_tokens, out_path, n_accepted, dev_status);
+    if (vec)
+        mss_chunks_kernel<true><<<chunks, kDrawThreads, 0, stream>>>(
+            logits, temperature, q_probs, Rq, q_row, tokens, n_nodes, first_child, next_sibling,
+            Tmax, V, w);
+    else
+        mss_chunks_kernel<false><<<chunks, kDrawThreads, 0, stream>>>(
+            logits, temperature, q_probs, Rq, q_row, tokens, n_nodes, first_child, next_sibling,
+            Tmax, V, w);
+    TSD_LAUNCH_CHECK();
+    if (vec)
+        mss_finalize_kernel<true><<<B, kDrawThreads, 0, stream>>>(
+            logits, temperature, q_probs, Rq, q_row, tokens, n_nodes, first_child, next_sibling,
+            u_sample, Tmax, V, w, out_tokens, out_path, n_accepted, dev_status);
+    else
+        mss_finalize_kernel<false><<<B, kDrawThreads, 0, stream>>>(
+            logits, temperature, q_probs, Rq, q_row, tokens, n_nodes, first_child, next_sibling,
+            u_sample, Tmax, V, w, out_tokens, out_path, n_accepted, dev_status);
     TSD_LAUNCH_CHECK();
     return TSD_OK;
 }
