@@ -58,6 +58,47 @@ def num_threads() -> int:
     return int(_load().oracle_num_threads())
 
 
+class use_library:
+    """Context manager: route every oracle call to another build of the oracle
+    source (the mutation tests plant mistakes in a copy and check that the
+    pins catch them)."""
+
+    def __init__(self, path: str):
+        self.path = path
+        self.saved: Optional[ctypes.CDLL] = None
+
+    def __enter__(self):
+        global _lib
+        _load()
+        with _lock:
+            self.saved = _lib
+            lib = ctypes.CDLL(self.path)
+            lib.oracle_num_threads.restype = ctypes.c_int
+            _lib = lib
+        return self
+
+    def __exit__(self, *exc):
+        global _lib
+        with _lock:
+            _lib = self.saved
+        return False
+
+
+def build_variant(source: str, out_path: str) -> str:
+    """Compile oracle C source text (same flags as build()) to out_path."""
+    src = out_path + ".c"
+    with open(src, "w") as f:
+        f.write(source)
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fPIC",
+                           "-shared", "-o", out_path, src, "-lm"])
+    return out_path
+
+
+def source() -> str:
+    with open(_SRC) as f:
+        return f.read()
+
+
 def _np(t, dtype=None) -> np.ndarray:
     """Contiguous numpy view of a CPU tensor/array (bf16 as raw uint16 bits)."""
     if isinstance(t, torch.Tensor):

@@ -1,0 +1,77 @@
+"""Plant plausible mistakes in the oracle and check that its pins catch them
+(CPU only).
+
+Each case copies oracle/tsd_oracle.c, applies one textual change that a
+careless implementation of the pages could contain, compiles the copy, routes
+the oracle through it and runs the pin that should fail.  A mutation that no
+pin detects would mean the oracle is not pinned where it matters.
+"""
+
+import pytest
+
+import oracle
+import test_oracle_attention as pa
+import test_oracle_greedy as pg
+import test_oracle_mask as pm
+import test_oracle_stochastic as ps
+
+MUTATIONS = {
+    # attention (SpecInfer explainer, "トークンツリー構造の仕組み")
+    "prefix_not_attended": ("int P = prefix_len[b];", "int P = 0;",
+                            lambda: pa.test_chain_equals_causal_attention("f32", 4)),
+    "node_not_in_own_S_u": ("int n = P + np;", "int n = P + np - 1;",
+                            pa.test_single_node_is_decode_attention),
+    "gqa_head_mapping": ("int G = Hq / Hkv, hk = h / G;", "int G = Hq / Hkv, hk = h % Hkv;",
+                         lambda: pa.test_chain_equals_causal_attention("bf16", 4)),
+    "softmax_scale_dropped": ("s *= scale;", "s *= 1.0;",
+                              lambda: pa.test_every_node_is_causal_attention_over_its_path(0)),
+    "value_of_wrong_position": ("size_t voff = (kvbase + pos) * D;",
+                                "size_t voff = (kvbase + (pos > 0 ? pos - 1 : 0)) * D;",
+                                lambda: pa.test_every_node_is_causal_attention_over_its_path(1)),
+    # ancestor mask
+    "depth_off_by_one": ("dp[u] = d;", "dp[u] = d - 1;",
+                         lambda: pm.test_mask_vs_subtree_enumeration(4)),
+    "mask_misses_self": ("for (int v = u; v >= 0; v = par[v]) {\n                mk",
+                         "for (int v = par[u]; v >= 0; v = par[v]) {\n                mk",
+                         pm.test_merge_diagram_golden),
+    # greedy (ツリー検証アルゴリズム, greedy)
+    "argmax_ties_to_highest": ("if (l[i] > l[best])", "if (l[i] >= l[best])",
+                               lambda: [pg.test_greedy_vs_exhaustive_search(s) for s in range(8)]),
+    "greedy_ignores_ancestors": ("int parent_ok = p < 0 ? 1 : matched[p];", "int parent_ok = 1;",
+                                 lambda: [pg.test_greedy_vs_exhaustive_search(s)
+                                          for s in range(8)]),
+    "greedy_first_not_longest": ("if (matched[u] && len[u] > best_len) {",
+                                 "if (matched[u] && best < 0) {",
+                                 lambda: [pg.test_greedy_vs_exhaustive_search(s)
+                                          for s in range(8)]),
+    # stochastic (ツリー検証アルゴリズム, P_accept and P_residual)
+    "no_residual_update": ("if (S > 0.0)\n", "if (0)\n",
+                           lambda: ps.test_exact_enumeration_equals_target(16, 2, 1.0)),
+    "residual_not_normalised": ("p[i] = (r > 0.0 ? r : 0.0) / S;", "p[i] = (r > 0.0 ? r : 0.0);",
+                                lambda: ps.test_exact_enumeration_equals_target(6, 3, 0.7)),
+    "accept_ignores_ssm_prob": ("if (px > 0.0 && u * qx <= px) {", "if (px > 0.0 && u <= px) {",
+                                lambda: ps.test_exact_enumeration_equals_target(16, 1, 1.3)),
+    "temperature_ignored": ("- m) / temperature)", "- m) / 1.0)",
+                            lambda: ps.test_no_tree_draw_is_inverse_cdf(0.5)),
+    "child_uses_root_row": ("int row = cur + 1;", "int row = 0;", ps.test_chi_square_depth_two),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pin_catches_mutation(name, tmp_path):
+    old, new, pin = MUTATIONS[name]
+    src = oracle.source()
+    assert src.count(old) >= 1, f"mutation anchor not found: {old!r}"
+    lib = oracle.build_variant(src.replace(old, new), str(tmp_path / f"{name}.so"))
+    with oracle.use_library(lib):
+        with pytest.raises(AssertionError):
+            pin()
+
+
+def test_unmutated_source_passes_the_same_pins(tmp_path):
+    lib = oracle.build_variant(oracle.source(), str(tmp_path / "same.so"))
+    with oracle.use_library(lib):
+        pa.test_chain_equals_causal_attention("f32", 4)
+        pm.test_mask_vs_subtree_enumeration(4)
+        pg.test_greedy_vs_exhaustive_search(0)
+        ps.test_exact_enumeration_equals_target(16, 2, 1.0)
