@@ -5,26 +5,36 @@
 // S_u = committed prefix + the node's ancestors-or-self) for bf16 inputs with
 // head_dim 128.
 //
-// Work unit = (row block, (b, KV head), KV split).  The query rows of one KV
-// head are packed GQA-style, r = u * G + g, so a 128-row block is a dense
-// [128 x 128] A operand no matter how the tree and the head group split it.
-// Per key tile of 128 positions:
-//     S   = Q K^T           tcgen05.mma, A = Q (smem), B = K tile (smem, TMA),
-//                           fp32 accumulator in TMEM (two S buffers ping-pong)
+// The query rows of one KV head are packed GQA-style, r = u * G + g, so a
+// block of 128 rows is one dense [128 x 128] A operand however the tree and
+// the head group divide it.  Per key tile of 128 positions:
+//     S   = Q K^T      tcgen05.mma, A = Q (smem), B = K tile (smem, TMA),
+//                      fp32 accumulator in TMEM
 //     P   = 2^(S*scale*log2e - m)   softmax warps: TMEM -> registers, ancestor
-//                           mask (only on the tiles that reach the tree), online
-//                           max/sum, P packed to bf16 and stored back into the
-//                           S buffer's TMEM columns
-//     O  += P V             tcgen05.mma with A = P read from TMEM and B = the V
-//                           tile (smem, MN-major), O accumulated in TMEM
-// The running max is only raised (and O rescaled) when a tile's max exceeds it
-// by more than 2^8, which keeps O rescales rare while P stays < 256.
+//                      mask only on tiles that reach the tree (one 32-bit
+//                      visibility word per 32 keys), online max/sum, P packed
+//                      to bf16 and written back over the S columns
+//     O  += P V        tcgen05.mma with A = P from TMEM, B = V tile (MN-major)
+// The running max is only raised (O rescaled in TMEM) when a tile exceeds it
+// by more than 2^8, so rescales are rare while P stays below 256.  One
+// exponential in four is evaluated on the FMA pipe (ptx::exp2_fma), the other
+// three on MUFU.  Cache rows at or beyond P_b + T_b are zeroed in shared
+// memory before the PV product, so garbage there (NaN included) never leaks.
 //
-// Warp roles (192 threads): warp 0 issues TMA loads of K and V into two
-// separate rings, warp 1 owns TMEM and issues the MMAs (one elected lane),
-// warps 2-5 run the softmax, one query row per thread (TMEM lane = row).
-// Every mbarrier wait is bounded: after ~2 s it raises a CTA-wide abort flag,
-// reports TSD_DEV_TIMEOUT and the CTA unwinds, frees its TMEM and exits.
+// Two kernels share this machinery:
+//   * tree_attn_rows_kernel (packed blocks of more than 128 rows): one CTA per
+//     (128-row block, (b, KV head), KV split); 6 warps -- TMA producer, MMA
+//     issuer, 4 softmax warps; TMEM holds two S buffers (so the next tile's
+//     scores are ready while the softmax works) and O.
+//   * tree_attn_keysplit_kernel (at most 128 rows, e.g. MHA with small
+//     trees, where the KV stream is the bound): one CTA per ((b, KV head),
+//     split); two 4-warp softmax groups take the even and odd key tiles of
+//     the same query tile, each with its own S and O in TMEM, and their
+//     (O, m, l) are merged by log-sum-exp at the end -- twice the softmax
+//     throughput per KV byte.
+// K and V stream through separate TMA rings (128-byte swizzle).  Every
+// mbarrier wait is bounded: after ~2 s it raises a CTA-wide abort flag, the
+// CTA reports TSD_DEV_TIMEOUT, unwinds, frees its TMEM and exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -42,28 +52,30 @@ int launch_combine(int dtype, int D, const float *part_o, const float2 *part_ml,
 
 namespace {
 
-constexpr int BM = 128;        // query rows per CTA
+constexpr int BQ = 128;        // query rows per tile
 constexpr int BN = 128;        // keys per tile
 constexpr int HD = 128;        // head dim
 constexpr int NSK = 3;         // K ring stages
 constexpr int NSV = 2;         // V ring stages
-constexpr int kThreads = 192;  // 6 warps
 constexpr uint32_t kSub = BN * 128;          // [128 rows][64 bf16] sub-tile, 16 KB
 constexpr uint32_t kTile = 2 * kSub;         // [128][128] bf16, 32 KB
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kOffQ + kTile;
 constexpr uint32_t kOffV = kOffK + NSK * kTile;
 constexpr uint32_t kOffBar = kOffV + NSV * kTile;
-constexpr int kNumBars = 1 + 2 * NSK + 2 * NSV + 2 + 2 + 1;
+constexpr int kNumBars = 1 + 2 * NSK + 2 * NSV + 2 + 4 + 2;
 constexpr uint32_t kOffMisc = kOffBar + 8 * kNumBars;
-constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;   // + alignment slack
+constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;   // + alignment slack
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+constexpr int kRowsThreads = 192;       // rows kernel: 6 warps
+constexpr int kSplitThreads = 384;      // key-split kernel: 12 warps
 
 // mbarrier addresses: q_full, k_full[NSK], k_empty[NSK], v_full[NSV],
-// v_empty[NSV], s_full[2], p_full[2], o_ready -- consecutive 8-byte words.
+// v_empty[NSV], s_full[2], p_full[4], o_ready[2] -- consecutive 8-byte words.
 struct Bars {
     uint32_t base;
     __device__ uint32_t q_full() const { return base; }
@@ -73,7 +85,7 @@ struct Bars {
     __device__ uint32_t v_empty(int s) const { return base + 8u * (1 + 2 * NSK + NSV + s); }
     __device__ uint32_t s_full(int i) const { return base + 8u * (1 + 2 * NSK + 2 * NSV + i); }
     __device__ uint32_t p_full(int i) const { return base + 8u * (3 + 2 * NSK + 2 * NSV + i); }
-    __device__ uint32_t o_ready() const { return base + 8u * (5 + 2 * NSK + 2 * NSV); }
+    __device__ uint32_t o_ready(int i) const { return base + 8u * (7 + 2 * NSK + 2 * NSV + i); }
 };
 
 // A wait whose outcome is the same on every lane of the warp (the TMEM
@@ -104,8 +116,363 @@ __device__ __forceinline__ uint32_t mask_word(const uint32_t (&mw)[4], int v)
     return v < 32 ? mw[0] : v < 64 ? mw[1] : v < 96 ? mw[2] : mw[3];
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
-    tree_attn_umma_kernel(const __grid_constant__ CUtensorMap tmK,
+// Visibility of the 32 keys pos0 .. pos0 + 31 for one query row: bit k is set
+// iff key pos0 + k is below ke and is either a prefix position (< P) or a
+// tree node on the row's root path (bit pos0 + k - P of the ancestor mask).
+__device__ __forceinline__ uint32_t valid_bits(int pos0, int P, int ke, const uint32_t (&mw)[4])
+{
+    auto low_ones = [](int n) -> uint32_t {
+        return n >= 32 ? 0xffffffffu : (n <= 0 ? 0u : ((1u << n) - 1u));
+    };
+    const uint32_t prefix = low_ones(P - pos0);
+    const int lo = pos0 - P;   // ancestor-mask bit of key pos0
+    uint32_t tree = 0u;
+    if (lo >= 0 && lo < 128) {
+        const int w = lo >> 5, sh = lo & 31;
+        const uint32_t a = mask_word(mw, w * 32);
+        const uint32_t c = w < 3 ? mask_word(mw, w * 32 + 32) : 0u;
+        tree = sh ? (a >> sh) | (c << (32 - sh)) : a;
+    } else if (lo < 0 && lo > -32) {
+        tree = mw[0] << (-lo);
+    }
+    return (prefix | tree) & low_ones(ke - pos0);
+}
+
+// Per-CTA set-up shared by both kernels: 1024-byte aligned carve-up of the
+// dynamic shared memory, barrier initialisation, TMEM allocation (warp 1).
+struct Setup {
+    uint8_t *gbase;
+    uint32_t base, sQ, sK, sV, tmem;
+    Bars bars;
+    volatile int *abort_flag;
+};
+
+__device__ __forceinline__ Setup cta_setup(uint8_t *smem_raw, uint32_t q_arrivals,
+                                           uint32_t p_arrivals)
+{
+    Setup su;
+    const uint32_t raw = ptx::smem_addr(smem_raw);
+    su.base = (raw + 1023u) & ~1023u;
+    su.gbase = smem_raw + (su.base - raw);
+    su.sQ = su.base + kOffQ;
+    su.sK = su.base + kOffK;
+    su.sV = su.base + kOffV;
+    su.bars = Bars{su.base + kOffBar};
+    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(su.gbase + kOffMisc);
+    su.abort_flag = reinterpret_cast<volatile int *>(su.gbase + kOffMisc + 4);
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(su.bars.q_full(), q_arrivals);
+        for (int i = 0; i < NSK; ++i) {
+            ptx::mbar_init(su.bars.k_full(i), 1);
+            ptx::mbar_init(su.bars.k_empty(i), 1);
+        }
+        for (int i = 0; i < NSV; ++i) {
+            ptx::mbar_init(su.bars.v_full(i), 1);
+            ptx::mbar_init(su.bars.v_empty(i), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(su.bars.s_full(i), 1);
+            ptx::mbar_init(su.bars.o_ready(i), 1);
+        }
+        for (int i = 0; i < 4; ++i)
+            ptx::mbar_init(su.bars.p_full(i), p_arrivals);
+        *su.abort_flag = 0;
+        ptx::fence_barrier_init();
+        ptx::fence_proxy_async_smem();
+    }
+    if ((threadIdx.x >> 5) == 1) {
+        ptx::tmem_alloc(ptx::smem_addr((const void *)tmem_slot), kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    su.tmem = *tmem_slot;
+    return su;
+}
+
+__device__ __forceinline__ void cta_teardown(const Setup &su, int32_t *dev_status)
+{
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (*su.abort_flag && threadIdx.x == 0)
+        flag(dev_status, TSD_DEV_TIMEOUT);
+    if ((threadIdx.x >> 5) == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(su.tmem, kTmemCols);
+    }
+}
+
+// TMA producer (one lane): K_0, K_1, V_0, K_2, V_1, ... -- the order in which
+// the MMA warp first needs them.
+__device__ __forceinline__ void produce_kv(const Setup &su, const CUtensorMap *tmK,
+                                           const CUtensorMap *tmV, int z, int kb, int ntiles)
+{
+    ptx::prefetch_tmap(tmK);
+    ptx::prefetch_tmap(tmV);
+    for (int i = 0; i <= ntiles; ++i) {
+        if (i < ntiles) {
+            const int s = i % NSK;
+            if (i >= NSK &&
+                !ptx::mbar_wait(su.bars.k_empty(s), ((i / NSK) - 1) & 1, su.abort_flag))
+                break;
+            ptx::mbar_arrive_expect_tx(su.bars.k_full(s), kTile);
+            const uint32_t dst = su.sK + s * kTile;
+            const int pos = kb + i * BN;
+            ptx::tma_load_3d(dst, tmK, 0, pos, z, su.bars.k_full(s));
+            ptx::tma_load_3d(dst + kSub, tmK, 64, pos, z, su.bars.k_full(s));
+        }
+        if (i >= 1) {
+            const int j = i - 1, s = j % NSV;
+            if (j >= NSV &&
+                !ptx::mbar_wait(su.bars.v_empty(s), ((j / NSV) - 1) & 1, su.abort_flag))
+                break;
+            ptx::mbar_arrive_expect_tx(su.bars.v_full(s), kTile);
+            const uint32_t dst = su.sV + s * kTile;
+            const int pos = kb + j * BN;
+            ptx::tma_load_3d(dst, tmV, 0, pos, z, su.bars.v_full(s));
+            ptx::tma_load_3d(dst + kSub, tmV, 64, pos, z, su.bars.v_full(s));
+        }
+    }
+}
+
+// MMA warp, S = Q K^T for key tile `t` into TMEM columns `col_s`.
+__device__ __forceinline__ void issue_qk(const Setup &su, int lane, uint32_t col_s, int t,
+                                         uint32_t s_full)
+{
+    constexpr uint32_t idesc = ptx::idesc_bf16(BQ, BN, false, false);
+    const int st = t % NSK;
+    if (lane == 0) {
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk)
+            ptx::mma_ss(su.tmem + col_s, desc_kmajor(su.sQ, kk),
+                        desc_kmajor(su.sK + st * kTile, kk), idesc, kk > 0 ? 1u : 0u);
+        ptx::mma_commit(s_full);
+        ptx::mma_commit(su.bars.k_empty(st));
+    }
+    __syncwarp();
+}
+
+// MMA warp, O += P V for key tile `t` (P in TMEM columns col_p); zeroes the
+// V rows at or beyond P_b + T_b first.  Returns false on abort.
+__device__ __forceinline__ void issue_pv(const Setup &su, int lane, uint32_t col_p,
+                                         uint32_t col_o, int t, bool accumulate, int first_bad,
+                                         uint32_t o_ready)
+{
+    constexpr uint32_t idesc = ptx::idesc_bf16(BQ, HD, false, true);
+    const int vs = t % NSV;
+    if (first_bad < BN) {
+        uint8_t *vt = su.gbase + kOffV + vs * kTile;
+        for (int row = max(first_bad, 0) + (lane >> 3); row < BN; row += 4) {
+            const int c = lane & 7;
+            *reinterpret_cast<uint4 *>(vt + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4 *>(vt + kSub + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+        }
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+    }
+    ptx::tc_fence_after();
+    if (lane == 0) {
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+            ptx::mma_ts(su.tmem + col_o, su.tmem + col_p + kk * 8, desc_v(su.sV + vs * kTile, kk),
+                        idesc, (accumulate || kk > 0) ? 1u : 0u);
+        ptx::mma_commit(su.bars.v_empty(vs));
+        ptx::mma_commit(o_ready);
+    }
+    __syncwarp();
+}
+
+// Softmax-warp helpers.  Row state of one query row of a tile.
+struct RowCtx {
+    int P, ke;
+    uint32_t mw[4];
+    float scale_log2;
+};
+
+// Q row `t` of the tile -> shared memory, 128-byte swizzled K-major layout.
+__device__ __forceinline__ void load_q_row(const Setup &su, const __nv_bfloat16 *__restrict__ q,
+                                           bool row_ok, size_t q_off, int t)
+{
+    const uint4 *src = reinterpret_cast<const uint4 *>(q + q_off);
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+        const uint4 x = row_ok ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+        const int sub = c >> 3, cc = c & 7;
+        *reinterpret_cast<uint4 *>(su.gbase + kOffQ + sub * kSub + t * 128 +
+                                   ((cc ^ (t & 7)) * 16)) = x;
+    }
+    ptx::fence_proxy_async_smem();
+}
+
+// Rescale this row's O (TMEM columns col_o) by alpha.
+__device__ __forceinline__ void rescale_o(uint32_t taddr_o, float alpha)
+{
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        ptx::tmem_ld32(taddr_o + c * 32, o);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+            o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+        ptx::tmem_st32(taddr_o + c * 32, o);
+    }
+    ptx::tmem_wait_st();
+}
+
+// P = 2^(s * scale - m) for 64 scores (two 32-column chunks already loaded
+// and masked), packed to bf16 into pk[32]; returns their sum.
+__device__ __forceinline__ float exp_pack64(const uint32_t (&sa)[32], const uint32_t (&sb)[32],
+                                            float scale_log2, float neg_m, uint32_t (&pk)[32])
+{
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const float p0 = ptx::ex2(fmaf(__uint_as_float(sa[2 * k]), scale_log2, neg_m));
+        const float p1 = ptx::ex2(fmaf(__uint_as_float(sa[2 * k + 1]), scale_log2, neg_m));
+        const float p2 = ptx::ex2(fmaf(__uint_as_float(sb[2 * k]), scale_log2, neg_m));
+        // one exponential in four on the FMA pipe, three on MUFU
+        const float p3 = ptx::exp2_fma(fmaf(__uint_as_float(sb[2 * k + 1]), scale_log2, neg_m));
+        acc[k & 3] += (p0 + p1) + (p2 + p3);
+        pk[k] = ptx::pack_bf16(p0, p1);
+        pk[16 + k] = ptx::pack_bf16(p2, p3);
+    }
+    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
+__device__ __forceinline__ void mask32(uint32_t (&s)[32], uint32_t bits)
+{
+#pragma unroll
+    for (int k = 0; k < 32; ++k)
+        s[k] = ((bits >> k) & 1u) ? s[k] : __float_as_uint(-INFINITY);
+}
+
+__device__ __forceinline__ float max32x2(const uint32_t (&sa)[32], const uint32_t (&sb)[32],
+                                         float (&mx)[8])
+{
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+        mx[k & 7] = fmaxf(mx[k & 7], __uint_as_float(sa[k]));
+        mx[k & 7] = fmaxf(mx[k & 7], __uint_as_float(sb[k]));
+    }
+    return 0.f;
+}
+
+__device__ __forceinline__ float max8(const float (&mx)[8])
+{
+    return fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+}
+
+// Online-softmax step for one tile whose scores sit in TMEM columns col_s:
+// max, (rare) rescale of O, P over the S columns, running sum.  `wait_o`
+// waits for the previous PV product when O must be rescaled.  Returns false
+// on abort.
+template <typename WaitO>
+__device__ __forceinline__ bool softmax_tile(uint32_t taddr_s, uint32_t taddr_o, int pos0,
+                                             const RowCtx &rc, bool first, float &m_run,
+                                             float &l_run, WaitO wait_o)
+{
+    const bool masked = !(pos0 + BN <= min(rc.P, rc.ke));
+    // max over the raw scores (scale > 0 is applied once), two chunks at a time
+    float mx[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        mx[i] = -INFINITY;
+#pragma unroll 1
+    for (int c2 = 0; c2 < 2; ++c2) {
+        uint32_t sa[32], sb[32];
+        ptx::tmem_ld32(taddr_s + c2 * 64, sa);
+        ptx::tmem_ld32(taddr_s + c2 * 64 + 32, sb);
+        ptx::tmem_wait_ld();
+        if (masked) {
+            mask32(sa, valid_bits(pos0 + c2 * 64, rc.P, rc.ke, rc.mw));
+            mask32(sb, valid_bits(pos0 + c2 * 64 + 32, rc.P, rc.ke, rc.mw));
+        }
+        max32x2(sa, sb, mx);
+    }
+    const float mt = max8(mx) * rc.scale_log2;
+    const bool need = mt > m_run + kRescaleThreshold;   // false if mt is -inf
+    const float m_new = need ? mt : m_run;
+    const float alpha = need ? ptx::ex2(m_run - m_new) : 1.f;   // 0 when m_run = -inf
+    if (__any_sync(0xffffffffu, need) && !first) {
+        if (!wait_o())
+            return false;
+        ptx::tc_fence_after();
+        rescale_o(taddr_o, alpha);
+    }
+    l_run *= alpha;
+    m_run = m_new;
+    // P over the S columns already read: keys 64 c2 .. -> columns 32 c2 ..
+    const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
+    float lsum = 0.f;
+#pragma unroll 1
+    for (int c2 = 0; c2 < 2; ++c2) {
+        uint32_t sa[32], sb[32];
+        ptx::tmem_ld32(taddr_s + c2 * 64, sa);
+        ptx::tmem_ld32(taddr_s + c2 * 64 + 32, sb);
+        ptx::tmem_wait_ld();
+        if (masked) {
+            mask32(sa, valid_bits(pos0 + c2 * 64, rc.P, rc.ke, rc.mw));
+            mask32(sb, valid_bits(pos0 + c2 * 64 + 32, rc.P, rc.ke, rc.mw));
+        }
+        uint32_t pk[32];
+        lsum += exp_pack64(sa, sb, rc.scale_log2, neg_m, pk);
+        ptx::tmem_st32(taddr_s + c2 * 32, pk);
+    }
+    ptx::tmem_wait_st();
+    l_run += lsum;
+    return true;
+}
+
+// Final O row (TMEM) -> output row (bf16, normalised) or split partial (fp32).
+__device__ __forceinline__ void write_row(uint32_t taddr_o, float inv, bool row_ok, size_t row,
+                                          int nsplit, int split, size_t nrows,
+                                          __nv_bfloat16 *__restrict__ out,
+                                          float *__restrict__ part_o, int col0, int ncols)
+{
+    for (int c = 0; c < ncols; c += 32) {
+        uint32_t o[32];
+        ptx::tmem_ld32(taddr_o + c, o);
+        ptx::tmem_wait_ld();
+        if (!row_ok)
+            continue;
+        if (nsplit == 1) {
+            uint4 *dst = reinterpret_cast<uint4 *>(out + row * HD + col0 + c);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                uint4 x;
+                x.x = ptx::pack_bf16(__uint_as_float(o[8 * v + 0]) * inv,
+                                     __uint_as_float(o[8 * v + 1]) * inv);
+                x.y = ptx::pack_bf16(__uint_as_float(o[8 * v + 2]) * inv,
+                                     __uint_as_float(o[8 * v + 3]) * inv);
+                x.z = ptx::pack_bf16(__uint_as_float(o[8 * v + 4]) * inv,
+                                     __uint_as_float(o[8 * v + 5]) * inv);
+                x.w = ptx::pack_bf16(__uint_as_float(o[8 * v + 6]) * inv,
+                                     __uint_as_float(o[8 * v + 7]) * inv);
+                dst[v] = x;
+            }
+        } else {
+            float4 *dst = reinterpret_cast<float4 *>(part_o + ((size_t)split * nrows + row) * HD +
+                                                     col0 + c);
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+                dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv,
+                                     __uint_as_float(o[4 * v + 1]) * inv,
+                                     __uint_as_float(o[4 * v + 2]) * inv,
+                                     __uint_as_float(o[4 * v + 3]) * inv);
+        }
+    }
+}
+
+// ============================================================ rows kernel
+// More than 128 packed rows: one 128-row query tile per CTA, 6 warps (TMA
+// producer, MMA issuer, 4 softmax warps).  The MMA warp computes S for tile
+// j + 1 into the other S buffer while the softmax works on tile j.
+// TMEM: S0 [0,128) | S1 [128,256) | O [256,384).
+__global__ void __launch_bounds__(kRowsThreads, 1)
+    tree_attn_rows_kernel(const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV,
                           const __nv_bfloat16 *__restrict__ q,
                           const int32_t *__restrict__ prefix_len,
@@ -128,315 +495,288 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int R = T * G;
     const int kb = split * keys_per_split;
     const int ke = min(kb + keys_per_split, P + T);
-    if (rb * BM >= R || kb >= ke)
+    if (rb * BQ >= R || kb >= ke)
         return;   // no rows or no keys: the partials stay empty
     const int ntiles = (ke - kb + BN - 1) / BN;
-
-    // 1024-byte aligned carve-up (128-byte swizzle atoms repeat every 1024 B).
-    const uint32_t raw = ptx::smem_addr(smem_raw);
-    const uint32_t base = (raw + 1023u) & ~1023u;
-    uint8_t *gbase = smem_raw + (base - raw);
-    const uint32_t sQ = base + kOffQ, sK = base + kOffK, sV = base + kOffV;
-    const Bars bars{base + kOffBar};
-    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(gbase + kOffMisc);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + kOffMisc + 4);
-
+    const Setup su = cta_setup(smem_raw, BQ, BQ);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (threadIdx.x == 0) {
-        ptx::mbar_init(bars.q_full(), 128);
-        for (int i = 0; i < NSK; ++i) {
-            ptx::mbar_init(bars.k_full(i), 1);
-            ptx::mbar_init(bars.k_empty(i), 1);
-        }
-        for (int i = 0; i < NSV; ++i) {
-            ptx::mbar_init(bars.v_full(i), 1);
-            ptx::mbar_init(bars.v_empty(i), 1);
-        }
-        for (int i = 0; i < 2; ++i) {
-            ptx::mbar_init(bars.s_full(i), 1);
-            ptx::mbar_init(bars.p_full(i), 128);
-        }
-        ptx::mbar_init(bars.o_ready(), 1);
-        *abort_flag = 0;
-        ptx::fence_barrier_init();
-        ptx::fence_proxy_async_smem();
-    }
-    if (warp == 1) {
-        ptx::tmem_alloc(ptx::smem_addr((const void *)tmem_slot), kTmemCols);
-        ptx::tmem_relinquish();
-    }
-    ptx::tc_fence_before();
-    __syncthreads();
-    ptx::tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
+    auto col_s = [](int i) { return (uint32_t)(i & 1) * 128u; };   // S buffer of tile i
+    constexpr uint32_t kO = 256u;
 
     if (warp == 0) {
-        // ------------------------------------------------ TMA producer
-        if (lane == 0) {
-            ptx::prefetch_tmap(&tmK);
-            ptx::prefetch_tmap(&tmV);
-            const int z = b * Hkv + hk;
-            // Order of consumption by the MMA warp: K0, K1, V0, K2, V1, ...
-            for (int i = 0; i <= ntiles; ++i) {
-                if (i < ntiles) {
-                    const int s = i % NSK;
-                    if (i >= NSK &&
-                        !ptx::mbar_wait(bars.k_empty(s), ((i / NSK) - 1) & 1, abort_flag))
-                        break;
-                    ptx::mbar_arrive_expect_tx(bars.k_full(s), kTile);
-                    const uint32_t dst = sK + s * kTile;
-                    const int pos = kb + i * BN;
-                    ptx::tma_load_3d(dst, &tmK, 0, pos, z, bars.k_full(s));
-                    ptx::tma_load_3d(dst + kSub, &tmK, 64, pos, z, bars.k_full(s));
-                }
-                if (i >= 1) {
-                    const int j = i - 1, s = j % NSV;
-                    if (j >= NSV &&
-                        !ptx::mbar_wait(bars.v_empty(s), ((j / NSV) - 1) & 1, abort_flag))
-                        break;
-                    ptx::mbar_arrive_expect_tx(bars.v_full(s), kTile);
-                    const uint32_t dst = sV + s * kTile;
-                    const int pos = kb + j * BN;
-                    ptx::tma_load_3d(dst, &tmV, 0, pos, z, bars.v_full(s));
-                    ptx::tma_load_3d(dst + kSub, &tmV, 64, pos, z, bars.v_full(s));
-                }
-            }
-        }
+        if (lane == 0)
+            produce_kv(su, &tmK, &tmV, b * Hkv + hk, kb, ntiles);
     } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
-        constexpr uint32_t idesc_qk = ptx::idesc_bf16(BM, BN, false, false);
-        constexpr uint32_t idesc_pv = ptx::idesc_bf16(BM, HD, false, true);
-        bool ok = warp_wait(bars.q_full(), 0, abort_flag);
+        // QK_0, then per tile j: QK_{j+1} (other S buffer), PV_j.
+        bool ok = warp_wait(su.bars.q_full(), 0, su.abort_flag);
         ptx::tc_fence_after();
         for (int i = 0; ok && i <= ntiles; ++i) {
             if (i < ntiles) {
-                const int s = i % NSK, sb = i & 1;
-                if (!warp_wait(bars.k_full(s), (i / NSK) & 1, abort_flag)) {
+                if (!warp_wait(su.bars.k_full(i % NSK), (i / NSK) & 1, su.abort_flag)) {
                     ok = false;
                     break;
                 }
                 ptx::tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t d = tmem + (sb ? kColS1 : kColS0);
-#pragma unroll
-                    for (int kk = 0; kk < HD / 16; ++kk)
-                        ptx::mma_ss(d, desc_kmajor(sQ, kk), desc_kmajor(sK + s * kTile, kk),
-                                    idesc_qk, kk > 0 ? 1u : 0u);
-                    ptx::mma_commit(bars.s_full(sb));
-                    ptx::mma_commit(bars.k_empty(s));
-                }
-                __syncwarp();
+                issue_qk(su, lane, col_s(i), i, su.bars.s_full(i & 1));
             }
             if (i >= 1) {
-                const int j = i - 1, pb = j & 1, s = j % NSV;
-                if (!warp_wait(bars.p_full(pb), (j >> 1) & 1, abort_flag) ||
-                    !warp_wait(bars.v_full(s), (j / NSV) & 1, abort_flag)) {
+                const int j = i - 1;
+                if (!warp_wait(su.bars.p_full(j & 1), (j >> 1) & 1, su.abort_flag) ||
+                    !warp_wait(su.bars.v_full(j % NSV), (j / NSV) & 1, su.abort_flag)) {
                     ok = false;
                     break;
                 }
-                ptx::tc_fence_after();
-                // Cache rows at or beyond P + T may hold anything (NaN included):
-                // zero them so that P = 0 there contributes exactly nothing.
-                const int first_bad = P + T - (kb + j * BN);
-                if (first_bad < BN) {
-                    uint8_t *vt = gbase + (sV - base) + s * kTile;
-                    for (int row = max(first_bad, 0) + (lane >> 3); row < BN; row += 4) {
-                        const int c = lane & 7;
-                        *reinterpret_cast<uint4 *>(vt + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
-                        *reinterpret_cast<uint4 *>(vt + kSub + row * 128 + c * 16) =
-                            make_uint4(0, 0, 0, 0);
-                    }
-                    ptx::fence_proxy_async_smem();
-                    __syncwarp();
-                }
-                if (lane == 0) {
-                    const uint32_t a = tmem + (pb ? kColS1 : kColS0);
-#pragma unroll
-                    for (int kk = 0; kk < BN / 16; ++kk)
-                        ptx::mma_ts(tmem + kColO, a + kk * 8, desc_v(sV + s * kTile, kk), idesc_pv,
-                                    (j > 0 || kk > 0) ? 1u : 0u);
-                    ptx::mma_commit(bars.v_empty(s));
-                    ptx::mma_commit(bars.o_ready());
-                }
-                __syncwarp();
+                issue_pv(su, lane, col_s(j), kO, j, j > 0, P + T - (kb + j * BN),
+                         su.bars.o_ready(0));
             }
         }
     } else {
-        // ------------------------------------------------ softmax warps 2..5
+        // softmax warps 2..5: one query row per thread == TMEM lane
         const int quarter = warp & 3;
-        const int t = quarter * 32 + lane;   // row within the block == TMEM lane
+        const int t = quarter * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        const int r = rb * BM + t;
+        const int r = rb * BQ + t;
         const bool row_ok = r < R;
         const int u = row_ok ? r / G : 0;
         const int h = hk * G + (row_ok ? r % G : 0);
-
-        // Q row -> shared memory in the 128-byte swizzled K-major layout.
-        {
-            const uint4 *src = reinterpret_cast<const uint4 *>(
-                q + (((size_t)b * Tmax + u) * Hq + h) * HD);
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                const uint4 x = row_ok ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
-                const int sub = c >> 3, cc = c & 7;
-                *reinterpret_cast<uint4 *>(gbase + kOffQ + sub * kSub + t * 128 +
-                                           ((cc ^ (t & 7)) * 16)) = x;
-            }
-            ptx::fence_proxy_async_smem();
-            ptx::mbar_arrive(bars.q_full());
-        }
-        uint32_t mw[4] = {0u, 0u, 0u, 0u};
+        load_q_row(su, q, row_ok, (((size_t)b * Tmax + u) * Hq + h) * HD, t);
+        ptx::mbar_arrive(su.bars.q_full());
+        uint32_t mw[4];
 #pragma unroll
         for (int w = 0; w < 4; ++w)
-            if (row_ok && w < W)
-                mw[w] = mask[((size_t)b * Tmax + u) * W + w];
-
+            mw[w] = (row_ok && w < W) ? mask[((size_t)b * Tmax + u) * W + w] : 0u;
+        const uint32_t taddr_o = su.tmem + lane_off + kO;
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
-        for (int j = 0; j < ntiles; ++j) {
+        for (int j = 0; ok && j < ntiles; ++j) {
             const int sb = j & 1;
-            const uint32_t scol = sb ? kColS1 : kColS0;
-            if (!warp_wait(bars.s_full(sb), (j >> 1) & 1, abort_flag)) {
+            if (!warp_wait(su.bars.s_full(sb), (j >> 1) & 1, su.abort_flag)) {
                 ok = false;
                 break;
             }
             ptx::tc_fence_after();
+            // all 128 scores of the row in registers at once
+            const uint32_t taddr_s = su.tmem + lane_off + col_s(j);
             uint32_t sr[4][32];
 #pragma unroll
             for (int c = 0; c < 4; ++c)
-                ptx::tmem_ld32(tmem + lane_off + scol + c * 32, sr[c]);
+                ptx::tmem_ld32(taddr_s + c * 32, sr[c]);
             ptx::tmem_wait_ld();
-
-            // Raw scores (masked ones -inf); the softmax scale (> 0) is applied
-            // inside the exponent's FMA, and to the max once.
             const int pos0 = kb + j * BN;
-            float s[BN];
-            if (pos0 + BN <= min(P, ke)) {
+            if (!(pos0 + BN <= min(P, ke))) {   // only where the tree or the range end is
 #pragma unroll
-                for (int k = 0; k < BN; ++k)
-                    s[k] = __uint_as_float(sr[k >> 5][k & 31]);
-            } else {
-#pragma unroll
-                for (int k = 0; k < BN; ++k) {
-                    const int pos = pos0 + k;
-                    bool valid = pos < ke;
-                    if (valid && pos >= P) {
-                        const int v = pos - P;
-                        valid = (mask_word(mw, v) >> (v & 31)) & 1u;
-                    }
-                    s[k] = valid ? __uint_as_float(sr[k >> 5][k & 31]) : -INFINITY;
-                }
+                for (int c = 0; c < 4; ++c)
+                    mask32(sr[c], valid_bits(pos0 + c * 32, P, ke, mw));
             }
-            // Tile max with 8 independent partial maxima (short dependency chains).
             float mx[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i)
-                mx[i] = s[i];
-#pragma unroll
-            for (int k = 8; k < BN; ++k)
-                mx[k & 7] = fmaxf(mx[k & 7], s[k]);
-            const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
-                             scale_log2;
+                mx[i] = -INFINITY;
+            max32x2(sr[0], sr[1], mx);
+            max32x2(sr[2], sr[3], mx);
+            const float mt = max8(mx) * scale_log2;
             const bool need = mt > m_run + kRescaleThreshold;   // false if mt is -inf
             const float m_new = need ? mt : m_run;
             const float alpha = need ? ptx::ex2(m_run - m_new) : 1.f;   // 0 when m_run = -inf
             if (__any_sync(0xffffffffu, need) && j > 0) {
-                // O holds PV_0..PV_{j-1}: wait for the last of them, then rescale.
-                if (!warp_wait(bars.o_ready(), (j - 1) & 1, abort_flag)) {
+                // O holds PV_0 .. PV_{j-1}: wait for the last of them.
+                if (!warp_wait(su.bars.o_ready(0), (j - 1) & 1, su.abort_flag)) {
                     ok = false;
                     break;
                 }
                 ptx::tc_fence_after();
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t o[32];
-                    ptx::tmem_ld32(tmem + lane_off + kColO + c * 32, o);
-                    ptx::tmem_wait_ld();
-#pragma unroll
-                    for (int k = 0; k < 32; ++k)
-                        o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-                    ptx::tmem_st32(tmem + lane_off + kColO + c * 32, o);
-                }
-                ptx::tmem_wait_st();
+                rescale_o(taddr_o, alpha);
             }
             l_run *= alpha;
             m_run = m_new;
             const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
-            float lsum[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            for (int c2 = 0; c2 < 2; ++c2) {
                 uint32_t pk[32];
-#pragma unroll
-                for (int k = 0; k < 32; ++k) {
-                    const float p0 = ptx::ex2(fmaf(s[c * 64 + 2 * k], scale_log2, neg_m));
-                    const float p1 = ptx::ex2(fmaf(s[c * 64 + 2 * k + 1], scale_log2, neg_m));
-                    lsum[k & 3] += p0 + p1;
-                    pk[k] = ptx::pack_bf16(p0, p1);
-                }
-                ptx::tmem_st32(tmem + lane_off + scol + c * 32, pk);
+                l_run += exp_pack64(sr[2 * c2], sr[2 * c2 + 1], scale_log2, neg_m, pk);
+                ptx::tmem_st32(taddr_s + c2 * 32, pk);
             }
             ptx::tmem_wait_st();
-            l_run += (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
             ptx::tc_fence_before();
-            ptx::mbar_arrive(bars.p_full(sb));
+            ptx::mbar_arrive(su.bars.p_full(sb));
         }
-
-        // ------------------------------------------------ epilogue
-        if (ok && warp_wait(bars.o_ready(), (ntiles - 1) & 1, abort_flag)) {
+        if (ok && warp_wait(su.bars.o_ready(0), (ntiles - 1) & 1, su.abort_flag)) {
             ptx::tc_fence_after();
             const size_t row = ((size_t)b * Tmax + u) * Hq + h;
             const size_t nrows = (size_t)gridDim.y / Hkv * Tmax * Hq;
-            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t o[32];
-                ptx::tmem_ld32(tmem + lane_off + kColO + c * 32, o);
-                ptx::tmem_wait_ld();
-                if (!row_ok)
-                    continue;
-                if (nsplit == 1) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(out + row * HD + c * 32);
-#pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        uint4 x;
-                        x.x = ptx::pack_bf16(__uint_as_float(o[8 * v + 0]) * inv,
-                                             __uint_as_float(o[8 * v + 1]) * inv);
-                        x.y = ptx::pack_bf16(__uint_as_float(o[8 * v + 2]) * inv,
-                                             __uint_as_float(o[8 * v + 3]) * inv);
-                        x.z = ptx::pack_bf16(__uint_as_float(o[8 * v + 4]) * inv,
-                                             __uint_as_float(o[8 * v + 5]) * inv);
-                        x.w = ptx::pack_bf16(__uint_as_float(o[8 * v + 6]) * inv,
-                                             __uint_as_float(o[8 * v + 7]) * inv);
-                        dst[v] = x;
-                    }
-                } else {
-                    float4 *dst = reinterpret_cast<float4 *>(
-                        part_o + ((size_t)split * nrows + row) * HD + c * 32);
-#pragma unroll
-                    for (int v = 0; v < 8; ++v)
-                        dst[v] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
-                                             __uint_as_float(o[4 * v + 2]),
-                                             __uint_as_float(o[4 * v + 3]));
-                }
-            }
+            const float inv = nsplit == 1 ? (l_run > 0.f ? 1.f / l_run : 0.f) : 1.f;
+            write_row(taddr_o, inv, row_ok, row, nsplit, split, nrows, out, part_o, 0, HD);
             if (row_ok && nsplit > 1)
                 part_ml[(size_t)split * nrows + row] = make_float2(m_run, l_run);
         }
     }
+    cta_teardown(su, dev_status);
+}
 
-    ptx::tc_fence_before();
-    __syncthreads();
-    if (*abort_flag && threadIdx.x == 0)
-        flag(dev_status, TSD_DEV_TIMEOUT);
-    if (warp == 1) {
-        ptx::tc_fence_after();
-        ptx::tmem_dealloc(tmem, kTmemCols);
+// ======================================================== key-split kernel
+// At most 128 packed rows: softmax group s (warps 4+4s .. 7+4s) takes the key
+// tiles s, s+2, s+4, ... of the CTA's range with its own S_s and O_s.
+// TMEM: S0 [0,128) | S1 [128,256) | O0 [256,384) | O1 [384,512).
+// MMA order: QK(0) QK(1) | PV(0) QK(2) | PV(1) QK(3) | ...  (tile k belongs to
+// group k & 1; S_s is reused after PV of its previous tile, in issue order).
+__global__ void __launch_bounds__(kSplitThreads, 1)
+    tree_attn_keysplit_kernel(const __grid_constant__ CUtensorMap tmK,
+                              const __grid_constant__ CUtensorMap tmV,
+                              const __nv_bfloat16 *__restrict__ q,
+                              const int32_t *__restrict__ prefix_len,
+                              const int32_t *__restrict__ n_nodes,
+                              const uint32_t *__restrict__ mask, int Tmax, int Hq, int Hkv,
+                              int Lmax, int W, float scale_log2, int keys_per_split, int nsplit,
+                              __nv_bfloat16 *__restrict__ out, float *__restrict__ part_o,
+                              float2 *__restrict__ part_ml, int32_t *dev_status)
+{
+    extern __shared__ uint8_t smem_raw[];
+    const int pair = blockIdx.y, split = blockIdx.z;
+    const int b = pair / Hkv, hk = pair % Hkv;
+    const int G = Hq / Hkv;
+    const int T = n_nodes[b], P = prefix_len[b];
+    if (!tree_header_ok(T, Tmax) || P < 0 || P + T > Lmax) {
+        if (split == 0 && hk == 0 && threadIdx.x == 0)
+            flag(dev_status, TSD_DEV_BAD_PREFIX);
+        return;
     }
+    const int R = T * G;
+    const int kb = split * keys_per_split;
+    const int ke = min(kb + keys_per_split, P + T);
+    if (R <= 0 || kb >= ke)
+        return;
+    const int ntiles = (ke - kb + BN - 1) / BN;
+    const Setup su = cta_setup(smem_raw, 2 * BQ, BQ);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    auto col_s = [](int s) { return (uint32_t)s * 128u; };
+    auto col_o = [](int s) { return 256u + (uint32_t)s * 128u; };
+
+    if (warp == 0) {
+        if (lane == 0)
+            produce_kv(su, &tmK, &tmV, b * Hkv + hk, kb, ntiles);
+    } else if (warp == 1) {
+        bool ok = warp_wait(su.bars.q_full(), 0, su.abort_flag);
+        ptx::tc_fence_after();
+        auto qk = [&](int k) -> bool {
+            if (!warp_wait(su.bars.k_full(k % NSK), (k / NSK) & 1, su.abort_flag))
+                return false;
+            ptx::tc_fence_after();
+            issue_qk(su, lane, col_s(k & 1), k, su.bars.s_full(k & 1));
+            return true;
+        };
+        if (ok)
+            ok = qk(0);
+        if (ok && ntiles > 1)
+            ok = qk(1);
+        for (int k = 0; ok && k < ntiles; ++k) {
+            const int s = k & 1;
+            if (!warp_wait(su.bars.p_full(s), (k >> 1) & 1, su.abort_flag) ||
+                !warp_wait(su.bars.v_full(k % NSV), (k / NSV) & 1, su.abort_flag)) {
+                ok = false;
+                break;
+            }
+            issue_pv(su, lane, col_s(s), col_o(s), k, k >= 2, P + T - (kb + k * BN),
+                     su.bars.o_ready(s));
+            if (k + 2 < ntiles)
+                ok = qk(k + 2);
+        }
+    } else if (warp >= 4) {
+        const int s = (warp - 4) >> 2;   // group
+        const int quarter = warp & 3;
+        const int t = quarter * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const bool row_ok = t < R;
+        const int u = row_ok ? t / G : 0;
+        const int h = hk * G + (row_ok ? t % G : 0);
+        if (s == 0)
+            load_q_row(su, q, row_ok, (((size_t)b * Tmax + u) * Hq + h) * HD, t);
+        ptx::mbar_arrive(su.bars.q_full());
+        RowCtx rc;
+        rc.P = P;
+        rc.ke = ke;
+        rc.scale_log2 = scale_log2;
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+            rc.mw[w] = (row_ok && w < W) ? mask[((size_t)b * Tmax + u) * W + w] : 0u;
+        const int my_tiles = (ntiles - s + 1) / 2;
+        float m_run = -INFINITY, l_run = 0.f;
+        bool ok = true;
+        for (int mi = 0; ok && mi < my_tiles; ++mi) {
+            if (!warp_wait(su.bars.s_full(s), mi & 1, su.abort_flag)) {
+                ok = false;
+                break;
+            }
+            ptx::tc_fence_after();
+            auto wait_o = [&]() { return warp_wait(su.bars.o_ready(s), (mi - 1) & 1, su.abort_flag); };
+            ok = softmax_tile(su.tmem + lane_off + col_s(s), su.tmem + lane_off + col_o(s),
+                              kb + (2 * mi + s) * BN, rc, mi == 0, m_run, l_run, wait_o);
+            if (!ok)
+                break;
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(su.bars.p_full(s));
+        }
+        const bool have = ok && my_tiles > 0 &&
+                          warp_wait(su.bars.o_ready(s), (my_tiles - 1) & 1, su.abort_flag);
+        ptx::tc_fence_after();
+        // Merge (m, l) of the two groups through shared memory in the Q tile.
+        // Q is only free once group 0 has seen its last product: every QK
+        // (the only reader of Q) is issued before that PV, while group 1 may
+        // have had no tile at all and get here at once.
+        ptx::named_barrier(1, 2 * BQ);
+        float2 *ml = reinterpret_cast<float2 *>(su.gbase + kOffQ);
+        ml[s * BQ + t] = make_float2(have ? m_run : -INFINITY, have ? l_run : 0.f);
+        ptx::named_barrier(1, 2 * BQ);
+        const float2 a = ml[t], c2 = ml[BQ + t];
+        const float M = fmaxf(a.x, c2.x);
+        const float w0 = a.y > 0.f ? ptx::ex2(a.x - M) : 0.f;
+        const float w1 = c2.y > 0.f ? ptx::ex2(c2.x - M) : 0.f;
+        const float L = a.y * w0 + c2.y * w1;
+        const float inv = nsplit == 1 ? (L > 0.f ? 1.f / L : 0.f) : 1.f;
+        const size_t row = ((size_t)b * Tmax + u) * Hq + h;
+        const size_t nrows = (size_t)gridDim.y / Hkv * Tmax * Hq;
+        // group s writes head_dim columns [64 s, 64 s + 64)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            const uint32_t col = s * 64 + c * 32;
+            uint32_t o0[32], o1[32];
+            ptx::tmem_ld32(su.tmem + lane_off + col_o(0) + col, o0);
+            ptx::tmem_ld32(su.tmem + lane_off + col_o(1) + col, o1);
+            ptx::tmem_wait_ld();
+            if (!row_ok)
+                continue;
+            float o[32];
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+                o[k] = ((w0 > 0.f ? __uint_as_float(o0[k]) * w0 : 0.f) +
+                        (w1 > 0.f ? __uint_as_float(o1[k]) * w1 : 0.f)) * inv;
+            if (nsplit == 1) {
+                uint4 *dst = reinterpret_cast<uint4 *>(out + row * HD + col);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    uint4 x;
+                    x.x = ptx::pack_bf16(o[8 * v + 0], o[8 * v + 1]);
+                    x.y = ptx::pack_bf16(o[8 * v + 2], o[8 * v + 3]);
+                    x.z = ptx::pack_bf16(o[8 * v + 4], o[8 * v + 5]);
+                    x.w = ptx::pack_bf16(o[8 * v + 6], o[8 * v + 7]);
+                    dst[v] = x;
+                }
+            } else {
+                float4 *dst = reinterpret_cast<float4 *>(
+                    part_o + ((size_t)split * nrows + row) * HD + col);
+#pragma unroll
+                for (int v = 0; v < 8; ++v)
+                    dst[v] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+            }
+        }
+        if (row_ok && nsplit > 1 && s == 0)
+            part_ml[(size_t)split * nrows + row] = make_float2(M, L);
+    }
+    cta_teardown(su, dev_status);
 }
 
 // ------------------------------------------------------------------ host
 struct UmmaPlan {
+    bool keysplit;   // at most 128 packed rows
     int nrb, nsplit, keys_per_split;
 };
 
@@ -444,9 +784,12 @@ UmmaPlan umma_plan(const AttnArgs &a, int num_sms)
 {
     UmmaPlan p;
     const int G = a.Hq / a.Hkv;
-    p.nrb = (a.Tmax * G + BM - 1) / BM;
+    p.keysplit = a.Tmax * G <= BQ;
+    p.nrb = p.keysplit ? 1 : (a.Tmax * G + BQ - 1) / BQ;
     const long base = (long)p.nrb * a.B * a.Hkv;
     const int tiles = (a.Lmax + BN - 1) / BN;
+    // waves x (tiles per CTA + fixed cost): the fewest splits that balance
+    // the grid over the SMs.
     int best = 1;
     double best_cost = 1e30;
     for (int ns = 1; ns <= 64 && ns <= tiles; ++ns) {
@@ -496,6 +839,21 @@ bool make_kv_map(CUtensorMap *m, const void *ptr, int Lmax, int BH)
     return r == CUDA_SUCCESS;
 }
 
+cudaError_t set_smem_attributes()
+{
+    static std::once_flag once;
+    static cudaError_t err = cudaSuccess;
+    std::call_once(once, [] {
+        err = cudaFuncSetAttribute(tree_attn_rows_kernel,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+        if (err == cudaSuccess)
+            err = cudaFuncSetAttribute(tree_attn_keysplit_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kSmemBytes);
+    });
+    return err;
+}
+
 }  // namespace
 
 bool umma_attention_supported(const AttnArgs &a)
@@ -525,13 +883,7 @@ int launch_umma_attention(const AttnArgs &a, void *ws, size_t ws_bytes, int num_
     if (!make_kv_map(&tmK, a.k, a.Lmax, a.B * a.Hkv) ||
         !make_kv_map(&tmV, a.v, a.Lmax, a.B * a.Hkv))
         return TSD_ERR_CUDA;
-    static bool attr_set = false;
-    if (!attr_set) {
-        TSD_CUDA_TRY(cudaFuncSetAttribute(tree_attn_umma_kernel,
-                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          (int)kSmemBytes));
-        attr_set = true;
-    }
+    TSD_CUDA_TRY(set_smem_attributes());
     const size_t nrows = (size_t)a.B * a.Tmax * a.Hq;
     float *part_o = nullptr;
     float2 *part_ml = nullptr;
@@ -544,10 +896,18 @@ int launch_umma_attention(const AttnArgs &a, void *ws, size_t ws_bytes, int num_
         TSD_LAUNCH_CHECK();
     }
     dim3 grid(p.nrb, a.B * a.Hkv, p.nsplit);
-    tree_attn_umma_kernel<<<grid, kThreads, kSmemBytes, stream>>>(
-        tmK, tmV, static_cast<const __nv_bfloat16 *>(a.q), a.prefix_len, a.n_nodes, a.mask,
-        a.Tmax, a.Hq, a.Hkv, a.Lmax, (a.Tmax + 31) / 32, a.scale * kLog2e, p.keys_per_split,
-        p.nsplit, static_cast<__nv_bfloat16 *>(a.out), part_o, part_ml, a.dev_status);
+    const float sl2 = a.scale * kLog2e;
+    const int W = (a.Tmax + 31) / 32;
+    if (p.keysplit)
+        tree_attn_keysplit_kernel<<<grid, kSplitThreads, kSmemBytes, stream>>>(
+            tmK, tmV, static_cast<const __nv_bfloat16 *>(a.q), a.prefix_len, a.n_nodes, a.mask,
+            a.Tmax, a.Hq, a.Hkv, a.Lmax, W, sl2, p.keys_per_split, p.nsplit,
+            static_cast<__nv_bfloat16 *>(a.out), part_o, part_ml, a.dev_status);
+    else
+        tree_attn_rows_kernel<<<grid, kRowsThreads, kSmemBytes, stream>>>(
+            tmK, tmV, static_cast<const __nv_bfloat16 *>(a.q), a.prefix_len, a.n_nodes, a.mask,
+            a.Tmax, a.Hq, a.Hkv, a.Lmax, W, sl2, p.keys_per_split, p.nsplit,
+            static_cast<__nv_bfloat16 *>(a.out), part_o, part_ml, a.dev_status);
     TSD_LAUNCH_CHECK();
     if (p.nsplit > 1) {
         const int rc = launch_combine(a.dtype, a.D, part_o, part_ml, p.nsplit, a.prefix_len,

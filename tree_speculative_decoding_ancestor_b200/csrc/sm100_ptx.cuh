@@ -195,6 +195,23 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+        : "memory");
+}
+
+// Named barrier over `count` threads (a multiple of 32) of this CTA.
+__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -205,6 +222,28 @@ __device__ __forceinline__ float ex2(float x)
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// 2^x on the FMA/ALU pipes, for spreading the softmax's exponentials over
+// more than the MUFU unit.  Cody-Waite style split x = j + f with j the
+// nearest integer (the 1.5 * 2^23 rounding trick, so j also lands in the low
+// bits of t) and f in [-1/2, 1/2]; 2^f from a degree-3 polynomial whose
+// coefficients were fitted for minimum relative error on [-1/2, 1/2]
+// (Lawson's iteratively reweighted least squares): max relative error 7.5e-5,
+// far below the bf16 rounding (2^-9) the result goes through.  j is added to
+// the exponent field with one integer multiply-add.  Returns 0 for x < -125
+// (below that the result would leave the normal range; as a softmax weight
+// next to a row maximum of 1 it is 0 in bf16 anyway).
+__device__ __forceinline__ float exp2_fma(float x)
+{
+    constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
+    const float t = x + kRound;
+    const float f = x - (t - kRound);
+    float p = fmaf(0x1.c3f6e2p-5f, f, 0x1.f0ddf0p-3f);
+    p = fmaf(p, f, 0x1.62f31ap-1f);
+    p = fmaf(p, f, 0x1.fff694p-1f);
+    const int bits = __float_as_int(t) * (1 << 23) + __float_as_int(p);
+    return x < -125.0f ? 0.0f : __int_as_float(bits);
 }
 
 // Two floats -> packed bf16x2 (lo in the low half), round to nearest even.
