@@ -145,7 +145,9 @@ int tsd_tree_attention(const void *q, const void *k_cache, const void *v_cache,
                        int dtype, void *out, void *workspace, size_t workspace_bytes,
                        int32_t *dev_status, tsd_stream_t stream);
 
-/* Bytes of workspace either verify call needs (per-row statistics). */
+/* Bytes of workspace either verify call needs: a fixed ~40 KB (per-CTA
+ * partial sums and barrier counters of the stochastic walk) plus 4 bytes per
+ * logits row (greedy row argmax). */
 size_t tsd_tree_verify_workspace_size(int B, int Tmax, int V);
 
 /*
@@ -192,7 +194,11 @@ int tsd_tree_verify_greedy(const float *logits, const int32_t *tokens, const int
  *   n_nodes, first_child, next_sibling   from tsd_tree_mask_build
  *   u_accept      [B][Tmax] fp64, u_sample [B][Tmax+1] fp64: uniforms in (0,1)
  *   out_tokens, out_path, n_accepted      as for the greedy call
- * Device: TSD_DEV_BAD_TOKEN, TSD_DEV_BAD_QROW.
+ * Work: one cooperative kernel launch; each sequence's walk reads only the
+ * logits rows (and q rows) of the nodes it reaches.  The CTAs of a sequence
+ * meet at barriers whose waits are bounded (about 2 s).
+ * Device: TSD_DEV_BAD_TOKEN, TSD_DEV_BAD_QROW, TSD_DEV_TIMEOUT (a barrier
+ * wait expired; the affected sequences get n_accepted = -1).
  */
 int tsd_tree_verify_stochastic(const float *logits, double temperature, const float *q_probs,
                                int Rq, const int32_t *q_row, const int32_t *tokens,
@@ -215,11 +221,10 @@ int tsd_tree_verify_stochastic(const float *logits, double temperature, const fl
  * inside the library's device code; every GPU that loads the library holds
  * that array until the process exits.  Nothing is allocated: no cudaMalloc,
  * no cudaFree, no allocating library routine.
- *   - Sizes whose scratch exceeds the array (tsd_tree_verify_workspace_size:
- *     about 28 bytes per logits row plus 12 bytes per 4096 vocabulary entries
- *     per sequence, i.e. B * (Tmax + 1) up to roughly 37000 rows) return
- *     TSD_ERR_WORKSPACE and launch nothing; use tsd_tree_verify_stochastic
- *     for those.
+ *   - The scratch it needs is fixed (about 40 KB: the per-CTA partial sums
+ *     and barrier counters of the walk), whatever B, Tmax and V are, so no
+ *     shape is refused for size; TSD_ERR_WORKSPACE would mean a build whose
+ *     array is smaller than that, and then nothing is launched.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call
  *     before any stream capture.
@@ -227,7 +232,7 @@ int tsd_tree_verify_stochastic(const float *logits, double temperature, const fl
  *     contents.  Calls whose kernels may overlap on the GPU (different
  *     streams, or concurrent host threads) race on it: serialise them.
  */
-#define TSD_NOALLOC_SCRATCH_BYTES (1u << 20)
+#define TSD_NOALLOC_SCRATCH_BYTES (1u << 16)
 
 int tsd_tree_verify_stochastic_noalloc(const float *logits, double temperature,
                                        const float *q_probs, int Rq, const int32_t *q_row,

@@ -160,6 +160,9 @@ VERIFY_CASES = [
     (34, 4, 128, 32000, "sample", 1.0),
     (35, 32, 20, 5, "sample", 1.3),
     (36, 6, 40, 777, "topk", 0.5),
+    (37, 2, 16, 128256, "topk", 1.0),    # 32-CTA teams, 4008 entries each
+    (38, 3, 12, 50001, "sample", 0.9),   # last chunk ends at V, V % 4 != 0
+    (39, 700, 8, 64, "sample", 1.0),     # more sequences than the grid holds
 ]
 
 

@@ -100,6 +100,7 @@ int launch_umma_attention(const AttnArgs &a, void *ws, size_t ws_bytes, int num_
                           cudaStream_t stream);
 
 size_t verify_workspace(int B, int Tmax, int V);
+size_t verify_stochastic_scratch();   // fixed: independent of the shape
 int launch_verify_greedy(const float *logits, const int32_t *tokens, const int32_t *parent,
                          const int32_t *n_nodes, const uint32_t *mask,
                          const int32_t *first_child, int B, int Tmax, int V,

@@ -9,30 +9,36 @@
 //                           path matches, the deepest (lowest index on ties),
 //                           and the argmax of its row (computed here for a leaf).
 // stochastic (multi-step speculative sampling)
-//   mss_rows_kernel         one CTA per logits row (every node and the root):
-//                           m = max l and Z = sum exp((l-m)/T) in fp64; for a
-//                           row with children, the children in ascending index:
-//                           child c with token x is accepted iff p(x) > 0 and
-//                           u_c * q_c(x) <= p(x) (one thread, exact fp64
-//                           formula); after a rejection the block computes
-//                           S = sum max(0, p - q_c), and p becomes
-//                           max(0, p - q_c) / S.
-//   mss_chunks_kernel       one CTA per (vocabulary chunk, sequence): follows
-//                           the accepted children from the root to the row where
-//                           the sequence stops and sums that row's final
-//                           distribution over its chunk;
-//   mss_finalize_kernel     one CTA per sequence: emits the path, then draws the
-//                           last token by inverse CDF at u_sample[row] -- the
-//                           chunk whose running sum passes u, then an fp64
-//                           block scan inside that chunk.
+//   mss_walk_kernel         one cooperative launch.  Each sequence is walked by
+//                           a team of K CTAs, CTA k owning one contiguous chunk
+//                           of the vocabulary.  At the current node's row the
+//                           team computes m = max l and Z = sum exp((l-m)/T)
+//                           in fp64 (one pass: each thread keeps a running max
+//                           and rescales its sum when the max rises), then
+//                           tries the children in ascending index: child c
+//                           with token x is accepted iff p(x) > 0 and
+//                           u_c * q_c(x) <= p(x) (exact fp64 formula, every
+//                           CTA taking the same decision from the same
+//                           numbers); after a rejection the team sums
+//                           S = sum max(0, p - q_c) and p becomes
+//                           max(0, p - q_c) / S.  An accepted child's row is
+//                           next.  Where the walk stops, the team sums the
+//                           final distribution per chunk; the chunk whose
+//                           running sum passes u_sample[row] is scanned (fp64
+//                           block scan) by its CTA for the token.
+//                           Only rows on the accepted path are read.  Partial
+//                           results cross CTAs through one workspace slot per
+//                           CTA and a per-team arrival counter; every wait on
+//                           a counter is bounded (TSD_DEV_TIMEOUT).
 //
 // Residual distributions are never materialised: p^(n)(x) is recomputed per
 // element from the logits row, the rejected siblings' q rows and their
-// normalisers.  The bulk sums (Z, S, the CDF) use a table-driven fp64 exp
-// (its table pre-scaled by 1/Z) and reciprocals; the acceptance tests use the
-// exact formula.  Both agree with a sequential fp64 evaluation to ~1e-15
+// normalisers (all L2-resident while a team works on a row).  The bulk sums
+// (Z, S, the CDF) use a table-driven fp64 exp (its table pre-scaled by 1/Z)
+// and reciprocals; the acceptance tests use the exact formula.  Both agree with a sequential fp64 evaluation to ~1e-15
 // relative, so a decision can only differ when its uniform lies within that
 // distance of the boundary.
+#include <algorithm>
 #include <climits>
 
 #include "fp64_exp.cuh"
@@ -43,46 +49,35 @@ namespace tsd {
 namespace {
 
 constexpr int kRowThreads = 512;
-constexpr int kWarps = kRowThreads / 32;
 constexpr int kFinThreads = 1024;
-constexpr int kDrawThreads = 256;
-constexpr int kChunk = 4096;   // vocabulary chunk of the deferred draw (multiple of 4)
+constexpr int kWalkThreads = 256;
+constexpr int kWalkWarps = kWalkThreads / 32;
+constexpr int kTeamMax = 32;          // CTAs per team: one partial per lane of a warp
+constexpr int kTeamMinChunk = 2048;   // vocabulary entries per CTA, at least
+constexpr int kWalkMaxCtas = 1024;    // grid cap (sets the workspace slots)
+constexpr unsigned long long kTeamWaitNs = 2000000000ull;   // bound of one barrier wait
 
 struct VerifyWs {
-    double *Z;            // [B][Tmax+1]  sum exp((l - m)/T)
-    double *S;            // [B][Tmax]    residual normaliser after rejecting child c
-    double *chunk_sum;    // [B][nch]     final distribution summed over a chunk
-    int32_t *argmax;      // [B][Tmax+1]  greedy: argmax of rows with children
-    int32_t *accepted;    // [B][Tmax+1]  accepted child per row, -1 none
-    float *rmax;          // [B][Tmax+1]  row max
-    int32_t *chunk_last;  // [B][nch]     largest token of the chunk with p > 0, or -1
-    int nch;
+    double2 *slot;     // [2][kWalkMaxCtas]  per-CTA partials, by barrier parity
+    int2 *team;        // [kWalkMaxCtas]     {arrivals, abort} per team, zeroed per call
+    int32_t *argmax;   // [B][Tmax+1]        greedy: argmax of rows with children
 };
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-int num_chunks(int V) { return (V + kChunk - 1) / kChunk; }
+// Fixed part first: the stochastic call uses only that.
+constexpr size_t kWalkBytes = ((2 * kWalkMaxCtas * sizeof(double2) + 255) & ~(size_t)255) +
+                              ((kWalkMaxCtas * sizeof(int2) + 255) & ~(size_t)255);
 
-VerifyWs carve(void *ws, int B, int Tmax, int V)
+VerifyWs carve(void *ws)
 {
-    const size_t R = (size_t)B * (Tmax + 1), N = (size_t)B * Tmax;
-    const size_t C = (size_t)B * num_chunks(V);
     char *p = static_cast<char *>(ws);
     VerifyWs w;
-    w.nch = num_chunks(V);
-    w.Z = reinterpret_cast<double *>(p);
-    p += align256(R * sizeof(double));
-    w.S = reinterpret_cast<double *>(p);
-    p += align256(N * sizeof(double));
-    w.chunk_sum = reinterpret_cast<double *>(p);
-    p += align256(C * sizeof(double));
+    w.slot = reinterpret_cast<double2 *>(p);
+    p += align256(2 * kWalkMaxCtas * sizeof(double2));
+    w.team = reinterpret_cast<int2 *>(p);
+    p += align256(kWalkMaxCtas * sizeof(int2));
     w.argmax = reinterpret_cast<int32_t *>(p);
-    p += align256(R * sizeof(int32_t));
-    w.accepted = reinterpret_cast<int32_t *>(p);
-    p += align256(R * sizeof(int32_t));
-    w.rmax = reinterpret_cast<float *>(p);
-    p += align256(R * sizeof(float));
-    w.chunk_last = reinterpret_cast<int32_t *>(p);
     return w;
 }
 
@@ -134,15 +129,17 @@ __device__ void block_argmax(float &v, int &i, float *shv, int *shi)
     __syncthreads();
 }
 
+template <int NT>
 __device__ float block_max(float v, float *sh)
 {
+    constexpr int NW = NT / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     v = warp_max(v);
     if (lane == 0)
         sh[warp] = v;
     __syncthreads();
     if (warp == 0) {
-        v = lane < kWarps ? sh[lane] : -INFINITY;
+        v = lane < NW ? sh[lane] : -INFINITY;
         v = warp_max(v);
         if (lane == 0)
             sh[0] = v;
@@ -153,15 +150,17 @@ __device__ float block_max(float v, float *sh)
     return v;
 }
 
+template <int NT>
 __device__ double block_sum(double v, double *sh)
 {
+    constexpr int NW = NT / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     v = warp_sum(v);
     if (lane == 0)
         sh[warp] = v;
     __syncthreads();
     if (warp == 0) {
-        v = lane < kWarps ? sh[lane] : 0.0;
+        v = lane < NW ? sh[lane] : 0.0;
         v = warp_sum(v);
         if (lane == 0)
             sh[0] = v;
@@ -245,33 +244,6 @@ __device__ int row_argmax(const float *__restrict__ row, int V, float *shv, int 
     return bi == INT_MAX ? 0 : bi;
 }
 
-__device__ float row_max(const float *__restrict__ row, int V, float *sh)
-{
-    float m = -INFINITY;
-    if ((V & 3) == 0) {
-        const float4 *r4 = reinterpret_cast<const float4 *>(row);
-        const int n4 = V >> 2;
-        int j = threadIdx.x;
-        for (; j + 3 * kRowThreads < n4; j += 4 * kRowThreads) {
-            float4 x[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                x[k] = __ldg(r4 + j + k * kRowThreads);
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                m = fmaxf(m, fmaxf(fmaxf(x[k].x, x[k].y), fmaxf(x[k].z, x[k].w)));
-        }
-        for (; j < n4; j += kRowThreads) {
-            const float4 x = __ldg(r4 + j);
-            m = fmaxf(m, fmaxf(fmaxf(x.x, x.y), fmaxf(x.z, x.w)));
-        }
-    } else {
-        for (int j = threadIdx.x; j < V; j += kRowThreads)
-            m = fmaxf(m, __ldg(row + j));
-    }
-    return block_max(m, sh);
-}
-
 // Per-row state of multi-step speculative sampling.
 struct RowState {
     double m, inv_temp, temp, Z;
@@ -326,22 +298,70 @@ __device__ __forceinline__ void p_bulk4(const float *__restrict__ row, int x0, i
     }
 }
 
-// sum_x max(0, p^(n)(x) - q(x)) (q == nullptr: sum_x p^(n)(x)), eight tokens
-// per thread per iteration as two groups of four.
+// One pass over the CTA's chunk [x_lo, x_hi) of a logits row: the chunk's
+// max m_k and z_k = sum exp((l - m_k)/T).  Each thread keeps a running max
+// and rescales its sum when the max rises; `table` is scaled by 1.
 template <bool VEC>
-__device__ double bulk_mass(const float *__restrict__ row, const float *__restrict__ q, int V,
-                            const RowState &st, const double *table, double *sh)
+__device__ double2 chunk_max_z(const float *__restrict__ row, int x_lo, int x_hi, int V,
+                               double inv_temp, const double *table, float *shf, double *shd)
+{
+    float mt = -INFINITY;
+    double zt = 0.0;
+    auto group = [&](const float (&l)[4]) {
+        const float m4 = fmaxf(fmaxf(l[0], l[1]), fmaxf(l[2], l[3]));
+        if (m4 > mt) {
+            if (mt != -INFINITY)
+                zt *= table_exp(((double)mt - (double)m4) * inv_temp, table);
+            mt = m4;
+        }
+        if (mt != -INFINITY) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                zt += table_exp(((double)l[k] - (double)mt) * inv_temp, table);
+        }
+    };
+    for (int x0 = x_lo + 4 * threadIdx.x; x0 < x_hi; x0 += 8 * kWalkThreads) {
+        const int x1 = x0 + 4 * kWalkThreads;
+        float l0[4], l1[4];
+        load4<VEC>(row, x0, V, l0);
+        load4<VEC>(row, x1, V, l1);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            if (x0 + k >= x_hi)
+                l0[k] = -INFINITY;
+            if (x1 + k >= x_hi)
+                l1[k] = -INFINITY;
+        }
+        group(l0);
+        group(l1);
+    }
+    const float mk = block_max<kWalkThreads>(mt, shf);
+    const double zs =
+        mt == -INFINITY ? 0.0 : zt * table_exp(((double)mt - (double)mk) * inv_temp, table);
+    return make_double2((double)mk, block_sum<kWalkThreads>(zs, shd));
+}
+
+// Over the CTA's chunk: sum max(0, p^(n)(x) - q(x)), or with q == nullptr
+// sum p^(n)(x) and (in *last) the largest x with p^(n)(x) > 0, -1 if none.
+// `table` is scaled by 1/Z.  x_lo is a multiple of 4 and x_hi is one or V,
+// so the groups of four never straddle x_hi inside the vocabulary.
+template <bool VEC>
+__device__ double chunk_mass(const float *__restrict__ row, const float *__restrict__ q,
+                             int x_lo, int x_hi, int V, const RowState &st, const double *table,
+                             double *shd, int *shi, int *last_out)
 {
     double s = 0.0;
-    for (int x0 = 4 * threadIdx.x; x0 < V; x0 += 8 * kRowThreads) {
-        const int x1 = x0 + 4 * kRowThreads;
-        double p0[4], p1[4];
+    int last = -1;
+    for (int x0 = x_lo + 4 * threadIdx.x; x0 < x_hi; x0 += 8 * kWalkThreads) {
+        const int x1 = x0 + 4 * kWalkThreads;
+        double p0[4], p1[4] = {0.0, 0.0, 0.0, 0.0};
         p_bulk4<VEC>(row, x0, V, st, table, p0);
-        p_bulk4<VEC>(row, x1, V, st, table, p1);
+        if (x1 < x_hi)
+            p_bulk4<VEC>(row, x1, V, st, table, p1);
         if (q) {
             float q0[4], q1[4];
             load4<VEC>(q, x0, V, q0);
-            load4<VEC>(q, x1, V, q1);
+            load4<VEC>(q, x1 < x_hi ? x1 : V, V, q1);
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const double d0 = p0[k] - (double)q0[k], d1 = p1[k] - (double)q1[k];
@@ -349,11 +369,66 @@ __device__ double bulk_mass(const float *__restrict__ row, const float *__restri
             }
         } else {
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
+            for (int k = 0; k < 4; ++k) {
                 s += p0[k] + p1[k];
+                if (p0[k] > 0.0)
+                    last = max(last, x0 + k);
+                if (p1[k] > 0.0)
+                    last = max(last, x1 + k);
+            }
         }
     }
-    return block_sum(s, sh);
+    if (last_out)
+        *last_out = block_max_int<kWalkThreads>(last, shi);
+    return block_sum<kWalkThreads>(s, shd);
+}
+
+// The draw inside the chunk [x_lo, x_hi): the smallest x with
+// carry + sum_{x_lo <= y <= x} p^(n)(y) > u (fp64 block scan in order), or
+// INT_MAX when rounding leaves the chunk's sum short of u.
+template <bool VEC>
+__device__ int chunk_scan(const float *__restrict__ row, int x_lo, int x_hi, int V,
+                          const RowState &st, const double *table, double carry, double u,
+                          double *warp_tot, int *shi)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int base = x_lo; base < x_hi; base += 4 * kWalkThreads) {
+        const int x0 = base + 4 * threadIdx.x;
+        double p[4] = {0.0, 0.0, 0.0, 0.0};
+        if (x0 < x_hi)
+            p_bulk4<VEC>(row, x0, V, st, table, p);
+        const double mine = ((p[0] + p[1]) + p[2]) + p[3];
+        double incl = mine;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const double y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o)
+                incl += y;
+        }
+        if (lane == 31)
+            warp_tot[warp] = incl;
+        __syncthreads();
+        double wbase = 0.0, tile = 0.0;
+        for (int w2 = 0; w2 < kWalkWarps; ++w2) {
+            const double t = warp_tot[w2];
+            if (w2 < warp)
+                wbase += t;
+            tile += t;
+        }
+        double C = carry + wbase + (incl - mine);
+        int found = INT_MAX;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            C += p[k];
+            if (found == INT_MAX && x0 + k < x_hi && C > u)
+                found = x0 + k;
+        }
+        found = block_min_int<kWalkThreads>(found, shi);   // ends with a barrier
+        if (found != INT_MAX)
+            return found;
+        carry += tile;
+    }
+    return INT_MAX;
 }
 
 // p^(n)(x) for one acceptance test: the exact fp64 formula of the definition.
@@ -382,8 +457,8 @@ __global__ void __launch_bounds__(kRowThreads)
                        const int32_t *__restrict__ first_child, int Tmax, int V,
                        int32_t *__restrict__ argmax_ws)
 {
-    __shared__ float shv[kWarps];
-    __shared__ int shi[kWarps];
+    __shared__ float shv[kRowThreads / 32];
+    __shared__ int shi[kRowThreads / 32];
     const int r = blockIdx.x, b = blockIdx.y;
     int T;
     if (!sequence_ok(n_nodes, first_child, b, Tmax, T) || r > T)
@@ -480,323 +555,265 @@ __global__ void __launch_bounds__(kFinThreads)
 }
 
 // -------------------------------------------------------------- stochastic
+__device__ __forceinline__ unsigned long long global_ns()
+{
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Barrier over the K CTAs of one team (co-resident: cooperative launch).
+// `target` = K x the number of barriers the team has entered, this one
+// included.  Thread 0 publishes the CTA's slot write (fence, then its
+// arrival) and spins on the counter; after kTeamWaitNs it raises the team's
+// abort flag, which releases the other CTAs as well.  False after an abort.
+__device__ bool team_barrier(int2 *team, int target, int *sh_ok)
+{
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int *arrive = &team->x;
+        volatile int *abort = &team->y;
+        __threadfence();
+        atomicAdd(arrive, 1);
+        const unsigned long long t0 = global_ns();
+        int ok = 1;
+        for (;;) {
+            int v;
+            asm volatile("ld.acquire.gpu.b32 %0, [%1];" : "=r"(v) : "l"(arrive) : "memory");
+            if (v >= target)
+                break;
+            if (*abort) {
+                ok = 0;
+                break;
+            }
+            if (global_ns() - t0 > kTeamWaitNs) {
+                atomicExch(&team->y, 1);
+                ok = 0;
+                break;
+            }
+            __nanosleep(64);
+        }
+        *sh_ok = ok;
+    }
+    __syncthreads();
+    return *sh_ok != 0;
+}
+
 // VEC: V % 4 == 0, so every logits / q row is 16-byte aligned (the entry
-// point checks the base pointers) and the bulk passes use float4 loads.
+// point checks the base pointers) and the passes use float4 loads.
+// Grid: teams x K CTAs; team t walks sequences t, t + teams, ...
 template <bool VEC>
-__global__ void __launch_bounds__(kRowThreads)
-    mss_rows_kernel(const float *__restrict__ logits, double temp,
+__global__ void __launch_bounds__(kWalkThreads)
+    mss_walk_kernel(const float *__restrict__ logits, double temp,
                     const float *__restrict__ q_probs, int Rq, const int32_t *__restrict__ q_row,
                     const int32_t *__restrict__ tokens, const int32_t *__restrict__ n_nodes,
                     const int32_t *__restrict__ first_child,
                     const int32_t *__restrict__ next_sibling,
-                    const double *__restrict__ u_accept, int Tmax, int V, VerifyWs ws)
+                    const double *__restrict__ u_accept, const double *__restrict__ u_sample,
+                    int B, int Tmax, int V, int K, int chunk, VerifyWs ws,
+                    int32_t *__restrict__ out_tokens, int32_t *__restrict__ out_path,
+                    int32_t *__restrict__ n_accepted, int32_t *dev_status)
 {
     __shared__ double table[kExpTable];
-    __shared__ float shf[kWarps];
-    __shared__ double shd[kWarps];
+    __shared__ float shf[kWalkWarps];
+    __shared__ double shd[kWalkWarps];
+    __shared__ int shi[kWalkWarps];
     __shared__ RowState st;
-    __shared__ int decision;
-    const int r = blockIdx.x, b = blockIdx.y;
-    int T;
-    if (!sequence_ok(n_nodes, first_child, b, Tmax, T) || r > T)
-        return;
-    fill_exp_table(table, 1.0);
-    const float *row = logits + ((size_t)b * (Tmax + 1) + r) * V;
-    const float mf = row_max(row, V, shf);   // its barriers also publish the table
-    if (threadIdx.x == 0) {
-        st.m = (double)mf;
-        st.inv_temp = 1.0 / temp;
-        st.temp = temp;
-        st.n = 0;
-    }
-    __syncthreads();
-    const double Z = bulk_mass<VEC>(row, nullptr, V, st, table, shd);
-    const size_t ri = (size_t)b * (Tmax + 1) + r;
-    if (threadIdx.x == 0) {
-        st.Z = Z;
-        ws.rmax[ri] = mf;
-        ws.Z[ri] = Z;
-    }
-    int c = first_child[ri];
-    if (c < 0) {
-        if (threadIdx.x == 0)
-            ws.accepted[ri] = -1;
-        return;   // a leaf (or an empty tree's root): it only needs m and Z
-    }
-    fill_exp_table(table, 1.0 / Z);   // bulk_mass ended with a barrier: table is free
-    __syncthreads();
-    int accepted = -1;
-    while (c >= 0) {
-        const int x = tokens[(size_t)b * Tmax + c];
-        const int qr = q_row[(size_t)b * Tmax + c];
-        if (x < 0 || x >= V || qr < 0 || qr >= Rq)
-            break;   // malformed; the finalize kernel reports it
-        const float *qc = q_probs + ((size_t)b * Rq + qr) * V;
-        if (threadIdx.x == 0) {
-            const double px = p_exact(row[x], x, st);
-            const double qx = (double)qc[x];
-            const double u = u_accept[(size_t)b * Tmax + c];
-            decision = (px > 0.0 && u * qx <= px) ? 1 : 0;
-        }
-        __syncthreads();
-        if (decision) {
-            accepted = c;
-            break;
-        }
-        const double S = bulk_mass<VEC>(row, qc, V, st, table, shd);
-        if (threadIdx.x == 0) {
-            st.q[st.n] = qc;
-            st.S[st.n] = S;
-            st.inv_S[st.n] = S > 0.0 ? 1.0 / S : 0.0;
-            st.n += 1;
-            ws.S[(size_t)b * Tmax + c] = S;
-        }
-        __syncthreads();
-        c = next_sibling[(size_t)b * Tmax + c];
-    }
-    if (threadIdx.x == 0)
-        ws.accepted[ri] = accepted;
-}
+    __shared__ int sh_ok, sh_dec, sh_pick, sh_token;
+    __shared__ double sh_carry;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int teams = gridDim.x / K;
+    const int team = blockIdx.x / K, k = blockIdx.x % K;
+    const int x_lo = min(k * chunk, V), x_hi = min(x_lo + chunk, V);
+    const double inv_temp = 1.0 / temp;
+    const bool lead = k == 0 && tid == 0;   // writes the path and the error codes
+    int2 *tm = ws.team + team;
+    int nbar = 0;
+    // this CTA's slot / the team's K slots of the next barrier
+    auto slots = [&]() { return ws.slot + (nbar & 1) * kWalkMaxCtas + team * K; };
 
-// Thread 0: walk the accepted children from the root (accepted row in shared
-// memory), fill `st` with the final distribution's state at the row where the
-// sequence stops, and return that row; n_out = accepted nodes.  Optionally
-// writes the path.  st.n = -1 if a q row index is malformed.
-__device__ int walk_to_terminal(int b, int T, int Tmax, int Rq, int V, double temp,
-                                const float *__restrict__ q_probs,
-                                const int32_t *__restrict__ q_row,
-                                const int32_t *__restrict__ tokens,
-                                const int32_t *__restrict__ first_child,
-                                const int32_t *__restrict__ next_sibling, const VerifyWs &ws,
-                                const int *acc, RowState &st, int &n_out,
-                                int32_t *__restrict__ out_path, int32_t *__restrict__ out_tokens)
-{
-    int row = 0, n = 0;
-    while (n < T && acc[row] >= 0) {
-        const int c = acc[row];
-        if (out_path) {
-            out_path[(size_t)b * Tmax + n] = c;
-            out_tokens[(size_t)b * (Tmax + 1) + n] = tokens[(size_t)b * Tmax + c];
+    for (int b = team; b < B; b += teams) {
+        int T;
+        if (!sequence_ok(n_nodes, first_child, b, Tmax, T)) {
+            if (lead)
+                n_accepted[b] = -1;
+            continue;
         }
-        row = c + 1;
-        ++n;
-    }
-    const size_t ri = (size_t)b * (Tmax + 1) + row;
-    st.m = (double)ws.rmax[ri];
-    st.Z = ws.Z[ri];
-    st.temp = temp;
-    st.inv_temp = 1.0 / temp;
-    st.n = 0;
-    for (int c = first_child[ri]; c >= 0; c = next_sibling[(size_t)b * Tmax + c]) {
-        const int qr = q_row[(size_t)b * Tmax + c];
-        if (qr < 0 || qr >= Rq) {
-            st.n = -1;
-            break;
+        int bad = 0;
+        for (int u = tid; u < T; u += kWalkThreads) {
+            const int x = tokens[(size_t)b * Tmax + u];
+            const int qr = q_row[(size_t)b * Tmax + u];
+            bad |= (x < 0 || x >= V) ? TSD_DEV_BAD_TOKEN : 0;
+            bad |= (qr < 0 || qr >= Rq) ? TSD_DEV_BAD_QROW : 0;
         }
-        const double S = ws.S[(size_t)b * Tmax + c];
-        st.q[st.n] = q_probs + ((size_t)b * Rq + qr) * V;
-        st.S[st.n] = S;
-        st.inv_S[st.n] = S > 0.0 ? 1.0 / S : 0.0;
-        st.n += 1;
-    }
-    n_out = n;
-    return row;
-}
-
-template <bool VEC>
-__global__ void __launch_bounds__(kDrawThreads)
-    mss_chunks_kernel(const float *__restrict__ logits, double temp,
-                      const float *__restrict__ q_probs, int Rq,
-                      const int32_t *__restrict__ q_row, const int32_t *__restrict__ tokens,
-                      const int32_t *__restrict__ n_nodes,
-                      const int32_t *__restrict__ first_child,
-                      const int32_t *__restrict__ next_sibling, int Tmax, int V, VerifyWs ws)
-{
-    __shared__ double table[kExpTable];
-    __shared__ double shd[kDrawThreads / 32];
-    __shared__ int shi[kDrawThreads / 32];
-    __shared__ int acc[kMaxTree + 1];
-    __shared__ RowState st;
-    __shared__ int term;
-    const int ch = blockIdx.x, b = blockIdx.y;
-    int T;
-    if (!sequence_ok(n_nodes, first_child, b, Tmax, T))
-        return;
-    for (int i = threadIdx.x; i <= T; i += kDrawThreads)
-        acc[i] = ws.accepted[(size_t)b * (Tmax + 1) + i];
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int n;
-        term = walk_to_terminal(b, T, Tmax, Rq, V, temp, q_probs, q_row, tokens, first_child,
-                                next_sibling, ws, acc, st, n, nullptr, nullptr);
-    }
-    __syncthreads();
-    if (st.n < 0)
-        return;   // malformed; the finalize kernel reports it
-    fill_exp_table(table, 1.0 / st.Z);
-    __syncthreads();
-    const float *row = logits + ((size_t)b * (Tmax + 1) + term) * V;
-    const int x_begin = ch * kChunk, x_end = min(x_begin + kChunk, V);
-    double s = 0.0;
-    int last = -1;
-    for (int x0 = x_begin + 4 * threadIdx.x; x0 < x_end; x0 += 4 * kDrawThreads) {
-        double p[4];
-        p_bulk4<VEC>(row, x0, V, st, table, p);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            s += p[k];
-            if (p[k] > 0.0)
-                last = x0 + k;
+        if (__syncthreads_or(bad)) {   // the same answer in every CTA of the team
+            if (k == 0 && bad)
+                flag(dev_status, bad);
+            if (lead)
+                n_accepted[b] = -1;
+            continue;
         }
-    }
-    // block reductions over kDrawThreads threads
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    s = warp_sum(s);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-        last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
-    if (lane == 0) {
-        shd[warp] = s;
-        shi[warp] = last;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        double tot = 0.0;
-        int lst = -1;
-        for (int w2 = 0; w2 < kDrawThreads / 32; ++w2) {
-            tot += shd[w2];
-            lst = max(lst, shi[w2]);
-        }
-        ws.chunk_sum[(size_t)b * ws.nch + ch] = tot;
-        ws.chunk_last[(size_t)b * ws.nch + ch] = lst;
-    }
-}
-
-template <bool VEC>
-__global__ void __launch_bounds__(kDrawThreads)
-    mss_finalize_kernel(const float *__restrict__ logits, double temp,
-                        const float *__restrict__ q_probs, int Rq,
-                        const int32_t *__restrict__ q_row, const int32_t *__restrict__ tokens,
-                        const int32_t *__restrict__ n_nodes,
-                        const int32_t *__restrict__ first_child,
-                        const int32_t *__restrict__ next_sibling,
-                        const double *__restrict__ u_sample, int Tmax, int V, VerifyWs ws,
-                        int32_t *__restrict__ out_tokens, int32_t *__restrict__ out_path,
-                        int32_t *__restrict__ n_accepted, int32_t *dev_status)
-{
-    constexpr int NW = kDrawThreads / 32;
-    __shared__ double table[kExpTable];
-    __shared__ double warp_tot[NW];
-    __shared__ int shi[NW];
-    __shared__ int acc[kMaxTree + 1];
-    __shared__ RowState st;
-    __shared__ int term, n_path, chosen;
-    __shared__ double carry0;
-    const int b = blockIdx.x, tid = threadIdx.x;
-    const int lane = tid & 31, warp = tid >> 5;
-    int T;
-    if (!sequence_ok(n_nodes, first_child, b, Tmax, T)) {
-        if (tid == 0)
-            n_accepted[b] = -1;
-        return;
-    }
-    int bad = 0;
-    if (tid < T) {
-        const int x = tokens[(size_t)b * Tmax + tid];
-        const int qr = q_row[(size_t)b * Tmax + tid];
-        bad = (x < 0 || x >= V) ? TSD_DEV_BAD_TOKEN : 0;
-        bad |= (qr < 0 || qr >= Rq) ? TSD_DEV_BAD_QROW : 0;
-    }
-    if (__syncthreads_or(bad)) {
-        if (bad)
-            flag(dev_status, bad);
-        if (tid == 0)
-            n_accepted[b] = -1;
-        return;
-    }
-    for (int i = tid; i <= T; i += kDrawThreads)
-        acc[i] = ws.accepted[(size_t)b * (Tmax + 1) + i];
-    __syncthreads();
-    if (tid == 0) {
-        int n;
-        term = walk_to_terminal(b, T, Tmax, Rq, V, temp, q_probs, q_row, tokens, first_child,
-                                next_sibling, ws, acc, st, n, out_path, out_tokens);
-        n_path = n;
-        // The chunk whose running sum passes u.
-        const double u = u_sample[(size_t)b * (Tmax + 1) + term];
-        double C = 0.0;
-        int pick = -1;
-        for (int c = 0; c < ws.nch; ++c) {
-            const double s = ws.chunk_sum[(size_t)b * ws.nch + c];
-            if (C + s > u) {
-                pick = c;
-                break;
-            }
-            C += s;
-        }
-        chosen = pick;
-        carry0 = C;
-    }
-    __syncthreads();
-    const double u = u_sample[(size_t)b * (Tmax + 1) + term];
-    int token;
-    if (chosen < 0) {
-        // Rounding left the total at or below u: the largest token with p > 0.
-        int last = -1;
-        for (int c = tid; c < ws.nch; c += kDrawThreads)
-            last = max(last, ws.chunk_last[(size_t)b * ws.nch + c]);
-        token = block_max_int<kDrawThreads>(last, shi);
-    } else {
-        fill_exp_table(table, 1.0 / st.Z);
-        __syncthreads();
-        const float *row = logits + ((size_t)b * (Tmax + 1) + term) * V;
-        const int x_begin = chosen * kChunk, x_end = min(x_begin + kChunk, V);
-        double carry = carry0;
-        token = INT_MAX;
-        for (int base = x_begin; base < x_end; base += 4 * kDrawThreads) {
-            const int x0 = base + 4 * tid;
-            double p[4] = {0.0, 0.0, 0.0, 0.0};
-            if (x0 < x_end)
-                p_bulk4<VEC>(row, x0, V, st, table, p);
-            const double mine = ((p[0] + p[1]) + p[2]) + p[3];
-            double incl = mine;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const double y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o)
-                    incl += y;
-            }
-            if (lane == 31)
-                warp_tot[warp] = incl;
+        int row = 0, n_path = 0;
+        bool alive = true;
+        for (;;) {
+            const size_t ri = (size_t)b * (Tmax + 1) + row;
+            const float *lrow = logits + ri * V;
+            // m and Z of this row
+            fill_exp_table(table, 1.0);
             __syncthreads();
-            double wbase = 0.0, tile = 0.0;
-            for (int w2 = 0; w2 < NW; ++w2) {
-                const double t = warp_tot[w2];
-                if (w2 < warp)
-                    wbase += t;
-                tile += t;
-            }
-            double C = carry + wbase + (incl - mine);
-            int found = INT_MAX;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                C += p[k];
-                if (found == INT_MAX && x0 + k < x_end && C > u)
-                    found = x0 + k;
-            }
-            found = block_min_int<kDrawThreads>(found, shi);
-            if (found != INT_MAX) {
-                token = found;
+            const double2 mz = chunk_max_z<VEC>(lrow, x_lo, x_hi, V, inv_temp, table, shf, shd);
+            double2 *sl = slots();
+            if (tid == 0)
+                sl[k] = mz;
+            ++nbar;
+            if (!team_barrier(tm, nbar * K, &sh_ok)) {
+                alive = false;
                 break;
             }
-            carry += tile;
+            if (warp == 0) {
+                double mk = -INFINITY, zk = 0.0;
+                if (lane < K) {
+                    const double2 v = __ldcg(sl + lane);
+                    mk = v.x;
+                    zk = v.y;
+                }
+                double m = mk;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1)
+                    m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
+                const double zs =
+                    mk == -INFINITY ? 0.0 : zk * table_exp((mk - m) * inv_temp, table);
+                const double Z = warp_sum(zs);
+                if (lane == 0) {
+                    st.m = m;
+                    st.Z = Z;
+                    st.temp = temp;
+                    st.inv_temp = inv_temp;
+                    st.n = 0;
+                }
+            }
+            __syncthreads();
+            fill_exp_table(table, 1.0 / st.Z);
+            __syncthreads();
+            // the children in ascending index
+            int accepted = -1;
+            for (int c = first_child[ri]; c >= 0; c = next_sibling[(size_t)b * Tmax + c]) {
+                const int x = tokens[(size_t)b * Tmax + c];
+                const float *qc = q_probs + ((size_t)b * Rq + q_row[(size_t)b * Tmax + c]) * V;
+                if (tid == 0) {
+                    const double px = p_exact(lrow[x], x, st);
+                    const double qx = (double)qc[x];
+                    const double u = u_accept[(size_t)b * Tmax + c];
+                    sh_dec = (px > 0.0 && u * qx <= px) ? 1 : 0;
+                }
+                __syncthreads();
+                if (sh_dec) {
+                    accepted = c;
+                    break;
+                }
+                const double s =
+                    chunk_mass<VEC>(lrow, qc, x_lo, x_hi, V, st, table, shd, shi, nullptr);
+                sl = slots();
+                if (tid == 0)
+                    sl[k] = make_double2(s, 0.0);
+                ++nbar;
+                if (!team_barrier(tm, nbar * K, &sh_ok)) {
+                    alive = false;
+                    break;
+                }
+                if (warp == 0) {
+                    const double S = warp_sum(lane < K ? __ldcg(sl + lane).x : 0.0);
+                    if (lane == 0) {
+                        st.q[st.n] = qc;
+                        st.S[st.n] = S;
+                        st.inv_S[st.n] = S > 0.0 ? 1.0 / S : 0.0;
+                        st.n += 1;
+                    }
+                }
+                __syncthreads();
+            }
+            if (!alive)
+                break;
+            if (accepted >= 0 && n_path < T) {
+                if (lead) {
+                    out_path[(size_t)b * Tmax + n_path] = accepted;
+                    out_tokens[(size_t)b * (Tmax + 1) + n_path] =
+                        tokens[(size_t)b * Tmax + accepted];
+                }
+                ++n_path;
+                row = accepted + 1;
+                continue;
+            }
+            // The walk stops here: draw the final token from p^(n).
+            int last;
+            const double s =
+                chunk_mass<VEC>(lrow, nullptr, x_lo, x_hi, V, st, table, shd, shi, &last);
+            sl = slots();
+            if (tid == 0)
+                sl[k] = make_double2(s, (double)last);
+            ++nbar;
+            if (!team_barrier(tm, nbar * K, &sh_ok)) {
+                alive = false;
+                break;
+            }
+            const double u = u_sample[ri];
+            if (warp == 0) {
+                double sk = 0.0;
+                int lk = -1;
+                if (lane < K) {
+                    const double2 v = __ldcg(sl + lane);
+                    sk = v.x;
+                    lk = (int)v.y;
+                }
+                double incl = sk;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const double y = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o)
+                        incl += y;
+                }
+                double excl = __shfl_up_sync(0xffffffffu, incl, 1);
+                if (lane == 0)
+                    excl = 0.0;
+                const unsigned hit = __ballot_sync(0xffffffffu, lane < K && excl + sk > u);
+                int lmax = lk;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1)
+                    lmax = max(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+                const int pick = hit ? __ffs(hit) - 1 : -1;
+                const double carry = __shfl_sync(0xffffffffu, excl, pick >= 0 ? pick : 0);
+                const int lpick = __shfl_sync(0xffffffffu, lk, pick >= 0 ? pick : 0);
+                if (lane == 0) {
+                    sh_pick = pick;
+                    sh_carry = carry;
+                    sh_token = pick >= 0 ? lpick : lmax;
+                }
+            }
+            __syncthreads();
+            const int pick = sh_pick;
+            if (pick == k) {
+                int token = chunk_scan<VEC>(lrow, x_lo, x_hi, V, st, table, sh_carry, u, shd, shi);
+                if (token == INT_MAX)   // the chunk's own sum fell short by rounding
+                    token = sh_token;
+                if (tid == 0) {
+                    out_tokens[(size_t)b * (Tmax + 1) + n_path] = token;
+                    n_accepted[b] = n_path;
+                }
+            } else if (pick < 0 && k == 0 && tid == 0) {
+                // Rounding left the total at or below u: the largest token with p > 0.
+                out_tokens[(size_t)b * (Tmax + 1) + n_path] = sh_token;
+                n_accepted[b] = n_path;
+            }
+            break;
         }
-        if (token == INT_MAX)   // the chunk's own total fell short by rounding
-            token = ws.chunk_last[(size_t)b * ws.nch + chosen];
-    }
-    if (tid == 0) {
-        out_tokens[(size_t)b * (Tmax + 1) + n_path] = token;
-        n_accepted[b] = n_path;
+        if (!alive) {
+            if (tid == 0)
+                flag(dev_status, TSD_DEV_TIMEOUT);
+            if (lead)
+                for (int bb = b; bb < B; bb += teams)
+                    n_accepted[bb] = -1;
+            return;
+        }
     }
 }
 
@@ -804,12 +821,11 @@ __global__ void __launch_bounds__(kDrawThreads)
 
 size_t verify_workspace(int B, int Tmax, int V)
 {
-    const size_t R = (size_t)B * (Tmax + 1), N = (size_t)B * Tmax;
-    const size_t C = (size_t)B * num_chunks(V);
-    return align256(R * sizeof(double)) + align256(N * sizeof(double)) +
-           align256(C * sizeof(double)) + 3 * align256(R * sizeof(int32_t)) +
-           align256(C * sizeof(int32_t));
+    (void)V;
+    return kWalkBytes + align256((size_t)B * (Tmax + 1) * sizeof(int32_t));
 }
+
+size_t verify_stochastic_scratch() { return kWalkBytes; }
 
 int launch_verify_greedy(const float *logits, const int32_t *tokens, const int32_t *parent,
                          const int32_t *n_nodes, const uint32_t *mask,
@@ -819,7 +835,7 @@ int launch_verify_greedy(const float *logits, const int32_t *tokens, const int32
 {
     if (B == 0)
         return TSD_OK;
-    const VerifyWs w = carve(ws, B, Tmax, V);
+    const VerifyWs w = carve(ws);
     greedy_rows_kernel<<<dim3(Tmax + 1, B), kRowThreads, 0, stream>>>(logits, n_nodes,
                                                                       first_child, Tmax, V,
                                                                       w.argmax);
@@ -831,6 +847,33 @@ int launch_verify_greedy(const float *logits, const int32_t *tokens, const int32
     return TSD_OK;
 }
 
+namespace {
+
+// CTAs of the walk kernel that fit on the device at once (cooperative
+// launch limit), capped by the workspace slots; looked up once per device.
+int walk_capacity(bool vec)
+{
+    constexpr int kMaxDevices = 64;
+    static int cap[2][kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return 0;
+    int &c = cap[vec ? 1 : 0][dev];
+    if (c == 0) {
+        int sms = 0, occ = 0, coop = 0;
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
+        const void *fn = vec ? reinterpret_cast<const void *>(mss_walk_kernel<true>)
+                             : reinterpret_cast<const void *>(mss_walk_kernel<false>);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, kWalkThreads, 0);
+        (void)cudaGetLastError();
+        c = coop ? std::min(sms * occ, kWalkMaxCtas) : -1;
+    }
+    return c;
+}
+
+}  // namespace
+
 int launch_verify_stochastic(const float *logits, double temperature, const float *q_probs,
                              int Rq, const int32_t *q_row, const int32_t *tokens,
                              const int32_t *n_nodes, const int32_t *first_child,
@@ -841,35 +884,42 @@ int launch_verify_stochastic(const float *logits, double temperature, const floa
 {
     if (B == 0)
         return TSD_OK;
-    const VerifyWs w = carve(ws, B, Tmax, V);
     const bool vec = (V & 3) == 0;
-    const dim3 rows(Tmax + 1, B), chunks(w.nch, B);
-    if (vec)
-        mss_rows_kernel<true><<<rows, kRowThreads, 0, stream>>>(
-            logits, temperature, q_probs, Rq, q_row, tokens, n_nodes, first_child, next_sibling,
-            u_accept, Tmax, V, w);
-    else
-        mss_rows_kernel<false><<<rows, kRowThreads, 0, stream>>>(
-            logits, temperature, q_probs, Rq, q_row, tokens, n_nodes, first_child, next_sibling,
-            u_accept, Tmax, V, w);
-    TSD_LAUNCH_CHECK();
-    if (vec)
-        mss_chunks_kernel<true><<<chunks, kDrawThreads, 0, stream>>>(
-            logits, temperature, q_probs, Rq, q_row, tokens, n_nodes, first_child, next_sibling,
-            Tmax, V, w);
-    else
-        mss_chunks_kernel<false><<<chunks, kDrawThreads, 0, stream>>>(
-            logits, temperature, q_probs, Rq, q_row, tokens, n_nodes, first_child, next_sibling,
-            Tmax, V, w);
-    TSD_LAUNCH_CHECK();
-    if (vec)
-        mss_finalize_kernel<true><<<B, kDrawThreads, 0, stream>>>(
-            logits, temperature, q_probs, Rq, q_row, tokens, n_nodes, first_child, next_sibling,
-            u_sample, Tmax, V, w, out_tokens, out_path, n_accepted, dev_status);
-    else
-        mss_finalize_kernel<false><<<B, kDrawThreads, 0, stream>>>(
-            logits, temperature, q_probs, Rq, q_row, tokens, n_nodes, first_child, next_sibling,
-            u_sample, Tmax, V, w, out_tokens, out_path, n_accepted, dev_status);
+    const int cap = walk_capacity(vec);
+    if (cap <= 0)
+        return TSD_ERR_CUDA;
+    // Team size: enough CTAs that each owns at least kTeamMinChunk entries
+    // (at most kTeamMax), as long as every sequence still gets a team.
+    const int k_want = std::max(1, std::min(kTeamMax, V / kTeamMinChunk));
+    int K, teams;
+    if ((long)B * k_want <= cap) {
+        K = k_want;
+        teams = B;
+    } else {
+        K = std::max(1, cap / B);
+        teams = std::min(B, cap / K);
+    }
+    int chunk = (V + K - 1) / K;
+    chunk = (chunk + 3) & ~3;
+    VerifyWs w = carve(ws);
+    if (cudaMemsetAsync(w.team, 0, (size_t)teams * sizeof(int2), stream) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return TSD_ERR_CUDA;
+    }
+    void *args[] = {(void *)&logits,      (void *)&temperature, (void *)&q_probs,
+                    (void *)&Rq,          (void *)&q_row,       (void *)&tokens,
+                    (void *)&n_nodes,     (void *)&first_child, (void *)&next_sibling,
+                    (void *)&u_accept,    (void *)&u_sample,    (void *)&B,
+                    (void *)&Tmax,        (void *)&V,           (void *)&K,
+                    (void *)&chunk,       (void *)&w,           (void *)&out_tokens,
+                    (void *)&out_path,    (void *)&n_accepted,  (void *)&dev_status};
+    const void *fn = vec ? reinterpret_cast<const void *>(mss_walk_kernel<true>)
+                         : reinterpret_cast<const void *>(mss_walk_kernel<false>);
+    if (cudaLaunchCooperativeKernel(fn, dim3(teams * K), dim3(kWalkThreads), args, 0, stream) !=
+        cudaSuccess) {
+        (void)cudaGetLastError();
+        return TSD_ERR_CUDA;
+    }
     TSD_LAUNCH_CHECK();
     return TSD_OK;
 }

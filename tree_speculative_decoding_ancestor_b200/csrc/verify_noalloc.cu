@@ -1,7 +1,8 @@
 // Stochastic tree verification for callers that cannot allocate device memory.
 //
-// tsd_tree_verify_stochastic needs a small scratch area (per-row statistics of
-// the logits and the residual normalisers).  Some callers have no way to
+// tsd_tree_verify_stochastic needs a small scratch area (the per-CTA partial
+// sums its teams exchange and their barrier counters; its size does not
+// depend on the problem).  Some callers have no way to
 // provide one: a serving engine that has already handed nearly all device
 // memory to its KV-cache pool, or code that reaches this library through a
 // plain C interface with no device allocator of its own.  For them this file
@@ -68,14 +69,14 @@ extern "C" int tsd_tree_verify_stochastic_noalloc(
         return TSD_ERR_NULL;
     if ((reinterpret_cast<uintptr_t>(logits) & 15u) || (reinterpret_cast<uintptr_t>(q_probs) & 15u))
         return TSD_ERR_ALIGN;
-    if (tsd::verify_workspace(B, Tmax, V) > kNoallocScratchBytes)
-        return TSD_ERR_WORKSPACE;   // beyond the fixed scratch: use the workspace call
+    if (tsd::verify_stochastic_scratch() > kNoallocScratchBytes)
+        return TSD_ERR_WORKSPACE;   // cannot happen with the constants above
     void *scratch = nullptr;
     const int rc = scratch_for_current_device(&scratch);
     if (rc != TSD_OK)
         return rc;
-    // The kernels write every scratch entry before reading it, so the
-    // contents a previous call left behind need no clearing.
+    // The launcher zeroes the team counters on the stream before the kernel;
+    // every other scratch entry is written before it is read.
     return tsd::launch_verify_stochastic(logits, temperature, q_probs, Rq, q_row, tokens, n_nodes,
                                          first_child, next_sibling, u_accept, u_sample, B, Tmax,
                                          V, out_tokens, out_path, n_accepted, scratch, dev_status,
