@@ -16,16 +16,18 @@
 //                      to bf16 and written back over the S columns
 //     O  += P V        tcgen05.mma with A = P from TMEM, B = V tile (MN-major)
 // The running max is only raised (O rescaled in TMEM) when a tile exceeds it
-// by more than 2^8, so rescales are rare while P stays below 256.  One
-// exponential in four is evaluated on the FMA pipe (ptx::exp2_fma), the other
-// three on MUFU.  Cache rows at or beyond P_b + T_b are zeroed in shared
-// memory before the PV product, so garbage there (NaN included) never leaks.
+// by more than 2^8, so rescales are rare while P stays below 256.  The
+// softmax issues few instructions per score (packed fp32x2 scaling and sums,
+// three-input max); with one softmax warp per SM sub-partition it is bound
+// by that warp's issue rate.  Cache rows at or beyond P_b + T_b are zeroed
+// in shared memory before the PV product, so garbage there (NaN included)
+// never leaks.  One mbarrier arrival per softmax warp (not per thread).
 //
 // Two kernels share this machinery:
 //   * tree_attn_rows_kernel (packed blocks of more than 128 rows): one CTA per
 //     (128-row block, (b, KV head), KV split); 6 warps -- TMA producer, MMA
-//     issuer, 4 softmax warps; TMEM holds two S buffers (so the next tile's
-//     scores are ready while the softmax works) and O.
+//     issuer, 4 softmax warps; TMEM holds three S buffers (the scores of the
+//     next two key tiles are ready while the softmax works) and O.
 //   * tree_attn_keysplit_kernel (at most 128 rows, e.g. MHA with small
 //     trees, where the KV stream is the bound): one CTA per ((b, KV head),
 //     split); two 4-warp softmax groups take the even and odd key tiles of
@@ -63,7 +65,7 @@ constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kOffQ + kTile;
 constexpr uint32_t kOffV = kOffK + NSK * kTile;
 constexpr uint32_t kOffBar = kOffV + NSV * kTile;
-constexpr int kNumBars = 1 + 2 * NSK + 2 * NSV + 2 + 4 + 2;
+constexpr int kNumBars = 1 + 2 * NSK + 2 * NSV + 12;
 constexpr uint32_t kOffMisc = kOffBar + 8 * kNumBars;
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;   // + alignment slack
 constexpr uint32_t kTmemCols = 512;
@@ -75,7 +77,7 @@ constexpr int kRowsThreads = 192;       // rows kernel: 6 warps
 constexpr int kSplitThreads = 384;      // key-split kernel: 12 warps
 
 // mbarrier addresses: q_full, k_full[NSK], k_empty[NSK], v_full[NSV],
-// v_empty[NSV], s_full[2], p_full[4], o_ready[2] -- consecutive 8-byte words.
+// v_empty[NSV], s_full[4], p_full[4], o_ready[4] -- consecutive 8-byte words.
 struct Bars {
     uint32_t base;
     __device__ uint32_t q_full() const { return base; }
@@ -84,8 +86,8 @@ struct Bars {
     __device__ uint32_t v_full(int s) const { return base + 8u * (1 + 2 * NSK + s); }
     __device__ uint32_t v_empty(int s) const { return base + 8u * (1 + 2 * NSK + NSV + s); }
     __device__ uint32_t s_full(int i) const { return base + 8u * (1 + 2 * NSK + 2 * NSV + i); }
-    __device__ uint32_t p_full(int i) const { return base + 8u * (3 + 2 * NSK + 2 * NSV + i); }
-    __device__ uint32_t o_ready(int i) const { return base + 8u * (7 + 2 * NSK + 2 * NSV + i); }
+    __device__ uint32_t p_full(int i) const { return base + 8u * (5 + 2 * NSK + 2 * NSV + i); }
+    __device__ uint32_t o_ready(int i) const { return base + 8u * (9 + 2 * NSK + 2 * NSV + i); }
 };
 
 // A wait whose outcome is the same on every lane of the warp (the TMEM
@@ -94,6 +96,16 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 {
     const bool ok = ptx::mbar_wait(bar, parity, abort);
     return __all_sync(0xffffffffu, ok);
+}
+
+// One arrival per warp: the lanes' prior writes (TMEM stores after their
+// wait::st and fence, or shared-memory stores after their proxy fence) are
+// ordered before lane 0's arrival by the warp barrier.
+__device__ __forceinline__ void warp_arrive(uint32_t bar)
+{
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0)
+        ptx::mbar_arrive(bar);
 }
 
 // K-major, 128-byte-swizzled operand made of two [rows][64] sub-tiles: the
@@ -170,12 +182,11 @@ __device__ __forceinline__ Setup cta_setup(uint8_t *smem_raw, uint32_t q_arrival
             ptx::mbar_init(su.bars.v_full(i), 1);
             ptx::mbar_init(su.bars.v_empty(i), 1);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < 4; ++i) {
             ptx::mbar_init(su.bars.s_full(i), 1);
             ptx::mbar_init(su.bars.o_ready(i), 1);
-        }
-        for (int i = 0; i < 4; ++i)
             ptx::mbar_init(su.bars.p_full(i), p_arrivals);
+        }
         *su.abort_flag = 0;
         ptx::fence_barrier_init();
         ptx::fence_proxy_async_smem();
@@ -294,13 +305,13 @@ struct RowCtx {
 __device__ __forceinline__ void load_q_row(const Setup &su, const __nv_bfloat16 *__restrict__ q,
                                            bool row_ok, size_t q_off, int t)
 {
+    uint8_t *dst = su.gbase + kOffQ;
     const uint4 *src = reinterpret_cast<const uint4 *>(q + q_off);
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
         const uint4 x = row_ok ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
         const int sub = c >> 3, cc = c & 7;
-        *reinterpret_cast<uint4 *>(su.gbase + kOffQ + sub * kSub + t * 128 +
-                                   ((cc ^ (t & 7)) * 16)) = x;
+        *reinterpret_cast<uint4 *>(dst + sub * kSub + t * 128 + ((cc ^ (t & 7)) * 16)) = x;
     }
     ptx::fence_proxy_async_smem();
 }
@@ -322,19 +333,23 @@ __device__ __forceinline__ void rescale_o(uint32_t taddr_o, float alpha)
 }
 
 // P = 2^(s * scale - m) for 64 scores (two 32-column chunks already loaded
-// and masked), packed to bf16 into pk[32]; returns their sum.
+// and masked), packed to bf16 into pk[32]; returns their sum.  The scaling
+// and the sums run on packed fp32 pairs, the exponentials on MUFU.
 __device__ __forceinline__ float exp_pack64(const uint32_t (&sa)[32], const uint32_t (&sb)[32],
                                             float scale_log2, float neg_m, uint32_t (&pk)[32])
 {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
-        const float p0 = ptx::ex2(fmaf(__uint_as_float(sa[2 * k]), scale_log2, neg_m));
-        const float p1 = ptx::ex2(fmaf(__uint_as_float(sa[2 * k + 1]), scale_log2, neg_m));
-        const float p2 = ptx::ex2(fmaf(__uint_as_float(sb[2 * k]), scale_log2, neg_m));
-        // one exponential in four on the FMA pipe, three on MUFU
-        const float p3 = ptx::exp2_fma(fmaf(__uint_as_float(sb[2 * k + 1]), scale_log2, neg_m));
-        acc[k & 3] += (p0 + p1) + (p2 + p3);
+        float x0, x1, x2, x3;
+        ptx::fma2_bc(x0, x1, __uint_as_float(sa[2 * k]), __uint_as_float(sa[2 * k + 1]),
+                     scale_log2, neg_m);
+        ptx::fma2_bc(x2, x3, __uint_as_float(sb[2 * k]), __uint_as_float(sb[2 * k + 1]),
+                     scale_log2, neg_m);
+        const float p0 = ptx::ex2(x0), p1 = ptx::ex2(x1), p2 = ptx::ex2(x2), p3 = ptx::ex2(x3);
+        const int a = (k & 1) * 2;
+        ptx::add2(acc[a], acc[a + 1], p0, p1);
+        ptx::add2(acc[a], acc[a + 1], p2, p3);
         pk[k] = ptx::pack_bf16(p0, p1);
         pk[16 + k] = ptx::pack_bf16(p2, p3);
     }
@@ -348,21 +363,21 @@ __device__ __forceinline__ void mask32(uint32_t (&s)[32], uint32_t bits)
         s[k] = ((bits >> k) & 1u) ? s[k] : __float_as_uint(-INFINITY);
 }
 
-__device__ __forceinline__ float max32x2(const uint32_t (&sa)[32], const uint32_t (&sb)[32],
-                                         float (&mx)[8])
+// Running maxima of 64 scores, 16 independent chains of 3-input maxima.
+__device__ __forceinline__ void max32x2(const uint32_t (&sa)[32], const uint32_t (&sb)[32],
+                                        float (&mx)[16])
 {
 #pragma unroll
-    for (int k = 0; k < 32; ++k) {
-        mx[k & 7] = fmaxf(mx[k & 7], __uint_as_float(sa[k]));
-        mx[k & 7] = fmaxf(mx[k & 7], __uint_as_float(sb[k]));
-    }
-    return 0.f;
+    for (int k = 0; k < 32; ++k)
+        mx[k & 15] = ptx::max3(mx[k & 15], __uint_as_float(sa[k]), __uint_as_float(sb[k]));
 }
 
-__device__ __forceinline__ float max8(const float (&mx)[8])
+__device__ __forceinline__ float max16(const float (&mx)[16])
 {
-    return fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+    float a = ptx::max3(mx[0], mx[1], mx[2]), b = ptx::max3(mx[3], mx[4], mx[5]);
+    float c = ptx::max3(mx[6], mx[7], mx[8]), d = ptx::max3(mx[9], mx[10], mx[11]);
+    float e = ptx::max3(mx[12], mx[13], mx[14]);
+    return ptx::max3(ptx::max3(a, b, c), ptx::max3(d, e, mx[15]), -INFINITY);
 }
 
 // Online-softmax step for one tile whose scores sit in TMEM columns col_s:
@@ -376,9 +391,9 @@ __device__ __forceinline__ bool softmax_tile(uint32_t taddr_s, uint32_t taddr_o,
 {
     const bool masked = !(pos0 + BN <= min(rc.P, rc.ke));
     // max over the raw scores (scale > 0 is applied once), two chunks at a time
-    float mx[8];
+    float mx[16];
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < 16; ++i)
         mx[i] = -INFINITY;
 #pragma unroll 1
     for (int c2 = 0; c2 < 2; ++c2) {
@@ -392,7 +407,7 @@ __device__ __forceinline__ bool softmax_tile(uint32_t taddr_s, uint32_t taddr_o,
         }
         max32x2(sa, sb, mx);
     }
-    const float mt = max8(mx) * rc.scale_log2;
+    const float mt = max16(mx) * rc.scale_log2;
     const bool need = mt > m_run + kRescaleThreshold;   // false if mt is -inf
     const float m_new = need ? mt : m_run;
     const float alpha = need ? ptx::ex2(m_run - m_new) : 1.f;   // 0 when m_run = -inf
@@ -468,9 +483,14 @@ __device__ __forceinline__ void write_row(uint32_t taddr_o, float inv, bool row_
 
 // ============================================================ rows kernel
 // More than 128 packed rows: one 128-row query tile per CTA, 6 warps (TMA
-// producer, MMA issuer, 4 softmax warps).  The MMA warp computes S for tile
-// j + 1 into the other S buffer while the softmax works on tile j.
-// TMEM: S0 [0,128) | S1 [128,256) | O [256,384).
+// producer, MMA issuer, 4 softmax warps).  Three S buffers: the MMA warp
+// keeps the scores of the next two key tiles ready while the softmax works
+// on tile j, so the softmax never waits on the PV -> QK chain.
+// TMEM: S0 [0,128) | S1 [128,256) | S2 [256,384) | O [384,512).
+// MMA order: QK_0 QK_1 QK_2, then per tile j: PV_j QK_{j+3}; P_j is read out
+// of S_{j%3} by PV_j before QK_{j+3}, issued after it by the same thread,
+// overwrites it.  PV_j commits to o_ready[j%3], so a wait for "PV_{j-1}
+// done" names a phase that can be neither stale nor ahead.
 __global__ void __launch_bounds__(kRowsThreads, 1)
     tree_attn_rows_kernel(const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV,
@@ -498,37 +518,37 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
     if (rb * BQ >= R || kb >= ke)
         return;   // no rows or no keys: the partials stay empty
     const int ntiles = (ke - kb + BN - 1) / BN;
-    const Setup su = cta_setup(smem_raw, BQ, BQ);
+    const Setup su = cta_setup(smem_raw, 4, 4);   // arrivals: softmax warps
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    auto col_s = [](int i) { return (uint32_t)(i & 1) * 128u; };   // S buffer of tile i
-    constexpr uint32_t kO = 256u;
+    constexpr int NS = 3;   // S buffers
+    auto col_s = [](int i) { return (uint32_t)(i % NS) * 128u; };
+    constexpr uint32_t kO = 384u;
 
     if (warp == 0) {
         if (lane == 0)
             produce_kv(su, &tmK, &tmV, b * Hkv + hk, kb, ntiles);
     } else if (warp == 1) {
-        // QK_0, then per tile j: QK_{j+1} (other S buffer), PV_j.
         bool ok = warp_wait(su.bars.q_full(), 0, su.abort_flag);
         ptx::tc_fence_after();
-        for (int i = 0; ok && i <= ntiles; ++i) {
-            if (i < ntiles) {
-                if (!warp_wait(su.bars.k_full(i % NSK), (i / NSK) & 1, su.abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                ptx::tc_fence_after();
-                issue_qk(su, lane, col_s(i), i, su.bars.s_full(i & 1));
+        auto qk = [&](int i) {
+            if (!warp_wait(su.bars.k_full(i % NSK), (i / NSK) & 1, su.abort_flag))
+                return false;
+            ptx::tc_fence_after();
+            issue_qk(su, lane, col_s(i), i, su.bars.s_full(i % NS));
+            return true;
+        };
+        for (int i = 0; ok && i < min(NS, ntiles); ++i)
+            ok = qk(i);
+        for (int j = 0; ok && j < ntiles; ++j) {
+            if (!warp_wait(su.bars.p_full(j % NS), (j / NS) & 1, su.abort_flag) ||
+                !warp_wait(su.bars.v_full(j % NSV), (j / NSV) & 1, su.abort_flag)) {
+                ok = false;
+                break;
             }
-            if (i >= 1) {
-                const int j = i - 1;
-                if (!warp_wait(su.bars.p_full(j & 1), (j >> 1) & 1, su.abort_flag) ||
-                    !warp_wait(su.bars.v_full(j % NSV), (j / NSV) & 1, su.abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                issue_pv(su, lane, col_s(j), kO, j, j > 0, P + T - (kb + j * BN),
-                         su.bars.o_ready(0));
-            }
+            issue_pv(su, lane, col_s(j), kO, j, j > 0, P + T - (kb + j * BN),
+                     su.bars.o_ready(j % NS));
+            if (j + NS < ntiles)
+                ok = qk(j + NS);
         }
     } else {
         // softmax warps 2..5: one query row per thread == TMEM lane
@@ -540,17 +560,20 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
         const int u = row_ok ? r / G : 0;
         const int h = hk * G + (row_ok ? r % G : 0);
         load_q_row(su, q, row_ok, (((size_t)b * Tmax + u) * Hq + h) * HD, t);
-        ptx::mbar_arrive(su.bars.q_full());
+        warp_arrive(su.bars.q_full());
         uint32_t mw[4];
 #pragma unroll
         for (int w = 0; w < 4; ++w)
             mw[w] = (row_ok && w < W) ? mask[((size_t)b * Tmax + u) * W + w] : 0u;
         const uint32_t taddr_o = su.tmem + lane_off + kO;
+        // PV_i done (o_ready[i % 3] completes once per tile of that class)
+        auto wait_pv = [&](int i) {
+            return warp_wait(su.bars.o_ready(i % NS), (i / NS) & 1, su.abort_flag);
+        };
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
         for (int j = 0; ok && j < ntiles; ++j) {
-            const int sb = j & 1;
-            if (!warp_wait(su.bars.s_full(sb), (j >> 1) & 1, su.abort_flag)) {
+            if (!warp_wait(su.bars.s_full(j % NS), (j / NS) & 1, su.abort_flag)) {
                 ok = false;
                 break;
             }
@@ -568,19 +591,19 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
                 for (int c = 0; c < 4; ++c)
                     mask32(sr[c], valid_bits(pos0 + c * 32, P, ke, mw));
             }
-            float mx[8];
+            float mx[16];
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
+            for (int i = 0; i < 16; ++i)
                 mx[i] = -INFINITY;
             max32x2(sr[0], sr[1], mx);
             max32x2(sr[2], sr[3], mx);
-            const float mt = max8(mx) * scale_log2;
+            const float mt = max16(mx) * scale_log2;
             const bool need = mt > m_run + kRescaleThreshold;   // false if mt is -inf
             const float m_new = need ? mt : m_run;
             const float alpha = need ? ptx::ex2(m_run - m_new) : 1.f;   // 0 when m_run = -inf
             if (__any_sync(0xffffffffu, need) && j > 0) {
                 // O holds PV_0 .. PV_{j-1}: wait for the last of them.
-                if (!warp_wait(su.bars.o_ready(0), (j - 1) & 1, su.abort_flag)) {
+                if (!wait_pv(j - 1)) {
                     ok = false;
                     break;
                 }
@@ -598,9 +621,9 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
             }
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
-            ptx::mbar_arrive(su.bars.p_full(sb));
+            warp_arrive(su.bars.p_full(j % NS));
         }
-        if (ok && warp_wait(su.bars.o_ready(0), (ntiles - 1) & 1, su.abort_flag)) {
+        if (ok && wait_pv(ntiles - 1)) {
             ptx::tc_fence_after();
             const size_t row = ((size_t)b * Tmax + u) * Hq + h;
             const size_t nrows = (size_t)gridDim.y / Hkv * Tmax * Hq;
@@ -646,7 +669,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
     if (R <= 0 || kb >= ke)
         return;
     const int ntiles = (ke - kb + BN - 1) / BN;
-    const Setup su = cta_setup(smem_raw, 2 * BQ, BQ);
+    const Setup su = cta_setup(smem_raw, 8, 4);   // arrivals: softmax warps
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     auto col_s = [](int s) { return (uint32_t)s * 128u; };
     auto col_o = [](int s) { return 256u + (uint32_t)s * 128u; };
@@ -690,7 +713,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
         const int h = hk * G + (row_ok ? t % G : 0);
         if (s == 0)
             load_q_row(su, q, row_ok, (((size_t)b * Tmax + u) * Hq + h) * HD, t);
-        ptx::mbar_arrive(su.bars.q_full());
+        warp_arrive(su.bars.q_full());
         RowCtx rc;
         rc.P = P;
         rc.ke = ke;
@@ -713,7 +736,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
             if (!ok)
                 break;
             ptx::tc_fence_before();
-            ptx::mbar_arrive(su.bars.p_full(s));
+            warp_arrive(su.bars.p_full(s));
         }
         const bool have = ok && my_tiles > 0 &&
                           warp_wait(su.bars.o_ready(s), (my_tiles - 1) & 1, su.abort_flag);
@@ -850,6 +873,7 @@ cudaError_t set_smem_attributes()
             err = cudaFuncSetAttribute(tree_attn_keysplit_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
+
     });
     return err;
 }

@@ -224,29 +224,39 @@ __device__ __forceinline__ float ex2(float x)
     return y;
 }
 
-// 2^x on the FMA/ALU pipes, for spreading the softmax's exponentials over
-// more than the MUFU unit.  Cody-Waite style split x = j + f with j the
-// nearest integer (the 1.5 * 2^23 rounding trick, so j also lands in the low
-// bits of t) and f in [-1/2, 1/2]; 2^f from a degree-3 polynomial whose
-// coefficients were fitted for minimum relative error on [-1/2, 1/2]
-// (Lawson's iteratively reweighted least squares): max relative error 7.5e-5,
-// far below the bf16 rounding (2^-9) the result goes through.  j is added to
-// the exponent field with one integer multiply-add.  Returns 0 for x < -125
-// (below that the result would leave the normal range; as a softmax weight
-// next to a row maximum of 1 it is 0 in bf16 anyway).
-__device__ __forceinline__ float exp2_fma(float x)
+// Packed fp32 pairs (sm_100): (d0, d1) = (a0, a1) * b + c, b and c broadcast.
+__device__ __forceinline__ void fma2_bc(float &d0, float &d1, float a0, float a1, float b, float c)
 {
-    constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
-    const float t = x + kRound;
-    const float f = x - (t - kRound);
-    float p = fmaf(0x1.c3f6e2p-5f, f, 0x1.f0ddf0p-3f);
-    p = fmaf(p, f, 0x1.62f31ap-1f);
-    p = fmaf(p, f, 0x1.fff694p-1f);
-    const int bits = __float_as_int(t) * (1 << 23) + __float_as_int(p);
-    return x < -125.0f ? 0.0f : __int_as_float(bits);
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %4};\n\t"
+        "mov.b64 rc, {%5, %5};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b), "f"(c));
 }
 
-// Two floats -> packed bf16x2 (lo in the low half), round to nearest even.
+// (s0, s1) += (a0, a1)
+__device__ __forceinline__ void add2(float &s0, float &s1, float a0, float a1)
+{
+    asm("{\n\t.reg .b64 ra, rs;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rs, {%0, %1};\n\t"
+        "add.f32x2 rs, rs, ra;\n\t"
+        "mov.b64 {%0, %1}, rs;\n\t}"
+        : "+f"(s0), "+f"(s1)
+        : "f"(a0), "f"(a1));
+}
+
+// Three-input maximum (sm_100).
+__device__ __forceinline__ float max3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
 {
     uint32_t r;
