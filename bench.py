@@ -58,6 +58,24 @@ def _dist():
     return ws, rank, local
 
 
+def rank_workload(cfg: int, rank: int, B=None):
+    """Weak scaling: every rank verifies its own batch of independent
+    sequences, drawn with a seed of its own (rank 0 = the single-GPU batch)."""
+    return gen.config_workload(cfg, seed=gen.SEED_BASE + cfg + 1000 * rank, B=B)
+
+
+def reduce_over_ranks(pg, device, tokens: int, ms: float):
+    """Whole-job tokens (sum over ranks) and the slowest rank's time (max over
+    ranks).  Every rank makes the same two collective calls, in this order."""
+    if pg is None:
+        return tokens, ms
+    n = torch.tensor([float(tokens)], dtype=torch.float64, device=device)
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    pg.all_reduce(n, op=pg.ReduceOp.SUM)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return int(n.item()), float(t.item())
+
+
 # ----------------------------------------------------------------- work
 def attn_flops(w) -> int:
     """4*D flops per (query row, attended key): prefix + ancestors-or-self."""
@@ -285,7 +303,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         pg = dist
     # weak scaling: every rank verifies its own batch (a different seed per rank)
-    w = gen.config_workload(cfg, seed=gen.SEED_BASE + cfg + 1000 * rank, B=args.batch)
+    w = rank_workload(cfg, rank, args.batch)
     step = Step(w, dev, tsd)
     tokens_per_step = int(w.n_nodes.sum())
 
@@ -324,13 +342,9 @@ def main():
     clk = _clock_summary(clocks)
     step_ms = [a.elapsed_time(b) for a, b in st_ev]
     att_ms = [a.elapsed_time(b) for a, b in att_ev]
-    total_ms = float(sum(step_ms))
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if pg:
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-    total_ms = float(t.item())
+    job_tokens, total_ms = reduce_over_ranks(pg, dev, tokens_per_step, float(sum(step_ms)))
     ms_per_step = total_ms / args.steps
-    value = ws * tokens_per_step / (ms_per_step / 1e3)
+    value = job_tokens / (ms_per_step / 1e3)
     if int(tsd.device_status(dev).item()) != 0:
         raise RuntimeError("device status set during the timed steps")
 
@@ -422,12 +436,9 @@ def e2e(w, dev, tsd, args, pg, ws):
         one()
     e1.record()
     torch.cuda.synchronize(dev)
-    ms = e0.elapsed_time(e1) / steps
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if pg:
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-    ms = float(t.item())
-    return {"value": ws * int(w.n_nodes.sum()) / (ms / 1e3), "unit": UNIT,
+    job_tokens, ms = reduce_over_ranks(pg, dev, int(w.n_nodes.sum()),
+                                       e0.elapsed_time(e1) / steps)
+    return {"value": job_tokens / (ms / 1e3), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
             "ms_per_step": ms}
 
