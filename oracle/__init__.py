@@ -30,7 +30,7 @@ _lock = threading.Lock()
 _lib: Optional[ctypes.CDLL] = None
 
 SENTINEL = -7
-BAD_TREE, BAD_TOKEN, BAD_QROW = 1, 2, 4
+BAD_TREE, BAD_TOKEN, BAD_QROW, BAD_PATH = 1, 2, 4, 32
 
 
 def build(force: bool = False) -> str:
@@ -220,6 +220,25 @@ def verify_stochastic(logits, temperature: float, q_probs, q_row, tokens, parent
                                  _p(st))
     return dict(out_tokens=out_tokens, out_path=out_path, n_accepted=n_acc, n_flagged=nflag,
                 n_decisions=ndec, status=st)
+
+
+def kv_commit(k_cache, v_cache, prefix_len, out_path, n_accepted) -> Dict[str, np.ndarray]:
+    """Move the accepted nodes' K/V rows to the positions right after the
+    prefix.  Works on copies: returns the new caches (same dtype/shape as
+    the inputs, as numpy arrays; bf16 as raw uint16), new_prefix and status."""
+    lib = _load()
+    ka = _np(k_cache).copy()
+    va = _np(v_cache).copy()
+    B, Hkv, Lmax, D = ka.shape
+    path = _np(out_path, np.int32)
+    Tmax = path.shape[1]
+    nacc = _np(n_accepted, np.int32)
+    pl = _np(prefix_len, np.int32)
+    newp = np.full(B, SENTINEL, dtype=np.int32)
+    st = np.zeros(B, dtype=np.int32)
+    lib.oracle_kv_commit(_p(ka), _p(va), _p(pl), _p(path), _p(nacc), B, Tmax, Hkv, Lmax,
+                         D * ka.itemsize, _p(newp), _p(st))
+    return dict(k_cache=ka, v_cache=va, new_prefix=newp, status=st)
 
 
 # Convenience wrappers over a workloads.Workload -----------------------------

@@ -18,6 +18,10 @@
  *     flatkey.ai speculative decoding guide (its verification diagram).
  *   - stochastic verification: "ツリー検証アルゴリズム", the P_accept equation
  *     min(1, P_LLM/P_SSM) and the residual equation norm(max(0, P_LLM-P_SSM)).
+ *   - committing the accepted path: "Tree Attention のカーネル融合", item 2
+ *     (the tree's KV entries stay consistent with the existing KV cache),
+ *     and the flatkey.ai guide's verification diagram (the accepted prefix
+ *     is committed).
  *
  * Readings taken where the page is silent (each one is listed in the design
  * notes of the repository):
@@ -36,7 +40,10 @@
  *     sequence with a draw at its own row using u_sample[row];
  *   - greedy: the longest root path all of whose tokens equal the argmax of
  *     their parent's row (lowest token id on argmax ties, lowest terminal
- *     node index on length ties), then the argmax of the terminal's row.
+ *     node index on length ties), then the argmax of the terminal's row;
+ *   - commit: the accepted nodes' K and V rows move to the positions right
+ *     after the prefix, in path order, and the prefix grows by their number
+ *     (the final sampled token has no KV entry yet).
  */
 #include <math.h>
 #include <stdint.h>
@@ -49,6 +56,7 @@
 #define ORACLE_BAD_TREE 1
 #define ORACLE_BAD_TOKEN 2
 #define ORACLE_BAD_QROW 4
+#define ORACLE_BAD_PATH 32
 
 /* dtype 0: IEEE fp32, dtype 1: bfloat16 (upper 16 bits of an fp32). */
 static double load_value(const void *base, size_t i, int dtype)
@@ -454,5 +462,55 @@ int oracle_verify_stochastic(const float *logits, double temperature, const floa
         }
         free(p);
     }
+    return any;
+}
+
+/* Commit of the accepted path.  For each sequence b with n = n_accepted[b]
+ * >= 0 and path u_0..u_{n-1} = out_path[b][0..n-1]: for every KV head, the
+ * K row and the V row at cache position P_b + u_i move to P_b + i, all at
+ * once (every source is read before any destination is written), and
+ * new_prefix[b] = P_b + n.  Rows are moved as raw bytes.  Sequences with
+ * n < 0 are left alone (new_prefix = P_b).  A path that is not a strictly
+ * increasing list of node indices in [0, Tmax), longer than Tmax, or that
+ * reaches past Lmax, sets status[b] = ORACLE_BAD_PATH and moves nothing. */
+int oracle_kv_commit(unsigned char *k, unsigned char *v, const int32_t *prefix_len,
+                     const int32_t *out_path, const int32_t *n_accepted, int B, int Tmax, int Hkv,
+                     int Lmax, int row_bytes, int32_t *new_prefix, int32_t *status)
+{
+    int any = 0;
+    unsigned char *tmp = (unsigned char *)malloc((size_t)(Tmax > 0 ? Tmax : 1) * row_bytes);
+    for (int b = 0; b < B; ++b) {
+        const int n = n_accepted[b], P = prefix_len[b];
+        const int32_t *path = out_path + (size_t)b * Tmax;
+        new_prefix[b] = P;
+        status[b] = 0;
+        if (n < 0)
+            continue;
+        int ok = n <= Tmax && P >= 0;
+        for (int i = 0; ok && i < n; ++i) {
+            const int u = path[i];
+            if (u < 0 || u >= Tmax || (i > 0 && u <= path[i - 1]) || P + u >= Lmax)
+                ok = 0;
+        }
+        if (!ok) {
+            status[b] = ORACLE_BAD_PATH;
+            any |= ORACLE_BAD_PATH;
+            continue;
+        }
+        for (int h = 0; h < Hkv; ++h) {
+            unsigned char *planes[2] = {k, v};
+            for (int t = 0; t < 2; ++t) {
+                unsigned char *base = planes[t] + ((size_t)b * Hkv + h) * Lmax * row_bytes;
+                for (int i = 0; i < n; ++i)
+                    memcpy(tmp + (size_t)i * row_bytes,
+                           base + (size_t)(P + path[i]) * row_bytes, row_bytes);
+                for (int i = 0; i < n; ++i)
+                    memcpy(base + (size_t)(P + i) * row_bytes, tmp + (size_t)i * row_bytes,
+                           row_bytes);
+            }
+        }
+        new_prefix[b] = P + n;
+    }
+    free(tmp);
     return any;
 }

@@ -11,6 +11,7 @@ import pytest
 
 import oracle
 import test_oracle_attention as pa
+import test_oracle_commit as pc
 import test_oracle_greedy as pg
 import test_oracle_mask as pm
 import test_oracle_stochastic as ps
@@ -54,6 +55,11 @@ MUTATIONS = {
     "temperature_ignored": ("- m) / temperature)", "- m) / 1.0)",
                             lambda: ps.test_no_tree_draw_is_inverse_cdf(0.5)),
     "child_uses_root_row": ("int row = cur + 1;", "int row = 0;", ps.test_chi_square_depth_two),
+    # commit of the accepted path
+    "commit_ignores_prefix": ("base + (size_t)(P + path[i]) * row_bytes", "base + (size_t)(path[i]) * row_bytes",
+                              lambda: pc.test_commit_then_decode_equals_tree_attention(1, "bf16")),
+    "commit_reverses_order": ("memcpy(base + (size_t)(P + i) * row_bytes", "memcpy(base + (size_t)(P + n - 1 - i) * row_bytes",
+                              lambda: pc.test_committed_rows_follow_the_verified_tokens_in_order("greedy")),
 }
 
 
