@@ -347,6 +347,7 @@ def main():
     value = job_tokens / (ms_per_step / 1e3)
     if int(tsd.device_status(dev).item()) != 0:
         raise RuntimeError("device status set during the timed steps")
+    commit = time_commit(step, dev, tsd)
 
     peaks, peak_kind = _peaks()
     att_s = statistics.mean(att_ms) / 1e3
@@ -384,7 +385,8 @@ def main():
                        else f"inputs larger than L2 ({working / 1e6:.0f} MB read per step)",
                        "parallelism": f"batch-sharded x{ws} (independent sequences)"},
             "kv_cache_gbs": kv_gbs, "kv_cache_frac_of_hbm": kv_gbs / peaks["hbm_gbs"],
-            "roofline": roof, "gpu_launches": launches, "clocks": clk}
+            "roofline": roof, "gpu_launches": launches, "clocks": clk,
+            "kv_commit": commit}
 
     if not args.no_e2e:
         line["e2e"] = e2e(w, dev, tsd, args, pg, ws)
@@ -394,6 +396,40 @@ def main():
         print(json.dumps(line), flush=True)
     if pg:
         pg.destroy_process_group()
+
+
+def time_commit(step, dev, tsd, reps: int = 20):
+    """The step after verification (outside the metric's step): move the
+    accepted nodes' K/V rows after the prefix.  Timed alone with CUDA events
+    on the verify result of the last step (repeating it moves the same rows
+    again, which costs the same).  The kernel takes a few microseconds, less
+    than the Python call around it, so the reps are captured in a CUDA graph
+    and the replay is timed."""
+    w, d = step.w, step.d
+    res = step.s if "stochastic" in w.verify else step.g
+    n = int(res.n_accepted.clamp(min=0).sum().item())
+    row = w.D * d["k_cache"].element_size()
+    newp = torch.empty_like(d["prefix_len"])
+    tsd.kv_commit(d["k_cache"], d["v_cache"], d["prefix_len"], res, new_prefix_len=newp)
+    torch.cuda.synchronize(dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(reps):
+            tsd.kv_commit(d["k_cache"], d["v_cache"], d["prefix_len"], res, new_prefix_len=newp)
+    graph.replay()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    graph.replay()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    del graph
+    if int(tsd.device_status(dev).item()) != 0:
+        raise RuntimeError("device status set by the commit")
+    us = e0.elapsed_time(e1) * 1e3 / reps
+    moved = 4 * n * w.Hkv * row   # K and V rows, read once and written once
+    return {"us": us, "accepted_nodes": n, "algorithmic_bytes": moved,
+            "gbs": moved / (us * 1e-6) / 1e9 if us > 0 else None}
 
 
 def e2e(w, dev, tsd, args, pg, ws):

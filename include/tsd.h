@@ -69,7 +69,8 @@ enum tsd_dev_status {
     TSD_DEV_BAD_TOKEN = 2,    /* a token id outside [0, V)                  */
     TSD_DEV_BAD_QROW = 4,     /* a q_row index outside [0, Rq)              */
     TSD_DEV_BAD_PREFIX = 8,   /* prefix_len[b] + n_nodes[b] > Lmax or < 0   */
-    TSD_DEV_TIMEOUT = 16      /* a bounded pipeline wait expired (kernel bailed out) */
+    TSD_DEV_TIMEOUT = 16,     /* a bounded pipeline wait expired (kernel bailed out) */
+    TSD_DEV_BAD_PATH = 32     /* an accepted path that is not a valid commit list     */
 };
 
 /* Element types of Q / K / V / attention output. */
@@ -208,6 +209,31 @@ int tsd_tree_verify_stochastic(const float *logits, double temperature, const fl
                                int32_t *out_tokens, int32_t *out_path, int32_t *n_accepted,
                                void *workspace, size_t workspace_bytes, int32_t *dev_status,
                                tsd_stream_t stream);
+
+/*
+ * Commit of the accepted path ("Tree Attention のカーネル融合", item 2: the
+ * tree's KV entries stay consistent with the existing KV cache; the
+ * flatkey.ai guide's verification diagram: the accepted prefix is committed).
+ * For every sequence b with n = n_accepted[b] >= 0 and accepted nodes
+ * u_i = out_path[b][i] (i < n, as the verify calls write them), the K and V
+ * rows of every KV head at cache position P_b + u_i move to P_b + i, in place,
+ * all at once (no row is written before every source has been read), and
+ * new_prefix_len[b] = P_b + n.  The final sampled token has no KV entry yet.
+ *   k_cache, v_cache  [B][Hkv][Lmax][D] (dtype TSD_BF16 or TSD_F32), in/out
+ *   prefix_len        [B] int32, P_b before the commit
+ *   out_path          [B][Tmax] int32, n_accepted [B] int32 (verify outputs)
+ *   new_prefix_len    [B] int32, out (P_b for a skipped sequence)
+ * Sequences with n_accepted < 0 are skipped silently (their verify call
+ * already reported why).  A path that is not strictly increasing, leaves
+ * [0, Tmax), is longer than Tmax or reaches past Lmax moves nothing and sets
+ * TSD_DEV_BAD_PATH.  Pointers 16-byte aligned; D * element size a multiple
+ * of 16 and at most 512 bytes.  Host errors: TSD_ERR_NULL, TSD_ERR_SHAPE,
+ * TSD_ERR_DTYPE, TSD_ERR_ALIGN, TSD_ERR_CUDA.  Device: TSD_DEV_BAD_PATH.
+ */
+int tsd_kv_commit(void *k_cache, void *v_cache, const int32_t *prefix_len,
+                  const int32_t *out_path, const int32_t *n_accepted, int B, int Tmax, int Hkv,
+                  int D, int Lmax, int dtype, int32_t *new_prefix_len, int32_t *dev_status,
+                  tsd_stream_t stream);
 
 /*
  * Stochastic verification without a workspace, for callers that cannot

@@ -1,12 +1,13 @@
 """B200-native verification hot path of tree speculative decoding (SpecInfer).
 
-Four calls, each a thin wrapper over the C ABI of ``lib/libtsd.so``
+Five calls, each a thin wrapper over the C ABI of ``lib/libtsd.so``
 (``include/tsd.h``):
 
 * :func:`tree_mask_build`     -- ancestor bitmask / depth / child lists from ``parent[]``;
 * :func:`tree_attention`      -- topology-aware tree attention over prefix KV + ancestors;
 * :func:`tree_verify_greedy`  -- longest argmax-matching root path + one bonus token;
-* :func:`tree_verify_stochastic` -- multi-step speculative sampling (exact target distribution).
+* :func:`tree_verify_stochastic` -- multi-step speculative sampling (exact target distribution);
+* :func:`kv_commit`           -- move the accepted nodes' K/V rows after the prefix.
 """
 
 from .binding import (  # noqa: F401
@@ -17,6 +18,7 @@ from .binding import (  # noqa: F401
     attention_workspace_size,
     device_status,
     exported_symbols,
+    kv_commit,
     launch_count,
     load_library,
     tree_attention,

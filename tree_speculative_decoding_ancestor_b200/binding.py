@@ -24,6 +24,7 @@ TSD_F32, TSD_BF16 = 0, 1
 TSD_MAX_TREE = 128
 TSD_TREE_INVALID = -2
 DEV_BAD_TREE, DEV_BAD_TOKEN, DEV_BAD_QROW, DEV_BAD_PREFIX, DEV_TIMEOUT = 1, 2, 4, 8, 16
+DEV_BAD_PATH = 32
 
 _lock = threading.Lock()
 _lib: Optional[ctypes.CDLL] = None
@@ -48,6 +49,7 @@ _SIGNATURES: Dict[str, Tuple[object, list]] = {
                                         _I, _I, _I, _P, _P, _P, _P, _SZ, _P, _P]),
     "tsd_tree_verify_stochastic_noalloc": (_I, [_P, ctypes.c_double, _P, _I, _P, _P, _P, _P, _P,
                                                 _P, _P, _I, _I, _I, _P, _P, _P, _P, _P]),
+    "tsd_kv_commit": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
 }
 
 
@@ -291,8 +293,8 @@ def tree_verify_stochastic_noalloc(logits: torch.Tensor, temperature: float,
     """tree_verify_stochastic for callers that cannot allocate device memory:
     the scratch lives in a fixed array inside the library, so the caller
     passes preallocated outputs and nothing is allocated here (see
-    tsd_tree_verify_stochastic_noalloc in include/tsd.h for the size limit,
-    the first-call set-up and why overlapping calls race)."""
+    tsd_tree_verify_stochastic_noalloc in include/tsd.h for the fixed
+    scratch, the first-call set-up and why overlapping calls race)."""
     lib = load_library()
     dev = logits.device
     B, R, V = logits.shape
@@ -313,3 +315,31 @@ def tree_verify_stochastic_noalloc(logits: torch.Tensor, temperature: float,
         _ptr(out.n_accepted), _ptr(st), _stream(dev))
     _check(rc, "tsd_tree_verify_stochastic_noalloc")
     return out
+
+
+def kv_commit(k_cache: torch.Tensor, v_cache: torch.Tensor, prefix_len: torch.Tensor,
+              result: VerifyResult, new_prefix_len: Optional[torch.Tensor] = None,
+              status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Move the accepted nodes' K/V rows (in place) to the positions right
+    after each sequence's prefix; returns the new prefix lengths [B] int32."""
+    lib = load_library()
+    dev = k_cache.device
+    B, Hkv, Lmax, D = k_cache.shape
+    Tmax = result.out_path.shape[1]
+    dt = {torch.float32: TSD_F32, torch.bfloat16: TSD_BF16}.get(k_cache.dtype)
+    if dt is None:
+        raise TypeError("k_cache must be float32 or bfloat16")
+    _need(k_cache, "k_cache", k_cache.dtype, (B, Hkv, Lmax, D), dev)
+    _need(v_cache, "v_cache", k_cache.dtype, (B, Hkv, Lmax, D), dev)
+    _need(prefix_len, "prefix_len", torch.int32, (B,), dev)
+    _need(result.out_path, "out_path", torch.int32, (B, Tmax), dev)
+    _need(result.n_accepted, "n_accepted", torch.int32, (B,), dev)
+    if new_prefix_len is None:
+        new_prefix_len = torch.empty((B,), dtype=torch.int32, device=dev)
+    _need(new_prefix_len, "new_prefix_len", torch.int32, (B,), dev)
+    st = device_status(dev) if status is None else status
+    rc = lib.tsd_kv_commit(_ptr(k_cache), _ptr(v_cache), _ptr(prefix_len), _ptr(result.out_path),
+                           _ptr(result.n_accepted), B, Tmax, Hkv, D, Lmax, dt,
+                           _ptr(new_prefix_len), _ptr(st), _stream(dev))
+    _check(rc, "tsd_kv_commit")
+    return new_prefix_len

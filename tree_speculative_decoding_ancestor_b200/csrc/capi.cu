@@ -187,4 +187,27 @@ int tsd_tree_verify_stochastic(const float *logits, double temperature, const fl
                                          dev_status, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int tsd_kv_commit(void *k_cache, void *v_cache, const int32_t *prefix_len,
+                  const int32_t *out_path, const int32_t *n_accepted, int B, int Tmax, int Hkv,
+                  int D, int Lmax, int dtype, int32_t *new_prefix_len, int32_t *dev_status,
+                  tsd_stream_t stream)
+{
+    if (B < 0 || Tmax < 1 || Tmax > TSD_MAX_TREE || Hkv < 1 || D < 1 || Lmax < 1)
+        return TSD_ERR_SHAPE;
+    if (dtype != TSD_F32 && dtype != TSD_BF16)
+        return TSD_ERR_DTYPE;
+    const int row_bytes = D * (dtype == TSD_F32 ? 4 : 2);
+    if (row_bytes % 16 != 0 || row_bytes > 512)
+        return TSD_ERR_SHAPE;
+    if (B == 0)
+        return TSD_OK;
+    if (!k_cache || !v_cache || !prefix_len || !out_path || !n_accepted || !new_prefix_len)
+        return TSD_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(k_cache) & 15u) || (reinterpret_cast<uintptr_t>(v_cache) & 15u))
+        return TSD_ERR_ALIGN;
+    return tsd::launch_kv_commit(k_cache, v_cache, prefix_len, out_path, n_accepted, B, Tmax,
+                                 Hkv, Lmax, row_bytes, new_prefix_len, dev_status,
+                                 reinterpret_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

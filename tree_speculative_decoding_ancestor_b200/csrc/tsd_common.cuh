@@ -101,6 +101,10 @@ int launch_umma_attention(const AttnArgs &a, void *ws, size_t ws_bytes, int num_
 
 size_t verify_workspace(int B, int Tmax, int V);
 size_t verify_stochastic_scratch();   // fixed: independent of the shape
+int launch_kv_commit(void *k_cache, void *v_cache, const int32_t *prefix_len,
+                     const int32_t *out_path, const int32_t *n_accepted, int B, int Tmax, int Hkv,
+                     int Lmax, int row_bytes, int32_t *new_prefix, int32_t *dev_status,
+                     cudaStream_t stream);
 int launch_verify_greedy(const float *logits, const int32_t *tokens, const int32_t *parent,
                          const int32_t *n_nodes, const uint32_t *mask,
                          const int32_t *first_child, int B, int Tmax, int V,
