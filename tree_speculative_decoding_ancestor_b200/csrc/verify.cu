@@ -22,10 +22,12 @@
 //                           numbers); after a rejection the team sums
 //                           S = sum max(0, p - q_c) and p becomes
 //                           max(0, p - q_c) / S.  An accepted child's row is
-//                           next.  Where the walk stops, the team sums the
-//                           final distribution per chunk; the chunk whose
-//                           running sum passes u_sample[row] is scanned (fp64
-//                           block scan) by its CTA for the token.
+//                           next.  Every pass also leaves the current
+//                           distribution's sum over each chunk (z_k/Z, or
+//                           S_k/S after a rejection); where the walk stops,
+//                           the chunk whose running sum passes u_sample[row]
+//                           is scanned (fp64 block scan) by its CTA for the
+//                           token -- the draw costs no barrier.
 //                           Only rows on the accepted path are read.  Partial
 //                           results cross CTAs through one workspace slot per
 //                           CTA and a per-team arrival counter; every wait on
@@ -246,7 +248,7 @@ __device__ int row_argmax(const float *__restrict__ row, int V, float *shv, int 
 
 // Per-row state of multi-step speculative sampling.
 struct RowState {
-    double m, inv_temp, temp, Z;
+    double m, inv_temp, temp, Z, inv_Z;
     int n;                         // siblings rejected so far (-1: malformed input)
     const float *q[kMaxTree];      // their SSM rows
     double S[kMaxTree];            // their residual normalisers
@@ -272,9 +274,9 @@ __device__ __forceinline__ void load4(const float *__restrict__ p, int x0, int V
     }
 }
 
-// p^(n)(x) for x in [x0, x0+4) (0 beyond V) for the bulk sums.  `table` is
-// the exp table pre-scaled by 1/Z (by 1 while Z itself is being summed); the
-// loads of each rejected sibling's row are issued together.
+// p^(n)(x) for x in [x0, x0+4) (0 beyond V) for the bulk sums (`table`
+// unscaled: p^(0) = table_exp(..) / Z); the loads of each rejected sibling's
+// row are issued together.
 template <bool VEC>
 __device__ __forceinline__ void p_bulk4(const float *__restrict__ row, int x0, int V,
                                         const RowState &st, const double *table, double (&p)[4])
@@ -283,7 +285,8 @@ __device__ __forceinline__ void p_bulk4(const float *__restrict__ row, int x0, i
     load4<VEC>(row, x0, V, l);
 #pragma unroll
     for (int k = 0; k < 4; ++k)
-        p[k] = x0 + k < V ? table_exp(((double)l[k] - st.m) * st.inv_temp, table) : 0.0;
+        p[k] = x0 + k < V ? table_exp(((double)l[k] - st.m) * st.inv_temp, table) * st.inv_Z
+                          : 0.0;
     for (int j = 0; j < st.n; ++j) {
         if (st.S[j] > 0.0) {
             float q[4];
@@ -299,15 +302,22 @@ __device__ __forceinline__ void p_bulk4(const float *__restrict__ row, int x0, i
 }
 
 // One pass over the CTA's chunk [x_lo, x_hi) of a logits row: the chunk's
-// max m_k and z_k = sum exp((l - m_k)/T).  Each thread keeps a running max
-// and rescales its sum when the max rises; `table` is scaled by 1.
+// max m_k, z_k = sum exp((l - m_k)/T) and (in *last) the largest x with a
+// finite logit, -1 if none.  Each thread keeps a running max and rescales
+// its sum when the max rises.
 template <bool VEC>
 __device__ double2 chunk_max_z(const float *__restrict__ row, int x_lo, int x_hi, int V,
-                               double inv_temp, const double *table, float *shf, double *shd)
+                               double inv_temp, const double *table, float *shf, double *shd,
+                               int *shi, int *last_out)
 {
     float mt = -INFINITY;
     double zt = 0.0;
-    auto group = [&](const float (&l)[4]) {
+    int last = -1;
+    auto group = [&](const float (&l)[4], int x0) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            if (l[k] > -INFINITY)
+                last = x0 + k;
         const float m4 = fmaxf(fmaxf(l[0], l[1]), fmaxf(l[2], l[3]));
         if (m4 > mt) {
             if (mt != -INFINITY)
@@ -332,54 +342,47 @@ __device__ double2 chunk_max_z(const float *__restrict__ row, int x_lo, int x_hi
             if (x1 + k >= x_hi)
                 l1[k] = -INFINITY;
         }
-        group(l0);
-        group(l1);
+        group(l0, x0);
+        group(l1, x1);
     }
+    *last_out = block_max_int<kWalkThreads>(last, shi);
     const float mk = block_max<kWalkThreads>(mt, shf);
     const double zs =
         mt == -INFINITY ? 0.0 : zt * table_exp(((double)mt - (double)mk) * inv_temp, table);
     return make_double2((double)mk, block_sum<kWalkThreads>(zs, shd));
 }
 
-// Over the CTA's chunk: sum max(0, p^(n)(x) - q(x)), or with q == nullptr
-// sum p^(n)(x) and (in *last) the largest x with p^(n)(x) > 0, -1 if none.
-// `table` is scaled by 1/Z.  x_lo is a multiple of 4 and x_hi is one or V,
-// so the groups of four never straddle x_hi inside the vocabulary.
+// Over the CTA's chunk: sum max(0, p^(n)(x) - q(x)) and (in *last) the
+// largest x where that is positive (-1 if none).  x_lo is a multiple of 4
+// and x_hi is one or V, so the groups of four never straddle x_hi inside the
+// vocabulary.
 template <bool VEC>
-__device__ double chunk_mass(const float *__restrict__ row, const float *__restrict__ q,
-                             int x_lo, int x_hi, int V, const RowState &st, const double *table,
-                             double *shd, int *shi, int *last_out)
+__device__ double chunk_residual(const float *__restrict__ row, const float *__restrict__ q,
+                                 int x_lo, int x_hi, int V, const RowState &st,
+                                 const double *table, double *shd, int *shi, int *last_out)
 {
     double s = 0.0;
     int last = -1;
     for (int x0 = x_lo + 4 * threadIdx.x; x0 < x_hi; x0 += 8 * kWalkThreads) {
         const int x1 = x0 + 4 * kWalkThreads;
         double p0[4], p1[4] = {0.0, 0.0, 0.0, 0.0};
+        float q0[4], q1[4];
         p_bulk4<VEC>(row, x0, V, st, table, p0);
         if (x1 < x_hi)
             p_bulk4<VEC>(row, x1, V, st, table, p1);
-        if (q) {
-            float q0[4], q1[4];
-            load4<VEC>(q, x0, V, q0);
-            load4<VEC>(q, x1 < x_hi ? x1 : V, V, q1);
+        load4<VEC>(q, x0, V, q0);
+        load4<VEC>(q, x1 < x_hi ? x1 : V, V, q1);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const double d0 = p0[k] - (double)q0[k], d1 = p1[k] - (double)q1[k];
-                s += (d0 > 0.0 ? d0 : 0.0) + (d1 > 0.0 ? d1 : 0.0);
-            }
-        } else {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                s += p0[k] + p1[k];
-                if (p0[k] > 0.0)
-                    last = max(last, x0 + k);
-                if (p1[k] > 0.0)
-                    last = max(last, x1 + k);
-            }
+        for (int k = 0; k < 4; ++k) {
+            const double d0 = p0[k] - (double)q0[k], d1 = p1[k] - (double)q1[k];
+            s += (d0 > 0.0 ? d0 : 0.0) + (d1 > 0.0 ? d1 : 0.0);
+            if (d0 > 0.0)
+                last = max(last, x0 + k);
+            if (d1 > 0.0)
+                last = max(last, x1 + k);
         }
     }
-    if (last_out)
-        *last_out = block_max_int<kWalkThreads>(last, shi);
+    *last_out = block_max_int<kWalkThreads>(last, shi);
     return block_sum<kWalkThreads>(s, shd);
 }
 
@@ -564,7 +567,7 @@ __device__ __forceinline__ unsigned long long global_ns()
 
 // Barrier over the K CTAs of one team (co-resident: cooperative launch).
 // `target` = K x the number of barriers the team has entered, this one
-// included.  Thread 0 publishes the CTA's slot write (fence, then its
+// included.  Thread 0 publishes the CTA's slot write (a release-ordered
 // arrival) and spins on the counter; after kTeamWaitNs it raises the team's
 // abort flag, which releases the other CTAs as well.  False after an abort.
 __device__ bool team_barrier(int2 *team, int target, int *sh_ok)
@@ -573,8 +576,8 @@ __device__ bool team_barrier(int2 *team, int target, int *sh_ok)
     if (threadIdx.x == 0) {
         int *arrive = &team->x;
         volatile int *abort = &team->y;
-        __threadfence();
-        atomicAdd(arrive, 1);
+        // release: this CTA's slot write is visible before its arrival
+        asm volatile("red.release.gpu.add.s32 [%0], 1;" ::"l"(arrive) : "memory");
         const unsigned long long t0 = global_ns();
         int ok = 1;
         for (;;) {
@@ -621,6 +624,11 @@ __global__ void __launch_bounds__(kWalkThreads)
     __shared__ RowState st;
     __shared__ int sh_ok, sh_dec, sh_pick, sh_token;
     __shared__ double sh_carry;
+    // the final distribution p^(n) of the current row summed over each of
+    // the team's K chunks (and each chunk's largest x with p > 0): kept up to
+    // date by every pass, so the draw needs no pass of its own
+    __shared__ double draw_sum[32];
+    __shared__ int draw_last[32];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int teams = gridDim.x / K;
     const int team = blockIdx.x / K, k = blockIdx.x % K;
@@ -631,6 +639,7 @@ __global__ void __launch_bounds__(kWalkThreads)
     int nbar = 0;
     // this CTA's slot / the team's K slots of the next barrier
     auto slots = [&]() { return ws.slot + (nbar & 1) * kWalkMaxCtas + team * K; };
+    fill_exp_table(table, 1.0);   // read only from here on (barriers below publish it)
 
     for (int b = team; b < B; b += teams) {
         int T;
@@ -658,13 +667,13 @@ __global__ void __launch_bounds__(kWalkThreads)
         for (;;) {
             const size_t ri = (size_t)b * (Tmax + 1) + row;
             const float *lrow = logits + ri * V;
-            // m and Z of this row
-            fill_exp_table(table, 1.0);
-            __syncthreads();
-            const double2 mz = chunk_max_z<VEC>(lrow, x_lo, x_hi, V, inv_temp, table, shf, shd);
+            // m and Z of this row (slot: z_k, then m_k as fp32 bits | last_k)
+            int lastk;
+            const double2 mz =
+                chunk_max_z<VEC>(lrow, x_lo, x_hi, V, inv_temp, table, shf, shd, shi, &lastk);
             double2 *sl = slots();
             if (tid == 0)
-                sl[k] = mz;
+                sl[k] = make_double2(mz.y, __hiloint2double(__float_as_int((float)mz.x), lastk));
             ++nbar;
             if (!team_barrier(tm, nbar * K, &sh_ok)) {
                 alive = false;
@@ -672,10 +681,12 @@ __global__ void __launch_bounds__(kWalkThreads)
             }
             if (warp == 0) {
                 double mk = -INFINITY, zk = 0.0;
+                int lk = -1;
                 if (lane < K) {
                     const double2 v = __ldcg(sl + lane);
-                    mk = v.x;
-                    zk = v.y;
+                    zk = v.x;
+                    mk = (double)__int_as_float(__double2hiint(v.y));
+                    lk = __double2loint(v.y);
                 }
                 double m = mk;
 #pragma unroll
@@ -684,16 +695,17 @@ __global__ void __launch_bounds__(kWalkThreads)
                 const double zs =
                     mk == -INFINITY ? 0.0 : zk * table_exp((mk - m) * inv_temp, table);
                 const double Z = warp_sum(zs);
+                draw_sum[lane] = zs / Z;
+                draw_last[lane] = lk;
                 if (lane == 0) {
                     st.m = m;
                     st.Z = Z;
+                    st.inv_Z = 1.0 / Z;
                     st.temp = temp;
                     st.inv_temp = inv_temp;
                     st.n = 0;
                 }
             }
-            __syncthreads();
-            fill_exp_table(table, 1.0 / st.Z);
             __syncthreads();
             // the children in ascending index
             int accepted = -1;
@@ -712,17 +724,28 @@ __global__ void __launch_bounds__(kWalkThreads)
                     break;
                 }
                 const double s =
-                    chunk_mass<VEC>(lrow, qc, x_lo, x_hi, V, st, table, shd, shi, nullptr);
+                    chunk_residual<VEC>(lrow, qc, x_lo, x_hi, V, st, table, shd, shi, &lastk);
                 sl = slots();
                 if (tid == 0)
-                    sl[k] = make_double2(s, 0.0);
+                    sl[k] = make_double2(s, (double)lastk);
                 ++nbar;
                 if (!team_barrier(tm, nbar * K, &sh_ok)) {
                     alive = false;
                     break;
                 }
                 if (warp == 0) {
-                    const double S = warp_sum(lane < K ? __ldcg(sl + lane).x : 0.0);
+                    double sk = 0.0;
+                    int lk = -1;
+                    if (lane < K) {
+                        const double2 v = __ldcg(sl + lane);
+                        sk = v.x;
+                        lk = (int)v.y;
+                    }
+                    const double S = warp_sum(sk);
+                    if (S > 0.0) {   // else p stays as it was
+                        draw_sum[lane] = sk * (1.0 / S);
+                        draw_last[lane] = lk;
+                    }
                     if (lane == 0) {
                         st.q[st.n] = qc;
                         st.S[st.n] = S;
@@ -744,27 +767,12 @@ __global__ void __launch_bounds__(kWalkThreads)
                 row = accepted + 1;
                 continue;
             }
-            // The walk stops here: draw the final token from p^(n).
-            int last;
-            const double s =
-                chunk_mass<VEC>(lrow, nullptr, x_lo, x_hi, V, st, table, shd, shi, &last);
-            sl = slots();
-            if (tid == 0)
-                sl[k] = make_double2(s, (double)last);
-            ++nbar;
-            if (!team_barrier(tm, nbar * K, &sh_ok)) {
-                alive = false;
-                break;
-            }
+            // The walk stops here: draw the final token from p^(n), first
+            // the chunk (from the sums the last pass left), then the token.
             const double u = u_sample[ri];
             if (warp == 0) {
-                double sk = 0.0;
-                int lk = -1;
-                if (lane < K) {
-                    const double2 v = __ldcg(sl + lane);
-                    sk = v.x;
-                    lk = (int)v.y;
-                }
+                const double sk = draw_sum[lane];
+                const int lk = draw_last[lane];
                 double incl = sk;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
