@@ -241,6 +241,44 @@ def kv_commit(k_cache, v_cache, prefix_len, out_path, n_accepted) -> Dict[str, n
     return dict(k_cache=ka, v_cache=va, new_prefix=newp, status=st)
 
 
+def gather_pages(k_pages, v_pages, block_table, page_size: int, Lmax: int):
+    """Paged K/V pools [num_pages][Hkv][page_size][D] + block table
+    [B][max_blocks] -> contiguous caches [B][Hkv][Lmax][D] (logical position
+    pos of sequence b lives in physical page block_table[b][pos // page_size]
+    at row pos % page_size).  Logical pages beyond the table are zero."""
+    kp, vp = _np(k_pages), _np(v_pages)
+    bt = _np(block_table, np.int32)
+    B, nblk = bt.shape
+    _, Hkv, ps, D = kp.shape
+    assert ps == page_size
+    k = np.zeros((B, Hkv, Lmax, D), dtype=kp.dtype)
+    v = np.zeros((B, Hkv, Lmax, D), dtype=vp.dtype)
+    for b in range(B):
+        for j in range(nblk):
+            lo = j * page_size
+            if lo >= Lmax:
+                break
+            hi = min(lo + page_size, Lmax)
+            pg = int(bt[b, j])
+            k[b, :, lo:hi] = kp[pg, :, :hi - lo]
+            v[b, :, lo:hi] = vp[pg, :, :hi - lo]
+    return k, v
+
+
+def tree_attention_paged(q, k_pages, v_pages, block_table, page_size: int, prefix_len, n_nodes,
+                         parent, scale: float) -> np.ndarray:
+    """Tree attention over a paged KV cache: the same definition as
+    tree_attention, on the cache the block table describes."""
+    qa = _np(q)
+    Tmax = qa.shape[1]
+    Lmax = int(np.asarray(_np(block_table)).shape[1]) * page_size
+    k, v = gather_pages(k_pages, v_pages, block_table, page_size, Lmax)
+    if isinstance(q, torch.Tensor) and q.dtype == torch.bfloat16:
+        k = torch.from_numpy(k.view(np.int16)).view(torch.bfloat16)
+        v = torch.from_numpy(v.view(np.int16)).view(torch.bfloat16)
+    return tree_attention(q, k, v, prefix_len, n_nodes, parent, scale)
+
+
 # Convenience wrappers over a workloads.Workload -----------------------------
 
 def workload_attention(w) -> np.ndarray:
