@@ -348,6 +348,7 @@ def main():
     if int(tsd.device_status(dev).item()) != 0:
         raise RuntimeError("device status set during the timed steps")
     commit = time_commit(step, dev, tsd)
+    paged = time_paged_attention(step, dev, tsd) if w.dtype == "bf16" else None
 
     peaks, peak_kind = _peaks()
     att_s = statistics.mean(att_ms) / 1e3
@@ -386,7 +387,7 @@ def main():
                        "parallelism": f"batch-sharded x{ws} (independent sequences)"},
             "kv_cache_gbs": kv_gbs, "kv_cache_frac_of_hbm": kv_gbs / peaks["hbm_gbs"],
             "roofline": roof, "gpu_launches": launches, "clocks": clk,
-            "kv_commit": commit}
+            "kv_commit": commit, "paged_attention": paged}
 
     if not args.no_e2e:
         line["e2e"] = e2e(w, dev, tsd, args, pg, ws)
@@ -430,6 +431,56 @@ def time_commit(step, dev, tsd, reps: int = 20):
     moved = 4 * n * w.Hkv * row   # K and V rows, read once and written once
     return {"us": us, "accepted_nodes": n, "algorithmic_bytes": moved,
             "gbs": moved / (us * 1e-6) / 1e9 if us > 0 else None}
+
+
+def time_paged_attention(step, dev, tsd, page_size: int = 128, reps: int = 10):
+    """The same attention call through a paged KV cache (pools of page_size
+    rows, physical pages in a shuffled order, a block table per sequence),
+    timed alone with CUDA events; also reports the contiguous call's time
+    measured the same way."""
+    w, d = step.w, step.d
+    B, Hkv, Lmax, D = d["k_cache"].shape
+    nblk = (Lmax + page_size - 1) // page_size
+    gen_ = torch.Generator().manual_seed(1234)
+    perm = torch.randperm(B * nblk, generator=gen_).to(dev)
+
+    def pool(cache):
+        padded = torch.zeros((B, Hkv, nblk * page_size, D), dtype=cache.dtype, device=dev)
+        padded[:, :, :Lmax] = cache
+        logical = padded.view(B, Hkv, nblk, page_size, D).permute(0, 2, 1, 3, 4)
+        out = torch.empty((B * nblk, Hkv, page_size, D), dtype=cache.dtype, device=dev)
+        out[perm] = logical.reshape(B * nblk, Hkv, page_size, D)
+        return out
+
+    kp, vp = pool(d["k_cache"]), pool(d["v_cache"])
+    table = perm.view(B, nblk).to(torch.int32)
+    out = torch.empty_like(d["q"])
+
+    def paged():
+        tsd.tree_attention_paged(d["q"], kp, vp, table, d["prefix_len"], d["n_nodes"],
+                                 step.tree.mask, out=out)
+
+    def flat():
+        tsd.tree_attention(d["q"], d["k_cache"], d["v_cache"], d["prefix_len"], d["n_nodes"],
+                           step.tree.mask, out=out, workspace=step.ws_attn)
+
+    res = {}
+    for name, fn in (("us", paged), ("contiguous_us", flat)):
+        fn()
+        torch.cuda.synchronize(dev)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(reps)]
+        for a, b in ev:
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize(dev)
+        res[name] = statistics.median(a.elapsed_time(b) * 1e3 for a, b in ev)
+    if int(tsd.device_status(dev).item()) != 0:
+        raise RuntimeError("device status set by the paged attention")
+    res["page_size"] = page_size
+    del kp, vp
+    return res
 
 
 def e2e(w, dev, tsd, args, pg, ws):

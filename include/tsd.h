@@ -70,7 +70,8 @@ enum tsd_dev_status {
     TSD_DEV_BAD_QROW = 4,     /* a q_row index outside [0, Rq)              */
     TSD_DEV_BAD_PREFIX = 8,   /* prefix_len[b] + n_nodes[b] > Lmax or < 0   */
     TSD_DEV_TIMEOUT = 16,     /* a bounded pipeline wait expired (kernel bailed out) */
-    TSD_DEV_BAD_PATH = 32     /* an accepted path that is not a valid commit list     */
+    TSD_DEV_BAD_PATH = 32,    /* an accepted path that is not a valid commit list     */
+    TSD_DEV_BAD_PAGE = 64     /* a block-table entry outside [0, num_pages)          */
 };
 
 /* Element types of Q / K / V / attention output. */
@@ -145,6 +146,33 @@ int tsd_tree_attention(const void *q, const void *k_cache, const void *v_cache,
                        int B, int Tmax, int Hq, int Hkv, int D, int Lmax, float scale,
                        int dtype, void *out, void *workspace, size_t workspace_bytes,
                        int32_t *dev_status, tsd_stream_t stream);
+
+/*
+ * Tree attention over a paged KV cache ("実運用への応用" / "vLLMとの関連" and the
+ * outlook list: the tree verification combined with PagedAttention's
+ * block-wise KV memory).  The same operation as tsd_tree_attention on the
+ * logical cache the block table describes: logical position pos of sequence
+ * b (prefix at 0..P_b-1, node u at P_b+u, as before) is row pos % page_size
+ * of physical page block_table[b][pos / page_size].
+ *   k_pages, v_pages  [num_pages][Hkv][page_size][D], dtype as for
+ *                     tsd_tree_attention (caller-owned pools)
+ *   block_table       [B][max_blocks] int32, physical page ids
+ *   page_size         a power of two in [16, 4096]; the logical capacity is
+ *                     max_blocks * page_size (the Lmax of the workspace size:
+ *                     tsd_tree_attention_workspace_size(B, Tmax, Hq, Hkv, D,
+ *                     max_blocks * page_size, dtype))
+ * Entries of the table beyond a sequence's last key are never read.  An
+ * entry outside [0, num_pages) for a key the sequence uses sets
+ * TSD_DEV_BAD_PAGE (that key reads as zero, or as page 0 on the tensor-core
+ * path).  Host errors: those of tsd_tree_attention, and TSD_ERR_SHAPE for a
+ * page size that is not a power of two in range.
+ */
+int tsd_tree_attention_paged(const void *q, const void *k_pages, const void *v_pages,
+                             const int32_t *block_table, int num_pages, int page_size,
+                             int max_blocks, const int32_t *prefix_len, const int32_t *n_nodes,
+                             const uint32_t *mask, int B, int Tmax, int Hq, int Hkv, int D,
+                             float scale, int dtype, void *out, void *workspace,
+                             size_t workspace_bytes, int32_t *dev_status, tsd_stream_t stream);
 
 /* Bytes of workspace either verify call needs: a fixed ~40 KB (per-CTA
  * partial sums and barrier counters of the stochastic walk) plus 4 bytes per

@@ -1,10 +1,11 @@
 """B200-native verification hot path of tree speculative decoding (SpecInfer).
 
-Five calls, each a thin wrapper over the C ABI of ``lib/libtsd.so``
+Five operations, each a thin wrapper over the C ABI of ``lib/libtsd.so``
 (``include/tsd.h``):
 
 * :func:`tree_mask_build`     -- ancestor bitmask / depth / child lists from ``parent[]``;
-* :func:`tree_attention`      -- topology-aware tree attention over prefix KV + ancestors;
+* :func:`tree_attention`      -- topology-aware tree attention over prefix KV + ancestors
+  (:func:`tree_attention_paged` for a paged KV cache with a block table);
 * :func:`tree_verify_greedy`  -- longest argmax-matching root path + one bonus token;
 * :func:`tree_verify_stochastic` -- multi-step speculative sampling (exact target distribution);
 * :func:`kv_commit`           -- move the accepted nodes' K/V rows after the prefix.
@@ -22,6 +23,7 @@ from .binding import (  # noqa: F401
     launch_count,
     load_library,
     tree_attention,
+    tree_attention_paged,
     tree_mask_build,
     tree_verify_greedy,
     tree_verify_stochastic,

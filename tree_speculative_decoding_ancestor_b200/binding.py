@@ -24,7 +24,7 @@ TSD_F32, TSD_BF16 = 0, 1
 TSD_MAX_TREE = 128
 TSD_TREE_INVALID = -2
 DEV_BAD_TREE, DEV_BAD_TOKEN, DEV_BAD_QROW, DEV_BAD_PREFIX, DEV_TIMEOUT = 1, 2, 4, 8, 16
-DEV_BAD_PATH = 32
+DEV_BAD_PATH, DEV_BAD_PAGE = 32, 64
 
 _lock = threading.Lock()
 _lib: Optional[ctypes.CDLL] = None
@@ -50,6 +50,8 @@ _SIGNATURES: Dict[str, Tuple[object, list]] = {
     "tsd_tree_verify_stochastic_noalloc": (_I, [_P, ctypes.c_double, _P, _I, _P, _P, _P, _P, _P,
                                                 _P, _P, _I, _I, _I, _P, _P, _P, _P, _P]),
     "tsd_kv_commit": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
+    "tsd_tree_attention_paged": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _I, _I, _I, _I,
+                                      _I, ctypes.c_float, _I, _P, _P, _SZ, _P, _P]),
 }
 
 
@@ -343,3 +345,41 @@ def kv_commit(k_cache: torch.Tensor, v_cache: torch.Tensor, prefix_len: torch.Te
                            _ptr(new_prefix_len), _ptr(st), _stream(dev))
     _check(rc, "tsd_kv_commit")
     return new_prefix_len
+
+
+def tree_attention_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,
+                         block_table: torch.Tensor, prefix_len: torch.Tensor,
+                         n_nodes: torch.Tensor, mask: torch.Tensor,
+                         scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                         workspace: Optional[torch.Tensor] = None,
+                         status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """tree_attention over a paged KV cache: pools [num_pages][Hkv][page_size][D]
+    and a block table [B][max_blocks] of physical page ids."""
+    lib = load_library()
+    dev = q.device
+    B, Tmax, Hq, D = q.shape
+    num_pages, Hkv, page_size, _ = k_pages.shape
+    max_blocks = block_table.shape[1]
+    dt = {torch.float32: TSD_F32, torch.bfloat16: TSD_BF16}.get(q.dtype)
+    if dt is None:
+        raise TypeError("q must be float32 or bfloat16")
+    _need(k_pages, "k_pages", q.dtype, (num_pages, Hkv, page_size, D), dev)
+    _need(v_pages, "v_pages", q.dtype, (num_pages, Hkv, page_size, D), dev)
+    _need(block_table, "block_table", torch.int32, (B, max_blocks), dev)
+    _need(prefix_len, "prefix_len", torch.int32, (B,), dev)
+    _need(n_nodes, "n_nodes", torch.int32, (B,), dev)
+    _need(mask, "mask", torch.int32, (B, Tmax, (Tmax + 31) // 32), dev)
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", q.dtype, (B, Tmax, Hq, D), dev)
+    Lmax = max_blocks * page_size
+    need = int(lib.tsd_tree_attention_workspace_size(B, Tmax, Hq, Hkv, D, Lmax, dt))
+    ws = _get_workspace(dev, "attention", need) if workspace is None else workspace
+    st = device_status(dev) if status is None else status
+    sc = (1.0 / D ** 0.5) if scale is None else float(scale)
+    rc = lib.tsd_tree_attention_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table),
+                                      num_pages, page_size, max_blocks, _ptr(prefix_len),
+                                      _ptr(n_nodes), _ptr(mask), B, Tmax, Hq, Hkv, D, sc, dt,
+                                      _ptr(out), _ptr(ws), ws.numel(), _ptr(st), _stream(dev))
+    _check(rc, "tsd_tree_attention_paged")
+    return out

@@ -58,7 +58,7 @@ __global__ void __launch_bounds__(kSimtThreads)
                           int Tmax, int Hq, int Hkv, int Lmax, int W, float scale_log2,
                           int keys_per_split, int nsplit, Elt *__restrict__ out,
                           float *__restrict__ part_o, float2 *__restrict__ part_ml,
-                          int32_t *dev_status)
+                          int32_t *dev_status, KvPages pages)
 {
     constexpr int DL = D / 32;
     __shared__ float sq[kSimtRows][D];
@@ -112,15 +112,19 @@ __global__ void __launch_bounds__(kSimtThreads)
             o[rr][i] = 0.f;
     }
 
-    const size_t kv_base = ((size_t)b * Hkv + hk) * (size_t)Lmax;
     for (int kt = k_begin; kt < k_end; kt += kSimtKeys) {
         __syncthreads();
         for (int i = threadIdx.x; i < kSimtKeys * D; i += kSimtThreads) {
             const int j = i / D, d = i % D, pos = kt + j;
             float kx = 0.f, vx = 0.f;
             if (pos < k_end) {
-                kx = to_float(kc[(kv_base + pos) * D + d]);
-                vx = to_float(vc[(kv_base + pos) * D + d]);
+                const long long row = kv_row(pages, b, hk, Hkv, Lmax, pos);
+                if (row >= 0) {
+                    kx = to_float(kc[row * D + d]);
+                    vx = to_float(vc[row * D + d]);
+                } else if (d == 0) {
+                    flag(dev_status, TSD_DEV_BAD_PAGE);   // that key reads as zero
+                }
             }
             sk[j][d] = kx;
             sv[j][d] = vx;
@@ -259,7 +263,7 @@ int launch_typed(const AttnArgs &a, const SimtPlan &p, void *ws, cudaStream_t st
         static_cast<const Elt *>(a.q), static_cast<const Elt *>(a.k), static_cast<const Elt *>(a.v),
         a.prefix_len, a.n_nodes, a.mask, a.Tmax, a.Hq, a.Hkv, a.Lmax, (a.Tmax + 31) / 32,
         scale_log2, p.keys_per_split, p.nsplit, static_cast<Elt *>(a.out), part_o, part_ml,
-        a.dev_status);
+        a.dev_status, a.pages);
     TSD_LAUNCH_CHECK();
     if (p.nsplit > 1) {
         const unsigned blocks = (unsigned)((nrows + 7) / 8);

@@ -40,6 +40,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "sm100_ptx.cuh"
@@ -214,10 +215,46 @@ __device__ __forceinline__ void cta_teardown(const Setup &su, int32_t *dev_statu
     }
 }
 
+// The TMA loads of one [128 keys][128] K or V tile starting at logical key
+// position pos0 into `dst` (two 64-column halves).  Contiguous cache: one box
+// per half at (x, pos0, b * Hkv + hk).  Paged cache: one box per page the
+// tile touches (box rows = min(128, page_size); a box never straddles a page
+// since both are powers of two and pos0 is a multiple of 128) at (x, row in
+// page, page * Hkv + hk).  A box that starts at or beyond the sequence's end
+// loads any valid page: those keys are masked and their V rows zeroed.
+__device__ __forceinline__ void load_kv_tile(uint32_t dst, const CUtensorMap *tm, uint32_t bar,
+                                             int pos0, int b, int hk, int Hkv,
+                                             const KvPages &pages, int seq_end,
+                                             int32_t *dev_status)
+{
+    if (!pages.table) {
+        ptx::tma_load_3d(dst, tm, 0, pos0, b * Hkv + hk, bar);
+        ptx::tma_load_3d(dst + kSub, tm, 64, pos0, b * Hkv + hk, bar);
+        return;
+    }
+    const int rows = min(BN, pages.page_size);
+    for (int r0 = 0; r0 < BN; r0 += rows) {
+        const int pos = pos0 + r0;
+        int z = hk, y = 0;
+        if (pos < seq_end) {
+            const int page = pages.table[(size_t)b * pages.max_blocks + (pos >> pages.log2_page)];
+            if (page < 0 || page >= pages.num_pages)
+                flag(dev_status, TSD_DEV_BAD_PAGE);   // page 0 stands in
+            else
+                z = page * Hkv + hk;
+            y = pos & (pages.page_size - 1);
+        }
+        ptx::tma_load_3d(dst + r0 * 128, tm, 0, y, z, bar);
+        ptx::tma_load_3d(dst + kSub + r0 * 128, tm, 64, y, z, bar);
+    }
+}
+
 // TMA producer (one lane): K_0, K_1, V_0, K_2, V_1, ... -- the order in which
 // the MMA warp first needs them.
 __device__ __forceinline__ void produce_kv(const Setup &su, const CUtensorMap *tmK,
-                                           const CUtensorMap *tmV, int z, int kb, int ntiles)
+                                           const CUtensorMap *tmV, int b, int hk, int Hkv,
+                                           int kb, int ntiles, const KvPages &pages,
+                                           int seq_end, int32_t *dev_status)
 {
     ptx::prefetch_tmap(tmK);
     ptx::prefetch_tmap(tmV);
@@ -228,10 +265,8 @@ __device__ __forceinline__ void produce_kv(const Setup &su, const CUtensorMap *t
                 !ptx::mbar_wait(su.bars.k_empty(s), ((i / NSK) - 1) & 1, su.abort_flag))
                 break;
             ptx::mbar_arrive_expect_tx(su.bars.k_full(s), kTile);
-            const uint32_t dst = su.sK + s * kTile;
-            const int pos = kb + i * BN;
-            ptx::tma_load_3d(dst, tmK, 0, pos, z, su.bars.k_full(s));
-            ptx::tma_load_3d(dst + kSub, tmK, 64, pos, z, su.bars.k_full(s));
+            load_kv_tile(su.sK + s * kTile, tmK, su.bars.k_full(s), kb + i * BN, b, hk, Hkv,
+                         pages, seq_end, dev_status);
         }
         if (i >= 1) {
             const int j = i - 1, s = j % NSV;
@@ -239,10 +274,8 @@ __device__ __forceinline__ void produce_kv(const Setup &su, const CUtensorMap *t
                 !ptx::mbar_wait(su.bars.v_empty(s), ((j / NSV) - 1) & 1, su.abort_flag))
                 break;
             ptx::mbar_arrive_expect_tx(su.bars.v_full(s), kTile);
-            const uint32_t dst = su.sV + s * kTile;
-            const int pos = kb + j * BN;
-            ptx::tma_load_3d(dst, tmV, 0, pos, z, su.bars.v_full(s));
-            ptx::tma_load_3d(dst + kSub, tmV, 64, pos, z, su.bars.v_full(s));
+            load_kv_tile(su.sV + s * kTile, tmV, su.bars.v_full(s), kb + j * BN, b, hk, Hkv,
+                         pages, seq_end, dev_status);
         }
     }
 }
@@ -500,7 +533,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
                           int Tmax, int Hq, int Hkv, int Lmax, int W, float scale_log2,
                           int keys_per_split, int nsplit, __nv_bfloat16 *__restrict__ out,
                           float *__restrict__ part_o, float2 *__restrict__ part_ml,
-                          int32_t *dev_status)
+                          int32_t *dev_status, KvPages pages)
 {
     extern __shared__ uint8_t smem_raw[];
     const int rb = blockIdx.x, pair = blockIdx.y, split = blockIdx.z;
@@ -526,7 +559,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
 
     if (warp == 0) {
         if (lane == 0)
-            produce_kv(su, &tmK, &tmV, b * Hkv + hk, kb, ntiles);
+            produce_kv(su, &tmK, &tmV, b, hk, Hkv, kb, ntiles, pages, P + T, dev_status);
     } else if (warp == 1) {
         bool ok = warp_wait(su.bars.q_full(), 0, su.abort_flag);
         ptx::tc_fence_after();
@@ -651,7 +684,8 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                               const uint32_t *__restrict__ mask, int Tmax, int Hq, int Hkv,
                               int Lmax, int W, float scale_log2, int keys_per_split, int nsplit,
                               __nv_bfloat16 *__restrict__ out, float *__restrict__ part_o,
-                              float2 *__restrict__ part_ml, int32_t *dev_status)
+                              float2 *__restrict__ part_ml, int32_t *dev_status,
+                              KvPages pages)
 {
     extern __shared__ uint8_t smem_raw[];
     const int pair = blockIdx.y, split = blockIdx.z;
@@ -676,7 +710,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
 
     if (warp == 0) {
         if (lane == 0)
-            produce_kv(su, &tmK, &tmV, b * Hkv + hk, kb, ntiles);
+            produce_kv(su, &tmK, &tmV, b, hk, Hkv, kb, ntiles, pages, P + T, dev_status);
     } else if (warp == 1) {
         bool ok = warp_wait(su.bars.q_full(), 0, su.abort_flag);
         ptx::tc_fence_after();
@@ -846,14 +880,17 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 }
 
 // [B*Hkv][Lmax][128] bf16 cache viewed as a 3-D tensor, boxes of [1][128][64].
-bool make_kv_map(CUtensorMap *m, const void *ptr, int Lmax, int BH)
+// [planes][rows][128] bf16 viewed as a 3-D tensor, boxes of [1][box_rows][64]:
+// a contiguous cache has planes = B * Hkv and rows = Lmax, a paged pool has
+// planes = num_pages * Hkv and rows = page_size.
+bool make_kv_map(CUtensorMap *m, const void *ptr, int rows, int planes, int box_rows)
 {
     auto fn = encode_fn();
     if (!fn)
         return false;
-    cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)Lmax, (cuuint64_t)BH};
-    cuuint64_t strides[2] = {(cuuint64_t)HD * 2, (cuuint64_t)Lmax * HD * 2};
-    cuuint32_t box[3] = {64, BN, 1};
+    cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)rows, (cuuint64_t)planes};
+    cuuint64_t strides[2] = {(cuuint64_t)HD * 2, (cuuint64_t)rows * HD * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims,
                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -904,8 +941,12 @@ int launch_umma_attention(const AttnArgs &a, void *ws, size_t ws_bytes, int num_
     if (ws_bytes < umma_attention_workspace(a, num_sms))
         return TSD_ERR_WORKSPACE;
     CUtensorMap tmK, tmV;
-    if (!make_kv_map(&tmK, a.k, a.Lmax, a.B * a.Hkv) ||
-        !make_kv_map(&tmV, a.v, a.Lmax, a.B * a.Hkv))
+    const bool paged = a.pages.table != nullptr;
+    const int rows = paged ? a.pages.page_size : a.Lmax;
+    const int planes = paged ? a.pages.num_pages * a.Hkv : a.B * a.Hkv;
+    const int box_rows = paged ? std::min(BN, a.pages.page_size) : BN;
+    if (!make_kv_map(&tmK, a.k, rows, planes, box_rows) ||
+        !make_kv_map(&tmV, a.v, rows, planes, box_rows))
         return TSD_ERR_CUDA;
     TSD_CUDA_TRY(set_smem_attributes());
     const size_t nrows = (size_t)a.B * a.Tmax * a.Hq;
@@ -926,12 +967,12 @@ int launch_umma_attention(const AttnArgs &a, void *ws, size_t ws_bytes, int num_
         tree_attn_keysplit_kernel<<<grid, kSplitThreads, kSmemBytes, stream>>>(
             tmK, tmV, static_cast<const __nv_bfloat16 *>(a.q), a.prefix_len, a.n_nodes, a.mask,
             a.Tmax, a.Hq, a.Hkv, a.Lmax, W, sl2, p.keys_per_split, p.nsplit,
-            static_cast<__nv_bfloat16 *>(a.out), part_o, part_ml, a.dev_status);
+            static_cast<__nv_bfloat16 *>(a.out), part_o, part_ml, a.dev_status, a.pages);
     else
         tree_attn_rows_kernel<<<grid, kRowsThreads, kSmemBytes, stream>>>(
             tmK, tmV, static_cast<const __nv_bfloat16 *>(a.q), a.prefix_len, a.n_nodes, a.mask,
             a.Tmax, a.Hq, a.Hkv, a.Lmax, W, sl2, p.keys_per_split, p.nsplit,
-            static_cast<__nv_bfloat16 *>(a.out), part_o, part_ml, a.dev_status);
+            static_cast<__nv_bfloat16 *>(a.out), part_o, part_ml, a.dev_status, a.pages);
     TSD_LAUNCH_CHECK();
     if (p.nsplit > 1) {
         const int rc = launch_combine(a.dtype, a.D, part_o, part_ml, p.nsplit, a.prefix_len,

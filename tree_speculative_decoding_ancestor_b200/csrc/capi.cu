@@ -131,6 +131,45 @@ int tsd_tree_attention(const void *q, const void *k_cache, const void *v_cache,
     return tsd::launch_simt_attention(a, workspace, workspace_bytes, sms, s);
 }
 
+int tsd_tree_attention_paged(const void *q, const void *k_pages, const void *v_pages,
+                             const int32_t *block_table, int num_pages, int page_size,
+                             int max_blocks, const int32_t *prefix_len, const int32_t *n_nodes,
+                             const uint32_t *mask, int B, int Tmax, int Hq, int Hkv, int D,
+                             float scale, int dtype, void *out, void *workspace,
+                             size_t workspace_bytes, int32_t *dev_status, tsd_stream_t stream)
+{
+    if (page_size < 16 || page_size > 4096 || (page_size & (page_size - 1)) != 0 ||
+        max_blocks < 1 || num_pages < 1 || (long long)max_blocks * page_size > (1LL << 30))
+        return TSD_ERR_SHAPE;
+    tsd::AttnArgs a;
+    a.q = q; a.k = k_pages; a.v = v_pages; a.prefix_len = prefix_len; a.n_nodes = n_nodes;
+    a.mask = mask; a.B = B; a.Tmax = Tmax; a.Hq = Hq; a.Hkv = Hkv; a.D = D;
+    a.Lmax = max_blocks * page_size;
+    a.dtype = dtype; a.scale = scale; a.out = out; a.dev_status = dev_status;
+    a.pages.table = block_table;
+    a.pages.max_blocks = max_blocks;
+    a.pages.page_size = page_size;
+    a.pages.log2_page = __builtin_ctz((unsigned)page_size);
+    a.pages.num_pages = num_pages;
+    if (B == 0)
+        return TSD_OK;
+    if (!block_table)
+        return TSD_ERR_NULL;
+    const int rc = check_attn(a);
+    if (rc != TSD_OK)
+        return rc;
+    const int sms = device_sms();
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (choose_umma(a)) {
+        if (workspace_bytes < tsd::umma_attention_workspace(a, sms))
+            return TSD_ERR_WORKSPACE;
+        return tsd::launch_umma_attention(a, workspace, workspace_bytes, sms, s);
+    }
+    if (workspace_bytes < tsd::simt_attention_workspace(a, sms))
+        return TSD_ERR_WORKSPACE;
+    return tsd::launch_simt_attention(a, workspace, workspace_bytes, sms, s);
+}
+
 size_t tsd_tree_verify_workspace_size(int B, int Tmax, int V)
 {
     if (B <= 0 || Tmax < 1 || Tmax > TSD_MAX_TREE || V < 1)

@@ -82,14 +82,37 @@ int launch_tree_mask(const int32_t *parent, const int32_t *n_nodes, int B, int T
                      uint32_t *mask, int32_t *depth, int32_t *first_child, int32_t *next_sibling,
                      int32_t *dev_status, cudaStream_t stream);
 
+// Where K/V row `pos` of (sequence b, KV head hk) lives.  table == nullptr:
+// a contiguous cache [B][Hkv][Lmax][D].  Otherwise a paged pool
+// [num_pages][Hkv][page_size][D]: logical page pos / page_size of sequence b
+// is physical page table[b][pos / page_size] (page_size a power of two).
+struct KvPages {
+    const int32_t *table = nullptr;
+    int max_blocks = 0, page_size = 0, log2_page = 0, num_pages = 0;
+};
+
+// Row index (in rows of D elements) of K/V position `pos`; a page id outside
+// [0, num_pages) yields -1.
+__device__ __forceinline__ long long kv_row(const KvPages &pg, int b, int hk, int Hkv, int Lmax,
+                                            int pos)
+{
+    if (!pg.table)
+        return ((long long)b * Hkv + hk) * Lmax + pos;
+    const int page = pg.table[(size_t)b * pg.max_blocks + (pos >> pg.log2_page)];
+    if (page < 0 || page >= pg.num_pages)
+        return -1;
+    return ((long long)page * Hkv + hk) * pg.page_size + (pos & (pg.page_size - 1));
+}
+
 struct AttnArgs {
     const void *q, *k, *v;
     const int32_t *prefix_len, *n_nodes;
     const uint32_t *mask;
-    int B, Tmax, Hq, Hkv, D, Lmax, dtype;
+    int B, Tmax, Hq, Hkv, D, Lmax, dtype;   // Lmax: logical capacity (max_blocks * page_size if paged)
     float scale;
     void *out;
     int32_t *dev_status;
+    KvPages pages;
 };
 size_t simt_attention_workspace(const AttnArgs &a, int num_sms);
 int launch_simt_attention(const AttnArgs &a, void *ws, size_t ws_bytes, int num_sms,
