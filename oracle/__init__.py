@@ -279,6 +279,62 @@ def tree_attention_paged(q, k_pages, v_pages, block_table, page_size: int, prefi
     return tree_attention(q, k, v, prefix_len, n_nodes, parent, scale)
 
 
+def tree_expand(q_probs, frow, k: int, parent, tokens, q_row, n_nodes, lvl_begin):
+    """One expansion level (on copies of the tree arrays): every frontier node
+    gets the k best tokens of its q row as children.  Returns the new arrays
+    and status."""
+    lib = _load()
+    qp = _np(q_probs, np.float32)
+    B, Rq, V = qp.shape
+    par = _np(parent, np.int32).copy()
+    tok = _np(tokens, np.int32).copy()
+    qr = _np(q_row, np.int32).copy()
+    nn = _np(n_nodes, np.int32).copy()
+    lb = _np(lvl_begin, np.int32).copy()
+    fr = _np(frow, np.int32)
+    Tmax = par.shape[1]
+    st = np.zeros(B, dtype=np.int32)
+    lib.oracle_tree_expand(_p(qp), Rq, V, _p(fr), int(k), _p(par), _p(tok), _p(qr), _p(nn),
+                           _p(lb), B, Tmax, _p(st))
+    return dict(parent=par, tokens=tok, q_row=qr, n_nodes=nn, lvl_begin=lb, status=st)
+
+
+def tree_dfs_order(parent, tokens, q_row, n_nodes) -> Dict[str, np.ndarray]:
+    """Depth-first pre-order renumbering (children in increasing index)."""
+    lib = _load()
+    par = _np(parent, np.int32)
+    tok = _np(tokens, np.int32)
+    qr = _np(q_row, np.int32)
+    nn = _np(n_nodes, np.int32)
+    B, Tmax = par.shape
+    perm = np.full((B, Tmax), SENTINEL, dtype=np.int32)
+    op = np.full((B, Tmax), SENTINEL, dtype=np.int32)
+    ot = np.full((B, Tmax), SENTINEL, dtype=np.int32)
+    oq = np.full((B, Tmax), SENTINEL, dtype=np.int32)
+    st = np.zeros(B, dtype=np.int32)
+    lib.oracle_tree_dfs_order(_p(par), _p(tok), _p(qr), _p(nn), B, Tmax, _p(perm), _p(op),
+                              _p(ot), _p(oq), _p(st))
+    return dict(perm=perm, parent=op, tokens=ot, q_row=oq, status=st)
+
+
+def tree_merge_chains(chain_tokens, chain_q_row, chain_len, Tmax: int) -> Dict[str, np.ndarray]:
+    """Merge M chains per sequence ([B][M][L] tokens and q rows, [B][M]
+    lengths) into one token tree in depth-first pre-order."""
+    lib = _load()
+    ct = _np(chain_tokens, np.int32)
+    cq = _np(chain_q_row, np.int32)
+    cl = _np(chain_len, np.int32)
+    B, M, L = ct.shape
+    par = np.full((B, Tmax), SENTINEL, dtype=np.int32)
+    tok = np.full((B, Tmax), SENTINEL, dtype=np.int32)
+    qr = np.full((B, Tmax), SENTINEL, dtype=np.int32)
+    nn = np.zeros(B, dtype=np.int32)
+    st = np.zeros(B, dtype=np.int32)
+    lib.oracle_tree_merge_chains(_p(ct), _p(cq), _p(cl), M, L, B, Tmax, _p(par), _p(tok),
+                                 _p(qr), _p(nn), _p(st))
+    return dict(parent=par, tokens=tok, q_row=qr, n_nodes=nn, status=st)
+
+
 # Convenience wrappers over a workloads.Workload -----------------------------
 
 def workload_attention(w) -> np.ndarray:

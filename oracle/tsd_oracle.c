@@ -514,3 +514,177 @@ int oracle_kv_commit(unsigned char *k, unsigned char *v, const int32_t *prefix_l
     free(tmp);
     return any;
 }
+
+/* ---------------------------------------------------------------- tree construction
+ * Section "マルチドラフトモデルアプローチ" of the SpecInfer explainer: an
+ * expansion-based tree <k_1, ..., k_n> takes the top-k_i tokens of one SSM at
+ * every node of depth i-1 (item 1); a merge-based tree merges the outputs of
+ * several SSMs into one token tree (item 2); "Tree Attention のカーネル融合",
+ * item 2: the tree is laid out in depth-first order. */
+
+/* (v, i) comes before (w, j) in "descending probability, lower token first". */
+static int before(float v, int i, float w, int j) { return v > w || (v == w && i < j); }
+
+/* One expansion level.  The frontier is the root (lvl_begin[b] == n_nodes[b]
+ * == 0 only for an empty tree) or the nodes lvl_begin[b] .. n_nodes[b]-1;
+ * frontier node i (in index order) has its SSM distribution in q row
+ * frow[b][i].  Each frontier node gets k children, appended in frontier order,
+ * holding the k best tokens of its row in descending probability (lower
+ * token id on ties), with q_row = frow[b][i].  lvl_begin[b] becomes the old
+ * n_nodes[b].  More than Tmax nodes, a bad q row or k > V: status 1, nothing
+ * changes. */
+int oracle_tree_expand(const float *q_probs, int Rq, int V, const int32_t *frow, int k,
+                       int32_t *parent, int32_t *tokens, int32_t *q_row, int32_t *n_nodes,
+                       int32_t *lvl_begin, int B, int Tmax, int32_t *status)
+{
+    int any = 0;
+    for (int b = 0; b < B; ++b) {
+        const int n = n_nodes[b];
+        const int root_level = (n == 0);
+        const int F = root_level ? 1 : n - lvl_begin[b];
+        const int32_t *fr = frow + (size_t)b * Tmax;
+        int ok = k >= 1 && k <= V && F >= 1 && lvl_begin[b] >= 0 && n + F * k <= Tmax;
+        for (int i = 0; ok && i < F; ++i)
+            ok = fr[i] >= 0 && fr[i] < Rq;
+        status[b] = ok ? 0 : 1;
+        if (!ok) {
+            any |= 1;
+            continue;
+        }
+        for (int i = 0; i < F; ++i) {
+            const float *p = q_probs + ((size_t)b * Rq + fr[i]) * V;
+            float pv = 0.f;
+            int pi = -1;   /* the previous pick; the next is the best after it */
+            for (int j = 0; j < k; ++j) {
+                int best = -1;
+                for (int x = 0; x < V; ++x) {
+                    if (pi >= 0 && !before(pv, pi, p[x], x))
+                        continue;
+                    if (best < 0 || before(p[x], x, p[best], best))
+                        best = x;
+                }
+                const int u = n + i * k + j;
+                parent[(size_t)b * Tmax + u] = root_level ? -1 : lvl_begin[b] + i;
+                tokens[(size_t)b * Tmax + u] = best;
+                q_row[(size_t)b * Tmax + u] = fr[i];
+                pv = p[best];
+                pi = best;
+            }
+        }
+        lvl_begin[b] = n;
+        n_nodes[b] = n + F * k;
+    }
+    return any;
+}
+
+/* Depth-first pre-order of a tree given in any topological order (children
+ * visited in increasing index): perm[new] = old, and parent/tokens/q_row
+ * renumbered (out_*).  status 1 for a tree that is not topological. */
+int oracle_tree_dfs_order(const int32_t *parent, const int32_t *tokens, const int32_t *q_row,
+                          const int32_t *n_nodes, int B, int Tmax, int32_t *perm,
+                          int32_t *out_parent, int32_t *out_tokens, int32_t *out_q_row,
+                          int32_t *status)
+{
+    int any = 0;
+    int32_t *stack = (int32_t *)malloc(sizeof(int32_t) * (Tmax + 1));
+    int32_t *inv = (int32_t *)malloc(sizeof(int32_t) * (Tmax + 1));
+    for (int b = 0; b < B; ++b) {
+        const int T = n_nodes[b];
+        const int32_t *par = parent + (size_t)b * Tmax;
+        status[b] = (T < 0 || T > Tmax || !tree_is_valid(par, T)) ? 1 : 0;
+        if (status[b]) {
+            any |= 1;
+            continue;
+        }
+        int top = 0, cnt = 0;
+        /* push the root's children in decreasing index so the smallest pops first */
+        for (int v = T - 1; v >= 0; --v)
+            if (par[v] == -1)
+                stack[top++] = v;
+        while (top > 0) {
+            const int u = stack[--top];
+            perm[(size_t)b * Tmax + cnt] = u;
+            inv[u] = cnt++;
+            for (int v = T - 1; v > u; --v)
+                if (par[v] == u)
+                    stack[top++] = v;
+        }
+        for (int i = 0; i < T; ++i) {
+            const int u = perm[(size_t)b * Tmax + i];
+            out_parent[(size_t)b * Tmax + i] = par[u] < 0 ? -1 : inv[par[u]];
+            out_tokens[(size_t)b * Tmax + i] = tokens[(size_t)b * Tmax + u];
+            out_q_row[(size_t)b * Tmax + i] = q_row[(size_t)b * Tmax + u];
+        }
+    }
+    free(stack);
+    free(inv);
+    return any;
+}
+
+/* Merge M chains per sequence into one token tree: chain m proposes tokens
+ * ctok[b][m][0..clen[b][m]-1], step i drawn from q row cq[b][m][i].  A chain
+ * reuses the node of an earlier chain while its prefix matches (same parent,
+ * same token) and creates new nodes from the first difference on; a node
+ * keeps the q row of the chain that created it.  Output in depth-first
+ * pre-order, children in creation order.  More than Tmax nodes or a bad
+ * length: status 1, n_nodes = -1. */
+int oracle_tree_merge_chains(const int32_t *ctok, const int32_t *cq, const int32_t *clen, int M,
+                             int L, int B, int Tmax, int32_t *parent, int32_t *tokens,
+                             int32_t *q_row, int32_t *n_nodes, int32_t *status)
+{
+    int any = 0;
+    int32_t *tp = (int32_t *)malloc(sizeof(int32_t) * (Tmax + 1));
+    int32_t *tt = (int32_t *)malloc(sizeof(int32_t) * (Tmax + 1));
+    int32_t *tq = (int32_t *)malloc(sizeof(int32_t) * (Tmax + 1));
+    int32_t *perm = (int32_t *)malloc(sizeof(int32_t) * (Tmax + 1));
+    int32_t *op = (int32_t *)malloc(sizeof(int32_t) * (Tmax + 1));
+    int32_t *ot = (int32_t *)malloc(sizeof(int32_t) * (Tmax + 1));
+    int32_t *oq = (int32_t *)malloc(sizeof(int32_t) * (Tmax + 1));
+    for (int b = 0; b < B; ++b) {
+        int T = 0, ok = 1;
+        for (int m = 0; ok && m < M; ++m) {
+            const int len = clen[(size_t)b * M + m];
+            if (len < 0 || len > L) {
+                ok = 0;
+                break;
+            }
+            int cur = -1;
+            for (int i = 0; i < len; ++i) {
+                const int t = ctok[((size_t)b * M + m) * L + i];
+                int found = -1;
+                for (int v = 0; v < T; ++v)
+                    if (tp[v] == cur && tt[v] == t) {
+                        found = v;
+                        break;
+                    }
+                if (found < 0) {
+                    if (T == Tmax) {
+                        ok = 0;
+                        break;
+                    }
+                    tp[T] = cur;
+                    tt[T] = t;
+                    tq[T] = cq[((size_t)b * M + m) * L + i];
+                    found = T++;
+                }
+                cur = found;
+            }
+        }
+        status[b] = ok ? 0 : 1;
+        if (!ok) {
+            any |= 1;
+            n_nodes[b] = -1;
+            continue;
+        }
+        int32_t st;
+        oracle_tree_dfs_order(tp, tt, tq, &T, 1, Tmax > 0 ? Tmax : 1, perm, op, ot, oq, &st);
+        for (int u = 0; u < T; ++u) {
+            parent[(size_t)b * Tmax + u] = op[u];
+            tokens[(size_t)b * Tmax + u] = ot[u];
+            q_row[(size_t)b * Tmax + u] = oq[u];
+        }
+        n_nodes[b] = T;
+    }
+    free(tp); free(tt); free(tq); free(perm); free(op); free(ot); free(oq);
+    return any;
+}

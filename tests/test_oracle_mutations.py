@@ -15,6 +15,7 @@ import test_oracle_commit as pc
 import test_oracle_greedy as pg
 import test_oracle_mask as pm
 import test_oracle_stochastic as ps
+import test_oracle_tree_build as pt
 
 MUTATIONS = {
     # attention (SpecInfer explainer, "トークンツリー構造の仕組み")
@@ -58,6 +59,13 @@ MUTATIONS = {
     # commit of the accepted path
     "commit_ignores_prefix": ("base + (size_t)(P + path[i]) * row_bytes", "base + (size_t)(path[i]) * row_bytes",
                               lambda: pc.test_commit_then_decode_equals_tree_attention(1, "bf16")),
+    # tree construction
+    "topk_ties_to_higher_id": ("return v > w || (v == w && i < j);", "return v > w || (v == w && i > j);",
+                               pt.test_topk_ties_take_the_lower_token_id),
+    "merge_never_shares": ("if (tp[v] == cur && tt[v] == t) {", "if (0) {",
+                           pt.test_merge_rebuilds_the_page_figure),
+    "dfs_children_reversed": ("for (int v = T - 1; v > u; --v)", "for (int v = u + 1; v < T; ++v)",
+                              lambda: pt.test_dfs_order_is_the_recursive_preorder(0)),
     "commit_reverses_order": ("memcpy(base + (size_t)(P + i) * row_bytes", "memcpy(base + (size_t)(P + n - 1 - i) * row_bytes",
                               lambda: pc.test_committed_rows_follow_the_verified_tokens_in_order("greedy")),
 }
