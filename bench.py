@@ -349,6 +349,7 @@ def main():
         raise RuntimeError("device status set during the timed steps")
     commit = time_commit(step, dev, tsd)
     paged = time_paged_attention(step, dev, tsd) if w.dtype == "bf16" else None
+    build = time_tree_build(w, dev, tsd)
 
     peaks, peak_kind = _peaks()
     att_s = statistics.mean(att_ms) / 1e3
@@ -387,7 +388,7 @@ def main():
                        "parallelism": f"batch-sharded x{ws} (independent sequences)"},
             "kv_cache_gbs": kv_gbs, "kv_cache_frac_of_hbm": kv_gbs / peaks["hbm_gbs"],
             "roofline": roof, "gpu_launches": launches, "clocks": clk,
-            "kv_commit": commit, "paged_attention": paged}
+            "kv_commit": commit, "paged_attention": paged, "tree_build": build}
 
     if not args.no_e2e:
         line["e2e"] = e2e(w, dev, tsd, args, pg, ws)
@@ -431,6 +432,67 @@ def time_commit(step, dev, tsd, reps: int = 20):
     moved = 4 * n * w.Hkv * row   # K and V rows, read once and written once
     return {"us": us, "accepted_nodes": n, "algorithmic_bytes": moved,
             "gbs": moved / (us * 1e-6) / 1e9 if us > 0 else None}
+
+
+def time_tree_build(w, dev, tsd, reps: int = 10):
+    """Token-tree construction on the GPU for the workload's batch and
+    vocabulary: an expansion <4, 2, 2, ...> level by level (as many levels as
+    the tree slots hold; the top-k of a random SSM row per frontier node),
+    then the depth-first renumbering; the launches are captured in a CUDA
+    graph and its replay is timed."""
+    B, V = w.B, w.V
+    ks, n, F = [4], 4, 4
+    while n + 2 * F <= w.Tmax:
+        ks.append(2)
+        n, F = n + 2 * F, 2 * F
+    n, F, frows = 0, 1, []
+    for k in ks:
+        lb = n
+        fr = torch.zeros((B, w.Tmax), dtype=torch.int32)
+        if n > 0:
+            fr[:, :F] = torch.arange(lb, n, dtype=torch.int32) + 1   # node u's row is u + 1
+        frows.append(fr.to(dev))
+        n, F = n + F * k, F * k
+        if n > w.Tmax:
+            return None
+    q = torch.rand((B, n + 1, V), device=dev, generator=None)
+    z = lambda: torch.zeros((B, w.Tmax), dtype=torch.int32, device=dev)  # noqa: E731
+    tree = tsd.Tree(z(), z(), z(), torch.zeros(B, dtype=torch.int32, device=dev))
+    lvl = torch.zeros(B, dtype=torch.int32, device=dev)
+    perm = z()
+    out = tsd.Tree(z(), z(), z(), tree.n_nodes)
+    lib = tsd.load_library()
+    st = tsd.device_status(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def run():
+        tree.n_nodes.zero_()
+        lvl.zero_()
+        for k, fr in zip(ks, frows):
+            tsd.tree_expand(q, fr, k, tree, lvl)
+        lib.tsd_tree_dfs_order(tree.parent.data_ptr(), tree.tokens.data_ptr(),
+                               tree.q_row.data_ptr(), tree.n_nodes.data_ptr(), B, w.Tmax,
+                               perm.data_ptr(), out.parent.data_ptr(), out.tokens.data_ptr(),
+                               out.q_row.data_ptr(), st.data_ptr(), stream.cuda_stream)
+
+    run()
+    torch.cuda.synchronize(dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(reps):
+            run()
+    graph.replay()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    graph.replay()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    del graph
+    if int(st.item()) != 0 or int(tree.n_nodes[0].item()) != n:
+        raise RuntimeError("tree construction failed in the benchmark")
+    return {"expansion": list(ks), "nodes_per_sequence": n, "sequences": B, "vocab": V,
+            "us": e0.elapsed_time(e1) * 1e3 / reps}
 
 
 def time_paged_attention(step, dev, tsd, page_size: int = 128, reps: int = 10):

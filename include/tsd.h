@@ -239,6 +239,59 @@ int tsd_tree_verify_stochastic(const float *logits, double temperature, const fl
                                tsd_stream_t stream);
 
 /*
+ * Token-tree construction ("マルチドラフトモデルアプローチ": item 1,
+ * expansion-based trees <k_1, ..., k_n> take one SSM's top-k_i tokens at
+ * every node of depth i-1; item 2, merge-based trees merge the outputs of
+ * several SSMs into one token tree; "Tree Attention のカーネル融合", item 2: the
+ * tree is laid out depth-first).  Tree arrays are those of the other calls:
+ * parent, tokens, q_row [B][Tmax] int32, n_nodes [B] int32.
+ *
+ * tsd_tree_expand adds one level.  The frontier is the root when
+ * n_nodes[b] == 0, else the nodes lvl_begin[b] .. n_nodes[b]-1 (the level
+ * added last); frontier node i (in index order) has its SSM distribution in
+ * q_probs[b][frow[b][i]] (q_probs [B][Rq][V] fp32, frow [B][Tmax] int32).
+ * Each frontier node gets k children, appended in frontier order at
+ * n_nodes + i*k + j, holding the k most probable tokens of its row in
+ * descending probability (lower token id on ties), with q_row = frow[b][i];
+ * then lvl_begin[b] = old n_nodes[b] and n_nodes[b] += F*k.  A level that
+ * would exceed Tmax, a q row outside [0, Rq) or k > V changes nothing and
+ * sets TSD_DEV_BAD_TREE.  Nodes come out level by level; renumber with
+ * tsd_tree_dfs_order before the other calls if depth-first order is wanted.
+ */
+int tsd_tree_expand(const float *q_probs, int Rq, int V, const int32_t *frow, int k,
+                    int32_t *parent, int32_t *tokens, int32_t *q_row, int32_t *n_nodes,
+                    int32_t *lvl_begin, int B, int Tmax, int32_t *dev_status,
+                    tsd_stream_t stream);
+
+/*
+ * tsd_tree_dfs_order renumbers each tree (any order in which parents precede
+ * children) into depth-first pre-order, children in increasing old index:
+ * perm[b][new] = old, out_parent / out_tokens / out_q_row renumbered
+ * (entries beyond n_nodes untouched).  A malformed tree sets
+ * TSD_DEV_BAD_TREE and writes nothing for that sequence.
+ */
+int tsd_tree_dfs_order(const int32_t *parent, const int32_t *tokens, const int32_t *q_row,
+                       const int32_t *n_nodes, int B, int Tmax, int32_t *perm,
+                       int32_t *out_parent, int32_t *out_tokens, int32_t *out_q_row,
+                       int32_t *dev_status, tsd_stream_t stream);
+
+/*
+ * tsd_tree_merge_chains builds the tree from M chains per sequence: chain m
+ * proposes chain_tokens[b][m][0 .. chain_len[b][m]-1], step i drawn from q row
+ * chain_q_row[b][m][i] ([B][M][L] int32, lengths [B][M]).  A chain reuses
+ * earlier nodes while its prefix matches (same parent, same token) and
+ * creates nodes from its first difference on; a node keeps the q row of the
+ * chain that created it.  Output in depth-first pre-order, children in
+ * creation order; n_nodes[b] = the node count, or -1 (with
+ * TSD_DEV_BAD_TREE) when the tree would exceed Tmax or a length is outside
+ * [0, L].
+ */
+int tsd_tree_merge_chains(const int32_t *chain_tokens, const int32_t *chain_q_row,
+                          const int32_t *chain_len, int M, int L, int B, int Tmax,
+                          int32_t *parent, int32_t *tokens, int32_t *q_row, int32_t *n_nodes,
+                          int32_t *dev_status, tsd_stream_t stream);
+
+/*
  * Commit of the accepted path ("Tree Attention のカーネル融合", item 2: the
  * tree's KV entries stay consistent with the existing KV cache; the
  * flatkey.ai guide's verification diagram: the accepted prefix is committed).

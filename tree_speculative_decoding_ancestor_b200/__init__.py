@@ -1,6 +1,6 @@
 """B200-native verification hot path of tree speculative decoding (SpecInfer).
 
-Five operations, each a thin wrapper over the C ABI of ``lib/libtsd.so``
+Six operations, each a thin wrapper over the C ABI of ``lib/libtsd.so``
 (``include/tsd.h``):
 
 * :func:`tree_mask_build`     -- ancestor bitmask / depth / child lists from ``parent[]``;
@@ -8,12 +8,15 @@ Five operations, each a thin wrapper over the C ABI of ``lib/libtsd.so``
   (:func:`tree_attention_paged` for a paged KV cache with a block table);
 * :func:`tree_verify_greedy`  -- longest argmax-matching root path + one bonus token;
 * :func:`tree_verify_stochastic` -- multi-step speculative sampling (exact target distribution);
-* :func:`kv_commit`           -- move the accepted nodes' K/V rows after the prefix.
+* :func:`kv_commit`           -- move the accepted nodes' K/V rows after the prefix;
+* :func:`tree_expand`, :func:`tree_merge_chains`, :func:`tree_dfs_order` -- build the
+  token tree (expansion top-k levels, merge of several SSMs' chains, depth-first order).
 """
 
 from .binding import (  # noqa: F401
     LIB_PATH,
     TsdError,
+    Tree,
     TreeMask,
     VerifyResult,
     attention_workspace_size,
@@ -24,7 +27,10 @@ from .binding import (  # noqa: F401
     load_library,
     tree_attention,
     tree_attention_paged,
+    tree_dfs_order,
+    tree_expand,
     tree_mask_build,
+    tree_merge_chains,
     tree_verify_greedy,
     tree_verify_stochastic,
     tree_verify_stochastic_noalloc,

@@ -52,6 +52,9 @@ _SIGNATURES: Dict[str, Tuple[object, list]] = {
     "tsd_kv_commit": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
     "tsd_tree_attention_paged": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _I, _I, _I, _I,
                                       _I, ctypes.c_float, _I, _P, _P, _SZ, _P, _P]),
+    "tsd_tree_expand": (_I, [_P, _I, _I, _P, _I, _P, _P, _P, _P, _P, _I, _I, _P, _P]),
+    "tsd_tree_dfs_order": (_I, [_P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "tsd_tree_merge_chains": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
 }
 
 
@@ -382,4 +385,74 @@ def tree_attention_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.
                                       _ptr(n_nodes), _ptr(mask), B, Tmax, Hq, Hkv, D, sc, dt,
                                       _ptr(out), _ptr(ws), ws.numel(), _ptr(st), _stream(dev))
     _check(rc, "tsd_tree_attention_paged")
+    return out
+
+
+class Tree(NamedTuple):
+    parent: torch.Tensor     # [B][Tmax] int32
+    tokens: torch.Tensor     # [B][Tmax] int32
+    q_row: torch.Tensor      # [B][Tmax] int32
+    n_nodes: torch.Tensor    # [B] int32
+
+
+def tree_expand(q_probs: torch.Tensor, frow: torch.Tensor, k: int, tree: Tree,
+                lvl_begin: torch.Tensor, status: Optional[torch.Tensor] = None) -> Tree:
+    """Add one expansion level in place (the k most probable tokens of each
+    frontier node's SSM row become its children)."""
+    lib = load_library()
+    dev = q_probs.device
+    B, Rq, V = q_probs.shape
+    Tmax = tree.parent.shape[1]
+    _need(q_probs, "q_probs", torch.float32, (B, Rq, V), dev)
+    _need(frow, "frow", torch.int32, (B, Tmax), dev)
+    for name in ("parent", "tokens", "q_row"):
+        _need(getattr(tree, name), name, torch.int32, (B, Tmax), dev)
+    _need(tree.n_nodes, "n_nodes", torch.int32, (B,), dev)
+    _need(lvl_begin, "lvl_begin", torch.int32, (B,), dev)
+    st = device_status(dev) if status is None else status
+    rc = lib.tsd_tree_expand(_ptr(q_probs), Rq, V, _ptr(frow), int(k), _ptr(tree.parent),
+                             _ptr(tree.tokens), _ptr(tree.q_row), _ptr(tree.n_nodes),
+                             _ptr(lvl_begin), B, Tmax, _ptr(st), _stream(dev))
+    _check(rc, "tsd_tree_expand")
+    return tree
+
+
+def tree_dfs_order(tree: Tree, status: Optional[torch.Tensor] = None):
+    """Depth-first renumbering: returns (perm [B][Tmax], renumbered Tree)."""
+    lib = load_library()
+    dev = tree.parent.device
+    B, Tmax = tree.parent.shape
+    for name in ("parent", "tokens", "q_row"):
+        _need(getattr(tree, name), name, torch.int32, (B, Tmax), dev)
+    _need(tree.n_nodes, "n_nodes", torch.int32, (B,), dev)
+    perm = torch.full((B, Tmax), -1, dtype=torch.int32, device=dev)
+    out = Tree(torch.full_like(tree.parent, -1), torch.zeros_like(tree.tokens),
+               torch.zeros_like(tree.q_row), tree.n_nodes.clone())
+    st = device_status(dev) if status is None else status
+    rc = lib.tsd_tree_dfs_order(_ptr(tree.parent), _ptr(tree.tokens), _ptr(tree.q_row),
+                                _ptr(tree.n_nodes), B, Tmax, _ptr(perm), _ptr(out.parent),
+                                _ptr(out.tokens), _ptr(out.q_row), _ptr(st), _stream(dev))
+    _check(rc, "tsd_tree_dfs_order")
+    return perm, out
+
+
+def tree_merge_chains(chain_tokens: torch.Tensor, chain_q_row: torch.Tensor,
+                      chain_len: torch.Tensor, Tmax: int,
+                      status: Optional[torch.Tensor] = None) -> Tree:
+    """Merge M draft chains per sequence into one token tree (depth-first)."""
+    lib = load_library()
+    dev = chain_tokens.device
+    B, M, L = chain_tokens.shape
+    _need(chain_tokens, "chain_tokens", torch.int32, (B, M, L), dev)
+    _need(chain_q_row, "chain_q_row", torch.int32, (B, M, L), dev)
+    _need(chain_len, "chain_len", torch.int32, (B, M), dev)
+    out = Tree(torch.full((B, Tmax), -1, dtype=torch.int32, device=dev),
+               torch.zeros((B, Tmax), dtype=torch.int32, device=dev),
+               torch.zeros((B, Tmax), dtype=torch.int32, device=dev),
+               torch.zeros((B,), dtype=torch.int32, device=dev))
+    st = device_status(dev) if status is None else status
+    rc = lib.tsd_tree_merge_chains(_ptr(chain_tokens), _ptr(chain_q_row), _ptr(chain_len), M, L,
+                                   B, Tmax, _ptr(out.parent), _ptr(out.tokens), _ptr(out.q_row),
+                                   _ptr(out.n_nodes), _ptr(st), _stream(dev))
+    _check(rc, "tsd_tree_merge_chains")
     return out

@@ -249,4 +249,53 @@ int tsd_kv_commit(void *k_cache, void *v_cache, const int32_t *prefix_len,
                                  reinterpret_cast<cudaStream_t>(stream));
 }
 
+int tsd_tree_expand(const float *q_probs, int Rq, int V, const int32_t *frow, int k,
+                    int32_t *parent, int32_t *tokens, int32_t *q_row, int32_t *n_nodes,
+                    int32_t *lvl_begin, int B, int Tmax, int32_t *dev_status,
+                    tsd_stream_t stream)
+{
+    if (B < 0 || Tmax < 1 || Tmax > TSD_MAX_TREE || Rq < 1 || V < 1 || k < 1 || k > Tmax)
+        return TSD_ERR_SHAPE;
+    if (B == 0)
+        return TSD_OK;
+    if (!q_probs || !frow || !parent || !tokens || !q_row || !n_nodes || !lvl_begin)
+        return TSD_ERR_NULL;
+    return tsd::launch_tree_expand(q_probs, Rq, V, frow, k, parent, tokens, q_row, n_nodes,
+                                   lvl_begin, B, Tmax, dev_status,
+                                   reinterpret_cast<cudaStream_t>(stream));
+}
+
+int tsd_tree_dfs_order(const int32_t *parent, const int32_t *tokens, const int32_t *q_row,
+                       const int32_t *n_nodes, int B, int Tmax, int32_t *perm,
+                       int32_t *out_parent, int32_t *out_tokens, int32_t *out_q_row,
+                       int32_t *dev_status, tsd_stream_t stream)
+{
+    if (B < 0 || Tmax < 1 || Tmax > TSD_MAX_TREE)
+        return TSD_ERR_SHAPE;
+    if (B == 0)
+        return TSD_OK;
+    if (!parent || !tokens || !q_row || !n_nodes || !perm || !out_parent || !out_tokens ||
+        !out_q_row)
+        return TSD_ERR_NULL;
+    return tsd::launch_tree_dfs(parent, tokens, q_row, n_nodes, B, Tmax, perm, out_parent,
+                                out_tokens, out_q_row, dev_status,
+                                reinterpret_cast<cudaStream_t>(stream));
+}
+
+int tsd_tree_merge_chains(const int32_t *chain_tokens, const int32_t *chain_q_row,
+                          const int32_t *chain_len, int M, int L, int B, int Tmax,
+                          int32_t *parent, int32_t *tokens, int32_t *q_row, int32_t *n_nodes,
+                          int32_t *dev_status, tsd_stream_t stream)
+{
+    if (B < 0 || M < 1 || L < 1 || Tmax < 1 || Tmax > TSD_MAX_TREE)
+        return TSD_ERR_SHAPE;
+    if (B == 0)
+        return TSD_OK;
+    if (!chain_tokens || !chain_q_row || !chain_len || !parent || !tokens || !q_row || !n_nodes)
+        return TSD_ERR_NULL;
+    return tsd::launch_tree_merge(chain_tokens, chain_q_row, chain_len, M, L, B, Tmax, parent,
+                                  tokens, q_row, n_nodes, dev_status,
+                                  reinterpret_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

@@ -1,0 +1,340 @@
+// Token-tree construction (SpecInfer explainer, "マルチドラフトモデルアプローチ":
+// item 1, an expansion-based tree <k_1, ..., k_n> takes one SSM's top-k_i
+// tokens at every node of depth i-1; item 2, a merge-based tree merges the
+// outputs of several SSMs into one token tree; "Tree Attention のカーネル融合",
+// item 2: the tree is laid out depth-first).
+//
+//   tree_expand_kernel        one CTA per (frontier node, sequence): the k best
+//                             tokens of the node's SSM row (descending
+//                             probability, lower token id on ties) in k block
+//                             passes, each taking the best element strictly
+//                             after the previous pick in that order; writes the
+//                             children at n_nodes + i*k + j;
+//   tree_expand_commit_kernel one thread per sequence: n_nodes and lvl_begin
+//                             advance once every CTA has read them;
+//   tree_dfs_kernel           one thread per sequence: child lists in index
+//                             order, then a stackless pre-order walk;
+//   tree_merge_kernel         one thread per sequence: trie insertion of the
+//                             chains (children kept in creation order), then
+//                             the same pre-order walk.
+// The per-sequence work is at most TSD_MAX_TREE nodes; it runs in shared
+// memory, one sequence per CTA.
+#include <climits>
+
+#include "tsd_common.cuh"
+
+namespace tsd {
+
+namespace {
+
+constexpr int kExpandThreads = 256;
+
+// (v, i) comes before (w, j) in "descending probability, lower token first".
+__device__ __forceinline__ bool before(float v, int i, float w, int j)
+{
+    return v > w || (v == w && i < j);
+}
+
+// Validation shared by both expansion kernels (every CTA reaches the same
+// answer): frontier size F, or 0 if the level cannot be added.
+__device__ int expand_frontier(const int32_t *__restrict__ frow, int Rq, int V, int k,
+                               const int32_t *__restrict__ n_nodes,
+                               const int32_t *__restrict__ lvl_begin, int b, int Tmax, int &n,
+                               int &lb)
+{
+    n = n_nodes[b];
+    lb = lvl_begin[b];
+    const int F = n == 0 ? 1 : n - lb;
+    if (n < 0 || n > Tmax || k < 1 || k > V || F < 1 || lb < 0 || (long)n + (long)F * k > Tmax)
+        return 0;
+    for (int i = 0; i < F; ++i) {
+        const int r = frow[(size_t)b * Tmax + i];
+        if (r < 0 || r >= Rq)
+            return 0;
+    }
+    return F;
+}
+
+__global__ void __launch_bounds__(kExpandThreads)
+    tree_expand_kernel(const float *__restrict__ q_probs, int Rq, int V,
+                       const int32_t *__restrict__ frow, int k, int32_t *__restrict__ parent,
+                       int32_t *__restrict__ tokens, int32_t *__restrict__ q_row,
+                       const int32_t *__restrict__ n_nodes, const int32_t *__restrict__ lvl_begin,
+                       int Tmax)
+{
+    __shared__ float shv[kExpandThreads / 32];
+    __shared__ int shi[kExpandThreads / 32];
+    __shared__ int s_F, s_n, s_lb;
+    const int i = blockIdx.x, b = blockIdx.y;
+    if (threadIdx.x == 0) {
+        int n, lb;
+        s_F = expand_frontier(frow, Rq, V, k, n_nodes, lvl_begin, b, Tmax, n, lb);
+        s_n = n;
+        s_lb = lb;
+    }
+    __syncthreads();
+    const int F = s_F, n = s_n, lb = s_lb;
+    if (i >= F)
+        return;
+    const int r = frow[(size_t)b * Tmax + i];
+    const float *p = q_probs + ((size_t)b * Rq + r) * V;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float pv = 0.f;
+    int pi = -1;
+    for (int j = 0; j < k; ++j) {
+        float bv = -INFINITY;
+        int bi = INT_MAX;
+        for (int x = threadIdx.x; x < V; x += kExpandThreads) {
+            const float v = __ldg(p + x);
+            if (pi >= 0 && !before(pv, pi, v, x))
+                continue;   // at or before the previous pick
+            if (bi == INT_MAX || before(v, x, bv, bi)) {
+                bv = v;
+                bi = x;
+            }
+        }
+        // block arg-best (value desc, index asc); INT_MAX = nothing found
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (oi != INT_MAX && (bi == INT_MAX || before(ov, oi, bv, bi))) {
+                bv = ov;
+                bi = oi;
+            }
+        }
+        if (lane == 0) {
+            shv[warp] = bv;
+            shi[warp] = bi;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            bv = lane < kExpandThreads / 32 ? shv[lane] : -INFINITY;
+            bi = lane < kExpandThreads / 32 ? shi[lane] : INT_MAX;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                if (oi != INT_MAX && (bi == INT_MAX || before(ov, oi, bv, bi))) {
+                    bv = ov;
+                    bi = oi;
+                }
+            }
+            if (lane == 0) {
+                shv[0] = bv;
+                shi[0] = bi;
+            }
+        }
+        __syncthreads();
+        pv = shv[0];
+        pi = shi[0];
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            const size_t u = (size_t)b * Tmax + n + i * k + j;
+            parent[u] = n == 0 ? -1 : lb + i;
+            tokens[u] = pi;   // k <= V: a pick always exists
+            q_row[u] = r;
+        }
+    }
+}
+
+__global__ void tree_expand_commit_kernel(const int32_t *__restrict__ frow, int Rq, int V, int k,
+                                          int32_t *__restrict__ n_nodes,
+                                          int32_t *__restrict__ lvl_begin, int B, int Tmax,
+                                          int32_t *dev_status)
+{
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= B)
+        return;
+    int n, lb;
+    const int F = expand_frontier(frow, Rq, V, k, n_nodes, lvl_begin, b, Tmax, n, lb);
+    if (F == 0) {
+        flag(dev_status, TSD_DEV_BAD_TREE);
+        return;
+    }
+    lvl_begin[b] = n;
+    n_nodes[b] = n + F * k;
+}
+
+// Pre-order of the tree held in shared memory (par, first child, next
+// sibling; -1 = none), written to order[]: returns the node count visited.
+__device__ int preorder(const int *par, const int *fc, const int *ns, int root_first, int *order)
+{
+    int cnt = 0;
+    int u = root_first;
+    while (u >= 0) {
+        order[cnt++] = u;
+        if (fc[u] >= 0) {
+            u = fc[u];
+            continue;
+        }
+        while (u >= 0 && ns[u] < 0)
+            u = par[u];
+        if (u >= 0)
+            u = ns[u];
+    }
+    return cnt;
+}
+
+__global__ void tree_dfs_kernel(const int32_t *__restrict__ parent,
+                                const int32_t *__restrict__ tokens,
+                                const int32_t *__restrict__ q_row,
+                                const int32_t *__restrict__ n_nodes, int Tmax,
+                                int32_t *__restrict__ perm, int32_t *__restrict__ out_parent,
+                                int32_t *__restrict__ out_tokens, int32_t *__restrict__ out_q_row,
+                                int32_t *dev_status)
+{
+    __shared__ int par[kMaxTree], fc[kMaxTree], ns[kMaxTree], order[kMaxTree], inv[kMaxTree];
+    const int b = blockIdx.x;
+    if (threadIdx.x != 0)
+        return;
+    const int T = n_nodes[b];
+    bool ok = T >= 0 && T <= Tmax;
+    for (int v = 0; ok && v < T; ++v) {
+        par[v] = parent[(size_t)b * Tmax + v];
+        ok = par[v] >= -1 && par[v] < v;
+    }
+    if (!ok) {
+        flag(dev_status, TSD_DEV_BAD_TREE);
+        return;
+    }
+    int root_first = -1;
+    for (int v = T - 1; v >= 0; --v)   // children lists in increasing index
+        fc[v] = -1;
+    for (int v = T - 1; v >= 0; --v) {
+        const int p = par[v];
+        if (p < 0) {
+            ns[v] = root_first;
+            root_first = v;
+        } else {
+            ns[v] = fc[p];
+            fc[p] = v;
+        }
+    }
+    const int cnt = preorder(par, fc, ns, root_first, order);
+    for (int i = 0; i < cnt; ++i)
+        inv[order[i]] = i;
+    for (int i = 0; i < cnt; ++i) {
+        const int u = order[i];
+        const size_t o = (size_t)b * Tmax + i;
+        perm[o] = u;
+        out_parent[o] = par[u] < 0 ? -1 : inv[par[u]];
+        out_tokens[o] = tokens[(size_t)b * Tmax + u];
+        out_q_row[o] = q_row[(size_t)b * Tmax + u];
+    }
+}
+
+__global__ void tree_merge_kernel(const int32_t *__restrict__ ctok, const int32_t *__restrict__ cq,
+                                  const int32_t *__restrict__ clen, int M, int L, int Tmax,
+                                  int32_t *__restrict__ parent, int32_t *__restrict__ tokens,
+                                  int32_t *__restrict__ q_row, int32_t *__restrict__ n_nodes,
+                                  int32_t *dev_status)
+{
+    __shared__ int par[kMaxTree], tok[kMaxTree], qr[kMaxTree], fc[kMaxTree], lc[kMaxTree],
+        ns[kMaxTree], order[kMaxTree], inv[kMaxTree];
+    const int b = blockIdx.x;
+    if (threadIdx.x != 0)
+        return;
+    int T = 0, root_first = -1, root_last = -1;
+    bool ok = true;
+    for (int m = 0; ok && m < M; ++m) {
+        const int len = clen[(size_t)b * M + m];
+        if (len < 0 || len > L) {
+            ok = false;
+            break;
+        }
+        int cur = -1;
+        for (int i = 0; i < len; ++i) {
+            const int t = ctok[((size_t)b * M + m) * L + i];
+            int v = cur < 0 ? root_first : fc[cur];
+            while (v >= 0 && tok[v] != t)
+                v = ns[v];
+            if (v < 0) {   // a new node, last child of cur
+                if (T == Tmax) {
+                    ok = false;
+                    break;
+                }
+                v = T++;
+                par[v] = cur;
+                tok[v] = t;
+                qr[v] = cq[((size_t)b * M + m) * L + i];
+                fc[v] = lc[v] = ns[v] = -1;
+                if (cur < 0) {
+                    if (root_last < 0)
+                        root_first = v;
+                    else
+                        ns[root_last] = v;
+                    root_last = v;
+                } else {
+                    if (lc[cur] < 0)
+                        fc[cur] = v;
+                    else
+                        ns[lc[cur]] = v;
+                    lc[cur] = v;
+                }
+            }
+            cur = v;
+        }
+    }
+    if (!ok) {
+        n_nodes[b] = -1;
+        flag(dev_status, TSD_DEV_BAD_TREE);
+        return;
+    }
+    const int cnt = preorder(par, fc, ns, root_first, order);
+    for (int i = 0; i < cnt; ++i)
+        inv[order[i]] = i;
+    for (int i = 0; i < cnt; ++i) {
+        const int u = order[i];
+        const size_t o = (size_t)b * Tmax + i;
+        parent[o] = par[u] < 0 ? -1 : inv[par[u]];
+        tokens[o] = tok[u];
+        q_row[o] = qr[u];
+    }
+    n_nodes[b] = cnt;
+}
+
+}  // namespace
+
+int launch_tree_expand(const float *q_probs, int Rq, int V, const int32_t *frow, int k,
+                       int32_t *parent, int32_t *tokens, int32_t *q_row, int32_t *n_nodes,
+                       int32_t *lvl_begin, int B, int Tmax, int32_t *dev_status,
+                       cudaStream_t stream)
+{
+    if (B == 0)
+        return TSD_OK;
+    tree_expand_kernel<<<dim3(Tmax, B), kExpandThreads, 0, stream>>>(
+        q_probs, Rq, V, frow, k, parent, tokens, q_row, n_nodes, lvl_begin, Tmax);
+    TSD_LAUNCH_CHECK();
+    tree_expand_commit_kernel<<<(B + 127) / 128, 128, 0, stream>>>(frow, Rq, V, k, n_nodes,
+                                                                  lvl_begin, B, Tmax, dev_status);
+    TSD_LAUNCH_CHECK();
+    return TSD_OK;
+}
+
+int launch_tree_dfs(const int32_t *parent, const int32_t *tokens, const int32_t *q_row,
+                    const int32_t *n_nodes, int B, int Tmax, int32_t *perm, int32_t *out_parent,
+                    int32_t *out_tokens, int32_t *out_q_row, int32_t *dev_status,
+                    cudaStream_t stream)
+{
+    if (B == 0)
+        return TSD_OK;
+    tree_dfs_kernel<<<B, 32, 0, stream>>>(parent, tokens, q_row, n_nodes, Tmax, perm, out_parent,
+                                          out_tokens, out_q_row, dev_status);
+    TSD_LAUNCH_CHECK();
+    return TSD_OK;
+}
+
+int launch_tree_merge(const int32_t *ctok, const int32_t *cq, const int32_t *clen, int M, int L,
+                      int B, int Tmax, int32_t *parent, int32_t *tokens, int32_t *q_row,
+                      int32_t *n_nodes, int32_t *dev_status, cudaStream_t stream)
+{
+    if (B == 0)
+        return TSD_OK;
+    tree_merge_kernel<<<B, 32, 0, stream>>>(ctok, cq, clen, M, L, Tmax, parent, tokens, q_row,
+                                            n_nodes, dev_status);
+    TSD_LAUNCH_CHECK();
+    return TSD_OK;
+}
+
+}  // namespace tsd

@@ -124,6 +124,17 @@ int launch_umma_attention(const AttnArgs &a, void *ws, size_t ws_bytes, int num_
 
 size_t verify_workspace(int B, int Tmax, int V);
 size_t verify_stochastic_scratch();   // fixed: independent of the shape
+int launch_tree_expand(const float *q_probs, int Rq, int V, const int32_t *frow, int k,
+                       int32_t *parent, int32_t *tokens, int32_t *q_row, int32_t *n_nodes,
+                       int32_t *lvl_begin, int B, int Tmax, int32_t *dev_status,
+                       cudaStream_t stream);
+int launch_tree_dfs(const int32_t *parent, const int32_t *tokens, const int32_t *q_row,
+                    const int32_t *n_nodes, int B, int Tmax, int32_t *perm, int32_t *out_parent,
+                    int32_t *out_tokens, int32_t *out_q_row, int32_t *dev_status,
+                    cudaStream_t stream);
+int launch_tree_merge(const int32_t *ctok, const int32_t *cq, const int32_t *clen, int M, int L,
+                      int B, int Tmax, int32_t *parent, int32_t *tokens, int32_t *q_row,
+                      int32_t *n_nodes, int32_t *dev_status, cudaStream_t stream);
 int launch_kv_commit(void *k_cache, void *v_cache, const int32_t *prefix_len,
                      const int32_t *out_path, const int32_t *n_accepted, int B, int Tmax, int Hkv,
                      int Lmax, int row_bytes, int32_t *new_prefix, int32_t *dev_status,
