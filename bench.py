@@ -445,16 +445,14 @@ def time_tree_build(w, dev, tsd, reps: int = 10):
     while n + 2 * F <= w.Tmax:
         ks.append(2)
         n, F = n + 2 * F, 2 * F
-    n, F, frows = 0, 1, []
+    n, F, start, frows = 0, 1, 0, []
     for k in ks:
-        lb = n
-        fr = torch.zeros((B, w.Tmax), dtype=torch.int32)
-        if n > 0:
-            fr[:, :F] = torch.arange(lb, n, dtype=torch.int32) + 1   # node u's row is u + 1
+        fr = torch.zeros((B, w.Tmax), dtype=torch.int32)   # root level: row 0
+        if n > 0:   # frontier = the level added last, nodes start .. n-1; node u's row is u + 1
+            fr[:, :F] = torch.arange(start, n, dtype=torch.int32) + 1
         frows.append(fr.to(dev))
+        start = n
         n, F = n + F * k, F * k
-        if n > w.Tmax:
-            return None
     q = torch.rand((B, n + 1, V), device=dev, generator=None)
     z = lambda: torch.zeros((B, w.Tmax), dtype=torch.int32, device=dev)  # noqa: E731
     tree = tsd.Tree(z(), z(), z(), torch.zeros(B, dtype=torch.int32, device=dev))

@@ -7,9 +7,11 @@
 //   tree_expand_kernel        one CTA per (frontier node, sequence): the k best
 //                             tokens of the node's SSM row (descending
 //                             probability, lower token id on ties) in k block
-//                             passes, each taking the best element strictly
-//                             after the previous pick in that order; writes the
-//                             children at n_nodes + i*k + j;
+//                             passes (8 loads in flight per thread), each
+//                             taking the best element strictly after the
+//                             previous pick in that order -- a compare and a
+//                             select per element; writes the children at
+//                             n_nodes + i*k + j;
 //   tree_expand_commit_kernel one thread per sequence: n_nodes and lvl_begin
 //                             advance once every CTA has read them;
 //   tree_dfs_kernel           one thread per sequence: child lists in index
@@ -27,7 +29,9 @@ namespace tsd {
 
 namespace {
 
-constexpr int kExpandThreads = 256;
+constexpr int kExpandThreads = 512;
+constexpr int kLoadBatch = 8;       // loads in flight per thread in the row scans
+constexpr int kMergeStage = 1024;   // chain entries staged in shared memory
 
 // (v, i) comes before (w, j) in "descending probability, lower token first".
 __device__ __forceinline__ bool before(float v, int i, float w, int j)
@@ -35,8 +39,9 @@ __device__ __forceinline__ bool before(float v, int i, float w, int j)
     return v > w || (v == w && i < j);
 }
 
-// Validation shared by both expansion kernels (every CTA reaches the same
-// answer): frontier size F, or 0 if the level cannot be added.
+// Validation of one level (the commit kernel's; the expansion kernel makes the
+// same checks in parallel): frontier size F, or 0 if the level cannot be
+// added.
 __device__ int expand_frontier(const int32_t *__restrict__ frow, int Rq, int V, int k,
                                const int32_t *__restrict__ n_nodes,
                                const int32_t *__restrict__ lvl_begin, int b, int Tmax, int &n,
@@ -55,6 +60,48 @@ __device__ int expand_frontier(const int32_t *__restrict__ frow, int Rq, int V, 
     return F;
 }
 
+// Block arg-best of (v, i) over the CTA (value desc, index asc; INT_MAX =
+// none); the result in every thread.
+__device__ __forceinline__ void block_best(float &v, int &i, float *shv, int *shi)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, v, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, i, o);
+        if (oi != INT_MAX && (i == INT_MAX || before(ov, oi, v, i))) {
+            v = ov;
+            i = oi;
+        }
+    }
+    if (lane == 0) {
+        shv[warp] = v;
+        shi[warp] = i;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        v = lane < kExpandThreads / 32 ? shv[lane] : -INFINITY;
+        i = lane < kExpandThreads / 32 ? shi[lane] : INT_MAX;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, v, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, i, o);
+            if (oi != INT_MAX && (i == INT_MAX || before(ov, oi, v, i))) {
+                v = ov;
+                i = oi;
+            }
+        }
+        if (lane == 0) {
+            shv[0] = v;
+            shi[0] = i;
+        }
+    }
+    __syncthreads();
+    v = shv[0];
+    i = shi[0];
+    __syncthreads();
+}
+
 __global__ void __launch_bounds__(kExpandThreads)
     tree_expand_kernel(const float *__restrict__ q_probs, int Rq, int V,
                        const int32_t *__restrict__ frow, int k, int32_t *__restrict__ parent,
@@ -64,71 +111,82 @@ __global__ void __launch_bounds__(kExpandThreads)
 {
     __shared__ float shv[kExpandThreads / 32];
     __shared__ int shi[kExpandThreads / 32];
-    __shared__ int s_F, s_n, s_lb;
-    const int i = blockIdx.x, b = blockIdx.y;
-    if (threadIdx.x == 0) {
-        int n, lb;
-        s_F = expand_frontier(frow, Rq, V, k, n_nodes, lvl_begin, b, Tmax, n, lb);
-        s_n = n;
-        s_lb = lb;
+    // sequence fastest: the working CTAs (i < F) of every sequence come first
+    // in launch order, the idle ones after them
+    const int b = blockIdx.x, i = blockIdx.y;
+    // the frontier size from two loads; CTAs beyond it leave at once
+    const int n = n_nodes[b], lb = lvl_begin[b];
+    const int F = n == 0 ? 1 : n - lb;
+    if (n < 0 || n > Tmax || k < 1 || k > V || F < 1 || lb < 0 ||
+        (long)n + (long)F * k > Tmax || i >= F)
+        return;
+    // every q row of the frontier in range (the same answer in every CTA)
+    int bad = 0;
+    for (int f = threadIdx.x; f < F; f += kExpandThreads) {
+        const int r = frow[(size_t)b * Tmax + f];
+        bad |= r < 0 || r >= Rq;
     }
-    __syncthreads();
-    const int F = s_F, n = s_n, lb = s_lb;
-    if (i >= F)
+    if (__syncthreads_or(bad))
         return;
     const int r = frow[(size_t)b * Tmax + i];
     const float *p = q_probs + ((size_t)b * Rq + r) * V;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const bool vec = (V & 3) == 0 && (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
     float pv = 0.f;
     int pi = -1;
     for (int j = 0; j < k; ++j) {
         float bv = -INFINITY;
         int bi = INT_MAX;
-        for (int x = threadIdx.x; x < V; x += kExpandThreads) {
-            const float v = __ldg(p + x);
+        auto consider = [&](float v, int x) {
             if (pi >= 0 && !before(pv, pi, v, x))
-                continue;   // at or before the previous pick
+                return;   // at or before the previous pick
             if (bi == INT_MAX || before(v, x, bv, bi)) {
                 bv = v;
                 bi = x;
             }
-        }
-        // block arg-best (value desc, index asc); INT_MAX = nothing found
+        };
+        if (vec) {   // float4 loads, kLoadBatch in flight per thread
+            const float4 *p4 = reinterpret_cast<const float4 *>(p);
+            const int n4 = V >> 2;
+            int x4 = threadIdx.x;
+            for (; x4 + (kLoadBatch - 1) * kExpandThreads < n4;
+                 x4 += kLoadBatch * kExpandThreads) {
+                float4 t[kLoadBatch];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (oi != INT_MAX && (bi == INT_MAX || before(ov, oi, bv, bi))) {
-                bv = ov;
-                bi = oi;
-            }
-        }
-        if (lane == 0) {
-            shv[warp] = bv;
-            shi[warp] = bi;
-        }
-        __syncthreads();
-        if (warp == 0) {
-            bv = lane < kExpandThreads / 32 ? shv[lane] : -INFINITY;
-            bi = lane < kExpandThreads / 32 ? shi[lane] : INT_MAX;
+                for (int u = 0; u < kLoadBatch; ++u)
+                    t[u] = __ldg(p4 + x4 + u * kExpandThreads);
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                if (oi != INT_MAX && (bi == INT_MAX || before(ov, oi, bv, bi))) {
-                    bv = ov;
-                    bi = oi;
+                for (int u = 0; u < kLoadBatch; ++u) {
+                    const int x = 4 * (x4 + u * kExpandThreads);
+                    consider(t[u].x, x);
+                    consider(t[u].y, x + 1);
+                    consider(t[u].z, x + 2);
+                    consider(t[u].w, x + 3);
                 }
             }
-            if (lane == 0) {
-                shv[0] = bv;
-                shi[0] = bi;
+            for (; x4 < n4; x4 += kExpandThreads) {
+                const float4 t = __ldg(p4 + x4);
+                consider(t.x, 4 * x4);
+                consider(t.y, 4 * x4 + 1);
+                consider(t.z, 4 * x4 + 2);
+                consider(t.w, 4 * x4 + 3);
             }
+        } else {
+            int x = threadIdx.x;
+            for (; x + (kLoadBatch - 1) * kExpandThreads < V; x += kLoadBatch * kExpandThreads) {
+                float t[kLoadBatch];
+#pragma unroll
+                for (int u = 0; u < kLoadBatch; ++u)
+                    t[u] = __ldg(p + x + u * kExpandThreads);
+#pragma unroll
+                for (int u = 0; u < kLoadBatch; ++u)
+                    consider(t[u], x + u * kExpandThreads);
+            }
+            for (; x < V; x += kExpandThreads)
+                consider(__ldg(p + x), x);
         }
-        __syncthreads();
-        pv = shv[0];
-        pi = shi[0];
-        __syncthreads();
+        block_best(bv, bi, shv, shi);
+        pv = bv;
+        pi = bi;
         if (threadIdx.x == 0) {
             const size_t u = (size_t)b * Tmax + n + i * k + j;
             parent[u] = n == 0 ? -1 : lb + i;
@@ -185,36 +243,45 @@ __global__ void tree_dfs_kernel(const int32_t *__restrict__ parent,
                                 int32_t *dev_status)
 {
     __shared__ int par[kMaxTree], fc[kMaxTree], ns[kMaxTree], order[kMaxTree], inv[kMaxTree];
-    const int b = blockIdx.x;
-    if (threadIdx.x != 0)
-        return;
+    __shared__ int s_cnt;
+    const int b = blockIdx.x, lane = threadIdx.x;   // one warp
     const int T = n_nodes[b];
-    bool ok = T >= 0 && T <= Tmax;
-    for (int v = 0; ok && v < T; ++v) {
-        par[v] = parent[(size_t)b * Tmax + v];
-        ok = par[v] >= -1 && par[v] < v;
-    }
-    if (!ok) {
-        flag(dev_status, TSD_DEV_BAD_TREE);
+    if (T < 0 || T > Tmax) {
+        if (lane == 0)
+            flag(dev_status, TSD_DEV_BAD_TREE);
         return;
     }
-    int root_first = -1;
-    for (int v = T - 1; v >= 0; --v)   // children lists in increasing index
-        fc[v] = -1;
-    for (int v = T - 1; v >= 0; --v) {
-        const int p = par[v];
-        if (p < 0) {
-            ns[v] = root_first;
-            root_first = v;
-        } else {
-            ns[v] = fc[p];
-            fc[p] = v;
-        }
+    bool bad = false;
+    for (int v = lane; v < T; v += 32) {   // the loads in parallel
+        par[v] = parent[(size_t)b * Tmax + v];
+        bad |= par[v] < -1 || par[v] >= v;
     }
-    const int cnt = preorder(par, fc, ns, root_first, order);
-    for (int i = 0; i < cnt; ++i)
-        inv[order[i]] = i;
-    for (int i = 0; i < cnt; ++i) {
+    if (__any_sync(0xffffffffu, bad)) {
+        if (lane == 0)
+            flag(dev_status, TSD_DEV_BAD_TREE);
+        return;
+    }
+    __syncwarp();
+    if (lane == 0) {   // the walk, on shared memory
+        int root_first = -1;
+        for (int v = T - 1; v >= 0; --v)   // children lists in increasing index
+            fc[v] = -1;
+        for (int v = T - 1; v >= 0; --v) {
+            const int p = par[v];
+            if (p < 0) {
+                ns[v] = root_first;
+                root_first = v;
+            } else {
+                ns[v] = fc[p];
+                fc[p] = v;
+            }
+        }
+        s_cnt = preorder(par, fc, ns, root_first, order);
+        for (int i = 0; i < s_cnt; ++i)
+            inv[order[i]] = i;
+    }
+    __syncwarp();
+    for (int i = lane; i < s_cnt; i += 32) {
         const int u = order[i];
         const size_t o = (size_t)b * Tmax + i;
         perm[o] = u;
@@ -232,20 +299,35 @@ __global__ void tree_merge_kernel(const int32_t *__restrict__ ctok, const int32_
 {
     __shared__ int par[kMaxTree], tok[kMaxTree], qr[kMaxTree], fc[kMaxTree], lc[kMaxTree],
         ns[kMaxTree], order[kMaxTree], inv[kMaxTree];
-    const int b = blockIdx.x;
-    if (threadIdx.x != 0)
+    __shared__ int s_ct[kMergeStage], s_cq[kMergeStage], s_len[kMergeStage];
+    const int b = blockIdx.x, lane = threadIdx.x;   // one warp
+    // the chains into shared memory in parallel when they fit
+    const bool staged = M * L <= kMergeStage;
+    if (staged) {
+        for (int i = lane; i < M * L; i += 32) {
+            s_ct[i] = ctok[(size_t)b * M * L + i];
+            s_cq[i] = cq[(size_t)b * M * L + i];
+        }
+        for (int m = lane; m < M; m += 32)
+            s_len[m] = clen[(size_t)b * M + m];
+    }
+    __syncwarp();
+    if (lane != 0)
         return;
+    const int *ct = staged ? s_ct : ctok + (size_t)b * M * L;
+    const int *cqr = staged ? s_cq : cq + (size_t)b * M * L;
+    const int *cl = staged ? s_len : clen + (size_t)b * M;
     int T = 0, root_first = -1, root_last = -1;
     bool ok = true;
     for (int m = 0; ok && m < M; ++m) {
-        const int len = clen[(size_t)b * M + m];
+        const int len = cl[m];
         if (len < 0 || len > L) {
             ok = false;
             break;
         }
         int cur = -1;
         for (int i = 0; i < len; ++i) {
-            const int t = ctok[((size_t)b * M + m) * L + i];
+            const int t = ct[(size_t)m * L + i];
             int v = cur < 0 ? root_first : fc[cur];
             while (v >= 0 && tok[v] != t)
                 v = ns[v];
@@ -257,7 +339,7 @@ __global__ void tree_merge_kernel(const int32_t *__restrict__ ctok, const int32_
                 v = T++;
                 par[v] = cur;
                 tok[v] = t;
-                qr[v] = cq[((size_t)b * M + m) * L + i];
+                qr[v] = cqr[(size_t)m * L + i];
                 fc[v] = lc[v] = ns[v] = -1;
                 if (cur < 0) {
                     if (root_last < 0)
@@ -303,7 +385,7 @@ int launch_tree_expand(const float *q_probs, int Rq, int V, const int32_t *frow,
 {
     if (B == 0)
         return TSD_OK;
-    tree_expand_kernel<<<dim3(Tmax, B), kExpandThreads, 0, stream>>>(
+    tree_expand_kernel<<<dim3(B, Tmax), kExpandThreads, 0, stream>>>(
         q_probs, Rq, V, frow, k, parent, tokens, q_row, n_nodes, lvl_begin, Tmax);
     TSD_LAUNCH_CHECK();
     tree_expand_commit_kernel<<<(B + 127) / 128, 128, 0, stream>>>(frow, Rq, V, k, n_nodes,
