@@ -72,6 +72,7 @@ constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;   // + alignment slack
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
+constexpr float kLazyLimit = 18446744073709551616.0f;   // 2^64: headroom of a P tile sum
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 constexpr int kRowsThreads = 192;       // rows kernel: 6 warps
@@ -287,10 +288,15 @@ __device__ __forceinline__ void issue_qk(const Setup &su, int lane, uint32_t col
     constexpr uint32_t idesc = ptx::idesc_bf16(BQ, BN, false, false);
     const int st = t % NSK;
     if (lane == 0) {
+        // base descriptors once; the k-slices are constant offsets (the
+        // address field is addr >> 4 and shared addresses stay below 256 KB,
+        // so adding to the packed word never carries out of it)
+        const uint64_t dq = desc_kmajor(su.sQ, 0), dk = desc_kmajor(su.sK + st * kTile, 0);
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk)
-            ptx::mma_ss(su.tmem + col_s, desc_kmajor(su.sQ, kk),
-                        desc_kmajor(su.sK + st * kTile, kk), idesc, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < HD / 16; ++kk) {
+            const uint64_t off = ((uint32_t)(kk >> 2) * kSub + (uint32_t)(kk & 3) * 32u) >> 4;
+            ptx::mma_ss(su.tmem + col_s, dq + off, dk + off, idesc, kk > 0 ? 1u : 0u);
+        }
         ptx::mma_commit(s_full);
         ptx::mma_commit(su.bars.k_empty(st));
     }
@@ -317,10 +323,12 @@ __device__ __forceinline__ void issue_pv(const Setup &su, int lane, uint32_t col
     }
     ptx::tc_fence_after();
     if (lane == 0) {
+        const uint64_t dv = desc_v(su.sV + vs * kTile, 0);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-            ptx::mma_ts(su.tmem + col_o, su.tmem + col_p + kk * 8, desc_v(su.sV + vs * kTile, kk),
-                        idesc, (accumulate || kk > 0) ? 1u : 0u);
+            ptx::mma_ts(su.tmem + col_o, su.tmem + col_p + kk * 8,
+                        dv + (uint64_t)((kk * 16u * 128u) >> 4), idesc,
+                        (accumulate || kk > 0) ? 1u : 0u);
         ptx::mma_commit(su.bars.v_empty(vs));
         ptx::mma_commit(o_ready);
     }
@@ -385,6 +393,25 @@ __device__ __forceinline__ float exp_pack64(const uint32_t (&sa)[32], const uint
         ptx::add2(acc[a], acc[a + 1], p2, p3);
         pk[k] = ptx::pack_bf16(p0, p1);
         pk[16 + k] = ptx::pack_bf16(p2, p3);
+    }
+    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
+// P for 32 scores (one 32-column chunk, loaded and masked), packed to bf16
+// into pk[16]; returns their sum.
+__device__ __forceinline__ float exp_pack32(const uint32_t (&sa)[32], float scale_log2,
+                                            float neg_m, uint32_t (&pk)[16])
+{
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        float x0, x1;
+        ptx::fma2_bc(x0, x1, __uint_as_float(sa[2 * k]), __uint_as_float(sa[2 * k + 1]),
+                     scale_log2, neg_m);
+        const float p0 = ptx::ex2(x0), p1 = ptx::ex2(x1);
+        const int a = (k & 1) * 2;
+        ptx::add2(acc[a], acc[a + 1], p0, p1);
+        pk[k] = ptx::pack_bf16(p0, p1);
     }
     return (acc[0] + acc[1]) + (acc[2] + acc[3]);
 }
@@ -624,34 +651,51 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
                 for (int c = 0; c < 4; ++c)
                     mask32(sr[c], valid_bits(pos0 + c * 32, P, ke, mw));
             }
-            float mx[16];
+            // P against the running max, written speculatively; the row max
+            // is only taken (and O rescaled) when some exponent may exceed
+            // the headroom: the tile's sum above 2^64 (or not finite), which
+            // always happens on the first tile (m_run = -inf).  One exp loop,
+            // run a second time only by a warp that took the max.
+            float lsum = 0.f;
+#pragma unroll 1
+            for (int pass = 0; pass < 2; ++pass) {
+                const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
+                lsum = 0.f;
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-                mx[i] = -INFINITY;
-            max32x2(sr[0], sr[1], mx);
-            max32x2(sr[2], sr[3], mx);
-            const float mt = max16(mx) * scale_log2;
-            const bool need = mt > m_run + kRescaleThreshold;   // false if mt is -inf
-            const float m_new = need ? mt : m_run;
-            const float alpha = need ? ptx::ex2(m_run - m_new) : 1.f;   // 0 when m_run = -inf
-            if (__any_sync(0xffffffffu, need) && j > 0) {
-                // O holds PV_0 .. PV_{j-1}: wait for the last of them.
-                if (!wait_pv(j - 1)) {
-                    ok = false;
-                    break;
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t pk[16];
+                    lsum += exp_pack32(sr[c], scale_log2, neg_m, pk);
+                    ptx::tmem_st16(taddr_s + c * 16, pk);
                 }
-                ptx::tc_fence_after();
-                rescale_o(taddr_o, alpha);
-            }
-            l_run *= alpha;
-            m_run = m_new;
-            const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
+                const bool redo = !(lsum <= kLazyLimit) || m_run == -INFINITY;
+                if (pass == 1 || !__any_sync(0xffffffffu, redo))
+                    break;
+                float mx[16];
 #pragma unroll
-            for (int c2 = 0; c2 < 2; ++c2) {
-                uint32_t pk[32];
-                l_run += exp_pack64(sr[2 * c2], sr[2 * c2 + 1], scale_log2, neg_m, pk);
-                ptx::tmem_st32(taddr_s + c2 * 32, pk);
+                for (int i = 0; i < 16; ++i)
+                    mx[i] = -INFINITY;
+                max32x2(sr[0], sr[1], mx);
+                max32x2(sr[2], sr[3], mx);
+                const float mt = max16(mx) * scale_log2;
+                const bool need = mt > m_run + kRescaleThreshold;   // false if mt is -inf
+                const float m_new = need ? mt : m_run;
+                const float alpha = need ? ptx::ex2(m_run - m_new) : 1.f;   // 0 when m_run = -inf
+                if (__any_sync(0xffffffffu, need) && j > 0) {
+                    // O holds PV_0 .. PV_{j-1}: wait for the last of them.
+                    if (!wait_pv(j - 1)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    rescale_o(taddr_o, alpha);
+                }
+                l_run *= alpha;
+                m_run = m_new;
+                ptx::tmem_wait_st();   // the speculative P is overwritten next pass
             }
+            if (!ok)
+                break;
+            l_run += lsum;
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             warp_arrive(su.bars.p_full(j % NS));
