@@ -317,6 +317,24 @@ int tsd_kv_commit(void *k_cache, void *v_cache, const int32_t *prefix_len,
                   tsd_stream_t stream);
 
 /*
+ * Self-test of the bounded waits (no counterpart in the paper).  Every wait
+ * in the kernels above gives up after a time limit, sets TSD_DEV_TIMEOUT and
+ * returns, so that a stalled pipeline ends with a status instead of a hung
+ * GPU.  This call runs those same wait routines on something that never
+ * completes, with a short limit, so that tests can check the behaviour:
+ *   kind 0  the mbarrier wait of the tensor-core attention kernels, on an
+ *           mbarrier nobody arrives on;
+ *   kind 1  the team barrier of the stochastic walk, on a counter whose
+ *           target one CTA cannot reach.
+ *   limit_ns  in [1 ms, 2 s]; scratch: 8 bytes of device memory (8-aligned).
+ * Expected result: the kernel ends after about limit_ns with TSD_DEV_TIMEOUT
+ * set in *dev_status.  Host errors: TSD_ERR_SHAPE, TSD_ERR_NULL,
+ * TSD_ERR_ALIGN, TSD_ERR_CUDA.
+ */
+int tsd_debug_wait_probe(int kind, unsigned long long limit_ns, void *scratch,
+                         int32_t *dev_status, tsd_stream_t stream);
+
+/*
  * Stochastic verification without a workspace, for callers that cannot
  * allocate device memory (for example a serving engine whose KV-cache pool
  * already owns nearly all of the GPU's memory, or a caller reaching the

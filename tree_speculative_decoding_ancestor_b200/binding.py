@@ -55,6 +55,7 @@ _SIGNATURES: Dict[str, Tuple[object, list]] = {
     "tsd_tree_expand": (_I, [_P, _I, _I, _P, _I, _P, _P, _P, _P, _P, _I, _I, _P, _P]),
     "tsd_tree_dfs_order": (_I, [_P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P]),
     "tsd_tree_merge_chains": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "tsd_debug_wait_probe": (_I, [_I, ctypes.c_ulonglong, _P, _P, _P]),
 }
 
 
@@ -456,3 +457,16 @@ def tree_merge_chains(chain_tokens: torch.Tensor, chain_q_row: torch.Tensor,
                                    _ptr(out.n_nodes), _ptr(st), _stream(dev))
     _check(rc, "tsd_tree_merge_chains")
     return out
+
+
+def debug_wait_probe(kind: int, limit_ns: int = 50_000_000, device=None,
+                     status: Optional[torch.Tensor] = None) -> None:
+    """Run the kernels' bounded wait routines on something that never completes
+    (kind 0: mbarrier wait; kind 1: team barrier); they must end after about
+    limit_ns with DEV_TIMEOUT set in the status word."""
+    lib = load_library()
+    dev = torch.device(device or torch.cuda.current_device())
+    scratch = torch.zeros(2, dtype=torch.int32, device=dev)
+    st = device_status(dev) if status is None else status
+    rc = lib.tsd_debug_wait_probe(int(kind), int(limit_ns), _ptr(scratch), _ptr(st), _stream(dev))
+    _check(rc, "tsd_debug_wait_probe")

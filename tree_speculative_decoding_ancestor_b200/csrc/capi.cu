@@ -298,4 +298,17 @@ int tsd_tree_merge_chains(const int32_t *chain_tokens, const int32_t *chain_q_ro
                                   reinterpret_cast<cudaStream_t>(stream));
 }
 
+int tsd_debug_wait_probe(int kind, unsigned long long limit_ns, void *scratch,
+                         int32_t *dev_status, tsd_stream_t stream)
+{
+    if ((kind != 0 && kind != 1) || limit_ns < 1000000ull || limit_ns > 2000000000ull)
+        return TSD_ERR_SHAPE;
+    if (!scratch || !dev_status)
+        return TSD_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(scratch) & 7u)
+        return TSD_ERR_ALIGN;
+    return tsd::launch_wait_probe(kind, limit_ns, scratch, dev_status,
+                                  reinterpret_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

@@ -135,6 +135,8 @@ int launch_tree_dfs(const int32_t *parent, const int32_t *tokens, const int32_t 
 int launch_tree_merge(const int32_t *ctok, const int32_t *cq, const int32_t *clen, int M, int L,
                       int B, int Tmax, int32_t *parent, int32_t *tokens, int32_t *q_row,
                       int32_t *n_nodes, int32_t *dev_status, cudaStream_t stream);
+int launch_wait_probe(int kind, unsigned long long limit_ns, void *scratch,
+                      int32_t *dev_status, cudaStream_t stream);
 int launch_kv_commit(void *k_cache, void *v_cache, const int32_t *prefix_len,
                      const int32_t *out_path, const int32_t *n_accepted, int B, int Tmax, int Hkv,
                      int Lmax, int row_bytes, int32_t *new_prefix, int32_t *dev_status,

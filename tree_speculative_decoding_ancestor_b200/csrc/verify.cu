@@ -44,6 +44,7 @@
 #include <climits>
 
 #include "fp64_exp.cuh"
+#include "team_barrier.cuh"
 #include "tsd_common.cuh"
 
 namespace tsd {
@@ -558,49 +559,6 @@ __global__ void __launch_bounds__(kFinThreads)
 }
 
 // -------------------------------------------------------------- stochastic
-__device__ __forceinline__ unsigned long long global_ns()
-{
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-// Barrier over the K CTAs of one team (co-resident: cooperative launch).
-// `target` = K x the number of barriers the team has entered, this one
-// included.  Thread 0 publishes the CTA's slot write (a release-ordered
-// arrival) and spins on the counter; after kTeamWaitNs it raises the team's
-// abort flag, which releases the other CTAs as well.  False after an abort.
-__device__ bool team_barrier(int2 *team, int target, int *sh_ok)
-{
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int *arrive = &team->x;
-        volatile int *abort = &team->y;
-        // release: this CTA's slot write is visible before its arrival
-        asm volatile("red.release.gpu.add.s32 [%0], 1;" ::"l"(arrive) : "memory");
-        const unsigned long long t0 = global_ns();
-        int ok = 1;
-        for (;;) {
-            int v;
-            asm volatile("ld.acquire.gpu.b32 %0, [%1];" : "=r"(v) : "l"(arrive) : "memory");
-            if (v >= target)
-                break;
-            if (*abort) {
-                ok = 0;
-                break;
-            }
-            if (global_ns() - t0 > kTeamWaitNs) {
-                atomicExch(&team->y, 1);
-                ok = 0;
-                break;
-            }
-            __nanosleep(64);
-        }
-        *sh_ok = ok;
-    }
-    __syncthreads();
-    return *sh_ok != 0;
-}
 
 // VEC: V % 4 == 0, so every logits / q row is 16-byte aligned (the entry
 // point checks the base pointers) and the passes use float4 loads.
@@ -675,7 +633,7 @@ __global__ void __launch_bounds__(kWalkThreads)
             if (tid == 0)
                 sl[k] = make_double2(mz.y, __hiloint2double(__float_as_int((float)mz.x), lastk));
             ++nbar;
-            if (!team_barrier(tm, nbar * K, &sh_ok)) {
+            if (!team_barrier(tm, nbar * K, &sh_ok, kTeamWaitNs)) {
                 alive = false;
                 break;
             }
@@ -729,7 +687,7 @@ __global__ void __launch_bounds__(kWalkThreads)
                 if (tid == 0)
                     sl[k] = make_double2(s, (double)lastk);
                 ++nbar;
-                if (!team_barrier(tm, nbar * K, &sh_ok)) {
+                if (!team_barrier(tm, nbar * K, &sh_ok, kTeamWaitNs)) {
                     alive = false;
                     break;
                 }
