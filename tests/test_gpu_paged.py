@@ -31,9 +31,9 @@ def _pools(w, page_size, seed):
 
 CASES = [
     # (seed, B, Tmax, Hq, Hkv, D, dtype, page_size)  kernel used
-    (41, 3, 40, 32, 4, 128, "bf16", 16),     # tcgen05 rows kernel (320 packed rows)
+    (41, 3, 40, 32, 4, 128, "bf16", 16),     # tcgen05 128-key rows kernel (320 packed rows)
     (42, 3, 40, 32, 4, 128, "bf16", 128),
-    (43, 2, 24, 8, 8, 128, "bf16", 64),      # tcgen05 key-split kernel (24 rows)
+    (43, 2, 24, 8, 8, 128, "bf16", 64),      # tcgen05 64-key rows kernel (24 rows)
     (44, 2, 24, 8, 8, 128, "bf16", 256),
     (45, 3, 20, 4, 2, 64, "f32", 32),        # CUDA-core kernel
     (46, 3, 20, 8, 2, 64, "bf16", 16),
@@ -65,6 +65,19 @@ def test_paged_attention_parity(cuda_device, case):
         T = int(w.n_nodes[b])
         assert np.abs(g[b, :T] - ref[b, :T]).max() <= tol
         assert np.array_equal(g[b, :T], f[b, :T])
+
+
+@pytest.mark.parametrize("case", CASES[:2], ids=[f"s{c[0]}_p{c[7]}" for c in CASES[:2]])
+def test_paged_attention_parity_paired_rows_kernel(cuda_device, case, monkeypatch):
+    # the 64-key rows kernel (two CTAs per SM) instead of the default 128-key one
+    monkeypatch.setenv("TSD_ATTN_ROWS_VARIANT", "2")
+    test_paged_attention_parity(cuda_device, case)
+
+
+@pytest.mark.parametrize("case", CASES[2:4], ids=[f"s{c[0]}_p{c[7]}" for c in CASES[2:4]])
+def test_paged_attention_parity_small_on_keysplit_kernel(cuda_device, case, monkeypatch):
+    monkeypatch.setenv("TSD_ATTN_SMALL_VARIANT", "keysplit")
+    test_paged_attention_parity(cuda_device, case)
 
 
 @pytest.mark.parametrize("D,dtype", [(128, "bf16"), (64, "f32")])

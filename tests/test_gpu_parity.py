@@ -92,6 +92,27 @@ def test_attention_parity(cuda_device, case):
     assert _status(cuda_device) == 0
 
 
+# cases with more than 128 packed rows, on the 64-key rows kernel (two CTAs
+# per SM) instead of the default 128-key one (one CTA per SM)
+ROWS_CASES = [c for c in ATTN_CASES if c[7] == "bf16" and c[5] == 128 and c[2] * c[3] // c[4] > 128]
+
+
+@pytest.mark.parametrize("case", ROWS_CASES, ids=[f"s{c[0]}" for c in ROWS_CASES])
+def test_attention_parity_paired_rows_kernel(cuda_device, case, monkeypatch):
+    monkeypatch.setenv("TSD_ATTN_ROWS_VARIANT", "2")
+    test_attention_parity(cuda_device, case)
+
+
+SMALL_CASES = [c for c in ATTN_CASES if c[7] == "bf16" and c[5] == 128 and c[2] * c[3] // c[4] <= 128]
+
+
+@pytest.mark.parametrize("case", SMALL_CASES, ids=[f"s{c[0]}" for c in SMALL_CASES])
+def test_attention_parity_small_on_keysplit_kernel(cuda_device, case, monkeypatch):
+    # at most 128 packed rows, on the key-split kernel instead of the 64-key rows one
+    monkeypatch.setenv("TSD_ATTN_SMALL_VARIANT", "keysplit")
+    test_attention_parity(cuda_device, case)
+
+
 def test_attention_empty_trees_and_prefix(cuda_device):
     # T_b = 0 sequences, P_b = 0 sequences, and a single-node tree with no prefix
     w = gen.random_workload(21, B=4, Tmax=8, Hq=4, Hkv=2, D=128, P_max=50, dtype="bf16",

@@ -24,16 +24,19 @@
 // never leaks.  One mbarrier arrival per softmax warp (not per thread).
 //
 // Two kernels share this machinery:
-//   * tree_attn_rows_kernel (packed blocks of more than 128 rows): one CTA per
-//     (128-row block, (b, KV head), KV split); 6 warps -- TMA producer, MMA
-//     issuer, 4 softmax warps; TMEM holds three S buffers (the scores of the
-//     next two key tiles are ready while the softmax works) and O.
-//   * tree_attn_keysplit_kernel (at most 128 rows, e.g. MHA with small
-//     trees, where the KV stream is the bound): one CTA per ((b, KV head),
-//     split); two 4-warp softmax groups take the even and odd key tiles of
-//     the same query tile, each with its own S and O in TMEM, and their
-//     (O, m, l) are merged by log-sum-exp at the end -- twice the softmax
-//     throughput per KV byte.
+//   * tree_attn_rows_kernel: one CTA per (128-row block, (b, KV head), KV
+//     split); 6 warps -- TMA producer, MMA issuer, 4 softmax warps; TMEM
+//     holds NS score buffers (the scores of the next key tiles are ready
+//     while the softmax works) and O.  Two instances: 128-key tiles with
+//     three S buffers at one CTA per SM (more than 128 packed rows), and
+//     64-key tiles with two S buffers at two CTAs per SM (at most 128 packed
+//     rows, where the KV stream is the bound: two co-resident CTAs keep
+//     twice the loads in flight and hide each other's prologue and tail).
+//   * tree_attn_keysplit_kernel (at most 128 rows; selected with
+//     TSD_ATTN_SMALL_VARIANT=keysplit): one CTA per ((b, KV head), split);
+//     two 4-warp softmax groups take the even and odd key tiles of the same
+//     query tile, each with its own S and O in TMEM, and their (O, m, l) are
+//     merged by log-sum-exp at the end.
 // K and V stream through separate TMA rings (128-byte swizzle).  Every
 // mbarrier wait is bounded: after ~2 s it raises a CTA-wide abort flag, the
 // CTA reports TSD_DEV_TIMEOUT, unwinds, frees its TMEM and exits.
@@ -41,6 +44,8 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "sm100_ptx.cuh"
@@ -56,31 +61,47 @@ int launch_combine(int dtype, int D, const float *part_o, const float2 *part_ml,
 namespace {
 
 constexpr int BQ = 128;        // query rows per tile
-constexpr int BN = 128;        // keys per tile
 constexpr int HD = 128;        // head dim
-constexpr int NSK = 3;         // K ring stages
-constexpr int NSV = 2;         // V ring stages
-constexpr uint32_t kSub = BN * 128;          // [128 rows][64 bf16] sub-tile, 16 KB
-constexpr uint32_t kTile = 2 * kSub;         // [128][128] bf16, 32 KB
+constexpr uint32_t kSubQ = BQ * 128;         // Q [128 rows][64 bf16] sub-tile, 16 KB
+constexpr uint32_t kTileQ = 2 * kSubQ;       // Q tile [128][128] bf16, 32 KB
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kOffQ + kTile;
-constexpr uint32_t kOffV = kOffK + NSK * kTile;
-constexpr uint32_t kOffBar = kOffV + NSV * kTile;
-constexpr int kNumBars = 1 + 2 * NSK + 2 * NSV + 12;
-constexpr uint32_t kOffMisc = kOffBar + 8 * kNumBars;
-constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;   // + alignment slack
-constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 constexpr float kLazyLimit = 18446744073709551616.0f;   // 2^64: headroom of a P tile sum
-static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+// Tile geometry of a kernel: keys per tile, K and V ring stages, TMEM
+// columns; shared memory holds Q, the K ring, the V ring, the mbarriers.
+template <int BN_, int NSK_, int NSV_, uint32_t TMEM_COLS>
+struct Geo {
+    static constexpr int BN = BN_;                       // keys per tile
+    static constexpr int NSK = NSK_;                     // K ring stages
+    static constexpr int NSV = NSV_;                     // V ring stages
+    static constexpr uint32_t kSub = BN * 128;           // [BN rows][64 bf16] sub-tile
+    static constexpr uint32_t kTile = 2 * kSub;          // [BN][128] bf16
+    static constexpr uint32_t kOffK = kOffQ + kTileQ;
+    static constexpr uint32_t kOffV = kOffK + NSK * kTile;
+    static constexpr uint32_t kOffBar = kOffV + NSV * kTile;
+    static constexpr int kNumBars = 1 + 2 * NSK + 2 * NSV + 12;
+    static constexpr uint32_t kOffMisc = kOffBar + 8 * kNumBars;
+    static constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;   // + alignment slack
+    static constexpr uint32_t kTmemCols = TMEM_COLS;
+};
+// 128-key tiles, 197 KB of shared memory and all 512 TMEM columns: one CTA
+// per SM (rows and key-split kernels).
+using Wide = Geo<128, 3, 2, 512>;
+// 64-key tiles, 97 KB and 256 columns: two CTAs per SM (paired rows kernel).
+using Half = Geo<64, 2, 2, 256>;
+static_assert(Wide::kSmemBytes <= 232448, "shared memory budget");
+static_assert(2 * (Half::kSmemBytes + 1024) <= 233472, "two CTAs per SM");
 
 constexpr int kRowsThreads = 192;       // rows kernel: 6 warps
 constexpr int kSplitThreads = 384;      // key-split kernel: 12 warps
 
 // mbarrier addresses: q_full, k_full[NSK], k_empty[NSK], v_full[NSV],
 // v_empty[NSV], s_full[4], p_full[4], o_ready[4] -- consecutive 8-byte words.
+template <class Gm>
 struct Bars {
+    static constexpr int NSK = Gm::NSK, NSV = Gm::NSV;
     uint32_t base;
     __device__ uint32_t q_full() const { return base; }
     __device__ uint32_t k_full(int s) const { return base + 8u * (1 + s); }
@@ -110,19 +131,25 @@ __device__ __forceinline__ void warp_arrive(uint32_t bar)
         ptx::mbar_arrive(bar);
 }
 
-// K-major, 128-byte-swizzled operand made of two [rows][64] sub-tiles: the
-// descriptor for the kk-th 16-wide slice of the 128-wide contraction dim.
-__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int kk)
+// K-major, 128-byte-swizzled operand made of two [rows][64] sub-tiles `sub`
+// bytes apart: the descriptor for the 16-wide slice kk of the 128-wide
+// contraction dim is the base descriptor plus slice_off(kk, sub) (the
+// address field is addr >> 4 and shared addresses stay below 256 KB, so
+// adding to the packed word never carries out of it).
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile)
 {
-    const uint32_t addr = tile + (uint32_t)(kk >> 2) * kSub + (uint32_t)(kk & 3) * 32u;
-    return ptx::smem_desc_sw128(addr, 16u, 1024u);
+    return ptx::smem_desc_sw128(tile, 16u, 1024u);
+}
+__device__ __forceinline__ uint64_t slice_off(int kk, uint32_t sub)
+{
+    return ((uint32_t)(kk >> 2) * sub + (uint32_t)(kk & 3) * 32u) >> 4;
 }
 
-// V tile as the MN-major B operand of O += P V: the kk-th group of 16 keys;
-// the two 64-wide halves of head_dim are kSub bytes apart.
-__device__ __forceinline__ uint64_t desc_v(uint32_t tile, int kk)
+// V tile as the MN-major B operand of O += P V (group kk of 16 keys at
+// + kk * 2 KB); the two 64-wide halves of head_dim are `sub` bytes apart.
+__device__ __forceinline__ uint64_t desc_v(uint32_t tile, uint32_t sub)
 {
-    return ptx::smem_desc_sw128(tile + (uint32_t)kk * 16u * 128u, kSub, 1024u);
+    return ptx::smem_desc_sw128(tile, sub, 1024u);
 }
 
 __device__ __forceinline__ uint32_t mask_word(const uint32_t (&mw)[4], int v)
@@ -154,24 +181,28 @@ __device__ __forceinline__ uint32_t valid_bits(int pos0, int P, int ke, const ui
 
 // Per-CTA set-up shared by both kernels: 1024-byte aligned carve-up of the
 // dynamic shared memory, barrier initialisation, TMEM allocation (warp 1).
+template <class Gm>
 struct Setup {
     uint8_t *gbase;
     uint32_t base, sQ, sK, sV, tmem;
-    Bars bars;
+    Bars<Gm> bars;
     volatile int *abort_flag;
 };
 
-__device__ __forceinline__ Setup cta_setup(uint8_t *smem_raw, uint32_t q_arrivals,
-                                           uint32_t p_arrivals)
+template <class Gm>
+__device__ __forceinline__ Setup<Gm> cta_setup(uint8_t *smem_raw, uint32_t q_arrivals,
+                                               uint32_t p_arrivals)
 {
-    Setup su;
+    constexpr int NSK = Gm::NSK, NSV = Gm::NSV;
+    constexpr uint32_t kOffMisc = Gm::kOffMisc;
+    Setup<Gm> su;
     const uint32_t raw = ptx::smem_addr(smem_raw);
     su.base = (raw + 1023u) & ~1023u;
     su.gbase = smem_raw + (su.base - raw);
     su.sQ = su.base + kOffQ;
-    su.sK = su.base + kOffK;
-    su.sV = su.base + kOffV;
-    su.bars = Bars{su.base + kOffBar};
+    su.sK = su.base + Gm::kOffK;
+    su.sV = su.base + Gm::kOffV;
+    su.bars = Bars<Gm>{su.base + Gm::kOffBar};
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(su.gbase + kOffMisc);
     su.abort_flag = reinterpret_cast<volatile int *>(su.gbase + kOffMisc + 4);
     if (threadIdx.x == 0) {
@@ -194,7 +225,7 @@ __device__ __forceinline__ Setup cta_setup(uint8_t *smem_raw, uint32_t q_arrival
         ptx::fence_proxy_async_smem();
     }
     if ((threadIdx.x >> 5) == 1) {
-        ptx::tmem_alloc(ptx::smem_addr((const void *)tmem_slot), kTmemCols);
+        ptx::tmem_alloc(ptx::smem_addr((const void *)tmem_slot), Gm::kTmemCols);
         ptx::tmem_relinquish();
     }
     ptx::tc_fence_before();
@@ -204,7 +235,8 @@ __device__ __forceinline__ Setup cta_setup(uint8_t *smem_raw, uint32_t q_arrival
     return su;
 }
 
-__device__ __forceinline__ void cta_teardown(const Setup &su, int32_t *dev_status)
+template <class Gm>
+__device__ __forceinline__ void cta_teardown(const Setup<Gm> &su, int32_t *dev_status)
 {
     ptx::tc_fence_before();
     __syncthreads();
@@ -212,17 +244,18 @@ __device__ __forceinline__ void cta_teardown(const Setup &su, int32_t *dev_statu
         flag(dev_status, TSD_DEV_TIMEOUT);
     if ((threadIdx.x >> 5) == 1) {
         ptx::tc_fence_after();
-        ptx::tmem_dealloc(su.tmem, kTmemCols);
+        ptx::tmem_dealloc(su.tmem, Gm::kTmemCols);
     }
 }
 
-// The TMA loads of one [128 keys][128] K or V tile starting at logical key
+// The TMA loads of one [BN keys][128] K or V tile starting at logical key
 // position pos0 into `dst` (two 64-column halves).  Contiguous cache: one box
 // per half at (x, pos0, b * Hkv + hk).  Paged cache: one box per page the
-// tile touches (box rows = min(128, page_size); a box never straddles a page
-// since both are powers of two and pos0 is a multiple of 128) at (x, row in
+// tile touches (box rows = min(BN, page_size); a box never straddles a page
+// since both are powers of two and pos0 is a multiple of BN) at (x, row in
 // page, page * Hkv + hk).  A box that starts at or beyond the sequence's end
 // loads any valid page: those keys are masked and their V rows zeroed.
+template <class Gm>
 __device__ __forceinline__ void load_kv_tile(uint32_t dst, const CUtensorMap *tm, uint32_t bar,
                                              int pos0, int b, int hk, int Hkv,
                                              const KvPages &pages, int seq_end,
@@ -230,11 +263,11 @@ __device__ __forceinline__ void load_kv_tile(uint32_t dst, const CUtensorMap *tm
 {
     if (!pages.table) {
         ptx::tma_load_3d(dst, tm, 0, pos0, b * Hkv + hk, bar);
-        ptx::tma_load_3d(dst + kSub, tm, 64, pos0, b * Hkv + hk, bar);
+        ptx::tma_load_3d(dst + Gm::kSub, tm, 64, pos0, b * Hkv + hk, bar);
         return;
     }
-    const int rows = min(BN, pages.page_size);
-    for (int r0 = 0; r0 < BN; r0 += rows) {
+    const int rows = min(Gm::BN, pages.page_size);
+    for (int r0 = 0; r0 < Gm::BN; r0 += rows) {
         const int pos = pos0 + r0;
         int z = hk, y = 0;
         if (pos < seq_end) {
@@ -246,17 +279,20 @@ __device__ __forceinline__ void load_kv_tile(uint32_t dst, const CUtensorMap *tm
             y = pos & (pages.page_size - 1);
         }
         ptx::tma_load_3d(dst + r0 * 128, tm, 0, y, z, bar);
-        ptx::tma_load_3d(dst + kSub + r0 * 128, tm, 64, y, z, bar);
+        ptx::tma_load_3d(dst + Gm::kSub + r0 * 128, tm, 64, y, z, bar);
     }
 }
 
 // TMA producer (one lane): K_0, K_1, V_0, K_2, V_1, ... -- the order in which
 // the MMA warp first needs them.
-__device__ __forceinline__ void produce_kv(const Setup &su, const CUtensorMap *tmK,
+template <class Gm>
+__device__ __forceinline__ void produce_kv(const Setup<Gm> &su, const CUtensorMap *tmK,
                                            const CUtensorMap *tmV, int b, int hk, int Hkv,
                                            int kb, int ntiles, const KvPages &pages,
                                            int seq_end, int32_t *dev_status)
 {
+    constexpr int NSK = Gm::NSK, NSV = Gm::NSV, BN = Gm::BN;
+    constexpr uint32_t kTile = Gm::kTile;
     ptx::prefetch_tmap(tmK);
     ptx::prefetch_tmap(tmV);
     for (int i = 0; i <= ntiles; ++i) {
@@ -266,7 +302,7 @@ __device__ __forceinline__ void produce_kv(const Setup &su, const CUtensorMap *t
                 !ptx::mbar_wait(su.bars.k_empty(s), ((i / NSK) - 1) & 1, su.abort_flag))
                 break;
             ptx::mbar_arrive_expect_tx(su.bars.k_full(s), kTile);
-            load_kv_tile(su.sK + s * kTile, tmK, su.bars.k_full(s), kb + i * BN, b, hk, Hkv,
+            load_kv_tile<Gm>(su.sK + s * kTile, tmK, su.bars.k_full(s), kb + i * BN, b, hk, Hkv,
                          pages, seq_end, dev_status);
         }
         if (i >= 1) {
@@ -275,28 +311,25 @@ __device__ __forceinline__ void produce_kv(const Setup &su, const CUtensorMap *t
                 !ptx::mbar_wait(su.bars.v_empty(s), ((j / NSV) - 1) & 1, su.abort_flag))
                 break;
             ptx::mbar_arrive_expect_tx(su.bars.v_full(s), kTile);
-            load_kv_tile(su.sV + s * kTile, tmV, su.bars.v_full(s), kb + j * BN, b, hk, Hkv,
+            load_kv_tile<Gm>(su.sV + s * kTile, tmV, su.bars.v_full(s), kb + j * BN, b, hk, Hkv,
                          pages, seq_end, dev_status);
         }
     }
 }
 
 // MMA warp, S = Q K^T for key tile `t` into TMEM columns `col_s`.
-__device__ __forceinline__ void issue_qk(const Setup &su, int lane, uint32_t col_s, int t,
+template <class Gm>
+__device__ __forceinline__ void issue_qk(const Setup<Gm> &su, int lane, uint32_t col_s, int t,
                                          uint32_t s_full)
 {
-    constexpr uint32_t idesc = ptx::idesc_bf16(BQ, BN, false, false);
-    const int st = t % NSK;
+    constexpr uint32_t idesc = ptx::idesc_bf16(BQ, Gm::BN, false, false);
+    const int st = t % Gm::NSK;
     if (lane == 0) {
-        // base descriptors once; the k-slices are constant offsets (the
-        // address field is addr >> 4 and shared addresses stay below 256 KB,
-        // so adding to the packed word never carries out of it)
-        const uint64_t dq = desc_kmajor(su.sQ, 0), dk = desc_kmajor(su.sK + st * kTile, 0);
+        const uint64_t dq = desc_kmajor(su.sQ), dk = desc_kmajor(su.sK + st * Gm::kTile);
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-            const uint64_t off = ((uint32_t)(kk >> 2) * kSub + (uint32_t)(kk & 3) * 32u) >> 4;
-            ptx::mma_ss(su.tmem + col_s, dq + off, dk + off, idesc, kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < HD / 16; ++kk)
+            ptx::mma_ss(su.tmem + col_s, dq + slice_off(kk, kSubQ), dk + slice_off(kk, Gm::kSub),
+                        idesc, kk > 0 ? 1u : 0u);
         ptx::mma_commit(s_full);
         ptx::mma_commit(su.bars.k_empty(st));
     }
@@ -304,26 +337,29 @@ __device__ __forceinline__ void issue_qk(const Setup &su, int lane, uint32_t col
 }
 
 // MMA warp, O += P V for key tile `t` (P in TMEM columns col_p); zeroes the
-// V rows at or beyond P_b + T_b first.  Returns false on abort.
-__device__ __forceinline__ void issue_pv(const Setup &su, int lane, uint32_t col_p,
+// V rows at or beyond P_b + T_b first.
+template <class Gm>
+__device__ __forceinline__ void issue_pv(const Setup<Gm> &su, int lane, uint32_t col_p,
                                          uint32_t col_o, int t, bool accumulate, int first_bad,
                                          uint32_t o_ready)
 {
+    constexpr int BN = Gm::BN;
     constexpr uint32_t idesc = ptx::idesc_bf16(BQ, HD, false, true);
-    const int vs = t % NSV;
+    const int vs = t % Gm::NSV;
     if (first_bad < BN) {
-        uint8_t *vt = su.gbase + kOffV + vs * kTile;
+        uint8_t *vt = su.gbase + Gm::kOffV + vs * Gm::kTile;
         for (int row = max(first_bad, 0) + (lane >> 3); row < BN; row += 4) {
             const int c = lane & 7;
             *reinterpret_cast<uint4 *>(vt + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4 *>(vt + kSub + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4 *>(vt + Gm::kSub + row * 128 + c * 16) =
+                make_uint4(0, 0, 0, 0);
         }
         ptx::fence_proxy_async_smem();
         __syncwarp();
     }
     ptx::tc_fence_after();
     if (lane == 0) {
-        const uint64_t dv = desc_v(su.sV + vs * kTile, 0);
+        const uint64_t dv = desc_v(su.sV + vs * Gm::kTile, Gm::kSub);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
             ptx::mma_ts(su.tmem + col_o, su.tmem + col_p + kk * 8,
@@ -343,7 +379,8 @@ struct RowCtx {
 };
 
 // Q row `t` of the tile -> shared memory, 128-byte swizzled K-major layout.
-__device__ __forceinline__ void load_q_row(const Setup &su, const __nv_bfloat16 *__restrict__ q,
+template <class Gm>
+__device__ __forceinline__ void load_q_row(const Setup<Gm> &su, const __nv_bfloat16 *__restrict__ q,
                                            bool row_ok, size_t q_off, int t)
 {
     uint8_t *dst = su.gbase + kOffQ;
@@ -352,7 +389,7 @@ __device__ __forceinline__ void load_q_row(const Setup &su, const __nv_bfloat16 
     for (int c = 0; c < 16; ++c) {
         const uint4 x = row_ok ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
         const int sub = c >> 3, cc = c & 7;
-        *reinterpret_cast<uint4 *>(dst + sub * kSub + t * 128 + ((cc ^ (t & 7)) * 16)) = x;
+        *reinterpret_cast<uint4 *>(dst + sub * kSubQ + t * 128 + ((cc ^ (t & 7)) * 16)) = x;
     }
     ptx::fence_proxy_async_smem();
 }
@@ -449,7 +486,7 @@ __device__ __forceinline__ bool softmax_tile(uint32_t taddr_s, uint32_t taddr_o,
                                              const RowCtx &rc, bool first, float &m_run,
                                              float &l_run, WaitO wait_o)
 {
-    const bool masked = !(pos0 + BN <= min(rc.P, rc.ke));
+    const bool masked = !(pos0 + Wide::BN <= min(rc.P, rc.ke));
     // max over the raw scores (scale > 0 is applied once), two chunks at a time
     float mx[16];
 #pragma unroll
@@ -543,15 +580,25 @@ __device__ __forceinline__ void write_row(uint32_t taddr_o, float inv, bool row_
 
 // ============================================================ rows kernel
 // More than 128 packed rows: one 128-row query tile per CTA, 6 warps (TMA
-// producer, MMA issuer, 4 softmax warps).  Three S buffers: the MMA warp
-// keeps the scores of the next two key tiles ready while the softmax works
-// on tile j, so the softmax never waits on the PV -> QK chain.
-// TMEM: S0 [0,128) | S1 [128,256) | S2 [256,384) | O [384,512).
-// MMA order: QK_0 QK_1 QK_2, then per tile j: PV_j QK_{j+3}; P_j is read out
-// of S_{j%3} by PV_j before QK_{j+3}, issued after it by the same thread,
-// overwrites it.  PV_j commits to o_ready[j%3], so a wait for "PV_{j-1}
-// done" names a phase that can be neither stale nor ahead.
-__global__ void __launch_bounds__(kRowsThreads, 1)
+// producer, MMA issuer, 4 softmax warps).  NS score buffers of BN columns
+// each, then O: the MMA warp keeps the scores of the next NS - 1 key tiles
+// ready while the softmax works on tile j.  Two instances:
+//   * 128-key tiles, NS = 3, one CTA per SM:
+//         TMEM S0 [0,128) | S1 [128,256) | S2 [256,384) | O [384,512)
+//   * 64-key tiles, NS = 2, two CTAs per SM (each with 256 TMEM columns and
+//     97 KB of shared memory): S0 [0,64) | S1 [64,128) | O [128,256).  The
+//     two CTAs' MMA warps feed one tensor pipe and their softmax warps share
+//     the sub-partitions, so one CTA's barrier waits and exp latency are
+//     covered by the other's work.
+// MMA order: QK_0 .. QK_{NS-1}, then per tile j: PV_j QK_{j+NS}; P_j is read
+// out of S_{j%NS} by PV_j before QK_{j+NS}, issued after it by the same
+// thread, overwrites it.  PV_j commits to o_ready[j%NS].  The softmax at tile
+// j waits for "PV_{j-1} done" on o_ready[(j-1)%NS]: the phase before it
+// there is PV_{j-1-NS}, issued before QK_j, whose completion the softmax has
+// already seen, and the phase after it needs P_{j-1+NS}, not yet written --
+// so the wait names a phase that can be neither stale nor ahead.
+template <class Gm, int NS, int kMinBlocks>
+__global__ void __launch_bounds__(kRowsThreads, kMinBlocks)
     tree_attn_rows_kernel(const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV,
                           const __nv_bfloat16 *__restrict__ q,
@@ -577,12 +624,14 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
     const int ke = min(kb + keys_per_split, P + T);
     if (rb * BQ >= R || kb >= ke)
         return;   // no rows or no keys: the partials stay empty
+    constexpr int BN = Gm::BN, NSK = Gm::NSK, NSV = Gm::NSV;
+    constexpr int NC = BN / 32;   // 32-column score chunks per tile
+    static_assert(NS * BN + HD <= (int)Gm::kTmemCols && NC % 2 == 0, "TMEM layout");
     const int ntiles = (ke - kb + BN - 1) / BN;
-    const Setup su = cta_setup(smem_raw, 4, 4);   // arrivals: softmax warps
+    const Setup<Gm> su = cta_setup<Gm>(smem_raw, 4, 4);   // arrivals: softmax warps
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr int NS = 3;   // S buffers
-    auto col_s = [](int i) { return (uint32_t)(i % NS) * 128u; };
-    constexpr uint32_t kO = 384u;
+    auto col_s = [](int i) { return (uint32_t)(i % NS) * (uint32_t)BN; };
+    constexpr uint32_t kO = NS * BN;
 
     if (warp == 0) {
         if (lane == 0)
@@ -626,7 +675,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
         for (int w = 0; w < 4; ++w)
             mw[w] = (row_ok && w < W) ? mask[((size_t)b * Tmax + u) * W + w] : 0u;
         const uint32_t taddr_o = su.tmem + lane_off + kO;
-        // PV_i done (o_ready[i % 3] completes once per tile of that class)
+        // PV_i done (o_ready[i % NS] completes once per tile of that class)
         auto wait_pv = [&](int i) {
             return warp_wait(su.bars.o_ready(i % NS), (i / NS) & 1, su.abort_flag);
         };
@@ -638,17 +687,17 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
                 break;
             }
             ptx::tc_fence_after();
-            // all 128 scores of the row in registers at once
+            // all BN scores of the row in registers at once
             const uint32_t taddr_s = su.tmem + lane_off + col_s(j);
-            uint32_t sr[4][32];
+            uint32_t sr[NC][32];
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
+            for (int c = 0; c < NC; ++c)
                 ptx::tmem_ld32(taddr_s + c * 32, sr[c]);
             ptx::tmem_wait_ld();
             const int pos0 = kb + j * BN;
             if (!(pos0 + BN <= min(P, ke))) {   // only where the tree or the range end is
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
+                for (int c = 0; c < NC; ++c)
                     mask32(sr[c], valid_bits(pos0 + c * 32, P, ke, mw));
             }
             // P against the running max, written speculatively; the row max
@@ -662,7 +711,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
                 const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
                 lsum = 0.f;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < NC; ++c) {
                     uint32_t pk[16];
                     lsum += exp_pack32(sr[c], scale_log2, neg_m, pk);
                     ptx::tmem_st16(taddr_s + c * 16, pk);
@@ -674,8 +723,9 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
                     mx[i] = -INFINITY;
-                max32x2(sr[0], sr[1], mx);
-                max32x2(sr[2], sr[3], mx);
+#pragma unroll
+                for (int c = 0; c < NC; c += 2)
+                    max32x2(sr[c], sr[c + 1], mx);
                 const float mt = max16(mx) * scale_log2;
                 const bool need = mt > m_run + kRescaleThreshold;   // false if mt is -inf
                 const float m_new = need ? mt : m_run;
@@ -746,8 +796,10 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
     const int ke = min(kb + keys_per_split, P + T);
     if (R <= 0 || kb >= ke)
         return;
+    using Gm = Wide;
+    constexpr int BN = Gm::BN, NSK = Gm::NSK, NSV = Gm::NSV;
     const int ntiles = (ke - kb + BN - 1) / BN;
-    const Setup su = cta_setup(smem_raw, 8, 4);   // arrivals: softmax warps
+    const Setup<Gm> su = cta_setup<Gm>(smem_raw, 8, 4);   // arrivals: softmax warps
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     auto col_s = [](int s) { return (uint32_t)s * 128u; };
     auto col_o = [](int s) { return 256u + (uint32_t)s * 128u; };
@@ -878,33 +930,66 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
 // ------------------------------------------------------------------ host
 struct UmmaPlan {
     bool keysplit;   // at most 128 packed rows
+    bool paired;     // rows kernel with 64-key tiles, two CTAs per SM
     int nrb, nsplit, keys_per_split;
 };
 
+// Rows-kernel instance: 1 = 128-key tiles at one CTA per SM (default),
+// 2 = 64-key tiles at two CTAs per SM when the environment variable
+// TSD_ATTN_ROWS_VARIANT is "2" (read at every launch, so that one process
+// can run and compare both).
+int rows_variant()
+{
+    const char *e = std::getenv("TSD_ATTN_ROWS_VARIANT");
+    return (e && e[0] == '2' && e[1] == '\0') ? 2 : 1;
+}
+
+// At most 128 packed rows: the paired 64-key rows kernel (default), or the
+// key-split kernel when TSD_ATTN_SMALL_VARIANT is "keysplit".
+bool small_paired()
+{
+    const char *e = std::getenv("TSD_ATTN_SMALL_VARIANT");
+    return !(e && std::strcmp(e, "keysplit") == 0);
+}
+
+// Kernel choice and grid.  More than 128 packed rows go to the rows kernel:
+// 64-key tiles at two CTAs per SM, or 128-key tiles at one.  Splits of the
+// key range balance the grid over the CTA slots.
 UmmaPlan umma_plan(const AttnArgs &a, int num_sms)
 {
     UmmaPlan p;
     const int G = a.Hq / a.Hkv;
-    p.keysplit = a.Tmax * G <= BQ;
+    const bool small = a.Tmax * G <= BQ;
+    p.keysplit = small && !small_paired();
+    p.paired = small ? !p.keysplit : rows_variant() == 2;
     p.nrb = p.keysplit ? 1 : (a.Tmax * G + BQ - 1) / BQ;
+    const int bn = p.paired ? Half::BN : Wide::BN;
+    const int slots = num_sms * (p.paired ? 2 : 1);
     const long base = (long)p.nrb * a.B * a.Hkv;
-    const int tiles = (a.Lmax + BN - 1) / BN;
-    // waves x (tiles per CTA + fixed cost): the fewest splits that balance
-    // the grid over the SMs.
+    const int tiles = (a.Lmax + bn - 1) / bn;
+    // Cost of ns splits in tile times.  One CTA per SM: waves x (tiles per
+    // CTA + fixed cost).  Two per SM: the scheduler refills a slot as soon as
+    // a CTA ends and a CTA alone on an SM runs faster, so the wave count is
+    // taken fractionally (but at least one CTA length), and a split pays for
+    // its fp32 partials and the combine pass.
+    const int fixed = 256 / bn;
     int best = 1;
     double best_cost = 1e30;
     for (int ns = 1; ns <= 64 && ns <= tiles; ++ns) {
         const long units = base * ns;
-        const long waves = (units + num_sms - 1) / num_sms;
         const int per = (tiles + ns - 1) / ns;
-        const double cost = (double)waves * (per + 2);
+        double cost;
+        if (p.paired)
+            cost = std::max((double)units / slots, 1.0) * (per + fixed) + (ns > 1 ? fixed : 0);
+        else
+            cost = (double)((units + slots - 1) / slots) * (per + fixed);
         if (cost < best_cost - 1e-9) {
             best_cost = cost;
             best = ns;
         }
     }
     p.nsplit = best;
-    p.keys_per_split = ((tiles + best - 1) / best) * BN;
+    p.keys_per_split = ((tiles + best - 1) / best) * bn;
     return p;
 }
 
@@ -948,13 +1033,21 @@ cudaError_t set_smem_attributes()
     static std::once_flag once;
     static cudaError_t err = cudaSuccess;
     std::call_once(once, [] {
-        err = cudaFuncSetAttribute(tree_attn_rows_kernel,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+        auto wide = tree_attn_rows_kernel<Wide, 3, 1>;
+        auto half = tree_attn_rows_kernel<Half, 2, 2>;
+        err = cudaFuncSetAttribute(wide, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)Wide::kSmemBytes);
         if (err == cudaSuccess)
             err = cudaFuncSetAttribute(tree_attn_keysplit_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)kSmemBytes);
-
+                                       (int)Wide::kSmemBytes);
+        if (err == cudaSuccess)
+            err = cudaFuncSetAttribute(half, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)Half::kSmemBytes);
+        // two CTAs per SM need the largest shared-memory carve-out
+        if (err == cudaSuccess)
+            err = cudaFuncSetAttribute(half, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                       (int)cudaSharedmemCarveoutMaxShared);
     });
     return err;
 }
@@ -988,7 +1081,8 @@ int launch_umma_attention(const AttnArgs &a, void *ws, size_t ws_bytes, int num_
     const bool paged = a.pages.table != nullptr;
     const int rows = paged ? a.pages.page_size : a.Lmax;
     const int planes = paged ? a.pages.num_pages * a.Hkv : a.B * a.Hkv;
-    const int box_rows = paged ? std::min(BN, a.pages.page_size) : BN;
+    const int bn = p.paired ? Half::BN : Wide::BN;
+    const int box_rows = paged ? std::min(bn, a.pages.page_size) : bn;
     if (!make_kv_map(&tmK, a.k, rows, planes, box_rows) ||
         !make_kv_map(&tmV, a.v, rows, planes, box_rows))
         return TSD_ERR_CUDA;
@@ -1008,12 +1102,17 @@ int launch_umma_attention(const AttnArgs &a, void *ws, size_t ws_bytes, int num_
     const float sl2 = a.scale * kLog2e;
     const int W = (a.Tmax + 31) / 32;
     if (p.keysplit)
-        tree_attn_keysplit_kernel<<<grid, kSplitThreads, kSmemBytes, stream>>>(
+        tree_attn_keysplit_kernel<<<grid, kSplitThreads, Wide::kSmemBytes, stream>>>(
+            tmK, tmV, static_cast<const __nv_bfloat16 *>(a.q), a.prefix_len, a.n_nodes, a.mask,
+            a.Tmax, a.Hq, a.Hkv, a.Lmax, W, sl2, p.keys_per_split, p.nsplit,
+            static_cast<__nv_bfloat16 *>(a.out), part_o, part_ml, a.dev_status, a.pages);
+    else if (p.paired)
+        tree_attn_rows_kernel<Half, 2, 2><<<grid, kRowsThreads, Half::kSmemBytes, stream>>>(
             tmK, tmV, static_cast<const __nv_bfloat16 *>(a.q), a.prefix_len, a.n_nodes, a.mask,
             a.Tmax, a.Hq, a.Hkv, a.Lmax, W, sl2, p.keys_per_split, p.nsplit,
             static_cast<__nv_bfloat16 *>(a.out), part_o, part_ml, a.dev_status, a.pages);
     else
-        tree_attn_rows_kernel<<<grid, kRowsThreads, kSmemBytes, stream>>>(
+        tree_attn_rows_kernel<Wide, 3, 1><<<grid, kRowsThreads, Wide::kSmemBytes, stream>>>(
             tmK, tmV, static_cast<const __nv_bfloat16 *>(a.q), a.prefix_len, a.n_nodes, a.mask,
             a.Tmax, a.Hq, a.Hkv, a.Lmax, W, sl2, p.keys_per_split, p.nsplit,
             static_cast<__nv_bfloat16 *>(a.out), part_o, part_ml, a.dev_status, a.pages);
