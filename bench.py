@@ -132,15 +132,53 @@ class Step:
                                   dtype=torch.uint8, device=dev)
         self.ev = None
 
+    def run_mask(self):
+        d = self.d
+        self.tsd.tree_mask_build(d["parent"], d["n_nodes"], out=self.tree)
+
+    def run_attention(self):
+        d = self.d
+        self.tsd.tree_attention(d["q"], d["k_cache"], d["v_cache"], d["prefix_len"],
+                                d["n_nodes"], self.tree.mask, out=self.out,
+                                workspace=self.ws_attn)
+
     def run(self, attn_events=None):
-        w, d, tsd = self.w, self.d, self.tsd
-        tsd.tree_mask_build(d["parent"], d["n_nodes"], out=self.tree)
+        self.run_mask()
         if attn_events is not None:
             attn_events[0].record()
-        tsd.tree_attention(d["q"], d["k_cache"], d["v_cache"], d["prefix_len"], d["n_nodes"],
-                           self.tree.mask, out=self.out, workspace=self.ws_attn)
+        self.run_attention()
         if attn_events is not None:
             attn_events[1].record()
+        self.run_verify()
+
+    def capture(self):
+        """CUDA graphs of the mask build and of the attention call (plain
+        kernel launches), so that the timed steps measure device work and not
+        the Python and launch overhead in front of each call (which exceeds
+        the kernels' own time on the small workloads).  The verify calls stay
+        eager.  Returns the kernel launches one replay of both graphs makes."""
+        torch.cuda.synchronize(self.dev)
+        n0 = self.tsd.launch_count()
+        self.g_mask, self.g_attn = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.g_mask):
+            self.run_mask()
+        with torch.cuda.graph(self.g_attn):
+            self.run_attention()
+        torch.cuda.synchronize(self.dev)
+        return self.tsd.launch_count() - n0
+
+    def run_graphed(self, attn_events):
+        self.g_mask.replay()
+        attn_events[0].record()
+        self.g_attn.replay()
+        attn_events[1].record()
+        self.run_verify()
+
+    def release(self):
+        self.g_mask = self.g_attn = None
+
+    def run_verify(self):
+        w, d, tsd = self.w, self.d, self.tsd
         if "greedy" in w.verify:
             tsd.tree_verify_greedy(d["logits"], d["tokens"], d["parent"], d["n_nodes"],
                                    self.tree, out=self.g, workspace=self.ws_ver)
@@ -318,6 +356,10 @@ def main():
     if working < 3 * L2_BYTES:
         flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
 
+    graph_launches = step.capture()
+    for _ in range(2):
+        step.run_graphed((torch.cuda.Event(), torch.cuda.Event()))
+    torch.cuda.synchronize(dev)
     n_att = args.steps
     att_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(n_att)]
@@ -333,10 +375,11 @@ def main():
         if flush is not None:
             flush.fill_(float(i))
         st_ev[i][0].record()
-        step.run(att_ev[i])
+        step.run_graphed(att_ev[i])
         st_ev[i][1].record()
     torch.cuda.synchronize(dev)
-    launches = tsd.launch_count() - launches0
+    launches = tsd.launch_count() - launches0 + graph_launches * args.steps
+    step.release()
     if pg:
         pg.barrier()
     clk = _clock_summary(clocks)

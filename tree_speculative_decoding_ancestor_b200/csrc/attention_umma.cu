@@ -538,6 +538,73 @@ __device__ __forceinline__ bool softmax_tile(uint32_t taddr_s, uint32_t taddr_o,
     return true;
 }
 
+// One key tile of the online softmax of the rows kernels, for this thread's
+// query row: the BN scores in TMEM columns taddr_s are read into registers
+// at once and masked where the tile reaches the tree or the range end.  P is
+// written against the running max speculatively; the row max is only taken
+// (and O rescaled) when some exponent may exceed the headroom -- the tile's
+// sum above 2^64 or not finite, which always happens on a query tile's first
+// key tile (m_run = -inf).  One exp loop, run a second time only by a warp
+// that took the max.  `wait_prev` waits for the previous PV product before
+// O is rescaled.  Returns false on abort.
+template <int BN, typename WaitPrev>
+__device__ __forceinline__ bool softmax_rows_tile(uint32_t taddr_s, uint32_t taddr_o, int pos0,
+                                                  int P, int ke, const uint32_t (&mw)[4],
+                                                  float scale_log2, bool first, float &m_run,
+                                                  float &l_run, WaitPrev wait_prev)
+{
+    constexpr int NC = BN / 32;   // 32-column score chunks
+    uint32_t sr[NC][32];
+#pragma unroll
+    for (int c = 0; c < NC; ++c)
+        ptx::tmem_ld32(taddr_s + c * 32, sr[c]);
+    ptx::tmem_wait_ld();
+    if (!(pos0 + BN <= min(P, ke))) {   // only where the tree or the range end is
+#pragma unroll
+        for (int c = 0; c < NC; ++c)
+            mask32(sr[c], valid_bits(pos0 + c * 32, P, ke, mw));
+    }
+    float lsum = 0.f;
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+        const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
+        lsum = 0.f;
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+            uint32_t pk[16];
+            lsum += exp_pack32(sr[c], scale_log2, neg_m, pk);
+            ptx::tmem_st16(taddr_s + c * 16, pk);
+        }
+        const bool redo = !(lsum <= kLazyLimit) || m_run == -INFINITY;
+        if (pass == 1 || !__any_sync(0xffffffffu, redo))
+            break;
+        float mx[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            mx[i] = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < NC; c += 2)
+            max32x2(sr[c], sr[c + 1], mx);
+        const float mt = max16(mx) * scale_log2;
+        const bool need = mt > m_run + kRescaleThreshold;   // false if mt is -inf
+        const float m_new = need ? mt : m_run;
+        const float alpha = need ? ptx::ex2(m_run - m_new) : 1.f;   // 0 when m_run = -inf
+        if (__any_sync(0xffffffffu, need) && !first) {
+            // O holds the products of the earlier key tiles: wait for the last.
+            if (!wait_prev())
+                return false;
+            ptx::tc_fence_after();
+            rescale_o(taddr_o, alpha);
+        }
+        l_run *= alpha;
+        m_run = m_new;
+        ptx::tmem_wait_st();   // the speculative P is overwritten next pass
+    }
+    l_run += lsum;
+    ptx::tmem_wait_st();
+    return true;
+}
+
 // Final O row (TMEM) -> output row (bf16, normalised) or split partial (fp32).
 __device__ __forceinline__ void write_row(uint32_t taddr_o, float inv, bool row_ok, size_t row,
                                           int nsplit, int split, size_t nrows,
@@ -625,8 +692,7 @@ __global__ void __launch_bounds__(kRowsThreads, kMinBlocks)
     if (rb * BQ >= R || kb >= ke)
         return;   // no rows or no keys: the partials stay empty
     constexpr int BN = Gm::BN, NSK = Gm::NSK, NSV = Gm::NSV;
-    constexpr int NC = BN / 32;   // 32-column score chunks per tile
-    static_assert(NS * BN + HD <= (int)Gm::kTmemCols && NC % 2 == 0, "TMEM layout");
+    static_assert(NS * BN + HD <= (int)Gm::kTmemCols && BN % 64 == 0, "TMEM layout");
     const int ntiles = (ke - kb + BN - 1) / BN;
     const Setup<Gm> su = cta_setup<Gm>(smem_raw, 4, 4);   // arrivals: softmax warps
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -687,66 +753,11 @@ __global__ void __launch_bounds__(kRowsThreads, kMinBlocks)
                 break;
             }
             ptx::tc_fence_after();
-            // all BN scores of the row in registers at once
-            const uint32_t taddr_s = su.tmem + lane_off + col_s(j);
-            uint32_t sr[NC][32];
-#pragma unroll
-            for (int c = 0; c < NC; ++c)
-                ptx::tmem_ld32(taddr_s + c * 32, sr[c]);
-            ptx::tmem_wait_ld();
-            const int pos0 = kb + j * BN;
-            if (!(pos0 + BN <= min(P, ke))) {   // only where the tree or the range end is
-#pragma unroll
-                for (int c = 0; c < NC; ++c)
-                    mask32(sr[c], valid_bits(pos0 + c * 32, P, ke, mw));
-            }
-            // P against the running max, written speculatively; the row max
-            // is only taken (and O rescaled) when some exponent may exceed
-            // the headroom: the tile's sum above 2^64 (or not finite), which
-            // always happens on the first tile (m_run = -inf).  One exp loop,
-            // run a second time only by a warp that took the max.
-            float lsum = 0.f;
-#pragma unroll 1
-            for (int pass = 0; pass < 2; ++pass) {
-                const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
-                lsum = 0.f;
-#pragma unroll
-                for (int c = 0; c < NC; ++c) {
-                    uint32_t pk[16];
-                    lsum += exp_pack32(sr[c], scale_log2, neg_m, pk);
-                    ptx::tmem_st16(taddr_s + c * 16, pk);
-                }
-                const bool redo = !(lsum <= kLazyLimit) || m_run == -INFINITY;
-                if (pass == 1 || !__any_sync(0xffffffffu, redo))
-                    break;
-                float mx[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    mx[i] = -INFINITY;
-#pragma unroll
-                for (int c = 0; c < NC; c += 2)
-                    max32x2(sr[c], sr[c + 1], mx);
-                const float mt = max16(mx) * scale_log2;
-                const bool need = mt > m_run + kRescaleThreshold;   // false if mt is -inf
-                const float m_new = need ? mt : m_run;
-                const float alpha = need ? ptx::ex2(m_run - m_new) : 1.f;   // 0 when m_run = -inf
-                if (__any_sync(0xffffffffu, need) && j > 0) {
-                    // O holds PV_0 .. PV_{j-1}: wait for the last of them.
-                    if (!wait_pv(j - 1)) {
-                        ok = false;
-                        break;
-                    }
-                    ptx::tc_fence_after();
-                    rescale_o(taddr_o, alpha);
-                }
-                l_run *= alpha;
-                m_run = m_new;
-                ptx::tmem_wait_st();   // the speculative P is overwritten next pass
-            }
+            ok = softmax_rows_tile<BN>(su.tmem + lane_off + col_s(j), taddr_o, kb + j * BN, P, ke,
+                                       mw, scale_log2, j == 0, m_run, l_run,
+                                       [&]() { return wait_pv(j - 1); });
             if (!ok)
                 break;
-            l_run += lsum;
-            ptx::tmem_wait_st();
             ptx::tc_fence_before();
             warp_arrive(su.bars.p_full(j % NS));
         }
@@ -934,10 +945,10 @@ struct UmmaPlan {
     int nrb, nsplit, keys_per_split;
 };
 
-// Rows-kernel instance: 1 = 128-key tiles at one CTA per SM (default),
-// 2 = 64-key tiles at two CTAs per SM when the environment variable
-// TSD_ATTN_ROWS_VARIANT is "2" (read at every launch, so that one process
-// can run and compare both).
+// Rows-kernel instance for more than 128 packed rows: 1 = 128-key tiles at
+// one CTA per SM (default), 2 = 64-key tiles at two CTAs per SM when the
+// environment variable TSD_ATTN_ROWS_VARIANT is "2" (read at every launch,
+// so that one process can run and compare both).
 int rows_variant()
 {
     const char *e = std::getenv("TSD_ATTN_ROWS_VARIANT");
@@ -1044,6 +1055,7 @@ cudaError_t set_smem_attributes()
         if (err == cudaSuccess)
             err = cudaFuncSetAttribute(half, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)Half::kSmemBytes);
+
         // two CTAs per SM need the largest shared-memory carve-out
         if (err == cudaSuccess)
             err = cudaFuncSetAttribute(half, cudaFuncAttributePreferredSharedMemoryCarveout,
