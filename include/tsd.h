@@ -140,6 +140,14 @@ size_t tsd_tree_attention_workspace_size(int B, int Tmax, int Hq, int Hkv, int D
  * out of range), TSD_ERR_DTYPE, TSD_ERR_ALIGN, TSD_ERR_WORKSPACE, TSD_ERR_CUDA.
  * Device: TSD_DEV_BAD_PREFIX (that sequence's rows are not written),
  * TSD_DEV_TIMEOUT.
+ * Kernel choice (results agree within the bf16 tolerance whichever runs):
+ * bf16 with D = 128 and at least 8 packed query rows per KV head (Tmax *
+ * Hq / Hkv) runs on the tensor cores -- 64-key tiles at two CTAs per SM up
+ * to 128 packed rows, 128-key tiles at one CTA per SM above; everything else
+ * on the CUDA cores.  The environment variables TSD_ATTN_ROWS_VARIANT=2
+ * (64-key tiles above 128 rows too) and TSD_ATTN_SMALL_VARIANT=keysplit
+ * (two softmax groups splitting the key tiles, up to 128 rows) select the
+ * alternatives; they are read at every call.
  */
 int tsd_tree_attention(const void *q, const void *k_cache, const void *v_cache,
                        const int32_t *prefix_len, const int32_t *n_nodes, const uint32_t *mask,
