@@ -145,8 +145,9 @@ size_t tsd_tree_attention_workspace_size(int B, int Tmax, int Hq, int Hkv, int D
  * Hq / Hkv) runs on the tensor cores -- 64-key tiles at two CTAs per SM up
  * to 128 packed rows, 128-key tiles at one CTA per SM above; everything else
  * on the CUDA cores.  The environment variables TSD_ATTN_ROWS_VARIANT=2
- * (64-key tiles above 128 rows too) and TSD_ATTN_SMALL_VARIANT=keysplit
- * (two softmax groups splitting the key tiles, up to 128 rows) select the
+ * (64-key tiles above 128 rows too), TSD_ATTN_SMALL_VARIANT=keysplit (two
+ * softmax groups splitting the key tiles, up to 128 rows) and
+ * TSD_FORCE_PATH=simt (the CUDA-core kernel for every shape) select the
  * alternatives; they are read at every call.
  */
 int tsd_tree_attention(const void *q, const void *k_cache, const void *v_cache,

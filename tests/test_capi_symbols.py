@@ -62,3 +62,74 @@ def test_host_only_calls(lib):
     assert lib.tsd_tree_verify_stochastic(None, 0.0, None, 1, None, None, None, None, None,
                                           None, None, 1, 4, 8, None, None, None, None, 0, None,
                                           None) == -2
+
+
+# Host-side argument checks of the other entry points: each call below is
+# refused before any CUDA call, so fake (but aligned) addresses never reach a
+# kernel.  Skipped where a GPU is present: if a check were ever missing, such
+# a call would launch on addresses that are not device memory.
+_A = 0x10000           # a 16-byte aligned stand-in address
+_U = 0x10004           # a misaligned one
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(),
+                    reason="fake addresses must not reach a GPU")
+def test_host_checks_of_every_entry_point(lib):
+    ERR_NULL, ERR_SHAPE, ERR_DTYPE, ERR_ALIGN = -1, -2, -3, -6
+    BF16, F32 = 1, 0
+
+    def attn(q=_A, B=2, Tmax=8, Hq=8, Hkv=2, D=128, Lmax=64, dtype=BF16):
+        return lib.tsd_tree_attention(q, _A, _A, _A, _A, _A, B, Tmax, Hq, Hkv, D, Lmax, 0.1,
+                                      dtype, _A, _A, 1 << 20, _A, None)
+    assert attn(B=0) == 0
+    assert attn(q=None) == ERR_NULL
+    assert attn(Hq=6, Hkv=4) == ERR_SHAPE          # heads not a multiple
+    assert attn(Tmax=129) == ERR_SHAPE             # more tree slots than the mask holds
+    assert attn(Lmax=4) == ERR_SHAPE               # cache shorter than the tree slots
+    assert attn(D=96) == ERR_DTYPE
+    assert attn(dtype=7) == ERR_DTYPE
+    assert attn(q=_U) == ERR_ALIGN
+
+    def paged(table=_A, num_pages=4, page_size=64, max_blocks=4, B=2):
+        return lib.tsd_tree_attention_paged(_A, _A, _A, table, num_pages, page_size, max_blocks,
+                                            _A, _A, _A, B, 8, 8, 2, 128, 0.1, BF16, _A, _A,
+                                            1 << 20, _A, None)
+    for ps in (8, 24, 8192):                        # not a power of two in [16, 4096]
+        assert paged(page_size=ps) == ERR_SHAPE
+    assert paged(max_blocks=0) == ERR_SHAPE
+    assert paged(num_pages=0) == ERR_SHAPE
+    assert paged(table=None) == ERR_NULL
+    assert paged(B=0) == 0
+
+    def commit(k=_A, D=128, dtype=BF16, B=2, path=_A):
+        return lib.tsd_kv_commit(k, _A, _A, path, _A, B, 8, 2, D, 64, dtype, _A, _A, None)
+    assert commit(D=4) == ERR_SHAPE                 # 8-byte rows: not a 16-byte multiple
+    assert commit(D=512) == ERR_SHAPE               # 1 KB rows: beyond the staging limit
+    assert commit(dtype=7) == ERR_DTYPE
+    assert commit(path=None) == ERR_NULL
+    assert commit(k=_U) == ERR_ALIGN
+    assert commit(B=0) == 0
+
+    def expand(k=2, Tmax=8, q=_A, B=2):
+        return lib.tsd_tree_expand(q, 9, 100, _A, k, _A, _A, _A, _A, _A, B, Tmax, _A, None)
+    assert expand(k=0) == ERR_SHAPE
+    assert expand(k=9) == ERR_SHAPE                 # k > Tmax
+    assert expand(q=None) == ERR_NULL
+    assert expand(B=0) == 0
+
+    assert lib.tsd_tree_dfs_order(_A, _A, _A, _A, 2, 129, _A, _A, _A, _A, _A, None) == ERR_SHAPE
+    assert lib.tsd_tree_dfs_order(_A, None, _A, _A, 2, 8, _A, _A, _A, _A, _A, None) == ERR_NULL
+
+    def merge(M=3, L=4, Tmax=16, ct=_A):
+        return lib.tsd_tree_merge_chains(ct, _A, _A, M, L, 2, Tmax, _A, _A, _A, _A, _A, None)
+    assert merge(M=0) == ERR_SHAPE
+    assert merge(L=0) == ERR_SHAPE
+    assert merge(Tmax=200) == ERR_SHAPE
+    assert merge(ct=None) == ERR_NULL
+
+    probe = lib.tsd_debug_wait_probe
+    assert probe(2, 50_000_000, _A, _A, None) == ERR_SHAPE       # unknown kind
+    assert probe(0, 10, _A, _A, None) == ERR_SHAPE               # below 1 ms
+    assert probe(1, 3_000_000_000, _A, _A, None) == ERR_SHAPE    # above 2 s
+    assert probe(0, 50_000_000, None, _A, None) == ERR_NULL
+    assert probe(0, 50_000_000, _U, _A, None) == ERR_ALIGN
