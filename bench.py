@@ -390,6 +390,7 @@ def main():
     value = job_tokens / (ms_per_step / 1e3)
     if int(tsd.device_status(dev).item()) != 0:
         raise RuntimeError("device status set during the timed steps")
+    acceptance = accepted_summary(w, step)
     commit = time_commit(step, dev, tsd)
     paged = time_paged_attention(step, dev, tsd) if w.dtype == "bf16" else None
     build = time_tree_build(w, dev, tsd)
@@ -431,6 +432,7 @@ def main():
                        "parallelism": f"batch-sharded x{ws} (independent sequences)"},
             "kv_cache_gbs": kv_gbs, "kv_cache_frac_of_hbm": kv_gbs / peaks["hbm_gbs"],
             "roofline": roof, "gpu_launches": launches, "clocks": clk,
+            "acceptance": acceptance,
             "kv_commit": commit, "paged_attention": paged, "tree_build": build}
 
     if not args.no_e2e:
@@ -441,6 +443,24 @@ def main():
         print(json.dumps(line), flush=True)
     if pg:
         pg.destroy_process_group()
+
+
+def accepted_summary(w, step) -> dict:
+    """Mean tree nodes accepted per sequence by each verify mode of the
+    workload, and the tokens one verification step emits per sequence (the
+    accepted nodes plus the target's own token).  Read from the last timed
+    step's results; malformed sequences (n_accepted = -1) are left out."""
+    out = {}
+    for mode, res in (("greedy", step.g), ("stochastic", step.s)):
+        if mode not in w.verify:
+            continue
+        n = res.n_accepted.detach().to("cpu", torch.float64)
+        ok = n >= 0
+        if bool(ok.any()):
+            m = float(n[ok].mean())
+            out[mode] = {"mean_accepted_nodes": m, "mean_tokens_per_step": m + 1.0,
+                         "sequences": int(ok.sum())}
+    return out
 
 
 def time_commit(step, dev, tsd, reps: int = 20):

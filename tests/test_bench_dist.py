@@ -86,3 +86,26 @@ def test_ranks_verify_different_sequences():
 
 def test_single_process_passthrough():
     assert bench.reduce_over_ranks(None, torch.device("cpu"), 11, 1.5) == (11, 1.5)
+
+
+def test_accepted_summary_skips_malformed_sequences():
+    from tree_speculative_decoding_ancestor_b200 import VerifyResult
+
+    class _W:
+        verify = ("greedy", "stochastic")
+
+    class _Step:
+        pass
+
+    z = torch.zeros((4, 5), dtype=torch.int32)
+    st = _Step()
+    st.g = VerifyResult(z, z, torch.tensor([3, 0, -1, 1], dtype=torch.int32))
+    st.s = VerifyResult(z, z, torch.tensor([2, 2, 2, 2], dtype=torch.int32))
+    got = bench.accepted_summary(_W(), st)
+    assert got["greedy"] == {"mean_accepted_nodes": 4 / 3, "mean_tokens_per_step": 4 / 3 + 1,
+                             "sequences": 3}
+    assert got["stochastic"]["mean_accepted_nodes"] == 2.0
+    _W.verify = ("stochastic",)
+    assert set(bench.accepted_summary(_W(), st)) == {"stochastic"}
+    st.s = VerifyResult(z, z, torch.full((4,), -1, dtype=torch.int32))
+    assert bench.accepted_summary(_W(), st) == {}
