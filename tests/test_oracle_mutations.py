@@ -89,3 +89,39 @@ def test_unmutated_source_passes_the_same_pins(tmp_path):
         pm.test_mask_vs_subtree_enumeration(4)
         pg.test_greedy_vs_exhaustive_search(0)
         ps.test_exact_enumeration_equals_target(16, 2, 1.0)
+
+
+# The paged-KV gather is Python (numpy) code in the oracle package: plant the
+# mistakes in a copy of its source and route the oracle through the copy.
+import inspect  # noqa: E402
+
+import test_oracle_paged as pp  # noqa: E402
+
+PY_MUTATIONS = {
+    "paged_table_ignored": ("pg = int(bt[b, j])", "pg = j"),
+    "paged_row_offset": ("k[b, :, lo:hi] = kp[pg, :, :hi - lo]",
+                         "k[b, :, lo:hi] = kp[pg, :, ::-1][:, :hi - lo]"),
+    "paged_values_from_keys": ("v[b, :, lo:hi] = vp[pg, :, :hi - lo]",
+                               "v[b, :, lo:hi] = kp[pg, :, :hi - lo]"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTATIONS))
+def test_paged_pin_catches_mutation(name, monkeypatch):
+    old, new = PY_MUTATIONS[name]
+    src = inspect.getsource(oracle.gather_pages)
+    assert src.count(old) == 1, f"mutation anchor not found: {old!r}"
+    ns = {}
+    exec(compile(src.replace(old, new), "<mutated gather_pages>", "exec"), vars(oracle).copy(),
+         ns)
+    monkeypatch.setattr(oracle, "gather_pages", ns["gather_pages"])
+    with pytest.raises(AssertionError):
+        pp.test_paged_equals_contiguous(31, "bf16", 16)
+
+
+def test_unmutated_paged_copy_passes_the_pin(monkeypatch):
+    ns = {}
+    exec(compile(inspect.getsource(oracle.gather_pages), "<copied gather_pages>", "exec"),
+         vars(oracle).copy(), ns)
+    monkeypatch.setattr(oracle, "gather_pages", ns["gather_pages"])
+    pp.test_paged_equals_contiguous(31, "bf16", 16)
