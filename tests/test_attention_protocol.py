@@ -1,0 +1,166 @@
+"""The mbarrier protocol of the tcgen05 rows kernel, on the host (CPU only).
+
+The kernel's three roles meet only at mbarriers:
+- the TMA producer fills a K ring and a V ring;
+- the MMA issuer runs QK_0 .. QK_{NS-1}, then PV_j, QK_{j+NS} for each key
+  tile j, committing each product to barriers;
+- four softmax warps consume the scores, publish P, sometimes wait for the
+  previous PV product (to rescale O), and wait for the last one before
+  writing O.
+
+This test replays exactly that sequence of arrivals and parity waits
+(`csrc/attention_umma.cu`, both tile geometries) under random interleavings
+of the roles, the TMA copies and the in-order tensor pipe. It checks three
+things:
+- no wait is left waiting for ever;
+- every wait that passes sees exactly the phase it names: an mbarrier wait
+  on parity p passes whenever the barrier's completed-phase count has the
+  other parity, so a stale or an early pass would go unnoticed on the GPU;
+- no S buffer is overwritten by a QK product before the PV product that
+  reads its P has run.
+"""
+
+import random
+
+import pytest
+
+
+class _Barrier:
+    def __init__(self, count):
+        self.count, self.pending, self.done = count, 0, 0
+
+    def arrive(self):
+        self.pending += 1
+        if self.pending == self.count:
+            self.pending, self.done = 0, self.done + 1
+
+
+def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready"):
+    rnd = random.Random(seed)
+    bars = {"q_full": _Barrier(4)}
+    for s in range(NSK):
+        bars["k_full", s], bars["k_empty", s] = _Barrier(1), _Barrier(1)
+    for s in range(NSV):
+        bars["v_full", s], bars["v_empty", s] = _Barrier(1), _Barrier(1)
+    for i in range(NS):
+        bars["s_full", i], bars["o_ready", i] = _Barrier(1), _Barrier(1)
+        bars["p_full", i] = _Barrier(4)
+
+    def passes(name, k):
+        """Wait for phase k of `name` (parity k & 1): True once it passes."""
+        b = bars[name]
+        if (b.done & 1) == (k & 1):
+            return False
+        assert b.done == k + 1, f"wait on {name} for phase {k} passed at {b.done} completions"
+        return True
+
+    tma, pipe = [], []
+    s_owner = {}       # S buffer -> tile whose scores/P it holds
+    pv_done = set()
+
+    def producer():
+        for i in range(ntiles + 1):
+            if i < ntiles:
+                s = i % NSK
+                if i >= NSK:
+                    while not passes(("k_empty", s), i // NSK - 1):
+                        yield
+                tma.append(("k_full", s))
+            if i >= 1:
+                j = i - 1
+                s = j % NSV
+                if j >= NSV:
+                    while not passes(("v_empty", s), j // NSV - 1):
+                        yield
+                tma.append(("v_full", s))
+            yield
+
+    def mma():
+        while not passes("q_full", 0):
+            yield
+
+        def qk(i):
+            while not passes(("k_full", i % NSK), i // NSK):
+                yield
+            buf = i % NS
+            prev = s_owner.get(buf)
+            assert prev is None or prev in pv_done or ("pv", prev) in [p[0] for p in pipe], \
+                f"QK_{i} issued over the P of tile {prev} before its PV"
+            pipe.append((("qk", i), [("s_full", buf), ("k_empty", i % NSK)]))
+            s_owner[buf] = i
+        for i in range(min(NS, ntiles)):
+            yield from qk(i)
+        for j in range(ntiles):
+            while not passes(("p_full", j % NS), j // NS):
+                yield
+            while not passes(("v_full", j % NSV), j // NSV):
+                yield
+            pipe.append((("pv", j), [("v_empty", j % NSV), ("o_ready", j % NS)]))
+            if j + NS < ntiles:
+                yield from qk(j + NS)
+            yield
+
+    def softmax():
+        bars["q_full"].arrive()
+        yield
+        for j in range(ntiles):
+            while not passes(("s_full", j % NS), j // NS):
+                yield
+            yield
+            if j > 0 and rnd.random() < rescale_p:      # O rescaled: PV_{j-1} done
+                while not passes(("o_ready", (j - 1) % NS), (j - 1) // NS):
+                    yield
+                assert j - 1 in pv_done
+            bars["p_full", j % NS].arrive()
+            yield
+        if ntiles:
+            last = ntiles - 1
+            if final_wait == "o_ready":
+                while not passes(("o_ready", last % NS), last // NS):
+                    yield
+            else:                                        # the V ring's barrier instead
+                while not passes(("v_empty", last % NSV), last // NSV):
+                    yield
+            assert set(range(ntiles)) <= pv_done
+
+    roles = [producer(), mma()] + [softmax() for _ in range(4)]
+    idle = 0
+    while roles or tma or pipe:
+        choices = list(range(len(roles))) + (["tma"] if tma else []) + (["pipe"] if pipe else [])
+        c = rnd.choice(choices)
+        if c == "tma":        # copies land in any order
+            bars[tma.pop(rnd.randrange(len(tma)))].arrive()
+            idle = 0
+        elif c == "pipe":     # the tensor pipe completes in issue order
+            (kind, t), commits = pipe.pop(0)
+            if kind == "pv":
+                pv_done.add(t)
+            for name in commits:
+                bars[name].arrive()
+            idle = 0
+        else:
+            try:
+                next(roles[c])
+            except StopIteration:
+                roles.pop(c)
+            idle += 1
+        assert idle < 50_000, "no role can make progress: a wait never ends"
+
+
+@pytest.mark.parametrize("NS,NSK,NSV", [(3, 3, 2), (2, 2, 2)],
+                         ids=["128-key tiles", "64-key tiles"])
+@pytest.mark.parametrize("ntiles", [1, 2, 3, 4, 5, 8, 17])
+def test_rows_kernel_protocol(NS, NSK, NSV, ntiles):
+    for seed in range(150):
+        _run(NS, NSK, NSV, ntiles, seed)
+
+
+def test_the_checks_catch_a_stale_wait():
+    # Waiting for the last PV product on the V ring's empty barrier instead of
+    # o_ready looks equivalent (PV_j also arrives there) but is not: with two
+    # V stages the phase before PV_{n-1} on that barrier is PV_{n-3}, which
+    # may still be running, so the parity wait can pass one phase early.  The
+    # protocol check must flag it.
+    with pytest.raises(AssertionError):
+        for seed in range(300):
+            _run(3, 3, 2, 6, seed, final_wait="v_empty")
