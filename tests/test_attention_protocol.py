@@ -1,4 +1,4 @@
-"""The mbarrier protocol of the tcgen05 rows kernel, on the host (CPU only).
+"""The mbarrier protocols of the tcgen05 attention kernels, on the host (CPU only).
 
 The kernel's three roles meet only at mbarriers:
 - the TMA producer fills a K ring and a V ring;
@@ -164,3 +164,115 @@ def test_the_checks_catch_a_stale_wait():
     with pytest.raises(AssertionError):
         for seed in range(300):
             _run(3, 3, 2, 6, seed, final_wait="v_empty")
+
+
+def _run_keysplit(NSK, NSV, ntiles, seed, rescale_p=0.3):
+    """The key-split kernel: softmax group s (4 warps) takes tiles s, s+2, ...
+    with its own S_s, O_s and barriers s_full[s], p_full[s], o_ready[s]; MMA
+    order QK(0) QK(1), then PV(k), QK(k+2); both groups load Q (8 arrivals)."""
+    rnd = random.Random(seed)
+    bars = {"q_full": _Barrier(8)}
+    for s in range(NSK):
+        bars["k_full", s], bars["k_empty", s] = _Barrier(1), _Barrier(1)
+    for s in range(NSV):
+        bars["v_full", s], bars["v_empty", s] = _Barrier(1), _Barrier(1)
+    for g in range(2):
+        bars["s_full", g], bars["o_ready", g] = _Barrier(1), _Barrier(1)
+        bars["p_full", g] = _Barrier(4)
+
+    def passes(name, k):
+        b = bars[name]
+        if (b.done & 1) == (k & 1):
+            return False
+        assert b.done == k + 1, f"wait on {name} for phase {k} passed at {b.done} completions"
+        return True
+
+    tma, pipe, pv_done, issued_pv = [], [], set(), set()
+
+    def producer():
+        for i in range(ntiles + 1):
+            if i < ntiles:
+                s = i % NSK
+                if i >= NSK:
+                    while not passes(("k_empty", s), i // NSK - 1):
+                        yield
+                tma.append(("k_full", s))
+            if i >= 1:
+                j = i - 1
+                s = j % NSV
+                if j >= NSV:
+                    while not passes(("v_empty", s), j // NSV - 1):
+                        yield
+                tma.append(("v_full", s))
+            yield
+
+    def mma():
+        while not passes("q_full", 0):
+            yield
+
+        def qk(k):
+            while not passes(("k_full", k % NSK), k // NSK):
+                yield
+            assert k < 2 or k - 2 in issued_pv, f"QK({k}) over S_{k & 1} before PV({k - 2})"
+            pipe.append((("qk", k), [("s_full", k & 1), ("k_empty", k % NSK)]))
+        yield from qk(0)
+        if ntiles > 1:
+            yield from qk(1)
+        for k in range(ntiles):
+            while not passes(("p_full", k & 1), k >> 1):
+                yield
+            while not passes(("v_full", k % NSV), k // NSV):
+                yield
+            pipe.append((("pv", k), [("v_empty", k % NSV), ("o_ready", k & 1)]))
+            issued_pv.add(k)
+            if k + 2 < ntiles:
+                yield from qk(k + 2)
+            yield
+
+    def softmax(g):
+        bars["q_full"].arrive()
+        yield
+        mine = (ntiles - g + 1) // 2
+        for mi in range(mine):
+            while not passes(("s_full", g), mi):
+                yield
+            yield
+            if mi > 0 and rnd.random() < rescale_p:
+                while not passes(("o_ready", g), mi - 1):
+                    yield
+                assert 2 * (mi - 1) + g in pv_done
+            bars["p_full", g].arrive()
+            yield
+        if mine:
+            while not passes(("o_ready", g), mine - 1):
+                yield
+            assert {2 * i + g for i in range(mine)} <= pv_done
+
+    roles = [producer(), mma()] + [softmax(g) for g in (0, 1) for _ in range(4)]
+    idle = 0
+    while roles or tma or pipe:
+        choices = list(range(len(roles))) + (["tma"] if tma else []) + (["pipe"] if pipe else [])
+        c = rnd.choice(choices)
+        if c == "tma":
+            bars[tma.pop(rnd.randrange(len(tma)))].arrive()
+            idle = 0
+        elif c == "pipe":
+            (kind, t), commits = pipe.pop(0)
+            if kind == "pv":
+                pv_done.add(t)
+            for name in commits:
+                bars[name].arrive()
+            idle = 0
+        else:
+            try:
+                next(roles[c])
+            except StopIteration:
+                roles.pop(c)
+            idle += 1
+        assert idle < 50_000, "no role can make progress: a wait never ends"
+
+
+@pytest.mark.parametrize("ntiles", [1, 2, 3, 4, 5, 9, 16])
+def test_keysplit_kernel_protocol(ntiles):
+    for seed in range(150):
+        _run_keysplit(3, 2, ntiles, seed)
