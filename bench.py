@@ -230,9 +230,22 @@ def _clock_summary(proc):
             "samples": len(sm)}
 
 
+KERNEL_SECTION_END = "// ------------------------------------------------------------------ host"
+
+
+def kernel_source_hash(text: str) -> str:
+    """Hash of the kernels' source text in a CUDA file: from its first
+    anonymous namespace to the host-section marker (the includes above and
+    the host launch code below do not change what the kernels compute or
+    move)."""
+    i = text.index("namespace {\n")
+    j = text.index(KERNEL_SECTION_END, i)
+    return hashlib.sha256(text[i:j].encode()).hexdigest()[:16]
+
+
 def _traffic_record(kernel_src: str, workload: str):
     """DRAM traffic of the dominant kernel from the committed ncu summary, if
-    the summary was taken on the current source of that kernel."""
+    the summary was taken on the current source of the kernels."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
@@ -242,8 +255,11 @@ def _traffic_record(kernel_src: str, workload: str):
         return None
     if not rec:
         return None
-    h = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()[:16]
-    return rec.get("bytes_per_launch") if rec.get("source_sha") == h else None
+    try:
+        h = kernel_source_hash(open(kernel_src).read())
+    except (ValueError, OSError):
+        return None
+    return rec.get("bytes_per_launch") if rec.get("kernel_sha") == h else None
 
 
 # ------------------------------------------------------------ CPU oracle

@@ -109,3 +109,14 @@ def test_accepted_summary_skips_malformed_sequences():
     assert set(bench.accepted_summary(_W(), st)) == {"stochastic"}
     st.s = VerifyResult(z, z, torch.full((4,), -1, dtype=torch.int32))
     assert bench.accepted_summary(_W(), st) == {}
+
+
+def test_traffic_record_is_keyed_by_the_kernel_section():
+    src = ("#include <a>\nnamespace {\n__global__ void k() {}\n}\n"
+           + bench.KERNEL_SECTION_END + "\nint launch() { return 0; }\n")
+    h = bench.kernel_source_hash(src)
+    # edits to the includes or the host launch code keep the key ...
+    assert bench.kernel_source_hash("#include <b>\n" + src) == h
+    assert bench.kernel_source_hash(src.replace("return 0", "return 1")) == h
+    # ... an edit to a kernel does not
+    assert bench.kernel_source_hash(src.replace("k() {}", "k() { }")) != h

@@ -44,6 +44,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -1039,28 +1040,37 @@ bool make_kv_map(CUtensorMap *m, const void *ptr, int rows, int planes, int box_
     return r == CUDA_SUCCESS;
 }
 
+// The kernels' shared-memory limits are attributes of the current device's
+// copy of each kernel: raised once per device (a process may drive several).
 cudaError_t set_smem_attributes()
 {
-    static std::once_flag once;
-    static cudaError_t err = cudaSuccess;
-    std::call_once(once, [] {
-        auto wide = tree_attn_rows_kernel<Wide, 3, 1>;
-        auto half = tree_attn_rows_kernel<Half, 2, 2>;
-        err = cudaFuncSetAttribute(wide, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    constexpr int kMaxDevices = 64;
+    static std::atomic<bool> done[kMaxDevices];
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess)
+        return err;
+    if (dev < 0 || dev >= kMaxDevices)
+        return cudaErrorInvalidDevice;
+    if (done[dev].load())
+        return cudaSuccess;
+    auto wide = tree_attn_rows_kernel<Wide, 3, 1>;
+    auto half = tree_attn_rows_kernel<Half, 2, 2>;
+    err = cudaFuncSetAttribute(wide, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)Wide::kSmemBytes);
+    if (err == cudaSuccess)
+        err = cudaFuncSetAttribute(tree_attn_keysplit_kernel,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)Wide::kSmemBytes);
-        if (err == cudaSuccess)
-            err = cudaFuncSetAttribute(tree_attn_keysplit_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)Wide::kSmemBytes);
-        if (err == cudaSuccess)
-            err = cudaFuncSetAttribute(half, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)Half::kSmemBytes);
-
-        // two CTAs per SM need the largest shared-memory carve-out
-        if (err == cudaSuccess)
-            err = cudaFuncSetAttribute(half, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                       (int)cudaSharedmemCarveoutMaxShared);
-    });
+    if (err == cudaSuccess)
+        err = cudaFuncSetAttribute(half, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)Half::kSmemBytes);
+    // two CTAs per SM need the largest shared-memory carve-out
+    if (err == cudaSuccess)
+        err = cudaFuncSetAttribute(half, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                   (int)cudaSharedmemCarveoutMaxShared);
+    if (err == cudaSuccess)
+        done[dev].store(true);
     return err;
 }
 
