@@ -113,6 +113,30 @@ def test_attention_parity_small_on_keysplit_kernel(cuda_device, case, monkeypatc
     test_attention_parity(cuda_device, case)
 
 
+# Full trees at the row-block boundary: 32 nodes x G = 4 is exactly 128
+# packed rows, the largest query block of the small-shape kernels; 33 nodes
+# give 132 rows, the 128-key rows kernel with a second block of 4 real rows.
+@pytest.mark.parametrize("Tmax,env", [(32, None), (32, ("TSD_ATTN_SMALL_VARIANT", "keysplit")),
+                                      (33, None), (33, ("TSD_ATTN_ROWS_VARIANT", "2"))],
+                         ids=["128-rows", "128-rows-keysplit", "132-rows", "132-rows-paired"])
+def test_attention_parity_at_the_row_block_boundary(cuda_device, Tmax, env, monkeypatch):
+    if env:
+        monkeypatch.setenv(*env)
+    w = gen.random_workload(90 + Tmax, B=2, Tmax=Tmax, Hq=8, Hkv=2, D=128, P_max=400,
+                            dtype="bf16", min_nodes=Tmax, max_children=4, max_depth=12,
+                            lmax_pad=37, V=16)
+    assert (w.n_nodes == Tmax).all()
+    d = to_dev(w, cuda_device)
+    poison(w, d)
+    tree = run_tree(d)
+    sentinel = 1234.0
+    out = torch.full_like(d["q"], sentinel)
+    tsd.tree_attention(d["q"], d["k_cache"], d["v_cache"], d["prefix_len"], d["n_nodes"],
+                       tree.mask, out=out)
+    check_attention(w, out, sentinel=sentinel)
+    assert _status(cuda_device) == 0
+
+
 def test_attention_empty_trees_and_prefix(cuda_device):
     # T_b = 0 sequences, P_b = 0 sequences, and a single-node tree with no prefix
     w = gen.random_workload(21, B=4, Tmax=8, Hq=4, Hkv=2, D=128, P_max=50, dtype="bf16",
