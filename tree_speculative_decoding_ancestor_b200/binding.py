@@ -103,6 +103,13 @@ def _stream(device: torch.device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
 
+def _cuda(device: torch.device) -> None:
+    """The kernels read and write device memory only: refuse anything else
+    before a host address can reach a launch."""
+    if device.type != "cuda":
+        raise ValueError(f"tensors must be on a CUDA device, got {device}")
+
+
 def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape: Tuple[int, ...],
           device: torch.device) -> None:
     if not isinstance(t, torch.Tensor):
@@ -140,6 +147,27 @@ def _get_workspace(device: torch.device, kind: str, nbytes: int) -> torch.Tensor
     return ws
 
 
+def _workspace_for(device: torch.device, kind: str, nbytes: int,
+                   workspace: Optional[torch.Tensor]) -> torch.Tensor:
+    """The caller's workspace (a contiguous uint8 tensor on the device: its
+    element count is the byte count the library checks), or the cache's."""
+    if workspace is None:
+        return _get_workspace(device, kind, nbytes)
+    _need(workspace, "workspace", torch.uint8, (workspace.numel(),), device)
+    return workspace
+
+
+def _status_for(device: torch.device, status: Optional[torch.Tensor]) -> torch.Tensor:
+    """The caller's status word (an int32 tensor on the device), or the
+    per-device one."""
+    if status is None:
+        return device_status(device)
+    if not isinstance(status, torch.Tensor) or status.dtype != torch.int32 or \
+            status.device != device or status.numel() < 1:
+        raise ValueError(f"status must be an int32 tensor on {device}")
+    return status
+
+
 class TreeMask(NamedTuple):
     mask: torch.Tensor          # [B][Tmax][W] int32 (bit pattern of uint32)
     depth: torch.Tensor         # [B][Tmax] int32
@@ -153,12 +181,27 @@ class VerifyResult(NamedTuple):
     n_accepted: torch.Tensor    # [B] int32
 
 
+def _need_tree(tree: TreeMask, B: int, Tmax: int, device: torch.device, fields) -> None:
+    """Check the TreeMask fields a call reads or writes."""
+    shapes = {"mask": (B, Tmax, (Tmax + 31) // 32), "depth": (B, Tmax),
+              "first_child": (B, Tmax + 1), "next_sibling": (B, Tmax)}
+    for f in fields:
+        _need(getattr(tree, f), f, torch.int32, shapes[f], device)
+
+
+def _need_result(out: VerifyResult, B: int, Tmax: int, device: torch.device) -> None:
+    _need(out.out_tokens, "out_tokens", torch.int32, (B, Tmax + 1), device)
+    _need(out.out_path, "out_path", torch.int32, (B, Tmax), device)
+    _need(out.n_accepted, "n_accepted", torch.int32, (B,), device)
+
+
 def tree_mask_build(parent: torch.Tensor, n_nodes: torch.Tensor,
                     out: Optional[TreeMask] = None, status: Optional[torch.Tensor] = None
                     ) -> TreeMask:
     """Ancestor mask, depth and child lists of each token tree."""
     lib = load_library()
     dev = parent.device
+    _cuda(dev)
     B, Tmax = parent.shape
     W = (Tmax + 31) // 32
     _need(parent, "parent", torch.int32, (B, Tmax), dev)
@@ -168,7 +211,8 @@ def tree_mask_build(parent: torch.Tensor, n_nodes: torch.Tensor,
                        torch.empty((B, Tmax), dtype=torch.int32, device=dev),
                        torch.empty((B, Tmax + 1), dtype=torch.int32, device=dev),
                        torch.empty((B, Tmax), dtype=torch.int32, device=dev))
-    st = device_status(dev) if status is None else status
+    _need_tree(out, B, Tmax, dev, ("mask", "depth", "first_child", "next_sibling"))
+    st = _status_for(dev, status)
     rc = lib.tsd_tree_mask_build(_ptr(parent), _ptr(n_nodes), B, Tmax, _ptr(out.mask),
                                  _ptr(out.depth), _ptr(out.first_child), _ptr(out.next_sibling),
                                  _ptr(st), _stream(dev))
@@ -190,6 +234,7 @@ def tree_attention(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
     """Topology-aware tree attention over prefix KV + ancestors (out[B][Tmax][Hq][D])."""
     lib = load_library()
     dev = q.device
+    _cuda(dev)
     B, Tmax, Hq, D = q.shape
     Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
     if q.dtype not in (torch.float32, torch.bfloat16):
@@ -207,8 +252,8 @@ def tree_attention(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
         scale = D ** -0.5
     code = TSD_BF16 if q.dtype == torch.bfloat16 else TSD_F32
     need = int(lib.tsd_tree_attention_workspace_size(B, Tmax, Hq, Hkv, D, Lmax, code))
-    ws = _get_workspace(dev, "attn", need) if workspace is None else workspace
-    st = device_status(dev) if status is None else status
+    ws = _workspace_for(dev, "attn", need, workspace)
+    st = _status_for(dev, status)
     rc = lib.tsd_tree_attention(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(prefix_len),
                                 _ptr(n_nodes), _ptr(mask), B, Tmax, Hq, Hkv, D, Lmax,
                                 float(scale), code, _ptr(out), _ptr(ws), ws.numel(), _ptr(st),
@@ -237,16 +282,19 @@ def tree_verify_greedy(logits: torch.Tensor, tokens: torch.Tensor, parent: torch
     """Longest root path matching the target argmax, plus one bonus token."""
     lib = load_library()
     dev = logits.device
+    _cuda(dev)
     B, R, V = logits.shape
     Tmax = R - 1
     _need(logits, "logits", torch.float32, (B, Tmax + 1, V), dev)
     _need(tokens, "tokens", torch.int32, (B, Tmax), dev)
     _need(parent, "parent", torch.int32, (B, Tmax), dev)
     _need(n_nodes, "n_nodes", torch.int32, (B,), dev)
+    _need_tree(tree, B, Tmax, dev, ("mask", "first_child"))
     out = _verify_outputs(B, Tmax, dev, out)
+    _need_result(out, B, Tmax, dev)
     need = int(lib.tsd_tree_verify_workspace_size(B, Tmax, V))
-    ws = _get_workspace(dev, "verify", need) if workspace is None else workspace
-    st = device_status(dev) if status is None else status
+    ws = _workspace_for(dev, "verify", need, workspace)
+    st = _status_for(dev, status)
     rc = lib.tsd_tree_verify_greedy(_ptr(logits), _ptr(tokens), _ptr(parent), _ptr(n_nodes),
                                     _ptr(tree.mask), _ptr(tree.first_child), B, Tmax, V,
                                     _ptr(out.out_tokens), _ptr(out.out_path),
@@ -265,6 +313,7 @@ def tree_verify_stochastic(logits: torch.Tensor, temperature: float, q_probs: to
     """Multi-step speculative sampling over the tree (exact target distribution)."""
     lib = load_library()
     dev = logits.device
+    _cuda(dev)
     B, R, V = logits.shape
     Tmax = R - 1
     Rq = q_probs.shape[1]
@@ -275,10 +324,12 @@ def tree_verify_stochastic(logits: torch.Tensor, temperature: float, q_probs: to
     _need(n_nodes, "n_nodes", torch.int32, (B,), dev)
     _need(u_accept, "u_accept", torch.float64, (B, Tmax), dev)
     _need(u_sample, "u_sample", torch.float64, (B, Tmax + 1), dev)
+    _need_tree(tree, B, Tmax, dev, ("first_child", "next_sibling"))
     out = _verify_outputs(B, Tmax, dev, out)
+    _need_result(out, B, Tmax, dev)
     need = int(lib.tsd_tree_verify_workspace_size(B, Tmax, V))
-    ws = _get_workspace(dev, "verify", need) if workspace is None else workspace
-    st = device_status(dev) if status is None else status
+    ws = _workspace_for(dev, "verify", need, workspace)
+    st = _status_for(dev, status)
     rc = lib.tsd_tree_verify_stochastic(_ptr(logits), float(temperature), _ptr(q_probs), Rq,
                                         _ptr(q_row), _ptr(tokens), _ptr(n_nodes),
                                         _ptr(tree.first_child), _ptr(tree.next_sibling),
@@ -303,6 +354,7 @@ def tree_verify_stochastic_noalloc(logits: torch.Tensor, temperature: float,
     scratch, the first-call set-up and why overlapping calls race)."""
     lib = load_library()
     dev = logits.device
+    _cuda(dev)
     B, R, V = logits.shape
     Tmax = R - 1
     Rq = q_probs.shape[1]
@@ -313,7 +365,9 @@ def tree_verify_stochastic_noalloc(logits: torch.Tensor, temperature: float,
     _need(n_nodes, "n_nodes", torch.int32, (B,), dev)
     _need(u_accept, "u_accept", torch.float64, (B, Tmax), dev)
     _need(u_sample, "u_sample", torch.float64, (B, Tmax + 1), dev)
-    st = device_status(dev) if status is None else status
+    _need_tree(tree, B, Tmax, dev, ("first_child", "next_sibling"))
+    _need_result(out, B, Tmax, dev)
+    st = _status_for(dev, status)
     rc = lib.tsd_tree_verify_stochastic_noalloc(
         _ptr(logits), float(temperature), _ptr(q_probs), Rq, _ptr(q_row), _ptr(tokens),
         _ptr(n_nodes), _ptr(tree.first_child), _ptr(tree.next_sibling), _ptr(u_accept),
@@ -330,6 +384,7 @@ def kv_commit(k_cache: torch.Tensor, v_cache: torch.Tensor, prefix_len: torch.Te
     after each sequence's prefix; returns the new prefix lengths [B] int32."""
     lib = load_library()
     dev = k_cache.device
+    _cuda(dev)
     B, Hkv, Lmax, D = k_cache.shape
     Tmax = result.out_path.shape[1]
     dt = {torch.float32: TSD_F32, torch.bfloat16: TSD_BF16}.get(k_cache.dtype)
@@ -343,7 +398,7 @@ def kv_commit(k_cache: torch.Tensor, v_cache: torch.Tensor, prefix_len: torch.Te
     if new_prefix_len is None:
         new_prefix_len = torch.empty((B,), dtype=torch.int32, device=dev)
     _need(new_prefix_len, "new_prefix_len", torch.int32, (B,), dev)
-    st = device_status(dev) if status is None else status
+    st = _status_for(dev, status)
     rc = lib.tsd_kv_commit(_ptr(k_cache), _ptr(v_cache), _ptr(prefix_len), _ptr(result.out_path),
                            _ptr(result.n_accepted), B, Tmax, Hkv, D, Lmax, dt,
                            _ptr(new_prefix_len), _ptr(st), _stream(dev))
@@ -361,12 +416,14 @@ def tree_attention_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.
     and a block table [B][max_blocks] of physical page ids."""
     lib = load_library()
     dev = q.device
+    _cuda(dev)
     B, Tmax, Hq, D = q.shape
     num_pages, Hkv, page_size, _ = k_pages.shape
     max_blocks = block_table.shape[1]
     dt = {torch.float32: TSD_F32, torch.bfloat16: TSD_BF16}.get(q.dtype)
     if dt is None:
         raise TypeError("q must be float32 or bfloat16")
+    _need(q, "q", q.dtype, (B, Tmax, Hq, D), dev)
     _need(k_pages, "k_pages", q.dtype, (num_pages, Hkv, page_size, D), dev)
     _need(v_pages, "v_pages", q.dtype, (num_pages, Hkv, page_size, D), dev)
     _need(block_table, "block_table", torch.int32, (B, max_blocks), dev)
@@ -378,8 +435,8 @@ def tree_attention_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.
     _need(out, "out", q.dtype, (B, Tmax, Hq, D), dev)
     Lmax = max_blocks * page_size
     need = int(lib.tsd_tree_attention_workspace_size(B, Tmax, Hq, Hkv, D, Lmax, dt))
-    ws = _get_workspace(dev, "attention", need) if workspace is None else workspace
-    st = device_status(dev) if status is None else status
+    ws = _workspace_for(dev, "attention", need, workspace)
+    st = _status_for(dev, status)
     sc = (1.0 / D ** 0.5) if scale is None else float(scale)
     rc = lib.tsd_tree_attention_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table),
                                       num_pages, page_size, max_blocks, _ptr(prefix_len),
@@ -402,6 +459,7 @@ def tree_expand(q_probs: torch.Tensor, frow: torch.Tensor, k: int, tree: Tree,
     frontier node's SSM row become its children)."""
     lib = load_library()
     dev = q_probs.device
+    _cuda(dev)
     B, Rq, V = q_probs.shape
     Tmax = tree.parent.shape[1]
     _need(q_probs, "q_probs", torch.float32, (B, Rq, V), dev)
@@ -410,7 +468,7 @@ def tree_expand(q_probs: torch.Tensor, frow: torch.Tensor, k: int, tree: Tree,
         _need(getattr(tree, name), name, torch.int32, (B, Tmax), dev)
     _need(tree.n_nodes, "n_nodes", torch.int32, (B,), dev)
     _need(lvl_begin, "lvl_begin", torch.int32, (B,), dev)
-    st = device_status(dev) if status is None else status
+    st = _status_for(dev, status)
     rc = lib.tsd_tree_expand(_ptr(q_probs), Rq, V, _ptr(frow), int(k), _ptr(tree.parent),
                              _ptr(tree.tokens), _ptr(tree.q_row), _ptr(tree.n_nodes),
                              _ptr(lvl_begin), B, Tmax, _ptr(st), _stream(dev))
@@ -422,6 +480,7 @@ def tree_dfs_order(tree: Tree, status: Optional[torch.Tensor] = None):
     """Depth-first renumbering: returns (perm [B][Tmax], renumbered Tree)."""
     lib = load_library()
     dev = tree.parent.device
+    _cuda(dev)
     B, Tmax = tree.parent.shape
     for name in ("parent", "tokens", "q_row"):
         _need(getattr(tree, name), name, torch.int32, (B, Tmax), dev)
@@ -429,7 +488,7 @@ def tree_dfs_order(tree: Tree, status: Optional[torch.Tensor] = None):
     perm = torch.full((B, Tmax), -1, dtype=torch.int32, device=dev)
     out = Tree(torch.full_like(tree.parent, -1), torch.zeros_like(tree.tokens),
                torch.zeros_like(tree.q_row), tree.n_nodes.clone())
-    st = device_status(dev) if status is None else status
+    st = _status_for(dev, status)
     rc = lib.tsd_tree_dfs_order(_ptr(tree.parent), _ptr(tree.tokens), _ptr(tree.q_row),
                                 _ptr(tree.n_nodes), B, Tmax, _ptr(perm), _ptr(out.parent),
                                 _ptr(out.tokens), _ptr(out.q_row), _ptr(st), _stream(dev))
@@ -443,6 +502,7 @@ def tree_merge_chains(chain_tokens: torch.Tensor, chain_q_row: torch.Tensor,
     """Merge M draft chains per sequence into one token tree (depth-first)."""
     lib = load_library()
     dev = chain_tokens.device
+    _cuda(dev)
     B, M, L = chain_tokens.shape
     _need(chain_tokens, "chain_tokens", torch.int32, (B, M, L), dev)
     _need(chain_q_row, "chain_q_row", torch.int32, (B, M, L), dev)
@@ -451,7 +511,7 @@ def tree_merge_chains(chain_tokens: torch.Tensor, chain_q_row: torch.Tensor,
                torch.zeros((B, Tmax), dtype=torch.int32, device=dev),
                torch.zeros((B, Tmax), dtype=torch.int32, device=dev),
                torch.zeros((B,), dtype=torch.int32, device=dev))
-    st = device_status(dev) if status is None else status
+    st = _status_for(dev, status)
     rc = lib.tsd_tree_merge_chains(_ptr(chain_tokens), _ptr(chain_q_row), _ptr(chain_len), M, L,
                                    B, Tmax, _ptr(out.parent), _ptr(out.tokens), _ptr(out.q_row),
                                    _ptr(out.n_nodes), _ptr(st), _stream(dev))
@@ -466,7 +526,10 @@ def debug_wait_probe(kind: int, limit_ns: int = 50_000_000, device=None,
     limit_ns with DEV_TIMEOUT set in the status word."""
     lib = load_library()
     dev = torch.device(device or torch.cuda.current_device())
+    _cuda(dev)
+    if dev.index is None:
+        dev = torch.device("cuda", torch.cuda.current_device())
     scratch = torch.zeros(2, dtype=torch.int32, device=dev)
-    st = device_status(dev) if status is None else status
+    st = _status_for(dev, status)
     rc = lib.tsd_debug_wait_probe(int(kind), int(limit_ns), _ptr(scratch), _ptr(st), _stream(dev))
     _check(rc, "tsd_debug_wait_probe")
