@@ -77,6 +77,14 @@ enum tsd_dev_status {
 /* Element types of Q / K / V / attention output. */
 enum tsd_dtype { TSD_F32 = 0, TSD_BF16 = 1 };
 
+/* Attention kernels, as reported by tsd_tree_attention_plan. */
+enum tsd_attention_path {
+    TSD_PLAN_SIMT = 0,       /* CUDA cores, 16 query rows per CTA                       */
+    TSD_PLAN_ROWS128 = 1,    /* tensor cores, 128-key tiles, one CTA per SM             */
+    TSD_PLAN_ROWS64 = 2,     /* tensor cores, 64-key tiles, two CTAs per SM             */
+    TSD_PLAN_KEYSPLIT = 3    /* tensor cores, two softmax groups splitting the key tiles */
+};
+
 /* Marker written to first_child[b][0] by tsd_tree_mask_build for a malformed
  * tree; the verify calls then report n_accepted[b] = -1 for that sequence. */
 #define TSD_TREE_INVALID (-2)
@@ -116,6 +124,20 @@ int tsd_tree_mask_build(const int32_t *parent, const int32_t *n_nodes, int B, in
  * Bytes of workspace tsd_tree_attention needs for these sizes (split-KV
  * partial results).  Depends only on the arguments and the current device.
  */
+/*
+ * The launch tsd_tree_attention would make for these sizes on a device with
+ * num_sms SMs (host only, nothing is launched; the environment variables
+ * that select the attention kernel are read as in the call itself):
+ *   plan[0]  the kernel, a tsd_attention_path value
+ *   plan[1]  query-row blocks per (sequence, KV head)
+ *   plan[2]  key-range splits (combined by log-sum-exp when > 1)
+ *   plan[3]  keys per split
+ * Errors: TSD_ERR_NULL (plan), TSD_ERR_SHAPE (sizes as for the call,
+ * num_sms < 1), TSD_ERR_DTYPE.
+ */
+int tsd_tree_attention_plan(int B, int Tmax, int Hq, int Hkv, int D, int Lmax, int dtype,
+                            int num_sms, int32_t *plan);
+
 size_t tsd_tree_attention_workspace_size(int B, int Tmax, int Hq, int Hkv, int D, int Lmax,
                                          int dtype);
 

@@ -19,6 +19,7 @@ from .binding import (  # noqa: F401
     Tree,
     TreeMask,
     VerifyResult,
+    attention_plan,
     attention_workspace_size,
     device_status,
     exported_symbols,

@@ -40,6 +40,7 @@ _SIGNATURES: Dict[str, Tuple[object, list]] = {
     "tsd_launch_count": (ctypes.c_ulonglong, []),
     "tsd_tree_mask_build": (_I, [_P, _P, _I, _I, _P, _P, _P, _P, _P, _P]),
     "tsd_tree_attention_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
+    "tsd_tree_attention_plan": (_I, [_I, _I, _I, _I, _I, _I, _I, _I, _P]),
     "tsd_tree_attention": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float,
                                 _I, _P, _P, _SZ, _P, _P]),
     "tsd_tree_verify_workspace_size": (_SZ, [_I, _I, _I]),
@@ -224,6 +225,23 @@ def attention_workspace_size(B: int, Tmax: int, Hq: int, Hkv: int, D: int, Lmax:
                              dtype: torch.dtype) -> int:
     code = TSD_BF16 if dtype == torch.bfloat16 else TSD_F32
     return int(load_library().tsd_tree_attention_workspace_size(B, Tmax, Hq, Hkv, D, Lmax, code))
+
+
+PLAN_KERNELS = {0: "simt", 1: "rows128", 2: "rows64", 3: "keysplit"}
+
+
+def attention_plan(B: int, Tmax: int, Hq: int, Hkv: int, D: int, Lmax: int,
+                   dtype: torch.dtype, num_sms: int) -> Dict[str, object]:
+    """The kernel and grid tree_attention would use for these sizes on a
+    device with num_sms SMs (host only): kernel name, query-row blocks per
+    (sequence, KV head), key-range splits, keys per split."""
+    code = TSD_BF16 if dtype == torch.bfloat16 else TSD_F32
+    plan = (ctypes.c_int32 * 4)()
+    rc = load_library().tsd_tree_attention_plan(B, Tmax, Hq, Hkv, D, Lmax, code, num_sms,
+                                                ctypes.addressof(plan))
+    _check(rc, "tsd_tree_attention_plan")
+    return {"kernel": PLAN_KERNELS[plan[0]], "row_blocks": plan[1], "splits": plan[2],
+            "keys_per_split": plan[3]}
 
 
 def tree_attention(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,

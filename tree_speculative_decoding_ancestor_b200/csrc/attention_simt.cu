@@ -315,6 +315,15 @@ int launch_combine(int dtype, int D, const float *part_o, const float2 *part_ml,
     return TSD_ERR_DTYPE;
 }
 
+void simt_attention_plan(const AttnArgs &a, int num_sms, int32_t out[4])
+{
+    const SimtPlan p = simt_plan(a, num_sms);
+    out[0] = TSD_PLAN_SIMT;
+    out[1] = p.row_chunks;
+    out[2] = p.nsplit;
+    out[3] = p.keys_per_split;
+}
+
 size_t simt_attention_workspace(const AttnArgs &a, int num_sms)
 {
     const SimtPlan p = simt_plan(a, num_sms);

@@ -1083,6 +1083,15 @@ bool umma_attention_supported(const AttnArgs &a)
     return a.dtype == TSD_BF16 && a.D == HD && a.Tmax * (a.Hq / a.Hkv) >= 8;
 }
 
+void umma_attention_plan(const AttnArgs &a, int num_sms, int32_t out[4])
+{
+    const UmmaPlan p = umma_plan(a, num_sms);
+    out[0] = p.keysplit ? TSD_PLAN_KEYSPLIT : (p.paired ? TSD_PLAN_ROWS64 : TSD_PLAN_ROWS128);
+    out[1] = p.nrb;
+    out[2] = p.nsplit;
+    out[3] = p.keys_per_split;
+}
+
 size_t umma_attention_workspace(const AttnArgs &a, int num_sms)
 {
     const UmmaPlan p = umma_plan(a, num_sms);

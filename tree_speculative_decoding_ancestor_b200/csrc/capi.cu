@@ -104,6 +104,25 @@ size_t tsd_tree_attention_workspace_size(int B, int Tmax, int Hq, int Hkv, int D
                           : tsd::simt_attention_workspace(a, sms);
 }
 
+int tsd_tree_attention_plan(int B, int Tmax, int Hq, int Hkv, int D, int Lmax, int dtype,
+                            int num_sms, int32_t *plan)
+{
+    if (!plan)
+        return TSD_ERR_NULL;
+    if (B < 1 || Tmax < 1 || Tmax > TSD_MAX_TREE || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 ||
+        Lmax < Tmax || num_sms < 1)
+        return TSD_ERR_SHAPE;
+    if ((dtype != TSD_F32 && dtype != TSD_BF16) || (D != 64 && D != 128))
+        return TSD_ERR_DTYPE;
+    tsd::AttnArgs a{};
+    a.B = B; a.Tmax = Tmax; a.Hq = Hq; a.Hkv = Hkv; a.D = D; a.Lmax = Lmax; a.dtype = dtype;
+    if (choose_umma(a))
+        tsd::umma_attention_plan(a, num_sms, plan);
+    else
+        tsd::simt_attention_plan(a, num_sms, plan);
+    return TSD_OK;
+}
+
 int tsd_tree_attention(const void *q, const void *k_cache, const void *v_cache,
                        const int32_t *prefix_len, const int32_t *n_nodes, const uint32_t *mask,
                        int B, int Tmax, int Hq, int Hkv, int D, int Lmax, float scale,

@@ -115,6 +115,8 @@ struct AttnArgs {
     KvPages pages;
 };
 size_t simt_attention_workspace(const AttnArgs &a, int num_sms);
+void simt_attention_plan(const AttnArgs &a, int num_sms, int32_t out[4]);
+void umma_attention_plan(const AttnArgs &a, int num_sms, int32_t out[4]);
 int launch_simt_attention(const AttnArgs &a, void *ws, size_t ws_bytes, int num_sms,
                           cudaStream_t stream);
 bool umma_attention_supported(const AttnArgs &a);
