@@ -430,6 +430,10 @@ def main():
                               "attention_umma.cu")
     roof["traffic"] = _traffic_record(kernel_src, args.workload)
     roof["kernel"] = "tree attention (mask-aware split-KV), one layer"
+    roof["plan"] = tsd.attention_plan(
+        w.B, w.Tmax, w.Hq, w.Hkv, w.D, int(w.k_cache.shape[2]),
+        torch.bfloat16 if w.dtype == "bf16" else torch.float32,
+        torch.cuda.get_device_properties(dev).multi_processor_count)
     roof["attn_us"] = att_s * 1e6
     roof["algorithmic_bytes"] = abytes
     roof["algorithmic_flops"] = flops
