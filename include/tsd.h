@@ -159,7 +159,8 @@ size_t tsd_tree_attention_workspace_size(int B, int Tmax, int Hq, int Hkv, int D
  * Cache positions at or beyond prefix_len[b] + T_b are never read into the
  * result, whatever they hold.  q, k_cache, v_cache, out must be 16-byte
  * aligned.  Host errors: TSD_ERR_NULL, TSD_ERR_SHAPE (Hq % Hkv != 0, sizes
- * out of range), TSD_ERR_DTYPE, TSD_ERR_ALIGN, TSD_ERR_WORKSPACE, TSD_ERR_CUDA.
+ * out of range, B * Hkv > 65535), TSD_ERR_DTYPE, TSD_ERR_ALIGN,
+ * TSD_ERR_WORKSPACE, TSD_ERR_CUDA.
  * Device: TSD_DEV_BAD_PREFIX (that sequence's rows are not written),
  * TSD_DEV_TIMEOUT.
  * Kernel choice (results agree within the bf16 tolerance whichever runs):
@@ -224,6 +225,8 @@ size_t tsd_tree_verify_workspace_size(int B, int Tmax, int V);
  *   n_accepted  [B] int32           out: number of accepted nodes (-1 if the
  *                                   sequence is malformed; nothing else written)
  * Entries beyond n_accepted (+1 for out_tokens) are not written.
+ * Host errors: TSD_ERR_SHAPE (B < 0 or > 65535, Tmax, V < 1), TSD_ERR_NULL,
+ * TSD_ERR_ALIGN (logits), TSD_ERR_WORKSPACE, TSD_ERR_CUDA.
  * Device: TSD_DEV_BAD_TOKEN.
  */
 int tsd_tree_verify_greedy(const float *logits, const int32_t *tokens, const int32_t *parent,
@@ -339,8 +342,9 @@ int tsd_tree_merge_chains(const int32_t *chain_tokens, const int32_t *chain_q_ro
  * already reported why).  A path that is not strictly increasing, leaves
  * [0, Tmax), is longer than Tmax or reaches past Lmax moves nothing and sets
  * TSD_DEV_BAD_PATH.  Pointers 16-byte aligned; D * element size a multiple
- * of 16 and at most 512 bytes.  Host errors: TSD_ERR_NULL, TSD_ERR_SHAPE,
- * TSD_ERR_DTYPE, TSD_ERR_ALIGN, TSD_ERR_CUDA.  Device: TSD_DEV_BAD_PATH.
+ * of 16 and at most 512 bytes; B at most 65535.  Host errors: TSD_ERR_NULL,
+ * TSD_ERR_SHAPE, TSD_ERR_DTYPE, TSD_ERR_ALIGN, TSD_ERR_CUDA.  Device:
+ * TSD_DEV_BAD_PATH.
  */
 int tsd_kv_commit(void *k_cache, void *v_cache, const int32_t *prefix_len,
                   const int32_t *out_path, const int32_t *n_accepted, int B, int Tmax, int Hkv,

@@ -89,6 +89,10 @@ def test_host_checks_of_every_entry_point(lib):
     assert attn(D=96) == ERR_DTYPE
     assert attn(dtype=7) == ERR_DTYPE
     assert attn(q=_U) == ERR_ALIGN
+    assert attn(B=40000, Hq=2, Hkv=2) == ERR_SHAPE   # (b, KV head) pairs beyond the grid's y
+    assert lib.tsd_tree_attention_workspace_size(40000, 8, 2, 2, 128, 64, BF16) == 0
+    assert lib.tsd_tree_verify_greedy(_A, _A, _A, _A, _A, _A, 70000, 8, 100, _A, _A, _A, _A,
+                                      1 << 20, _A, None) == ERR_SHAPE
 
     def paged(table=_A, num_pages=4, page_size=64, max_blocks=4, B=2):
         return lib.tsd_tree_attention_paged(_A, _A, _A, table, num_pages, page_size, max_blocks,
@@ -109,6 +113,7 @@ def test_host_checks_of_every_entry_point(lib):
     assert commit(path=None) == ERR_NULL
     assert commit(k=_U) == ERR_ALIGN
     assert commit(B=0) == 0
+    assert commit(B=70000) == ERR_SHAPE
 
     def expand(k=2, Tmax=8, q=_A, B=2):
         return lib.tsd_tree_expand(q, 9, 100, _A, k, _A, _A, _A, _A, _A, B, Tmax, _A, None)

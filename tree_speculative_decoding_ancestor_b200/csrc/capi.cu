@@ -25,6 +25,10 @@ int device_sms()
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Largest y extent of a launch grid: the attention kernels run (b, KV head)
+// pairs on y, the greedy row kernel and the commit kernel the sequences.
+constexpr long long kMaxGridY = 65535;
+
 // Path selection for tree attention: the tensor-core kernel when the packed
 // query block is large enough and the layout fits it, otherwise CUDA cores.
 // TSD_FORCE_PATH=simt|umma overrides (for A/B measurement).
@@ -44,7 +48,7 @@ int check_attn(const tsd::AttnArgs &a)
     if (!a.q || !a.k || !a.v || !a.prefix_len || !a.n_nodes || !a.mask || !a.out)
         return TSD_ERR_NULL;
     if (a.B < 0 || a.Tmax < 1 || a.Tmax > TSD_MAX_TREE || a.Hq < 1 || a.Hkv < 1 ||
-        a.Hq % a.Hkv != 0 || a.Lmax < a.Tmax)
+        a.Hq % a.Hkv != 0 || a.Lmax < a.Tmax || (long long)a.B * a.Hkv > kMaxGridY)
         return TSD_ERR_SHAPE;
     if (a.dtype != TSD_F32 && a.dtype != TSD_BF16)
         return TSD_ERR_DTYPE;
@@ -97,7 +101,7 @@ size_t tsd_tree_attention_workspace_size(int B, int Tmax, int Hq, int Hkv, int D
     tsd::AttnArgs a{};
     a.B = B; a.Tmax = Tmax; a.Hq = Hq; a.Hkv = Hkv; a.D = D; a.Lmax = Lmax; a.dtype = dtype;
     if (B <= 0 || Tmax < 1 || Tmax > TSD_MAX_TREE || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 ||
-        (D != 64 && D != 128) || Lmax < Tmax)
+        (D != 64 && D != 128) || Lmax < Tmax || (long long)B * Hkv > kMaxGridY)
         return 0;
     const int sms = device_sms();
     return choose_umma(a) ? tsd::umma_attention_workspace(a, sms)
@@ -110,7 +114,7 @@ int tsd_tree_attention_plan(int B, int Tmax, int Hq, int Hkv, int D, int Lmax, i
     if (!plan)
         return TSD_ERR_NULL;
     if (B < 1 || Tmax < 1 || Tmax > TSD_MAX_TREE || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 ||
-        Lmax < Tmax || num_sms < 1)
+        Lmax < Tmax || num_sms < 1 || (long long)B * Hkv > kMaxGridY)
         return TSD_ERR_SHAPE;
     if ((dtype != TSD_F32 && dtype != TSD_BF16) || (D != 64 && D != 128))
         return TSD_ERR_DTYPE;
@@ -203,7 +207,7 @@ int tsd_tree_verify_greedy(const float *logits, const int32_t *tokens, const int
                            void *workspace, size_t workspace_bytes, int32_t *dev_status,
                            tsd_stream_t stream)
 {
-    if (B < 0 || Tmax < 1 || Tmax > TSD_MAX_TREE || V < 1)
+    if (B < 0 || B > kMaxGridY || Tmax < 1 || Tmax > TSD_MAX_TREE || V < 1)
         return TSD_ERR_SHAPE;
     if (B == 0)
         return TSD_OK;
@@ -250,7 +254,8 @@ int tsd_kv_commit(void *k_cache, void *v_cache, const int32_t *prefix_len,
                   int D, int Lmax, int dtype, int32_t *new_prefix_len, int32_t *dev_status,
                   tsd_stream_t stream)
 {
-    if (B < 0 || Tmax < 1 || Tmax > TSD_MAX_TREE || Hkv < 1 || D < 1 || Lmax < 1)
+    if (B < 0 || B > kMaxGridY || Tmax < 1 || Tmax > TSD_MAX_TREE || Hkv < 1 || D < 1 ||
+        Lmax < 1)
         return TSD_ERR_SHAPE;
     if (dtype != TSD_F32 && dtype != TSD_BF16)
         return TSD_ERR_DTYPE;
