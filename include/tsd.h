@@ -171,7 +171,8 @@ size_t tsd_tree_attention_workspace_size(int B, int Tmax, int Hq, int Hkv, int D
  * (64-key tiles above 128 rows too), TSD_ATTN_SMALL_VARIANT=keysplit (two
  * softmax groups splitting the key tiles, up to 128 rows) and
  * TSD_FORCE_PATH=simt (the CUDA-core kernel for every shape) select the
- * alternatives; they are read at every call.
+ * alternatives, and TSD_ATTN_SPLITS=n fixes the number of key-range splits
+ * (at most 64 and one per key tile); they are read at every call.
  */
 int tsd_tree_attention(const void *q, const void *k_cache, const void *v_cache,
                        const int32_t *prefix_len, const int32_t *n_nodes, const uint32_t *mask,

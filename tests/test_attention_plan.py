@@ -81,3 +81,18 @@ def test_plan_rejects_bad_sizes():
         tsd.attention_plan(2, 8, 8, 2, 96, 64, torch.bfloat16, SMS)    # head dim
     with pytest.raises(tsd.TsdError):
         tsd.attention_plan(2, 8, 8, 2, 128, 64, torch.bfloat16, 0)     # no SMs
+
+
+def test_forced_split_count(monkeypatch):
+    B, Tmax, Hq, Hkv, D, Lmax, dt = _sizes("llama7b")
+    monkeypatch.setenv("TSD_ATTN_SPLITS", "3")
+    p = tsd.attention_plan(B, Tmax, Hq, Hkv, D, Lmax, dt, SMS)
+    assert p["kernel"] == "rows64" and p["splits"] == 3
+    assert 3 * p["keys_per_split"] >= Lmax and p["keys_per_split"] % 64 == 0
+    # the partial results are sized for the forced splits
+    assert tsd.attention_workspace_size(B, Tmax, Hq, Hkv, D, Lmax, dt) > 0
+    monkeypatch.setenv("TSD_ATTN_SPLITS", "1000")     # clamped to one split per key tile
+    p = tsd.attention_plan(B, Tmax, Hq, Hkv, D, Lmax, dt, SMS)
+    assert p["splits"] == (Lmax + 63) // 64
+    monkeypatch.setenv("TSD_ATTN_SPLITS", "4")        # the CUDA-core path: 128 keys at least
+    assert tsd.attention_plan(*_sizes("tiny"), SMS)["splits"] == 1

@@ -16,6 +16,9 @@
 // the usual log-sum-exp rescaling.
 #include <cfloat>
 
+#include <algorithm>
+#include <cstdlib>
+
 #include "tsd_common.cuh"
 
 namespace tsd {
@@ -44,6 +47,11 @@ SimtPlan simt_plan(const AttnArgs &a, int num_sms)
     ns = ns < 1 ? 1 : ns;
     ns = ns > max_split ? max_split : ns;
     ns = ns > 64 ? 64 : ns;
+    if (const char *e = std::getenv("TSD_ATTN_SPLITS")) {   // forced split count
+        const int n = std::atoi(e);
+        if (n >= 1)
+            ns = std::min(std::min(n, 64), max_split);
+    }
     p.nsplit = ns;
     int kps = (a.Lmax + ns - 1) / ns;
     p.keys_per_split = (kps + kSimtKeys - 1) / kSimtKeys * kSimtKeys;

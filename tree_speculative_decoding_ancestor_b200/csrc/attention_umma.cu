@@ -1000,6 +1000,13 @@ UmmaPlan umma_plan(const AttnArgs &a, int num_sms)
             best = ns;
         }
     }
+    // TSD_ATTN_SPLITS=n forces n key-range splits (1..64, at most one per
+    // tile) in place of the cost model's choice.
+    if (const char *e = std::getenv("TSD_ATTN_SPLITS")) {
+        const int n = std::atoi(e);
+        if (n >= 1)
+            best = std::min(std::min(n, 64), tiles);
+    }
     p.nsplit = best;
     p.keys_per_split = ((tiles + best - 1) / best) * bn;
     return p;
