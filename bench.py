@@ -97,15 +97,83 @@ def attn_bytes(w) -> int:
     return w.kv_bytes() + qo
 
 
-def verify_bytes(w) -> int:
-    """Logits rows of the internal nodes (+ the root) once, plus the q rows read
-    by the first acceptance pass; a lower bound used for the report only."""
-    rows = 0
-    for b in range(w.B):
-        T = int(w.n_nodes[b])
-        par = set(w.parent[b, :T].tolist())
-        rows += len(par)   # includes -1 (root) when T > 0
-    return rows * w.V * 4
+def verify_traffic(w, step) -> dict:
+    """Algorithmic bytes of the verify calls of one step: every row a
+    verifier must read, once.  Greedy: the logits row of the root and of every
+    node with children (their argmax decides the path), plus the terminal's
+    row when the path ends at a leaf (the bonus token).  Stochastic: the
+    logits rows on the accepted path and the distinct q rows of the children
+    tried there (the children before the accepted one, or all of them where
+    the walk stops); read from the step's own results."""
+    row = w.V * 4
+    out = {}
+    if "greedy" in w.verify:
+        n = step.g.n_accepted.cpu().tolist()
+        path = step.g.out_path.cpu().tolist()
+        rows = 0
+        for b in range(w.B):
+            T = int(w.n_nodes[b])
+            par = w.parent[b, :T].tolist()
+            internal = set(par)            # -1 stands for the root
+            rows += len(internal) if T else 1
+            k = n[b]
+            if k > 0 and path[b][k - 1] not in internal:
+                rows += 1                  # a leaf's row for the bonus token
+        out["greedy"] = rows * row
+    if "stochastic" in w.verify:
+        n = step.s.n_accepted.cpu().tolist()
+        path = step.s.out_path.cpu().tolist()
+        qr = w.q_row.tolist()
+        rows = 0
+        for b in range(w.B):
+            T = int(w.n_nodes[b])
+            par = w.parent[b, :T].tolist()
+            k = max(n[b], 0)
+            nodes = [-1] + path[b][:k]
+            for i, c in enumerate(nodes):
+                rows += 1                  # the logits row of node c
+                kids = [u for u in range(T) if par[u] == c]
+                stop = path[b][i] if i < k else None
+                tried = kids[:kids.index(stop) + 1] if stop is not None else kids
+                rows += len({qr[b][u] for u in tried})
+        out["stochastic"] = rows * row
+    return out
+
+
+def step_roofline(w, step, ms_per_step: float, peaks: dict) -> dict:
+    """Roofline of the whole step: t_roof = max(bytes / HBM peak, FLOPs /
+    tensor peak) with the bytes of the mask build, the attention layer and
+    the verify calls, the FLOPs of the attention layer; frac = t_roof / the
+    measured step time."""
+    mask_bytes = w.B * w.Tmax * 4 * (1 + 1 + 1 + 1 + (w.Tmax + 31) // 32) + w.B * 8
+    vb = verify_traffic(w, step)
+    total = attn_bytes(w) + mask_bytes + sum(vb.values())
+    flops = attn_flops(w)
+    t_hbm = total / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    t_roof = max(t_hbm, t_tc)
+    return {"bound": "tensor" if t_tc > t_hbm else "hbm", "t_roof_us": t_roof * 1e6,
+            "step_us": ms_per_step * 1e3, "frac": t_roof / (ms_per_step * 1e-3),
+            "bytes": total, "verify_bytes": vb, "flops": flops,
+            "peaks": {"hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"]}}
+
+
+def kernel_roofline(w, att_s: float, peaks: dict) -> dict:
+    """Roofline of the attention kernel alone (the dominant launch)."""
+    flops, abytes = attn_flops(w), attn_bytes(w)
+    t_hbm = abytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    if t_tc > t_hbm:
+        roof = {"bound": "tensor", "achieved": flops / att_s / 1e12,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": abytes / att_s / 1e9, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["attn_us"] = att_s * 1e6
+    roof["algorithmic_bytes"] = abytes
+    roof["algorithmic_flops"] = flops
+    return roof
 
 
 class Step:
@@ -263,26 +331,32 @@ def _traffic_record(kernel_src: str, workload: str):
 
 
 # ------------------------------------------------------------ CPU oracle
-def cpu_baseline(w, budget_s: float = 15.0):
+def cpu_baseline(w, budget_s: float = 15.0, keep=None):
     """Time the oracle (as it stands) on a bounded sample of the workload:
     whole sequences (attention over all heads + the verify call(s)), added
-    one at a time until ~budget_s of CPU work."""
+    one at a time until ~budget_s of CPU work.  With `keep` (a list), the
+    oracle's outputs of each sequence are appended to it (outside the timed
+    calls) for the parity record."""
     import oracle
     oracle.build()
     done_nodes, elapsed, seqs = 0, 0.0, 0
     for b in range(w.B):
         T = int(w.n_nodes[b])
         sub = _subset(w, b)
+        out = {"b": b}
         t0 = time.perf_counter()
         if T:
             rows = [(0, u, h) for u in range(T) for h in range(w.Hq)]
-            oracle.tree_attention_rows(sub.q, sub.k_cache, sub.v_cache, sub.prefix_len,
-                                       sub.n_nodes, sub.parent, sub.scale, rows)
+            out["attn"] = oracle.tree_attention_rows(sub.q, sub.k_cache, sub.v_cache,
+                                                     sub.prefix_len, sub.n_nodes, sub.parent,
+                                                     sub.scale, rows)
         if "greedy" in w.verify:
-            oracle.workload_greedy(sub)
+            out["greedy"] = oracle.workload_greedy(sub)
         if "stochastic" in w.verify:
-            oracle.workload_stochastic(sub)
+            out["stochastic"] = oracle.workload_stochastic(sub)
         elapsed += time.perf_counter() - t0
+        if keep is not None:
+            keep.append(out)
         done_nodes += T
         seqs += 1
         if elapsed >= budget_s:
@@ -291,6 +365,74 @@ def cpu_baseline(w, budget_s: float = 15.0):
             "kind": "oracle",
             "sample": f"{seqs} of {w.B} sequences ({done_nodes} nodes), full attention layer "
                       f"over all {w.Hq} heads + {'/'.join(w.verify)} verify, {elapsed:.1f} s"}
+
+
+ATOL = {"bf16": 2e-2, "f32": 1e-4}   # attention max-abs tolerance against the fp64 oracle
+
+
+def parity_record(w, step, ref_seqs) -> dict:
+    """The GPU step's outputs against the oracle's on the sequences the oracle
+    ran (every node and head of each): attention max-abs error, greedy paths
+    and tokens bit-exact, stochastic ones bit-exact except on sequences whose
+    oracle path has a decision within 1e-9 of its boundary (excused)."""
+    rec = {"sequences": len(ref_seqs), "attn_tol": ATOL[w.dtype]}
+    got = step.out.float().cpu().numpy().astype(np.float64)
+    worst, rows = 0.0, 0
+    for r in ref_seqs:
+        if "attn" not in r:
+            continue
+        b, T = r["b"], int(w.n_nodes[r["b"]])
+        g = got[b, :T].reshape(T * w.Hq, w.D)
+        worst = max(worst, float(np.abs(g - r["attn"]).max()))
+        rows += T * w.Hq
+    rec.update(attn_max_abs=worst, attn_rows_compared=rows, attn_ok=worst <= ATOL[w.dtype])
+    for mode, res in (("greedy", step.g), ("stochastic", step.s)):
+        if mode not in w.verify:
+            continue
+        n = res.n_accepted.cpu().numpy()
+        path, toks = res.out_path.cpu().numpy(), res.out_tokens.cpu().numpy()
+        mism = excused = decisions = flagged = 0
+        for r in ref_seqs:
+            ref, b = r[mode], r["b"]
+            k = int(ref["n_accepted"][0])
+            same = int(n[b]) == k and (k < 0 or (
+                (path[b, :k] == ref["out_path"][0, :k]).all() and
+                (toks[b, :k + 1] == ref["out_tokens"][0, :k + 1]).all()))
+            if mode == "stochastic":
+                decisions += int(ref["n_decisions"].sum())
+                flagged += int(ref["n_flagged"].sum())
+                if not same and int(ref["n_flagged"][0]) > 0:
+                    excused += 1
+                    continue
+            mism += 0 if same else 1
+        if mode == "greedy":
+            rec["greedy"] = {"mismatches": mism, "exact": mism == 0}
+        else:
+            rec["stochastic"] = {"mismatches": mism, "excused": excused,
+                                 "flagged_decisions": flagged, "decisions": decisions,
+                                 "exact": mism == 0 and excused <= 1e-4 * max(decisions, 1)}
+    rec["ok"] = rec["attn_ok"] and all(rec[m]["exact"] for m in ("greedy", "stochastic")
+                                       if m in rec)
+    return rec
+
+
+def oracle_single_thread(name: str, budget_s: float = 6.0):
+    """The oracle on one host core (OMP_NUM_THREADS=1), on one sequence of
+    the named workload, through this script's reference arm in a child
+    process (the thread count is fixed when the oracle's OpenMP runtime
+    starts)."""
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    try:
+        r = subprocess.run([sys.executable, os.path.abspath(__file__), "--impl", "reference",
+                            "--workload", name, "--steps", "1", "--warmup", "0", "--batch", "1",
+                            "--oracle-budget", str(budget_s)],
+                           env=env, capture_output=True, text=True, timeout=300)
+        line = json.loads(r.stdout.strip().splitlines()[-1])
+        cb = line["cpu_baseline"]
+        return {"workload": name, "value": cb["value"], "unit": UNIT, "cores": cb["cores"],
+                "kind": "oracle", "sample": cb["sample"]}
+    except (subprocess.SubprocessError, ValueError, KeyError, IndexError, OSError) as e:
+        return {"workload": name, "error": str(e)[:200]}
 
 
 def _subset(w, b):
@@ -308,6 +450,110 @@ def _workload_name(w):
     return w.name
 
 
+def time_steps(step, w, dev, tsd, steps: int, warmup: int, pg=None, local: int = 0,
+               clocks: bool = False) -> dict:
+    """Warm-up, then `steps` timed steps: the mask build and the attention
+    call replayed from CUDA graphs, the verify calls eager; a barrier and a
+    synchronize on both sides of the timed region; CUDA events per step and
+    around the attention call.  The L2 is flushed between steps unless the
+    step already reads more than three times its size."""
+    for _ in range(max(3, warmup)):
+        step.run()
+    torch.cuda.synchronize(dev)
+    if int(tsd.device_status(dev).item()) != 0:
+        raise RuntimeError(f"device status set during warm-up ({w.name})")
+    flush = None
+    working = w.kv_bytes() + w.logits.numel() * 4 + w.q_probs.numel() * 4
+    if working < 3 * L2_BYTES:
+        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    graph_launches = step.capture()
+    for _ in range(2):
+        step.run_graphed((torch.cuda.Event(), torch.cuda.Event()))
+    torch.cuda.synchronize(dev)
+    att_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+    st_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(steps)]
+    sampler = _clock_sampler(local) if clocks else None
+    if sampler is not None:
+        time.sleep(0.3)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = tsd.launch_count()
+    for i in range(steps):
+        if flush is not None:
+            flush.fill_(float(i))
+        st_ev[i][0].record()
+        step.run_graphed(att_ev[i])
+        st_ev[i][1].record()
+    torch.cuda.synchronize(dev)
+    launches = tsd.launch_count() - launches0 + graph_launches * steps
+    step.release()
+    if pg:
+        pg.barrier()
+    clk = _clock_summary(sampler) if sampler is not None else None
+    if int(tsd.device_status(dev).item()) != 0:
+        raise RuntimeError(f"device status set during the timed steps ({w.name})")
+    return {"step_ms": [a.elapsed_time(b) for a, b in st_ev],
+            "att_ms": [a.elapsed_time(b) for a, b in att_ev],
+            "launches": launches, "clocks": clk,
+            "l2": "flushed between steps (2x L2 write)" if flush is not None
+            else f"inputs larger than L2 ({working / 1e6:.0f} MB read per step)"}
+
+
+def workload_record(name, w, step, t, peaks, dev, tsd, parity_budget_s: float) -> dict:
+    """One workload's figures for the `workloads` table of the line: tokens/s,
+    step time, attention time and roofline, the step roofline, KV-cache
+    bandwidth, acceptance, the attention plan, and parity against the oracle
+    on a bounded sample of whole sequences."""
+    ms = statistics.mean(t["step_ms"])
+    att_s = statistics.mean(t["att_ms"]) / 1e3
+    kv_gbs = w.kv_bytes() / att_s / 1e9
+    ref = []
+    cpu_baseline(w, budget_s=parity_budget_s, keep=ref)
+    return {"workload": w.name, "value": int(w.n_nodes.sum()) / (ms / 1e3), "unit": UNIT,
+            "ms_per_step": ms, "steps": len(t["step_ms"]), "dtype": w.dtype,
+            "roofline": kernel_roofline(w, att_s, peaks),
+            "roofline_step": step_roofline(w, step, ms, peaks),
+            "kv_cache_gbs": kv_gbs, "kv_cache_frac_of_hbm": kv_gbs / peaks["hbm_gbs"],
+            "acceptance": accepted_summary(w, step), "plan": _plan(w, dev, tsd),
+            "parity": parity_record(w, step, ref), "l2": t["l2"]}
+
+
+def _plan(w, dev, tsd):
+    return tsd.attention_plan(
+        w.B, w.Tmax, w.Hq, w.Hkv, w.D, int(w.k_cache.shape[2]),
+        torch.bfloat16 if w.dtype == "bf16" else torch.float32,
+        torch.cuda.get_device_properties(dev).multi_processor_count)
+
+
+def acceptance_other_proposal(cfg, dev, tsd) -> dict:
+    """Acceptance of the headline workload's trees under the other token
+    proposal (top-k tokens of rows perturbed by N(0, 0.3^2) instead of draws
+    from rows perturbed by N(0, 1)): the same trees and target logits, only
+    the speculated tokens and SSM rows differ.  Verify calls only."""
+    other = "topk" if cfg in (3, 4) else None
+    if other is None:
+        return None
+    w = gen.config_workload(cfg, with_attention=False, proposal=other)
+    d = {f: getattr(w, f).to(dev) for f in ("parent", "n_nodes", "tokens", "q_row", "logits",
+                                            "q_probs", "u_accept", "u_sample")}
+    tree = tsd.tree_mask_build(d["parent"], d["n_nodes"])
+    out = {}
+    if "greedy" in w.verify:
+        r = tsd.tree_verify_greedy(d["logits"], d["tokens"], d["parent"], d["n_nodes"], tree)
+        out["greedy"] = float(r.n_accepted.double().mean())
+    if "stochastic" in w.verify:
+        r = tsd.tree_verify_stochastic(d["logits"], w.temperature, d["q_probs"], d["q_row"],
+                                       d["tokens"], d["n_nodes"], tree, d["u_accept"],
+                                       d["u_sample"])
+        out["stochastic"] = float(r.n_accepted.double().mean())
+    torch.cuda.synchronize(dev)
+    return {"proposal": "top-k tokens, SSM noise N(0, 0.3^2)",
+            "mean_accepted_nodes": out}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -319,6 +565,12 @@ def main():
                     help="sequences per GPU (default: the workload's batch)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-side", action="store_true",
+                    help="skip the side measurements (commit, paged attention, tree build)")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="time only the headline workload (no table of the other four)")
+    ap.add_argument("--oracle-budget", type=float, default=None,
+                    help="reference arm: seconds of oracle work per timed step")
     args = ap.parse_args()
     ws, rank, local = _dist()
     cfg = gen.WORKLOAD_NAMES[args.workload]
@@ -329,8 +581,9 @@ def main():
         w = gen.config_workload(cfg, B=args.batch)
         times = []
         cb = None
+        budget = args.oracle_budget or 6.0
         for i in range(args.warmup + args.steps):
-            cb = cpu_baseline(w, budget_s=2.0 if i < args.warmup else 6.0)
+            cb = cpu_baseline(w, budget_s=min(2.0, budget) if i < args.warmup else budget)
             if i >= args.warmup:
                 times.append(cb["value"])
         val = statistics.median(times)
@@ -360,83 +613,28 @@ def main():
     w = rank_workload(cfg, rank, args.batch)
     step = Step(w, dev, tsd)
     tokens_per_step = int(w.n_nodes.sum())
-
-    for _ in range(max(3, args.warmup)):
-        step.run()
-    torch.cuda.synchronize(dev)
-    if int(tsd.device_status(dev).item()) != 0:
-        raise RuntimeError("device status set during warm-up")
-
-    flush = None
-    working = w.kv_bytes() + w.logits.numel() * 4 + w.q_probs.numel() * 4
-    if working < 3 * L2_BYTES:
-        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
-
-    graph_launches = step.capture()
-    for _ in range(2):
-        step.run_graphed((torch.cuda.Event(), torch.cuda.Event()))
-    torch.cuda.synchronize(dev)
-    n_att = args.steps
-    att_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(n_att)]
-    st_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-             for _ in range(args.steps)]
-    clocks = _clock_sampler(local)
-    time.sleep(0.3)
-    if pg:
-        pg.barrier()
-    torch.cuda.synchronize(dev)
-    launches0 = tsd.launch_count()
-    for i in range(args.steps):
-        if flush is not None:
-            flush.fill_(float(i))
-        st_ev[i][0].record()
-        step.run_graphed(att_ev[i])
-        st_ev[i][1].record()
-    torch.cuda.synchronize(dev)
-    launches = tsd.launch_count() - launches0 + graph_launches * args.steps
-    step.release()
-    if pg:
-        pg.barrier()
-    clk = _clock_summary(clocks)
-    step_ms = [a.elapsed_time(b) for a, b in st_ev]
-    att_ms = [a.elapsed_time(b) for a, b in att_ev]
-    job_tokens, total_ms = reduce_over_ranks(pg, dev, tokens_per_step, float(sum(step_ms)))
+    t = time_steps(step, w, dev, tsd, args.steps, args.warmup, pg, local, clocks=True)
+    job_tokens, total_ms = reduce_over_ranks(pg, dev, tokens_per_step, float(sum(t["step_ms"])))
     ms_per_step = total_ms / args.steps
     value = job_tokens / (ms_per_step / 1e3)
-    if int(tsd.device_status(dev).item()) != 0:
-        raise RuntimeError("device status set during the timed steps")
     acceptance = accepted_summary(w, step)
-    commit = time_commit(step, dev, tsd)
-    paged = time_paged_attention(step, dev, tsd) if w.dtype == "bf16" else None
-    build = time_tree_build(w, dev, tsd)
+    side = {}
+    if not args.no_side:
+        side["kv_commit"] = time_commit(step, dev, tsd)
+        side["paged_attention"] = time_paged_attention(step, dev, tsd) \
+            if w.dtype == "bf16" else None
+        side["tree_build"] = time_tree_build(w, dev, tsd)
 
     peaks, peak_kind = _peaks()
-    att_s = statistics.mean(att_ms) / 1e3
-    flops = attn_flops(w)
-    abytes = attn_bytes(w)
-    t_hbm = abytes / (peaks["hbm_gbs"] * 1e9)
-    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
-    if t_tc > t_hbm:
-        roof = {"bound": "tensor", "achieved": flops / att_s / 1e12,
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
-    else:
-        roof = {"bound": "hbm", "achieved": abytes / att_s / 1e9, "peak": peaks["hbm_gbs"],
-                "unit": "GB/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
+    att_s = statistics.mean(t["att_ms"]) / 1e3
+    roof = kernel_roofline(w, att_s, peaks)
     roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json burst)" if peak_kind == \
         "measured" else "fallback"
     kernel_src = os.path.join(ROOT, "tree_speculative_decoding_ancestor_b200", "csrc",
                               "attention_umma.cu")
     roof["traffic"] = _traffic_record(kernel_src, args.workload)
     roof["kernel"] = "tree attention (mask-aware split-KV), one layer"
-    roof["plan"] = tsd.attention_plan(
-        w.B, w.Tmax, w.Hq, w.Hkv, w.D, int(w.k_cache.shape[2]),
-        torch.bfloat16 if w.dtype == "bf16" else torch.float32,
-        torch.cuda.get_device_properties(dev).multi_processor_count)
-    roof["attn_us"] = att_s * 1e6
-    roof["algorithmic_bytes"] = abytes
-    roof["algorithmic_flops"] = flops
+    roof["plan"] = _plan(w, dev, tsd)
     kv_gbs = w.kv_bytes() / att_s / 1e9
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
@@ -446,19 +644,41 @@ def main():
             "config": {"workload": _workload_name(w), "batch_per_gpu": w.B,
                        "tree_nodes_per_step_per_gpu": tokens_per_step, "Hq": w.Hq,
                        "Hkv": w.Hkv, "head_dim": w.D, "prefix": int(w.prefix_len[0]),
-                       "vocab": w.V, "verify": list(w.verify),
-                       "l2": "flushed between steps (2x L2 write)" if flush is not None
-                       else f"inputs larger than L2 ({working / 1e6:.0f} MB read per step)",
+                       "vocab": w.V, "verify": list(w.verify), "l2": t["l2"],
                        "parallelism": f"batch-sharded x{ws} (independent sequences)"},
             "kv_cache_gbs": kv_gbs, "kv_cache_frac_of_hbm": kv_gbs / peaks["hbm_gbs"],
-            "roofline": roof, "gpu_launches": launches, "clocks": clk,
-            "acceptance": acceptance,
-            "kv_commit": commit, "paged_attention": paged, "tree_build": build}
+            "roofline": roof,
+            "roofline_step": step_roofline(w, step, statistics.mean(t["step_ms"]), peaks),
+            "gpu_launches": t["launches"], "clocks": t["clocks"],
+            "acceptance": acceptance}
+    line.update(side)
 
     if not args.no_e2e:
         line["e2e"] = e2e(w, dev, tsd, args, pg, ws)
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w)
+        ref = []
+        line["cpu_baseline"] = cpu_baseline(w, keep=ref)
+        line["parity"] = parity_record(w, step, ref)
+        line["cpu_baseline_1thread"] = oracle_single_thread("llama7b")
+    if ws == 1 and not args.no_workloads:
+        alt = acceptance_other_proposal(cfg, dev, tsd)
+        if alt:
+            line["acceptance_other_proposal"] = alt
+        rec = {args.workload: workload_record(args.workload, w, step, t, peaks, dev, tsd,
+                                              parity_budget_s=0.0)}
+        rec[args.workload]["parity"] = line.get("parity", rec[args.workload]["parity"])
+        del step
+        torch.cuda.empty_cache()
+        for name in sorted(gen.WORKLOAD_NAMES, key=gen.WORKLOAD_NAMES.get):
+            if name == args.workload:
+                continue
+            wk = gen.config_workload(gen.WORKLOAD_NAMES[name])
+            sk = Step(wk, dev, tsd)
+            tk = time_steps(sk, wk, dev, tsd, min(args.steps, 20), 3)
+            rec[name] = workload_record(name, wk, sk, tk, peaks, dev, tsd, parity_budget_s=3.0)
+            del sk, wk
+            torch.cuda.empty_cache()
+        line["workloads"] = rec
     if rank == 0:
         print(json.dumps(line), flush=True)
     if pg:

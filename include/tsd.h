@@ -274,6 +274,21 @@ int tsd_tree_verify_stochastic(const float *logits, double temperature, const fl
                                tsd_stream_t stream);
 
 /*
+ * The grid tsd_tree_verify_stochastic (and its _noalloc form) launches for B
+ * sequences over a vocabulary of V on the current device (host only,
+ * nothing is launched; it reads the device's SM count and the walk kernel's
+ * occupancy):
+ *   plan[0]  teams: sequences walked at the same time (team t walks
+ *            sequences t, t + teams, t + 2 teams, ...)
+ *   plan[1]  CTAs per team, each owning one chunk of the vocabulary
+ *   plan[2]  vocabulary entries per chunk
+ *   plan[3]  CTAs in the cooperative launch (teams x CTAs per team)
+ * Errors: TSD_ERR_NULL (plan), TSD_ERR_SHAPE (B < 1, Tmax out of range,
+ * V < 1), TSD_ERR_CUDA (no device or no cooperative launch).
+ */
+int tsd_tree_verify_stochastic_plan(int B, int Tmax, int V, int32_t *plan);
+
+/*
  * Token-tree construction ("マルチドラフトモデルアプローチ": item 1,
  * expansion-based trees <k_1, ..., k_n> take one SSM's top-k_i tokens at
  * every node of depth i-1; item 2, merge-based trees merge the outputs of

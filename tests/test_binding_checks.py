@@ -140,3 +140,25 @@ def test_host_tensors_are_refused_before_the_library():
     q = torch.zeros(B, Tmax, Hq, D, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA device"):
         tsd.tree_attention(q, q, q, parent[:, 0], parent[:, 0], parent)
+
+
+def test_cached_workspaces_are_per_stream(lib, monkeypatch):
+    # Calls without a workspace on two streams must not share a buffer (their
+    # kernels may overlap); calls on one stream reuse the same buffer.
+    monkeypatch.setattr(binding, "_workspace", {})
+    dev = torch.device("cpu")
+    seen = {}
+    for handle in (11, 22, 11):
+        monkeypatch.setattr(binding, "_stream", lambda d, h=handle: h)
+        ws = binding._workspace_for(dev, "verify", 512, None)
+        assert ws.numel() >= 512
+        seen.setdefault(handle, []).append(ws.data_ptr())
+    assert seen[11][0] == seen[11][1]
+    assert seen[11][0] != seen[22][0]
+    # through an entry point: the stochastic verifier on two streams
+    bufs = []
+    for handle in (33, 44):
+        monkeypatch.setattr(binding, "_stream", lambda d, h=handle: h)
+        _stochastic()
+        bufs.append(binding._workspace[(None, "verify", handle)].data_ptr())
+    assert bufs[0] != bufs[1]

@@ -138,3 +138,20 @@ def test_host_checks_of_every_entry_point(lib):
     assert probe(1, 3_000_000_000, _A, _A, None) == ERR_SHAPE    # above 2 s
     assert probe(0, 50_000_000, None, _A, None) == ERR_NULL
     assert probe(0, 50_000_000, _U, _A, None) == ERR_ALIGN
+
+
+def test_launching_entry_points_open_an_nvtx_range():
+    # Every C-ABI call that launches work is a named range on a profiler's
+    # timeline: its body starts with TSD_NVTX_RANGE().
+    csrc = os.path.join(ROOT, "tree_speculative_decoding_ancestor_b200", "csrc")
+    bodies = {}
+    for f in ("capi.cu", "verify_noalloc.cu"):
+        src = open(os.path.join(csrc, f)).read()
+        for m in re.finditer(r"\n(?:extern \"C\" )?int (tsd_[a-z0-9_]+)\(([^{]*)\)\n\{\n(.*?)\n\}\n",
+                             src, flags=re.S):
+            bodies[m.group(1)] = m.group(3)
+    launching = {n for n, body in bodies.items() if "launch" in body or "<<<" in body}
+    assert {"tsd_tree_attention", "tsd_tree_verify_stochastic_noalloc",
+            "tsd_kv_commit"} <= launching
+    for n in launching:
+        assert bodies[n].lstrip().startswith("TSD_NVTX_RANGE();"), n

@@ -137,6 +137,83 @@ def test_attention_parity_at_the_row_block_boundary(cuda_device, Tmax, env, monk
     assert _status(cuda_device) == 0
 
 
+# Forced key-range split counts (TSD_ATTN_SPLITS) on every kernel: one split
+# takes each kernel's direct normalised write, one key tile per split the
+# partials + log-sum-exp combine (and leaves the key-split kernel's second
+# softmax group without tiles).  The large shape has up to 256 packed rows
+# per (sequence, KV head) -- two row blocks on the 128-key rows kernel, the
+# plan the 70B-GQA benchmark runs with one split -- and is compared on every
+# row.
+LARGE = dict(seed=81, B=4, Tmax=64, Hq=32, Hkv=8, D=128, P_max=1500, P_min=900, min_nodes=36)
+SMALL = dict(seed=82, B=3, Tmax=24, Hq=16, Hkv=4, D=128, P_max=900, P_min=300, min_nodes=8)
+FORCED = [
+    # (shape, environment, expected kernel)
+    ("large", {}, "rows128"),
+    ("large", {"TSD_ATTN_ROWS_VARIANT": "2"}, "rows64"),
+    ("small", {}, "rows64"),
+    ("small", {"TSD_ATTN_SMALL_VARIANT": "keysplit"}, "keysplit"),
+    ("small", {"TSD_FORCE_PATH": "simt"}, "simt"),
+]
+
+
+def _shape_workload(name):
+    c = dict(LARGE if name == "large" else SMALL)
+    return gen.random_workload(c.pop("seed"), dtype="bf16", max_children=4, max_depth=12,
+                               lmax_pad=37, V=16, **c)
+
+
+@pytest.mark.parametrize("splits", ["1", "3", "64"])
+@pytest.mark.parametrize("forced", FORCED, ids=[f"{f[0]}-{f[2]}" for f in FORCED])
+def test_attention_parity_forced_splits(cuda_device, forced, splits, monkeypatch):
+    shape, env, kernel = forced
+    for k, v in env.items():
+        monkeypatch.setenv(k, v)
+    monkeypatch.setenv("TSD_ATTN_SPLITS", splits)
+    w = _shape_workload(shape)
+    sms = torch.cuda.get_device_properties(cuda_device).multi_processor_count
+    plan = tsd.attention_plan(w.B, w.Tmax, w.Hq, w.Hkv, w.D, w.Lmax, torch.bfloat16, sms)
+    assert plan["kernel"] == kernel
+    tiles = -(-w.Lmax // (128 if kernel in ("rows128", "keysplit") else
+                          64 if kernel == "rows64" else 32))
+    assert plan["splits"] == min(int(splits), tiles if kernel != "simt" else plan["splits"])
+    if shape == "large" and kernel == "rows128":
+        assert plan["row_blocks"] == 2 and max(w.n_nodes.tolist()) * w.G > 128
+    d = to_dev(w, cuda_device)
+    poison(w, d)
+    tree = run_tree(d)
+    out = torch.full_like(d["q"], 1234.0)
+    tsd.tree_attention(d["q"], d["k_cache"], d["v_cache"], d["prefix_len"], d["n_nodes"],
+                       tree.mask, out=out)
+    check_attention(w, out, sentinel=1234.0)
+    assert _status(cuda_device) == 0
+
+
+@pytest.mark.parametrize("splits", ["1", "2"])
+@pytest.mark.parametrize("forced", FORCED, ids=[f"{f[0]}-{f[2]}" for f in FORCED])
+def test_attention_row_without_keys_is_zero(cuda_device, forced, splits, monkeypatch):
+    # A caller-supplied mask row without the node's own bit, in a sequence with
+    # no prefix, leaves that query row no key at all: every kernel writes it as
+    # zeros, whatever the split count; the other rows keep the oracle's values.
+    shape, env, kernel = forced
+    for k, v in env.items():
+        monkeypatch.setenv(k, v)
+    monkeypatch.setenv("TSD_ATTN_SPLITS", splits)
+    w = _shape_workload(shape)
+    w.prefix_len[0] = 0
+    ref = oracle.workload_attention(w)
+    d = to_dev(w, cuda_device)
+    tree = run_tree(d)
+    u0 = 0   # the root's first child: its only key is itself
+    tree.mask[0, u0].zero_()
+    out = tsd.tree_attention(d["q"], d["k_cache"], d["v_cache"], d["prefix_len"], d["n_nodes"],
+                             tree.mask)
+    got = out.float().cpu()
+    assert (got[0, u0] == 0).all().item()
+    ref[0, u0] = got[0, u0].numpy()
+    check_attention(w, out, ref=ref)
+    assert _status(cuda_device) == 0
+
+
 def test_attention_empty_trees_and_prefix(cuda_device):
     # T_b = 0 sequences, P_b = 0 sequences, and a single-node tree with no prefix
     w = gen.random_workload(21, B=4, Tmax=8, Hq=4, Hkv=2, D=128, P_max=50, dtype="bf16",
@@ -207,13 +284,15 @@ VERIFY_CASES = [
     (36, 6, 40, 777, "topk", 0.5),
     (37, 2, 16, 128256, "topk", 1.0),    # 32-CTA teams, 4008 entries each
     (38, 3, 12, 50001, "sample", 0.9),   # last chunk ends at V, V % 4 != 0
-    (39, 700, 8, 64, "sample", 1.0),     # more sequences than the grid holds
+    (39, 1100, 8, 64, "sample", 1.0),    # more sequences than the grid holds
 ]
 
 
 @pytest.mark.parametrize("case", VERIFY_CASES, ids=[f"s{c[0]}" for c in VERIFY_CASES])
 def test_verify_parity(cuda_device, case):
     seed, B, Tmax, V, mode, temp = case
+    if seed == 39:   # one-CTA teams that each walk several sequences
+        assert tsd.verify_stochastic_plan(B, Tmax, V)["teams"] < B
     w = gen.random_workload(seed, B=B, Tmax=Tmax, V=V, min_nodes=0, max_children=5,
                             max_depth=10, token_mode=mode, q_sigma=0.3, temperature=temp,
                             with_attention=False)
@@ -299,6 +378,9 @@ def _sample_rows(w, n, seed):
 
 @pytest.mark.parametrize("cfg", [0, 1, 2, 3, 4])
 def test_config_full_size(cuda_device, cfg):
+    # The launch the benchmark times (same sizes, same plan), compared with
+    # the oracle on every row of the first and last sequence (all nodes, all
+    # heads) and on rows sampled from the whole batch.
     w = gen.config_workload(cfg)
     d = to_dev(w, cuda_device)
     tree = run_tree(d)
@@ -309,6 +391,8 @@ def test_config_full_size(cuda_device, cfg):
         check_attention(w, out)
     else:
         rows = _sample_rows(w, 48, cfg)
+        for b in sorted({0, w.B - 1}):
+            rows += [(b, u, h) for u in range(int(w.n_nodes[b])) for h in range(w.Hq)]
         ref = oracle.tree_attention_rows(w.q, w.k_cache, w.v_cache, w.prefix_len, w.n_nodes,
                                          w.parent, w.scale, rows)
         got = out.float().cpu().numpy()

@@ -5,10 +5,11 @@ KV-cache pool already owns nearly all device memory, or a caller that reaches
 the library through a plain C interface with no device allocator.  This entry
 point keeps its scratch in a fixed array inside the library instead.  These
 tests call it through the C ABI (ctypes, no Python wrapper in between) and
-check that it returns exactly what the workspace entry point returns, on two
-calls in a row (the second call finds the first call's leftovers in the
-shared array), and that its fixed scratch does not limit the shape: a batch
-with more sequences than the verifier's grid has CTAs still runs.
+check that it returns exactly what the workspace entry point returns, and
+what the fp64 oracle returns, on two calls in a row (the second call finds
+the first call's leftovers in the shared array), and that its fixed scratch
+does not limit the shape: a batch with more sequences than the verifier's
+grid has CTAs still runs, one-CTA teams walking several sequences each.
 
 This file is collected last on purpose, so that a run stopping at the first
 failure has already run every other test.
@@ -19,7 +20,9 @@ import ctypes
 import pytest
 import torch
 
+import oracle
 import tree_speculative_decoding_ancestor_b200 as tsd
+from gpu_util import check_stochastic
 from workloads import gen
 
 pytestmark = pytest.mark.gpu
@@ -72,15 +75,22 @@ def test_noalloc_matches_workspace_call_twice(cuda_device):
         assert torch.equal(got.out_tokens, want.out_tokens)
         assert torch.equal(got.out_path, want.out_path)
         assert (got.n_accepted >= 0).all().item()
+        check_stochastic(w, got, oracle.workload_stochastic(w))
     assert int(status.item()) == 0
 
 
 def test_noalloc_takes_a_batch_larger_than_the_grid(cuda_device):
     lib = tsd.load_library()
-    # 700 sequences: more than the cooperative grid holds at once, so teams
-    # walk several sequences each and the barrier counters run on.
+    # 1100 sequences over a 64-token vocabulary: one CTA per team, and more
+    # sequences than the cooperative grid holds (it is capped at 1024 CTAs),
+    # so teams walk several sequences each and their barrier counters run on
+    # from one sequence to the next.
     dev = cuda_device
-    w, d, tree = _inputs(77, dev, B=700, Tmax=24, V=64)
+    B, Tmax, V = 1100, 24, 64
+    plan = tsd.verify_stochastic_plan(B, Tmax, V)
+    assert plan["ctas_per_team"] == 1
+    assert plan["teams"] < B, plan
+    w, d, tree = _inputs(77, dev, B=B, Tmax=Tmax, V=V)
     want = tsd.tree_verify_stochastic(d["logits"], w.temperature, d["q_probs"], d["q_row"],
                                       d["tokens"], d["n_nodes"], tree, d["u_accept"],
                                       d["u_sample"], out=_outputs(w.B, w.Tmax, dev))
@@ -96,3 +106,4 @@ def test_noalloc_takes_a_batch_larger_than_the_grid(cuda_device):
     assert torch.equal(out.out_tokens, want.out_tokens)
     assert torch.equal(out.out_path, want.out_path)
     assert (out.n_accepted >= 0).all().item()
+    check_stochastic(w, out, oracle.workload_stochastic(w))

@@ -35,5 +35,6 @@ from .binding import (  # noqa: F401
     tree_verify_greedy,
     tree_verify_stochastic,
     tree_verify_stochastic_noalloc,
+    verify_stochastic_plan,
     verify_workspace_size,
 )

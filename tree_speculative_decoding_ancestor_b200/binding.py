@@ -50,6 +50,7 @@ _SIGNATURES: Dict[str, Tuple[object, list]] = {
                                         _I, _I, _I, _P, _P, _P, _P, _SZ, _P, _P]),
     "tsd_tree_verify_stochastic_noalloc": (_I, [_P, ctypes.c_double, _P, _I, _P, _P, _P, _P, _P,
                                                 _P, _P, _I, _I, _I, _P, _P, _P, _P, _P]),
+    "tsd_tree_verify_stochastic_plan": (_I, [_I, _I, _I, _P]),
     "tsd_kv_commit": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
     "tsd_tree_attention_paged": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _I, _I, _I, _I,
                                       _I, ctypes.c_float, _I, _P, _P, _SZ, _P, _P]),
@@ -127,7 +128,11 @@ def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape: Tuple[int, ...]
 
 # Per-device status word and workspace cache ---------------------------------
 _status: Dict[int, torch.Tensor] = {}
-_workspace: Dict[Tuple[int, str], torch.Tensor] = {}
+# Workspaces the binding allocates when the caller passes none, one per
+# (device, kind, stream): calls on one stream run one after another, so they
+# can share a buffer; calls on different streams may overlap on the GPU, and
+# a workspace must not be shared by calls that may overlap.
+_workspace: Dict[Tuple[int, str, int], torch.Tensor] = {}
 
 
 def device_status(device=None) -> torch.Tensor:
@@ -140,12 +145,17 @@ def device_status(device=None) -> torch.Tensor:
 
 
 def _get_workspace(device: torch.device, kind: str, nbytes: int) -> torch.Tensor:
-    key = (device.index, kind)
-    ws = _workspace.get(key)
-    if ws is None or ws.numel() < nbytes:
-        ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
-        _workspace[key] = ws
-    return ws
+    """The cached workspace of this kind for the caller's current stream on
+    `device` (grown when too small; the caching allocator keeps a replaced
+    buffer's memory for that stream's later work, so a kernel still running on
+    it is not disturbed)."""
+    with _lock:
+        key = (device.index, kind, int(_stream(device)))
+        ws = _workspace.get(key)
+        if ws is None or ws.numel() < nbytes:
+            ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+            _workspace[key] = ws
+        return ws
 
 
 def _workspace_for(device: torch.device, kind: str, nbytes: int,
@@ -359,6 +369,16 @@ def tree_verify_stochastic(logits: torch.Tensor, temperature: float, q_probs: to
     return out
 
 
+def verify_stochastic_plan(B: int, Tmax: int, V: int) -> Dict[str, int]:
+    """The grid tree_verify_stochastic launches for these sizes on the current
+    device (host only): teams walking at once, CTAs per team, vocabulary
+    entries per CTA, CTAs in the launch."""
+    plan = (ctypes.c_int32 * 4)()
+    rc = load_library().tsd_tree_verify_stochastic_plan(B, Tmax, V, ctypes.addressof(plan))
+    _check(rc, "tsd_tree_verify_stochastic_plan")
+    return {"teams": plan[0], "ctas_per_team": plan[1], "chunk": plan[2], "ctas": plan[3]}
+
+
 def tree_verify_stochastic_noalloc(logits: torch.Tensor, temperature: float,
                                    q_probs: torch.Tensor, q_row: torch.Tensor,
                                    tokens: torch.Tensor, n_nodes: torch.Tensor, tree: TreeMask,
@@ -453,7 +473,7 @@ def tree_attention_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.
     _need(out, "out", q.dtype, (B, Tmax, Hq, D), dev)
     Lmax = max_blocks * page_size
     need = int(lib.tsd_tree_attention_workspace_size(B, Tmax, Hq, Hkv, D, Lmax, dt))
-    ws = _workspace_for(dev, "attention", need, workspace)
+    ws = _workspace_for(dev, "attn", need, workspace)
     st = _status_for(dev, status)
     sc = (1.0 / D ** 0.5) if scale is None else float(scale)
     rc = lib.tsd_tree_attention_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table),

@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(kSimtThreads)
         const int u = r / G, h = hk * G + r % G;
         const size_t row = ((size_t)b * Tmax + u) * Hq + h;
         if (nsplit == 1) {
-            const float inv = 1.f / l[rr];
+            const float inv = l[rr] > 0.f ? 1.f / l[rr] : 0.f;   // a row with no key: 0
 #pragma unroll
             for (int i = 0; i < DL; ++i)
                 out[row * D + lane + 32 * i] = from_float<Elt>(o[rr][i] * inv);
@@ -237,7 +237,9 @@ __global__ void __launch_bounds__(256)
         for (int i = 0; i < DL; ++i)
             acc[i] = fmaf(w, part_o[((size_t)s * nrows + row) * D + lane + 32 * i], acc[i]);
     }
-    const float inv = 1.f / L;
+    // a row that no split saw a key for (a caller mask without the node's own
+    // bit and no prefix) is written as zeros, as the single-split paths do
+    const float inv = L > 0.f ? 1.f / L : 0.f;
 #pragma unroll
     for (int i = 0; i < DL; ++i)
         out[row * D + lane + 32 * i] = from_float<Elt>(acc[i] * inv);

@@ -85,6 +85,7 @@ int tsd_tree_mask_build(const int32_t *parent, const int32_t *n_nodes, int B, in
                         uint32_t *mask, int32_t *depth, int32_t *first_child,
                         int32_t *next_sibling, int32_t *dev_status, tsd_stream_t stream)
 {
+    TSD_NVTX_RANGE();
     if (B < 0 || Tmax < 1 || Tmax > TSD_MAX_TREE)
         return TSD_ERR_SHAPE;
     if (B == 0)
@@ -133,6 +134,7 @@ int tsd_tree_attention(const void *q, const void *k_cache, const void *v_cache,
                        int dtype, void *out, void *workspace, size_t workspace_bytes,
                        int32_t *dev_status, tsd_stream_t stream)
 {
+    TSD_NVTX_RANGE();
     tsd::AttnArgs a;
     a.q = q; a.k = k_cache; a.v = v_cache; a.prefix_len = prefix_len; a.n_nodes = n_nodes;
     a.mask = mask; a.B = B; a.Tmax = Tmax; a.Hq = Hq; a.Hkv = Hkv; a.D = D; a.Lmax = Lmax;
@@ -161,6 +163,7 @@ int tsd_tree_attention_paged(const void *q, const void *k_pages, const void *v_p
                              float scale, int dtype, void *out, void *workspace,
                              size_t workspace_bytes, int32_t *dev_status, tsd_stream_t stream)
 {
+    TSD_NVTX_RANGE();
     if (page_size < 16 || page_size > 4096 || (page_size & (page_size - 1)) != 0 ||
         max_blocks < 1 || num_pages < 1 || (long long)max_blocks * page_size > (1LL << 30))
         return TSD_ERR_SHAPE;
@@ -207,6 +210,7 @@ int tsd_tree_verify_greedy(const float *logits, const int32_t *tokens, const int
                            void *workspace, size_t workspace_bytes, int32_t *dev_status,
                            tsd_stream_t stream)
 {
+    TSD_NVTX_RANGE();
     if (B < 0 || B > kMaxGridY || Tmax < 1 || Tmax > TSD_MAX_TREE || V < 1)
         return TSD_ERR_SHAPE;
     if (B == 0)
@@ -232,6 +236,7 @@ int tsd_tree_verify_stochastic(const float *logits, double temperature, const fl
                                void *workspace, size_t workspace_bytes, int32_t *dev_status,
                                tsd_stream_t stream)
 {
+    TSD_NVTX_RANGE();
     if (B < 0 || Tmax < 1 || Tmax > TSD_MAX_TREE || V < 1 || Rq < 1 || !(temperature > 0.0))
         return TSD_ERR_SHAPE;
     if (B == 0)
@@ -249,11 +254,21 @@ int tsd_tree_verify_stochastic(const float *logits, double temperature, const fl
                                          dev_status, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int tsd_tree_verify_stochastic_plan(int B, int Tmax, int V, int32_t *plan)
+{
+    if (!plan)
+        return TSD_ERR_NULL;
+    if (B < 1 || Tmax < 1 || Tmax > TSD_MAX_TREE || V < 1)
+        return TSD_ERR_SHAPE;
+    return tsd::verify_stochastic_plan(B, V, plan);
+}
+
 int tsd_kv_commit(void *k_cache, void *v_cache, const int32_t *prefix_len,
                   const int32_t *out_path, const int32_t *n_accepted, int B, int Tmax, int Hkv,
                   int D, int Lmax, int dtype, int32_t *new_prefix_len, int32_t *dev_status,
                   tsd_stream_t stream)
 {
+    TSD_NVTX_RANGE();
     if (B < 0 || B > kMaxGridY || Tmax < 1 || Tmax > TSD_MAX_TREE || Hkv < 1 || D < 1 ||
         Lmax < 1)
         return TSD_ERR_SHAPE;
@@ -278,6 +293,7 @@ int tsd_tree_expand(const float *q_probs, int Rq, int V, const int32_t *frow, in
                     int32_t *lvl_begin, int B, int Tmax, int32_t *dev_status,
                     tsd_stream_t stream)
 {
+    TSD_NVTX_RANGE();
     if (B < 0 || Tmax < 1 || Tmax > TSD_MAX_TREE || Rq < 1 || V < 1 || k < 1 || k > Tmax)
         return TSD_ERR_SHAPE;
     if (B == 0)
@@ -294,6 +310,7 @@ int tsd_tree_dfs_order(const int32_t *parent, const int32_t *tokens, const int32
                        int32_t *out_parent, int32_t *out_tokens, int32_t *out_q_row,
                        int32_t *dev_status, tsd_stream_t stream)
 {
+    TSD_NVTX_RANGE();
     if (B < 0 || Tmax < 1 || Tmax > TSD_MAX_TREE)
         return TSD_ERR_SHAPE;
     if (B == 0)
@@ -311,6 +328,7 @@ int tsd_tree_merge_chains(const int32_t *chain_tokens, const int32_t *chain_q_ro
                           int32_t *parent, int32_t *tokens, int32_t *q_row, int32_t *n_nodes,
                           int32_t *dev_status, tsd_stream_t stream)
 {
+    TSD_NVTX_RANGE();
     if (B < 0 || M < 1 || L < 1 || Tmax < 1 || Tmax > TSD_MAX_TREE)
         return TSD_ERR_SHAPE;
     if (B == 0)
@@ -325,6 +343,7 @@ int tsd_tree_merge_chains(const int32_t *chain_tokens, const int32_t *chain_q_ro
 int tsd_debug_wait_probe(int kind, unsigned long long limit_ns, void *scratch,
                          int32_t *dev_status, tsd_stream_t stream)
 {
+    TSD_NVTX_RANGE();
     if ((kind != 0 && kind != 1) || limit_ns < 1000000ull || limit_ns > 2000000000ull)
         return TSD_ERR_SHAPE;
     if (!scratch || !dev_status)

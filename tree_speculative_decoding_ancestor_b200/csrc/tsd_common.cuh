@@ -3,6 +3,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 #include "tsd.h"
@@ -58,6 +59,20 @@ __device__ __forceinline__ bool tree_header_ok(int T, int Tmax) { return T >= 0 
 }  // namespace tsd
 
 // Host-side launch helpers.
+
+// Every C-ABI call that launches work shows up as a range named after the
+// entry point on a profiler's timeline (NVTX; without an attached tool the
+// push and pop cost a call each and record nothing).
+namespace tsd {
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
+}  // namespace tsd
+#define TSD_NVTX_RANGE() tsd::NvtxRange tsd_nvtx_range_(__func__)
+
 #define TSD_CUDA_TRY(expr)                                                                    \
     do {                                                                                      \
         cudaError_t e_ = (expr);                                                              \
@@ -126,6 +141,7 @@ int launch_umma_attention(const AttnArgs &a, void *ws, size_t ws_bytes, int num_
 
 size_t verify_workspace(int B, int Tmax, int V);
 size_t verify_stochastic_scratch();   // fixed: independent of the shape
+int verify_stochastic_plan(int B, int V, int32_t out[4]);   // teams, K, chunk, CTAs
 int launch_tree_expand(const float *q_probs, int Rq, int V, const int32_t *frow, int k,
                        int32_t *parent, int32_t *tokens, int32_t *q_row, int32_t *n_nodes,
                        int32_t *lvl_begin, int B, int Tmax, int32_t *dev_status,

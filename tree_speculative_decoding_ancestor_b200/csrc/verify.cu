@@ -41,6 +41,7 @@
 // relative, so a decision can only differ when its uniform lies within that
 // distance of the boundary.
 #include <algorithm>
+#include <atomic>
 #include <climits>
 
 #include "fp64_exp.cuh"
@@ -819,12 +820,15 @@ namespace {
 // launch limit), capped by the workspace slots; looked up once per device.
 int walk_capacity(bool vec)
 {
+    // Threads making their first call on a device at the same time may both
+    // compute the value (the same one); the atomic makes that race benign.
     constexpr int kMaxDevices = 64;
-    static int cap[2][kMaxDevices] = {};
+    static std::atomic<int> cap[2][kMaxDevices];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
         return 0;
-    int &c = cap[vec ? 1 : 0][dev];
+    std::atomic<int> &slot = cap[vec ? 1 : 0][dev];
+    int c = slot.load(std::memory_order_relaxed);
     if (c == 0) {
         int sms = 0, occ = 0, coop = 0;
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -834,11 +838,47 @@ int walk_capacity(bool vec)
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, kWalkThreads, 0);
         (void)cudaGetLastError();
         c = coop ? std::min(sms * occ, kWalkMaxCtas) : -1;
+        slot.store(c, std::memory_order_relaxed);
     }
     return c;
 }
 
+// Grid of the walk for B sequences over a vocabulary of V on the current
+// device.  Team size: enough CTAs that each owns at least kTeamMinChunk
+// entries (at most kTeamMax), as long as every sequence still gets a team;
+// with more sequences than the grid holds, one-CTA teams each walk several.
+int walk_grid(int B, int V, int &K, int &teams, int &chunk)
+{
+    const int cap = walk_capacity((V & 3) == 0);
+    if (cap <= 0 || B < 1)
+        return TSD_ERR_CUDA;
+    const int k_want = std::max(1, std::min(kTeamMax, V / kTeamMinChunk));
+    if ((long)B * k_want <= cap) {
+        K = k_want;
+        teams = B;
+    } else {
+        K = std::max(1, cap / B);
+        teams = std::min(B, cap / K);
+    }
+    chunk = (V + K - 1) / K;
+    chunk = (chunk + 3) & ~3;
+    return TSD_OK;
+}
+
 }  // namespace
+
+int verify_stochastic_plan(int B, int V, int32_t out[4])
+{
+    int K, teams, chunk;
+    const int rc = walk_grid(B, V, K, teams, chunk);
+    if (rc != TSD_OK)
+        return rc;
+    out[0] = teams;
+    out[1] = K;
+    out[2] = chunk;
+    out[3] = teams * K;
+    return TSD_OK;
+}
 
 int launch_verify_stochastic(const float *logits, double temperature, const float *q_probs,
                              int Rq, const int32_t *q_row, const int32_t *tokens,
@@ -851,22 +891,9 @@ int launch_verify_stochastic(const float *logits, double temperature, const floa
     if (B == 0)
         return TSD_OK;
     const bool vec = (V & 3) == 0;
-    const int cap = walk_capacity(vec);
-    if (cap <= 0)
+    int K, teams, chunk;
+    if (walk_grid(B, V, K, teams, chunk) != TSD_OK)
         return TSD_ERR_CUDA;
-    // Team size: enough CTAs that each owns at least kTeamMinChunk entries
-    // (at most kTeamMax), as long as every sequence still gets a team.
-    const int k_want = std::max(1, std::min(kTeamMax, V / kTeamMinChunk));
-    int K, teams;
-    if ((long)B * k_want <= cap) {
-        K = k_want;
-        teams = B;
-    } else {
-        K = std::max(1, cap / B);
-        teams = std::min(B, cap / K);
-    }
-    int chunk = (V + K - 1) / K;
-    chunk = (chunk + 3) & ~3;
     VerifyWs w = carve(ws);
     if (cudaMemsetAsync(w.team, 0, (size_t)teams * sizeof(int2), stream) != cudaSuccess) {
         (void)cudaGetLastError();

@@ -60,6 +60,7 @@ extern "C" int tsd_tree_verify_stochastic_noalloc(
     int V, int32_t *out_tokens, int32_t *out_path, int32_t *n_accepted, int32_t *dev_status,
     tsd_stream_t stream)
 {
+    TSD_NVTX_RANGE();
     if (B < 0 || Tmax < 1 || Tmax > TSD_MAX_TREE || V < 1 || Rq < 1 || !(temperature > 0.0))
         return TSD_ERR_SHAPE;
     if (B == 0)

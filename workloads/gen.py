@@ -305,9 +305,11 @@ def _assemble(name: str, seed: int, B: int, Tmax: int, Hq: int, Hkv: int, D: int
                 pr = q_probs[b, int(q_row[b, u])].astype(np.float64)
                 pr = pr / pr.sum()
                 tokens[b, u] = int(rng.choice(V, p=pr))
-        elif token_mode == "chains":
+        elif token_mode in ("chains", "distinct"):
             # Merge trees: every chain samples its own tokens; a node where a
             # chain branches off must differ from its existing siblings.
+            # Other trees ("distinct"): every child is drawn from its row,
+            # again distinct from the siblings drawn before it.
             for u in range(T):
                 pr = q_probs[b, int(q_row[b, u])].astype(np.float64)
                 pr = pr / pr.sum()
@@ -381,19 +383,36 @@ SEED_BASE = 20261202
 WORKLOAD_NAMES = {"tiny": 0, "llama7b": 1, "merge": 2, "gqa70b": 3, "long32k": 4}
 
 
+# How the speculated tokens of the 70B-GQA and long-context workloads are
+# proposed: "sampled" (the default) follows their stated recipe -- SSM rows
+# softmax(target logits + N(0, 1)), each child's token drawn from its row,
+# siblings distinct; "topk" is the alternative reading kept for comparison
+# (the rows' top-k tokens at noise N(0, 0.3^2)), under which greedy
+# acceptance is not near zero.
+PROPOSALS = ("sampled", "topk")
+
+
 def config_workload(index: int, seed: Optional[int] = None, B: Optional[int] = None,
-                    with_attention: bool = True) -> Workload:
+                    with_attention: bool = True, proposal: str = "sampled") -> Workload:
     """Build configuration ``index`` (0..4).  ``B`` may shrink the batch (the
-    per-sequence recipe is unchanged)."""
+    per-sequence recipe is unchanged); ``proposal`` (one of PROPOSALS) picks
+    how configurations 3 and 4 choose their tokens."""
+    if proposal not in PROPOSALS:
+        raise ValueError(proposal)
     c = CONFIGS[index]
     seed = SEED_BASE + index if seed is None else seed
     Bn = c["B"] if B is None else B
     rng = np.random.default_rng(seed ^ 0x5EED)
     trees: List[Tuple[List[int], List[int]]] = []
-    # SSM perturbation: N(0,1) for the tiny case and N(0,0.5^2) for the merge
-    # case as stated with those workloads; the others only say "perturbed",
-    # and take sigma = 0.3 so that greedy acceptance is not trivially zero.
+    # SSM perturbation and tokens, as each workload states them: the tiny
+    # case N(0,1) with i.i.d. draws, the merge case N(0,0.5^2) with chain
+    # draws, the 70B-GQA and long-context cases N(0,1) with draws (distinct
+    # siblings).  The LLaMA-7B case says only "top-k tokens of a perturbed
+    # target softmax": sigma = 0.3, so that greedy acceptance is not
+    # trivially zero.
     token_mode, q_sigma = "topk", 0.3
+    if index in (3, 4) and proposal == "sampled":
+        token_mode, q_sigma = "distinct", 1.0
     for _b in range(Bn):
         if index == 0:
             # Kept in the breadth-first numbering the workload states:
