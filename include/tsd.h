@@ -71,7 +71,10 @@ enum tsd_dev_status {
     TSD_DEV_BAD_PREFIX = 8,   /* prefix_len[b] + n_nodes[b] > Lmax or < 0   */
     TSD_DEV_TIMEOUT = 16,     /* a bounded pipeline wait expired (kernel bailed out) */
     TSD_DEV_BAD_PATH = 32,    /* an accepted path that is not a valid commit list     */
-    TSD_DEV_BAD_PAGE = 64     /* a block-table entry outside [0, num_pages)          */
+    TSD_DEV_BAD_PAGE = 64,    /* a block-table entry outside [0, num_pages)          */
+    TSD_DEV_BOUNDS = 128      /* checked build only (libtsd_checked.so): a kernel computed
+                                 an index outside the buffer its arguments describe; the
+                                 access was skipped                                    */
 };
 
 /* Element types of Q / K / V / attention output. */
@@ -82,7 +85,8 @@ enum tsd_attention_path {
     TSD_PLAN_SIMT = 0,       /* CUDA cores, 16 query rows per CTA                       */
     TSD_PLAN_ROWS128 = 1,    /* tensor cores, 128-key tiles, one CTA per SM             */
     TSD_PLAN_ROWS64 = 2,     /* tensor cores, 64-key tiles, two CTAs per SM             */
-    TSD_PLAN_KEYSPLIT = 3    /* tensor cores, two softmax groups splitting the key tiles */
+    TSD_PLAN_KEYSPLIT = 3,   /* tensor cores, two softmax groups splitting the key tiles */
+    TSD_PLAN_ROWS128_PAIRED = 4  /* 128-key tiles, two softmax warps per TMEM lane quarter */
 };
 
 /* Marker written to first_child[b][0] by tsd_tree_mask_build for a malformed

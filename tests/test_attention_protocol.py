@@ -35,16 +35,34 @@ class _Barrier:
             self.pending, self.done = 0, self.done + 1
 
 
-def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready"):
+def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged=True, sw=1,
+         redo_p=0.2):
+    """merged: the producer reuses a K slot once s_full of the QK that read it
+    completes and a V slot once o_ready of the PV that read it completes (the
+    rows kernels; the MMA thread then commits only to s_full and o_ready).
+    sw = 2: two softmax warps per TMEM lane quarter, each on half of every
+    key tile; per tile they exchange their redo votes and, when either voted,
+    their row maxima (then both may rescale O), and at the end their row
+    sums -- each exchange a phase of the quarter's pair mbarrier."""
     rnd = random.Random(seed)
-    bars = {"q_full": _Barrier(4)}
+    nsm = 4 * sw
+    bars = {"q_full": _Barrier(nsm)}
     for s in range(NSK):
         bars["k_full", s], bars["k_empty", s] = _Barrier(1), _Barrier(1)
     for s in range(NSV):
         bars["v_full", s], bars["v_empty", s] = _Barrier(1), _Barrier(1)
     for i in range(NS):
         bars["s_full", i], bars["o_ready", i] = _Barrier(1), _Barrier(1)
-        bars["p_full", i] = _Barrier(4)
+        bars["p_full", i] = _Barrier(nsm)
+    for q in range(4):
+        bars["pair", q] = _Barrier(2)
+    decide = {}   # (quarter, tile) -> (redo, rescale): the same for both warps of a pair
+
+    def shared(q, j):
+        if (q, j) not in decide:
+            redo = j == 0 or rnd.random() < redo_p
+            decide[q, j] = (redo, redo and j > 0 and rnd.random() < rescale_p)
+        return decide[q, j]
 
     def passes(name, k):
         """Wait for phase k of `name` (parity k & 1): True once it passes."""
@@ -58,20 +76,37 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready"):
     s_owner = {}       # S buffer -> tile whose scores/P it holds
     pv_done = set()
 
+    k_read, v_read = {}, {}   # ring slot -> tile loaded there
+    qk_done, pv_done_set = set(), set()
+
     def producer():
         for i in range(ntiles + 1):
             if i < ntiles:
                 s = i % NSK
                 if i >= NSK:
-                    while not passes(("k_empty", s), i // NSK - 1):
-                        yield
+                    if merged:   # QK_{i-NSK} done: s_full[i % NS], NS == NSK
+                        assert NS == NSK
+                        while not passes(("s_full", s), i // NS - 1):
+                            yield
+                    else:
+                        while not passes(("k_empty", s), i // NSK - 1):
+                            yield
+                    assert k_read[s] in qk_done, f"K slot {s} reloaded before its QK ran"
+                k_read[s] = i
                 tma.append(("k_full", s))
             if i >= 1:
                 j = i - 1
                 s = j % NSV
                 if j >= NSV:
-                    while not passes(("v_empty", s), j // NSV - 1):
-                        yield
+                    if merged:   # PV_{j-NSV} done: o_ready[(j - NSV) % NS]
+                        r = j - NSV
+                        while not passes(("o_ready", r % NS), r // NS):
+                            yield
+                    else:
+                        while not passes(("v_empty", s), j // NSV - 1):
+                            yield
+                    assert v_read[s] in pv_done, f"V slot {s} reloaded before its PV ran"
+                v_read[s] = j
                 tma.append(("v_full", s))
             yield
 
@@ -86,7 +121,8 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready"):
             prev = s_owner.get(buf)
             assert prev is None or prev in pv_done or ("pv", prev) in [p[0] for p in pipe], \
                 f"QK_{i} issued over the P of tile {prev} before its PV"
-            pipe.append((("qk", i), [("s_full", buf), ("k_empty", i % NSK)]))
+            commits = [("s_full", buf)] if merged else [("s_full", buf), ("k_empty", i % NSK)]
+            pipe.append((("qk", i), commits))
             s_owner[buf] = i
         for i in range(min(NS, ntiles)):
             yield from qk(i)
@@ -95,19 +131,37 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready"):
                 yield
             while not passes(("v_full", j % NSV), j // NSV):
                 yield
-            pipe.append((("pv", j), [("v_empty", j % NSV), ("o_ready", j % NS)]))
+            commits = [("o_ready", j % NS)] if merged else \
+                [("v_empty", j % NSV), ("o_ready", j % NS)]
+            pipe.append((("pv", j), commits))
             if j + NS < ntiles:
                 yield from qk(j + NS)
             yield
 
-    def softmax():
+    def exchange(q, n):
+        """Exchange n of quarter q's pair: arrive, then wait for phase n."""
+        bars["pair", q].arrive()
+        while not passes(("pair", q), n):
+            yield
+
+    def softmax(q):
         bars["q_full"].arrive()
         yield
+        nx = 0
         for j in range(ntiles):
             while not passes(("s_full", j % NS), j // NS):
                 yield
             yield
-            if j > 0 and rnd.random() < rescale_p:      # O rescaled: PV_{j-1} done
+            if sw == 1:
+                rescale = j > 0 and rnd.random() < rescale_p
+            else:
+                redo, rescale = shared(q, j)
+                yield from exchange(q, nx)              # the votes
+                nx += 1
+                if redo:
+                    yield from exchange(q, nx)          # the row maxima
+                    nx += 1
+            if rescale:                                 # O rescaled: PV_{j-1} done
                 while not passes(("o_ready", (j - 1) % NS), (j - 1) // NS):
                     yield
                 assert j - 1 in pv_done
@@ -122,8 +176,10 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready"):
                 while not passes(("v_empty", last % NSV), last // NSV):
                     yield
             assert set(range(ntiles)) <= pv_done
+            if sw == 2:
+                yield from exchange(q, nx)              # the row sums
 
-    roles = [producer(), mma()] + [softmax() for _ in range(4)]
+    roles = [producer(), mma()] + [softmax(q) for q in range(4) for _ in range(sw)]
     idle = 0
     while roles or tma or pipe:
         choices = list(range(len(roles))) + (["tma"] if tma else []) + (["pipe"] if pipe else [])
@@ -135,6 +191,8 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready"):
             (kind, t), commits = pipe.pop(0)
             if kind == "pv":
                 pv_done.add(t)
+            else:
+                qk_done.add(t)
             for name in commits:
                 bars[name].arrive()
             idle = 0
@@ -147,12 +205,20 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready"):
         assert idle < 50_000, "no role can make progress: a wait never ends"
 
 
-@pytest.mark.parametrize("NS,NSK,NSV", [(3, 3, 2), (2, 2, 2)],
-                         ids=["128-key tiles", "64-key tiles"])
+@pytest.mark.parametrize("NS,NSK,NSV,sw", [(3, 3, 2, 1), (2, 2, 2, 1), (3, 3, 2, 2)],
+                         ids=["128-key tiles", "64-key tiles", "128-key tiles, paired softmax"])
 @pytest.mark.parametrize("ntiles", [1, 2, 3, 4, 5, 8, 17])
-def test_rows_kernel_protocol(NS, NSK, NSV, ntiles):
+def test_rows_kernel_protocol(NS, NSK, NSV, sw, ntiles):
     for seed in range(150):
-        _run(NS, NSK, NSV, ntiles, seed)
+        _run(NS, NSK, NSV, ntiles, seed, sw=sw)
+
+
+@pytest.mark.parametrize("ntiles", [1, 3, 6])
+def test_rows_kernel_protocol_with_ring_commits(ntiles):
+    # the producer waiting on the rings' own empty barriers (the MMA thread
+    # committing every product to them as well) is equally sound
+    for seed in range(100):
+        _run(3, 3, 2, ntiles, seed, merged=False)
 
 
 def test_the_checks_catch_a_stale_wait():
@@ -163,7 +229,7 @@ def test_the_checks_catch_a_stale_wait():
     # protocol check must flag it.
     with pytest.raises(AssertionError):
         for seed in range(300):
-            _run(3, 3, 2, 6, seed, final_wait="v_empty")
+            _run(3, 3, 2, 6, seed, final_wait="v_empty", merged=False)
 
 
 def _run_keysplit(NSK, NSV, ntiles, seed, rescale_p=0.3):

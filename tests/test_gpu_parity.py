@@ -103,6 +103,14 @@ def test_attention_parity_paired_rows_kernel(cuda_device, case, monkeypatch):
     test_attention_parity(cuda_device, case)
 
 
+@pytest.mark.parametrize("case", ROWS_CASES, ids=[f"s{c[0]}" for c in ROWS_CASES])
+def test_attention_parity_rows_kernel_paired_softmax(cuda_device, case, monkeypatch):
+    # more than 128 packed rows on the 128-key rows kernel with two softmax
+    # warps per TMEM lane quarter
+    monkeypatch.setenv("TSD_ATTN_SOFTMAX_WARPS", "2")
+    test_attention_parity(cuda_device, case)
+
+
 SMALL_CASES = [c for c in ATTN_CASES if c[7] == "bf16" and c[5] == 128 and c[2] * c[3] // c[4] <= 128]
 
 
@@ -150,6 +158,7 @@ FORCED = [
     # (shape, environment, expected kernel)
     ("large", {}, "rows128"),
     ("large", {"TSD_ATTN_ROWS_VARIANT": "2"}, "rows64"),
+    ("large", {"TSD_ATTN_SOFTMAX_WARPS": "2"}, "rows128x2"),
     ("small", {}, "rows64"),
     ("small", {"TSD_ATTN_SMALL_VARIANT": "keysplit"}, "keysplit"),
     ("small", {"TSD_FORCE_PATH": "simt"}, "simt"),
@@ -173,10 +182,10 @@ def test_attention_parity_forced_splits(cuda_device, forced, splits, monkeypatch
     sms = torch.cuda.get_device_properties(cuda_device).multi_processor_count
     plan = tsd.attention_plan(w.B, w.Tmax, w.Hq, w.Hkv, w.D, w.Lmax, torch.bfloat16, sms)
     assert plan["kernel"] == kernel
-    tiles = -(-w.Lmax // (128 if kernel in ("rows128", "keysplit") else
+    tiles = -(-w.Lmax // (128 if kernel in ("rows128", "rows128x2", "keysplit") else
                           64 if kernel == "rows64" else 32))
     assert plan["splits"] == min(int(splits), tiles if kernel != "simt" else plan["splits"])
-    if shape == "large" and kernel == "rows128":
+    if shape == "large" and kernel in ("rows128", "rows128x2"):
         assert plan["row_blocks"] == 2 and max(w.n_nodes.tolist()) * w.G > 128
     d = to_dev(w, cuda_device)
     poison(w, d)
@@ -374,6 +383,12 @@ def _sample_rows(w, n, seed):
     T0 = int(w.n_nodes[0])
     rows.append((0, T0 - 1, w.Hq - 1))
     return rows
+
+
+@pytest.mark.parametrize("cfg", [3, 4])
+def test_config_full_size_paired_softmax(cuda_device, cfg, monkeypatch):
+    monkeypatch.setenv("TSD_ATTN_SOFTMAX_WARPS", "2")
+    test_config_full_size(cuda_device, cfg)
 
 
 @pytest.mark.parametrize("cfg", [0, 1, 2, 3, 4])

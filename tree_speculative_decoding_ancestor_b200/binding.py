@@ -17,14 +17,16 @@ from typing import Dict, NamedTuple, Optional, Tuple
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "lib", "libtsd.so")
+# The library the binding loads: lib/libtsd.so, or the file TSD_LIBRARY names
+# (for instance lib/libtsd_checked.so, the bounds-checked debug build).
+LIB_PATH = os.environ.get("TSD_LIBRARY") or os.path.join(_HERE, "lib", "libtsd.so")
 
 TSD_OK = 0
 TSD_F32, TSD_BF16 = 0, 1
 TSD_MAX_TREE = 128
 TSD_TREE_INVALID = -2
 DEV_BAD_TREE, DEV_BAD_TOKEN, DEV_BAD_QROW, DEV_BAD_PREFIX, DEV_TIMEOUT = 1, 2, 4, 8, 16
-DEV_BAD_PATH, DEV_BAD_PAGE = 32, 64
+DEV_BAD_PATH, DEV_BAD_PAGE, DEV_BOUNDS = 32, 64, 128
 
 _lock = threading.Lock()
 _lib: Optional[ctypes.CDLL] = None
@@ -237,7 +239,7 @@ def attention_workspace_size(B: int, Tmax: int, Hq: int, Hkv: int, D: int, Lmax:
     return int(load_library().tsd_tree_attention_workspace_size(B, Tmax, Hq, Hkv, D, Lmax, code))
 
 
-PLAN_KERNELS = {0: "simt", 1: "rows128", 2: "rows64", 3: "keysplit"}
+PLAN_KERNELS = {0: "simt", 1: "rows128", 2: "rows64", 3: "keysplit", 4: "rows128x2"}
 
 
 def attention_plan(B: int, Tmax: int, Hq: int, Hkv: int, D: int, Lmax: int,

@@ -22,6 +22,12 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(HERE, "_build")
 LIB_DIR = os.path.join(HERE, "lib")
 LIB = os.path.join(LIB_DIR, "libtsd.so")
+# The checked build (-DTSD_CHECKS): every global access whose index a kernel
+# computes is compared with its buffer's extent first; an index outside it
+# sets TSD_DEV_BOUNDS in the status word and the access is skipped.  Slower;
+# for small-case debugging.  Load it with TSD_LIBRARY=<path> before the
+# binding's first call.
+LIB_CHECKED = os.path.join(LIB_DIR, "libtsd_checked.so")
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -46,11 +52,11 @@ def _stale(target: str, deps: List[str]) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def _compile(src: str, force: bool, verbose: bool) -> str:
-    obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+def _compile(src: str, force: bool, verbose: bool, checked: bool = False) -> str:
+    obj = os.path.join(BUILD, os.path.basename(src)[:-3] + (".checked.o" if checked else ".o"))
     if force or _stale(obj, [src] + _headers()):
-        cmd = [NVCC] + ARCH + CFLAGS + (["-Xptxas", "-v"] if verbose else []) + \
-            ["-c", src, "-o", obj + ".tmp"]
+        cmd = [NVCC] + ARCH + CFLAGS + (["-DTSD_CHECKS"] if checked else []) + \
+            (["-Xptxas", "-v"] if verbose else []) + ["-c", src, "-o", obj + ".tmp"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"nvcc failed for {src}:\n{r.stdout}\n{r.stderr}")
@@ -60,25 +66,29 @@ def _compile(src: str, force: bool, verbose: bool) -> str:
     return obj
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
+def build(force: bool = False, verbose: bool = False, checked: bool = False) -> str:
+    """Compile every source and link the library (the checked build with
+    `checked`); returns its path."""
     os.makedirs(BUILD, exist_ok=True)
     os.makedirs(LIB_DIR, exist_ok=True)
     srcs = _sources()
+    lib = LIB_CHECKED if checked else LIB
     with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        objs = list(ex.map(lambda s: _compile(s, force, verbose), srcs))
-    if force or _stale(LIB, objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+        objs = list(ex.map(lambda s: _compile(s, force, verbose, checked), srcs))
+    if force or _stale(lib, objs):
+        tmp = lib + f".tmp{os.getpid()}"
         cmd = [NVCC] + ARCH + ["-shared", "-o", tmp] + objs
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
+    ap.add_argument("--checked", action="store_true", help="the bounds-checked debug build")
     args = ap.parse_args()
-    print(build(args.force, args.verbose))
+    print(build(args.force, args.verbose, args.checked))

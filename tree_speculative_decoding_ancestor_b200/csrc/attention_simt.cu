@@ -94,19 +94,26 @@ __global__ void __launch_bounds__(kSimtThreads)
     const int k_begin = split * keys_per_split;
     const int k_end = min(k_begin + keys_per_split, P + T);
 
+    // extents of the buffers (checked build)
+    const int B = gridDim.y / Hkv;
+    const long long n_rows = (long long)B * Tmax * Hq;          // q / out rows
+    const long long n_kv = kv_rows_total(pages, B, Hkv, Lmax);   // K / V rows
     // Stage this CTA's query rows and their ancestor masks.
     for (int i = threadIdx.x; i < kSimtRows * D; i += kSimtThreads) {
         const int lr = i / D, d = i % D, r = row0 + lr;
         float x = 0.f;
         if (r < R) {
             const int u = r / G, h = hk * G + r % G;
-            x = to_float(q[(((size_t)b * Tmax + u) * Hq + h) * D + d]);
+            if (in_bounds(((long long)b * Tmax + u) * Hq + h, n_rows, dev_status))
+                x = to_float(q[(((size_t)b * Tmax + u) * Hq + h) * D + d]);
         }
         sq[lr][d] = x;
     }
     for (int i = threadIdx.x; i < kSimtRows * kMaskWords; i += kSimtThreads) {
         const int lr = i / kMaskWords, w = i % kMaskWords, r = row0 + lr;
-        smask[lr][w] = (r < R && w < W) ? mask[((size_t)b * Tmax + r / G) * W + w] : 0u;
+        const long long mi = ((long long)b * Tmax + r / G) * W + w;
+        smask[lr][w] = (r < R && w < W && in_bounds(mi, (long long)B * Tmax * W, dev_status))
+                           ? mask[mi] : 0u;
     }
 
     float o[4][DL];
@@ -127,7 +134,7 @@ __global__ void __launch_bounds__(kSimtThreads)
             float kx = 0.f, vx = 0.f;
             if (pos < k_end) {
                 const long long row = kv_row(pages, b, hk, Hkv, Lmax, pos);
-                if (row >= 0) {
+                if (row >= 0 && in_bounds(row, n_kv, dev_status)) {
                     kx = to_float(kc[row * D + d]);
                     vx = to_float(vc[row * D + d]);
                 } else if (d == 0) {
@@ -181,6 +188,8 @@ __global__ void __launch_bounds__(kSimtThreads)
             continue;
         const int u = r / G, h = hk * G + r % G;
         const size_t row = ((size_t)b * Tmax + u) * Hq + h;
+        if (!in_bounds((long long)row, n_rows, dev_status))
+            continue;
         if (nsplit == 1) {
             const float inv = l[rr] > 0.f ? 1.f / l[rr] : 0.f;   // a row with no key: 0
 #pragma unroll
@@ -213,6 +222,8 @@ __global__ void __launch_bounds__(256)
         return;
     const int b = (int)(row / ((size_t)Tmax * Hq));
     const int u = (int)((row / Hq) % Tmax);
+    if (!in_bounds(b, B, nullptr))
+        return;
     const int T = n_nodes[b], P = prefix_len[b];
     if (!tree_header_ok(T, Tmax) || P < 0 || P + T > Lmax || u >= T)
         return;

@@ -82,9 +82,11 @@ struct Geo {
     static constexpr uint32_t kOffK = kOffQ + kTileQ;
     static constexpr uint32_t kOffV = kOffK + NSK * kTile;
     static constexpr uint32_t kOffBar = kOffV + NSV * kTile;
-    static constexpr int kNumBars = 1 + 2 * NSK + 2 * NSV + 12;
+    static constexpr int kNumBars = 1 + 2 * NSK + 2 * NSV + 16;
     static constexpr uint32_t kOffMisc = kOffBar + 8 * kNumBars;
-    static constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;   // + alignment slack
+    static constexpr uint32_t kOffXchg = kOffMisc + 16;    // the softmax pairs' exchange slots
+    static constexpr uint32_t kXchgBytes = 4 * 528;        // 4 x sizeof(PairXchg)
+    static constexpr uint32_t kSmemBytes = kOffXchg + kXchgBytes + 1024;   // + alignment slack
     static constexpr uint32_t kTmemCols = TMEM_COLS;
 };
 // 128-key tiles, 197 KB of shared memory and all 512 TMEM columns: one CTA
@@ -95,11 +97,11 @@ using Half = Geo<64, 2, 2, 256>;
 static_assert(Wide::kSmemBytes <= 232448, "shared memory budget");
 static_assert(2 * (Half::kSmemBytes + 1024) <= 233472, "two CTAs per SM");
 
-constexpr int kRowsThreads = 192;       // rows kernel: 6 warps
 constexpr int kSplitThreads = 384;      // key-split kernel: 12 warps
 
 // mbarrier addresses: q_full, k_full[NSK], k_empty[NSK], v_full[NSV],
-// v_empty[NSV], s_full[4], p_full[4], o_ready[4] -- consecutive 8-byte words.
+// v_empty[NSV], s_full[4], p_full[4], o_ready[4], pair[4] -- consecutive
+// 8-byte words.
 template <class Gm>
 struct Bars {
     static constexpr int NSK = Gm::NSK, NSV = Gm::NSV;
@@ -112,6 +114,8 @@ struct Bars {
     __device__ uint32_t s_full(int i) const { return base + 8u * (1 + 2 * NSK + 2 * NSV + i); }
     __device__ uint32_t p_full(int i) const { return base + 8u * (5 + 2 * NSK + 2 * NSV + i); }
     __device__ uint32_t o_ready(int i) const { return base + 8u * (9 + 2 * NSK + 2 * NSV + i); }
+    // the two softmax warps of TMEM lane quarter i meet here (two arrivals)
+    __device__ uint32_t pair(int i) const { return base + 8u * (13 + 2 * NSK + 2 * NSV + i); }
 };
 
 // A wait whose outcome is the same on every lane of the warp (the TMEM
@@ -220,6 +224,7 @@ __device__ __forceinline__ Setup<Gm> cta_setup(uint8_t *smem_raw, uint32_t q_arr
             ptx::mbar_init(su.bars.s_full(i), 1);
             ptx::mbar_init(su.bars.o_ready(i), 1);
             ptx::mbar_init(su.bars.p_full(i), p_arrivals);
+            ptx::mbar_init(su.bars.pair(i), 2);
         }
         *su.abort_flag = 0;
         ptx::fence_barrier_init();
@@ -285,8 +290,15 @@ __device__ __forceinline__ void load_kv_tile(uint32_t dst, const CUtensorMap *tm
 }
 
 // TMA producer (one lane): K_0, K_1, V_0, K_2, V_1, ... -- the order in which
-// the MMA warp first needs them.
-template <class Gm>
+// the MMA warp first needs them.  A ring slot is reused once the product that
+// read it is complete.  NS_PROD = 0: the MMA warp commits every product to
+// the rings' own empty barriers as well.  NS_PROD = NS (the number of score
+// buffers, equal to the K ring's depth): the producer waits on the products'
+// own barriers instead -- QK_{i-NSK} completes on s_full[i % NS], PV_{j-NSV}
+// on o_ready[(j - NSV) % NS] -- which saves the MMA thread two commits per
+// tile.  Either wait names a phase that cannot be stale or ahead: the phase
+// after it needs K_i (or V_{j+1}), which this producer has not loaded yet.
+template <class Gm, int NS_PROD>
 __device__ __forceinline__ void produce_kv(const Setup<Gm> &su, const CUtensorMap *tmK,
                                            const CUtensorMap *tmV, int b, int hk, int Hkv,
                                            int kb, int ntiles, const KvPages &pages,
@@ -294,13 +306,14 @@ __device__ __forceinline__ void produce_kv(const Setup<Gm> &su, const CUtensorMa
 {
     constexpr int NSK = Gm::NSK, NSV = Gm::NSV, BN = Gm::BN;
     constexpr uint32_t kTile = Gm::kTile;
+    static_assert(NS_PROD == 0 || NS_PROD == NSK, "score buffers and K ring in step");
     ptx::prefetch_tmap(tmK);
     ptx::prefetch_tmap(tmV);
     for (int i = 0; i <= ntiles; ++i) {
         if (i < ntiles) {
             const int s = i % NSK;
-            if (i >= NSK &&
-                !ptx::mbar_wait(su.bars.k_empty(s), ((i / NSK) - 1) & 1, su.abort_flag))
+            const uint32_t k_free = NS_PROD ? su.bars.s_full(s) : su.bars.k_empty(s);
+            if (i >= NSK && !ptx::mbar_wait(k_free, ((i / NSK) - 1) & 1, su.abort_flag))
                 break;
             ptx::mbar_arrive_expect_tx(su.bars.k_full(s), kTile);
             load_kv_tile<Gm>(su.sK + s * kTile, tmK, su.bars.k_full(s), kb + i * BN, b, hk, Hkv,
@@ -308,9 +321,16 @@ __device__ __forceinline__ void produce_kv(const Setup<Gm> &su, const CUtensorMa
         }
         if (i >= 1) {
             const int j = i - 1, s = j % NSV;
-            if (j >= NSV &&
-                !ptx::mbar_wait(su.bars.v_empty(s), ((j / NSV) - 1) & 1, su.abort_flag))
-                break;
+            if (j >= NSV) {
+                const int r = j - NSV;   // PV_r read this slot last
+                const bool ok =
+                    NS_PROD ? ptx::mbar_wait(su.bars.o_ready(r % (NS_PROD ? NS_PROD : 1)),
+                                             (r / (NS_PROD ? NS_PROD : 1)) & 1, su.abort_flag)
+                            : ptx::mbar_wait(su.bars.v_empty(s), ((j / NSV) - 1) & 1,
+                                             su.abort_flag);
+                if (!ok)
+                    break;
+            }
             ptx::mbar_arrive_expect_tx(su.bars.v_full(s), kTile);
             load_kv_tile<Gm>(su.sV + s * kTile, tmV, su.bars.v_full(s), kb + j * BN, b, hk, Hkv,
                          pages, seq_end, dev_status);
@@ -319,7 +339,7 @@ __device__ __forceinline__ void produce_kv(const Setup<Gm> &su, const CUtensorMa
 }
 
 // MMA warp, S = Q K^T for key tile `t` into TMEM columns `col_s`.
-template <class Gm>
+template <class Gm, bool RING_COMMIT = true>
 __device__ __forceinline__ void issue_qk(const Setup<Gm> &su, int lane, uint32_t col_s, int t,
                                          uint32_t s_full)
 {
@@ -332,14 +352,17 @@ __device__ __forceinline__ void issue_qk(const Setup<Gm> &su, int lane, uint32_t
             ptx::mma_ss(su.tmem + col_s, dq + slice_off(kk, kSubQ), dk + slice_off(kk, Gm::kSub),
                         idesc, kk > 0 ? 1u : 0u);
         ptx::mma_commit(s_full);
-        ptx::mma_commit(su.bars.k_empty(st));
+        if (RING_COMMIT)
+            ptx::mma_commit(su.bars.k_empty(st));
     }
     __syncwarp();
 }
 
 // MMA warp, O += P V for key tile `t` (P in TMEM columns col_p); zeroes the
-// V rows at or beyond P_b + T_b first.
-template <class Gm>
+// V rows at or beyond P_b + T_b first.  P_SPLIT: the packed P of keys
+// 64 .. 127 sits 64 columns after that of keys 0 .. 63 (each softmax half
+// writes into its own score columns) instead of right after it.
+template <class Gm, bool RING_COMMIT = true, bool P_SPLIT = false>
 __device__ __forceinline__ void issue_pv(const Setup<Gm> &su, int lane, uint32_t col_p,
                                          uint32_t col_o, int t, bool accumulate, int first_bad,
                                          uint32_t o_ready)
@@ -362,11 +385,15 @@ __device__ __forceinline__ void issue_pv(const Setup<Gm> &su, int lane, uint32_t
     if (lane == 0) {
         const uint64_t dv = desc_v(su.sV + vs * Gm::kTile, Gm::kSub);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-            ptx::mma_ts(su.tmem + col_o, su.tmem + col_p + kk * 8,
+        for (int kk = 0; kk < BN / 16; ++kk) {
+            const uint32_t pc = P_SPLIT ? (uint32_t)((kk >> 2) * 64 + (kk & 3) * 8)
+                                        : (uint32_t)(kk * 8);
+            ptx::mma_ts(su.tmem + col_o, su.tmem + col_p + pc,
                         dv + (uint64_t)((kk * 16u * 128u) >> 4), idesc,
                         (accumulate || kk > 0) ? 1u : 0u);
-        ptx::mma_commit(su.bars.v_empty(vs));
+        }
+        if (RING_COMMIT)
+            ptx::mma_commit(su.bars.v_empty(vs));
         ptx::mma_commit(o_ready);
     }
     __syncwarp();
@@ -379,15 +406,16 @@ struct RowCtx {
     float scale_log2;
 };
 
-// Q row `t` of the tile -> shared memory, 128-byte swizzled K-major layout.
-template <class Gm>
+// Q row `t` of the tile -> shared memory, 128-byte swizzled K-major layout;
+// with SW = 2 warps per row, half hf loads the 64 dims hf*64 .. hf*64 + 63.
+template <class Gm, int SW = 1>
 __device__ __forceinline__ void load_q_row(const Setup<Gm> &su, const __nv_bfloat16 *__restrict__ q,
-                                           bool row_ok, size_t q_off, int t)
+                                           bool row_ok, size_t q_off, int t, int hf = 0)
 {
     uint8_t *dst = su.gbase + kOffQ;
     const uint4 *src = reinterpret_cast<const uint4 *>(q + q_off);
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
+    for (int c = (SW == 2 ? hf * 8 : 0); c < (SW == 2 ? hf * 8 + 8 : 16); ++c) {
         const uint4 x = row_ok ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
         const int sub = c >> 3, cc = c & 7;
         *reinterpret_cast<uint4 *>(dst + sub * kSubQ + t * 128 + ((cc ^ (t & 7)) * 16)) = x;
@@ -646,13 +674,128 @@ __device__ __forceinline__ void write_row(uint32_t taddr_o, float inv, bool row_
     }
 }
 
+// One 128-key tile of the online softmax split over two warps per TMEM lane
+// quarter: this warp takes the 64 keys of its half (hf) of the tile, for the
+// same 32 query rows as its partner warp, which takes the other half.  Both
+// halves write P against the same running max m_run and keep their own part
+// of the row sum (l_half).  Whether the row max must be taken (a half's P sum
+// above 2^64 or not finite, always on the first tile) is decided for both at
+// once: each warp publishes its ballot in the pair's exchange slots (by tile
+// parity) and the two warps meet at a named barrier of 64 threads; when the
+// max pass runs, each half publishes its rows' maxima the same way, so both
+// take the same new maximum and rescale their 64 columns of O alike.
+struct PairXchg {
+    uint32_t vote[2][2];      // [exchange parity][half]: the warp's redo ballot
+    float mx[2][2][32];       // [exchange parity][half][lane]: a value per row
+};
+static_assert(sizeof(PairXchg) == 528, "exchange slots");
+
+// One exchange between the two warps of a lane quarter: each warp has
+// written its slots of parity (n & 1) and arrives on the quarter's
+// mbarrier; both wait for the phase (bounded, like every wait here).  The
+// two warps make the same exchanges in the same order, so phase n of the
+// barrier is exchange n; slots alternate by parity, so a warp writing the
+// slots of exchange n + 2 has passed exchange n + 1, which its partner
+// entered only after reading those of exchange n.
+template <class Gm>
+__device__ __forceinline__ bool pair_exchange(const Setup<Gm> &su, int quarter, int &n)
+{
+    warp_arrive(su.bars.pair(quarter));
+    const bool ok = warp_wait(su.bars.pair(quarter), n & 1, su.abort_flag);
+    ++n;
+    return ok;
+}
+
+template <class Gm, typename WaitPrev>
+__device__ __forceinline__ bool softmax_half_tile(const Setup<Gm> &su, uint32_t taddr_s,
+                                                  uint32_t taddr_o, int pos0, int P, int ke,
+                                                  const uint32_t (&mw)[4], float scale_log2,
+                                                  bool first, int hf, int quarter, PairXchg *xc,
+                                                  int &nx, float &m_run, float &l_half,
+                                                  WaitPrev wait_prev)
+{
+    const int lane = threadIdx.x & 31;
+    uint32_t sr[2][32];
+    ptx::tmem_ld32(taddr_s, sr[0]);
+    ptx::tmem_ld32(taddr_s + 32, sr[1]);
+    ptx::tmem_wait_ld();
+    if (!(pos0 + 64 <= min(P, ke))) {
+        mask32(sr[0], valid_bits(pos0, P, ke, mw));
+        mask32(sr[1], valid_bits(pos0 + 32, P, ke, mw));
+    }
+    float lsum = 0.f;
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+        const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
+        lsum = 0.f;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            uint32_t pk[16];
+            lsum += exp_pack32(sr[c], scale_log2, neg_m, pk);
+            ptx::tmem_st16(taddr_s + c * 16, pk);
+        }
+        if (pass == 1)
+            break;
+        const bool redo = !(lsum <= kLazyLimit) || m_run == -INFINITY;
+        const uint32_t vote = __ballot_sync(0xffffffffu, redo);
+        int par = nx & 1;
+        if (lane == 0)
+            xc->vote[par][hf] = vote;
+        if (!pair_exchange(su, quarter, nx))
+            return false;
+        if ((xc->vote[par][0] | xc->vote[par][1]) == 0u)
+            break;
+        float mx[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            mx[i] = -INFINITY;
+        max32x2(sr[0], sr[1], mx);
+        par = nx & 1;
+        xc->mx[par][hf][lane] = max16(mx);
+        if (!pair_exchange(su, quarter, nx))
+            return false;
+        const float mt = fmaxf(xc->mx[par][0][lane], xc->mx[par][1][lane]) * scale_log2;
+        const bool need = mt > m_run + kRescaleThreshold;   // false if mt is -inf
+        const float m_new = need ? mt : m_run;
+        const float alpha = need ? ptx::ex2(m_run - m_new) : 1.f;   // 0 when m_run = -inf
+        if (__any_sync(0xffffffffu, need) && !first) {
+            // O holds the products of the earlier key tiles: wait for the last,
+            // then rescale this half's 64 columns of it.
+            if (!wait_prev())
+                return false;
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t o[32];
+                ptx::tmem_ld32(taddr_o + c * 32, o);
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int k = 0; k < 32; ++k)
+                    o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+                ptx::tmem_st32(taddr_o + c * 32, o);
+            }
+        }
+        l_half *= alpha;
+        m_run = m_new;
+        ptx::tmem_wait_st();   // the speculative P is overwritten next pass
+    }
+    l_half += lsum;
+    ptx::tmem_wait_st();
+    return true;
+}
+
 // ============================================================ rows kernel
-// More than 128 packed rows: one 128-row query tile per CTA, 6 warps (TMA
-// producer, MMA issuer, 4 softmax warps).  NS score buffers of BN columns
-// each, then O: the MMA warp keeps the scores of the next NS - 1 key tiles
-// ready while the softmax works on tile j.  Two instances:
+// More than 128 packed rows: one 128-row query tile per CTA; warp 0 the TMA
+// producer, warp 1 the MMA issuer, then the softmax warps.  NS score buffers
+// of BN columns each, then O: the MMA warp keeps the scores of the next NS - 1
+// key tiles ready while the softmax works on tile j.  Instances:
 //   * 128-key tiles, NS = 3, one CTA per SM:
 //         TMEM S0 [0,128) | S1 [128,256) | S2 [256,384) | O [384,512)
+//     with SW = 1 softmax warp per TMEM lane quarter (each thread a whole
+//     row of 128 scores), or SW = 2 (8 softmax warps, two per SM
+//     sub-partition: each takes one 64-key half of the tile for 32 rows, so
+//     a sub-partition interleaves two warps' exponentials; P of each half is
+//     written over that half's own score columns);
 //   * 64-key tiles, NS = 2, two CTAs per SM (each with 256 TMEM columns and
 //     97 KB of shared memory): S0 [0,64) | S1 [64,128) | O [128,256).  The
 //     two CTAs' MMA warps feed one tensor pipe and their softmax warps share
@@ -660,13 +803,17 @@ __device__ __forceinline__ void write_row(uint32_t taddr_o, float inv, bool row_
 //     covered by the other's work.
 // MMA order: QK_0 .. QK_{NS-1}, then per tile j: PV_j QK_{j+NS}; P_j is read
 // out of S_{j%NS} by PV_j before QK_{j+NS}, issued after it by the same
-// thread, overwrites it.  PV_j commits to o_ready[j%NS].  The softmax at tile
-// j waits for "PV_{j-1} done" on o_ready[(j-1)%NS]: the phase before it
+// thread, overwrites it.  QK_i commits to s_full[i%NS], PV_j to o_ready[j%NS]
+// (the producer reuses ring slots on those same barriers).  The softmax at
+// tile j waits for "PV_{j-1} done" on o_ready[(j-1)%NS]: the phase before it
 // there is PV_{j-1-NS}, issued before QK_j, whose completion the softmax has
 // already seen, and the phase after it needs P_{j-1+NS}, not yet written --
 // so the wait names a phase that can be neither stale nor ahead.
-template <class Gm, int NS, int kMinBlocks>
-__global__ void __launch_bounds__(kRowsThreads, kMinBlocks)
+template <int SW>
+constexpr int rows_threads() { return 64 + 128 * SW; }
+
+template <class Gm, int NS, int kMinBlocks, int SW>
+__global__ void __launch_bounds__(rows_threads<SW>(), kMinBlocks)
     tree_attn_rows_kernel(const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV,
                           const __nv_bfloat16 *__restrict__ q,
@@ -694,15 +841,19 @@ __global__ void __launch_bounds__(kRowsThreads, kMinBlocks)
         return;   // no rows or no keys: the partials stay empty
     constexpr int BN = Gm::BN, NSK = Gm::NSK, NSV = Gm::NSV;
     static_assert(NS * BN + HD <= (int)Gm::kTmemCols && BN % 64 == 0, "TMEM layout");
+    static_assert(SW == 1 || (SW == 2 && BN == 128), "split softmax: 128-key tiles");
+    static_assert(NS == NSK, "the producer reuses K slots on the score barriers");
     const int ntiles = (ke - kb + BN - 1) / BN;
-    const Setup<Gm> su = cta_setup<Gm>(smem_raw, 4, 4);   // arrivals: softmax warps
+    // arrivals: every softmax warp loads its part of Q and publishes its P
+    const Setup<Gm> su = cta_setup<Gm>(smem_raw, 4 * SW, 4 * SW);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     auto col_s = [](int i) { return (uint32_t)(i % NS) * (uint32_t)BN; };
     constexpr uint32_t kO = NS * BN;
 
     if (warp == 0) {
         if (lane == 0)
-            produce_kv(su, &tmK, &tmV, b, hk, Hkv, kb, ntiles, pages, P + T, dev_status);
+            produce_kv<Gm, NS>(su, &tmK, &tmV, b, hk, Hkv, kb, ntiles, pages, P + T,
+                               dev_status);
     } else if (warp == 1) {
         bool ok = warp_wait(su.bars.q_full(), 0, su.abort_flag);
         ptx::tc_fence_after();
@@ -710,7 +861,7 @@ __global__ void __launch_bounds__(kRowsThreads, kMinBlocks)
             if (!warp_wait(su.bars.k_full(i % NSK), (i / NSK) & 1, su.abort_flag))
                 return false;
             ptx::tc_fence_after();
-            issue_qk(su, lane, col_s(i), i, su.bars.s_full(i % NS));
+            issue_qk<Gm, false>(su, lane, col_s(i), i, su.bars.s_full(i % NS));
             return true;
         };
         for (int i = 0; ok && i < min(NS, ntiles); ++i)
@@ -721,32 +872,39 @@ __global__ void __launch_bounds__(kRowsThreads, kMinBlocks)
                 ok = false;
                 break;
             }
-            issue_pv(su, lane, col_s(j), kO, j, j > 0, P + T - (kb + j * BN),
-                     su.bars.o_ready(j % NS));
+            issue_pv<Gm, false, SW == 2>(su, lane, col_s(j), kO, j, j > 0,
+                                         P + T - (kb + j * BN), su.bars.o_ready(j % NS));
             if (j + NS < ntiles)
                 ok = qk(j + NS);
         }
     } else {
-        // softmax warps 2..5: one query row per thread == TMEM lane
+        // softmax warps: one query row per thread == TMEM lane; with SW = 2
+        // the two warps of a lane quarter split the tile's keys (hf = half)
         const int quarter = warp & 3;
+        const int hf = SW == 2 ? (warp - 2) >> 2 : 0;
         const int t = quarter * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const int r = rb * BQ + t;
-        const bool row_ok = r < R;
+        // the row's q / out / mask entries (bounds of the checked build:
+        // every one of them is in range iff the q row index is)
+        const bool row_ok = r < R && in_bounds(((long long)b * Tmax + r / G) * Hq + hk * G + r % G,
+                                               (long long)gridDim.y / Hkv * Tmax * Hq, dev_status);
         const int u = row_ok ? r / G : 0;
         const int h = hk * G + (row_ok ? r % G : 0);
-        load_q_row(su, q, row_ok, (((size_t)b * Tmax + u) * Hq + h) * HD, t);
+        load_q_row<Gm, SW>(su, q, row_ok, (((size_t)b * Tmax + u) * Hq + h) * HD, t, hf);
         warp_arrive(su.bars.q_full());
         uint32_t mw[4];
 #pragma unroll
         for (int w = 0; w < 4; ++w)
             mw[w] = (row_ok && w < W) ? mask[((size_t)b * Tmax + u) * W + w] : 0u;
-        const uint32_t taddr_o = su.tmem + lane_off + kO;
+        const uint32_t taddr_o = su.tmem + lane_off + kO + hf * 64;
+        PairXchg *xc = reinterpret_cast<PairXchg *>(su.gbase + Gm::kOffXchg) + quarter;
         // PV_i done (o_ready[i % NS] completes once per tile of that class)
         auto wait_pv = [&](int i) {
             return warp_wait(su.bars.o_ready(i % NS), (i / NS) & 1, su.abort_flag);
         };
         float m_run = -INFINITY, l_run = 0.f;
+        int nx = 0;   // pair exchanges made
         bool ok = true;
         for (int j = 0; ok && j < ntiles; ++j) {
             if (!warp_wait(su.bars.s_full(j % NS), (j / NS) & 1, su.abort_flag)) {
@@ -754,21 +912,37 @@ __global__ void __launch_bounds__(kRowsThreads, kMinBlocks)
                 break;
             }
             ptx::tc_fence_after();
-            ok = softmax_rows_tile<BN>(su.tmem + lane_off + col_s(j), taddr_o, kb + j * BN, P, ke,
-                                       mw, scale_log2, j == 0, m_run, l_run,
-                                       [&]() { return wait_pv(j - 1); });
+            auto wait_prev = [&]() { return wait_pv(j - 1); };
+            if (SW == 1)
+                ok = softmax_rows_tile<BN>(su.tmem + lane_off + col_s(j), taddr_o, kb + j * BN,
+                                           P, ke, mw, scale_log2, j == 0, m_run, l_run,
+                                           wait_prev);
+            else
+                ok = softmax_half_tile(su, su.tmem + lane_off + col_s(j) + hf * 64, taddr_o,
+                                       kb + j * BN + hf * 64, P, ke, mw, scale_log2, j == 0, hf,
+                                       quarter, xc, nx, m_run, l_run, wait_prev);
             if (!ok)
                 break;
             ptx::tc_fence_before();
             warp_arrive(su.bars.p_full(j % NS));
         }
-        if (ok && wait_pv(ntiles - 1)) {
+        bool done = ok && wait_pv(ntiles - 1);
+        if (SW == 2 && done) {
+            // the row sum is the two halves' sums (a warp that gave up skips
+            // this; its partner's bounded wait then sees the abort flag)
+            const int par = nx & 1;
+            xc->mx[par][hf][lane] = l_run;
+            done = pair_exchange(su, quarter, nx);
+            l_run = xc->mx[par][0][lane] + xc->mx[par][1][lane];
+        }
+        if (done) {
             ptx::tc_fence_after();
             const size_t row = ((size_t)b * Tmax + u) * Hq + h;
             const size_t nrows = (size_t)gridDim.y / Hkv * Tmax * Hq;
             const float inv = nsplit == 1 ? (l_run > 0.f ? 1.f / l_run : 0.f) : 1.f;
-            write_row(taddr_o, inv, row_ok, row, nsplit, split, nrows, out, part_o, 0, HD);
-            if (row_ok && nsplit > 1)
+            write_row(taddr_o, inv, row_ok, row, nsplit, split, nrows, out, part_o, hf * 64,
+                      HD / SW);
+            if (row_ok && nsplit > 1 && hf == 0)
                 part_ml[(size_t)split * nrows + row] = make_float2(m_run, l_run);
         }
     }
@@ -818,7 +992,8 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
 
     if (warp == 0) {
         if (lane == 0)
-            produce_kv(su, &tmK, &tmV, b, hk, Hkv, kb, ntiles, pages, P + T, dev_status);
+            produce_kv<Gm, 0>(su, &tmK, &tmV, b, hk, Hkv, kb, ntiles, pages, P + T,
+                              dev_status);
     } else if (warp == 1) {
         bool ok = warp_wait(su.bars.q_full(), 0, su.abort_flag);
         ptx::tc_fence_after();
@@ -850,7 +1025,8 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
         const int quarter = warp & 3;
         const int t = quarter * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        const bool row_ok = t < R;
+        const bool row_ok = t < R && in_bounds(((long long)b * Tmax + t / G) * Hq + hk * G + t % G,
+                                               (long long)gridDim.y / Hkv * Tmax * Hq, dev_status);
         const int u = row_ok ? t / G : 0;
         const int h = hk * G + (row_ok ? t % G : 0);
         if (s == 0)
@@ -943,8 +1119,18 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
 struct UmmaPlan {
     bool keysplit;   // at most 128 packed rows
     bool paired;     // rows kernel with 64-key tiles, two CTAs per SM
+    int sw;          // 128-key rows kernel: softmax warps per TMEM lane quarter
     int nrb, nsplit, keys_per_split;
 };
+
+// Softmax warps per TMEM lane quarter of the 128-key rows kernel: 1, or 2
+// when the environment variable TSD_ATTN_SOFTMAX_WARPS is "2" (read at every
+// launch).
+int rows_softmax_warps()
+{
+    const char *e = std::getenv("TSD_ATTN_SOFTMAX_WARPS");
+    return (e && e[0] == '2' && e[1] == '\0') ? 2 : 1;
+}
 
 // Rows-kernel instance for more than 128 packed rows: 1 = 128-key tiles at
 // one CTA per SM (default), 2 = 64-key tiles at two CTAs per SM when the
@@ -974,6 +1160,7 @@ UmmaPlan umma_plan(const AttnArgs &a, int num_sms)
     const bool small = a.Tmax * G <= BQ;
     p.keysplit = small && !small_paired();
     p.paired = small ? !p.keysplit : rows_variant() == 2;
+    p.sw = (p.keysplit || p.paired) ? 1 : rows_softmax_warps();
     p.nrb = p.keysplit ? 1 : (a.Tmax * G + BQ - 1) / BQ;
     const int bn = p.paired ? Half::BN : Wide::BN;
     const int slots = num_sms * (p.paired ? 2 : 1);
@@ -1061,10 +1248,14 @@ cudaError_t set_smem_attributes()
         return cudaErrorInvalidDevice;
     if (done[dev].load())
         return cudaSuccess;
-    auto wide = tree_attn_rows_kernel<Wide, 3, 1>;
-    auto half = tree_attn_rows_kernel<Half, 2, 2>;
+    auto wide = tree_attn_rows_kernel<Wide, 3, 1, 1>;
+    auto wide2 = tree_attn_rows_kernel<Wide, 3, 1, 2>;
+    auto half = tree_attn_rows_kernel<Half, 2, 2, 1>;
     err = cudaFuncSetAttribute(wide, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)Wide::kSmemBytes);
+    if (err == cudaSuccess)
+        err = cudaFuncSetAttribute(wide2, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)Wide::kSmemBytes);
     if (err == cudaSuccess)
         err = cudaFuncSetAttribute(tree_attn_keysplit_kernel,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1093,7 +1284,9 @@ bool umma_attention_supported(const AttnArgs &a)
 void umma_attention_plan(const AttnArgs &a, int num_sms, int32_t out[4])
 {
     const UmmaPlan p = umma_plan(a, num_sms);
-    out[0] = p.keysplit ? TSD_PLAN_KEYSPLIT : (p.paired ? TSD_PLAN_ROWS64 : TSD_PLAN_ROWS128);
+    out[0] = p.keysplit ? TSD_PLAN_KEYSPLIT
+                        : (p.paired ? TSD_PLAN_ROWS64
+                                    : (p.sw == 2 ? TSD_PLAN_ROWS128_PAIRED : TSD_PLAN_ROWS128));
     out[1] = p.nrb;
     out[2] = p.nsplit;
     out[3] = p.keys_per_split;
@@ -1145,15 +1338,23 @@ int launch_umma_attention(const AttnArgs &a, void *ws, size_t ws_bytes, int num_
             a.Tmax, a.Hq, a.Hkv, a.Lmax, W, sl2, p.keys_per_split, p.nsplit,
             static_cast<__nv_bfloat16 *>(a.out), part_o, part_ml, a.dev_status, a.pages);
     else if (p.paired)
-        tree_attn_rows_kernel<Half, 2, 2><<<grid, kRowsThreads, Half::kSmemBytes, stream>>>(
-            tmK, tmV, static_cast<const __nv_bfloat16 *>(a.q), a.prefix_len, a.n_nodes, a.mask,
-            a.Tmax, a.Hq, a.Hkv, a.Lmax, W, sl2, p.keys_per_split, p.nsplit,
-            static_cast<__nv_bfloat16 *>(a.out), part_o, part_ml, a.dev_status, a.pages);
+        tree_attn_rows_kernel<Half, 2, 2, 1>
+            <<<grid, rows_threads<1>(), Half::kSmemBytes, stream>>>(
+                tmK, tmV, static_cast<const __nv_bfloat16 *>(a.q), a.prefix_len, a.n_nodes,
+                a.mask, a.Tmax, a.Hq, a.Hkv, a.Lmax, W, sl2, p.keys_per_split, p.nsplit,
+                static_cast<__nv_bfloat16 *>(a.out), part_o, part_ml, a.dev_status, a.pages);
+    else if (p.sw == 2)
+        tree_attn_rows_kernel<Wide, 3, 1, 2>
+            <<<grid, rows_threads<2>(), Wide::kSmemBytes, stream>>>(
+                tmK, tmV, static_cast<const __nv_bfloat16 *>(a.q), a.prefix_len, a.n_nodes,
+                a.mask, a.Tmax, a.Hq, a.Hkv, a.Lmax, W, sl2, p.keys_per_split, p.nsplit,
+                static_cast<__nv_bfloat16 *>(a.out), part_o, part_ml, a.dev_status, a.pages);
     else
-        tree_attn_rows_kernel<Wide, 3, 1><<<grid, kRowsThreads, Wide::kSmemBytes, stream>>>(
-            tmK, tmV, static_cast<const __nv_bfloat16 *>(a.q), a.prefix_len, a.n_nodes, a.mask,
-            a.Tmax, a.Hq, a.Hkv, a.Lmax, W, sl2, p.keys_per_split, p.nsplit,
-            static_cast<__nv_bfloat16 *>(a.out), part_o, part_ml, a.dev_status, a.pages);
+        tree_attn_rows_kernel<Wide, 3, 1, 1>
+            <<<grid, rows_threads<1>(), Wide::kSmemBytes, stream>>>(
+                tmK, tmV, static_cast<const __nv_bfloat16 *>(a.q), a.prefix_len, a.n_nodes,
+                a.mask, a.Tmax, a.Hq, a.Hkv, a.Lmax, W, sl2, p.keys_per_split, p.nsplit,
+                static_cast<__nv_bfloat16 *>(a.out), part_o, part_ml, a.dev_status, a.pages);
     TSD_LAUNCH_CHECK();
     if (p.nsplit > 1) {
         const int rc = launch_combine(a.dtype, a.D, part_o, part_ml, p.nsplit, a.prefix_len,

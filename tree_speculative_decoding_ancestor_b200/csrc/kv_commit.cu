@@ -58,16 +58,18 @@ __global__ void __launch_bounds__(kCommitThreads)
     const size_t plane = (size_t)Lmax * row_bytes;
     uint8_t *const kb = k + ((size_t)b * Hkv + h) * plane;
     uint8_t *const vb = v + ((size_t)b * Hkv + h) * plane;
+    // extent of one (sequence, KV head) plane in 16-byte vectors
+    const long long plane_vec = (long long)Lmax * vec;
     for (int idx = threadIdx.x; idx < 2 * total; idx += kCommitThreads) {
         const int t = idx >= total, r = idx - t * total, i = r / vec, c = r - i * vec;
         const int u = s_path[i];
-        if (u != i)
+        if (u != i && in_bounds((long long)(P + u) * vec + c, plane_vec, dev_status))
             stage[idx] = reinterpret_cast<const uint4 *>((t ? vb : kb) + (size_t)(P + u) * row_bytes)[c];
     }
     __syncthreads();
     for (int idx = threadIdx.x; idx < 2 * total; idx += kCommitThreads) {
         const int t = idx >= total, r = idx - t * total, i = r / vec, c = r - i * vec;
-        if (s_path[i] != i)
+        if (s_path[i] != i && in_bounds((long long)(P + i) * vec + c, plane_vec, dev_status))
             reinterpret_cast<uint4 *>((t ? vb : kb) + (size_t)(P + i) * row_bytes)[c] = stage[idx];
     }
 }

@@ -187,7 +187,7 @@ __global__ void __launch_bounds__(kExpandThreads)
         block_best(bv, bi, shv, shi);
         pv = bv;
         pi = bi;
-        if (threadIdx.x == 0) {
+        if (threadIdx.x == 0 && in_bounds(n + i * k + j, Tmax, nullptr)) {
             const size_t u = (size_t)b * Tmax + n + i * k + j;
             parent[u] = n == 0 ? -1 : lb + i;
             tokens[u] = pi;   // k <= V: a pick always exists
@@ -283,6 +283,8 @@ __global__ void tree_dfs_kernel(const int32_t *__restrict__ parent,
     __syncwarp();
     for (int i = lane; i < s_cnt; i += 32) {
         const int u = order[i];
+        if (!in_bounds(i, Tmax, nullptr) || !in_bounds(u, Tmax, nullptr))
+            continue;
         const size_t o = (size_t)b * Tmax + i;
         perm[o] = u;
         out_parent[o] = par[u] < 0 ? -1 : inv[par[u]];
@@ -368,6 +370,8 @@ __global__ void tree_merge_kernel(const int32_t *__restrict__ ctok, const int32_
         inv[order[i]] = i;
     for (int i = 0; i < cnt; ++i) {
         const int u = order[i];
+        if (!in_bounds(i, Tmax, dev_status))
+            break;
         const size_t o = (size_t)b * Tmax + i;
         parent[o] = par[u] < 0 ? -1 : inv[par[u]];
         tokens[o] = tok[u];

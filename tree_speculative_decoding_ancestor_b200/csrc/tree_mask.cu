@@ -25,8 +25,9 @@ __global__ void __launch_bounds__(kMaxTree)
     const int u = threadIdx.x;
     const int T = n_nodes[b];
     const bool bad_T = !tree_header_ok(T, Tmax);
+    const long long nb = (long long)gridDim.x * Tmax;   // B * Tmax
     int p = -1;
-    if (u < Tmax && !bad_T && u < T)
+    if (u < Tmax && !bad_T && u < T && in_bounds((long long)b * Tmax + u, nb, dev_status))
         p = parent[(size_t)b * Tmax + u];
     par[u] = p;
     fc[u] = INT_MAX;
@@ -52,9 +53,10 @@ __global__ void __launch_bounds__(kMaxTree)
                 ns = v;
                 break;
             }
-    if (u < Tmax) {
+    if (u < Tmax && in_bounds((long long)b * Tmax + u, nb, dev_status)) {
         for (int w = 0; w < W; ++w)
-            mask[((size_t)b * Tmax + u) * W + w] = m[w];
+            if (in_bounds(((long long)b * Tmax + u) * W + w, nb * W, dev_status))
+                mask[((size_t)b * Tmax + u) * W + w] = m[w];
         depth[(size_t)b * Tmax + u] = d;
         next_sibling[(size_t)b * Tmax + u] = ns;
     }
@@ -62,7 +64,9 @@ __global__ void __launch_bounds__(kMaxTree)
         int v = (bad || fc[s] == INT_MAX) ? -1 : fc[s];
         if (bad && s == 0)
             v = TSD_TREE_INVALID;
-        first_child[(size_t)b * (Tmax + 1) + s] = v;
+        if (in_bounds((long long)b * (Tmax + 1) + s, (long long)gridDim.x * (Tmax + 1),
+                      dev_status))
+            first_child[(size_t)b * (Tmax + 1) + s] = v;
     }
     if (bad && u == 0)
         flag(dev_status, TSD_DEV_BAD_TREE);

@@ -53,6 +53,29 @@ __device__ __forceinline__ double warp_sum(double v)
     return v;
 }
 
+// Bounds checks of the checked build.  Compiled with -DTSD_CHECKS (the
+// library libtsd_checked.so, for small-case debugging), every global access
+// whose index a kernel computes is first compared with the extent of the
+// buffer the call's arguments describe; an index outside it sets
+// TSD_DEV_BOUNDS in the status word and the access is skipped (nothing
+// traps).  In the normal build in_bounds() is constant true and the checks
+// compile away.
+#ifdef TSD_CHECKS
+constexpr bool kChecked = true;
+#else
+constexpr bool kChecked = false;
+#endif
+
+__device__ __forceinline__ bool in_bounds(long long i, long long n, int32_t *dev_status)
+{
+    if (!kChecked)
+        return true;
+    if (i >= 0 && i < n)
+        return true;
+    flag(dev_status, TSD_DEV_BOUNDS);
+    return false;
+}
+
 // Sequence-level validity shared by the attention and verify kernels.
 __device__ __forceinline__ bool tree_header_ok(int T, int Tmax) { return T >= 0 && T <= Tmax; }
 
@@ -117,6 +140,15 @@ __device__ __forceinline__ long long kv_row(const KvPages &pg, int b, int hk, in
     if (page < 0 || page >= pg.num_pages)
         return -1;
     return ((long long)page * Hkv + hk) * pg.page_size + (pos & (pg.page_size - 1));
+}
+
+// Rows of D elements the K (or V) buffer holds: the contiguous cache
+// [B][Hkv][Lmax] or the paged pool [num_pages][Hkv][page_size] (for the
+// checked build's bounds).
+__host__ __device__ __forceinline__ long long kv_rows_total(const KvPages &pg, int B, int Hkv,
+                                                            int Lmax)
+{
+    return pg.table ? (long long)pg.num_pages * Hkv * pg.page_size : (long long)B * Hkv * Lmax;
 }
 
 struct AttnArgs {

@@ -542,8 +542,10 @@ __global__ void __launch_bounds__(kFinThreads)
             for (int w = 0; w < (u >> 5); ++w)
                 pos += __popc(mt[w]);
             pos += __popc(mt[u >> 5] & ((1u << (u & 31)) - 1u));
-            out_path[(size_t)b * Tmax + pos] = u;
-            out_tokens[(size_t)b * (Tmax + 1) + pos] = tok;
+            if (in_bounds(pos, Tmax, dev_status)) {
+                out_path[(size_t)b * Tmax + pos] = u;
+                out_tokens[(size_t)b * (Tmax + 1) + pos] = tok;
+            }
         }
     }
     const int row = t + 1;
@@ -553,7 +555,7 @@ __global__ void __launch_bounds__(kFinThreads)
     else
         bonus = row_argmax<kFinThreads>(logits + ((size_t)b * (Tmax + 1) + row) * V, V, shv,
                                         shi);
-    if (u == 0) {
+    if (u == 0 && in_bounds(n, Tmax + 1, dev_status)) {
         out_tokens[(size_t)b * (Tmax + 1) + n] = bonus;
         n_accepted[b] = n;
     }
@@ -669,6 +671,8 @@ __global__ void __launch_bounds__(kWalkThreads)
             // the children in ascending index
             int accepted = -1;
             for (int c = first_child[ri]; c >= 0; c = next_sibling[(size_t)b * Tmax + c]) {
+                if (!in_bounds(c, Tmax, dev_status))
+                    break;   // the same in every CTA of the team (they read the same c)
                 const int x = tokens[(size_t)b * Tmax + c];
                 const float *qc = q_probs + ((size_t)b * Rq + q_row[(size_t)b * Tmax + c]) * V;
                 if (tid == 0) {
@@ -717,7 +721,7 @@ __global__ void __launch_bounds__(kWalkThreads)
             if (!alive)
                 break;
             if (accepted >= 0 && n_path < T) {
-                if (lead) {
+                if (lead && in_bounds(n_path, Tmax, dev_status)) {
                     out_path[(size_t)b * Tmax + n_path] = accepted;
                     out_tokens[(size_t)b * (Tmax + 1) + n_path] =
                         tokens[(size_t)b * Tmax + accepted];
@@ -762,11 +766,11 @@ __global__ void __launch_bounds__(kWalkThreads)
                 int token = chunk_scan<VEC>(lrow, x_lo, x_hi, V, st, table, sh_carry, u, shd, shi);
                 if (token == INT_MAX)   // the chunk's own sum fell short by rounding
                     token = sh_token;
-                if (tid == 0) {
+                if (tid == 0 && in_bounds(n_path, Tmax + 1, dev_status)) {
                     out_tokens[(size_t)b * (Tmax + 1) + n_path] = token;
                     n_accepted[b] = n_path;
                 }
-            } else if (pick < 0 && k == 0 && tid == 0) {
+            } else if (pick < 0 && k == 0 && tid == 0 && in_bounds(n_path, Tmax + 1, dev_status)) {
                 // Rounding left the total at or below u: the largest token with p > 0.
                 out_tokens[(size_t)b * (Tmax + 1) + n_path] = sh_token;
                 n_accepted[b] = n_path;
