@@ -23,8 +23,7 @@
  *     and the flatkey.ai guide's verification diagram (the accepted prefix
  *     is committed).
  *
- * Readings taken where the page is silent (each one is listed in the design
- * notes of the repository):
+ * Readings taken where the page is silent:
  *   - the committed prefix is always attended; S_u = prefix, then the tree
  *     path root-first, ending with u itself;
  *   - the root is the last committed token (logits row 0); node u owns

@@ -2,9 +2,9 @@
 
 The plan names the kernel, the query-row blocks and the key-range splits
 that tree_attention uses for given sizes and SM count. Pinned here for the
-five workloads on a 148-SM B200 (the grids the measurements in the design
-notes were taken with), for the environment selections, and against the
-workspace size (partials exist only when the keys are split).
+five workloads on a 148-SM B200 (the grids the benchmark measures), for the
+environment selections, and against the workspace size (partials exist only
+when the keys are split).
 """
 
 import pytest

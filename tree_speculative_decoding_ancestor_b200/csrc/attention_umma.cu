@@ -69,6 +69,7 @@ constexpr uint32_t kOffQ = 0;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 constexpr float kLazyLimit = 18446744073709551616.0f;   // 2^64: headroom of a P tile sum
+constexpr int kTableCache = 1024;   // block-table entries of a CTA's key range kept in smem
 
 // Tile geometry of a kernel: keys per tile, K and V ring stages, TMEM
 // columns; shared memory holds Q, the K ring, the V ring, the mbarriers.
@@ -86,7 +87,8 @@ struct Geo {
     static constexpr uint32_t kOffMisc = kOffBar + 8 * kNumBars;
     static constexpr uint32_t kOffXchg = kOffMisc + 16;    // the softmax pairs' exchange slots
     static constexpr uint32_t kXchgBytes = 4 * 528;        // 4 x sizeof(PairXchg)
-    static constexpr uint32_t kSmemBytes = kOffXchg + kXchgBytes + 1024;   // + alignment slack
+    static constexpr uint32_t kOffTable = kOffXchg + kXchgBytes;   // paged: block-table slice
+    static constexpr uint32_t kSmemBytes = kOffTable + 4 * kTableCache + 1024;   // + alignment slack
     static constexpr uint32_t kTmemCols = TMEM_COLS;
 };
 // 128-key tiles, 197 KB of shared memory and all 512 TMEM columns: one CTA
@@ -261,11 +263,36 @@ __device__ __forceinline__ void cta_teardown(const Setup<Gm> &su, int32_t *dev_s
 // since both are powers of two and pos0 is a multiple of BN) at (x, row in
 // page, page * Hkv + hk).  A box that starts at or beyond the sequence's end
 // loads any valid page: those keys are masked and their V rows zeroed.
+// The block-table entries of the pages a CTA's key range [kb, seq_end)
+// touches, staged in shared memory by the producer warp before its first
+// load (at most kTableCache of them; entries past that are read from global
+// memory), so that a ring slot's reload does not wait for a global load.
+struct PageCache {
+    const int32_t *sm;   // entries blk0 .. blk0 + n - 1
+    int blk0, n;
+};
+
+template <class Gm>
+__device__ __forceinline__ PageCache stage_pages(const Setup<Gm> &su, const KvPages &pages, int b,
+                                                 int kb, int seq_end, int lane)
+{
+    PageCache pc{reinterpret_cast<const int32_t *>(su.gbase + Gm::kOffTable), 0, 0};
+    if (!pages.table || seq_end <= kb)
+        return pc;
+    pc.blk0 = kb >> pages.log2_page;
+    pc.n = min(((seq_end - 1) >> pages.log2_page) - pc.blk0 + 1, kTableCache);
+    int32_t *dst = reinterpret_cast<int32_t *>(su.gbase + Gm::kOffTable);
+    for (int i = lane; i < pc.n; i += 32)
+        dst[i] = pages.table[(size_t)b * pages.max_blocks + pc.blk0 + i];
+    __syncwarp();
+    return pc;
+}
+
 template <class Gm>
 __device__ __forceinline__ void load_kv_tile(uint32_t dst, const CUtensorMap *tm, uint32_t bar,
                                              int pos0, int b, int hk, int Hkv,
-                                             const KvPages &pages, int seq_end,
-                                             int32_t *dev_status)
+                                             const KvPages &pages, const PageCache &pc,
+                                             int seq_end, int32_t *dev_status)
 {
     if (!pages.table) {
         ptx::tma_load_3d(dst, tm, 0, pos0, b * Hkv + hk, bar);
@@ -277,7 +304,10 @@ __device__ __forceinline__ void load_kv_tile(uint32_t dst, const CUtensorMap *tm
         const int pos = pos0 + r0;
         int z = hk, y = 0;
         if (pos < seq_end) {
-            const int page = pages.table[(size_t)b * pages.max_blocks + (pos >> pages.log2_page)];
+            const int blk = pos >> pages.log2_page, ci = blk - pc.blk0;
+            const int page = (ci >= 0 && ci < pc.n)
+                                 ? pc.sm[ci]
+                                 : pages.table[(size_t)b * pages.max_blocks + blk];
             if (page < 0 || page >= pages.num_pages)
                 flag(dev_status, TSD_DEV_BAD_PAGE);   // page 0 stands in
             else
@@ -302,7 +332,8 @@ template <class Gm, int NS_PROD>
 __device__ __forceinline__ void produce_kv(const Setup<Gm> &su, const CUtensorMap *tmK,
                                            const CUtensorMap *tmV, int b, int hk, int Hkv,
                                            int kb, int ntiles, const KvPages &pages,
-                                           int seq_end, int32_t *dev_status)
+                                           const PageCache &pc, int seq_end,
+                                           int32_t *dev_status)
 {
     constexpr int NSK = Gm::NSK, NSV = Gm::NSV, BN = Gm::BN;
     constexpr uint32_t kTile = Gm::kTile;
@@ -317,7 +348,7 @@ __device__ __forceinline__ void produce_kv(const Setup<Gm> &su, const CUtensorMa
                 break;
             ptx::mbar_arrive_expect_tx(su.bars.k_full(s), kTile);
             load_kv_tile<Gm>(su.sK + s * kTile, tmK, su.bars.k_full(s), kb + i * BN, b, hk, Hkv,
-                         pages, seq_end, dev_status);
+                             pages, pc, seq_end, dev_status);
         }
         if (i >= 1) {
             const int j = i - 1, s = j % NSV;
@@ -333,7 +364,7 @@ __device__ __forceinline__ void produce_kv(const Setup<Gm> &su, const CUtensorMa
             }
             ptx::mbar_arrive_expect_tx(su.bars.v_full(s), kTile);
             load_kv_tile<Gm>(su.sV + s * kTile, tmV, su.bars.v_full(s), kb + j * BN, b, hk, Hkv,
-                         pages, seq_end, dev_status);
+                             pages, pc, seq_end, dev_status);
         }
     }
 }
@@ -475,6 +506,30 @@ __device__ __forceinline__ float exp_pack32(const uint32_t (&sa)[32], float scal
         ptx::fma2_bc(x0, x1, __uint_as_float(sa[2 * k]), __uint_as_float(sa[2 * k + 1]),
                      scale_log2, neg_m);
         const float p0 = ptx::ex2(x0), p1 = ptx::ex2(x1);
+        const int a = (k & 1) * 2;
+        ptx::add2(acc[a], acc[a + 1], p0, p1);
+        pk[k] = ptx::pack_bf16(p0, p1);
+    }
+    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
+// exp_pack32 with NF of its 16 score pairs (spread evenly) exponentiated on
+// the FMA pipe (ptx::exp2_fma) and the rest on MUFU: with two softmax warps
+// per sub-partition the MUFU unit, not issue, bounds the exponentials, and
+// the FMA pipe has room for part of them.
+template <int NF>
+__device__ __forceinline__ float exp_pack32_mix(const uint32_t (&sa)[32], float scale_log2,
+                                                float neg_m, uint32_t (&pk)[16])
+{
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        float x0, x1;
+        ptx::fma2_bc(x0, x1, __uint_as_float(sa[2 * k]), __uint_as_float(sa[2 * k + 1]),
+                     scale_log2, neg_m);
+        const bool poly = (k * NF) % 16 < NF;
+        const float p0 = poly ? ptx::exp2_fma(x0) : ptx::ex2(x0);
+        const float p1 = poly ? ptx::exp2_fma(x1) : ptx::ex2(x1);
         const int a = (k & 1) * 2;
         ptx::add2(acc[a], acc[a + 1], p0, p1);
         pk[k] = ptx::pack_bf16(p0, p1);
@@ -706,7 +761,7 @@ __device__ __forceinline__ bool pair_exchange(const Setup<Gm> &su, int quarter, 
     return ok;
 }
 
-template <class Gm, typename WaitPrev>
+template <class Gm, int NF, typename WaitPrev>
 __device__ __forceinline__ bool softmax_half_tile(const Setup<Gm> &su, uint32_t taddr_s,
                                                   uint32_t taddr_o, int pos0, int P, int ke,
                                                   const uint32_t (&mw)[4], float scale_log2,
@@ -731,7 +786,7 @@ __device__ __forceinline__ bool softmax_half_tile(const Setup<Gm> &su, uint32_t 
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
             uint32_t pk[16];
-            lsum += exp_pack32(sr[c], scale_log2, neg_m, pk);
+            lsum += exp_pack32_mix<NF>(sr[c], scale_log2, neg_m, pk);
             ptx::tmem_st16(taddr_s + c * 16, pk);
         }
         if (pass == 1)
@@ -812,7 +867,7 @@ __device__ __forceinline__ bool softmax_half_tile(const Setup<Gm> &su, uint32_t 
 template <int SW>
 constexpr int rows_threads() { return 64 + 128 * SW; }
 
-template <class Gm, int NS, int kMinBlocks, int SW>
+template <class Gm, int NS, int kMinBlocks, int SW, int NF = 0>
 __global__ void __launch_bounds__(rows_threads<SW>(), kMinBlocks)
     tree_attn_rows_kernel(const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV,
@@ -851,8 +906,9 @@ __global__ void __launch_bounds__(rows_threads<SW>(), kMinBlocks)
     constexpr uint32_t kO = NS * BN;
 
     if (warp == 0) {
+        const PageCache pc = stage_pages(su, pages, b, kb, min(ke, P + T), lane);
         if (lane == 0)
-            produce_kv<Gm, NS>(su, &tmK, &tmV, b, hk, Hkv, kb, ntiles, pages, P + T,
+            produce_kv<Gm, NS>(su, &tmK, &tmV, b, hk, Hkv, kb, ntiles, pages, pc, P + T,
                                dev_status);
     } else if (warp == 1) {
         bool ok = warp_wait(su.bars.q_full(), 0, su.abort_flag);
@@ -918,7 +974,7 @@ __global__ void __launch_bounds__(rows_threads<SW>(), kMinBlocks)
                                            P, ke, mw, scale_log2, j == 0, m_run, l_run,
                                            wait_prev);
             else
-                ok = softmax_half_tile(su, su.tmem + lane_off + col_s(j) + hf * 64, taddr_o,
+                ok = softmax_half_tile<Gm, NF>(su, su.tmem + lane_off + col_s(j) + hf * 64, taddr_o,
                                        kb + j * BN + hf * 64, P, ke, mw, scale_log2, j == 0, hf,
                                        quarter, xc, nx, m_run, l_run, wait_prev);
             if (!ok)
@@ -991,8 +1047,9 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
     auto col_o = [](int s) { return 256u + (uint32_t)s * 128u; };
 
     if (warp == 0) {
+        const PageCache pc = stage_pages(su, pages, b, kb, min(ke, P + T), lane);
         if (lane == 0)
-            produce_kv<Gm, 0>(su, &tmK, &tmV, b, hk, Hkv, kb, ntiles, pages, P + T,
+            produce_kv<Gm, 0>(su, &tmK, &tmV, b, hk, Hkv, kb, ntiles, pages, pc, P + T,
                               dev_status);
     } else if (warp == 1) {
         bool ok = warp_wait(su.bars.q_full(), 0, su.abort_flag);
@@ -1120,6 +1177,7 @@ struct UmmaPlan {
     bool keysplit;   // at most 128 packed rows
     bool paired;     // rows kernel with 64-key tiles, two CTAs per SM
     int sw;          // 128-key rows kernel: softmax warps per TMEM lane quarter
+    int nf;          // with sw = 2: score pairs of 16 exponentiated on the FMA pipe
     int nrb, nsplit, keys_per_split;
 };
 
@@ -1130,6 +1188,16 @@ int rows_softmax_warps()
 {
     const char *e = std::getenv("TSD_ATTN_SOFTMAX_WARPS");
     return (e && e[0] == '2' && e[1] == '\0') ? 2 : 1;
+}
+
+// With two softmax warps per quarter: of every 16 score pairs, how many are
+// exponentiated on the FMA pipe (0, 4 or 6; TSD_ATTN_EXP_FMA, read at every
+// launch).
+int rows_exp_fma()
+{
+    const char *e = std::getenv("TSD_ATTN_EXP_FMA");
+    const int n = e ? std::atoi(e) : 0;
+    return (n == 4 || n == 6) ? n : 0;
 }
 
 // Rows-kernel instance for more than 128 packed rows: 1 = 128-key tiles at
@@ -1161,6 +1229,7 @@ UmmaPlan umma_plan(const AttnArgs &a, int num_sms)
     p.keysplit = small && !small_paired();
     p.paired = small ? !p.keysplit : rows_variant() == 2;
     p.sw = (p.keysplit || p.paired) ? 1 : rows_softmax_warps();
+    p.nf = p.sw == 2 ? rows_exp_fma() : 0;
     p.nrb = p.keysplit ? 1 : (a.Tmax * G + BQ - 1) / BQ;
     const int bn = p.paired ? Half::BN : Wide::BN;
     const int slots = num_sms * (p.paired ? 2 : 1);
@@ -1249,13 +1318,16 @@ cudaError_t set_smem_attributes()
     if (done[dev].load())
         return cudaSuccess;
     auto wide = tree_attn_rows_kernel<Wide, 3, 1, 1>;
-    auto wide2 = tree_attn_rows_kernel<Wide, 3, 1, 2>;
+    auto wide2 = tree_attn_rows_kernel<Wide, 3, 1, 2, 0>;
+    auto wide2f4 = tree_attn_rows_kernel<Wide, 3, 1, 2, 4>;
+    auto wide2f6 = tree_attn_rows_kernel<Wide, 3, 1, 2, 6>;
     auto half = tree_attn_rows_kernel<Half, 2, 2, 1>;
     err = cudaFuncSetAttribute(wide, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)Wide::kSmemBytes);
-    if (err == cudaSuccess)
-        err = cudaFuncSetAttribute(wide2, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)Wide::kSmemBytes);
+    for (auto k : {wide2, wide2f4, wide2f6})
+        if (err == cudaSuccess)
+            err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)Wide::kSmemBytes);
     if (err == cudaSuccess)
         err = cudaFuncSetAttribute(tree_attn_keysplit_kernel,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1343,12 +1415,15 @@ int launch_umma_attention(const AttnArgs &a, void *ws, size_t ws_bytes, int num_
                 tmK, tmV, static_cast<const __nv_bfloat16 *>(a.q), a.prefix_len, a.n_nodes,
                 a.mask, a.Tmax, a.Hq, a.Hkv, a.Lmax, W, sl2, p.keys_per_split, p.nsplit,
                 static_cast<__nv_bfloat16 *>(a.out), part_o, part_ml, a.dev_status, a.pages);
-    else if (p.sw == 2)
-        tree_attn_rows_kernel<Wide, 3, 1, 2>
-            <<<grid, rows_threads<2>(), Wide::kSmemBytes, stream>>>(
-                tmK, tmV, static_cast<const __nv_bfloat16 *>(a.q), a.prefix_len, a.n_nodes,
-                a.mask, a.Tmax, a.Hq, a.Hkv, a.Lmax, W, sl2, p.keys_per_split, p.nsplit,
-                static_cast<__nv_bfloat16 *>(a.out), part_o, part_ml, a.dev_status, a.pages);
+    else if (p.sw == 2) {
+        auto kern = p.nf == 6 ? tree_attn_rows_kernel<Wide, 3, 1, 2, 6>
+                  : p.nf == 4 ? tree_attn_rows_kernel<Wide, 3, 1, 2, 4>
+                              : tree_attn_rows_kernel<Wide, 3, 1, 2, 0>;
+        kern<<<grid, rows_threads<2>(), Wide::kSmemBytes, stream>>>(
+            tmK, tmV, static_cast<const __nv_bfloat16 *>(a.q), a.prefix_len, a.n_nodes, a.mask,
+            a.Tmax, a.Hq, a.Hkv, a.Lmax, W, sl2, p.keys_per_split, p.nsplit,
+            static_cast<__nv_bfloat16 *>(a.out), part_o, part_ml, a.dev_status, a.pages);
+    }
     else
         tree_attn_rows_kernel<Wide, 3, 1, 1>
             <<<grid, rows_threads<1>(), Wide::kSmemBytes, stream>>>(
