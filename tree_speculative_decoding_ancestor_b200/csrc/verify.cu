@@ -30,8 +30,10 @@
 //                           token -- the draw costs no barrier.
 //                           Only rows on the accepted path are read.  Partial
 //                           results cross CTAs through one workspace slot per
-//                           CTA and a per-team arrival counter; every wait on
-//                           a counter is bounded (TSD_DEV_TIMEOUT).
+//                           CTA, published by a release-stored exchange number
+//                           that the team's readers poll directly (one round
+//                           trip per exchange); every wait is bounded
+//                           (TSD_DEV_TIMEOUT).
 //
 // Residual distributions are never materialised: p^(n)(x) is recomputed per
 // element from the logits row, the rejected siblings' q rows and their
@@ -62,26 +64,28 @@ constexpr int kWalkMaxCtas = 1024;    // grid cap (sets the workspace slots)
 constexpr unsigned long long kTeamWaitNs = 2000000000ull;   // bound of one barrier wait
 
 struct VerifyWs {
-    double2 *slot;     // [2][kWalkMaxCtas]  per-CTA partials, by barrier parity
-    int2 *team;        // [kWalkMaxCtas]     {arrivals, abort} per team, zeroed per call
+    double2 *slot;     // [2][kWalkMaxCtas]  per-CTA partials, by exchange parity
+    int *tag;          // [2][kWalkMaxCtas]  exchange number each slot holds  } zeroed
+    int *abort;        // [kWalkMaxCtas]     per-team abort flag              } per call
     int32_t *argmax;   // [B][Tmax+1]        greedy: argmax of rows with children
 };
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-// Fixed part first: the stochastic call uses only that.
-constexpr size_t kWalkBytes = ((2 * kWalkMaxCtas * sizeof(double2) + 255) & ~(size_t)255) +
-                              ((kWalkMaxCtas * sizeof(int2) + 255) & ~(size_t)255);
+// Fixed part first: the stochastic call uses only that.  The tags and the
+// abort flags are contiguous (one memset per call).
+constexpr size_t kSlotBytes = (2 * kWalkMaxCtas * sizeof(double2) + 255) & ~(size_t)255;
+constexpr size_t kZeroedBytes = (3 * kWalkMaxCtas * sizeof(int) + 255) & ~(size_t)255;
+constexpr size_t kWalkBytes = kSlotBytes + kZeroedBytes;
 
 VerifyWs carve(void *ws)
 {
     char *p = static_cast<char *>(ws);
     VerifyWs w;
     w.slot = reinterpret_cast<double2 *>(p);
-    p += align256(2 * kWalkMaxCtas * sizeof(double2));
-    w.team = reinterpret_cast<int2 *>(p);
-    p += align256(kWalkMaxCtas * sizeof(int2));
-    w.argmax = reinterpret_cast<int32_t *>(p);
+    w.tag = reinterpret_cast<int *>(p + kSlotBytes);
+    w.abort = w.tag + 2 * kWalkMaxCtas;
+    w.argmax = reinterpret_cast<int32_t *>(p + kWalkBytes);
     return w;
 }
 
@@ -204,6 +208,97 @@ template <int NT>
 __device__ int block_max_int(int v, int *sh)
 {
     return -block_min_int<NT>(-v, sh);
+}
+
+// The CTA's (max m, z = sum exp((l - m)/T), largest index last) from every
+// thread's own triple, in one block reduction: merging two triples keeps the
+// larger max and rescales the other side's sum to it.
+template <int NT>
+__device__ void block_max_z_last(float &m, double &z, int &last, double inv_temp,
+                                 const double *table, float *shf, double *shd, int *shi)
+{
+    constexpr int NW = NT / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    auto merge = [&](float m2, double z2, int l2) {
+        last = max(last, l2);
+        if (m2 == -INFINITY)
+            return;
+        if (m == -INFINITY) {
+            m = m2;
+            z = z2;
+        } else if (m2 > m) {
+            z = z * table_exp(((double)m - (double)m2) * inv_temp, table) + z2;
+            m = m2;
+        } else {
+            z += z2 * table_exp(((double)m2 - (double)m) * inv_temp, table);
+        }
+    };
+    auto warp_reduce = [&]() {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+            const double z2 = __shfl_xor_sync(0xffffffffu, z, o);
+            const int l2 = __shfl_xor_sync(0xffffffffu, last, o);
+            merge(m2, z2, l2);
+        }
+    };
+    warp_reduce();
+    if (lane == 0) {
+        shf[warp] = m;
+        shd[warp] = z;
+        shi[warp] = last;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        m = lane < NW ? shf[lane] : -INFINITY;
+        z = lane < NW ? shd[lane] : 0.0;
+        last = lane < NW ? shi[lane] : -1;
+        warp_reduce();
+        if (lane == 0) {
+            shf[0] = m;
+            shd[0] = z;
+            shi[0] = last;
+        }
+    }
+    __syncthreads();
+    m = shf[0];
+    z = shd[0];
+    last = shi[0];
+    __syncthreads();
+}
+
+// The CTA's (sum s, largest index last) in one block reduction.
+template <int NT>
+__device__ void block_sum_last(double &s, int &last, double *shd, int *shi)
+{
+    constexpr int NW = NT / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    auto warp_reduce = [&]() {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            s += __shfl_xor_sync(0xffffffffu, s, o);
+            last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
+        }
+    };
+    warp_reduce();
+    if (lane == 0) {
+        shd[warp] = s;
+        shi[warp] = last;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        s = lane < NW ? shd[lane] : 0.0;
+        last = lane < NW ? shi[lane] : -1;
+        warp_reduce();
+        if (lane == 0) {
+            shd[0] = s;
+            shi[0] = last;
+        }
+    }
+    __syncthreads();
+    s = shd[0];
+    last = shi[0];
+    __syncthreads();
 }
 
 // Row argmax (lowest index among the maxima); four float4 loads in flight.
@@ -347,11 +442,9 @@ __device__ double2 chunk_max_z(const float *__restrict__ row, int x_lo, int x_hi
         group(l0, x0);
         group(l1, x1);
     }
-    *last_out = block_max_int<kWalkThreads>(last, shi);
-    const float mk = block_max<kWalkThreads>(mt, shf);
-    const double zs =
-        mt == -INFINITY ? 0.0 : zt * table_exp(((double)mt - (double)mk) * inv_temp, table);
-    return make_double2((double)mk, block_sum<kWalkThreads>(zs, shd));
+    block_max_z_last<kWalkThreads>(mt, zt, last, inv_temp, table, shf, shd, shi);
+    *last_out = last;
+    return make_double2((double)mt, mt == -INFINITY ? 0.0 : zt);
 }
 
 // Over the CTA's chunk: sum max(0, p^(n)(x) - q(x)) and (in *last) the
@@ -384,8 +477,9 @@ __device__ double chunk_residual(const float *__restrict__ row, const float *__r
                 last = max(last, x1 + k);
         }
     }
-    *last_out = block_max_int<kWalkThreads>(last, shi);
-    return block_sum<kWalkThreads>(s, shd);
+    block_sum_last<kWalkThreads>(s, last, shd, shi);
+    *last_out = last;
+    return s;
 }
 
 // The draw inside the chunk [x_lo, x_hi): the smallest x with
@@ -596,10 +690,11 @@ __global__ void __launch_bounds__(kWalkThreads)
     const int x_lo = min(k * chunk, V), x_hi = min(x_lo + chunk, V);
     const double inv_temp = 1.0 / temp;
     const bool lead = k == 0 && tid == 0;   // writes the path and the error codes
-    int2 *tm = ws.team + team;
-    int nbar = 0;
-    // this CTA's slot / the team's K slots of the next barrier
-    auto slots = [&]() { return ws.slot + (nbar & 1) * kWalkMaxCtas + team * K; };
+    int *abort = ws.abort + team;
+    int nbar = 0;   // exchanges made
+    // the team's K slots and tags of the next exchange
+    auto slots = [&]() { return ws.slot + ((nbar + 1) & 1) * kWalkMaxCtas + team * K; };
+    auto tags = [&]() { return ws.tag + ((nbar + 1) & 1) * kWalkMaxCtas + team * K; };
     fill_exp_table(table, 1.0);   // read only from here on (barriers below publish it)
 
     for (int b = team; b < B; b += teams) {
@@ -635,16 +730,16 @@ __global__ void __launch_bounds__(kWalkThreads)
             double2 *sl = slots();
             if (tid == 0)
                 sl[k] = make_double2(mz.y, __hiloint2double(__float_as_int((float)mz.x), lastk));
-            ++nbar;
-            if (!team_barrier(tm, nbar * K, &sh_ok, kTeamWaitNs)) {
+            double2 v = make_double2(0.0, 0.0);
+            if (!team_exchange(sl, tags(), k, K, nbar + 1, abort, v, &sh_ok, kTeamWaitNs)) {
                 alive = false;
                 break;
             }
+            ++nbar;
             if (warp == 0) {
                 double mk = -INFINITY, zk = 0.0;
                 int lk = -1;
                 if (lane < K) {
-                    const double2 v = __ldcg(sl + lane);
                     zk = v.x;
                     mk = (double)__int_as_float(__double2hiint(v.y));
                     lk = __double2loint(v.y);
@@ -691,16 +786,16 @@ __global__ void __launch_bounds__(kWalkThreads)
                 sl = slots();
                 if (tid == 0)
                     sl[k] = make_double2(s, (double)lastk);
-                ++nbar;
-                if (!team_barrier(tm, nbar * K, &sh_ok, kTeamWaitNs)) {
+                double2 v = make_double2(0.0, 0.0);
+                if (!team_exchange(sl, tags(), k, K, nbar + 1, abort, v, &sh_ok, kTeamWaitNs)) {
                     alive = false;
                     break;
                 }
+                ++nbar;
                 if (warp == 0) {
                     double sk = 0.0;
                     int lk = -1;
                     if (lane < K) {
-                        const double2 v = __ldcg(sl + lane);
                         sk = v.x;
                         lk = (int)v.y;
                     }
@@ -899,7 +994,7 @@ int launch_verify_stochastic(const float *logits, double temperature, const floa
     if (walk_grid(B, V, K, teams, chunk) != TSD_OK)
         return TSD_ERR_CUDA;
     VerifyWs w = carve(ws);
-    if (cudaMemsetAsync(w.team, 0, (size_t)teams * sizeof(int2), stream) != cudaSuccess) {
+    if (cudaMemsetAsync(w.tag, 0, kZeroedBytes, stream) != cudaSuccess) {
         (void)cudaGetLastError();
         return TSD_ERR_CUDA;
     }
