@@ -618,6 +618,13 @@ def main():
     ms_per_step = total_ms / args.steps
     value = job_tokens / (ms_per_step / 1e3)
     acceptance = accepted_summary(w, step)
+    gathered = None
+    if pg is not None:
+        # the batch-sharded path's optional collective, outside the timed
+        # steps: every rank's verify results on every rank (same call order
+        # on every rank)
+        res = step.s if "stochastic" in w.verify else step.g
+        gathered = int(tsd.all_gather_accepted(res).n_accepted.shape[0])
     side = {}
     if not args.no_side:
         side["kv_commit"] = time_commit(step, dev, tsd)
@@ -651,6 +658,8 @@ def main():
             "roofline_step": step_roofline(w, step, statistics.mean(t["step_ms"]), peaks),
             "gpu_launches": t["launches"], "clocks": t["clocks"],
             "acceptance": acceptance}
+    if gathered is not None:
+        line["gathered_sequences"] = gathered
     line.update(side)
 
     if not args.no_e2e:

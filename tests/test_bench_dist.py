@@ -84,6 +84,54 @@ def test_ranks_verify_different_sequences():
     assert res[0][1] == int(w0.n_nodes.sum())
 
 
+def _gather_main(rank, world, port, out_q):
+    import torch.distributed as dist
+
+    from tree_speculative_decoding_ancestor_b200 import VerifyResult, all_gather_accepted
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        B, Tmax = (2, 3, 1)[rank], 4
+        base = 100 * rank
+        res = VerifyResult(torch.arange(B * (Tmax + 1), dtype=torch.int32).view(B, Tmax + 1) + base,
+                           torch.arange(B * Tmax, dtype=torch.int32).view(B, Tmax) + base,
+                           torch.arange(B, dtype=torch.int32) + base)
+        got = all_gather_accepted(res)
+        out_q.put((rank, [t.tolist() for t in got]))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_all_gather_accepted_concatenates_in_rank_order(world):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_gather_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = {}
+    try:
+        for _ in range(world):
+            rank, got = q.get(timeout=120)
+            res[rank] = got
+    finally:
+        for p in procs:
+            p.join(timeout=60)
+            if p.is_alive():
+                p.kill()
+    assert all(p.exitcode == 0 for p in procs)
+    sizes, Tmax = (2, 3, 1)[:world], 4
+    want_n = [100 * r + b for r in range(world) for b in range(sizes[r])]
+    want_path = [[100 * r + b * Tmax + j for j in range(Tmax)]
+                 for r in range(world) for b in range(sizes[r])]
+    for r in range(world):
+        assert res[r][2] == want_n
+        assert res[r][1] == want_path
+        assert len(res[r][0]) == sum(sizes) and len(res[r][0][0]) == Tmax + 1
+
+
 def test_single_process_passthrough():
     assert bench.reduce_over_ranks(None, torch.device("cpu"), 11, 1.5) == (11, 1.5)
 

@@ -10,7 +10,9 @@ Six operations, each a thin wrapper over the C ABI of ``lib/libtsd.so``
 * :func:`tree_verify_stochastic` -- multi-step speculative sampling (exact target distribution);
 * :func:`kv_commit`           -- move the accepted nodes' K/V rows after the prefix;
 * :func:`tree_expand`, :func:`tree_merge_chains`, :func:`tree_dfs_order` -- build the
-  token tree (expansion top-k levels, merge of several SSMs' chains, depth-first order).
+  token tree (expansion top-k levels, merge of several SSMs' chains, depth-first order);
+* :func:`all_gather_accepted` -- with one batch per GPU, every rank's verification
+  results on every rank (the batch-sharded path's only collective, optional).
 """
 
 from .binding import (  # noqa: F401
@@ -38,3 +40,4 @@ from .binding import (  # noqa: F401
     verify_stochastic_plan,
     verify_workspace_size,
 )
+from .dist import all_gather_accepted  # noqa: F401
