@@ -62,6 +62,8 @@ constexpr int kTeamMax = 32;          // CTAs per team: one partial per lane of 
 constexpr int kTeamMinChunk = 2048;   // vocabulary entries per CTA, at least
 constexpr int kWalkMaxCtas = 1024;    // grid cap (sets the workspace slots)
 constexpr unsigned long long kTeamWaitNs = 2000000000ull;   // bound of one barrier wait
+constexpr int kDecCache = 8;          // children per row whose test operands are prefetched
+constexpr int kDecOps = 2 * kDecCache + kDecCache * (kDecCache + 1) / 2;   // 52 loads
 
 struct VerifyWs {
     double2 *slot;     // [2][kWalkMaxCtas]  per-CTA partials, by exchange parity
@@ -684,6 +686,13 @@ __global__ void __launch_bounds__(kWalkThreads)
     // date by every pass, so the draw needs no pass of its own
     __shared__ double draw_sum[32];
     __shared__ int draw_last[32];
+    // the sequence's tree (child lists, tokens, q rows), staged once
+    __shared__ int s_fc[kMaxTree + 1], s_ns[kMaxTree], s_tok[kMaxTree], s_qr[kMaxTree];
+    // the operands of the acceptance tests of the current row's first
+    // kDecCache children, loaded while the row's m/Z pass runs:
+    // dc[i] = l(x_i), dc[kDecCache + i] = u_i, dc[2 kDecCache + i(i+1)/2 + j] =
+    // q_j(x_i) for j <= i (q_j: the q row of child j; j = i: the child's own)
+    __shared__ double dc[kDecOps];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int teams = gridDim.x / K;
     const int team = blockIdx.x / K, k = blockIdx.x % K;
@@ -705,9 +714,15 @@ __global__ void __launch_bounds__(kWalkThreads)
             continue;
         }
         int bad = 0;
-        for (int u = tid; u < T; u += kWalkThreads) {
+        for (int u = tid; u <= T; u += kWalkThreads) {
+            s_fc[u] = first_child[(size_t)b * (Tmax + 1) + u];
+            if (u == T)
+                break;
             const int x = tokens[(size_t)b * Tmax + u];
             const int qr = q_row[(size_t)b * Tmax + u];
+            s_tok[u] = x;
+            s_qr[u] = qr;
+            s_ns[u] = next_sibling[(size_t)b * Tmax + u];
             bad |= (x < 0 || x >= V) ? TSD_DEV_BAD_TOKEN : 0;
             bad |= (qr < 0 || qr >= Rq) ? TSD_DEV_BAD_QROW : 0;
         }
@@ -718,15 +733,84 @@ __global__ void __launch_bounds__(kWalkThreads)
                 n_accepted[b] = -1;
             continue;
         }
+        // child i (ascending index) of the node whose logits row is `row`; -1
+        // past the last (the lists come from the mask build: they are
+        // increasing and inside the tree)
+        auto child = [&](int row, int i) {
+            int c = s_fc[row];
+            for (; c >= 0 && i > 0; --i)
+                c = (c < T) ? s_ns[c] : -1;
+            return (c >= 0 && in_bounds(c, T, dev_status)) ? c : -1;
+        };
+        auto qrow = [&](int c) { return q_probs + ((size_t)b * Rq + s_qr[c]) * V; };
         int row = 0, n_path = 0;
         bool alive = true;
         for (;;) {
             const size_t ri = (size_t)b * (Tmax + 1) + row;
             const float *lrow = logits + ri * V;
+            // issue the acceptance-test operands' loads (consumed after the
+            // exchange below: their latency hides behind the pass)
+            double pre = 0.0;
+            int op = -1;
+            if (tid < kDecOps) {
+                int i = -1, j = -1;
+                if (tid < kDecCache)
+                    i = tid;
+                else if (tid < 2 * kDecCache)
+                    i = tid - kDecCache;
+                else {
+                    const int t2 = tid - 2 * kDecCache;   // i (i + 1) / 2 + j, j <= i
+                    i = 0;
+                    while ((i + 1) * (i + 2) / 2 <= t2)
+                        ++i;
+                    j = t2 - i * (i + 1) / 2;
+                }
+                const int ci = child(row, i);
+                if (ci >= 0) {
+                    const int x = s_tok[ci];
+                    if (tid < kDecCache) {
+                        pre = (double)__ldg(lrow + x);
+                    } else if (tid < 2 * kDecCache) {
+                        pre = __ldg(u_accept + (size_t)b * Tmax + ci);
+                    } else {
+                        const int cj = child(row, j);
+                        pre = (double)__ldg(qrow(cj) + x);
+                    }
+                    op = tid;
+                }
+            }
+            // lane 0 of warp 0: the acceptance test of child i, given the
+            // row's m, Z and the i siblings rejected before it (in st)
+            auto accept = [&](int i, int c) {
+                const int x = s_tok[c];
+                double lx, qx, u;
+                if (i < kDecCache) {
+                    lx = dc[i];
+                    u = dc[kDecCache + i];
+                    qx = dc[2 * kDecCache + i * (i + 1) / 2 + i];
+                } else {
+                    lx = (double)lrow[x];
+                    u = u_accept[(size_t)b * Tmax + c];
+                    qx = (double)qrow(c)[x];
+                }
+                double p = exp((lx - st.m) / st.temp) / st.Z;
+                for (int j = 0; j < st.n; ++j) {
+                    if (st.S[j] > 0.0) {
+                        const double qj = i < kDecCache
+                                              ? dc[2 * kDecCache + i * (i + 1) / 2 + j]
+                                              : (double)st.q[j][x];
+                        const double r = p - qj;
+                        p = (r > 0.0 ? r : 0.0) / st.S[j];
+                    }
+                }
+                return (p > 0.0 && u * qx <= p) ? 1 : 0;
+            };
             // m and Z of this row (slot: z_k, then m_k as fp32 bits | last_k)
             int lastk;
             const double2 mz =
                 chunk_max_z<VEC>(lrow, x_lo, x_hi, V, inv_temp, table, shf, shd, shi, &lastk);
+            if (op >= 0)
+                dc[op] = pre;
             double2 *sl = slots();
             if (tid == 0)
                 sl[k] = make_double2(mz.y, __hiloint2double(__float_as_int((float)mz.x), lastk));
@@ -736,6 +820,7 @@ __global__ void __launch_bounds__(kWalkThreads)
                 break;
             }
             ++nbar;
+            int c = child(row, 0);   // the children in ascending index
             if (warp == 0) {
                 double mk = -INFINITY, zk = 0.0;
                 int lk = -1;
@@ -760,27 +845,17 @@ __global__ void __launch_bounds__(kWalkThreads)
                     st.temp = temp;
                     st.inv_temp = inv_temp;
                     st.n = 0;
+                    sh_dec = c >= 0 ? accept(0, c) : 0;
                 }
             }
             __syncthreads();
-            // the children in ascending index
             int accepted = -1;
-            for (int c = first_child[ri]; c >= 0; c = next_sibling[(size_t)b * Tmax + c]) {
-                if (!in_bounds(c, Tmax, dev_status))
-                    break;   // the same in every CTA of the team (they read the same c)
-                const int x = tokens[(size_t)b * Tmax + c];
-                const float *qc = q_probs + ((size_t)b * Rq + q_row[(size_t)b * Tmax + c]) * V;
-                if (tid == 0) {
-                    const double px = p_exact(lrow[x], x, st);
-                    const double qx = (double)qc[x];
-                    const double u = u_accept[(size_t)b * Tmax + c];
-                    sh_dec = (px > 0.0 && u * qx <= px) ? 1 : 0;
-                }
-                __syncthreads();
+            for (int i = 0; c >= 0; ++i) {
                 if (sh_dec) {
                     accepted = c;
                     break;
                 }
+                const float *qc = qrow(c);
                 const double s =
                     chunk_residual<VEC>(lrow, qc, x_lo, x_hi, V, st, table, shd, shi, &lastk);
                 sl = slots();
@@ -792,6 +867,7 @@ __global__ void __launch_bounds__(kWalkThreads)
                     break;
                 }
                 ++nbar;
+                const int next = child(row, i + 1);
                 if (warp == 0) {
                     double sk = 0.0;
                     int lk = -1;
@@ -809,17 +885,18 @@ __global__ void __launch_bounds__(kWalkThreads)
                         st.S[st.n] = S;
                         st.inv_S[st.n] = S > 0.0 ? 1.0 / S : 0.0;
                         st.n += 1;
+                        sh_dec = next >= 0 ? accept(i + 1, next) : 0;
                     }
                 }
                 __syncthreads();
+                c = next;
             }
             if (!alive)
                 break;
             if (accepted >= 0 && n_path < T) {
                 if (lead && in_bounds(n_path, Tmax, dev_status)) {
                     out_path[(size_t)b * Tmax + n_path] = accepted;
-                    out_tokens[(size_t)b * (Tmax + 1) + n_path] =
-                        tokens[(size_t)b * Tmax + accepted];
+                    out_tokens[(size_t)b * (Tmax + 1) + n_path] = s_tok[accepted];
                 }
                 ++n_path;
                 row = accepted + 1;
