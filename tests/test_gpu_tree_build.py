@@ -24,8 +24,12 @@ def _q(seed, B, R, V, ties):
     return q
 
 
+# k <= 8 takes the one-pass register top-k (lists of 2, 4 or 8 per thread),
+# k > 8 one block pass per child; V % 4 != 0 takes the scalar loads.
 @pytest.mark.parametrize("ks,V,ties", [((2, 3, 2), 1000, False), ((1, 1, 3, 1, 1, 1, 1, 1), 32000, False),
-                                       ((4, 2), 37, True), ((5, 5, 2), 128256, False)])
+                                       ((4, 2), 37, True), ((5, 5, 2), 128256, False),
+                                       ((8, 2), 600, True), ((9, 3), 1000, True),
+                                       ((7, 6), 1001, False), ((16,), 40, True)])
 def test_expansion_matches_oracle(cuda_device, ks, V, ties):
     B, Tmax = 3, 128
     dev = cuda_device

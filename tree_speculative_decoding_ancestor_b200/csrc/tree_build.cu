@@ -6,11 +6,13 @@
 //
 //   tree_expand_kernel        one CTA per (frontier node, sequence): the k best
 //                             tokens of the node's SSM row (descending
-//                             probability, lower token id on ties) in k block
-//                             passes (8 loads in flight per thread), each
-//                             taking the best element strictly after the
-//                             previous pick in that order -- a compare and a
-//                             select per element; writes the children at
+//                             probability, lower token id on ties).  k <= 8:
+//                             one pass (8 loads in flight per thread), each
+//                             thread keeping its best k in registers, then k
+//                             block arg-best rounds over the threads' lists;
+//                             k > 8: k block passes, each taking the best
+//                             element strictly after the previous pick in
+//                             that order.  Writes the children at
 //                             n_nodes + i*k + j;
 //   tree_expand_commit_kernel one thread per sequence: n_nodes and lvl_begin
 //                             advance once every CTA has read them;
@@ -102,6 +104,83 @@ __device__ __forceinline__ void block_best(float &v, int &i, float *shv, int *sh
     __syncthreads();
 }
 
+// The k <= KM best entries of a row (descending probability, lower token id
+// on ties) in one pass: every thread keeps its own best KM in registers,
+// sorted, inserting each element with a branch-free compare-and-shift (no
+// divergence however often lanes insert); then k rounds of a block arg-best
+// over the threads' list heads, the winner popping its head.  `emit(j, x)`
+// is called by thread 0 with the j-th best token.
+template <int KM, typename Emit>
+__device__ __forceinline__ void row_topk_one_pass(const float *__restrict__ p, int V, bool vec,
+                                                  int k, float *shv, int *shi, Emit emit)
+{
+    float lv[KM];
+    int li[KM];
+#pragma unroll
+    for (int m = 0; m < KM; ++m) {
+        lv[m] = -INFINITY;
+        li[m] = INT_MAX;
+    }
+    auto insert = [&](float v, int x) {
+        bool c[KM];   // c[m]: (v, x) goes before entry m; monotone in m
+#pragma unroll
+        for (int m = 0; m < KM; ++m)
+            c[m] = li[m] == INT_MAX || before(v, x, lv[m], li[m]);
+#pragma unroll
+        for (int m = KM - 1; m > 0; --m) {
+            lv[m] = c[m - 1] ? lv[m - 1] : (c[m] ? v : lv[m]);
+            li[m] = c[m - 1] ? li[m - 1] : (c[m] ? x : li[m]);
+        }
+        lv[0] = c[0] ? v : lv[0];
+        li[0] = c[0] ? x : li[0];
+    };
+    if (vec) {   // float4 loads, kLoadBatch in flight per thread
+        const float4 *p4 = reinterpret_cast<const float4 *>(p);
+        const int n4 = V >> 2;
+        int x4 = threadIdx.x;
+        for (; x4 + (kLoadBatch - 1) * kExpandThreads < n4; x4 += kLoadBatch * kExpandThreads) {
+            float4 t[kLoadBatch];
+#pragma unroll
+            for (int u = 0; u < kLoadBatch; ++u)
+                t[u] = __ldg(p4 + x4 + u * kExpandThreads);
+#pragma unroll
+            for (int u = 0; u < kLoadBatch; ++u) {
+                const int x = 4 * (x4 + u * kExpandThreads);
+                insert(t[u].x, x);
+                insert(t[u].y, x + 1);
+                insert(t[u].z, x + 2);
+                insert(t[u].w, x + 3);
+            }
+        }
+        for (; x4 < n4; x4 += kExpandThreads) {
+            const float4 t = __ldg(p4 + x4);
+            insert(t.x, 4 * x4);
+            insert(t.y, 4 * x4 + 1);
+            insert(t.z, 4 * x4 + 2);
+            insert(t.w, 4 * x4 + 3);
+        }
+    } else {
+        for (int x = threadIdx.x; x < V; x += kExpandThreads)
+            insert(__ldg(p + x), x);
+    }
+    for (int j = 0; j < k; ++j) {
+        float bv = lv[0];
+        int bi = li[0];
+        block_best(bv, bi, shv, shi);
+        if (li[0] == bi && bi != INT_MAX) {   // this thread's head won: pop it
+#pragma unroll
+            for (int m = 0; m < KM - 1; ++m) {
+                lv[m] = lv[m + 1];
+                li[m] = li[m + 1];
+            }
+            lv[KM - 1] = -INFINITY;
+            li[KM - 1] = INT_MAX;
+        }
+        if (threadIdx.x == 0)
+            emit(j, bi);
+    }
+}
+
 __global__ void __launch_bounds__(kExpandThreads)
     tree_expand_kernel(const float *__restrict__ q_probs, int Rq, int V,
                        const int32_t *__restrict__ frow, int k, int32_t *__restrict__ parent,
@@ -131,6 +210,27 @@ __global__ void __launch_bounds__(kExpandThreads)
     const int r = frow[(size_t)b * Tmax + i];
     const float *p = q_probs + ((size_t)b * Rq + r) * V;
     const bool vec = (V & 3) == 0 && (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+    auto emit = [&](int j, int tok) {
+        if (in_bounds(n + i * k + j, Tmax, nullptr)) {
+            const size_t u = (size_t)b * Tmax + n + i * k + j;
+            parent[u] = n == 0 ? -1 : lb + i;
+            tokens[u] = tok;   // k <= V: a pick always exists
+            q_row[u] = r;
+        }
+    };
+    // up to 8 children: one pass over the row; more: one pass per child
+    if (k <= 2) {
+        row_topk_one_pass<2>(p, V, vec, k, shv, shi, emit);
+        return;
+    }
+    if (k <= 4) {
+        row_topk_one_pass<4>(p, V, vec, k, shv, shi, emit);
+        return;
+    }
+    if (k <= 8) {
+        row_topk_one_pass<8>(p, V, vec, k, shv, shi, emit);
+        return;
+    }
     float pv = 0.f;
     int pi = -1;
     for (int j = 0; j < k; ++j) {
@@ -187,12 +287,8 @@ __global__ void __launch_bounds__(kExpandThreads)
         block_best(bv, bi, shv, shi);
         pv = bv;
         pi = bi;
-        if (threadIdx.x == 0 && in_bounds(n + i * k + j, Tmax, nullptr)) {
-            const size_t u = (size_t)b * Tmax + n + i * k + j;
-            parent[u] = n == 0 ? -1 : lb + i;
-            tokens[u] = pi;   // k <= V: a pick always exists
-            q_row[u] = r;
-        }
+        if (threadIdx.x == 0)
+            emit(j, pi);
     }
 }
 
