@@ -36,14 +36,21 @@ class _Barrier:
 
 
 def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged=True, sw=1,
-         redo_p=0.2):
+         redo_p=0.2, cm=2):
     """merged: the producer reuses a K slot once s_full of the QK that read it
     completes and a V slot once o_ready of the PV that read it completes (the
     rows kernels; the MMA thread then commits only to s_full and o_ready).
     sw = 2: two softmax warps per TMEM lane quarter, each on half of every
     key tile; per tile they exchange their redo votes and, when either voted,
     their row maxima (then both may rescale O), and at the end their row
-    sums -- each exchange a phase of the quarter's pair mbarrier."""
+    sums -- each exchange a phase of the quarter's pair mbarrier.
+    cm = 1: one commit point per key tile -- the first NS QK products
+    commit to s_full alone (phase 0), then after PV_j and QK_{j+NS} one commit
+    point to s_full[j % NS] (phase j / NS + 1: PV_j done, and QK_{j+NS} if it
+    exists) and to the V ring's v_empty[j % NSV]; the softmax's waits for "PV_r
+    done" wait for that s_full phase, the producer reuses V slots on v_empty
+    (a wait for s_full phase j / NS + 1 there could come two phases early on
+    the last tiles, where no K wait precedes it)."""
     rnd = random.Random(seed)
     nsm = 4 * sw
     bars = {"q_full": _Barrier(nsm)}
@@ -77,6 +84,13 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
     pv_done = set()
 
     k_read, v_read = {}, {}   # ring slot -> tile loaded there
+
+    def pv_passed(r):
+        """The wait for "PV_r done" under the commit scheme."""
+        if cm == 1:
+            return passes(("s_full", r % NS), r // NS + 1)
+        return passes(("o_ready", r % NS), r // NS)
+
     qk_done, pv_done_set = set(), set()
 
     def producer():
@@ -98,9 +112,9 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
                 j = i - 1
                 s = j % NSV
                 if j >= NSV:
-                    if merged:   # PV_{j-NSV} done: o_ready[(j - NSV) % NS]
+                    if merged and cm == 2:   # PV_{j-NSV} done: o_ready[(j - NSV) % NS]
                         r = j - NSV
-                        while not passes(("o_ready", r % NS), r // NS):
+                        while not pv_passed(r):
                             yield
                     else:
                         while not passes(("v_empty", s), j // NSV - 1):
@@ -121,7 +135,11 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
             prev = s_owner.get(buf)
             assert prev is None or prev in pv_done or ("pv", prev) in [p[0] for p in pipe], \
                 f"QK_{i} issued over the P of tile {prev} before its PV"
-            commits = [("s_full", buf)] if merged else [("s_full", buf), ("k_empty", i % NSK)]
+            if cm == 1 and i >= NS:
+                commits = []             # covered by the tile's single commit
+            else:
+                commits = [("s_full", buf)] if merged else \
+                    [("s_full", buf), ("k_empty", i % NSK)]
             pipe.append((("qk", i), commits))
             s_owner[buf] = i
         for i in range(min(NS, ntiles)):
@@ -131,11 +149,16 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
                 yield
             while not passes(("v_full", j % NSV), j // NSV):
                 yield
-            commits = [("o_ready", j % NS)] if merged else \
-                [("v_empty", j % NSV), ("o_ready", j % NS)]
+            if cm == 1:
+                commits = []
+            else:
+                commits = [("o_ready", j % NS)] if merged else \
+                    [("v_empty", j % NSV), ("o_ready", j % NS)]
             pipe.append((("pv", j), commits))
             if j + NS < ntiles:
                 yield from qk(j + NS)
+            if cm == 1:   # one commit point: tracks everything issued so far
+                pipe.append((("commit", j), [("s_full", j % NS), ("v_empty", j % NSV)]))
             yield
 
     def exchange(q, n):
@@ -162,7 +185,7 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
                     yield from exchange(q, nx)          # the row maxima
                     nx += 1
             if rescale:                                 # O rescaled: PV_{j-1} done
-                while not passes(("o_ready", (j - 1) % NS), (j - 1) // NS):
+                while not pv_passed(j - 1):
                     yield
                 assert j - 1 in pv_done
             bars["p_full", j % NS].arrive()
@@ -170,7 +193,7 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
         if ntiles:
             last = ntiles - 1
             if final_wait == "o_ready":
-                while not passes(("o_ready", last % NS), last // NS):
+                while not pv_passed(last):
                     yield
             else:                                        # the V ring's barrier instead
                 while not passes(("v_empty", last % NSV), last // NSV):
@@ -191,7 +214,7 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
             (kind, t), commits = pipe.pop(0)
             if kind == "pv":
                 pv_done.add(t)
-            else:
+            elif kind == "qk":
                 qk_done.add(t)
             for name in commits:
                 bars[name].arrive()
@@ -211,6 +234,14 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
 def test_rows_kernel_protocol(NS, NSK, NSV, sw, ntiles):
     for seed in range(150):
         _run(NS, NSK, NSV, ntiles, seed, sw=sw)
+
+
+@pytest.mark.parametrize("NS,NSK,NSV,sw", [(3, 3, 2, 1), (2, 2, 2, 1), (3, 3, 2, 2)],
+                         ids=["128-key tiles", "64-key tiles", "128-key tiles, paired softmax"])
+@pytest.mark.parametrize("ntiles", [1, 2, 3, 4, 5, 8, 17])
+def test_rows_kernel_protocol_one_commit_per_tile(NS, NSK, NSV, sw, ntiles):
+    for seed in range(150):
+        _run(NS, NSK, NSV, ntiles, seed, sw=sw, cm=1)
 
 
 @pytest.mark.parametrize("ntiles", [1, 3, 6])

@@ -80,3 +80,16 @@ def test_verify_traffic_counts_rows_on_the_path():
     # q row 1; node 1's row (a leaf: no children tried)
     st = types.SimpleNamespace(g=res(0, []), s=res(2, [0, 1]))
     assert bench.verify_traffic(w, st)["stochastic"] == 5 * row
+
+
+def test_input_copies_defeat_the_l2():
+    # each workload's inputs are rotated over enough device copies that the
+    # copies read since a copy's last use exceed twice the L2; the tiny one
+    # cannot be, and falls back to the flush
+    for name in ("llama7b", "merge", "gqa70b", "long32k"):
+        w = gen.config_workload(gen.WORKLOAD_NAMES[name])
+        n = bench.input_sets_for(w)
+        nb = bench.input_bytes(w)
+        assert n >= 2 and (n - 1) * nb >= 2 * bench.L2_BYTES, (name, n, nb)
+        assert n * nb <= 4e9
+    assert bench.input_sets_for(gen.config_workload(0)) == 1

@@ -160,6 +160,9 @@ FORCED = [
     ("large", {"TSD_ATTN_ROWS_VARIANT": "2"}, "rows64"),
     ("large", {"TSD_ATTN_SOFTMAX_WARPS": "2"}, "rows128x2"),
     ("large", {"TSD_ATTN_SOFTMAX_WARPS": "2", "TSD_ATTN_EXP_FMA": "6"}, "rows128x2"),
+    ("large", {"TSD_ATTN_COMMITS": "1"}, "rows128"),
+    ("large", {"TSD_ATTN_COMMITS": "1", "TSD_ATTN_SOFTMAX_WARPS": "2"}, "rows128x2"),
+    ("small", {"TSD_ATTN_COMMITS": "1"}, "rows64"),
     ("small", {}, "rows64"),
     ("small", {"TSD_ATTN_SMALL_VARIANT": "keysplit"}, "keysplit"),
     ("small", {"TSD_FORCE_PATH": "simt"}, "simt"),
@@ -173,7 +176,7 @@ def _shape_workload(name):
 
 
 FORCED_IDS = [f"{f[0]}-{f[2]}" + ("-expfma" if "TSD_ATTN_EXP_FMA" in f[1] else "")
-              for f in FORCED]
+              + ("-1commit" if "TSD_ATTN_COMMITS" in f[1] else "") for f in FORCED]
 
 
 @pytest.mark.parametrize("splits", ["1", "3", "64"])
@@ -395,6 +398,12 @@ def _sample_rows(w, n, seed):
 def test_config_full_size_paired_softmax(cuda_device, cfg, nf, monkeypatch):
     monkeypatch.setenv("TSD_ATTN_SOFTMAX_WARPS", "2")
     monkeypatch.setenv("TSD_ATTN_EXP_FMA", nf)
+    test_config_full_size(cuda_device, cfg)
+
+
+@pytest.mark.parametrize("cfg", [1, 3, 4])
+def test_config_full_size_one_commit_per_tile(cuda_device, cfg, monkeypatch):
+    monkeypatch.setenv("TSD_ATTN_COMMITS", "1")
     test_config_full_size(cuda_device, cfg)
 
 

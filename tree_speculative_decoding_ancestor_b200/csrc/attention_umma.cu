@@ -328,7 +328,7 @@ __device__ __forceinline__ void load_kv_tile(uint32_t dst, const CUtensorMap *tm
 // on o_ready[(j - NSV) % NS] -- which saves the MMA thread two commits per
 // tile.  Either wait names a phase that cannot be stale or ahead: the phase
 // after it needs K_i (or V_{j+1}), which this producer has not loaded yet.
-template <class Gm, int NS_PROD>
+template <class Gm, int NS_PROD, int CM = 2>
 __device__ __forceinline__ void produce_kv(const Setup<Gm> &su, const CUtensorMap *tmK,
                                            const CUtensorMap *tmV, int b, int hk, int Hkv,
                                            int kb, int ntiles, const KvPages &pages,
@@ -354,11 +354,17 @@ __device__ __forceinline__ void produce_kv(const Setup<Gm> &su, const CUtensorMa
             const int j = i - 1, s = j % NSV;
             if (j >= NSV) {
                 const int r = j - NSV;   // PV_r read this slot last
+                constexpr int NSP = NS_PROD ? NS_PROD : 1;
+                // PV_r done: the ring's own v_empty (committed by the MMA warp
+                // without NS_PROD, and with one commit point per tile, CM = 1),
+                // or o_ready[r % NS] phase r / NS.  (With CM = 1 a wait for
+                // s_full[r % NS] phase r / NS + 1 could come two phases early on
+                // the last tiles, where no K wait precedes it.)
                 const bool ok =
-                    NS_PROD ? ptx::mbar_wait(su.bars.o_ready(r % (NS_PROD ? NS_PROD : 1)),
-                                             (r / (NS_PROD ? NS_PROD : 1)) & 1, su.abort_flag)
-                            : ptx::mbar_wait(su.bars.v_empty(s), ((j / NSV) - 1) & 1,
-                                             su.abort_flag);
+                    (!NS_PROD || CM == 1)
+                        ? ptx::mbar_wait(su.bars.v_empty(s), ((j / NSV) - 1) & 1, su.abort_flag)
+                        : ptx::mbar_wait(su.bars.o_ready(r % NSP), (r / NSP) & 1,
+                                         su.abort_flag);
                 if (!ok)
                     break;
             }
@@ -370,7 +376,7 @@ __device__ __forceinline__ void produce_kv(const Setup<Gm> &su, const CUtensorMa
 }
 
 // MMA warp, S = Q K^T for key tile `t` into TMEM columns `col_s`.
-template <class Gm, bool RING_COMMIT = true>
+template <class Gm, bool RING_COMMIT = true, bool COMMIT = true>
 __device__ __forceinline__ void issue_qk(const Setup<Gm> &su, int lane, uint32_t col_s, int t,
                                          uint32_t s_full)
 {
@@ -382,8 +388,9 @@ __device__ __forceinline__ void issue_qk(const Setup<Gm> &su, int lane, uint32_t
         for (int kk = 0; kk < HD / 16; ++kk)
             ptx::mma_ss(su.tmem + col_s, dq + slice_off(kk, kSubQ), dk + slice_off(kk, Gm::kSub),
                         idesc, kk > 0 ? 1u : 0u);
-        ptx::mma_commit(s_full);
-        if (RING_COMMIT)
+        if (COMMIT)
+            ptx::mma_commit(s_full);
+        if (COMMIT && RING_COMMIT)
             ptx::mma_commit(su.bars.k_empty(st));
     }
     __syncwarp();
@@ -393,7 +400,7 @@ __device__ __forceinline__ void issue_qk(const Setup<Gm> &su, int lane, uint32_t
 // V rows at or beyond P_b + T_b first.  P_SPLIT: the packed P of keys
 // 64 .. 127 sits 64 columns after that of keys 0 .. 63 (each softmax half
 // writes into its own score columns) instead of right after it.
-template <class Gm, bool RING_COMMIT = true, bool P_SPLIT = false>
+template <class Gm, bool RING_COMMIT = true, bool P_SPLIT = false, bool COMMIT = true>
 __device__ __forceinline__ void issue_pv(const Setup<Gm> &su, int lane, uint32_t col_p,
                                          uint32_t col_o, int t, bool accumulate, int first_bad,
                                          uint32_t o_ready)
@@ -423,9 +430,10 @@ __device__ __forceinline__ void issue_pv(const Setup<Gm> &su, int lane, uint32_t
                         dv + (uint64_t)((kk * 16u * 128u) >> 4), idesc,
                         (accumulate || kk > 0) ? 1u : 0u);
         }
-        if (RING_COMMIT)
+        if (COMMIT && RING_COMMIT)
             ptx::mma_commit(su.bars.v_empty(vs));
-        ptx::mma_commit(o_ready);
+        if (COMMIT)
+            ptx::mma_commit(o_ready);
     }
     __syncwarp();
 }
@@ -867,7 +875,7 @@ __device__ __forceinline__ bool softmax_half_tile(const Setup<Gm> &su, uint32_t 
 template <int SW>
 constexpr int rows_threads() { return 64 + 128 * SW; }
 
-template <class Gm, int NS, int kMinBlocks, int SW, int NF = 0>
+template <class Gm, int NS, int kMinBlocks, int SW, int NF = 0, int CM = 2>
 __global__ void __launch_bounds__(rows_threads<SW>(), kMinBlocks)
     tree_attn_rows_kernel(const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV,
@@ -908,30 +916,45 @@ __global__ void __launch_bounds__(rows_threads<SW>(), kMinBlocks)
     if (warp == 0) {
         const PageCache pc = stage_pages(su, pages, b, kb, min(ke, P + T), lane);
         if (lane == 0)
-            produce_kv<Gm, NS>(su, &tmK, &tmV, b, hk, Hkv, kb, ntiles, pages, pc, P + T,
-                               dev_status);
+            produce_kv<Gm, NS, CM>(su, &tmK, &tmV, b, hk, Hkv, kb, ntiles, pages, pc, P + T,
+                                   dev_status);
     } else if (warp == 1) {
         bool ok = warp_wait(su.bars.q_full(), 0, su.abort_flag);
         ptx::tc_fence_after();
-        auto qk = [&](int i) {
+        // CM = 2: QK_i commits to s_full[i % NS], PV_j to o_ready[j % NS].
+        // CM = 1: one commit point per tile -- after PV_j and QK_{j+NS} (or
+        // PV_j alone for the last NS tiles) to s_full[j % NS], so its phase
+        // j / NS + 1 says both are done (the first NS QKs commit alone, phase
+        // 0), and to the V ring's v_empty[j % NSV] for the producer.
+        auto qk = [&](int i, bool commit) {
             if (!warp_wait(su.bars.k_full(i % NSK), (i / NSK) & 1, su.abort_flag))
                 return false;
             ptx::tc_fence_after();
-            issue_qk<Gm, false>(su, lane, col_s(i), i, su.bars.s_full(i % NS));
+            if (commit)
+                issue_qk<Gm, false, true>(su, lane, col_s(i), i, su.bars.s_full(i % NS));
+            else
+                issue_qk<Gm, false, false>(su, lane, col_s(i), i, su.bars.s_full(i % NS));
             return true;
         };
         for (int i = 0; ok && i < min(NS, ntiles); ++i)
-            ok = qk(i);
+            ok = qk(i, true);
         for (int j = 0; ok && j < ntiles; ++j) {
             if (!warp_wait(su.bars.p_full(j % NS), (j / NS) & 1, su.abort_flag) ||
                 !warp_wait(su.bars.v_full(j % NSV), (j / NSV) & 1, su.abort_flag)) {
                 ok = false;
                 break;
             }
-            issue_pv<Gm, false, SW == 2>(su, lane, col_s(j), kO, j, j > 0,
-                                         P + T - (kb + j * BN), su.bars.o_ready(j % NS));
+            issue_pv<Gm, false, SW == 2, CM == 2>(su, lane, col_s(j), kO, j, j > 0,
+                                                  P + T - (kb + j * BN), su.bars.o_ready(j % NS));
             if (j + NS < ntiles)
-                ok = qk(j + NS);
+                ok = qk(j + NS, CM == 2);
+            if (CM == 1 && ok) {
+                if (lane == 0) {
+                    ptx::mma_commit(su.bars.s_full(j % NS));
+                    ptx::mma_commit(su.bars.v_empty(j % NSV));
+                }
+                __syncwarp();
+            }
         }
     } else {
         // softmax warps: one query row per thread == TMEM lane; with SW = 2
@@ -955,9 +978,12 @@ __global__ void __launch_bounds__(rows_threads<SW>(), kMinBlocks)
             mw[w] = (row_ok && w < W) ? mask[((size_t)b * Tmax + u) * W + w] : 0u;
         const uint32_t taddr_o = su.tmem + lane_off + kO + hf * 64;
         PairXchg *xc = reinterpret_cast<PairXchg *>(su.gbase + Gm::kOffXchg) + quarter;
-        // PV_i done (o_ready[i % NS] completes once per tile of that class)
+        // PV_i done: o_ready[i % NS] phase i / NS, or (CM = 1) s_full[i % NS]
+        // phase i / NS + 1
         auto wait_pv = [&](int i) {
-            return warp_wait(su.bars.o_ready(i % NS), (i / NS) & 1, su.abort_flag);
+            return CM == 1
+                       ? warp_wait(su.bars.s_full(i % NS), ((i / NS) + 1) & 1, su.abort_flag)
+                       : warp_wait(su.bars.o_ready(i % NS), (i / NS) & 1, su.abort_flag);
         };
         float m_run = -INFINITY, l_run = 0.f;
         int nx = 0;   // pair exchanges made
@@ -1178,6 +1204,7 @@ struct UmmaPlan {
     bool paired;     // rows kernel with 64-key tiles, two CTAs per SM
     int sw;          // 128-key rows kernel: softmax warps per TMEM lane quarter
     int nf;          // with sw = 2: score pairs of 16 exponentiated on the FMA pipe
+    int cm;          // rows kernels: commit points per key tile (1 or 2)
     int nrb, nsplit, keys_per_split;
 };
 
@@ -1188,6 +1215,14 @@ int rows_softmax_warps()
 {
     const char *e = std::getenv("TSD_ATTN_SOFTMAX_WARPS");
     return (e && e[0] == '2' && e[1] == '\0') ? 2 : 1;
+}
+
+// Commit points per key tile on the MMA thread: 2 (after QK, after PV), or
+// 1 when TSD_ATTN_COMMITS is "1" (read at every launch).
+int rows_commit_points()
+{
+    const char *e = std::getenv("TSD_ATTN_COMMITS");
+    return (e && e[0] == '1' && e[1] == '\0') ? 1 : 2;
 }
 
 // With two softmax warps per quarter: of every 16 score pairs, how many are
@@ -1230,6 +1265,9 @@ UmmaPlan umma_plan(const AttnArgs &a, int num_sms)
     p.paired = small ? !p.keysplit : rows_variant() == 2;
     p.sw = (p.keysplit || p.paired) ? 1 : rows_softmax_warps();
     p.nf = p.sw == 2 ? rows_exp_fma() : 0;
+    p.cm = p.keysplit ? 2 : rows_commit_points();
+    if (p.nf != 0)
+        p.cm = 2;   // the FMA-exponential instances are built with two
     p.nrb = p.keysplit ? 1 : (a.Tmax * G + BQ - 1) / BQ;
     const int bn = p.paired ? Half::BN : Wide::BN;
     const int slots = num_sms * (p.paired ? 2 : 1);
@@ -1321,9 +1359,16 @@ cudaError_t set_smem_attributes()
     auto wide2 = tree_attn_rows_kernel<Wide, 3, 1, 2, 0>;
     auto wide2f4 = tree_attn_rows_kernel<Wide, 3, 1, 2, 4>;
     auto wide2f6 = tree_attn_rows_kernel<Wide, 3, 1, 2, 6>;
+    auto wide_c1 = tree_attn_rows_kernel<Wide, 3, 1, 1, 0, 1>;
+    auto wide2_c1 = tree_attn_rows_kernel<Wide, 3, 1, 2, 0, 1>;
     auto half = tree_attn_rows_kernel<Half, 2, 2, 1>;
+    auto half_c1 = tree_attn_rows_kernel<Half, 2, 2, 1, 0, 1>;
     err = cudaFuncSetAttribute(wide, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)Wide::kSmemBytes);
+    for (auto k : {wide_c1, wide2_c1})
+        if (err == cudaSuccess)
+            err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)Wide::kSmemBytes);
     for (auto k : {wide2, wide2f4, wide2f6})
         if (err == cudaSuccess)
             err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1332,13 +1377,15 @@ cudaError_t set_smem_attributes()
         err = cudaFuncSetAttribute(tree_attn_keysplit_kernel,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)Wide::kSmemBytes);
-    if (err == cudaSuccess)
-        err = cudaFuncSetAttribute(half, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)Half::kSmemBytes);
-    // two CTAs per SM need the largest shared-memory carve-out
-    if (err == cudaSuccess)
-        err = cudaFuncSetAttribute(half, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                   (int)cudaSharedmemCarveoutMaxShared);
+    for (auto k : {half, half_c1}) {
+        if (err == cudaSuccess)
+            err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)Half::kSmemBytes);
+        // two CTAs per SM need the largest shared-memory carve-out
+        if (err == cudaSuccess)
+            err = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                       (int)cudaSharedmemCarveoutMaxShared);
+    }
     if (err == cudaSuccess)
         done[dev].store(true);
     return err;
@@ -1409,27 +1456,22 @@ int launch_umma_attention(const AttnArgs &a, void *ws, size_t ws_bytes, int num_
             tmK, tmV, static_cast<const __nv_bfloat16 *>(a.q), a.prefix_len, a.n_nodes, a.mask,
             a.Tmax, a.Hq, a.Hkv, a.Lmax, W, sl2, p.keys_per_split, p.nsplit,
             static_cast<__nv_bfloat16 *>(a.out), part_o, part_ml, a.dev_status, a.pages);
-    else if (p.paired)
-        tree_attn_rows_kernel<Half, 2, 2, 1>
-            <<<grid, rows_threads<1>(), Half::kSmemBytes, stream>>>(
-                tmK, tmV, static_cast<const __nv_bfloat16 *>(a.q), a.prefix_len, a.n_nodes,
-                a.mask, a.Tmax, a.Hq, a.Hkv, a.Lmax, W, sl2, p.keys_per_split, p.nsplit,
-                static_cast<__nv_bfloat16 *>(a.out), part_o, part_ml, a.dev_status, a.pages);
-    else if (p.sw == 2) {
-        auto kern = p.nf == 6 ? tree_attn_rows_kernel<Wide, 3, 1, 2, 6>
+    else {
+        auto kern = p.paired ? (p.cm == 1 ? tree_attn_rows_kernel<Half, 2, 2, 1, 0, 1>
+                                          : tree_attn_rows_kernel<Half, 2, 2, 1>)
+                  : p.sw == 1 ? (p.cm == 1 ? tree_attn_rows_kernel<Wide, 3, 1, 1, 0, 1>
+                                           : tree_attn_rows_kernel<Wide, 3, 1, 1>)
+                  : p.nf == 6 ? tree_attn_rows_kernel<Wide, 3, 1, 2, 6>
                   : p.nf == 4 ? tree_attn_rows_kernel<Wide, 3, 1, 2, 4>
+                  : p.cm == 1 ? tree_attn_rows_kernel<Wide, 3, 1, 2, 0, 1>
                               : tree_attn_rows_kernel<Wide, 3, 1, 2, 0>;
-        kern<<<grid, rows_threads<2>(), Wide::kSmemBytes, stream>>>(
+        const int threads = p.sw == 2 ? rows_threads<2>() : rows_threads<1>();
+        const uint32_t smem = p.paired ? Half::kSmemBytes : Wide::kSmemBytes;
+        kern<<<grid, threads, smem, stream>>>(
             tmK, tmV, static_cast<const __nv_bfloat16 *>(a.q), a.prefix_len, a.n_nodes, a.mask,
             a.Tmax, a.Hq, a.Hkv, a.Lmax, W, sl2, p.keys_per_split, p.nsplit,
             static_cast<__nv_bfloat16 *>(a.out), part_o, part_ml, a.dev_status, a.pages);
     }
-    else
-        tree_attn_rows_kernel<Wide, 3, 1, 1>
-            <<<grid, rows_threads<1>(), Wide::kSmemBytes, stream>>>(
-                tmK, tmV, static_cast<const __nv_bfloat16 *>(a.q), a.prefix_len, a.n_nodes,
-                a.mask, a.Tmax, a.Hq, a.Hkv, a.Lmax, W, sl2, p.keys_per_split, p.nsplit,
-                static_cast<__nv_bfloat16 *>(a.out), part_o, part_ml, a.dev_status, a.pages);
     TSD_LAUNCH_CHECK();
     if (p.nsplit > 1) {
         const int rc = launch_combine(a.dtype, a.D, part_o, part_ml, p.nsplit, a.prefix_len,
