@@ -212,59 +212,36 @@ __device__ int block_max_int(int v, int *sh)
     return -block_min_int<NT>(-v, sh);
 }
 
-// The CTA's (max m, z = sum exp((l - m)/T), largest index last) from every
-// thread's own triple, in one block reduction: merging two triples keeps the
-// larger max and rescales the other side's sum to it.
+// The CTA's largest m and largest index last in one block reduction.
 template <int NT>
-__device__ void block_max_z_last(float &m, double &z, int &last, double inv_temp,
-                                 const double *table, float *shf, double *shd, int *shi)
+__device__ void block_max_last(float &m, int &last, float *shf, int *shi)
 {
     constexpr int NW = NT / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    auto merge = [&](float m2, double z2, int l2) {
-        last = max(last, l2);
-        if (m2 == -INFINITY)
-            return;
-        if (m == -INFINITY) {
-            m = m2;
-            z = z2;
-        } else if (m2 > m) {
-            z = z * table_exp(((double)m - (double)m2) * inv_temp, table) + z2;
-            m = m2;
-        } else {
-            z += z2 * table_exp(((double)m2 - (double)m) * inv_temp, table);
-        }
-    };
     auto warp_reduce = [&]() {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
-            const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-            const double z2 = __shfl_xor_sync(0xffffffffu, z, o);
-            const int l2 = __shfl_xor_sync(0xffffffffu, last, o);
-            merge(m2, z2, l2);
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
         }
     };
     warp_reduce();
     if (lane == 0) {
         shf[warp] = m;
-        shd[warp] = z;
         shi[warp] = last;
     }
     __syncthreads();
     if (warp == 0) {
         m = lane < NW ? shf[lane] : -INFINITY;
-        z = lane < NW ? shd[lane] : 0.0;
         last = lane < NW ? shi[lane] : -1;
         warp_reduce();
         if (lane == 0) {
             shf[0] = m;
-            shd[0] = z;
             shi[0] = last;
         }
     }
     __syncthreads();
     m = shf[0];
-    z = shd[0];
     last = shi[0];
     __syncthreads();
 }
@@ -444,9 +421,14 @@ __device__ double2 chunk_max_z(const float *__restrict__ row, int x_lo, int x_hi
         group(l0, x0);
         group(l1, x1);
     }
-    block_max_z_last<kWalkThreads>(mt, zt, last, inv_temp, table, shf, shd, shi);
+    // the chunk's max and last in one reduction, then each thread rescales
+    // its own sum to the chunk max (in parallel), then one sum
+    float mk = mt;
+    block_max_last<kWalkThreads>(mk, last, shf, shi);
     *last_out = last;
-    return make_double2((double)mt, mt == -INFINITY ? 0.0 : zt);
+    const double zs =
+        mt == -INFINITY ? 0.0 : zt * table_exp(((double)mt - (double)mk) * inv_temp, table);
+    return make_double2((double)mk, block_sum<kWalkThreads>(zs, shd));
 }
 
 // Over the CTA's chunk: sum max(0, p^(n)(x) - q(x)) and (in *last) the
@@ -530,19 +512,6 @@ __device__ int chunk_scan(const float *__restrict__ row, int x_lo, int x_hi, int
         carry += tile;
     }
     return INT_MAX;
-}
-
-// p^(n)(x) for one acceptance test: the exact fp64 formula of the definition.
-__device__ __forceinline__ double p_exact(float lx, int x, const RowState &st)
-{
-    double p = exp(((double)lx - st.m) / st.temp) / st.Z;
-    for (int j = 0; j < st.n; ++j) {
-        if (st.S[j] > 0.0) {
-            const double r = p - (double)st.q[j][x];
-            p = (r > 0.0 ? r : 0.0) / st.S[j];
-        }
-    }
-    return p;
 }
 
 __device__ __forceinline__ bool sequence_ok(const int32_t *n_nodes, const int32_t *first_child,
