@@ -50,7 +50,11 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
     exists) and to the V ring's v_empty[j % NSV]; the softmax's waits for "PV_r
     done" wait for that s_full phase, the producer reuses V slots on v_empty
     (a wait for s_full phase j / NS + 1 there could come two phases early on
-    the last tiles, where no K wait precedes it)."""
+    the last tiles, where no K wait precedes it).
+    cm = 3: as cm = 1, but the MMA thread waits only for P_j (and for K of
+    the first NS tiles); the first softmax warp waits for V_j and K_{j+NS}
+    before it publishes P_j.  The MMA model checks that the tiles it reads
+    have landed."""
     rnd = random.Random(seed)
     nsm = 4 * sw
     bars = {"q_full": _Barrier(nsm)}
@@ -80,6 +84,7 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
         return True
 
     tma, pipe = [], []
+    landed = set()    # ("k" | "v", tile) whose copy has completed
     s_owner = {}       # S buffer -> tile whose scores/P it holds
     pv_done = set()
 
@@ -87,7 +92,7 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
 
     def pv_passed(r):
         """The wait for "PV_r done" under the commit scheme."""
-        if cm == 1:
+        if cm in (1, 3):
             return passes(("s_full", r % NS), r // NS + 1)
         return passes(("o_ready", r % NS), r // NS)
 
@@ -107,7 +112,7 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
                             yield
                     assert k_read[s] in qk_done, f"K slot {s} reloaded before its QK ran"
                 k_read[s] = i
-                tma.append(("k_full", s))
+                tma.append((("k_full", s), ("k", i)))
             if i >= 1:
                 j = i - 1
                 s = j % NSV
@@ -121,7 +126,7 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
                             yield
                     assert v_read[s] in pv_done, f"V slot {s} reloaded before its PV ran"
                 v_read[s] = j
-                tma.append(("v_full", s))
+                tma.append((("v_full", s), ("v", j)))
             yield
 
     def mma():
@@ -129,13 +134,15 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
             yield
 
         def qk(i):
-            while not passes(("k_full", i % NSK), i // NSK):
-                yield
+            if cm != 3 or i < NS:
+                while not passes(("k_full", i % NSK), i // NSK):
+                    yield
+            assert ("k", i) in landed, f"QK_{i} issued before K_{i} landed"
             buf = i % NS
             prev = s_owner.get(buf)
             assert prev is None or prev in pv_done or ("pv", prev) in [p[0] for p in pipe], \
                 f"QK_{i} issued over the P of tile {prev} before its PV"
-            if cm == 1 and i >= NS:
+            if cm in (1, 3) and i >= NS:
                 commits = []             # covered by the tile's single commit
             else:
                 commits = [("s_full", buf)] if merged else \
@@ -147,9 +154,11 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
         for j in range(ntiles):
             while not passes(("p_full", j % NS), j // NS):
                 yield
-            while not passes(("v_full", j % NSV), j // NSV):
-                yield
-            if cm == 1:
+            if cm != 3:
+                while not passes(("v_full", j % NSV), j // NSV):
+                    yield
+            assert ("v", j) in landed, f"PV_{j} issued before V_{j} landed"
+            if cm in (1, 3):
                 commits = []
             else:
                 commits = [("o_ready", j % NS)] if merged else \
@@ -157,7 +166,7 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
             pipe.append((("pv", j), commits))
             if j + NS < ntiles:
                 yield from qk(j + NS)
-            if cm == 1:   # one commit point: tracks everything issued so far
+            if cm in (1, 3):   # one commit point: tracks everything issued so far
                 pipe.append((("commit", j), [("s_full", j % NS), ("v_empty", j % NSV)]))
             yield
 
@@ -167,7 +176,7 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
         while not passes(("pair", q), n):
             yield
 
-    def softmax(q):
+    def softmax(q, first=False):
         bars["q_full"].arrive()
         yield
         nx = 0
@@ -188,6 +197,12 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
                 while not pv_passed(j - 1):
                     yield
                 assert j - 1 in pv_done
+            if cm == 3 and first:                       # for the MMA thread
+                while not passes(("v_full", j % NSV), j // NSV):
+                    yield
+                if j + NS < ntiles:
+                    while not passes(("k_full", (j + NS) % NSK), (j + NS) // NSK):
+                        yield
             bars["p_full", j % NS].arrive()
             yield
         if ntiles:
@@ -202,13 +217,16 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
             if sw == 2:
                 yield from exchange(q, nx)              # the row sums
 
-    roles = [producer(), mma()] + [softmax(q) for q in range(4) for _ in range(sw)]
+    roles = [producer(), mma()] + [softmax(q, first=(q == 0 and h == 0))
+                                   for q in range(4) for h in range(sw)]
     idle = 0
     while roles or tma or pipe:
         choices = list(range(len(roles))) + (["tma"] if tma else []) + (["pipe"] if pipe else [])
         c = rnd.choice(choices)
         if c == "tma":        # copies land in any order
-            bars[tma.pop(rnd.randrange(len(tma)))].arrive()
+            bar, what = tma.pop(rnd.randrange(len(tma)))
+            landed.add(what)
+            bars[bar].arrive()
             idle = 0
         elif c == "pipe":     # the tensor pipe completes in issue order
             (kind, t), commits = pipe.pop(0)
@@ -242,6 +260,14 @@ def test_rows_kernel_protocol(NS, NSK, NSV, sw, ntiles):
 def test_rows_kernel_protocol_one_commit_per_tile(NS, NSK, NSV, sw, ntiles):
     for seed in range(150):
         _run(NS, NSK, NSV, ntiles, seed, sw=sw, cm=1)
+
+
+@pytest.mark.parametrize("NS,NSK,NSV,sw", [(3, 3, 2, 1), (2, 2, 2, 1), (3, 3, 2, 2)],
+                         ids=["128-key tiles", "64-key tiles", "128-key tiles, paired softmax"])
+@pytest.mark.parametrize("ntiles", [1, 2, 3, 4, 5, 8, 17])
+def test_rows_kernel_protocol_one_wait_per_tile(NS, NSK, NSV, sw, ntiles):
+    for seed in range(150):
+        _run(NS, NSK, NSV, ntiles, seed, sw=sw, cm=3)
 
 
 @pytest.mark.parametrize("ntiles", [1, 3, 6])

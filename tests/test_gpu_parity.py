@@ -163,6 +163,9 @@ FORCED = [
     ("large", {"TSD_ATTN_COMMITS": "1"}, "rows128"),
     ("large", {"TSD_ATTN_COMMITS": "1", "TSD_ATTN_SOFTMAX_WARPS": "2"}, "rows128x2"),
     ("small", {"TSD_ATTN_COMMITS": "1"}, "rows64"),
+    ("large", {"TSD_ATTN_COMMITS": "3"}, "rows128"),
+    ("large", {"TSD_ATTN_COMMITS": "3", "TSD_ATTN_SOFTMAX_WARPS": "2"}, "rows128x2"),
+    ("small", {"TSD_ATTN_COMMITS": "3"}, "rows64"),
     ("small", {}, "rows64"),
     ("small", {"TSD_ATTN_SMALL_VARIANT": "keysplit"}, "keysplit"),
     ("small", {"TSD_FORCE_PATH": "simt"}, "simt"),
@@ -176,7 +179,8 @@ def _shape_workload(name):
 
 
 FORCED_IDS = [f"{f[0]}-{f[2]}" + ("-expfma" if "TSD_ATTN_EXP_FMA" in f[1] else "")
-              + ("-1commit" if "TSD_ATTN_COMMITS" in f[1] else "") for f in FORCED]
+              + (f"-sched{f[1]['TSD_ATTN_COMMITS']}" if "TSD_ATTN_COMMITS" in f[1] else "")
+              for f in FORCED]
 
 
 @pytest.mark.parametrize("splits", ["1", "3", "64"])
@@ -401,10 +405,17 @@ def test_config_full_size_paired_softmax(cuda_device, cfg, nf, monkeypatch):
     test_config_full_size(cuda_device, cfg)
 
 
+@pytest.mark.parametrize("sched", ["1", "3"])
 @pytest.mark.parametrize("cfg", [1, 3, 4])
-def test_config_full_size_one_commit_per_tile(cuda_device, cfg, monkeypatch):
-    monkeypatch.setenv("TSD_ATTN_COMMITS", "1")
+def test_config_full_size_mma_schedules(cuda_device, cfg, sched, monkeypatch):
+    monkeypatch.setenv("TSD_ATTN_COMMITS", sched)
     test_config_full_size(cuda_device, cfg)
+
+
+def test_config_full_size_paired_softmax_one_wait(cuda_device, monkeypatch):
+    monkeypatch.setenv("TSD_ATTN_COMMITS", "3")
+    monkeypatch.setenv("TSD_ATTN_SOFTMAX_WARPS", "2")
+    test_config_full_size(cuda_device, 3)
 
 
 @pytest.mark.parametrize("cfg", [0, 1, 2, 3, 4])

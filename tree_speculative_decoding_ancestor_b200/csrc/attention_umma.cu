@@ -361,7 +361,7 @@ __device__ __forceinline__ void produce_kv(const Setup<Gm> &su, const CUtensorMa
                 // s_full[r % NS] phase r / NS + 1 could come two phases early on
                 // the last tiles, where no K wait precedes it.)
                 const bool ok =
-                    (!NS_PROD || CM == 1)
+                    (!NS_PROD || CM != 2)
                         ? ptx::mbar_wait(su.bars.v_empty(s), ((j / NSV) - 1) & 1, su.abort_flag)
                         : ptx::mbar_wait(su.bars.o_ready(r % NSP), (r / NSP) & 1,
                                          su.abort_flag);
@@ -376,7 +376,7 @@ __device__ __forceinline__ void produce_kv(const Setup<Gm> &su, const CUtensorMa
 }
 
 // MMA warp, S = Q K^T for key tile `t` into TMEM columns `col_s`.
-template <class Gm, bool RING_COMMIT = true, bool COMMIT = true>
+template <class Gm, bool RING_COMMIT = true, bool COMMIT = true, bool WARP = true>
 __device__ __forceinline__ void issue_qk(const Setup<Gm> &su, int lane, uint32_t col_s, int t,
                                          uint32_t s_full)
 {
@@ -393,14 +393,32 @@ __device__ __forceinline__ void issue_qk(const Setup<Gm> &su, int lane, uint32_t
         if (COMMIT && RING_COMMIT)
             ptx::mma_commit(su.bars.k_empty(st));
     }
-    __syncwarp();
+    if (WARP)
+        __syncwarp();
 }
 
 // MMA warp, O += P V for key tile `t` (P in TMEM columns col_p); zeroes the
 // V rows at or beyond P_b + T_b first.  P_SPLIT: the packed P of keys
 // 64 .. 127 sits 64 columns after that of keys 0 .. 63 (each softmax half
 // writes into its own score columns) instead of right after it.
-template <class Gm, bool RING_COMMIT = true, bool P_SPLIT = false, bool COMMIT = true>
+// Zero the rows first_bad .. BN-1 of V ring slot vs (cache rows at or beyond
+// P_b + T_b: masked keys whose P is 0, but 0 * NaN would not be), by one warp,
+// then make the generic-proxy stores visible to the tensor cores.
+template <class Gm>
+__device__ __forceinline__ void zero_v_rows(const Setup<Gm> &su, int vs, int first_bad, int lane)
+{
+    uint8_t *vt = su.gbase + Gm::kOffV + vs * Gm::kTile;
+    for (int row = max(first_bad, 0) + (lane >> 3); row < Gm::BN; row += 4) {
+        const int c = lane & 7;
+        *reinterpret_cast<uint4 *>(vt + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4 *>(vt + Gm::kSub + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+    }
+    ptx::fence_proxy_async_smem();
+    __syncwarp();
+}
+
+template <class Gm, bool RING_COMMIT = true, bool P_SPLIT = false, bool COMMIT = true,
+          bool ZERO = true>
 __device__ __forceinline__ void issue_pv(const Setup<Gm> &su, int lane, uint32_t col_p,
                                          uint32_t col_o, int t, bool accumulate, int first_bad,
                                          uint32_t o_ready)
@@ -408,17 +426,8 @@ __device__ __forceinline__ void issue_pv(const Setup<Gm> &su, int lane, uint32_t
     constexpr int BN = Gm::BN;
     constexpr uint32_t idesc = ptx::idesc_bf16(BQ, HD, false, true);
     const int vs = t % Gm::NSV;
-    if (first_bad < BN) {
-        uint8_t *vt = su.gbase + Gm::kOffV + vs * Gm::kTile;
-        for (int row = max(first_bad, 0) + (lane >> 3); row < BN; row += 4) {
-            const int c = lane & 7;
-            *reinterpret_cast<uint4 *>(vt + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4 *>(vt + Gm::kSub + row * 128 + c * 16) =
-                make_uint4(0, 0, 0, 0);
-        }
-        ptx::fence_proxy_async_smem();
-        __syncwarp();
-    }
+    if (ZERO && first_bad < BN)
+        zero_v_rows<Gm>(su, vs, first_bad, lane);
     ptx::tc_fence_after();
     if (lane == 0) {
         const uint64_t dv = desc_v(su.sV + vs * Gm::kTile, Gm::kSub);
@@ -435,7 +444,8 @@ __device__ __forceinline__ void issue_pv(const Setup<Gm> &su, int lane, uint32_t
         if (COMMIT)
             ptx::mma_commit(o_ready);
     }
-    __syncwarp();
+    if (ZERO)
+        __syncwarp();
 }
 
 // Softmax-warp helpers.  Row state of one query row of a tile.
@@ -918,6 +928,33 @@ __global__ void __launch_bounds__(rows_threads<SW>(), kMinBlocks)
         if (lane == 0)
             produce_kv<Gm, NS, CM>(su, &tmK, &tmV, b, hk, Hkv, kb, ntiles, pages, pc, P + T,
                                    dev_status);
+    } else if (warp == 1 && CM == 3) {
+        // One mbarrier wait per key tile (each wait on this thread, even on a
+        // completed barrier, leaves the tensor pipe idle for about one MMA):
+        // lane 0 alone waits for P_j, whose last arrival comes from softmax
+        // warp 4 after it has seen V_j and K_{j+NS} land (and zeroed V_j's
+        // rows past the range end), then issues PV_j and QK_{j+NS} and one
+        // commit point, as for CM = 1.
+        if (lane == 0) {
+            bool ok = ptx::mbar_wait(su.bars.q_full(), 0, su.abort_flag);
+            for (int i = 0; ok && i < min(NS, ntiles); ++i) {
+                ok = ptx::mbar_wait(su.bars.k_full(i % NSK), (i / NSK) & 1, su.abort_flag);
+                ptx::tc_fence_after();
+                if (ok)
+                    issue_qk<Gm, false, true, false>(su, 0, col_s(i), i, su.bars.s_full(i % NS));
+            }
+            for (int j = 0; ok && j < ntiles; ++j) {
+                if (!ptx::mbar_wait(su.bars.p_full(j % NS), (j / NS) & 1, su.abort_flag))
+                    break;
+                ptx::tc_fence_after();
+                issue_pv<Gm, false, SW == 2, false, false>(su, 0, col_s(j), kO, j, j > 0, BN,
+                                                           0u);
+                if (j + NS < ntiles)
+                    issue_qk<Gm, false, false, false>(su, 0, col_s(j + NS), j + NS, 0u);
+                ptx::mma_commit(su.bars.s_full(j % NS));
+                ptx::mma_commit(su.bars.v_empty(j % NSV));
+            }
+        }
     } else if (warp == 1) {
         bool ok = warp_wait(su.bars.q_full(), 0, su.abort_flag);
         ptx::tc_fence_after();
@@ -978,10 +1015,10 @@ __global__ void __launch_bounds__(rows_threads<SW>(), kMinBlocks)
             mw[w] = (row_ok && w < W) ? mask[((size_t)b * Tmax + u) * W + w] : 0u;
         const uint32_t taddr_o = su.tmem + lane_off + kO + hf * 64;
         PairXchg *xc = reinterpret_cast<PairXchg *>(su.gbase + Gm::kOffXchg) + quarter;
-        // PV_i done: o_ready[i % NS] phase i / NS, or (CM = 1) s_full[i % NS]
+        // PV_i done: o_ready[i % NS] phase i / NS, or (CM = 1, 3) s_full[i % NS]
         // phase i / NS + 1
         auto wait_pv = [&](int i) {
-            return CM == 1
+            return CM != 2
                        ? warp_wait(su.bars.s_full(i % NS), ((i / NS) + 1) & 1, su.abort_flag)
                        : warp_wait(su.bars.o_ready(i % NS), (i / NS) & 1, su.abort_flag);
         };
@@ -1006,6 +1043,19 @@ __global__ void __launch_bounds__(rows_threads<SW>(), kMinBlocks)
             if (!ok)
                 break;
             ptx::tc_fence_before();
+            if (CM == 3 && warp == 4) {
+                // for the MMA thread: V_j and K_{j+NS} have landed, V_j's rows
+                // past the range end are zero
+                ok = warp_wait(su.bars.v_full(j % NSV), (j / NSV) & 1, su.abort_flag);
+                if (ok && j + NS < ntiles)
+                    ok = warp_wait(su.bars.k_full((j + NS) % NSK), ((j + NS) / NSK) & 1,
+                                   su.abort_flag);
+                if (!ok)
+                    break;
+                const int first_bad = P + T - (kb + j * BN);
+                if (first_bad < BN)
+                    zero_v_rows<Gm>(su, j % NSV, first_bad, lane);
+            }
             warp_arrive(su.bars.p_full(j % NS));
         }
         bool done = ok && wait_pv(ntiles - 1);
@@ -1217,12 +1267,16 @@ int rows_softmax_warps()
     return (e && e[0] == '2' && e[1] == '\0') ? 2 : 1;
 }
 
-// Commit points per key tile on the MMA thread: 2 (after QK, after PV), or
-// 1 when TSD_ATTN_COMMITS is "1" (read at every launch).
+// MMA-thread schedule of the rows kernels (TSD_ATTN_COMMITS, read at every
+// launch): 2 -- commits after QK and after PV, waits for P, V and K per tile;
+// "1" -- one commit point per tile; "3" -- one commit point and one wait
+// (for P) per tile, a softmax warp checking V and K first.
 int rows_commit_points()
 {
     const char *e = std::getenv("TSD_ATTN_COMMITS");
-    return (e && e[0] == '1' && e[1] == '\0') ? 1 : 2;
+    if (e && e[1] == '\0' && (e[0] == '1' || e[0] == '3'))
+        return e[0] - '0';
+    return 2;
 }
 
 // With two softmax warps per quarter: of every 16 score pairs, how many are
@@ -1361,11 +1415,14 @@ cudaError_t set_smem_attributes()
     auto wide2f6 = tree_attn_rows_kernel<Wide, 3, 1, 2, 6>;
     auto wide_c1 = tree_attn_rows_kernel<Wide, 3, 1, 1, 0, 1>;
     auto wide2_c1 = tree_attn_rows_kernel<Wide, 3, 1, 2, 0, 1>;
+    auto wide_c3 = tree_attn_rows_kernel<Wide, 3, 1, 1, 0, 3>;
+    auto wide2_c3 = tree_attn_rows_kernel<Wide, 3, 1, 2, 0, 3>;
     auto half = tree_attn_rows_kernel<Half, 2, 2, 1>;
     auto half_c1 = tree_attn_rows_kernel<Half, 2, 2, 1, 0, 1>;
+    auto half_c3 = tree_attn_rows_kernel<Half, 2, 2, 1, 0, 3>;
     err = cudaFuncSetAttribute(wide, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)Wide::kSmemBytes);
-    for (auto k : {wide_c1, wide2_c1})
+    for (auto k : {wide_c1, wide2_c1, wide_c3, wide2_c3})
         if (err == cudaSuccess)
             err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)Wide::kSmemBytes);
@@ -1377,7 +1434,7 @@ cudaError_t set_smem_attributes()
         err = cudaFuncSetAttribute(tree_attn_keysplit_kernel,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)Wide::kSmemBytes);
-    for (auto k : {half, half_c1}) {
+    for (auto k : {half, half_c1, half_c3}) {
         if (err == cudaSuccess)
             err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)Half::kSmemBytes);
@@ -1457,13 +1514,16 @@ int launch_umma_attention(const AttnArgs &a, void *ws, size_t ws_bytes, int num_
             a.Tmax, a.Hq, a.Hkv, a.Lmax, W, sl2, p.keys_per_split, p.nsplit,
             static_cast<__nv_bfloat16 *>(a.out), part_o, part_ml, a.dev_status, a.pages);
     else {
-        auto kern = p.paired ? (p.cm == 1 ? tree_attn_rows_kernel<Half, 2, 2, 1, 0, 1>
-                                          : tree_attn_rows_kernel<Half, 2, 2, 1>)
-                  : p.sw == 1 ? (p.cm == 1 ? tree_attn_rows_kernel<Wide, 3, 1, 1, 0, 1>
-                                           : tree_attn_rows_kernel<Wide, 3, 1, 1>)
+        auto kern = p.paired ? (p.cm == 1   ? tree_attn_rows_kernel<Half, 2, 2, 1, 0, 1>
+                                : p.cm == 3 ? tree_attn_rows_kernel<Half, 2, 2, 1, 0, 3>
+                                            : tree_attn_rows_kernel<Half, 2, 2, 1>)
+                  : p.sw == 1 ? (p.cm == 1   ? tree_attn_rows_kernel<Wide, 3, 1, 1, 0, 1>
+                                 : p.cm == 3 ? tree_attn_rows_kernel<Wide, 3, 1, 1, 0, 3>
+                                             : tree_attn_rows_kernel<Wide, 3, 1, 1>)
                   : p.nf == 6 ? tree_attn_rows_kernel<Wide, 3, 1, 2, 6>
                   : p.nf == 4 ? tree_attn_rows_kernel<Wide, 3, 1, 2, 4>
                   : p.cm == 1 ? tree_attn_rows_kernel<Wide, 3, 1, 2, 0, 1>
+                  : p.cm == 3 ? tree_attn_rows_kernel<Wide, 3, 1, 2, 0, 3>
                               : tree_attn_rows_kernel<Wide, 3, 1, 2, 0>;
         const int threads = p.sw == 2 ? rows_threads<2>() : rows_threads<1>();
         const uint32_t smem = p.paired ? Half::kSmemBytes : Wide::kSmemBytes;
