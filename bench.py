@@ -841,8 +841,8 @@ def time_tree_build(w, dev, tsd, reps: int = 10):
 def time_paged_attention(step, dev, tsd, page_size: int = 128, reps: int = 10):
     """The same attention call through a paged KV cache (pools of page_size
     rows, physical pages in a shuffled order, a block table per sequence),
-    timed alone with CUDA events; also reports the contiguous call's time
-    measured the same way."""
+    replayed from a CUDA graph and timed with CUDA events; also reports the
+    contiguous call's time measured the same way."""
     w, d = step.w, step.d
     B, Hkv, Lmax, D = d["k_cache"].shape
     nblk = (Lmax + page_size - 1) // page_size
@@ -871,15 +871,23 @@ def time_paged_attention(step, dev, tsd, page_size: int = 128, reps: int = 10):
 
     res = {}
     for name, fn in (("us", paged), ("contiguous_us", flat)):
+        # each call replayed from a CUDA graph of its own, so that the events
+        # time the kernels and not the Python and tensor-map work in front
         fn()
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            fn()
+        graph.replay()
         torch.cuda.synchronize(dev)
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(reps)]
         for a, b in ev:
             a.record()
-            fn()
+            graph.replay()
             b.record()
         torch.cuda.synchronize(dev)
+        del graph
         res[name] = statistics.median(a.elapsed_time(b) * 1e3 for a, b in ev)
     if int(tsd.device_status(dev).item()) != 0:
         raise RuntimeError("device status set by the paged attention")
