@@ -211,9 +211,9 @@ int tsd_tree_attention_paged(const void *q, const void *k_pages, const void *v_p
                              float scale, int dtype, void *out, void *workspace,
                              size_t workspace_bytes, int32_t *dev_status, tsd_stream_t stream);
 
-/* Bytes of workspace either verify call needs: a fixed ~44 KB (per-CTA
- * partial sums of the stochastic walk and the exchange tags that publish
- * them) plus 4 bytes per logits row (greedy row argmax). */
+/* Bytes of workspace either verify call needs: a fixed ~40 KB (per-CTA
+ * partial sums and barrier counters of the stochastic walk) plus 4 bytes per
+ * logits row (greedy row argmax). */
 size_t tsd_tree_verify_workspace_size(int B, int Tmax, int V);
 
 /*
@@ -379,9 +379,9 @@ int tsd_kv_commit(void *k_cache, void *v_cache, const int32_t *prefix_len,
  * completes, with a short limit, so that tests can check the behaviour:
  *   kind 0  the mbarrier wait of the tensor-core attention kernels, on an
  *           mbarrier nobody arrives on;
- *   kind 1  the team exchange of the stochastic walk, waiting for a partner
- *           CTA that does not exist.
- *   limit_ns  in [1 ms, 2 s]; scratch: 16 bytes of device memory (8-aligned).
+ *   kind 1  the team barrier of the stochastic walk, on a counter whose
+ *           target one CTA cannot reach.
+ *   limit_ns  in [1 ms, 2 s]; scratch: 8 bytes of device memory (8-aligned).
  * Expected result: the kernel ends after about limit_ns with TSD_DEV_TIMEOUT
  * set in *dev_status.  Host errors: TSD_ERR_SHAPE, TSD_ERR_NULL,
  * TSD_ERR_ALIGN, TSD_ERR_CUDA.
@@ -401,8 +401,8 @@ int tsd_debug_wait_probe(int kind, unsigned long long limit_ns, void *scratch,
  * inside the library's device code; every GPU that loads the library holds
  * that array until the process exits.  Nothing is allocated: no cudaMalloc,
  * no cudaFree, no allocating library routine.
- *   - The scratch it needs is fixed (about 44 KB: the per-CTA partial sums
- *     of the walk and the exchange tags that publish them), whatever B, Tmax and V are, so no
+ *   - The scratch it needs is fixed (about 40 KB: the per-CTA partial sums
+ *     and barrier counters of the walk), whatever B, Tmax and V are, so no
  *     shape is refused for size; TSD_ERR_WORKSPACE would mean a build whose
  *     array is smaller than that, and then nothing is launched.
  *   - The first call on each device looks up the array's device address

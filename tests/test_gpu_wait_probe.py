@@ -2,7 +2,7 @@
 
 Every wait in the kernels gives up after a time limit, sets TSD_DEV_TIMEOUT and
 returns.  The probe runs the same wait routines -- the attention kernels'
-mbarrier wait and the stochastic walk's team exchange -- on something nothing
+mbarrier wait and the stochastic walk's team barrier -- on something nothing
 ever signals, with a 50 ms limit; the kernel must end on its own with the
 status set, and the context must stay usable afterwards.
 """

@@ -2,19 +2,19 @@
 
 The walk's CTAs exchange their per-chunk partial sums with no grid-wide
 barrier (`csrc/verify.cu`, `csrc/team_barrier.cuh`). The K CTAs of a team
-do this at every exchange n = 1, 2, ...:
-1. write their (value, last index) pair into slot k of buffer n & 1;
-2. publish it: a release store of n into the tag of that slot;
-3. lane j of warp 0 polls the tag of slot j of that buffer until it reads
-   n (an acquire), then reads slot j.
+do this at every barrier n = 1, 2, ...:
+1. write their (value, last index) pair into slot k of buffer (n - 1) & 1;
+2. add 1 to the team's arrival counter (a release);
+3. poll until the counter reaches n·K (an acquire);
+4. read all K slots of that buffer.
 
-Every CTA of a team makes the same exchanges, since all of them take
-identical decisions from the same slots. A slot buffer is written again two
-exchanges later, and only by a CTA that has passed exchange n + 1, which
-every CTA enters after reading exchange n's slots. This test replays the
-exchange under random interleavings: every read must see the value written
-for its own exchange, and every wait must end. A one-buffer layout is the
-negative control.
+Every CTA of a team takes the same number of barriers, since all of them
+take identical decisions from the same slots. A slot buffer is written
+again two barriers later, and only by a CTA that has passed barrier n + 1,
+which every CTA reaches after reading barrier n's slots. This test replays
+the exchange under random interleavings: every read must see the value
+written for its own barrier, and every wait must end. A one-buffer layout
+is the negative control.
 """
 
 import random
@@ -22,25 +22,23 @@ import random
 import pytest
 
 
-def _run(K, nx, seed, buffers=2):
+def _run(K, nbar, seed, buffers=2):
     rnd = random.Random(seed)
     slots = [[None] * K for _ in range(buffers)]
-    tags = [[0] * K for _ in range(buffers)]
+    counter = [0]
 
     def cta(k):
-        for n in range(1, nx + 1):
-            buf = n % buffers
-            slots[buf][k] = (n, k)                    # this CTA's partial for exchange n
+        for n in range(1, nbar + 1):
+            buf = (n - 1) % buffers
+            slots[buf][k] = (n, k)                    # this CTA's partial for barrier n
             yield
-            tags[buf][k] = n                          # release store of the tag
+            counter[0] += 1                           # release-add
             yield
-            order = list(range(K))
-            rnd.shuffle(order)                        # the K lanes poll concurrently
-            for j in order:
-                while tags[buf][j] != n:              # acquire poll of slot j's tag
-                    yield
+            while counter[0] < n * K:                 # acquire-poll
+                yield
+            for j in range(K):                        # warp 0 reads the K slots
                 assert slots[buf][j] == (n, j), \
-                    f"CTA {k} at exchange {n} read {slots[buf][j]} from slot {j}"
+                    f"CTA {k} at barrier {n} read {slots[buf][j]} from slot {j}"
                 if rnd.random() < 0.3:
                     yield                             # reads spread over time
 
@@ -53,7 +51,7 @@ def _run(K, nx, seed, buffers=2):
         except StopIteration:
             ctas.pop(i)
         idle += 1
-        assert idle < 200_000, "a team exchange never completes"
+        assert idle < 200_000, "a team barrier never completes"
 
 
 @pytest.mark.parametrize("K", [1, 2, 5, 32])
@@ -63,8 +61,8 @@ def test_slots_are_read_before_they_are_reused(K):
 
 
 def test_one_slot_buffer_would_race():
-    # With a single buffer a fast CTA overwrites its slot for exchange n + 1
-    # while a slow one still reads exchange n's values.
+    # With a single buffer a fast CTA overwrites its slot for barrier n + 1
+    # while a slow one still reads barrier n's values.
     with pytest.raises(AssertionError):
         for seed in range(200):
             _run(4, 6, seed, buffers=1)

@@ -83,7 +83,7 @@ def test_noalloc_takes_a_batch_larger_than_the_grid(cuda_device):
     lib = tsd.load_library()
     # 1100 sequences over a 64-token vocabulary: one CTA per team, and more
     # sequences than the cooperative grid holds (it is capped at 1024 CTAs),
-    # so teams walk several sequences each and their exchange numbers run on
+    # so teams walk several sequences each and their barrier counters run on
     # from one sequence to the next.
     dev = cuda_device
     B, Tmax, V = 1100, 24, 64

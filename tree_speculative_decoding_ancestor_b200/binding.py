@@ -562,14 +562,14 @@ def tree_merge_chains(chain_tokens: torch.Tensor, chain_q_row: torch.Tensor,
 def debug_wait_probe(kind: int, limit_ns: int = 50_000_000, device=None,
                      status: Optional[torch.Tensor] = None) -> None:
     """Run the kernels' bounded wait routines on something that never completes
-    (kind 0: mbarrier wait; kind 1: team exchange); they must end after about
-    limit_ns with DEV_TIMEOUT set in the status word.  16 bytes of scratch."""
+    (kind 0: mbarrier wait; kind 1: team barrier); they must end after about
+    limit_ns with DEV_TIMEOUT set in the status word."""
     lib = load_library()
     dev = torch.device(device or torch.cuda.current_device())
     _cuda(dev)
     if dev.index is None:
         dev = torch.device("cuda", torch.cuda.current_device())
-    scratch = torch.zeros(4, dtype=torch.int32, device=dev)
+    scratch = torch.zeros(2, dtype=torch.int32, device=dev)
     st = _status_for(dev, status)
     rc = lib.tsd_debug_wait_probe(int(kind), int(limit_ns), _ptr(scratch), _ptr(st), _stream(dev))
     _check(rc, "tsd_debug_wait_probe")

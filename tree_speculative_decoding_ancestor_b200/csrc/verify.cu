@@ -30,10 +30,8 @@
 //                           token -- the draw costs no barrier.
 //                           Only rows on the accepted path are read.  Partial
 //                           results cross CTAs through one workspace slot per
-//                           CTA, published by a release-stored exchange number
-//                           that the team's readers poll directly (one round
-//                           trip per exchange); every wait is bounded
-//                           (TSD_DEV_TIMEOUT).
+//                           CTA and a per-team arrival counter; every wait on
+//                           a counter is bounded (TSD_DEV_TIMEOUT).
 //
 // Residual distributions are never materialised: p^(n)(x) is recomputed per
 // element from the logits row, the rejected siblings' q rows and their
@@ -66,28 +64,26 @@ constexpr int kDecCache = 8;          // children per row whose test operands ar
 constexpr int kDecOps = 2 * kDecCache + kDecCache * (kDecCache + 1) / 2;   // 52 loads
 
 struct VerifyWs {
-    double2 *slot;     // [2][kWalkMaxCtas]  per-CTA partials, by exchange parity
-    int *tag;          // [2][kWalkMaxCtas]  exchange number each slot holds  } zeroed
-    int *abort;        // [kWalkMaxCtas]     per-team abort flag              } per call
+    double2 *slot;     // [2][kWalkMaxCtas]  per-CTA partials, by barrier parity
+    int2 *team;        // [kWalkMaxCtas]     {arrivals, abort} per team, zeroed per call
     int32_t *argmax;   // [B][Tmax+1]        greedy: argmax of rows with children
 };
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-// Fixed part first: the stochastic call uses only that.  The tags and the
-// abort flags are contiguous (one memset per call).
-constexpr size_t kSlotBytes = (2 * kWalkMaxCtas * sizeof(double2) + 255) & ~(size_t)255;
-constexpr size_t kZeroedBytes = (3 * kWalkMaxCtas * sizeof(int) + 255) & ~(size_t)255;
-constexpr size_t kWalkBytes = kSlotBytes + kZeroedBytes;
+// Fixed part first: the stochastic call uses only that.
+constexpr size_t kWalkBytes = ((2 * kWalkMaxCtas * sizeof(double2) + 255) & ~(size_t)255) +
+                              ((kWalkMaxCtas * sizeof(int2) + 255) & ~(size_t)255);
 
 VerifyWs carve(void *ws)
 {
     char *p = static_cast<char *>(ws);
     VerifyWs w;
     w.slot = reinterpret_cast<double2 *>(p);
-    w.tag = reinterpret_cast<int *>(p + kSlotBytes);
-    w.abort = w.tag + 2 * kWalkMaxCtas;
-    w.argmax = reinterpret_cast<int32_t *>(p + kWalkBytes);
+    p += align256(2 * kWalkMaxCtas * sizeof(double2));
+    w.team = reinterpret_cast<int2 *>(p);
+    p += align256(kWalkMaxCtas * sizeof(int2));
+    w.argmax = reinterpret_cast<int32_t *>(p);
     return w;
 }
 
@@ -668,11 +664,10 @@ __global__ void __launch_bounds__(kWalkThreads)
     const int x_lo = min(k * chunk, V), x_hi = min(x_lo + chunk, V);
     const double inv_temp = 1.0 / temp;
     const bool lead = k == 0 && tid == 0;   // writes the path and the error codes
-    int *abort = ws.abort + team;
-    int nbar = 0;   // exchanges made
-    // the team's K slots and tags of the next exchange
-    auto slots = [&]() { return ws.slot + ((nbar + 1) & 1) * kWalkMaxCtas + team * K; };
-    auto tags = [&]() { return ws.tag + ((nbar + 1) & 1) * kWalkMaxCtas + team * K; };
+    int2 *tm = ws.team + team;
+    int nbar = 0;
+    // this CTA's slot / the team's K slots of the next barrier
+    auto slots = [&]() { return ws.slot + (nbar & 1) * kWalkMaxCtas + team * K; };
     fill_exp_table(table, 1.0);   // read only from here on (barriers below publish it)
 
     for (int b = team; b < B; b += teams) {
@@ -783,17 +778,17 @@ __global__ void __launch_bounds__(kWalkThreads)
             double2 *sl = slots();
             if (tid == 0)
                 sl[k] = make_double2(mz.y, __hiloint2double(__float_as_int((float)mz.x), lastk));
-            double2 v = make_double2(0.0, 0.0);
-            if (!team_exchange(sl, tags(), k, K, nbar + 1, abort, v, &sh_ok, kTeamWaitNs)) {
+            ++nbar;
+            if (!team_barrier(tm, nbar * K, &sh_ok, kTeamWaitNs)) {
                 alive = false;
                 break;
             }
-            ++nbar;
             int c = child(row, 0);   // the children in ascending index
             if (warp == 0) {
                 double mk = -INFINITY, zk = 0.0;
                 int lk = -1;
                 if (lane < K) {
+                    const double2 v = __ldcg(sl + lane);
                     zk = v.x;
                     mk = (double)__int_as_float(__double2hiint(v.y));
                     lk = __double2loint(v.y);
@@ -830,17 +825,17 @@ __global__ void __launch_bounds__(kWalkThreads)
                 sl = slots();
                 if (tid == 0)
                     sl[k] = make_double2(s, (double)lastk);
-                double2 v = make_double2(0.0, 0.0);
-                if (!team_exchange(sl, tags(), k, K, nbar + 1, abort, v, &sh_ok, kTeamWaitNs)) {
+                ++nbar;
+                if (!team_barrier(tm, nbar * K, &sh_ok, kTeamWaitNs)) {
                     alive = false;
                     break;
                 }
-                ++nbar;
                 const int next = child(row, i + 1);
                 if (warp == 0) {
                     double sk = 0.0;
                     int lk = -1;
                     if (lane < K) {
+                        const double2 v = __ldcg(sl + lane);
                         sk = v.x;
                         lk = (int)v.y;
                     }
@@ -1040,7 +1035,7 @@ int launch_verify_stochastic(const float *logits, double temperature, const floa
     if (walk_grid(B, V, K, teams, chunk) != TSD_OK)
         return TSD_ERR_CUDA;
     VerifyWs w = carve(ws);
-    if (cudaMemsetAsync(w.tag, 0, kZeroedBytes, stream) != cudaSuccess) {
+    if (cudaMemsetAsync(w.team, 0, (size_t)teams * sizeof(int2), stream) != cudaSuccess) {
         (void)cudaGetLastError();
         return TSD_ERR_CUDA;
     }

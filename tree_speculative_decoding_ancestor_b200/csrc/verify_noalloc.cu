@@ -1,7 +1,7 @@
 // Stochastic tree verification for callers that cannot allocate device memory.
 //
 // tsd_tree_verify_stochastic needs a small scratch area (the per-CTA partial
-// sums its teams exchange and the tags that publish them; its size does not
+// sums its teams exchange and their barrier counters; its size does not
 // depend on the problem).  Some callers have no way to
 // provide one: a serving engine that has already handed nearly all device
 // memory to its KV-cache pool, or code that reaches this library through a

@@ -3,9 +3,8 @@
 // must return with TSD_DEV_TIMEOUT set and leave the context usable.
 //   kind 0: the mbarrier wait of the tensor-core attention kernels, on an
 //           mbarrier nobody arrives on;
-//   kind 1: the team exchange of the stochastic walk, in a team of two
-//           CTAs of which only one exists, so the other's slot is never
-//           published.
+//   kind 1: the team barrier of the stochastic walk, on a counter whose
+//           target is one arrival more than the CTA can supply.
 #include "sm100_ptx.cuh"
 #include "team_barrier.cuh"
 #include "tsd_common.cuh"
@@ -14,12 +13,11 @@ namespace tsd {
 
 namespace {
 
-__global__ void wait_probe_kernel(int kind, unsigned long long limit_ns, int *scratch,
+__global__ void wait_probe_kernel(int kind, unsigned long long limit_ns, int2 *team,
                                   int32_t *dev_status)
 {
     __shared__ __align__(8) uint64_t bar;
     __shared__ int abort_flag, sh_ok;
-    __shared__ double2 slots[2];
     if (kind == 0) {
         if (threadIdx.x == 0) {
             ptx::mbar_init(ptx::smem_addr(&bar), 1);
@@ -33,10 +31,7 @@ __global__ void wait_probe_kernel(int kind, unsigned long long limit_ns, int *sc
         if (threadIdx.x == 0 && !ok)
             flag(dev_status, TSD_DEV_TIMEOUT);
     } else {
-        // scratch = {tag of CTA 0, tag of CTA 1, abort}: CTA 1 never publishes
-        double2 val;
-        if (!team_exchange(slots, scratch, 0, 2, 1, scratch + 2, val, &sh_ok, limit_ns) &&
-            threadIdx.x == 0)
+        if (!team_barrier(team, 2, &sh_ok, limit_ns) && threadIdx.x == 0)
             flag(dev_status, TSD_DEV_TIMEOUT);
     }
 }
@@ -46,12 +41,12 @@ __global__ void wait_probe_kernel(int kind, unsigned long long limit_ns, int *sc
 int launch_wait_probe(int kind, unsigned long long limit_ns, void *scratch,
                       int32_t *dev_status, cudaStream_t stream)
 {
-    int *ints = static_cast<int *>(scratch);
-    if (cudaMemsetAsync(ints, 0, 3 * sizeof(int), stream) != cudaSuccess) {
+    int2 *team = static_cast<int2 *>(scratch);
+    if (cudaMemsetAsync(team, 0, sizeof(int2), stream) != cudaSuccess) {
         (void)cudaGetLastError();
         return TSD_ERR_CUDA;
     }
-    wait_probe_kernel<<<1, 32, 0, stream>>>(kind, limit_ns, ints, dev_status);
+    wait_probe_kernel<<<1, 32, 0, stream>>>(kind, limit_ns, team, dev_status);
     TSD_LAUNCH_CHECK();
     return TSD_OK;
 }
