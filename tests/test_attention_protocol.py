@@ -44,17 +44,10 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
     key tile; per tile they exchange their redo votes and, when either voted,
     their row maxima (then both may rescale O), and at the end their row
     sums -- each exchange a phase of the quarter's pair mbarrier.
-    cm = 1: one commit point per key tile -- the first NS QK products
-    commit to s_full alone (phase 0), then after PV_j and QK_{j+NS} one commit
-    point to s_full[j % NS] (phase j / NS + 1: PV_j done, and QK_{j+NS} if it
-    exists) and to the V ring's v_empty[j % NSV]; the softmax's waits for "PV_r
-    done" wait for that s_full phase, the producer reuses V slots on v_empty
-    (a wait for s_full phase j / NS + 1 there could come two phases early on
-    the last tiles, where no K wait precedes it).
-    cm = 3: as cm = 1, but the MMA thread waits only for P_j (and for K of
-    the first NS tiles); the first softmax warp waits for V_j and K_{j+NS}
-    before it publishes P_j.  The MMA model checks that the tiles it reads
-    have landed."""
+    cm = 4: the MMA thread waits only for P_j (and for K of the first NS
+    tiles); the first softmax warp waits for V_j and K_{j+NS} before it
+    publishes P_j.  Commits and ring reuse as with cm = 2.  The MMA model
+    checks that the tiles it reads have landed."""
     rnd = random.Random(seed)
     nsm = 4 * sw
     bars = {"q_full": _Barrier(nsm)}
@@ -92,8 +85,6 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
 
     def pv_passed(r):
         """The wait for "PV_r done" under the commit scheme."""
-        if cm in (1, 3):
-            return passes(("s_full", r % NS), r // NS + 1)
         return passes(("o_ready", r % NS), r // NS)
 
     qk_done, pv_done_set = set(), set()
@@ -117,7 +108,7 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
                 j = i - 1
                 s = j % NSV
                 if j >= NSV:
-                    if merged and cm == 2:   # PV_{j-NSV} done: o_ready[(j - NSV) % NS]
+                    if merged:   # PV_{j-NSV} done: o_ready[(j - NSV) % NS]
                         r = j - NSV
                         while not pv_passed(r):
                             yield
@@ -134,7 +125,7 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
             yield
 
         def qk(i):
-            if cm != 3 or i < NS:
+            if cm != 4 or i < NS:
                 while not passes(("k_full", i % NSK), i // NSK):
                     yield
             assert ("k", i) in landed, f"QK_{i} issued before K_{i} landed"
@@ -142,11 +133,7 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
             prev = s_owner.get(buf)
             assert prev is None or prev in pv_done or ("pv", prev) in [p[0] for p in pipe], \
                 f"QK_{i} issued over the P of tile {prev} before its PV"
-            if cm in (1, 3) and i >= NS:
-                commits = []             # covered by the tile's single commit
-            else:
-                commits = [("s_full", buf)] if merged else \
-                    [("s_full", buf), ("k_empty", i % NSK)]
+            commits = [("s_full", buf)] if merged else [("s_full", buf), ("k_empty", i % NSK)]
             pipe.append((("qk", i), commits))
             s_owner[buf] = i
         for i in range(min(NS, ntiles)):
@@ -154,20 +141,15 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
         for j in range(ntiles):
             while not passes(("p_full", j % NS), j // NS):
                 yield
-            if cm != 3:
+            if cm != 4:
                 while not passes(("v_full", j % NSV), j // NSV):
                     yield
             assert ("v", j) in landed, f"PV_{j} issued before V_{j} landed"
-            if cm in (1, 3):
-                commits = []
-            else:
-                commits = [("o_ready", j % NS)] if merged else \
-                    [("v_empty", j % NSV), ("o_ready", j % NS)]
+            commits = [("o_ready", j % NS)] if merged else \
+                [("v_empty", j % NSV), ("o_ready", j % NS)]
             pipe.append((("pv", j), commits))
             if j + NS < ntiles:
                 yield from qk(j + NS)
-            if cm in (1, 3):   # one commit point: tracks everything issued so far
-                pipe.append((("commit", j), [("s_full", j % NS), ("v_empty", j % NSV)]))
             yield
 
     def exchange(q, n):
@@ -197,7 +179,7 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
                 while not pv_passed(j - 1):
                     yield
                 assert j - 1 in pv_done
-            if cm == 3 and first:                       # for the MMA thread
+            if cm == 4 and first:                       # for the MMA thread
                 while not passes(("v_full", j % NSV), j // NSV):
                     yield
                 if j + NS < ntiles:
@@ -257,17 +239,9 @@ def test_rows_kernel_protocol(NS, NSK, NSV, sw, ntiles):
 @pytest.mark.parametrize("NS,NSK,NSV,sw", [(3, 3, 2, 1), (2, 2, 2, 1), (3, 3, 2, 2)],
                          ids=["128-key tiles", "64-key tiles", "128-key tiles, paired softmax"])
 @pytest.mark.parametrize("ntiles", [1, 2, 3, 4, 5, 8, 17])
-def test_rows_kernel_protocol_one_commit_per_tile(NS, NSK, NSV, sw, ntiles):
+def test_rows_kernel_protocol_one_mma_wait_per_tile(NS, NSK, NSV, sw, ntiles):
     for seed in range(150):
-        _run(NS, NSK, NSV, ntiles, seed, sw=sw, cm=1)
-
-
-@pytest.mark.parametrize("NS,NSK,NSV,sw", [(3, 3, 2, 1), (2, 2, 2, 1), (3, 3, 2, 2)],
-                         ids=["128-key tiles", "64-key tiles", "128-key tiles, paired softmax"])
-@pytest.mark.parametrize("ntiles", [1, 2, 3, 4, 5, 8, 17])
-def test_rows_kernel_protocol_one_wait_per_tile(NS, NSK, NSV, sw, ntiles):
-    for seed in range(150):
-        _run(NS, NSK, NSV, ntiles, seed, sw=sw, cm=3)
+        _run(NS, NSK, NSV, ntiles, seed, sw=sw, cm=4)
 
 
 @pytest.mark.parametrize("ntiles", [1, 3, 6])

@@ -328,7 +328,7 @@ __device__ __forceinline__ void load_kv_tile(uint32_t dst, const CUtensorMap *tm
 // on o_ready[(j - NSV) % NS] -- which saves the MMA thread two commits per
 // tile.  Either wait names a phase that cannot be stale or ahead: the phase
 // after it needs K_i (or V_{j+1}), which this producer has not loaded yet.
-template <class Gm, int NS_PROD, int CM = 2>
+template <class Gm, int NS_PROD>
 __device__ __forceinline__ void produce_kv(const Setup<Gm> &su, const CUtensorMap *tmK,
                                            const CUtensorMap *tmV, int b, int hk, int Hkv,
                                            int kb, int ntiles, const KvPages &pages,
@@ -355,13 +355,10 @@ __device__ __forceinline__ void produce_kv(const Setup<Gm> &su, const CUtensorMa
             if (j >= NSV) {
                 const int r = j - NSV;   // PV_r read this slot last
                 constexpr int NSP = NS_PROD ? NS_PROD : 1;
-                // PV_r done: the ring's own v_empty (committed by the MMA warp
-                // without NS_PROD, and with one commit point per tile, CM = 1),
-                // or o_ready[r % NS] phase r / NS.  (With CM = 1 a wait for
-                // s_full[r % NS] phase r / NS + 1 could come two phases early on
-                // the last tiles, where no K wait precedes it.)
+                // PV_r done: o_ready[r % NS] phase r / NS, or the ring's own
+                // v_empty (which the MMA warp then commits as well)
                 const bool ok =
-                    (!NS_PROD || CM != 2)
+                    !NS_PROD
                         ? ptx::mbar_wait(su.bars.v_empty(s), ((j / NSV) - 1) & 1, su.abort_flag)
                         : ptx::mbar_wait(su.bars.o_ready(r % NSP), (r / NSP) & 1,
                                          su.abort_flag);
@@ -926,15 +923,15 @@ __global__ void __launch_bounds__(rows_threads<SW>(), kMinBlocks)
     if (warp == 0) {
         const PageCache pc = stage_pages(su, pages, b, kb, min(ke, P + T), lane);
         if (lane == 0)
-            produce_kv<Gm, NS, CM>(su, &tmK, &tmV, b, hk, Hkv, kb, ntiles, pages, pc, P + T,
-                                   dev_status);
-    } else if (warp == 1 && CM == 3) {
-        // One mbarrier wait per key tile (each wait on this thread, even on a
-        // completed barrier, leaves the tensor pipe idle for about one MMA):
-        // lane 0 alone waits for P_j, whose last arrival comes from softmax
+            produce_kv<Gm, NS>(su, &tmK, &tmV, b, hk, Hkv, kb, ntiles, pages, pc, P + T,
+                               dev_status);
+    } else if (warp == 1 && CM == 4) {
+        // One mbarrier wait per key tile: each wait on this thread, even on a
+        // completed barrier, leaves the tensor pipe idle for about one MMA.
+        // Lane 0 alone waits for P_j -- whose last arrival comes from softmax
         // warp 4 after it has seen V_j and K_{j+NS} land (and zeroed V_j's
-        // rows past the range end), then issues PV_j and QK_{j+NS} and one
-        // commit point, as for CM = 1.
+        // rows past the range end) -- then issues PV_j (commit o_ready) and
+        // QK_{j+NS} (commit s_full), as in the two-wait schedule.
         if (lane == 0) {
             bool ok = ptx::mbar_wait(su.bars.q_full(), 0, su.abort_flag);
             for (int i = 0; ok && i < min(NS, ntiles); ++i) {
@@ -947,51 +944,36 @@ __global__ void __launch_bounds__(rows_threads<SW>(), kMinBlocks)
                 if (!ptx::mbar_wait(su.bars.p_full(j % NS), (j / NS) & 1, su.abort_flag))
                     break;
                 ptx::tc_fence_after();
-                issue_pv<Gm, false, SW == 2, false, false>(su, 0, col_s(j), kO, j, j > 0, BN,
-                                                           0u);
+                issue_pv<Gm, false, SW == 2, true, false>(su, 0, col_s(j), kO, j, j > 0, BN,
+                                                          su.bars.o_ready(j % NS));
                 if (j + NS < ntiles)
-                    issue_qk<Gm, false, false, false>(su, 0, col_s(j + NS), j + NS, 0u);
-                ptx::mma_commit(su.bars.s_full(j % NS));
-                ptx::mma_commit(su.bars.v_empty(j % NSV));
+                    issue_qk<Gm, false, true, false>(su, 0, col_s(j + NS), j + NS,
+                                                     su.bars.s_full((j + NS) % NS));
             }
         }
     } else if (warp == 1) {
         bool ok = warp_wait(su.bars.q_full(), 0, su.abort_flag);
         ptx::tc_fence_after();
-        // CM = 2: QK_i commits to s_full[i % NS], PV_j to o_ready[j % NS].
-        // CM = 1: one commit point per tile -- after PV_j and QK_{j+NS} (or
-        // PV_j alone for the last NS tiles) to s_full[j % NS], so its phase
-        // j / NS + 1 says both are done (the first NS QKs commit alone, phase
-        // 0), and to the V ring's v_empty[j % NSV] for the producer.
-        auto qk = [&](int i, bool commit) {
+        // QK_i commits to s_full[i % NS], PV_j to o_ready[j % NS]
+        auto qk = [&](int i) {
             if (!warp_wait(su.bars.k_full(i % NSK), (i / NSK) & 1, su.abort_flag))
                 return false;
             ptx::tc_fence_after();
-            if (commit)
-                issue_qk<Gm, false, true>(su, lane, col_s(i), i, su.bars.s_full(i % NS));
-            else
-                issue_qk<Gm, false, false>(su, lane, col_s(i), i, su.bars.s_full(i % NS));
+            issue_qk<Gm, false>(su, lane, col_s(i), i, su.bars.s_full(i % NS));
             return true;
         };
         for (int i = 0; ok && i < min(NS, ntiles); ++i)
-            ok = qk(i, true);
+            ok = qk(i);
         for (int j = 0; ok && j < ntiles; ++j) {
             if (!warp_wait(su.bars.p_full(j % NS), (j / NS) & 1, su.abort_flag) ||
                 !warp_wait(su.bars.v_full(j % NSV), (j / NSV) & 1, su.abort_flag)) {
                 ok = false;
                 break;
             }
-            issue_pv<Gm, false, SW == 2, CM == 2>(su, lane, col_s(j), kO, j, j > 0,
-                                                  P + T - (kb + j * BN), su.bars.o_ready(j % NS));
+            issue_pv<Gm, false, SW == 2>(su, lane, col_s(j), kO, j, j > 0,
+                                         P + T - (kb + j * BN), su.bars.o_ready(j % NS));
             if (j + NS < ntiles)
-                ok = qk(j + NS, CM == 2);
-            if (CM == 1 && ok) {
-                if (lane == 0) {
-                    ptx::mma_commit(su.bars.s_full(j % NS));
-                    ptx::mma_commit(su.bars.v_empty(j % NSV));
-                }
-                __syncwarp();
-            }
+                ok = qk(j + NS);
         }
     } else {
         // softmax warps: one query row per thread == TMEM lane; with SW = 2
@@ -1015,12 +997,9 @@ __global__ void __launch_bounds__(rows_threads<SW>(), kMinBlocks)
             mw[w] = (row_ok && w < W) ? mask[((size_t)b * Tmax + u) * W + w] : 0u;
         const uint32_t taddr_o = su.tmem + lane_off + kO + hf * 64;
         PairXchg *xc = reinterpret_cast<PairXchg *>(su.gbase + Gm::kOffXchg) + quarter;
-        // PV_i done: o_ready[i % NS] phase i / NS, or (CM = 1, 3) s_full[i % NS]
-        // phase i / NS + 1
+        // PV_i done (o_ready[i % NS] completes once per tile of that class)
         auto wait_pv = [&](int i) {
-            return CM != 2
-                       ? warp_wait(su.bars.s_full(i % NS), ((i / NS) + 1) & 1, su.abort_flag)
-                       : warp_wait(su.bars.o_ready(i % NS), (i / NS) & 1, su.abort_flag);
+            return warp_wait(su.bars.o_ready(i % NS), (i / NS) & 1, su.abort_flag);
         };
         float m_run = -INFINITY, l_run = 0.f;
         int nx = 0;   // pair exchanges made
@@ -1043,7 +1022,7 @@ __global__ void __launch_bounds__(rows_threads<SW>(), kMinBlocks)
             if (!ok)
                 break;
             ptx::tc_fence_before();
-            if (CM == 3 && warp == 4) {
+            if (CM == 4 && warp == 4) {
                 // for the MMA thread: V_j and K_{j+NS} have landed, V_j's rows
                 // past the range end are zero
                 ok = warp_wait(su.bars.v_full(j % NSV), (j / NSV) & 1, su.abort_flag);
@@ -1254,7 +1233,7 @@ struct UmmaPlan {
     bool paired;     // rows kernel with 64-key tiles, two CTAs per SM
     int sw;          // 128-key rows kernel: softmax warps per TMEM lane quarter
     int nf;          // with sw = 2: score pairs of 16 exponentiated on the FMA pipe
-    int cm;          // rows kernels: commit points per key tile (1 or 2)
+    int cm;          // rows kernels: MMA schedule (2: waits for P, V, K; 4: for P only)
     int nrb, nsplit, keys_per_split;
 };
 
@@ -1267,16 +1246,13 @@ int rows_softmax_warps()
     return (e && e[0] == '2' && e[1] == '\0') ? 2 : 1;
 }
 
-// MMA-thread schedule of the rows kernels (TSD_ATTN_COMMITS, read at every
-// launch): 2 -- commits after QK and after PV, waits for P, V and K per tile;
-// "1" -- one commit point per tile; "3" -- one commit point and one wait
-// (for P) per tile, a softmax warp checking V and K first.
-int rows_commit_points()
+// MMA-thread schedule of the rows kernels (TSD_ATTN_MMA_WAITS, read at
+// every launch): 3 -- the MMA warp waits for P, V and K of every tile; "1"
+// -- lane 0 waits for P alone, a softmax warp having checked V and K.
+int rows_mma_waits()
 {
-    const char *e = std::getenv("TSD_ATTN_COMMITS");
-    if (e && e[1] == '\0' && (e[0] == '1' || e[0] == '3'))
-        return e[0] - '0';
-    return 2;
+    const char *e = std::getenv("TSD_ATTN_MMA_WAITS");
+    return (e && e[0] == '1' && e[1] == '\0') ? 1 : 3;
 }
 
 // With two softmax warps per quarter: of every 16 score pairs, how many are
@@ -1319,9 +1295,7 @@ UmmaPlan umma_plan(const AttnArgs &a, int num_sms)
     p.paired = small ? !p.keysplit : rows_variant() == 2;
     p.sw = (p.keysplit || p.paired) ? 1 : rows_softmax_warps();
     p.nf = p.sw == 2 ? rows_exp_fma() : 0;
-    p.cm = p.keysplit ? 2 : rows_commit_points();
-    if (p.nf != 0)
-        p.cm = 2;   // the FMA-exponential instances are built with two
+    p.cm = (!p.keysplit && rows_mma_waits() == 1) ? 4 : 2;
     p.nrb = p.keysplit ? 1 : (a.Tmax * G + BQ - 1) / BQ;
     const int bn = p.paired ? Half::BN : Wide::BN;
     const int slots = num_sms * (p.paired ? 2 : 1);
@@ -1409,32 +1383,23 @@ cudaError_t set_smem_attributes()
         return cudaErrorInvalidDevice;
     if (done[dev].load())
         return cudaSuccess;
-    auto wide = tree_attn_rows_kernel<Wide, 3, 1, 1>;
-    auto wide2 = tree_attn_rows_kernel<Wide, 3, 1, 2, 0>;
-    auto wide2f4 = tree_attn_rows_kernel<Wide, 3, 1, 2, 4>;
-    auto wide2f6 = tree_attn_rows_kernel<Wide, 3, 1, 2, 6>;
-    auto wide_c1 = tree_attn_rows_kernel<Wide, 3, 1, 1, 0, 1>;
-    auto wide2_c1 = tree_attn_rows_kernel<Wide, 3, 1, 2, 0, 1>;
-    auto wide_c3 = tree_attn_rows_kernel<Wide, 3, 1, 1, 0, 3>;
-    auto wide2_c3 = tree_attn_rows_kernel<Wide, 3, 1, 2, 0, 3>;
-    auto half = tree_attn_rows_kernel<Half, 2, 2, 1>;
-    auto half_c1 = tree_attn_rows_kernel<Half, 2, 2, 1, 0, 1>;
-    auto half_c3 = tree_attn_rows_kernel<Half, 2, 2, 1, 0, 3>;
-    err = cudaFuncSetAttribute(wide, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)Wide::kSmemBytes);
-    for (auto k : {wide_c1, wide2_c1, wide_c3, wide2_c3})
+    const void *wide_kernels[] = {
+        (const void *)tree_attn_rows_kernel<Wide, 3, 1, 1, 0, 2>,
+        (const void *)tree_attn_rows_kernel<Wide, 3, 1, 1, 0, 4>,
+        (const void *)tree_attn_rows_kernel<Wide, 3, 1, 2, 0, 2>,
+        (const void *)tree_attn_rows_kernel<Wide, 3, 1, 2, 0, 4>,
+        (const void *)tree_attn_rows_kernel<Wide, 3, 1, 2, 4, 2>,
+        (const void *)tree_attn_rows_kernel<Wide, 3, 1, 2, 4, 4>,
+        (const void *)tree_attn_rows_kernel<Wide, 3, 1, 2, 6, 2>,
+        (const void *)tree_attn_rows_kernel<Wide, 3, 1, 2, 6, 4>,
+        (const void *)tree_attn_keysplit_kernel};
+    for (const void *k : wide_kernels)
         if (err == cudaSuccess)
             err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)Wide::kSmemBytes);
-    for (auto k : {wide2, wide2f4, wide2f6})
-        if (err == cudaSuccess)
-            err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)Wide::kSmemBytes);
-    if (err == cudaSuccess)
-        err = cudaFuncSetAttribute(tree_attn_keysplit_kernel,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)Wide::kSmemBytes);
-    for (auto k : {half, half_c1, half_c3}) {
+    const void *half_kernels[] = {(const void *)tree_attn_rows_kernel<Half, 2, 2, 1, 0, 2>,
+                                  (const void *)tree_attn_rows_kernel<Half, 2, 2, 1, 0, 4>};
+    for (const void *k : half_kernels) {
         if (err == cudaSuccess)
             err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)Half::kSmemBytes);
@@ -1514,17 +1479,17 @@ int launch_umma_attention(const AttnArgs &a, void *ws, size_t ws_bytes, int num_
             a.Tmax, a.Hq, a.Hkv, a.Lmax, W, sl2, p.keys_per_split, p.nsplit,
             static_cast<__nv_bfloat16 *>(a.out), part_o, part_ml, a.dev_status, a.pages);
     else {
-        auto kern = p.paired ? (p.cm == 1   ? tree_attn_rows_kernel<Half, 2, 2, 1, 0, 1>
-                                : p.cm == 3 ? tree_attn_rows_kernel<Half, 2, 2, 1, 0, 3>
-                                            : tree_attn_rows_kernel<Half, 2, 2, 1>)
-                  : p.sw == 1 ? (p.cm == 1   ? tree_attn_rows_kernel<Wide, 3, 1, 1, 0, 1>
-                                 : p.cm == 3 ? tree_attn_rows_kernel<Wide, 3, 1, 1, 0, 3>
-                                             : tree_attn_rows_kernel<Wide, 3, 1, 1>)
-                  : p.nf == 6 ? tree_attn_rows_kernel<Wide, 3, 1, 2, 6>
-                  : p.nf == 4 ? tree_attn_rows_kernel<Wide, 3, 1, 2, 4>
-                  : p.cm == 1 ? tree_attn_rows_kernel<Wide, 3, 1, 2, 0, 1>
-                  : p.cm == 3 ? tree_attn_rows_kernel<Wide, 3, 1, 2, 0, 3>
-                              : tree_attn_rows_kernel<Wide, 3, 1, 2, 0>;
+        const bool c4 = p.cm == 4;
+        auto kern = p.paired    ? (c4 ? tree_attn_rows_kernel<Half, 2, 2, 1, 0, 4>
+                                      : tree_attn_rows_kernel<Half, 2, 2, 1, 0, 2>)
+                  : p.sw == 1   ? (c4 ? tree_attn_rows_kernel<Wide, 3, 1, 1, 0, 4>
+                                      : tree_attn_rows_kernel<Wide, 3, 1, 1, 0, 2>)
+                  : p.nf == 6   ? (c4 ? tree_attn_rows_kernel<Wide, 3, 1, 2, 6, 4>
+                                      : tree_attn_rows_kernel<Wide, 3, 1, 2, 6, 2>)
+                  : p.nf == 4   ? (c4 ? tree_attn_rows_kernel<Wide, 3, 1, 2, 4, 4>
+                                      : tree_attn_rows_kernel<Wide, 3, 1, 2, 4, 2>)
+                                : (c4 ? tree_attn_rows_kernel<Wide, 3, 1, 2, 0, 4>
+                                      : tree_attn_rows_kernel<Wide, 3, 1, 2, 0, 2>);
         const int threads = p.sw == 2 ? rows_threads<2>() : rows_threads<1>();
         const uint32_t smem = p.paired ? Half::kSmemBytes : Wide::kSmemBytes;
         kern<<<grid, threads, smem, stream>>>(
