@@ -928,28 +928,33 @@ __global__ void __launch_bounds__(rows_threads<SW>(), kMinBlocks)
     } else if (warp == 1 && CM == 4) {
         // One mbarrier wait per key tile: each wait on this thread, even on a
         // completed barrier, leaves the tensor pipe idle for about one MMA.
-        // Lane 0 alone waits for P_j -- whose last arrival comes from softmax
-        // warp 4 after it has seen V_j and K_{j+NS} land (and zeroed V_j's
-        // rows past the range end) -- then issues PV_j (commit o_ready) and
-        // QK_{j+NS} (commit s_full), as in the two-wait schedule.
-        if (lane == 0) {
-            bool ok = ptx::mbar_wait(su.bars.q_full(), 0, su.abort_flag);
-            for (int i = 0; ok && i < min(NS, ntiles); ++i) {
-                ok = ptx::mbar_wait(su.bars.k_full(i % NSK), (i / NSK) & 1, su.abort_flag);
-                ptx::tc_fence_after();
-                if (ok)
-                    issue_qk<Gm, false, true, false>(su, 0, col_s(i), i, su.bars.s_full(i % NS));
-            }
-            for (int j = 0; ok && j < ntiles; ++j) {
-                if (!ptx::mbar_wait(su.bars.p_full(j % NS), (j / NS) & 1, su.abort_flag))
-                    break;
-                ptx::tc_fence_after();
-                issue_pv<Gm, false, SW == 2, true, false>(su, 0, col_s(j), kO, j, j > 0, BN,
-                                                          su.bars.o_ready(j % NS));
-                if (j + NS < ntiles)
-                    issue_qk<Gm, false, true, false>(su, 0, col_s(j + NS), j + NS,
-                                                     su.bars.s_full((j + NS) % NS));
-            }
+        // Lane 0 waits for P_j -- whose last arrival comes from softmax warp
+        // 4 after it has seen V_j and K_{j+NS} land (and zeroed V_j's rows
+        // past the range end) -- and the warp stays converged on its result;
+        // lane 0 then issues PV_j (commit o_ready) and QK_{j+NS} (commit
+        // s_full), as in the three-wait schedule.
+        auto wait0 = [&](uint32_t bar, uint32_t parity) {
+            bool ok = true;
+            if (lane == 0)
+                ok = ptx::mbar_wait(bar, parity, su.abort_flag);
+            return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        };
+        bool ok = wait0(su.bars.q_full(), 0);
+        for (int i = 0; ok && i < min(NS, ntiles); ++i) {
+            ok = wait0(su.bars.k_full(i % NSK), (i / NSK) & 1);
+            ptx::tc_fence_after();
+            if (ok)
+                issue_qk<Gm, false, true, false>(su, lane, col_s(i), i, su.bars.s_full(i % NS));
+        }
+        for (int j = 0; ok && j < ntiles; ++j) {
+            if (!wait0(su.bars.p_full(j % NS), (j / NS) & 1))
+                break;
+            ptx::tc_fence_after();
+            issue_pv<Gm, false, SW == 2, true, false>(su, lane, col_s(j), kO, j, j > 0, BN,
+                                                      su.bars.o_ready(j % NS));
+            if (j + NS < ntiles)
+                issue_qk<Gm, false, true, false>(su, lane, col_s(j + NS), j + NS,
+                                                 su.bars.s_full((j + NS) % NS));
         }
     } else if (warp == 1) {
         bool ok = warp_wait(su.bars.q_full(), 0, su.abort_flag);

@@ -60,6 +60,8 @@ constexpr int kTeamMax = 32;          // CTAs per team: one partial per lane of 
 constexpr int kTeamMinChunk = 2048;   // vocabulary entries per CTA, at least
 constexpr int kWalkMaxCtas = 1024;    // grid cap (sets the workspace slots)
 constexpr unsigned long long kTeamWaitNs = 2000000000ull;   // bound of one barrier wait
+constexpr int kCacheGroups = 4;       // groups of 4 entries per thread in the cached walk
+constexpr int kCacheChunk = 4 * kCacheGroups * kWalkThreads;   // 4096 entries: 32 KB fp64
 constexpr int kDecCache = 8;          // children per row whose test operands are prefetched
 constexpr int kDecOps = 2 * kDecCache + kDecCache * (kDecCache + 1) / 2;   // 52 loads
 
@@ -462,6 +464,165 @@ __device__ double chunk_residual(const float *__restrict__ row, const float *__r
     return s;
 }
 
+// ---- the cached form: a CTA keeps its chunk of the current distribution in
+// shared memory (kCacheChunk entries at most), scaled: p(x) = pc[x - x_lo] * g.
+// Thread tid owns the groups of four entries tid, tid + 256, tid + 512 and
+// tid + 768 of the chunk in every pass, so each pass reads the global rows
+// once with coalesced loads and the cached values need no barrier between the
+// passes of a row.
+
+// m/Z pass: the chunk's logits -> registers, the chunk max m_k (and the
+// largest x with a finite logit), then pc = exp((l - m_k)/T) and its sum.
+template <bool VEC>
+__device__ double2 chunk_max_z_cached(const float *__restrict__ row, int x_lo, int x_hi, int V,
+                                      double inv_temp, const double *table, double *pc,
+                                      float *shf, double *shd, int *shi, int *last_out)
+{
+    float l[4 * kCacheGroups];
+    float mt = -INFINITY;
+    int last = -1;
+#pragma unroll
+    for (int m = 0; m < kCacheGroups; ++m) {
+        const int x0 = x_lo + 4 * (threadIdx.x + kWalkThreads * m);
+        float v[4];
+        if (x0 < x_hi)
+            load4<VEC>(row, x0, V, v);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float lv = (x0 + k < x_hi) ? v[k] : -INFINITY;
+            l[4 * m + k] = lv;
+            mt = fmaxf(mt, lv);
+            if (lv > -INFINITY)
+                last = x0 + k;
+        }
+    }
+    block_max_last<kWalkThreads>(mt, last, shf, shi);
+    *last_out = last;
+    double z = 0.0;
+#pragma unroll
+    for (int m = 0; m < kCacheGroups; ++m) {
+        const int i0 = 4 * (threadIdx.x + kWalkThreads * m);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            if (x_lo + i0 + k < x_hi) {
+                const float lv = l[4 * m + k];
+                const double e = (lv == -INFINITY)
+                                     ? 0.0
+                                     : table_exp(((double)lv - (double)mt) * inv_temp, table);
+                pc[i0 + k] = e;
+                z += e;
+            }
+        }
+    }
+    return make_double2((double)mt, mt == -INFINITY ? 0.0 : block_sum<kWalkThreads>(z, shd));
+}
+
+// Residual pass: S_k = sum over the chunk of max(0, p(x) - q(x)) with p(x) =
+// pc * g, and the largest x where that is positive.
+template <bool VEC>
+__device__ double chunk_residual_cached(const float *__restrict__ q, int x_lo, int x_hi, int V,
+                                        const double *pc, double g, double *shd, int *shi,
+                                        int *last_out)
+{
+    double s = 0.0;
+    int last = -1;
+#pragma unroll
+    for (int m = 0; m < kCacheGroups; ++m) {
+        const int i0 = 4 * (threadIdx.x + kWalkThreads * m);
+        const int x0 = x_lo + i0;
+        if (x0 >= x_hi)
+            continue;
+        float qv[4];
+        load4<VEC>(q, x0, V, qv);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            if (x0 + k < x_hi) {
+                const double r = pc[i0 + k] * g - (double)qv[k];
+                if (r > 0.0) {
+                    s += r;
+                    last = x0 + k;
+                }
+            }
+        }
+    }
+    block_sum_last<kWalkThreads>(s, last, shd, shi);
+    *last_out = last;
+    return s;
+}
+
+// After a rejection with residual sum S > 0: pc = max(0, pc * g - q) / S (the
+// q chunk comes from L1, just read), so that g becomes 1.  Each thread
+// rewrites only the entries it owns.
+template <bool VEC>
+__device__ void chunk_renormalise_cached(const float *__restrict__ q, int x_lo, int x_hi, int V,
+                                         double *pc, double g, double inv_S)
+{
+#pragma unroll
+    for (int m = 0; m < kCacheGroups; ++m) {
+        const int i0 = 4 * (threadIdx.x + kWalkThreads * m);
+        const int x0 = x_lo + i0;
+        if (x0 >= x_hi)
+            continue;
+        float qv[4];
+        load4<VEC>(q, x0, V, qv);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            if (x0 + k < x_hi) {
+                const double r = pc[i0 + k] * g - (double)qv[k];
+                pc[i0 + k] = (r > 0.0 ? r : 0.0) * inv_S;
+            }
+        }
+    }
+}
+
+// The draw inside the chunk, from the cached distribution: the smallest x
+// with carry + sum_{x_lo <= y <= x} p(y) > u (fp64 block scan in order), or
+// INT_MAX when rounding leaves the chunk's sum short of u.
+__device__ int chunk_scan_cached(const double *pc, double g, int x_lo, int x_hi, double carry,
+                                 double u, double *warp_tot, int *shi)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int base = x_lo; base < x_hi; base += 4 * kWalkThreads) {
+        const int x0 = base + 4 * threadIdx.x;
+        double p[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            if (x0 + k < x_hi)
+                p[k] = pc[x0 + k - x_lo] * g;
+        const double mine = ((p[0] + p[1]) + p[2]) + p[3];
+        double incl = mine;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const double y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o)
+                incl += y;
+        }
+        if (lane == 31)
+            warp_tot[warp] = incl;
+        __syncthreads();
+        double wbase = 0.0, tile = 0.0;
+        for (int w2 = 0; w2 < kWalkWarps; ++w2) {
+            const double t = warp_tot[w2];
+            if (w2 < warp)
+                wbase += t;
+            tile += t;
+        }
+        double C = carry + wbase + (incl - mine);
+        int found = INT_MAX;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            C += p[k];
+            if (found == INT_MAX && x0 + k < x_hi && C > u)
+                found = x0 + k;
+        }
+        found = block_min_int<kWalkThreads>(found, shi);   // ends with a barrier
+        if (found != INT_MAX)
+            return found;
+        carry += tile;
+    }
+    return INT_MAX;
+}
+
 // The draw inside the chunk [x_lo, x_hi): the smallest x with
 // carry + sum_{x_lo <= y <= x} p^(n)(y) > u (fp64 block scan in order), or
 // INT_MAX when rounding leaves the chunk's sum short of u.
@@ -627,8 +788,8 @@ __global__ void __launch_bounds__(kFinThreads)
 // VEC: V % 4 == 0, so every logits / q row is 16-byte aligned (the entry
 // point checks the base pointers) and the passes use float4 loads.
 // Grid: teams x K CTAs; team t walks sequences t, t + teams, ...
-template <bool VEC>
-__global__ void __launch_bounds__(kWalkThreads)
+template <bool VEC, bool CACHED>
+__global__ void __launch_bounds__(kWalkThreads, CACHED ? 3 : 4)
     mss_walk_kernel(const float *__restrict__ logits, double temp,
                     const float *__restrict__ q_probs, int Rq, const int32_t *__restrict__ q_row,
                     const int32_t *__restrict__ tokens, const int32_t *__restrict__ n_nodes,
@@ -658,6 +819,9 @@ __global__ void __launch_bounds__(kWalkThreads)
     // dc[i] = l(x_i), dc[kDecCache + i] = u_i, dc[2 kDecCache + i(i+1)/2 + j] =
     // q_j(x_i) for j <= i (q_j: the q row of child j; j = i: the child's own)
     __shared__ double dc[kDecOps];
+    // CACHED: this CTA's chunk of the current distribution, p(x) = pc[x - x_lo] * g
+    __shared__ double pc[CACHED ? kCacheChunk : 1];
+    double g = 0.0;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int teams = gridDim.x / K;
     const int team = blockIdx.x / K, k = blockIdx.x % K;
@@ -772,7 +936,10 @@ __global__ void __launch_bounds__(kWalkThreads)
             // m and Z of this row (slot: z_k, then m_k as fp32 bits | last_k)
             int lastk;
             const double2 mz =
-                chunk_max_z<VEC>(lrow, x_lo, x_hi, V, inv_temp, table, shf, shd, shi, &lastk);
+                CACHED ? chunk_max_z_cached<VEC>(lrow, x_lo, x_hi, V, inv_temp, table, pc, shf,
+                                                 shd, shi, &lastk)
+                       : chunk_max_z<VEC>(lrow, x_lo, x_hi, V, inv_temp, table, shf, shd, shi,
+                                          &lastk);
             if (op >= 0)
                 dc[op] = pre;
             double2 *sl = slots();
@@ -813,6 +980,10 @@ __global__ void __launch_bounds__(kWalkThreads)
                 }
             }
             __syncthreads();
+            if (CACHED)   // every thread: this CTA's scale of its cached chunk
+                g = mz.x == -INFINITY
+                        ? 0.0
+                        : table_exp((mz.x - st.m) * inv_temp, table) * st.inv_Z;
             int accepted = -1;
             for (int i = 0; c >= 0; ++i) {
                 if (sh_dec) {
@@ -821,7 +992,9 @@ __global__ void __launch_bounds__(kWalkThreads)
                 }
                 const float *qc = qrow(c);
                 const double s =
-                    chunk_residual<VEC>(lrow, qc, x_lo, x_hi, V, st, table, shd, shi, &lastk);
+                    CACHED ? chunk_residual_cached<VEC>(qc, x_lo, x_hi, V, pc, g, shd, shi, &lastk)
+                           : chunk_residual<VEC>(lrow, qc, x_lo, x_hi, V, st, table, shd, shi,
+                                                 &lastk);
                 sl = slots();
                 if (tid == 0)
                     sl[k] = make_double2(s, (double)lastk);
@@ -853,6 +1026,10 @@ __global__ void __launch_bounds__(kWalkThreads)
                     }
                 }
                 __syncthreads();
+                if (CACHED && st.S[st.n - 1] > 0.0) {   // else p stays as it was
+                    chunk_renormalise_cached<VEC>(qc, x_lo, x_hi, V, pc, g, st.inv_S[st.n - 1]);
+                    g = 1.0;
+                }
                 c = next;
             }
             if (!alive)
@@ -899,7 +1076,9 @@ __global__ void __launch_bounds__(kWalkThreads)
             __syncthreads();
             const int pick = sh_pick;
             if (pick == k) {
-                int token = chunk_scan<VEC>(lrow, x_lo, x_hi, V, st, table, sh_carry, u, shd, shi);
+                int token = CACHED ? chunk_scan_cached(pc, g, x_lo, x_hi, sh_carry, u, shd, shi)
+                                   : chunk_scan<VEC>(lrow, x_lo, x_hi, V, st, table, sh_carry, u,
+                                                     shd, shi);
                 if (token == INT_MAX)   // the chunk's own sum fell short by rounding
                     token = sh_token;
                 if (tid == 0 && in_bounds(n_path, Tmax + 1, dev_status)) {
@@ -958,23 +1137,30 @@ namespace {
 
 // CTAs of the walk kernel that fit on the device at once (cooperative
 // launch limit), capped by the workspace slots; looked up once per device.
-int walk_capacity(bool vec)
+const void *walk_kernel(bool vec, bool cached)
+{
+    return vec ? (cached ? reinterpret_cast<const void *>(mss_walk_kernel<true, true>)
+                         : reinterpret_cast<const void *>(mss_walk_kernel<true, false>))
+               : (cached ? reinterpret_cast<const void *>(mss_walk_kernel<false, true>)
+                         : reinterpret_cast<const void *>(mss_walk_kernel<false, false>));
+}
+
+int walk_capacity(bool vec, bool cached)
 {
     // Threads making their first call on a device at the same time may both
     // compute the value (the same one); the atomic makes that race benign.
     constexpr int kMaxDevices = 64;
-    static std::atomic<int> cap[2][kMaxDevices];
+    static std::atomic<int> cap[2][2][kMaxDevices];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
         return 0;
-    std::atomic<int> &slot = cap[vec ? 1 : 0][dev];
+    std::atomic<int> &slot = cap[vec ? 1 : 0][cached ? 1 : 0][dev];
     int c = slot.load(std::memory_order_relaxed);
     if (c == 0) {
         int sms = 0, occ = 0, coop = 0;
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
-        const void *fn = vec ? reinterpret_cast<const void *>(mss_walk_kernel<true>)
-                             : reinterpret_cast<const void *>(mss_walk_kernel<false>);
+        const void *fn = walk_kernel(vec, cached);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, kWalkThreads, 0);
         (void)cudaGetLastError();
         c = coop ? std::min(sms * occ, kWalkMaxCtas) : -1;
@@ -987,9 +1173,8 @@ int walk_capacity(bool vec)
 // device.  Team size: enough CTAs that each owns at least kTeamMinChunk
 // entries (at most kTeamMax), as long as every sequence still gets a team;
 // with more sequences than the grid holds, one-CTA teams each walk several.
-int walk_grid(int B, int V, int &K, int &teams, int &chunk)
+int walk_grid_for(int cap, int B, int V, int &K, int &teams, int &chunk)
 {
-    const int cap = walk_capacity((V & 3) == 0);
     if (cap <= 0 || B < 1)
         return TSD_ERR_CUDA;
     const int k_want = std::max(1, std::min(kTeamMax, V / kTeamMinChunk));
@@ -1005,12 +1190,26 @@ int walk_grid(int B, int V, int &K, int &teams, int &chunk)
     return TSD_OK;
 }
 
+// The walk keeps each CTA's chunk of the current distribution in shared
+// memory (`cached`) when the chunk fits kCacheChunk entries; otherwise it
+// recomputes the distribution from the rows in every pass.
+int walk_grid(int B, int V, int &K, int &teams, int &chunk, bool &cached)
+{
+    const bool vec = (V & 3) == 0;
+    int rc = walk_grid_for(walk_capacity(vec, true), B, V, K, teams, chunk);
+    cached = rc == TSD_OK && chunk <= kCacheChunk;
+    if (!cached)
+        rc = walk_grid_for(walk_capacity(vec, false), B, V, K, teams, chunk);
+    return rc;
+}
+
 }  // namespace
 
 int verify_stochastic_plan(int B, int V, int32_t out[4])
 {
     int K, teams, chunk;
-    const int rc = walk_grid(B, V, K, teams, chunk);
+    bool cached;
+    const int rc = walk_grid(B, V, K, teams, chunk, cached);
     if (rc != TSD_OK)
         return rc;
     out[0] = teams;
@@ -1032,7 +1231,8 @@ int launch_verify_stochastic(const float *logits, double temperature, const floa
         return TSD_OK;
     const bool vec = (V & 3) == 0;
     int K, teams, chunk;
-    if (walk_grid(B, V, K, teams, chunk) != TSD_OK)
+    bool cached;
+    if (walk_grid(B, V, K, teams, chunk, cached) != TSD_OK)
         return TSD_ERR_CUDA;
     VerifyWs w = carve(ws);
     if (cudaMemsetAsync(w.team, 0, (size_t)teams * sizeof(int2), stream) != cudaSuccess) {
@@ -1046,8 +1246,7 @@ int launch_verify_stochastic(const float *logits, double temperature, const floa
                     (void *)&Tmax,        (void *)&V,           (void *)&K,
                     (void *)&chunk,       (void *)&w,           (void *)&out_tokens,
                     (void *)&out_path,    (void *)&n_accepted,  (void *)&dev_status};
-    const void *fn = vec ? reinterpret_cast<const void *>(mss_walk_kernel<true>)
-                         : reinterpret_cast<const void *>(mss_walk_kernel<false>);
+    const void *fn = walk_kernel(vec, cached);
     if (cudaLaunchCooperativeKernel(fn, dim3(teams * K), dim3(kWalkThreads), args, 0, stream) !=
         cudaSuccess) {
         (void)cudaGetLastError();
