@@ -36,7 +36,7 @@ class _Barrier:
 
 
 def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged=True, sw=1,
-         redo_p=0.2, cm=2):
+         redo_p=0.2):
     """merged: the producer reuses a K slot once s_full of the QK that read it
     completes and a V slot once o_ready of the PV that read it completes (the
     rows kernels; the MMA thread then commits only to s_full and o_ready).
@@ -44,10 +44,7 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
     key tile; per tile they exchange their redo votes and, when either voted,
     their row maxima (then both may rescale O), and at the end their row
     sums -- each exchange a phase of the quarter's pair mbarrier.
-    cm = 4: the MMA thread waits only for P_j (and for K of the first NS
-    tiles); the first softmax warp waits for V_j and K_{j+NS} before it
-    publishes P_j.  Commits and ring reuse as with cm = 2.  The MMA model
-    checks that the tiles it reads have landed."""
+    The MMA model checks that the tiles it reads have landed."""
     rnd = random.Random(seed)
     nsm = 4 * sw
     bars = {"q_full": _Barrier(nsm)}
@@ -125,9 +122,8 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
             yield
 
         def qk(i):
-            if cm != 4 or i < NS:
-                while not passes(("k_full", i % NSK), i // NSK):
-                    yield
+            while not passes(("k_full", i % NSK), i // NSK):
+                yield
             assert ("k", i) in landed, f"QK_{i} issued before K_{i} landed"
             buf = i % NS
             prev = s_owner.get(buf)
@@ -141,9 +137,8 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
         for j in range(ntiles):
             while not passes(("p_full", j % NS), j // NS):
                 yield
-            if cm != 4:
-                while not passes(("v_full", j % NSV), j // NSV):
-                    yield
+            while not passes(("v_full", j % NSV), j // NSV):
+                yield
             assert ("v", j) in landed, f"PV_{j} issued before V_{j} landed"
             commits = [("o_ready", j % NS)] if merged else \
                 [("v_empty", j % NSV), ("o_ready", j % NS)]
@@ -158,7 +153,7 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
         while not passes(("pair", q), n):
             yield
 
-    def softmax(q, first=False):
+    def softmax(q):
         bars["q_full"].arrive()
         yield
         nx = 0
@@ -179,12 +174,6 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
                 while not pv_passed(j - 1):
                     yield
                 assert j - 1 in pv_done
-            if cm == 4 and first:                       # for the MMA thread
-                while not passes(("v_full", j % NSV), j // NSV):
-                    yield
-                if j + NS < ntiles:
-                    while not passes(("k_full", (j + NS) % NSK), (j + NS) // NSK):
-                        yield
             bars["p_full", j % NS].arrive()
             yield
         if ntiles:
@@ -199,8 +188,7 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
             if sw == 2:
                 yield from exchange(q, nx)              # the row sums
 
-    roles = [producer(), mma()] + [softmax(q, first=(q == 0 and h == 0))
-                                   for q in range(4) for h in range(sw)]
+    roles = [producer(), mma()] + [softmax(q) for q in range(4) for _ in range(sw)]
     idle = 0
     while roles or tma or pipe:
         choices = list(range(len(roles))) + (["tma"] if tma else []) + (["pipe"] if pipe else [])
@@ -234,14 +222,6 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
 def test_rows_kernel_protocol(NS, NSK, NSV, sw, ntiles):
     for seed in range(150):
         _run(NS, NSK, NSV, ntiles, seed, sw=sw)
-
-
-@pytest.mark.parametrize("NS,NSK,NSV,sw", [(3, 3, 2, 1), (2, 2, 2, 1), (3, 3, 2, 2)],
-                         ids=["128-key tiles", "64-key tiles", "128-key tiles, paired softmax"])
-@pytest.mark.parametrize("ntiles", [1, 2, 3, 4, 5, 8, 17])
-def test_rows_kernel_protocol_one_mma_wait_per_tile(NS, NSK, NSV, sw, ntiles):
-    for seed in range(150):
-        _run(NS, NSK, NSV, ntiles, seed, sw=sw, cm=4)
 
 
 @pytest.mark.parametrize("ntiles", [1, 3, 6])

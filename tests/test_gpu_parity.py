@@ -160,11 +160,6 @@ FORCED = [
     ("large", {"TSD_ATTN_ROWS_VARIANT": "2"}, "rows64"),
     ("large", {"TSD_ATTN_SOFTMAX_WARPS": "2"}, "rows128x2"),
     ("large", {"TSD_ATTN_SOFTMAX_WARPS": "2", "TSD_ATTN_EXP_FMA": "6"}, "rows128x2"),
-    ("large", {"TSD_ATTN_MMA_WAITS": "1"}, "rows128"),
-    ("large", {"TSD_ATTN_MMA_WAITS": "1", "TSD_ATTN_SOFTMAX_WARPS": "2"}, "rows128x2"),
-    ("large", {"TSD_ATTN_MMA_WAITS": "1", "TSD_ATTN_SOFTMAX_WARPS": "2",
-               "TSD_ATTN_EXP_FMA": "6"}, "rows128x2"),
-    ("small", {"TSD_ATTN_MMA_WAITS": "1"}, "rows64"),
     ("small", {}, "rows64"),
     ("small", {"TSD_ATTN_SMALL_VARIANT": "keysplit"}, "keysplit"),
     ("small", {"TSD_FORCE_PATH": "simt"}, "simt"),
@@ -178,7 +173,6 @@ def _shape_workload(name):
 
 
 FORCED_IDS = [f"{f[0]}-{f[2]}" + ("-expfma" if "TSD_ATTN_EXP_FMA" in f[1] else "")
-              + ("-1wait" if "TSD_ATTN_MMA_WAITS" in f[1] else "")
               for f in FORCED]
 
 
@@ -402,20 +396,6 @@ def test_config_full_size_paired_softmax(cuda_device, cfg, nf, monkeypatch):
     monkeypatch.setenv("TSD_ATTN_SOFTMAX_WARPS", "2")
     monkeypatch.setenv("TSD_ATTN_EXP_FMA", nf)
     test_config_full_size(cuda_device, cfg)
-
-
-@pytest.mark.parametrize("cfg", [1, 2, 3, 4])
-def test_config_full_size_one_mma_wait(cuda_device, cfg, monkeypatch):
-    monkeypatch.setenv("TSD_ATTN_MMA_WAITS", "1")
-    test_config_full_size(cuda_device, cfg)
-
-
-@pytest.mark.parametrize("nf", ["0", "6"])
-def test_config_full_size_paired_softmax_one_mma_wait(cuda_device, nf, monkeypatch):
-    monkeypatch.setenv("TSD_ATTN_MMA_WAITS", "1")
-    monkeypatch.setenv("TSD_ATTN_SOFTMAX_WARPS", "2")
-    monkeypatch.setenv("TSD_ATTN_EXP_FMA", nf)
-    test_config_full_size(cuda_device, 3)
 
 
 @pytest.mark.parametrize("cfg", [0, 1, 2, 3, 4])

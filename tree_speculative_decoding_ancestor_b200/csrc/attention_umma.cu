@@ -882,7 +882,7 @@ __device__ __forceinline__ bool softmax_half_tile(const Setup<Gm> &su, uint32_t 
 template <int SW>
 constexpr int rows_threads() { return 64 + 128 * SW; }
 
-template <class Gm, int NS, int kMinBlocks, int SW, int NF = 0, int CM = 2>
+template <class Gm, int NS, int kMinBlocks, int SW, int NF = 0>
 __global__ void __launch_bounds__(rows_threads<SW>(), kMinBlocks)
     tree_attn_rows_kernel(const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV,
@@ -925,14 +925,11 @@ __global__ void __launch_bounds__(rows_threads<SW>(), kMinBlocks)
         if (lane == 0)
             produce_kv<Gm, NS>(su, &tmK, &tmV, b, hk, Hkv, kb, ntiles, pages, pc, P + T,
                                dev_status);
-    } else if (warp == 1 && CM == 4) {
-        // One mbarrier wait per key tile: each wait on this thread, even on a
-        // completed barrier, leaves the tensor pipe idle for about one MMA.
-        // Lane 0 waits for P_j -- whose last arrival comes from softmax warp
-        // 4 after it has seen V_j and K_{j+NS} land (and zeroed V_j's rows
-        // past the range end) -- and the warp stays converged on its result;
-        // lane 0 then issues PV_j (commit o_ready) and QK_{j+NS} (commit
-        // s_full), as in the three-wait schedule.
+    } else if (warp == 1) {
+        // Every mbarrier wait on the MMA-issuing thread leaves the tensor
+        // pipe idle for a while (it queues little ahead of the thread), so
+        // lane 0 alone waits and the warp stays converged on its result
+        // (a warp-wide wait costs about twice as long).
         auto wait0 = [&](uint32_t bar, uint32_t parity) {
             bool ok = true;
             if (lane == 0)
@@ -940,28 +937,10 @@ __global__ void __launch_bounds__(rows_threads<SW>(), kMinBlocks)
             return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         };
         bool ok = wait0(su.bars.q_full(), 0);
-        for (int i = 0; ok && i < min(NS, ntiles); ++i) {
-            ok = wait0(su.bars.k_full(i % NSK), (i / NSK) & 1);
-            ptx::tc_fence_after();
-            if (ok)
-                issue_qk<Gm, false, true, false>(su, lane, col_s(i), i, su.bars.s_full(i % NS));
-        }
-        for (int j = 0; ok && j < ntiles; ++j) {
-            if (!wait0(su.bars.p_full(j % NS), (j / NS) & 1))
-                break;
-            ptx::tc_fence_after();
-            issue_pv<Gm, false, SW == 2, true, false>(su, lane, col_s(j), kO, j, j > 0, BN,
-                                                      su.bars.o_ready(j % NS));
-            if (j + NS < ntiles)
-                issue_qk<Gm, false, true, false>(su, lane, col_s(j + NS), j + NS,
-                                                 su.bars.s_full((j + NS) % NS));
-        }
-    } else if (warp == 1) {
-        bool ok = warp_wait(su.bars.q_full(), 0, su.abort_flag);
         ptx::tc_fence_after();
         // QK_i commits to s_full[i % NS], PV_j to o_ready[j % NS]
         auto qk = [&](int i) {
-            if (!warp_wait(su.bars.k_full(i % NSK), (i / NSK) & 1, su.abort_flag))
+            if (!wait0(su.bars.k_full(i % NSK), (i / NSK) & 1))
                 return false;
             ptx::tc_fence_after();
             issue_qk<Gm, false>(su, lane, col_s(i), i, su.bars.s_full(i % NS));
@@ -970,8 +949,8 @@ __global__ void __launch_bounds__(rows_threads<SW>(), kMinBlocks)
         for (int i = 0; ok && i < min(NS, ntiles); ++i)
             ok = qk(i);
         for (int j = 0; ok && j < ntiles; ++j) {
-            if (!warp_wait(su.bars.p_full(j % NS), (j / NS) & 1, su.abort_flag) ||
-                !warp_wait(su.bars.v_full(j % NSV), (j / NSV) & 1, su.abort_flag)) {
+            if (!wait0(su.bars.p_full(j % NS), (j / NS) & 1) ||
+                !wait0(su.bars.v_full(j % NSV), (j / NSV) & 1)) {
                 ok = false;
                 break;
             }
@@ -1027,19 +1006,6 @@ __global__ void __launch_bounds__(rows_threads<SW>(), kMinBlocks)
             if (!ok)
                 break;
             ptx::tc_fence_before();
-            if (CM == 4 && warp == 4) {
-                // for the MMA thread: V_j and K_{j+NS} have landed, V_j's rows
-                // past the range end are zero
-                ok = warp_wait(su.bars.v_full(j % NSV), (j / NSV) & 1, su.abort_flag);
-                if (ok && j + NS < ntiles)
-                    ok = warp_wait(su.bars.k_full((j + NS) % NSK), ((j + NS) / NSK) & 1,
-                                   su.abort_flag);
-                if (!ok)
-                    break;
-                const int first_bad = P + T - (kb + j * BN);
-                if (first_bad < BN)
-                    zero_v_rows<Gm>(su, j % NSV, first_bad, lane);
-            }
             warp_arrive(su.bars.p_full(j % NS));
         }
         bool done = ok && wait_pv(ntiles - 1);
@@ -1238,7 +1204,6 @@ struct UmmaPlan {
     bool paired;     // rows kernel with 64-key tiles, two CTAs per SM
     int sw;          // 128-key rows kernel: softmax warps per TMEM lane quarter
     int nf;          // with sw = 2: score pairs of 16 exponentiated on the FMA pipe
-    int cm;          // rows kernels: MMA schedule (2: waits for P, V, K; 4: for P only)
     int nrb, nsplit, keys_per_split;
 };
 
@@ -1249,15 +1214,6 @@ int rows_softmax_warps()
 {
     const char *e = std::getenv("TSD_ATTN_SOFTMAX_WARPS");
     return (e && e[0] == '2' && e[1] == '\0') ? 2 : 1;
-}
-
-// MMA-thread schedule of the rows kernels (TSD_ATTN_MMA_WAITS, read at
-// every launch): 3 -- the MMA warp waits for P, V and K of every tile; "1"
-// -- lane 0 waits for P alone, a softmax warp having checked V and K.
-int rows_mma_waits()
-{
-    const char *e = std::getenv("TSD_ATTN_MMA_WAITS");
-    return (e && e[0] == '1' && e[1] == '\0') ? 1 : 3;
 }
 
 // With two softmax warps per quarter: of every 16 score pairs, how many are
@@ -1300,7 +1256,6 @@ UmmaPlan umma_plan(const AttnArgs &a, int num_sms)
     p.paired = small ? !p.keysplit : rows_variant() == 2;
     p.sw = (p.keysplit || p.paired) ? 1 : rows_softmax_warps();
     p.nf = p.sw == 2 ? rows_exp_fma() : 0;
-    p.cm = (!p.keysplit && rows_mma_waits() == 1) ? 4 : 2;
     p.nrb = p.keysplit ? 1 : (a.Tmax * G + BQ - 1) / BQ;
     const int bn = p.paired ? Half::BN : Wide::BN;
     const int slots = num_sms * (p.paired ? 2 : 1);
@@ -1388,22 +1343,16 @@ cudaError_t set_smem_attributes()
         return cudaErrorInvalidDevice;
     if (done[dev].load())
         return cudaSuccess;
-    const void *wide_kernels[] = {
-        (const void *)tree_attn_rows_kernel<Wide, 3, 1, 1, 0, 2>,
-        (const void *)tree_attn_rows_kernel<Wide, 3, 1, 1, 0, 4>,
-        (const void *)tree_attn_rows_kernel<Wide, 3, 1, 2, 0, 2>,
-        (const void *)tree_attn_rows_kernel<Wide, 3, 1, 2, 0, 4>,
-        (const void *)tree_attn_rows_kernel<Wide, 3, 1, 2, 4, 2>,
-        (const void *)tree_attn_rows_kernel<Wide, 3, 1, 2, 4, 4>,
-        (const void *)tree_attn_rows_kernel<Wide, 3, 1, 2, 6, 2>,
-        (const void *)tree_attn_rows_kernel<Wide, 3, 1, 2, 6, 4>,
-        (const void *)tree_attn_keysplit_kernel};
+    const void *wide_kernels[] = {(const void *)tree_attn_rows_kernel<Wide, 3, 1, 1, 0>,
+                                  (const void *)tree_attn_rows_kernel<Wide, 3, 1, 2, 0>,
+                                  (const void *)tree_attn_rows_kernel<Wide, 3, 1, 2, 4>,
+                                  (const void *)tree_attn_rows_kernel<Wide, 3, 1, 2, 6>,
+                                  (const void *)tree_attn_keysplit_kernel};
     for (const void *k : wide_kernels)
         if (err == cudaSuccess)
             err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)Wide::kSmemBytes);
-    const void *half_kernels[] = {(const void *)tree_attn_rows_kernel<Half, 2, 2, 1, 0, 2>,
-                                  (const void *)tree_attn_rows_kernel<Half, 2, 2, 1, 0, 4>};
+    const void *half_kernels[] = {(const void *)tree_attn_rows_kernel<Half, 2, 2, 1, 0>};
     for (const void *k : half_kernels) {
         if (err == cudaSuccess)
             err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1484,17 +1433,11 @@ int launch_umma_attention(const AttnArgs &a, void *ws, size_t ws_bytes, int num_
             a.Tmax, a.Hq, a.Hkv, a.Lmax, W, sl2, p.keys_per_split, p.nsplit,
             static_cast<__nv_bfloat16 *>(a.out), part_o, part_ml, a.dev_status, a.pages);
     else {
-        const bool c4 = p.cm == 4;
-        auto kern = p.paired    ? (c4 ? tree_attn_rows_kernel<Half, 2, 2, 1, 0, 4>
-                                      : tree_attn_rows_kernel<Half, 2, 2, 1, 0, 2>)
-                  : p.sw == 1   ? (c4 ? tree_attn_rows_kernel<Wide, 3, 1, 1, 0, 4>
-                                      : tree_attn_rows_kernel<Wide, 3, 1, 1, 0, 2>)
-                  : p.nf == 6   ? (c4 ? tree_attn_rows_kernel<Wide, 3, 1, 2, 6, 4>
-                                      : tree_attn_rows_kernel<Wide, 3, 1, 2, 6, 2>)
-                  : p.nf == 4   ? (c4 ? tree_attn_rows_kernel<Wide, 3, 1, 2, 4, 4>
-                                      : tree_attn_rows_kernel<Wide, 3, 1, 2, 4, 2>)
-                                : (c4 ? tree_attn_rows_kernel<Wide, 3, 1, 2, 0, 4>
-                                      : tree_attn_rows_kernel<Wide, 3, 1, 2, 0, 2>);
+        auto kern = p.paired    ? tree_attn_rows_kernel<Half, 2, 2, 1, 0>
+                  : p.sw == 1   ? tree_attn_rows_kernel<Wide, 3, 1, 1, 0>
+                  : p.nf == 6   ? tree_attn_rows_kernel<Wide, 3, 1, 2, 6>
+                  : p.nf == 4   ? tree_attn_rows_kernel<Wide, 3, 1, 2, 4>
+                                : tree_attn_rows_kernel<Wide, 3, 1, 2, 0>;
         const int threads = p.sw == 2 ? rows_threads<2>() : rows_threads<1>();
         const uint32_t smem = p.paired ? Half::kSmemBytes : Wide::kSmemBytes;
         kern<<<grid, threads, smem, stream>>>(
