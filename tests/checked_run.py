@@ -30,7 +30,8 @@ def main():
     st = tsd.device_status(dev)
     kernels = [{}, {"TSD_ATTN_SOFTMAX_WARPS": "2"},
                {"TSD_ATTN_SOFTMAX_WARPS": "2", "TSD_ATTN_EXP_FMA": "6"}, {"TSD_ATTN_ROWS_VARIANT": "2"},
-               {"TSD_ATTN_SMALL_VARIANT": "keysplit"}, {"TSD_FORCE_PATH": "simt"}]
+               {"TSD_ATTN_SMALL_VARIANT": "keysplit"}, {"TSD_FORCE_PATH": "simt"},
+               {"TSD_ATTN_MMA_ORDER": "interleaved", "TSD_ATTN_EXP_FMA": "6"}]
     shapes = [dict(seed=3, B=3, Tmax=24, Hq=16, Hkv=2, D=128, P_max=513),    # 192 rows
               dict(seed=4, B=2, Tmax=20, Hq=8, Hkv=2, D=128, P_max=300),     # 80 rows
               dict(seed=5, B=2, Tmax=9, Hq=4, Hkv=4, D=64, P_max=70, dtype="f32")]

@@ -160,6 +160,11 @@ FORCED = [
     ("large", {"TSD_ATTN_ROWS_VARIANT": "2"}, "rows64"),
     ("large", {"TSD_ATTN_SOFTMAX_WARPS": "2"}, "rows128x2"),
     ("large", {"TSD_ATTN_SOFTMAX_WARPS": "2", "TSD_ATTN_EXP_FMA": "6"}, "rows128x2"),
+    ("large", {"TSD_ATTN_EXP_FMA": "4"}, "rows128"),
+    ("large", {"TSD_ATTN_MMA_ORDER": "interleaved"}, "rows128"),
+    ("large", {"TSD_ATTN_MMA_ORDER": "interleaved", "TSD_ATTN_EXP_FMA": "6"}, "rows128"),
+    ("large", {"TSD_ATTN_MMA_ORDER": "interleaved", "TSD_ATTN_SOFTMAX_WARPS": "2"},
+     "rows128x2"),
     ("small", {}, "rows64"),
     ("small", {"TSD_ATTN_SMALL_VARIANT": "keysplit"}, "keysplit"),
     ("small", {"TSD_FORCE_PATH": "simt"}, "simt"),
@@ -172,8 +177,9 @@ def _shape_workload(name):
                                lmax_pad=37, V=16, **c)
 
 
-FORCED_IDS = [f"{f[0]}-{f[2]}" + ("-expfma" if "TSD_ATTN_EXP_FMA" in f[1] else "")
-              for f in FORCED]
+FORCED_IDS = [f"{f[0]}-{f[2]}" + (f"-expfma{f[1]['TSD_ATTN_EXP_FMA']}"
+                                  if "TSD_ATTN_EXP_FMA" in f[1] else "")
+              + ("-interleaved" if "TSD_ATTN_MMA_ORDER" in f[1] else "") for f in FORCED]
 
 
 @pytest.mark.parametrize("splits", ["1", "3", "64"])
@@ -394,6 +400,14 @@ def _sample_rows(w, n, seed):
 @pytest.mark.parametrize("cfg", [3, 4])
 def test_config_full_size_paired_softmax(cuda_device, cfg, nf, monkeypatch):
     monkeypatch.setenv("TSD_ATTN_SOFTMAX_WARPS", "2")
+    monkeypatch.setenv("TSD_ATTN_EXP_FMA", nf)
+    test_config_full_size(cuda_device, cfg)
+
+
+@pytest.mark.parametrize("nf", ["0", "6"])
+@pytest.mark.parametrize("cfg", [3, 4])
+def test_config_full_size_interleaved_waits(cuda_device, cfg, nf, monkeypatch):
+    monkeypatch.setenv("TSD_ATTN_MMA_ORDER", "interleaved")
     monkeypatch.setenv("TSD_ATTN_EXP_FMA", nf)
     test_config_full_size(cuda_device, cfg)
 
