@@ -28,10 +28,8 @@ def main():
     assert tsd.LIB_PATH.endswith("libtsd_checked.so"), tsd.LIB_PATH
     dev = torch.device("cuda:0")
     st = tsd.device_status(dev)
-    kernels = [{}, {"TSD_ATTN_SOFTMAX_WARPS": "2"},
-               {"TSD_ATTN_SOFTMAX_WARPS": "2", "TSD_ATTN_EXP_FMA": "6"}, {"TSD_ATTN_ROWS_VARIANT": "2"},
-               {"TSD_ATTN_SMALL_VARIANT": "keysplit"}, {"TSD_FORCE_PATH": "simt"},
-               {"TSD_ATTN_MMA_ORDER": "interleaved", "TSD_ATTN_EXP_FMA": "6"}]
+    kernels = [{}, {"TSD_ATTN_SOFTMAX_WARPS": "2"}, {"TSD_ATTN_ROWS_VARIANT": "2"},
+               {"TSD_ATTN_SMALL_VARIANT": "keysplit"}, {"TSD_FORCE_PATH": "simt"}]
     shapes = [dict(seed=3, B=3, Tmax=24, Hq=16, Hkv=2, D=128, P_max=513),    # 192 rows
               dict(seed=4, B=2, Tmax=20, Hq=8, Hkv=2, D=128, P_max=300),     # 80 rows
               dict(seed=5, B=2, Tmax=9, Hq=4, Hkv=4, D=64, P_max=70, dtype="f32")]

@@ -36,7 +36,7 @@ class _Barrier:
 
 
 def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged=True, sw=1,
-         redo_p=0.2, order="plain"):
+         redo_p=0.2):
     """merged: the producer reuses a K slot once s_full of the QK that read it
     completes and a V slot once o_ready of the PV that read it completes (the
     rows kernels; the MMA thread then commits only to s_full and o_ready).
@@ -44,10 +44,7 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
     key tile; per tile they exchange their redo votes and, when either voted,
     their row maxima (then both may rescale O), and at the end their row
     sums -- each exchange a phase of the quarter's pair mbarrier.
-    The MMA model checks that the tiles it reads have landed.
-    order = "interleaved": the MMA thread waits for K_{j+NS} while PV_j is
-    being issued and for P_{j+1}, V_{j+1} while QK_{j+NS} is (the products
-    enter the pipe when their last part is issued)."""
+    The MMA model checks that the tiles it reads have landed."""
     rnd = random.Random(seed)
     nsm = 4 * sw
     bars = {"q_full": _Barrier(nsm)}
@@ -137,36 +134,6 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
             s_owner[buf] = i
         for i in range(min(NS, ntiles)):
             yield from qk(i)
-        if order == "interleaved":
-            if ntiles:
-                while not passes(("p_full", 0), 0):
-                    yield
-                while not passes(("v_full", 0), 0):
-                    yield
-            for j in range(ntiles):
-                assert ("v", j) in landed, f"PV_{j} issued before V_{j} landed"
-                has_qk, has_next = j + NS < ntiles, j + 1 < ntiles
-                if has_qk:
-                    while not passes(("k_full", (j + NS) % NSK), (j + NS) // NSK):
-                        yield
-                pipe.append((("pv", j), [("o_ready", j % NS)]))
-                yield
-                if has_next:
-                    while not passes(("p_full", (j + 1) % NS), (j + 1) // NS):
-                        yield
-                    while not passes(("v_full", (j + 1) % NSV), (j + 1) // NSV):
-                        yield
-                if has_qk:
-                    i = j + NS
-                    assert ("k", i) in landed, f"QK_{i} issued before K_{i} landed"
-                    prev = s_owner.get(i % NS)
-                    assert prev is None or prev in pv_done or \
-                        ("pv", prev) in [p[0] for p in pipe], \
-                        f"QK_{i} issued over the P of tile {prev} before its PV"
-                    pipe.append((("qk", i), [("s_full", i % NS)]))
-                    s_owner[i % NS] = i
-                yield
-            return
         for j in range(ntiles):
             while not passes(("p_full", j % NS), j // NS):
                 yield
@@ -255,14 +222,6 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
 def test_rows_kernel_protocol(NS, NSK, NSV, sw, ntiles):
     for seed in range(150):
         _run(NS, NSK, NSV, ntiles, seed, sw=sw)
-
-
-@pytest.mark.parametrize("NS,NSK,NSV,sw", [(3, 3, 2, 1), (3, 3, 2, 2)],
-                         ids=["128-key tiles", "128-key tiles, paired softmax"])
-@pytest.mark.parametrize("ntiles", [1, 2, 3, 4, 5, 8, 17])
-def test_rows_kernel_protocol_interleaved_waits(NS, NSK, NSV, sw, ntiles):
-    for seed in range(150):
-        _run(NS, NSK, NSV, ntiles, seed, sw=sw, order="interleaved")
 
 
 @pytest.mark.parametrize("ntiles", [1, 3, 6])

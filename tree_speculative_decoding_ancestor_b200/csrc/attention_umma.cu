@@ -445,35 +445,6 @@ __device__ __forceinline__ void issue_pv(const Setup<Gm> &su, int lane, uint32_t
         __syncwarp();
 }
 
-// Lane 0 of the MMA warp: part of a QK or PV product (slices kk0 .. kk1-1 of
-// the 16-wide contraction), no commit.  The interleaved schedule issues a
-// product in parts with a wait in between, so that the tensor pipe has
-// MMAs queued while the thread waits.
-template <class Gm>
-__device__ __forceinline__ void qk_range(const Setup<Gm> &su, uint32_t col_s, int t, int kk0,
-                                         int kk1)
-{
-    constexpr uint32_t idesc = ptx::idesc_bf16(BQ, Gm::BN, false, false);
-    const uint64_t dq = desc_kmajor(su.sQ), dk = desc_kmajor(su.sK + (t % Gm::NSK) * Gm::kTile);
-    for (int kk = kk0; kk < kk1; ++kk)
-        ptx::mma_ss(su.tmem + col_s, dq + slice_off(kk, kSubQ), dk + slice_off(kk, Gm::kSub),
-                    idesc, kk > 0 ? 1u : 0u);
-}
-
-template <class Gm, bool P_SPLIT>
-__device__ __forceinline__ void pv_range(const Setup<Gm> &su, uint32_t col_p, uint32_t col_o,
-                                         int t, bool accumulate, int kk0, int kk1)
-{
-    constexpr uint32_t idesc = ptx::idesc_bf16(BQ, HD, false, true);
-    const uint64_t dv = desc_v(su.sV + (t % Gm::NSV) * Gm::kTile, Gm::kSub);
-    for (int kk = kk0; kk < kk1; ++kk) {
-        const uint32_t pc =
-            P_SPLIT ? (uint32_t)((kk >> 2) * 64 + (kk & 3) * 8) : (uint32_t)(kk * 8);
-        ptx::mma_ts(su.tmem + col_o, su.tmem + col_p + pc, dv + (uint64_t)((kk * 16u * 128u) >> 4),
-                    idesc, (accumulate || kk > 0) ? 1u : 0u);
-    }
-}
-
 // Softmax-warp helpers.  Row state of one query row of a tile.
 struct RowCtx {
     int P, ke;
@@ -550,30 +521,6 @@ __device__ __forceinline__ float exp_pack32(const uint32_t (&sa)[32], float scal
         ptx::fma2_bc(x0, x1, __uint_as_float(sa[2 * k]), __uint_as_float(sa[2 * k + 1]),
                      scale_log2, neg_m);
         const float p0 = ptx::ex2(x0), p1 = ptx::ex2(x1);
-        const int a = (k & 1) * 2;
-        ptx::add2(acc[a], acc[a + 1], p0, p1);
-        pk[k] = ptx::pack_bf16(p0, p1);
-    }
-    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
-}
-
-// exp_pack32 with NF of its 16 score pairs (spread evenly) exponentiated on
-// the FMA pipe (ptx::exp2_fma) and the rest on MUFU: with two softmax warps
-// per sub-partition the MUFU unit, not issue, bounds the exponentials, and
-// the FMA pipe has room for part of them.
-template <int NF>
-__device__ __forceinline__ float exp_pack32_mix(const uint32_t (&sa)[32], float scale_log2,
-                                                float neg_m, uint32_t (&pk)[16])
-{
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-        float x0, x1;
-        ptx::fma2_bc(x0, x1, __uint_as_float(sa[2 * k]), __uint_as_float(sa[2 * k + 1]),
-                     scale_log2, neg_m);
-        const bool poly = (k * NF) % 16 < NF;
-        const float p0 = poly ? ptx::exp2_fma(x0) : ptx::ex2(x0);
-        const float p1 = poly ? ptx::exp2_fma(x1) : ptx::ex2(x1);
         const int a = (k & 1) * 2;
         ptx::add2(acc[a], acc[a + 1], p0, p1);
         pk[k] = ptx::pack_bf16(p0, p1);
@@ -675,7 +622,7 @@ __device__ __forceinline__ bool softmax_tile(uint32_t taddr_s, uint32_t taddr_o,
 // key tile (m_run = -inf).  One exp loop, run a second time only by a warp
 // that took the max.  `wait_prev` waits for the previous PV product before
 // O is rescaled.  Returns false on abort.
-template <int BN, int NF, typename WaitPrev>
+template <int BN, typename WaitPrev>
 __device__ __forceinline__ bool softmax_rows_tile(uint32_t taddr_s, uint32_t taddr_o, int pos0,
                                                   int P, int ke, const uint32_t (&mw)[4],
                                                   float scale_log2, bool first, float &m_run,
@@ -700,7 +647,7 @@ __device__ __forceinline__ bool softmax_rows_tile(uint32_t taddr_s, uint32_t tad
 #pragma unroll
         for (int c = 0; c < NC; ++c) {
             uint32_t pk[16];
-            lsum += exp_pack32_mix<NF>(sr[c], scale_log2, neg_m, pk);
+            lsum += exp_pack32(sr[c], scale_log2, neg_m, pk);
             ptx::tmem_st16(taddr_s + c * 16, pk);
         }
         const bool redo = !(lsum <= kLazyLimit) || m_run == -INFINITY;
@@ -805,7 +752,7 @@ __device__ __forceinline__ bool pair_exchange(const Setup<Gm> &su, int quarter, 
     return ok;
 }
 
-template <class Gm, int NF, typename WaitPrev>
+template <class Gm, typename WaitPrev>
 __device__ __forceinline__ bool softmax_half_tile(const Setup<Gm> &su, uint32_t taddr_s,
                                                   uint32_t taddr_o, int pos0, int P, int ke,
                                                   const uint32_t (&mw)[4], float scale_log2,
@@ -830,7 +777,7 @@ __device__ __forceinline__ bool softmax_half_tile(const Setup<Gm> &su, uint32_t 
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
             uint32_t pk[16];
-            lsum += exp_pack32_mix<NF>(sr[c], scale_log2, neg_m, pk);
+            lsum += exp_pack32(sr[c], scale_log2, neg_m, pk);
             ptx::tmem_st16(taddr_s + c * 16, pk);
         }
         if (pass == 1)
@@ -911,7 +858,7 @@ __device__ __forceinline__ bool softmax_half_tile(const Setup<Gm> &su, uint32_t 
 template <int SW>
 constexpr int rows_threads() { return 64 + 128 * SW; }
 
-template <class Gm, int NS, int kMinBlocks, int SW, int NF = 0, bool IL = false>
+template <class Gm, int NS, int kMinBlocks, int SW>
 __global__ void __launch_bounds__(rows_threads<SW>(), kMinBlocks)
     tree_attn_rows_kernel(const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV,
@@ -954,60 +901,6 @@ __global__ void __launch_bounds__(rows_threads<SW>(), kMinBlocks)
         if (lane == 0)
             produce_kv<Gm, NS>(su, &tmK, &tmV, b, hk, Hkv, kb, ntiles, pages, pc, P + T,
                                dev_status);
-    } else if (warp == 1 && IL) {
-        // Interleaved schedule: each wait sits between two parts of a product
-        // already being issued, so the tensor pipe has MMAs queued while the
-        // thread polls.  Per tile j: PV_j[0..5], wait K_{j+NS}, PV_j[6..7]
-        // (commit o_ready), QK_{j+NS}[0..3], wait P_{j+1}, QK_{j+NS}[4..5],
-        // wait V_{j+1}, QK_{j+NS}[6..7] (commit s_full).  The same barriers,
-        // phases and commits as the plain schedule; only the order in which
-        // this thread waits and issues differs.
-        bool ok = warp_wait(su.bars.q_full(), 0, su.abort_flag);
-        for (int i = 0; ok && i < min(NS, ntiles); ++i) {
-            ok = warp_wait(su.bars.k_full(i % NSK), (i / NSK) & 1, su.abort_flag);
-            ptx::tc_fence_after();
-            if (ok && lane == 0) {
-                qk_range<Gm>(su, col_s(i), i, 0, HD / 16);
-                ptx::mma_commit(su.bars.s_full(i % NS));
-            }
-            __syncwarp();
-        }
-        ok = ok && warp_wait(su.bars.p_full(0), 0, su.abort_flag) &&
-             warp_wait(su.bars.v_full(0), 0, su.abort_flag);
-        for (int j = 0; ok && j < ntiles; ++j) {
-            const int first_bad = P + T - (kb + j * BN);
-            if (first_bad < BN)
-                zero_v_rows<Gm>(su, j % NSV, first_bad, lane);
-            ptx::tc_fence_after();
-            const bool has_qk = j + NS < ntiles, has_next = j + 1 < ntiles;
-            constexpr int KP = BN / 16;   // PV slices
-            if (lane == 0)
-                pv_range<Gm, SW == 2>(su, col_s(j), kO, j, j > 0, 0, KP - 2);
-            if (has_qk)
-                ok = warp_wait(su.bars.k_full((j + NS) % NSK), ((j + NS) / NSK) & 1,
-                               su.abort_flag);
-            if (lane == 0) {
-                pv_range<Gm, SW == 2>(su, col_s(j), kO, j, j > 0, KP - 2, KP);
-                ptx::mma_commit(su.bars.o_ready(j % NS));
-            }
-            if (!ok)
-                break;
-            ptx::tc_fence_after();
-            if (has_qk && lane == 0)
-                qk_range<Gm>(su, col_s(j + NS), j + NS, 0, 4);
-            if (has_next)
-                ok = warp_wait(su.bars.p_full((j + 1) % NS), ((j + 1) / NS) & 1, su.abort_flag);
-            if (has_qk && lane == 0)
-                qk_range<Gm>(su, col_s(j + NS), j + NS, 4, 6);
-            if (has_next && ok)
-                ok = warp_wait(su.bars.v_full((j + 1) % NSV), ((j + 1) / NSV) & 1,
-                               su.abort_flag);
-            if (has_qk && lane == 0) {
-                qk_range<Gm>(su, col_s(j + NS), j + NS, 6, HD / 16);
-                ptx::mma_commit(su.bars.s_full((j + NS) % NS));
-            }
-            __syncwarp();
-        }
     } else if (warp == 1) {
         // Every mbarrier wait on the MMA-issuing thread leaves the tensor
         // pipe idle for a while (it queues little ahead of the thread).  The
@@ -1076,11 +969,11 @@ __global__ void __launch_bounds__(rows_threads<SW>(), kMinBlocks)
             ptx::tc_fence_after();
             auto wait_prev = [&]() { return wait_pv(j - 1); };
             if (SW == 1)
-                ok = softmax_rows_tile<BN, NF>(su.tmem + lane_off + col_s(j), taddr_o, kb + j * BN,
+                ok = softmax_rows_tile<BN>(su.tmem + lane_off + col_s(j), taddr_o, kb + j * BN,
                                            P, ke, mw, scale_log2, j == 0, m_run, l_run,
                                            wait_prev);
             else
-                ok = softmax_half_tile<Gm, NF>(su, su.tmem + lane_off + col_s(j) + hf * 64, taddr_o,
+                ok = softmax_half_tile<Gm>(su, su.tmem + lane_off + col_s(j) + hf * 64, taddr_o,
                                        kb + j * BN + hf * 64, P, ke, mw, scale_log2, j == 0, hf,
                                        quarter, xc, nx, m_run, l_run, wait_prev);
             if (!ok)
@@ -1283,8 +1176,6 @@ struct UmmaPlan {
     bool keysplit;   // at most 128 packed rows
     bool paired;     // rows kernel with 64-key tiles, two CTAs per SM
     int sw;          // 128-key rows kernel: softmax warps per TMEM lane quarter
-    int nf;          // score pairs of 16 exponentiated on the FMA pipe (128-key rows kernel)
-    bool il;         // 128-key rows kernel: interleaved MMA-warp waits
     int nrb, nsplit, keys_per_split;
 };
 
@@ -1297,23 +1188,6 @@ int rows_softmax_warps()
     return (e && e[0] == '2' && e[1] == '\0') ? 2 : 1;
 }
 
-// Order of the MMA warp's waits (TSD_ATTN_MMA_ORDER, read at every launch):
-// "interleaved" places each wait between parts of a product being issued.
-bool rows_interleaved()
-{
-    const char *e = std::getenv("TSD_ATTN_MMA_ORDER");
-    return e && std::strcmp(e, "interleaved") == 0;
-}
-
-// Of every 16 score pairs, how many are
-// exponentiated on the FMA pipe (0, 4 or 6; TSD_ATTN_EXP_FMA, read at every
-// launch).
-int rows_exp_fma()
-{
-    const char *e = std::getenv("TSD_ATTN_EXP_FMA");
-    const int n = e ? std::atoi(e) : 0;
-    return (n == 4 || n == 6) ? n : 0;
-}
 
 // Rows-kernel instance for more than 128 packed rows: 1 = 128-key tiles at
 // one CTA per SM (default), 2 = 64-key tiles at two CTAs per SM when the
@@ -1344,8 +1218,6 @@ UmmaPlan umma_plan(const AttnArgs &a, int num_sms)
     p.keysplit = small && !small_paired();
     p.paired = small ? !p.keysplit : rows_variant() == 2;
     p.sw = (p.keysplit || p.paired) ? 1 : rows_softmax_warps();
-    p.nf = (p.keysplit || p.paired) ? 0 : rows_exp_fma();
-    p.il = !(p.keysplit || p.paired) && rows_interleaved();
     p.nrb = p.keysplit ? 1 : (a.Tmax * G + BQ - 1) / BQ;
     const int bn = p.paired ? Half::BN : Wide::BN;
     const int slots = num_sms * (p.paired ? 2 : 1);
@@ -1419,22 +1291,6 @@ bool make_kv_map(CUtensorMap *m, const void *ptr, int rows, int planes, int box_
     return r == CUDA_SUCCESS;
 }
 
-// The 128-key rows kernel's instances: softmax warps per quarter (1, 2) x
-// FMA-pipe exponentials (0, 4, 6 of 16 pairs) x MMA-warp wait order.
-using WideKernel = decltype(&tree_attn_rows_kernel<Wide, 3, 1, 1, 0, false>);
-template <int SW, bool IL>
-WideKernel wide_by_nf(int nf)
-{
-    return nf == 6 ? tree_attn_rows_kernel<Wide, 3, 1, SW, 6, IL>
-         : nf == 4 ? tree_attn_rows_kernel<Wide, 3, 1, SW, 4, IL>
-                   : tree_attn_rows_kernel<Wide, 3, 1, SW, 0, IL>;
-}
-WideKernel wide_instance(int sw, int nf, bool il)
-{
-    return sw == 2 ? (il ? wide_by_nf<2, true>(nf) : wide_by_nf<2, false>(nf))
-                   : (il ? wide_by_nf<1, true>(nf) : wide_by_nf<1, false>(nf));
-}
-
 // The kernels' shared-memory limits are attributes of the current device's
 // copy of each kernel: raised once per device (a process may drive several).
 cudaError_t set_smem_attributes()
@@ -1449,18 +1305,14 @@ cudaError_t set_smem_attributes()
         return cudaErrorInvalidDevice;
     if (done[dev].load())
         return cudaSuccess;
-    const void *wide_kernels[13];
-    int nk = 0;
-    for (int sw : {1, 2})
-        for (int nf : {0, 4, 6})
-            for (bool il : {false, true})
-                wide_kernels[nk++] = (const void *)wide_instance(sw, nf, il);
-    wide_kernels[nk++] = (const void *)tree_attn_keysplit_kernel;
+    const void *wide_kernels[] = {(const void *)tree_attn_rows_kernel<Wide, 3, 1, 1>,
+                                  (const void *)tree_attn_rows_kernel<Wide, 3, 1, 2>,
+                                  (const void *)tree_attn_keysplit_kernel};
     for (const void *k : wide_kernels)
         if (err == cudaSuccess)
             err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)Wide::kSmemBytes);
-    const void *half_kernels[] = {(const void *)tree_attn_rows_kernel<Half, 2, 2, 1, 0>};
+    const void *half_kernels[] = {(const void *)tree_attn_rows_kernel<Half, 2, 2, 1>};
     for (const void *k : half_kernels) {
         if (err == cudaSuccess)
             err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1541,8 +1393,9 @@ int launch_umma_attention(const AttnArgs &a, void *ws, size_t ws_bytes, int num_
             a.Tmax, a.Hq, a.Hkv, a.Lmax, W, sl2, p.keys_per_split, p.nsplit,
             static_cast<__nv_bfloat16 *>(a.out), part_o, part_ml, a.dev_status, a.pages);
     else {
-        auto kern = p.paired ? tree_attn_rows_kernel<Half, 2, 2, 1, 0>
-                    : wide_instance(p.sw, p.nf, p.il);
+        auto kern = p.paired    ? tree_attn_rows_kernel<Half, 2, 2, 1>
+                    : p.sw == 2 ? tree_attn_rows_kernel<Wide, 3, 1, 2>
+                                : tree_attn_rows_kernel<Wide, 3, 1, 1>;
         const int threads = p.sw == 2 ? rows_threads<2>() : rows_threads<1>();
         const uint32_t smem = p.paired ? Half::kSmemBytes : Wide::kSmemBytes;
         kern<<<grid, threads, smem, stream>>>(

@@ -224,28 +224,6 @@ __device__ __forceinline__ float ex2(float x)
     return y;
 }
 
-// 2^x on the FMA/ALU pipes, so that part of the softmax's exponentials can
-// run beside the MUFU unit instead of queueing for it.  Cody-Waite style
-// split x = j + f with j the nearest integer (adding 1.5 * 2^23 rounds x to
-// an integer and leaves j in the low bits of t) and f in [-1/2, 1/2]; 2^f
-// from a degree-3 polynomial whose coefficients were fitted for minimum
-// relative error on [-1/2, 1/2] (Lawson's iteratively reweighted least
-// squares): max relative error 7.5e-5, far below the bf16 rounding (2^-9)
-// the softmax weights go through.  j is added to the exponent field with one
-// integer multiply-add.  Returns 0 for x < -125 (and for -inf): as a softmax
-// weight next to a row maximum of 1 that is 0 in bf16 anyway.
-__device__ __forceinline__ float exp2_fma(float x)
-{
-    constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
-    const float t = x + kRound;
-    const float f = x - (t - kRound);
-    float p = fmaf(0x1.c3f6e2p-5f, f, 0x1.f0ddf0p-3f);
-    p = fmaf(p, f, 0x1.62f31ap-1f);
-    p = fmaf(p, f, 0x1.fff694p-1f);
-    const int bits = __float_as_int(t) * (1 << 23) + __float_as_int(p);
-    return x < -125.0f ? 0.0f : __int_as_float(bits);
-}
-
 // Packed fp32 pairs (sm_100): (d0, d1) = (a0, a1) * b + c, b and c broadcast.
 __device__ __forceinline__ void fma2_bc(float &d0, float &d1, float a0, float a1, float b, float c)
 {
