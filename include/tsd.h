@@ -380,8 +380,12 @@ int tsd_kv_commit(void *k_cache, void *v_cache, const int32_t *prefix_len,
  *   kind 0  the mbarrier wait of the tensor-core attention kernels, on an
  *           mbarrier nobody arrives on;
  *   kind 1  the team barrier of the stochastic walk, on a counter whose
- *           target one CTA cannot reach.
- *   limit_ns  in [1 ms, 2 s]; scratch: 8 bytes of device memory (8-aligned).
+ *           target one CTA cannot reach;
+ *   kind 2  the cluster exchange of the stochastic walk (thread-block
+ *           cluster teams), in a cluster of two CTAs of which one never
+ *           takes part.
+ *   limit_ns  in [1 ms, 2 s]; scratch: 8 bytes of device memory (8-aligned;
+ *           unused by kind 2).
  * Expected result: the kernel ends after about limit_ns with TSD_DEV_TIMEOUT
  * set in *dev_status.  Host errors: TSD_ERR_SHAPE, TSD_ERR_NULL,
  * TSD_ERR_ALIGN, TSD_ERR_CUDA.

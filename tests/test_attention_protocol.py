@@ -73,6 +73,13 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
         assert b.done == k + 1, f"wait on {name} for phase {k} passed at {b.done} completions"
         return True
 
+    def test(name, k):
+        """A non-blocking test of phase k, issued ahead of the wait that
+        reads it: the phase before k must be complete (else a stale phase
+        would pass), and the result stands until it is read."""
+        assert bars[name].done >= k, f"early test of {name} phase {k} at {bars[name].done}"
+        return passes(name, k)
+
     tma, pipe = [], []
     landed = set()    # ("k" | "v", tile) whose copy has completed
     s_owner = {}       # S buffer -> tile whose scores/P it holds
@@ -87,8 +94,10 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
     qk_done, pv_done_set = set(), set()
 
     def producer():
-        for i in range(ntiles + 1):
-            if i < ntiles:
+        # K_0 .. K_{NSK-1}, V_0 .. V_{NSV-1}, then K runs NSK tiles ahead of V
+        i = j = 0
+        while i < ntiles or j < ntiles:
+            if i < ntiles and (j >= ntiles or i < NSK or (j >= NSV and i <= j + NSK)):
                 s = i % NSK
                 if i >= NSK:
                     if merged:   # QK_{i-NSK} done: s_full[i % NS], NS == NSK
@@ -101,8 +110,8 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
                     assert k_read[s] in qk_done, f"K slot {s} reloaded before its QK ran"
                 k_read[s] = i
                 tma.append((("k_full", s), ("k", i)))
-            if i >= 1:
-                j = i - 1
+                i += 1
+            else:
                 s = j % NSV
                 if j >= NSV:
                     if merged:   # PV_{j-NSV} done: o_ready[(j - NSV) % NS]
@@ -115,15 +124,17 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
                     assert v_read[s] in pv_done, f"V slot {s} reloaded before its PV ran"
                 v_read[s] = j
                 tma.append((("v_full", s), ("v", j)))
+                j += 1
             yield
 
     def mma():
         while not passes("q_full", 0):
             yield
 
-        def qk(i):
-            while not passes(("k_full", i % NSK), i // NSK):
-                yield
+        def qk(i, tested=False):
+            if not tested:
+                while not passes(("k_full", i % NSK), i // NSK):
+                    yield
             assert ("k", i) in landed, f"QK_{i} issued before K_{i} landed"
             buf = i % NS
             prev = s_owner.get(buf)
@@ -134,17 +145,30 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
             s_owner[buf] = i
         for i in range(min(NS, ntiles)):
             yield from qk(i)
+        # V_{j+1} and K_{j+NS} are tested while the products before them are
+        # issued, and waited for only when the test failed
+        v_t = test(("v_full", 0), 0) if ntiles else True
         for j in range(ntiles):
             while not passes(("p_full", j % NS), j // NS):
                 yield
-            while not passes(("v_full", j % NSV), j // NSV):
-                yield
+            if not v_t:
+                while not passes(("v_full", j % NSV), j // NSV):
+                    yield
             assert ("v", j) in landed, f"PV_{j} issued before V_{j} landed"
+            i = j + NS
+            k_t = test(("k_full", i % NSK), i // NSK) if i < ntiles else True
+            yield
             commits = [("o_ready", j % NS)] if merged else \
                 [("v_empty", j % NSV), ("o_ready", j % NS)]
             pipe.append((("pv", j), commits))
-            if j + NS < ntiles:
-                yield from qk(j + NS)
+            yield
+            if i < ntiles and not k_t:
+                while not passes(("k_full", i % NSK), i // NSK):
+                    yield
+            v_t = test(("v_full", (j + 1) % NSV), (j + 1) // NSV) if j + 1 < ntiles else True
+            yield
+            if i < ntiles:
+                yield from qk(i, tested=True)
             yield
 
     def exchange(q, n):
@@ -157,9 +181,12 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
         bars["q_full"].arrive()
         yield
         nx = 0
+        s_t = test(("s_full", 0), 0) if ntiles else True
         for j in range(ntiles):
-            while not passes(("s_full", j % NS), j // NS):
-                yield
+            if not s_t:
+                while not passes(("s_full", j % NS), j // NS):
+                    yield
+            s_t = test(("s_full", (j + 1) % NS), (j + 1) // NS) if j + 1 < ntiles else True
             yield
             if sw == 1:
                 rescale = j > 0 and rnd.random() < rescale_p
@@ -266,21 +293,23 @@ def _run_keysplit(NSK, NSV, ntiles, seed, rescale_p=0.3):
 
     tma, pipe, pv_done, issued_pv = [], [], set(), set()
 
-    def producer():
-        for i in range(ntiles + 1):
-            if i < ntiles:
+    def producer():   # the rows kernels' load order
+        i = j = 0
+        while i < ntiles or j < ntiles:
+            if i < ntiles and (j >= ntiles or i < NSK or (j >= NSV and i <= j + NSK)):
                 s = i % NSK
                 if i >= NSK:
                     while not passes(("k_empty", s), i // NSK - 1):
                         yield
                 tma.append(("k_full", s))
-            if i >= 1:
-                j = i - 1
+                i += 1
+            else:
                 s = j % NSV
                 if j >= NSV:
                     while not passes(("v_empty", s), j // NSV - 1):
                         yield
                 tma.append(("v_full", s))
+                j += 1
             yield
 
     def mma():

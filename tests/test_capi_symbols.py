@@ -133,7 +133,7 @@ def test_host_checks_of_every_entry_point(lib):
     assert merge(ct=None) == ERR_NULL
 
     probe = lib.tsd_debug_wait_probe
-    assert probe(2, 50_000_000, _A, _A, None) == ERR_SHAPE       # unknown kind
+    assert probe(3, 50_000_000, _A, _A, None) == ERR_SHAPE       # unknown kind
     assert probe(0, 10, _A, _A, None) == ERR_SHAPE               # below 1 ms
     assert probe(1, 3_000_000_000, _A, _A, None) == ERR_SHAPE    # above 2 s
     assert probe(0, 50_000_000, None, _A, None) == ERR_NULL

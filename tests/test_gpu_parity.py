@@ -300,9 +300,16 @@ VERIFY_CASES = [
 ]
 
 
+@pytest.mark.parametrize("exchange", ["cluster", "global"])
 @pytest.mark.parametrize("case", VERIFY_CASES, ids=[f"s{c[0]}" for c in VERIFY_CASES])
-def test_verify_parity(cuda_device, case):
+def test_verify_parity(cuda_device, case, exchange, monkeypatch):
+    # exchange: the walk's teams as thread-block clusters (the default up to
+    # 8 x 4096 vocabulary entries) or as CTAs of a cooperative launch
     seed, B, Tmax, V, mode, temp = case
+    if exchange == "global":
+        monkeypatch.setenv("TSD_WALK_EXCHANGE", "global")
+    elif V > 8 * 4096:
+        pytest.skip("the cluster form takes vocabularies up to 32768")
     if seed == 39:   # one-CTA teams that each walk several sequences
         assert tsd.verify_stochastic_plan(B, Tmax, V)["teams"] < B
     w = gen.random_workload(seed, B=B, Tmax=Tmax, V=V, min_nodes=0, max_children=5,
@@ -331,8 +338,11 @@ def test_verify_parity(cuda_device, case):
     assert _status(cuda_device) == 0
 
 
-def test_verify_many_seeds_stochastic(cuda_device):
+@pytest.mark.parametrize("exchange", ["cluster", "global"])
+def test_verify_many_seeds_stochastic(cuda_device, exchange, monkeypatch):
     # many small trees with accepted paths of every length; counts excusals
+    if exchange == "global":
+        monkeypatch.setenv("TSD_WALK_EXCHANGE", "global")
     total = dict(mismatches=0, excused=0, decisions=0)
     for seed in range(40, 52):
         w = gen.random_workload(seed, B=64, Tmax=12, V=64, min_nodes=0, max_children=4,

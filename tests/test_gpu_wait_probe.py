@@ -2,9 +2,9 @@
 
 Every wait in the kernels gives up after a time limit, sets TSD_DEV_TIMEOUT and
 returns.  The probe runs the same wait routines -- the attention kernels'
-mbarrier wait and the stochastic walk's team barrier -- on something nothing
-ever signals, with a 50 ms limit; the kernel must end on its own with the
-status set, and the context must stay usable afterwards.
+mbarrier wait, the stochastic walk's team barrier and its cluster exchange --
+on something nothing ever signals, with a 50 ms limit; the kernel must end on
+its own with the status set, and the context must stay usable afterwards.
 """
 
 import time
@@ -20,7 +20,7 @@ from workloads import gen
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("kind", [0, 1])
+@pytest.mark.parametrize("kind", [0, 1, 2])
 def test_bounded_wait_ends_with_timeout_status(cuda_device, kind):
     st = torch.zeros(1, dtype=torch.int32, device=cuda_device)
     torch.cuda.synchronize(cuda_device)
@@ -52,6 +52,6 @@ def test_probe_host_checks(cuda_device):
     lib = tsd.load_library()
     z = torch.zeros(2, dtype=torch.int32, device=cuda_device)
     s = torch.cuda.current_stream().cuda_stream
-    assert lib.tsd_debug_wait_probe(2, 50_000_000, z.data_ptr(), z.data_ptr(), s) == -2
+    assert lib.tsd_debug_wait_probe(3, 50_000_000, z.data_ptr(), z.data_ptr(), s) == -2
     assert lib.tsd_debug_wait_probe(0, 10, z.data_ptr(), z.data_ptr(), s) == -2      # < 1 ms
     assert lib.tsd_debug_wait_probe(0, 50_000_000, None, z.data_ptr(), s) == -1

@@ -14,7 +14,9 @@ again two barriers later, and only by a CTA that has passed barrier n + 1,
 which every CTA reaches after reading barrier n's slots. This test replays
 the exchange under random interleavings: every read must see the value
 written for its own barrier, and every wait must end. A one-buffer layout
-is the negative control.
+is the negative control. The cluster form of the same exchange (partials
+stored into every peer's shared memory, one mbarrier per buffer in every
+CTA) is replayed the same way.
 """
 
 import random
@@ -66,3 +68,62 @@ def test_one_slot_buffer_would_race():
     with pytest.raises(AssertionError):
         for seed in range(200):
             _run(4, 6, seed, buffers=1)
+
+
+def _run_cluster(K, nbar, seed, buffers=2):
+    """The cluster form (`csrc/cluster_xchg.cuh`): every CTA holds its own
+    slots[buffers][K] and mbarriers bar[buffers] (K arrivals per phase).  At
+    exchange n CTA k stores its partial into slot [n % buffers][k] of every
+    CTA and arrives on every CTA's bar[n % buffers]; then it waits on its own
+    barrier for phase n // buffers (by parity) and reads its own K slots."""
+    rnd = random.Random(seed)
+    slots = [[[None] * K for _ in range(buffers)] for _ in range(K)]   # [cta][buf][k]
+    done = [[0] * buffers for _ in range(K)]        # completed phases per barrier
+    pending = [[0] * buffers for _ in range(K)]     # arrivals in the open phase
+
+    def arrive(t, buf):
+        pending[t][buf] += 1
+        if pending[t][buf] == K:
+            pending[t][buf] = 0
+            done[t][buf] += 1
+
+    def cta(k):
+        for n in range(nbar):
+            buf = n % buffers
+            phase = n // buffers
+            for t in rnd.sample(range(K), K):          # threads 0..K-1, any order
+                slots[t][buf][k] = (n, k)              # remote store, then
+                arrive(t, buf)                         # remote release-arrive
+                yield
+            while (done[k][buf] & 1) == (phase & 1):   # parity wait (acquire)
+                yield
+            assert done[k][buf] == phase + 1, \
+                f"CTA {k} passed exchange {n} at {done[k][buf]} completions"
+            for j in range(K):
+                assert slots[k][buf][j] == (n, j), \
+                    f"CTA {k} at exchange {n} read {slots[k][buf][j]} from slot {j}"
+                if rnd.random() < 0.3:
+                    yield
+
+    ctas = [cta(k) for k in range(K)]
+    idle = 0
+    while ctas:
+        i = rnd.randrange(len(ctas))
+        try:
+            next(ctas[i])
+        except StopIteration:
+            ctas.pop(i)
+        idle += 1
+        assert idle < 200_000, "a cluster exchange never completes"
+
+
+@pytest.mark.parametrize("K", [1, 2, 5, 8, 16])
+def test_cluster_slots_are_read_before_they_are_reused(K):
+    for seed in range(60):
+        _run_cluster(K, 9, seed)
+
+
+def test_cluster_one_slot_buffer_would_race():
+    with pytest.raises(AssertionError):
+        for seed in range(200):
+            _run_cluster(4, 6, seed, buffers=1)

@@ -562,8 +562,9 @@ def tree_merge_chains(chain_tokens: torch.Tensor, chain_q_row: torch.Tensor,
 def debug_wait_probe(kind: int, limit_ns: int = 50_000_000, device=None,
                      status: Optional[torch.Tensor] = None) -> None:
     """Run the kernels' bounded wait routines on something that never completes
-    (kind 0: mbarrier wait; kind 1: team barrier); they must end after about
-    limit_ns with DEV_TIMEOUT set in the status word."""
+    (kind 0: mbarrier wait; kind 1: team barrier; kind 2: cluster exchange);
+    they must end after about limit_ns with DEV_TIMEOUT set in the status
+    word."""
     lib = load_library()
     dev = torch.device(device or torch.cuda.current_device())
     _cuda(dev)

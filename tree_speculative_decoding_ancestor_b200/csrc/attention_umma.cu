@@ -128,6 +128,18 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
     return __all_sync(0xffffffffu, ok);
 }
 
+// warp_wait for a phase that this warp already tested with ptx::mbar_test
+// (`tested`, this lane's result) while it did other work: when every lane
+// saw the phase complete the wait costs one vote.  The test must have been
+// issued after the phase before it completed (else a stale phase passes).
+__device__ __forceinline__ bool warp_wait_tested(uint32_t tested, uint32_t bar, uint32_t parity,
+                                                 volatile int *abort)
+{
+    if (__all_sync(0xffffffffu, tested != 0u))
+        return true;
+    return warp_wait(bar, parity, abort);
+}
+
 // One arrival per warp: the lanes' prior writes (TMEM stores after their
 // wait::st and fence, or shared-memory stores after their proxy fence) are
 // ordered before lane 0's arrival by the warp barrier.
@@ -319,15 +331,24 @@ __device__ __forceinline__ void load_kv_tile(uint32_t dst, const CUtensorMap *tm
     }
 }
 
-// TMA producer (one lane): K_0, K_1, V_0, K_2, V_1, ... -- the order in which
-// the MMA warp first needs them.  A ring slot is reused once the product that
-// read it is complete.  NS_PROD = 0: the MMA warp commits every product to
-// the rings' own empty barriers as well.  NS_PROD = NS (the number of score
-// buffers, equal to the K ring's depth): the producer waits on the products'
-// own barriers instead -- QK_{i-NSK} completes on s_full[i % NS], PV_{j-NSV}
-// on o_ready[(j - NSV) % NS] -- which saves the MMA thread two commits per
-// tile.  Either wait names a phase that cannot be stale or ahead: the phase
-// after it needs K_i (or V_{j+1}), which this producer has not loaded yet.
+// TMA producer (one lane).  Load order: K_0 .. K_{NSK-1} and V_0 .. V_{NSV-1}
+// into the empty rings, then K runs NSK tiles ahead of V: ... V_m, K_{m+NSK+1},
+// V_{m+1}, ...  A ring slot is reused once the product that read it is
+// complete; with the MMA order QK_{j+NS} right after PV_j, the V slot of V_m
+// and the K slot of K_{m+NSK+1} free up together (PV_{m-NSV}, then the QK
+// issued after it), so each reload is issued as soon as its slot is free and
+// a K tile has about NSK tile periods to land instead of one (a K ring that
+// only advanced after each V reload waited on the V ring).  Deadlock-free:
+// the product a K wait needs reads V tiles below m only, and the one a V wait
+// needs reads K tiles below the K index already issued.  NS_PROD = 0: the
+// MMA warp commits every product to the rings' own empty barriers as well.
+// NS_PROD = NS (the number of score buffers, equal to the K ring's depth):
+// the producer waits on the products' own barriers instead -- QK_{i-NSK}
+// completes on s_full[i % NS], PV_{j-NSV} on o_ready[(j - NSV) % NS] --
+// which saves the MMA thread two commits per tile.  Either wait names a phase
+// that cannot be stale or ahead: the phase before it was waited for by the
+// previous reload of the same ring slot, and the phase after it needs K_i
+// (or V_{j+1}), which this producer has not loaded yet.
 template <class Gm, int NS_PROD>
 __device__ __forceinline__ void produce_kv(const Setup<Gm> &su, const CUtensorMap *tmK,
                                            const CUtensorMap *tmV, int b, int hk, int Hkv,
@@ -340,8 +361,11 @@ __device__ __forceinline__ void produce_kv(const Setup<Gm> &su, const CUtensorMa
     static_assert(NS_PROD == 0 || NS_PROD == NSK, "score buffers and K ring in step");
     ptx::prefetch_tmap(tmK);
     ptx::prefetch_tmap(tmV);
-    for (int i = 0; i <= ntiles; ++i) {
-        if (i < ntiles) {
+    int i = 0, j = 0;   // next K tile, next V tile
+    while (i < ntiles || j < ntiles) {
+        const bool take_k =
+            i < ntiles && (j >= ntiles || i < NSK || (j >= NSV && i <= j + NSK));
+        if (take_k) {
             const int s = i % NSK;
             const uint32_t k_free = NS_PROD ? su.bars.s_full(s) : su.bars.k_empty(s);
             if (i >= NSK && !ptx::mbar_wait(k_free, ((i / NSK) - 1) & 1, su.abort_flag))
@@ -349,9 +373,9 @@ __device__ __forceinline__ void produce_kv(const Setup<Gm> &su, const CUtensorMa
             ptx::mbar_arrive_expect_tx(su.bars.k_full(s), kTile);
             load_kv_tile<Gm>(su.sK + s * kTile, tmK, su.bars.k_full(s), kb + i * BN, b, hk, Hkv,
                              pages, pc, seq_end, dev_status);
-        }
-        if (i >= 1) {
-            const int j = i - 1, s = j % NSV;
+            ++i;
+        } else {
+            const int s = j % NSV;
             if (j >= NSV) {
                 const int r = j - NSV;   // PV_r read this slot last
                 constexpr int NSP = NS_PROD ? NS_PROD : 1;
@@ -368,6 +392,7 @@ __device__ __forceinline__ void produce_kv(const Setup<Gm> &su, const CUtensorMa
             ptx::mbar_arrive_expect_tx(su.bars.v_full(s), kTile);
             load_kv_tile<Gm>(su.sV + s * kTile, tmV, su.bars.v_full(s), kb + j * BN, b, hk, Hkv,
                              pages, pc, seq_end, dev_status);
+            ++j;
         }
     }
 }
@@ -902,35 +927,50 @@ __global__ void __launch_bounds__(rows_threads<SW>(), kMinBlocks)
             produce_kv<Gm, NS>(su, &tmK, &tmV, b, hk, Hkv, kb, ntiles, pages, pc, P + T,
                                dev_status);
     } else if (warp == 1) {
-        // Every mbarrier wait on the MMA-issuing thread leaves the tensor
-        // pipe idle for a while (it queues little ahead of the thread).  The
-        // whole warp polls (a lane-0 poll with the other lanes held at a
-        // shuffle measured slower), three waits per key tile.
-        auto wait0 = [&](uint32_t bar, uint32_t parity) {
-            return warp_wait(bar, parity, su.abort_flag);
-        };
-        bool ok = wait0(su.bars.q_full(), 0);
+        // Every cycle the MMA-issuing thread spends between MMAs leaves the
+        // tensor pipe idle (it queues little ahead of the thread), and a
+        // wait costs a barrier round trip even when the phase is complete.
+        // So the barriers of V_{j+1} and K_{j+NS}, which have usually landed
+        // long before, are tested while the MMAs before them are issued, and
+        // only P_j (the softmax's, the one that is often late) is waited for
+        // in line.  The whole warp polls (a lane-0 poll with the other lanes
+        // held at a shuffle measured slower).
+        auto kbar = [&](int i) { return su.bars.k_full(i % NSK); };
+        auto kpar = [&](int i) { return (uint32_t)(i / NSK) & 1u; };
+        auto vbar = [&](int i) { return su.bars.v_full(i % NSV); };
+        auto vpar = [&](int i) { return (uint32_t)(i / NSV) & 1u; };
+        bool ok = warp_wait(su.bars.q_full(), 0, su.abort_flag);
         ptx::tc_fence_after();
         // QK_i commits to s_full[i % NS], PV_j to o_ready[j % NS]
-        auto qk = [&](int i) {
-            if (!wait0(su.bars.k_full(i % NSK), (i / NSK) & 1))
-                return false;
+        for (int i = 0; ok && i < min(NS, ntiles); ++i) {
+            ok = warp_wait(kbar(i), kpar(i), su.abort_flag);
             ptx::tc_fence_after();
-            issue_qk<Gm, false>(su, lane, col_s(i), i, su.bars.s_full(i % NS));
-            return true;
-        };
-        for (int i = 0; ok && i < min(NS, ntiles); ++i)
-            ok = qk(i);
+            if (ok)
+                issue_qk<Gm, false>(su, lane, col_s(i), i, su.bars.s_full(i % NS));
+        }
+        // tests of phases whose previous phase this warp has already waited
+        // for (V_{j+1-NSV} before PV_{j+1-NSV}, K_j before QK_j), and whose
+        // next phase needs a product not yet issued (PV_{j+1}, QK_{j+NS})
+        uint32_t v_tested = ntiles > 0 ? ptx::mbar_test(vbar(0), vpar(0)) : 1u;
         for (int j = 0; ok && j < ntiles; ++j) {
-            if (!wait0(su.bars.p_full(j % NS), (j / NS) & 1) ||
-                !wait0(su.bars.v_full(j % NSV), (j / NSV) & 1)) {
+            if (!warp_wait(su.bars.p_full(j % NS), (j / NS) & 1, su.abort_flag) ||
+                !warp_wait_tested(v_tested, vbar(j), vpar(j), su.abort_flag)) {
                 ok = false;
                 break;
             }
+            const int i = j + NS;
+            const uint32_t k_tested = i < ntiles ? ptx::mbar_test(kbar(i), kpar(i)) : 1u;
             issue_pv<Gm, false, SW == 2>(su, lane, col_s(j), kO, j, j > 0,
                                          P + T - (kb + j * BN), su.bars.o_ready(j % NS));
-            if (j + NS < ntiles)
-                ok = qk(j + NS);
+            if (i < ntiles && !warp_wait_tested(k_tested, kbar(i), kpar(i), su.abort_flag)) {
+                ok = false;
+                break;
+            }
+            v_tested = j + 1 < ntiles ? ptx::mbar_test(vbar(j + 1), vpar(j + 1)) : 1u;
+            if (i < ntiles) {
+                ptx::tc_fence_after();
+                issue_qk<Gm, false>(su, lane, col_s(i), i, su.bars.s_full(i % NS));
+            }
         }
     } else {
         // softmax warps: one query row per thread == TMEM lane; with SW = 2
@@ -961,12 +1001,21 @@ __global__ void __launch_bounds__(rows_threads<SW>(), kMinBlocks)
         float m_run = -INFINITY, l_run = 0.f;
         int nx = 0;   // pair exchanges made
         bool ok = true;
+        // S_{j+1} is tested at the start of tile j and read after it: QK_{j+1}
+        // completes long before (it was issued after PV_{j+1-NS}), so the wait
+        // costs a vote; the phase before it (QK_{j+1-NS}) was waited for at
+        // tile j+1-NS, and the one after it needs this warp's P_{j+1}.
+        uint32_t s_tested = ntiles > 0 ? ptx::mbar_test(su.bars.s_full(0), 0) : 1u;
         for (int j = 0; ok && j < ntiles; ++j) {
-            if (!warp_wait(su.bars.s_full(j % NS), (j / NS) & 1, su.abort_flag)) {
+            if (!warp_wait_tested(s_tested, su.bars.s_full(j % NS), (j / NS) & 1,
+                                  su.abort_flag)) {
                 ok = false;
                 break;
             }
             ptx::tc_fence_after();
+            s_tested = j + 1 < ntiles
+                           ? ptx::mbar_test(su.bars.s_full((j + 1) % NS), ((j + 1) / NS) & 1)
+                           : 1u;
             auto wait_prev = [&]() { return wait_pv(j - 1); };
             if (SW == 1)
                 ok = softmax_rows_tile<BN>(su.tmem + lane_off + col_s(j), taddr_o, kb + j * BN,

@@ -344,7 +344,7 @@ int tsd_debug_wait_probe(int kind, unsigned long long limit_ns, void *scratch,
                          int32_t *dev_status, tsd_stream_t stream)
 {
     TSD_NVTX_RANGE();
-    if ((kind != 0 && kind != 1) || limit_ns < 1000000ull || limit_ns > 2000000000ull)
+    if (kind < 0 || kind > 2 || limit_ns < 1000000ull || limit_ns > 2000000000ull)
         return TSD_ERR_SHAPE;
     if (!scratch || !dev_status)
         return TSD_ERR_NULL;

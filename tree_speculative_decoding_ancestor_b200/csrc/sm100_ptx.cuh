@@ -56,6 +56,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
+// Non-blocking check: 1 once the phase with `parity` has completed, else 0.
+// Issued ahead of independent work, its latency overlaps that work when the
+// result is read only afterwards.
+__device__ __forceinline__ uint32_t mbar_test(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok;
+}
+
 // Wait for the phase with `parity` to complete.  Gives up (returns false)
 // once `abort` is raised by another role, or after `limit_ns` nanoseconds,
 // in which case it raises `abort` itself.

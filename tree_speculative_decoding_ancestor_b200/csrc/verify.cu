@@ -43,7 +43,10 @@
 #include <algorithm>
 #include <atomic>
 #include <climits>
+#include <cstdlib>
+#include <cstring>
 
+#include "cluster_xchg.cuh"
 #include "fp64_exp.cuh"
 #include "team_barrier.cuh"
 #include "tsd_common.cuh"
@@ -58,6 +61,7 @@ constexpr int kWalkThreads = 256;
 constexpr int kWalkWarps = kWalkThreads / 32;
 constexpr int kTeamMax = 32;          // CTAs per team: one partial per lane of a warp
 constexpr int kTeamMinChunk = 2048;   // vocabulary entries per CTA, at least
+constexpr int kClusterTeam = 8;       // CTAs per cluster team at most (portable cluster size)
 constexpr int kWalkMaxCtas = 1024;    // grid cap (sets the workspace slots)
 constexpr unsigned long long kTeamWaitNs = 2000000000ull;   // bound of one barrier wait
 constexpr int kCacheGroups = 4;       // groups of 4 entries per thread in the cached walk
@@ -788,7 +792,12 @@ __global__ void __launch_bounds__(kFinThreads)
 // VEC: V % 4 == 0, so every logits / q row is 16-byte aligned (the entry
 // point checks the base pointers) and the passes use float4 loads.
 // Grid: teams x K CTAs; team t walks sequences t, t + teams, ...
-template <bool VEC, bool CACHED>
+// CLUSTER: a team is a thread-block cluster of K CTAs, which exchange their
+// partial sums through distributed shared memory (cluster_exchange: a store
+// and an mbarrier arrival per peer, then one local wait); otherwise a team is
+// K CTAs of a cooperative launch exchanging them through global memory
+// (per-CTA slots and an arrival counter, team_barrier).
+template <bool VEC, bool CACHED, bool CLUSTER>
 __global__ void __launch_bounds__(kWalkThreads, CACHED ? 3 : 4)
     mss_walk_kernel(const float *__restrict__ logits, double temp,
                     const float *__restrict__ q_probs, int Rq, const int32_t *__restrict__ q_row,
@@ -821,10 +830,12 @@ __global__ void __launch_bounds__(kWalkThreads, CACHED ? 3 : 4)
     __shared__ double dc[kDecOps];
     // CACHED: this CTA's chunk of the current distribution, p(x) = pc[x - x_lo] * g
     __shared__ double pc[CACHED ? kCacheChunk : 1];
+    __shared__ XchgShared xs;   // CLUSTER: the team's partials, in every CTA
     double g = 0.0;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int teams = gridDim.x / K;
-    const int team = blockIdx.x / K, k = blockIdx.x % K;
+    const int team = blockIdx.x / K;
+    const int k = CLUSTER ? (int)cluster_ctarank() : blockIdx.x % K;
     const int x_lo = min(k * chunk, V), x_hi = min(x_lo + chunk, V);
     const double inv_temp = 1.0 / temp;
     const bool lead = k == 0 && tid == 0;   // writes the path and the error codes
@@ -833,6 +844,26 @@ __global__ void __launch_bounds__(kWalkThreads, CACHED ? 3 : 4)
     // this CTA's slot / the team's K slots of the next barrier
     auto slots = [&]() { return ws.slot + (nbar & 1) * kWalkMaxCtas + team * K; };
     fill_exp_table(table, 1.0);   // read only from here on (barriers below publish it)
+    if (CLUSTER) {
+        xchg_init(&xs, K);
+        cluster_sync_all();
+    }
+    // Publish this CTA's partial v and wait for the team's K partials: their
+    // array (nullptr when the wait ran out, on every thread of the CTA).
+    auto exchange = [&](double2 v) -> const double2 * {
+        if (CLUSTER) {
+            const int n = nbar++;
+            return cluster_exchange(&xs, K, n, v, kTeamWaitNs) ? xs.slot[n & 1] : nullptr;
+        }
+        double2 *sl = slots();
+        if (tid == 0)
+            sl[k] = v;
+        ++nbar;
+        return team_barrier(tm, nbar * K, &sh_ok, kTeamWaitNs) ? sl : nullptr;
+    };
+    // partial `i` of the last exchange (global slots bypass L1: other CTAs
+    // wrote them)
+    auto partial = [&](const double2 *sl, int i) { return CLUSTER ? sl[i] : __ldcg(sl + i); };
 
     for (int b = team; b < B; b += teams) {
         int T;
@@ -942,11 +973,9 @@ __global__ void __launch_bounds__(kWalkThreads, CACHED ? 3 : 4)
                                           &lastk);
             if (op >= 0)
                 dc[op] = pre;
-            double2 *sl = slots();
-            if (tid == 0)
-                sl[k] = make_double2(mz.y, __hiloint2double(__float_as_int((float)mz.x), lastk));
-            ++nbar;
-            if (!team_barrier(tm, nbar * K, &sh_ok, kTeamWaitNs)) {
+            const double2 *sl =
+                exchange(make_double2(mz.y, __hiloint2double(__float_as_int((float)mz.x), lastk)));
+            if (!sl) {
                 alive = false;
                 break;
             }
@@ -955,7 +984,7 @@ __global__ void __launch_bounds__(kWalkThreads, CACHED ? 3 : 4)
                 double mk = -INFINITY, zk = 0.0;
                 int lk = -1;
                 if (lane < K) {
-                    const double2 v = __ldcg(sl + lane);
+                    const double2 v = partial(sl, lane);
                     zk = v.x;
                     mk = (double)__int_as_float(__double2hiint(v.y));
                     lk = __double2loint(v.y);
@@ -995,11 +1024,8 @@ __global__ void __launch_bounds__(kWalkThreads, CACHED ? 3 : 4)
                     CACHED ? chunk_residual_cached<VEC>(qc, x_lo, x_hi, V, pc, g, shd, shi, &lastk)
                            : chunk_residual<VEC>(lrow, qc, x_lo, x_hi, V, st, table, shd, shi,
                                                  &lastk);
-                sl = slots();
-                if (tid == 0)
-                    sl[k] = make_double2(s, (double)lastk);
-                ++nbar;
-                if (!team_barrier(tm, nbar * K, &sh_ok, kTeamWaitNs)) {
+                sl = exchange(make_double2(s, (double)lastk));
+                if (!sl) {
                     alive = false;
                     break;
                 }
@@ -1008,7 +1034,7 @@ __global__ void __launch_bounds__(kWalkThreads, CACHED ? 3 : 4)
                     double sk = 0.0;
                     int lk = -1;
                     if (lane < K) {
-                        const double2 v = __ldcg(sl + lane);
+                        const double2 v = partial(sl, lane);
                         sk = v.x;
                         lk = (int)v.y;
                     }
@@ -1098,9 +1124,11 @@ __global__ void __launch_bounds__(kWalkThreads, CACHED ? 3 : 4)
             if (lead)
                 for (int bb = b; bb < B; bb += teams)
                     n_accepted[bb] = -1;
-            return;
+            break;
         }
     }
+    if (CLUSTER)   // no CTA leaves while a peer may still store to it
+        cluster_sync_all();
 }
 
 }  // namespace
@@ -1135,16 +1163,21 @@ int launch_verify_greedy(const float *logits, const int32_t *tokens, const int32
 
 namespace {
 
-// CTAs of the walk kernel that fit on the device at once (cooperative
-// launch limit), capped by the workspace slots; looked up once per device.
-const void *walk_kernel(bool vec, bool cached)
+// The cluster form always keeps its chunks in shared memory.
+const void *walk_kernel(bool vec, bool cached, bool cluster)
 {
-    return vec ? (cached ? reinterpret_cast<const void *>(mss_walk_kernel<true, true>)
-                         : reinterpret_cast<const void *>(mss_walk_kernel<true, false>))
-               : (cached ? reinterpret_cast<const void *>(mss_walk_kernel<false, true>)
-                         : reinterpret_cast<const void *>(mss_walk_kernel<false, false>));
+    if (cluster)
+        return vec ? reinterpret_cast<const void *>(mss_walk_kernel<true, true, true>)
+                   : reinterpret_cast<const void *>(mss_walk_kernel<false, true, true>);
+    return vec ? (cached ? reinterpret_cast<const void *>(mss_walk_kernel<true, true, false>)
+                         : reinterpret_cast<const void *>(mss_walk_kernel<true, false, false>))
+               : (cached ? reinterpret_cast<const void *>(mss_walk_kernel<false, true, false>)
+                         : reinterpret_cast<const void *>(mss_walk_kernel<false, false, false>));
 }
 
+// CTAs of the walk kernel that fit on the device at once (the cooperative
+// launch limit), capped by the workspace slots; looked up once per device.
+// The cluster form is sized by the same per-SM occupancy.
 int walk_capacity(bool vec, bool cached)
 {
     // Threads making their first call on a device at the same time may both
@@ -1160,7 +1193,7 @@ int walk_capacity(bool vec, bool cached)
         int sms = 0, occ = 0, coop = 0;
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
-        const void *fn = walk_kernel(vec, cached);
+        const void *fn = walk_kernel(vec, cached, false);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, kWalkThreads, 0);
         (void)cudaGetLastError();
         c = coop ? std::min(sms * occ, kWalkMaxCtas) : -1;
@@ -1190,12 +1223,41 @@ int walk_grid_for(int cap, int B, int V, int &K, int &teams, int &chunk)
     return TSD_OK;
 }
 
-// The walk keeps each CTA's chunk of the current distribution in shared
-// memory (`cached`) when the chunk fits kCacheChunk entries; otherwise it
-// recomputes the distribution from the rows in every pass.
-int walk_grid(int B, int V, int &K, int &teams, int &chunk, bool &cached)
+// TSD_WALK_EXCHANGE=global keeps the cooperative form where the cluster form
+// applies (read at every launch; for A/B runs and the tests).
+bool walk_global_forced()
+{
+    const char *e = getenv("TSD_WALK_EXCHANGE");
+    return e && strcmp(e, "global") == 0;
+}
+
+// The walk plan.  Cluster form: a vocabulary of at most kClusterTeam x
+// kCacheChunk entries, split over K <= kClusterTeam CTAs of one cluster
+// (K = V / kTeamMinChunk rounded up, so that each CTA's chunk of the current
+// distribution stays in its shared memory); a team per sequence as long as
+// the teams fit on the device at once, else fewer teams that each walk
+// several sequences (clusters need no co-residency with each other).
+// Otherwise the cooperative form; it keeps each CTA's chunk in shared memory
+// (`cached`) when the chunk fits kCacheChunk entries, else it recomputes the
+// distribution from the rows in every pass.
+int walk_grid(int B, int V, int &K, int &teams, int &chunk, bool &cached, bool &cluster)
 {
     const bool vec = (V & 3) == 0;
+    cluster = !walk_global_forced() && (long)V <= (long)kClusterTeam * kCacheChunk;
+    if (cluster) {
+        const int cap = walk_capacity(vec, true);
+        if (cap <= 0 || B < 1)
+            return TSD_ERR_CUDA;
+        K = std::max(1, std::min(kClusterTeam, (V + kTeamMinChunk - 1) / kTeamMinChunk));
+        chunk = (((V + K - 1) / K) + 3) & ~3;
+        if (chunk > kCacheChunk) {   // V just below the limit: the largest team
+            K = kClusterTeam;
+            chunk = (((V + K - 1) / K) + 3) & ~3;
+        }
+        teams = std::max(1, std::min(B, cap / K));
+        cached = true;
+        return TSD_OK;
+    }
     int rc = walk_grid_for(walk_capacity(vec, true), B, V, K, teams, chunk);
     cached = rc == TSD_OK && chunk <= kCacheChunk;
     if (!cached)
@@ -1208,8 +1270,8 @@ int walk_grid(int B, int V, int &K, int &teams, int &chunk, bool &cached)
 int verify_stochastic_plan(int B, int V, int32_t out[4])
 {
     int K, teams, chunk;
-    bool cached;
-    const int rc = walk_grid(B, V, K, teams, chunk, cached);
+    bool cached, cluster;
+    const int rc = walk_grid(B, V, K, teams, chunk, cached, cluster);
     if (rc != TSD_OK)
         return rc;
     out[0] = teams;
@@ -1231,11 +1293,11 @@ int launch_verify_stochastic(const float *logits, double temperature, const floa
         return TSD_OK;
     const bool vec = (V & 3) == 0;
     int K, teams, chunk;
-    bool cached;
-    if (walk_grid(B, V, K, teams, chunk, cached) != TSD_OK)
+    bool cached, cluster;
+    if (walk_grid(B, V, K, teams, chunk, cached, cluster) != TSD_OK)
         return TSD_ERR_CUDA;
     VerifyWs w = carve(ws);
-    if (cudaMemsetAsync(w.team, 0, (size_t)teams * sizeof(int2), stream) != cudaSuccess) {
+    if (!cluster && cudaMemsetAsync(w.team, 0, (size_t)teams * sizeof(int2), stream) != cudaSuccess) {
         (void)cudaGetLastError();
         return TSD_ERR_CUDA;
     }
@@ -1246,9 +1308,26 @@ int launch_verify_stochastic(const float *logits, double temperature, const floa
                     (void *)&Tmax,        (void *)&V,           (void *)&K,
                     (void *)&chunk,       (void *)&w,           (void *)&out_tokens,
                     (void *)&out_path,    (void *)&n_accepted,  (void *)&dev_status};
-    const void *fn = walk_kernel(vec, cached);
-    if (cudaLaunchCooperativeKernel(fn, dim3(teams * K), dim3(kWalkThreads), args, 0, stream) !=
-        cudaSuccess) {
+    const void *fn = walk_kernel(vec, cached, cluster);
+    cudaError_t err;
+    if (cluster) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(teams * K);
+        cfg.blockDim = dim3(kWalkThreads);
+        cfg.dynamicSmemBytes = 0;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)K;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        err = cudaLaunchKernelExC(&cfg, fn, args);
+    } else {
+        err = cudaLaunchCooperativeKernel(fn, dim3(teams * K), dim3(kWalkThreads), args, 0, stream);
+    }
+    if (err != cudaSuccess) {
         (void)cudaGetLastError();
         return TSD_ERR_CUDA;
     }
