@@ -31,13 +31,20 @@ __device__ __forceinline__ void fill_exp_table(double *table, double scale)
 }
 
 // scale * e^x for x <= 0; 0 for x < -708 (where e^x leaves the normal range).
+// n = round(x * 128/ln2) by adding 1.5 * 2^52 (the sum's last significand
+// bit is worth 1, so the addition rounds to nearest and leaves n in the low
+// bits of the sum), which keeps the reduction on the FMA pipe instead of the
+// conversion unit; n may differ by one from rounding the rounded product,
+// which only moves r a rounding error past ln2/256.
 __device__ __forceinline__ double table_exp(double x, const double *table)
 {
-    if (x < -708.0)
-        return 0.0;
-    const double n = rint(x * kOneTwentyEightOverLn2);
+    constexpr double kRound = 6755399441055744.0;   // 1.5 * 2^52
+    const bool under = x < -708.0;
+    x = under ? -708.0 : x;
+    const double sum = fma(x, kOneTwentyEightOverLn2, kRound);
+    const double n = sum - kRound;
     const double r = fma(n, -kLn2Over128Lo, fma(n, -kLn2Over128Hi, x));
-    const int ni = (int)n;
+    const int ni = __double2loint(sum);
     double p = 1.0 / 24.0;
     p = fma(p, r, 1.0 / 6.0);
     p = fma(p, r, 0.5);
@@ -46,7 +53,7 @@ __device__ __forceinline__ double table_exp(double x, const double *table)
     const double t = table[ni & (kExpTable - 1)];
     const double y = fma(t, p, t);           // scale * 2^(j/128) * e^r
     const long long bits = __double_as_longlong(y) + ((long long)(ni >> 7) << 52);
-    return __longlong_as_double(bits);
+    return under ? 0.0 : __longlong_as_double(bits);
 }
 
 }  // namespace tsd

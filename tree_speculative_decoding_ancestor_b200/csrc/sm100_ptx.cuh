@@ -112,6 +112,17 @@ __device__ __forceinline__ void tc_fence_after()
 }
 
 // --------------------------------------------------------------------- TMA
+// Untiled bulk copy of `bytes` (a multiple of 16) from global memory to this
+// CTA's shared memory (both addresses 16-byte aligned); completes on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
+                                          uint32_t bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], "
+                 "%2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *m)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");

@@ -48,6 +48,7 @@
 
 #include "cluster_xchg.cuh"
 #include "fp64_exp.cuh"
+#include "sm100_ptx.cuh"
 #include "team_barrier.cuh"
 #include "tsd_common.cuh"
 
@@ -66,6 +67,7 @@ constexpr int kWalkMaxCtas = 1024;    // grid cap (sets the workspace slots)
 constexpr unsigned long long kTeamWaitNs = 2000000000ull;   // bound of one barrier wait
 constexpr int kCacheGroups = 4;       // groups of 4 entries per thread in the cached walk
 constexpr int kCacheChunk = 4 * kCacheGroups * kWalkThreads;   // 4096 entries: 32 KB fp64
+constexpr int kStageBytes = 2 * 2 * kCacheChunk * 4;   // staged chunks: 2 sets x (logits, q)
 constexpr int kDecCache = 8;          // children per row whose test operands are prefetched
 constexpr int kDecOps = 2 * kDecCache + kDecCache * (kDecCache + 1) / 2;   // 52 loads
 
@@ -324,6 +326,13 @@ __device__ int row_argmax(const float *__restrict__ row, int V, float *shv, int 
     return bi == INT_MAX ? 0 : bi;
 }
 
+// Starts an L2 prefetch of bytes [p, p + bytes) (p 16-byte aligned, bytes a
+// multiple of 16): one bulk request, nothing waits for it.
+__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // Per-row state of multi-step speculative sampling.
 struct RowState {
     double m, inv_temp, temp, Z, inv_Z;
@@ -349,6 +358,20 @@ __device__ __forceinline__ void load4(const float *__restrict__ p, int x0, int V
 #pragma unroll
         for (int k = 0; k < 4; ++k)
             v[k] = x0 + k < V ? __ldg(p + x0 + k) : 0.f;
+    }
+}
+
+// Four values of a chunk [x_lo, ..) starting at x0 < x_hi: from the global
+// row (SMEM false: p is the row) or from the chunk staged in shared memory
+// (SMEM: p is the chunk's first entry, 16-byte aligned).
+template <bool VEC, bool SMEM>
+__device__ __forceinline__ void load4c(const float *p, int x0, int x_lo, int V, float (&v)[4])
+{
+    if (SMEM) {
+        const float4 t = *reinterpret_cast<const float4 *>(p + (x0 - x_lo));
+        v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+    } else {
+        load4<VEC>(p, x0, V, v);
     }
 }
 
@@ -477,7 +500,7 @@ __device__ double chunk_residual(const float *__restrict__ row, const float *__r
 
 // m/Z pass: the chunk's logits -> registers, the chunk max m_k (and the
 // largest x with a finite logit), then pc = exp((l - m_k)/T) and its sum.
-template <bool VEC>
+template <bool VEC, bool SMEM>
 __device__ double2 chunk_max_z_cached(const float *__restrict__ row, int x_lo, int x_hi, int V,
                                       double inv_temp, const double *table, double *pc,
                                       float *shf, double *shd, int *shi, int *last_out)
@@ -490,7 +513,7 @@ __device__ double2 chunk_max_z_cached(const float *__restrict__ row, int x_lo, i
         const int x0 = x_lo + 4 * (threadIdx.x + kWalkThreads * m);
         float v[4];
         if (x0 < x_hi)
-            load4<VEC>(row, x0, V, v);
+            load4c<VEC, SMEM>(row, x0, x_lo, V, v);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const float lv = (x0 + k < x_hi) ? v[k] : -INFINITY;
@@ -502,20 +525,24 @@ __device__ double2 chunk_max_z_cached(const float *__restrict__ row, int x_lo, i
     }
     block_max_last<kWalkThreads>(mt, last, shf, shi);
     *last_out = last;
+    // no branches here, so that the 16 exponentials of a thread interleave:
+    // entries past x_hi hold -inf (their pc entries, 0, are never read) and
+    // -inf goes to 0 (also when the whole chunk is -inf)
+    const double md = (double)mt;
+    double e[4 * kCacheGroups];
+#pragma unroll
+    for (int i = 0; i < 4 * kCacheGroups; ++i) {
+        const double x = ((double)l[i] - md) * inv_temp;
+        e[i] = table_exp(l[i] == -INFINITY ? -INFINITY : x, table);
+    }
     double z = 0.0;
 #pragma unroll
     for (int m = 0; m < kCacheGroups; ++m) {
         const int i0 = 4 * (threadIdx.x + kWalkThreads * m);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            if (x_lo + i0 + k < x_hi) {
-                const float lv = l[4 * m + k];
-                const double e = (lv == -INFINITY)
-                                     ? 0.0
-                                     : table_exp(((double)lv - (double)mt) * inv_temp, table);
-                pc[i0 + k] = e;
-                z += e;
-            }
+            pc[i0 + k] = e[4 * m + k];
+            z += e[4 * m + k];
         }
     }
     return make_double2((double)mt, mt == -INFINITY ? 0.0 : block_sum<kWalkThreads>(z, shd));
@@ -523,7 +550,7 @@ __device__ double2 chunk_max_z_cached(const float *__restrict__ row, int x_lo, i
 
 // Residual pass: S_k = sum over the chunk of max(0, p(x) - q(x)) with p(x) =
 // pc * g, and the largest x where that is positive.
-template <bool VEC>
+template <bool VEC, bool SMEM>
 __device__ double chunk_residual_cached(const float *__restrict__ q, int x_lo, int x_hi, int V,
                                         const double *pc, double g, double *shd, int *shi,
                                         int *last_out)
@@ -537,7 +564,7 @@ __device__ double chunk_residual_cached(const float *__restrict__ q, int x_lo, i
         if (x0 >= x_hi)
             continue;
         float qv[4];
-        load4<VEC>(q, x0, V, qv);
+        load4c<VEC, SMEM>(q, x0, x_lo, V, qv);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             if (x0 + k < x_hi) {
@@ -557,7 +584,7 @@ __device__ double chunk_residual_cached(const float *__restrict__ q, int x_lo, i
 // After a rejection with residual sum S > 0: pc = max(0, pc * g - q) / S (the
 // q chunk comes from L1, just read), so that g becomes 1.  Each thread
 // rewrites only the entries it owns.
-template <bool VEC>
+template <bool VEC, bool SMEM>
 __device__ void chunk_renormalise_cached(const float *__restrict__ q, int x_lo, int x_hi, int V,
                                          double *pc, double g, double inv_S)
 {
@@ -568,7 +595,7 @@ __device__ void chunk_renormalise_cached(const float *__restrict__ q, int x_lo, 
         if (x0 >= x_hi)
             continue;
         float qv[4];
-        load4<VEC>(q, x0, V, qv);
+        load4c<VEC, SMEM>(q, x0, x_lo, V, qv);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             if (x0 + k < x_hi) {
@@ -831,6 +858,16 @@ __global__ void __launch_bounds__(kWalkThreads, CACHED ? 3 : 4)
     // CACHED: this CTA's chunk of the current distribution, p(x) = pc[x - x_lo] * g
     __shared__ double pc[CACHED ? kCacheChunk : 1];
     __shared__ XchgShared xs;   // CLUSTER: the team's partials, in every CTA
+    // STAGE (cached, 16-byte aligned rows): each pass reads its chunk from
+    // shared memory, where a bulk copy put it -- for every pass after the
+    // first of a sequence, issued at the start of the pass before, which
+    // fetches both chunks the next pass may need (the next child's own logits
+    // row and its q row), so their latency hides behind a whole pass,
+    // exchange and decision.  Set n & 1 serves pass n.
+    constexpr bool STAGE = CACHED && VEC;
+    extern __shared__ __align__(16) float walk_stage[];   // [2 sets][logits, q][kCacheChunk]
+    __shared__ __align__(8) unsigned long long stage_bar[2];
+    __shared__ int stage_abort;
     double g = 0.0;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int teams = gridDim.x / K;
@@ -844,6 +881,82 @@ __global__ void __launch_bounds__(kWalkThreads, CACHED ? 3 : 4)
     // this CTA's slot / the team's K slots of the next barrier
     auto slots = [&]() { return ws.slot + (nbar & 1) * kWalkMaxCtas + team * K; };
     fill_exp_table(table, 1.0);   // read only from here on (barriers below publish it)
+    if (STAGE) {
+        if (tid == 0) {
+            ptx::mbar_init(ptx::smem_addr(&stage_bar[0]), 1);
+            ptx::mbar_init(ptx::smem_addr(&stage_bar[1]), 1);
+            stage_abort = 0;
+            ptx::fence_barrier_init();
+        }
+        __syncthreads();
+    }
+    // per set: a copy in flight (pending), the sources it holds, and the
+    // phases of its barrier waited for (the same in every thread)
+    bool pending0 = false, pending1 = false;
+    const float *have_l0 = nullptr, *have_l1 = nullptr, *have_q0 = nullptr, *have_q1 = nullptr;
+    int waits0 = 0, waits1 = 0, npass = 0;
+    const uint32_t stage_bytes = (uint32_t)(x_hi - x_lo) * 4u;
+    // thread 0: copy this CTA's chunks of the rows lsrc / qsrc (either may be
+    // null) into set `set`; every thread has finished reading that set
+    auto stage_issue = [&](int set, const float *lsrc, const float *qsrc) {
+        const uint32_t bar = ptx::smem_addr(&stage_bar[set]);
+        const uint32_t dst = ptx::smem_addr(walk_stage + set * 2 * kCacheChunk);
+        ptx::fence_proxy_async_smem();   // the set's earlier reads before the copy's writes
+        ptx::mbar_arrive_expect_tx(bar, stage_bytes * ((lsrc ? 1u : 0u) + (qsrc ? 1u : 0u)));
+        if (lsrc && stage_bytes)
+            ptx::bulk_load(dst, lsrc + x_lo, stage_bytes, bar);
+        if (qsrc && stage_bytes)
+            ptx::bulk_load(dst + 4u * kCacheChunk, qsrc + x_lo, stage_bytes, bar);
+    };
+    // every thread: wait for set `set` (bounded); false on timeout
+    auto stage_wait = [&](int set) {
+        int &w = set ? waits1 : waits0;
+        const bool ok = ptx::mbar_wait(ptx::smem_addr(&stage_bar[set]), (uint32_t)(w & 1),
+                                       &stage_abort, kTeamWaitNs);
+        ++w;
+        (set ? pending1 : pending0) = false;
+        return ok;
+    };
+    // Start of a pass that reads row `need` (a logits row, or a q row if
+    // is_q), followed by a decision on the child whose own logits row and q
+    // row are next_l and next_q (null: no decision on a child follows):
+    // returns the chunk to read (the global row when not staging), nullptr
+    // on timeout.
+    auto stage_pass = [&](const float *need, bool is_q, const float *next_l, const float *next_q)
+        -> const float * {
+        if (!STAGE)
+            return need;
+        const int set = npass & 1;
+        ++npass;
+        bool &pend = set ? pending1 : pending0;
+        const float *&hl = set ? have_l1 : have_l0;
+        const float *&hq = set ? have_q1 : have_q0;
+        bool ok = true;
+        if (pend && (is_q ? hq : hl) != need) {   // staged for another outcome: drain
+            ok = stage_wait(set);
+        }
+        __syncthreads();   // every thread is done with the other set (the pass before)
+        if (tid == 0) {
+            if (!pend)
+                stage_issue(set, is_q ? nullptr : need, is_q ? need : nullptr);
+            if (next_l)
+                stage_issue(set ^ 1, next_l, next_q);
+        }
+        if (!pend) {
+            hl = is_q ? nullptr : need;
+            hq = is_q ? need : nullptr;
+            pend = true;
+        }
+        if (next_l) {
+            (set ? pending0 : pending1) = true;
+            (set ? have_l0 : have_l1) = next_l;
+            (set ? have_q0 : have_q1) = next_q;
+        }
+        ok = stage_wait(set) && ok;
+        if (!__syncthreads_and(ok))
+            return nullptr;
+        return walk_stage + set * 2 * kCacheChunk + (is_q ? kCacheChunk : 0);
+    };
     if (CLUSTER) {
         xchg_init(&xs, K);
         cluster_sync_all();
@@ -909,7 +1022,10 @@ __global__ void __launch_bounds__(kWalkThreads, CACHED ? 3 : 4)
             const float *lrow = logits + ri * V;
             // issue the acceptance-test operands' loads (consumed after the
             // exchange below: their latency hides behind the pass)
-            double pre = 0.0;
+            // (loaded raw: a conversion next to its load would stall the
+            // thread on it before it issues its chunk loads)
+            float pre_f = 0.f;
+            double pre_d = 0.0;
             int op = -1;
             if (tid < kDecOps) {
                 int i = -1, j = -1;
@@ -928,12 +1044,12 @@ __global__ void __launch_bounds__(kWalkThreads, CACHED ? 3 : 4)
                 if (ci >= 0) {
                     const int x = s_tok[ci];
                     if (tid < kDecCache) {
-                        pre = (double)__ldg(lrow + x);
+                        pre_f = __ldg(lrow + x);
                     } else if (tid < 2 * kDecCache) {
-                        pre = __ldg(u_accept + (size_t)b * Tmax + ci);
+                        pre_d = __ldg(u_accept + (size_t)b * Tmax + ci);
                     } else {
                         const int cj = child(row, j);
-                        pre = (double)__ldg(qrow(cj) + x);
+                        pre_f = __ldg(qrow(cj) + x);
                     }
                     op = tid;
                 }
@@ -964,15 +1080,38 @@ __global__ void __launch_bounds__(kWalkThreads, CACHED ? 3 : 4)
                 }
                 return (p > 0.0 && u * qx <= p) ? 1 : 0;
             };
+            // Without staging: the next pass reads this CTA's chunk of the
+            // first child's own logits row (if it is accepted) or of its q
+            // row (if not); start fetching both into L2 now, behind this pass
+            // and the exchange.
+            auto prefetch_next = [&](int c) {
+                if (VEC && tid == 0 && c >= 0 && x_hi > x_lo) {
+                    const uint32_t bytes = (uint32_t)(x_hi - x_lo) * 4u;
+                    prefetch_l2(logits + ((size_t)b * (Tmax + 1) + c + 1) * V + x_lo, bytes);
+                    prefetch_l2(qrow(c) + x_lo, bytes);
+                }
+            };
+            auto lrow_of = [&](int c) {
+                return logits + ((size_t)b * (Tmax + 1) + c + 1) * V;
+            };
+            const int c0 = child(row, 0);
+            if (!STAGE)
+                prefetch_next(c0);
+            const float *lsrc = stage_pass(lrow, false, c0 >= 0 ? lrow_of(c0) : nullptr,
+                                           c0 >= 0 ? qrow(c0) : nullptr);
+            if (!lsrc) {
+                alive = false;
+                break;
+            }
             // m and Z of this row (slot: z_k, then m_k as fp32 bits | last_k)
             int lastk;
             const double2 mz =
-                CACHED ? chunk_max_z_cached<VEC>(lrow, x_lo, x_hi, V, inv_temp, table, pc, shf,
-                                                 shd, shi, &lastk)
+                CACHED ? chunk_max_z_cached<VEC, STAGE>(lsrc, x_lo, x_hi, V, inv_temp, table, pc,
+                                                        shf, shd, shi, &lastk)
                        : chunk_max_z<VEC>(lrow, x_lo, x_hi, V, inv_temp, table, shf, shd, shi,
                                           &lastk);
             if (op >= 0)
-                dc[op] = pre;
+                dc[op] = (op >= kDecCache && op < 2 * kDecCache) ? pre_d : (double)pre_f;
             const double2 *sl =
                 exchange(make_double2(mz.y, __hiloint2double(__float_as_int((float)mz.x), lastk)));
             if (!sl) {
@@ -1020,8 +1159,18 @@ __global__ void __launch_bounds__(kWalkThreads, CACHED ? 3 : 4)
                     break;
                 }
                 const float *qc = qrow(c);
+                const int nx = child(row, i + 1);   // the sibling tested next
+                if (!STAGE)
+                    prefetch_next(nx);
+                const float *qsrc = stage_pass(qc, true, nx >= 0 ? lrow_of(nx) : nullptr,
+                                               nx >= 0 ? qrow(nx) : nullptr);
+                if (!qsrc) {
+                    alive = false;
+                    break;
+                }
                 const double s =
-                    CACHED ? chunk_residual_cached<VEC>(qc, x_lo, x_hi, V, pc, g, shd, shi, &lastk)
+                    CACHED ? chunk_residual_cached<VEC, STAGE>(qsrc, x_lo, x_hi, V, pc, g, shd, shi,
+                                                               &lastk)
                            : chunk_residual<VEC>(lrow, qc, x_lo, x_hi, V, st, table, shd, shi,
                                                  &lastk);
                 sl = exchange(make_double2(s, (double)lastk));
@@ -1053,7 +1202,8 @@ __global__ void __launch_bounds__(kWalkThreads, CACHED ? 3 : 4)
                 }
                 __syncthreads();
                 if (CACHED && st.S[st.n - 1] > 0.0) {   // else p stays as it was
-                    chunk_renormalise_cached<VEC>(qc, x_lo, x_hi, V, pc, g, st.inv_S[st.n - 1]);
+                    chunk_renormalise_cached<VEC, STAGE>(qsrc, x_lo, x_hi, V, pc, g,
+                                                         st.inv_S[st.n - 1]);
                     g = 1.0;
                 }
                 c = next;
@@ -1127,6 +1277,12 @@ __global__ void __launch_bounds__(kWalkThreads, CACHED ? 3 : 4)
             break;
         }
     }
+    if (STAGE) {   // copies still in flight (a walk that gave up): let them land
+        if (pending0)
+            stage_wait(0);
+        if (pending1)
+            stage_wait(1);
+    }
     if (CLUSTER)   // no CTA leaves while a peer may still store to it
         cluster_sync_all();
 }
@@ -1175,6 +1331,34 @@ const void *walk_kernel(bool vec, bool cached, bool cluster)
                          : reinterpret_cast<const void *>(mss_walk_kernel<false, false, false>));
 }
 
+// Dynamic shared memory of a walk instance: the staged chunks of the cached
+// form over 16-byte aligned rows.
+int walk_smem(bool vec, bool cached) { return (vec && cached) ? kStageBytes : 0; }
+
+// The dynamic shared-memory limit of every walk instance that stages, set
+// once per device (a function attribute of the current device).
+bool walk_attributes()
+{
+    constexpr int kMaxDevices = 64;
+    static std::atomic<int> done[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return false;
+    if (done[dev].load(std::memory_order_acquire))
+        return true;
+    const void *fns[] = {walk_kernel(true, true, false), walk_kernel(true, true, true)};
+    bool ok = true;
+    for (const void *fn : fns)
+        ok = ok && cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        kStageBytes) == cudaSuccess;
+    if (!ok) {
+        (void)cudaGetLastError();
+        return false;
+    }
+    done[dev].store(1, std::memory_order_release);
+    return true;
+}
+
 // CTAs of the walk kernel that fit on the device at once (the cooperative
 // launch limit), capped by the workspace slots; looked up once per device.
 // The cluster form is sized by the same per-SM occupancy.
@@ -1194,7 +1378,10 @@ int walk_capacity(bool vec, bool cached)
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
         const void *fn = walk_kernel(vec, cached, false);
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, kWalkThreads, 0);
+        if (!walk_attributes())
+            return 0;
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, kWalkThreads,
+                                                      walk_smem(vec, cached));
         (void)cudaGetLastError();
         c = coop ? std::min(sms * occ, kWalkMaxCtas) : -1;
         slot.store(c, std::memory_order_relaxed);
@@ -1309,12 +1496,15 @@ int launch_verify_stochastic(const float *logits, double temperature, const floa
                     (void *)&chunk,       (void *)&w,           (void *)&out_tokens,
                     (void *)&out_path,    (void *)&n_accepted,  (void *)&dev_status};
     const void *fn = walk_kernel(vec, cached, cluster);
+    const int smem = walk_smem(vec, cached);
+    if (smem && !walk_attributes())
+        return TSD_ERR_CUDA;
     cudaError_t err;
     if (cluster) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(teams * K);
         cfg.blockDim = dim3(kWalkThreads);
-        cfg.dynamicSmemBytes = 0;
+        cfg.dynamicSmemBytes = (size_t)smem;
         cfg.stream = stream;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1325,7 +1515,8 @@ int launch_verify_stochastic(const float *logits, double temperature, const floa
         cfg.numAttrs = 1;
         err = cudaLaunchKernelExC(&cfg, fn, args);
     } else {
-        err = cudaLaunchCooperativeKernel(fn, dim3(teams * K), dim3(kWalkThreads), args, 0, stream);
+        err = cudaLaunchCooperativeKernel(fn, dim3(teams * K), dim3(kWalkThreads), args,
+                                          (size_t)smem, stream);
     }
     if (err != cudaSuccess) {
         (void)cudaGetLastError();
