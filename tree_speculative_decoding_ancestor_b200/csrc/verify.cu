@@ -9,14 +9,12 @@
 //                           path matches, the deepest (lowest index on ties),
 //                           and the argmax of its row (computed here for a leaf).
 // stochastic (multi-step speculative sampling)
-//   mss_walk_kernel         one cooperative launch.  Each sequence is walked by
-//                           a team of K CTAs, CTA k owning one contiguous chunk
-//                           of the vocabulary.  At the current node's row the
-//                           team computes m = max l and Z = sum exp((l-m)/T)
-//                           in fp64 (one pass: each thread keeps a running max
-//                           and rescales its sum when the max rises), then
-//                           tries the children in ascending index: child c
-//                           with token x is accepted iff p(x) > 0 and
+//   mss_walk_kernel         one launch.  Each sequence is walked by a team of
+//                           K CTAs, CTA k owning one contiguous chunk of the
+//                           vocabulary.  At the current node's row the team
+//                           computes m = max l and Z = sum exp((l-m)/T) in
+//                           fp64, then tries the children in ascending index:
+//                           child c with token x is accepted iff p(x) > 0 and
 //                           u_c * q_c(x) <= p(x) (exact fp64 formula, every
 //                           CTA taking the same decision from the same
 //                           numbers); after a rejection the team sums
@@ -27,19 +25,26 @@
 //                           S_k/S after a rejection); where the walk stops,
 //                           the chunk whose running sum passes u_sample[row]
 //                           is scanned (fp64 block scan) by its CTA for the
-//                           token -- the draw costs no barrier.
-//                           Only rows on the accepted path are read.  Partial
-//                           results cross CTAs through one workspace slot per
-//                           CTA and a per-team arrival counter; every wait on
-//                           a counter is bounded (TSD_DEV_TIMEOUT).
+//                           token -- the draw costs no exchange.
+//                           Only rows on the accepted path are read.  A team
+//                           is a thread-block cluster exchanging its partials
+//                           through distributed shared memory (vocabularies
+//                           up to 8 x 4096 entries) or K CTAs of a cooperative
+//                           launch exchanging them through workspace slots
+//                           and a per-team arrival counter; every wait is
+//                           bounded (TSD_DEV_TIMEOUT).
 //
-// Residual distributions are never materialised: p^(n)(x) is recomputed per
-// element from the logits row, the rejected siblings' q rows and their
-// normalisers (all L2-resident while a team works on a row).  The bulk sums
-// (Z, S, the CDF) use a table-driven fp64 exp (its table pre-scaled by 1/Z)
-// and reciprocals; the acceptance tests use the exact formula.  Both agree with a sequential fp64 evaluation to ~1e-15
-// relative, so a decision can only differ when its uniform lies within that
-// distance of the boundary.
+// Cached form (chunks of at most 4096 entries): each CTA keeps its chunk of
+// the current distribution in shared memory in fp64, scaled (p = pc * g), so
+// a rejected sibling costs one pass over its q chunk and an in-place
+// renormalisation; with 16-byte aligned rows the chunks a pass reads arrive
+// in shared memory by bulk copies issued one pass ahead.  Otherwise p^(n)(x)
+// is recomputed per element from the logits row, the rejected siblings' q
+// rows and their normalisers.  The bulk sums (Z, S, the CDF) use a
+// table-driven fp64 exp and reciprocals; the acceptance tests use the exact
+// formula.  Both agree with a sequential fp64 evaluation to ~1e-15 relative,
+// so a decision can only differ when its uniform lies within that distance
+// of the boundary.
 #include <algorithm>
 #include <atomic>
 #include <climits>
