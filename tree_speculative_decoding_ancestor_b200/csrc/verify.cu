@@ -15,7 +15,7 @@
 //                           computes m = max l and Z = sum exp((l-m)/T) in
 //                           fp64, then tries the children in ascending index:
 //                           child c with token x is accepted iff p(x) > 0 and
-//                           u_c * q_c(x) <= p(x) (exact fp64 formula, every
+//                           u_c * q_c(x) <= p(x) (fp64, CUDA's exp, every
 //                           CTA taking the same decision from the same
 //                           numbers); after a rejection the team sums
 //                           S = sum max(0, p - q_c) and p becomes
@@ -41,10 +41,10 @@
 // in shared memory by bulk copies issued one pass ahead.  Otherwise p^(n)(x)
 // is recomputed per element from the logits row, the rejected siblings' q
 // rows and their normalisers.  The bulk sums (Z, S, the CDF) use a
-// table-driven fp64 exp and reciprocals; the acceptance tests use the exact
-// formula.  Both agree with a sequential fp64 evaluation to ~1e-15 relative,
-// so a decision can only differ when its uniform lies within that distance
-// of the boundary.
+// table-driven fp64 exp and reciprocals; the acceptance tests use CUDA's fp64
+// exp and the reciprocals of T, Z and the S_j.  Both agree with a sequential
+// fp64 evaluation of the formulas to ~1e-15 relative, so a decision can only
+// differ when its uniform lies within that distance of the boundary.
 #include <algorithm>
 #include <atomic>
 #include <climits>
@@ -1061,26 +1061,33 @@ __global__ void __launch_bounds__(kWalkThreads, CACHED ? 3 : 4)
             }
             // lane 0 of warp 0: the acceptance test of child i, given the
             // row's m, Z and the i siblings rejected before it (in st)
-            auto accept = [&](int i, int c) {
+            // exp((l(x_c) - m) / T) of child i, on every lane of warp 0 (it
+            // needs the row's max only, so it runs beside the sum's reduction)
+            auto test_exp = [&](int i, int c, double m) {
+                const double lx = i < kDecCache ? dc[i] : (double)lrow[s_tok[c]];
+                return exp((lx - m) * inv_temp);
+            };
+            // lane 0 of warp 0: the acceptance test of child i from its
+            // test_exp value e, given the row's 1/Z and the i siblings
+            // rejected before it (in st)
+            auto accept = [&](int i, int c, double e, double inv_Z) {
                 const int x = s_tok[c];
-                double lx, qx, u;
+                double qx, u;
                 if (i < kDecCache) {
-                    lx = dc[i];
                     u = dc[kDecCache + i];
                     qx = dc[2 * kDecCache + i * (i + 1) / 2 + i];
                 } else {
-                    lx = (double)lrow[x];
                     u = u_accept[(size_t)b * Tmax + c];
                     qx = (double)qrow(c)[x];
                 }
-                double p = exp((lx - st.m) / st.temp) / st.Z;
+                double p = e * inv_Z;
                 for (int j = 0; j < st.n; ++j) {
                     if (st.S[j] > 0.0) {
                         const double qj = i < kDecCache
                                               ? dc[2 * kDecCache + i * (i + 1) / 2 + j]
                                               : (double)st.q[j][x];
                         const double r = p - qj;
-                        p = (r > 0.0 ? r : 0.0) / st.S[j];
+                        p = (r > 0.0 ? r : 0.0) * st.inv_S[j];
                     }
                 }
                 return (p > 0.0 && u * qx <= p) ? 1 : 0;
@@ -1137,19 +1144,21 @@ __global__ void __launch_bounds__(kWalkThreads, CACHED ? 3 : 4)
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1)
                     m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
+                const double e0 = c >= 0 ? test_exp(0, c, m) : 0.0;
                 const double zs =
                     mk == -INFINITY ? 0.0 : zk * table_exp((mk - m) * inv_temp, table);
                 const double Z = warp_sum(zs);
-                draw_sum[lane] = zs / Z;
+                const double inv_Z = 1.0 / Z;
+                draw_sum[lane] = zs * inv_Z;
                 draw_last[lane] = lk;
                 if (lane == 0) {
                     st.m = m;
                     st.Z = Z;
-                    st.inv_Z = 1.0 / Z;
+                    st.inv_Z = inv_Z;
                     st.temp = temp;
                     st.inv_temp = inv_temp;
                     st.n = 0;
-                    sh_dec = c >= 0 ? accept(0, c) : 0;
+                    sh_dec = c >= 0 ? accept(0, c, e0, inv_Z) : 0;
                 }
             }
             __syncthreads();
@@ -1192,17 +1201,19 @@ __global__ void __launch_bounds__(kWalkThreads, CACHED ? 3 : 4)
                         sk = v.x;
                         lk = (int)v.y;
                     }
+                    const double en = next >= 0 ? test_exp(i + 1, next, st.m) : 0.0;
                     const double S = warp_sum(sk);
+                    const double inv_S = S > 0.0 ? 1.0 / S : 0.0;
                     if (S > 0.0) {   // else p stays as it was
-                        draw_sum[lane] = sk * (1.0 / S);
+                        draw_sum[lane] = sk * inv_S;
                         draw_last[lane] = lk;
                     }
                     if (lane == 0) {
                         st.q[st.n] = qc;
                         st.S[st.n] = S;
-                        st.inv_S[st.n] = S > 0.0 ? 1.0 / S : 0.0;
+                        st.inv_S[st.n] = inv_S;
                         st.n += 1;
-                        sh_dec = next >= 0 ? accept(i + 1, next) : 0;
+                        sh_dec = next >= 0 ? accept(i + 1, next, en, st.inv_Z) : 0;
                     }
                 }
                 __syncthreads();
