@@ -75,6 +75,7 @@ constexpr int kCacheChunk = 4 * kCacheGroups * kWalkThreads;   // 4096 entries: 
 constexpr int kStageBytes = 2 * 2 * kCacheChunk * 4;   // staged chunks: 2 sets x (logits, q)
 constexpr int kDecCache = 8;          // children per row whose test operands are prefetched
 constexpr int kDecOps = 2 * kDecCache + kDecCache * (kDecCache + 1) / 2;   // 52 loads
+static_assert(4 * kDecOps <= kWalkThreads, "one acceptance operand per fourth thread");
 
 struct VerifyWs {
     double2 *slot;     // [2][kWalkMaxCtas]  per-CTA partials, by barrier parity
@@ -329,6 +330,23 @@ __device__ int row_argmax(const float *__restrict__ row, int V, float *shv, int 
     }
     block_argmax<NT>(bv, bi, shv, shi);
     return bi == INT_MAX ? 0 : bi;
+}
+
+// Asynchronous 4- and 8-byte copies from global to shared memory (aligned to
+// their size), and the wait for all of this thread's copies.
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all()
+{
+    asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
 // Starts an L2 prefetch of bytes [p, p + bytes) (p 16-byte aligned, bytes a
@@ -855,11 +873,15 @@ __global__ void __launch_bounds__(kWalkThreads, CACHED ? 3 : 4)
     __shared__ int draw_last[32];
     // the sequence's tree (child lists, tokens, q rows), staged once
     __shared__ int s_fc[kMaxTree + 1], s_ns[kMaxTree], s_tok[kMaxTree], s_qr[kMaxTree];
+    // the first kDecCache children of every row (-1 past the last), so that
+    // looking one up walks no sibling chain
+    __shared__ int s_kid[kMaxTree + 1][kDecCache];
     // the operands of the acceptance tests of the current row's first
     // kDecCache children, loaded while the row's m/Z pass runs:
     // dc[i] = l(x_i), dc[kDecCache + i] = u_i, dc[2 kDecCache + i(i+1)/2 + j] =
     // q_j(x_i) for j <= i (q_j: the q row of child j; j = i: the child's own)
     __shared__ double dc[kDecOps];
+    __shared__ unsigned long long dc_raw[kDecOps];   // their raw bits, as fetched
     // CACHED: this CTA's chunk of the current distribution, p(x) = pc[x - x_lo] * g
     __shared__ double pc[CACHED ? kCacheChunk : 1];
     __shared__ XchgShared xs;   // CLUSTER: the team's partials, in every CTA
@@ -1010,12 +1032,21 @@ __global__ void __launch_bounds__(kWalkThreads, CACHED ? 3 : 4)
                 n_accepted[b] = -1;
             continue;
         }
+        for (int u = tid; u <= T; u += kWalkThreads) {
+            int c = s_fc[u];
+#pragma unroll
+            for (int i = 0; i < kDecCache; ++i) {
+                s_kid[u][i] = c;
+                c = (c >= 0 && c < T) ? s_ns[c] : -1;
+            }
+        }
+        __syncthreads();
         // child i (ascending index) of the node whose logits row is `row`; -1
         // past the last (the lists come from the mask build: they are
         // increasing and inside the tree)
         auto child = [&](int row, int i) {
-            int c = s_fc[row];
-            for (; c >= 0 && i > 0; --i)
+            int c = s_kid[row][min(i, kDecCache - 1)];
+            for (i -= kDecCache - 1; c >= 0 && i > 0; --i)
                 c = (c < T) ? s_ns[c] : -1;
             return (c >= 0 && in_bounds(c, T, dev_status)) ? c : -1;
         };
@@ -1025,42 +1056,7 @@ __global__ void __launch_bounds__(kWalkThreads, CACHED ? 3 : 4)
         for (;;) {
             const size_t ri = (size_t)b * (Tmax + 1) + row;
             const float *lrow = logits + ri * V;
-            // issue the acceptance-test operands' loads (consumed after the
-            // exchange below: their latency hides behind the pass)
-            // (loaded raw: a conversion next to its load would stall the
-            // thread on it before it issues its chunk loads)
-            float pre_f = 0.f;
-            double pre_d = 0.0;
             int op = -1;
-            if (tid < kDecOps) {
-                int i = -1, j = -1;
-                if (tid < kDecCache)
-                    i = tid;
-                else if (tid < 2 * kDecCache)
-                    i = tid - kDecCache;
-                else {
-                    const int t2 = tid - 2 * kDecCache;   // i (i + 1) / 2 + j, j <= i
-                    i = 0;
-                    while ((i + 1) * (i + 2) / 2 <= t2)
-                        ++i;
-                    j = t2 - i * (i + 1) / 2;
-                }
-                const int ci = child(row, i);
-                if (ci >= 0) {
-                    const int x = s_tok[ci];
-                    if (tid < kDecCache) {
-                        pre_f = __ldg(lrow + x);
-                    } else if (tid < 2 * kDecCache) {
-                        pre_d = __ldg(u_accept + (size_t)b * Tmax + ci);
-                    } else {
-                        const int cj = child(row, j);
-                        pre_f = __ldg(qrow(cj) + x);
-                    }
-                    op = tid;
-                }
-            }
-            // lane 0 of warp 0: the acceptance test of child i, given the
-            // row's m, Z and the i siblings rejected before it (in st)
             // exp((l(x_c) - m) / T) of child i, on every lane of warp 0 (it
             // needs the row's max only, so it runs beside the sum's reduction)
             auto test_exp = [&](int i, int c, double m) {
@@ -1115,6 +1111,38 @@ __global__ void __launch_bounds__(kWalkThreads, CACHED ? 3 : 4)
                 alive = false;
                 break;
             }
+            // fetch the acceptance-test operands (read after the pass below)
+            // by asynchronous copies into shared memory, which no barrier of
+            // the pass waits for; operand t on thread 4t (at most eight
+            // scattered loads per warp)
+            if ((tid & 3) == 0 && (tid >> 2) < kDecOps) {
+                const int t = tid >> 2;
+                int i = -1, j = -1;
+                if (t < kDecCache)
+                    i = t;
+                else if (t < 2 * kDecCache)
+                    i = t - kDecCache;
+                else {
+                    const int t2 = t - 2 * kDecCache;   // i (i + 1) / 2 + j, j <= i
+                    i = (int)((sqrtf(8.f * (float)t2 + 1.f) - 1.f) * 0.5f);
+                    i += ((i + 1) * (i + 2) / 2 <= t2) - (i * (i + 1) / 2 > t2);
+                    j = t2 - i * (i + 1) / 2;
+                }
+                const int ci = child(row, i);
+                if (ci >= 0) {
+                    const int x = s_tok[ci];
+                    const uint32_t dst = ptx::smem_addr(&dc_raw[t]);
+                    if (t < kDecCache) {
+                        cp_async4(dst, lrow + x);
+                    } else if (t < 2 * kDecCache) {
+                        cp_async8(dst, u_accept + (size_t)b * Tmax + ci);
+                    } else {
+                        const int cj = child(row, j);
+                        cp_async4(dst, qrow(cj) + x);
+                    }
+                    op = t;
+                }
+            }
             // m and Z of this row (slot: z_k, then m_k as fp32 bits | last_k)
             int lastk;
             const double2 mz =
@@ -1122,8 +1150,13 @@ __global__ void __launch_bounds__(kWalkThreads, CACHED ? 3 : 4)
                                                         shf, shd, shi, &lastk)
                        : chunk_max_z<VEC>(lrow, x_lo, x_hi, V, inv_temp, table, shf, shd, shi,
                                           &lastk);
-            if (op >= 0)
-                dc[op] = (op >= kDecCache && op < 2 * kDecCache) ? pre_d : (double)pre_f;
+            if (op >= 0) {   // long arrived: the pass took longer than the fetch
+                cp_async_wait_all();
+                const unsigned long long raw = dc_raw[op];
+                dc[op] = (op >= kDecCache && op < 2 * kDecCache)
+                             ? __longlong_as_double((long long)raw)
+                             : (double)__uint_as_float((uint32_t)raw);
+            }
             const double2 *sl =
                 exchange(make_double2(mz.y, __hiloint2double(__float_as_int((float)mz.x), lastk)));
             if (!sl) {
