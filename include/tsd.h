@@ -262,9 +262,13 @@ int tsd_tree_verify_greedy(const float *logits, const int32_t *tokens, const int
  *   n_nodes, first_child, next_sibling   from tsd_tree_mask_build
  *   u_accept      [B][Tmax] fp64, u_sample [B][Tmax+1] fp64: uniforms in (0,1)
  *   out_tokens, out_path, n_accepted      as for the greedy call
- * Work: one cooperative kernel launch; each sequence's walk reads only the
- * logits rows (and q rows) of the nodes it reaches.  The CTAs of a sequence
- * meet at barriers whose waits are bounded (about 2 s).
+ * Work: one kernel launch; each sequence's walk reads only the logits rows
+ * (and q rows) of the nodes it reaches.  The CTAs walking a sequence form a
+ * thread-block cluster and exchange their partial sums through distributed
+ * shared memory (V <= 32768), or are CTAs of a cooperative launch that
+ * exchange them through the workspace; either way every wait is bounded
+ * (about 2 s).  The environment variable TSD_WALK_EXCHANGE=global selects
+ * the cooperative form for every V (read at every call).
  * Device: TSD_DEV_BAD_TOKEN, TSD_DEV_BAD_QROW, TSD_DEV_TIMEOUT (a barrier
  * wait expired; the affected sequences get n_accepted = -1).
  */
@@ -286,7 +290,9 @@ int tsd_tree_verify_stochastic(const float *logits, double temperature, const fl
  *            sequences t, t + teams, t + 2 teams, ...)
  *   plan[1]  CTAs per team, each owning one chunk of the vocabulary
  *   plan[2]  vocabulary entries per chunk
- *   plan[3]  CTAs in the cooperative launch (teams x CTAs per team)
+ *   plan[3]  CTAs in the launch (teams x CTAs per team)
+ * A team is one thread-block cluster when V <= 32768 (then at most 8 CTAs)
+ * and CTAs of a cooperative launch otherwise.
  * Errors: TSD_ERR_NULL (plan), TSD_ERR_SHAPE (B < 1, Tmax out of range,
  * V < 1), TSD_ERR_CUDA (no device or no cooperative launch).
  */

@@ -9,7 +9,7 @@ check that it returns exactly what the workspace entry point returns, and
 what the fp64 oracle returns, on two calls in a row (the second call finds
 the first call's leftovers in the shared array), and that its fixed scratch
 does not limit the shape: a batch with more sequences than the verifier's
-grid has CTAs still runs, one-CTA teams walking several sequences each.
+grid has teams still runs, one-CTA teams walking several sequences each.
 
 This file is collected last on purpose, so that a run stopping at the first
 failure has already run every other test.
@@ -82,9 +82,9 @@ def test_noalloc_matches_workspace_call_twice(cuda_device):
 def test_noalloc_takes_a_batch_larger_than_the_grid(cuda_device):
     lib = tsd.load_library()
     # 1100 sequences over a 64-token vocabulary: one CTA per team, and more
-    # sequences than the cooperative grid holds (it is capped at 1024 CTAs),
-    # so teams walk several sequences each and their barrier counters run on
-    # from one sequence to the next.
+    # sequences than the teams the device holds at once (the plan caps the
+    # teams at that), so teams walk several sequences each and their
+    # exchange state runs on from one sequence to the next.
     dev = cuda_device
     B, Tmax, V = 1100, 24, 64
     plan = tsd.verify_stochastic_plan(B, Tmax, V)
