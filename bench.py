@@ -220,6 +220,11 @@ class Step:
             B, Tmax, w.Hq, w.Hkv, w.D, w.Lmax, d["q"].dtype)), dtype=torch.uint8, device=dev)
         self.ws_ver = torch.empty(max(256, tsd.verify_workspace_size(B, Tmax, w.V)),
                                   dtype=torch.uint8, device=dev)
+        # the greedy call's own workspace and stream: with both verify modes
+        # the two calls run side by side (they read the same inputs and
+        # nothing of each other's)
+        self.ws_ver_g = torch.empty_like(self.ws_ver)
+        self.side = torch.cuda.Stream(device=dev)
         self.ev = None
 
     def run_mask(self):
@@ -277,14 +282,30 @@ class Step:
         self.d = self.sets[0]
 
     def run_verify(self):
+        """The workload's verify calls.  With both modes, the greedy call runs
+        on a second stream beside the stochastic one (forked after the mask
+        build and the attention call, joined before the step ends): the
+        stochastic walk is latency-bound on a few CTAs per SM and the greedy
+        row scan bandwidth-bound, so they overlap."""
         w, d, tsd = self.w, self.d, self.tsd
-        if "greedy" in w.verify:
-            tsd.tree_verify_greedy(d["logits"], d["tokens"], d["parent"], d["n_nodes"],
-                                   self.tree, out=self.g, workspace=self.ws_ver)
-        if "stochastic" in w.verify:
-            tsd.tree_verify_stochastic(d["logits"], w.temperature, d["q_probs"], d["q_row"],
-                                       d["tokens"], d["n_nodes"], self.tree, d["u_accept"],
-                                       d["u_sample"], out=self.s, workspace=self.ws_ver)
+        greedy = lambda ws: tsd.tree_verify_greedy(  # noqa: E731
+            d["logits"], d["tokens"], d["parent"], d["n_nodes"], self.tree, out=self.g,
+            workspace=ws)
+        if "stochastic" not in w.verify:
+            if "greedy" in w.verify:
+                greedy(self.ws_ver)
+            return
+        main = torch.cuda.current_stream(self.dev)
+        both = "greedy" in w.verify
+        if both:
+            self.side.wait_stream(main)
+        tsd.tree_verify_stochastic(d["logits"], w.temperature, d["q_probs"], d["q_row"],
+                                   d["tokens"], d["n_nodes"], self.tree, d["u_accept"],
+                                   d["u_sample"], out=self.s, workspace=self.ws_ver)
+        if both:
+            with torch.cuda.stream(self.side):
+                greedy(self.ws_ver_g)
+            main.wait_stream(self.side)
 
 
 def _clock_sampler(index):
