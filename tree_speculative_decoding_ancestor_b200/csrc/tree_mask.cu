@@ -4,9 +4,11 @@
 // precomputed from the tree topology).
 //
 // One CTA of 128 threads per sequence, one thread per node slot.  The parent
-// array (<= 512 B) is staged in shared memory; every node walks its own root
-// path there (<= 128 steps, bounded because parent[v] < v is validated
-// first), so the whole build is a handful of shared-memory passes.
+// array (<= 512 B) is staged in shared memory (read beside the node count,
+// one global round trip); every node walks its own root path there (<= 128
+// steps, bounded because parent[v] < v is validated first).  Child lists
+// come from one 128-bit set of children per node: the first child is its
+// lowest bit, a node's next sibling the next bit set above its own.
 #include <climits>
 
 #include "tsd_common.cuh"
@@ -20,19 +22,23 @@ __global__ void __launch_bounds__(kMaxTree)
                      int32_t *dev_status)
 {
     __shared__ int32_t par[kMaxTree];
-    __shared__ int32_t fc[kMaxTree + 1];
+    __shared__ uint32_t kids[kMaxTree + 1][kMaskWords];   // children of node v - 1 (v = 0: root)
     const int b = blockIdx.x;
     const int u = threadIdx.x;
+    const long long nb = (long long)gridDim.x * Tmax;   // B * Tmax
+    // both reads at once: the slots past the node count are dropped below
+    int p = -1;
+    if (u < Tmax && in_bounds((long long)b * Tmax + u, nb, dev_status))
+        p = parent[(size_t)b * Tmax + u];
     const int T = n_nodes[b];
     const bool bad_T = !tree_header_ok(T, Tmax);
-    const long long nb = (long long)gridDim.x * Tmax;   // B * Tmax
-    int p = -1;
-    if (u < Tmax && !bad_T && u < T && in_bounds((long long)b * Tmax + u, nb, dev_status))
-        p = parent[(size_t)b * Tmax + u];
+    if (bad_T || u >= T)
+        p = -1;
     par[u] = p;
-    fc[u] = INT_MAX;
-    if (u == 0)
-        fc[kMaxTree] = INT_MAX;
+    for (int s = u; s <= kMaxTree; s += blockDim.x)
+#pragma unroll
+        for (int w = 0; w < kMaskWords; ++w)
+            kids[s][w] = 0u;
     const bool bad_u = !bad_T && u < T && (p < -1 || p >= u);
     const bool bad = __syncthreads_or(bad_T || bad_u);
 
@@ -43,16 +49,23 @@ __global__ void __launch_bounds__(kMaxTree)
             m[v >> 5] |= 1u << (v & 31);
             ++d;
         }
-        atomicMin(&fc[p + 1], u);
+        atomicOr(&kids[p + 1][u >> 5], 1u << (u & 31));
     }
     __syncthreads();
+    // the lowest child above index `after` in set s (-1: none)
+    auto next_kid = [&](int s, int after) {
+        for (int w = (after + 1) >> 5; w < kMaskWords; ++w) {
+            uint32_t bits = kids[s][w];
+            if (w == (after + 1) >> 5)
+                bits &= ~0u << ((after + 1) & 31);
+            if (bits)
+                return w * 32 + __ffs(bits) - 1;
+        }
+        return -1;
+    };
     int ns = -1;
-    if (!bad && u < T)
-        for (int v = u + 1; v < T; ++v)
-            if (par[v] == p) {
-                ns = v;
-                break;
-            }
+    if (!bad && u < T && u + 1 < kMaxTree)
+        ns = next_kid(p + 1, u);
     if (u < Tmax && in_bounds((long long)b * Tmax + u, nb, dev_status)) {
         for (int w = 0; w < W; ++w)
             if (in_bounds(((long long)b * Tmax + u) * W + w, nb * W, dev_status))
@@ -61,7 +74,7 @@ __global__ void __launch_bounds__(kMaxTree)
         next_sibling[(size_t)b * Tmax + u] = ns;
     }
     for (int s = u; s <= Tmax; s += blockDim.x) {
-        int v = (bad || fc[s] == INT_MAX) ? -1 : fc[s];
+        int v = bad ? -1 : next_kid(s, -1);
         if (bad && s == 0)
             v = TSD_TREE_INVALID;
         if (in_bounds((long long)b * (Tmax + 1) + s, (long long)gridDim.x * (Tmax + 1),
