@@ -170,6 +170,9 @@ __device__ float block_max(float v, float *sh)
     return v;
 }
 
+// Block reductions for the walk: warp partials through shared memory, then
+// every thread combines them itself in warp order (the same value on every
+// thread, and two barriers instead of three).
 template <int NT>
 __device__ double block_sum(double v, double *sh)
 {
@@ -179,14 +182,10 @@ __device__ double block_sum(double v, double *sh)
     if (lane == 0)
         sh[warp] = v;
     __syncthreads();
-    if (warp == 0) {
-        v = lane < NW ? sh[lane] : 0.0;
-        v = warp_sum(v);
-        if (lane == 0)
-            sh[0] = v;
-    }
-    __syncthreads();
-    v = sh[0];
+    v = 0.0;
+#pragma unroll
+    for (int w = 0; w < NW; ++w)
+        v += sh[w];
     __syncthreads();
     return v;
 }
@@ -241,18 +240,13 @@ __device__ void block_max_last(float &m, int &last, float *shf, int *shi)
         shi[warp] = last;
     }
     __syncthreads();
-    if (warp == 0) {
-        m = lane < NW ? shf[lane] : -INFINITY;
-        last = lane < NW ? shi[lane] : -1;
-        warp_reduce();
-        if (lane == 0) {
-            shf[0] = m;
-            shi[0] = last;
-        }
+    m = -INFINITY;
+    last = -1;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+        m = fmaxf(m, shf[w]);
+        last = max(last, shi[w]);
     }
-    __syncthreads();
-    m = shf[0];
-    last = shi[0];
     __syncthreads();
 }
 
@@ -275,18 +269,13 @@ __device__ void block_sum_last(double &s, int &last, double *shd, int *shi)
         shi[warp] = last;
     }
     __syncthreads();
-    if (warp == 0) {
-        s = lane < NW ? shd[lane] : 0.0;
-        last = lane < NW ? shi[lane] : -1;
-        warp_reduce();
-        if (lane == 0) {
-            shd[0] = s;
-            shi[0] = last;
-        }
+    s = 0.0;
+    last = -1;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+        s += shd[w];
+        last = max(last, shi[w]);
     }
-    __syncthreads();
-    s = shd[0];
-    last = shi[0];
     __syncthreads();
 }
 
@@ -984,6 +973,16 @@ __global__ void __launch_bounds__(kWalkThreads, CACHED ? 3 : 4)
             return nullptr;
         return walk_stage + set * 2 * kCacheChunk + (is_q ? kCacheChunk : 0);
     };
+    // the team's first root row is staged while the rest is set up (a
+    // sequence that turns out malformed leaves it pending: the next pass
+    // drains it)
+    if (STAGE && team < B) {
+        const float *root = logits + (size_t)team * (Tmax + 1) * V;
+        if (tid == 0)
+            stage_issue(0, root, nullptr);
+        pending0 = true;
+        have_l0 = root;
+    }
     if (CLUSTER) {
         xchg_init(&xs, K);
         cluster_sync_all();
