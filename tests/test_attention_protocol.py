@@ -94,10 +94,11 @@ def _run(NS, NSK, NSV, ntiles, seed, rescale_p=0.3, final_wait="o_ready", merged
     qk_done, pv_done_set = set(), set()
 
     def producer():
-        # K_0 .. K_{NSK-1}, V_0 .. V_{NSV-1}, then K runs NSK tiles ahead of V
+        # K_0 .. K_{NSK-1}, V_0 .. V_{NSV-1}, then V_m, K_{m+L} with L = NSK + NS - NSV
+        lead = NSK + NS - NSV
         i = j = 0
         while i < ntiles or j < ntiles:
-            if i < ntiles and (j >= ntiles or i < NSK or (j >= NSV and i <= j + NSK)):
+            if i < ntiles and (j >= ntiles or i < NSK or (j >= NSV and i <= j - 1 + lead)):
                 s = i % NSK
                 if i >= NSK:
                     if merged:   # QK_{i-NSK} done: s_full[i % NS], NS == NSK
@@ -293,10 +294,11 @@ def _run_keysplit(NSK, NSV, ntiles, seed, rescale_p=0.3):
 
     tma, pipe, pv_done, issued_pv = [], [], set(), set()
 
-    def producer():   # the rows kernels' load order
+    def producer():   # the rows kernels' load order, QK lookahead 2
+        lead = NSK + 2 - NSV
         i = j = 0
         while i < ntiles or j < ntiles:
-            if i < ntiles and (j >= ntiles or i < NSK or (j >= NSV and i <= j + NSK)):
+            if i < ntiles and (j >= ntiles or i < NSK or (j >= NSV and i <= j - 1 + lead)):
                 s = i % NSK
                 if i >= NSK:
                     while not passes(("k_empty", s), i // NSK - 1):

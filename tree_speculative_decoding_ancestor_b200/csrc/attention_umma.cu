@@ -332,14 +332,14 @@ __device__ __forceinline__ void load_kv_tile(uint32_t dst, const CUtensorMap *tm
 }
 
 // TMA producer (one lane).  Load order: K_0 .. K_{NSK-1} and V_0 .. V_{NSV-1}
-// into the empty rings, then K runs NSK tiles ahead of V: ... V_m, K_{m+NSK+1},
-// V_{m+1}, ...  A ring slot is reused once the product that read it is
-// complete; with the MMA order QK_{j+NS} right after PV_j, the V slot of V_m
-// and the K slot of K_{m+NSK+1} free up together (PV_{m-NSV}, then the QK
-// issued after it), so each reload is issued as soon as its slot is free and
-// a K tile has about NSK tile periods to land instead of one (a K ring that
-// only advanced after each V reload waited on the V ring).  Deadlock-free:
-// the product a K wait needs reads V tiles below m only, and the one a V wait
+// into the empty rings, then ... V_m, K_{m+L}, V_{m+1}, ... with L = NSK +
+// LA - NSV, LA the MMA warp's QK lookahead (QK_{j+LA} is issued right after
+// PV_j).  A ring slot is reused once the product that read it is complete,
+// so V_m's slot frees with PV_{m-NSV} and K_{m+L}'s with QK_{m+L-NSK}, the
+// QK issued right after that same PV: each reload is issued as soon as its
+// slot is free, a K tile has about LA tile periods to land, and no V reload
+// queues behind a K reload gated one product later.  Deadlock-free: the
+// product a K wait needs reads V tiles below m only, and the one a V wait
 // needs reads K tiles below the K index already issued.  NS_PROD = 0: the
 // MMA warp commits every product to the rings' own empty barriers as well.
 // NS_PROD = NS (the number of score buffers, equal to the K ring's depth):
@@ -359,12 +359,14 @@ __device__ __forceinline__ void produce_kv(const Setup<Gm> &su, const CUtensorMa
     constexpr int NSK = Gm::NSK, NSV = Gm::NSV, BN = Gm::BN;
     constexpr uint32_t kTile = Gm::kTile;
     static_assert(NS_PROD == 0 || NS_PROD == NSK, "score buffers and K ring in step");
+    // the QK lookahead: NS for the rows kernels, 2 for the key-split kernel
+    constexpr int kLead = NSK + (NS_PROD ? NS_PROD : 2) - NSV;
     ptx::prefetch_tmap(tmK);
     ptx::prefetch_tmap(tmV);
     int i = 0, j = 0;   // next K tile, next V tile
     while (i < ntiles || j < ntiles) {
         const bool take_k =
-            i < ntiles && (j >= ntiles || i < NSK || (j >= NSV && i <= j + NSK));
+            i < ntiles && (j >= ntiles || i < NSK || (j >= NSV && i <= j - 1 + kLead));
         if (take_k) {
             const int s = i % NSK;
             const uint32_t k_free = NS_PROD ? su.bars.s_full(s) : su.bars.k_empty(s);
