@@ -454,3 +454,49 @@ def test_table_exp_accuracy(cuda_device, tmp_path):
     r = subprocess.run([exe, "4e-15"], capture_output=True, text=True)
     assert r.returncode == 0, r.stdout + r.stderr
 
+
+
+def test_verify_greedy_and_stochastic_on_two_streams(cuda_device):
+    # The two verify calls read the same inputs and nothing of each other's:
+    # run side by side on two streams (each with its own workspace, as the
+    # benchmark's step does) they give what they give one after the other.
+    w = gen.random_workload(90, B=24, Tmax=48, V=32000, min_nodes=8, max_children=5,
+                            max_depth=8, token_mode="sample", q_sigma=1.0,
+                            with_attention=False)
+    d = to_dev(w, cuda_device)
+    tree = run_tree(d)
+    B, Tmax = w.B, w.Tmax
+
+    def outs():   # every entry preset, so that the untouched ones compare too
+        return tsd.VerifyResult(
+            torch.full((B, Tmax + 1), -7, dtype=torch.int32, device=cuda_device),
+            torch.full((B, Tmax), -7, dtype=torch.int32, device=cuda_device),
+            torch.full((B,), -7, dtype=torch.int32, device=cuda_device))
+
+    g_ref = tsd.tree_verify_greedy(d["logits"], d["tokens"], d["parent"], d["n_nodes"], tree,
+                                   out=outs())
+    s_ref = tsd.tree_verify_stochastic(d["logits"], w.temperature, d["q_probs"], d["q_row"],
+                                       d["tokens"], d["n_nodes"], tree, d["u_accept"],
+                                       d["u_sample"], out=outs())
+    torch.cuda.synchronize(cuda_device)
+    nb = tsd.verify_workspace_size(B, Tmax, w.V)
+    ws_g = torch.empty(nb, dtype=torch.uint8, device=cuda_device)
+    ws_s = torch.empty(nb, dtype=torch.uint8, device=cuda_device)
+    side = torch.cuda.Stream(device=cuda_device)
+    main = torch.cuda.current_stream(cuda_device)
+    for _ in range(3):
+        g_out, s_out = outs(), outs()
+        side.wait_stream(main)
+        s = tsd.tree_verify_stochastic(d["logits"], w.temperature, d["q_probs"], d["q_row"],
+                                       d["tokens"], d["n_nodes"], tree, d["u_accept"],
+                                       d["u_sample"], out=s_out, workspace=ws_s)
+        with torch.cuda.stream(side):
+            g = tsd.tree_verify_greedy(d["logits"], d["tokens"], d["parent"], d["n_nodes"],
+                                       tree, out=g_out, workspace=ws_g)
+        main.wait_stream(side)
+        torch.cuda.synchronize(cuda_device)
+        for a, b in ((g, g_ref), (s, s_ref)):
+            assert torch.equal(a.n_accepted, b.n_accepted)
+            assert torch.equal(a.out_tokens, b.out_tokens)
+            assert torch.equal(a.out_path, b.out_path)
+    assert _status(cuda_device) == 0
