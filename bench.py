@@ -254,40 +254,34 @@ class Step:
             attn_events[1].record()
         self.run_verify()
 
-    def capture(self):
-        """CUDA graphs of the mask build and of the attention call (plain
-        kernel launches) for every input copy, so that the timed steps
-        measure device work and not the Python and launch overhead in front
-        of each call (which exceeds the kernels' own time on the small
-        workloads).  The verify calls stay eager.  Returns the kernel launches
-        one replay of a copy's two graphs makes."""
+    def capture_steps(self, steps: int, st_ev, att_ev, flush=None):
+        """One CUDA graph of `steps` whole steps, step i on input copy
+        i % n_sets: the mask build, the attention call and the verify
+        call(s), between CUDA events recorded as graph nodes (external
+        events: st_ev[i] around the step, att_ev[i] around the attention
+        call, on the stream the kernels run on), with the L2 flush between
+        steps outside the step's events when `flush` is given.  Replaying it
+        times device work only: on the small workloads the Python and launch
+        work in front of each call took longer than the kernels.  Returns the
+        graph and the kernel launches it holds."""
         torch.cuda.synchronize(self.dev)
-        self.graphs = []
         n0 = self.tsd.launch_count()
-        for d in self.sets:
-            self.d = d
-            g_mask, g_attn = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g_mask):
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for i in range(steps):
+                self.d = self.sets[i % len(self.sets)]
+                if flush is not None:
+                    flush.fill_(float(i))
+                st_ev[i][0].record()
                 self.run_mask()
-            with torch.cuda.graph(g_attn):
+                att_ev[i][0].record()
                 self.run_attention()
-            self.graphs.append((g_mask, g_attn))
+                att_ev[i][1].record()
+                self.run_verify()
+                st_ev[i][1].record()
         torch.cuda.synchronize(self.dev)
         self.d = self.sets[0]
-        return (self.tsd.launch_count() - n0) // len(self.sets)
-
-    def run_graphed(self, attn_events, i: int = 0):
-        g_mask, g_attn = self.graphs[i % len(self.sets)]
-        self.d = self.sets[i % len(self.sets)]
-        g_mask.replay()
-        attn_events[0].record()
-        g_attn.replay()
-        attn_events[1].record()
-        self.run_verify()
-
-    def release(self):
-        self.graphs = []
-        self.d = self.sets[0]
+        return graph, self.tsd.launch_count() - n0
 
     def run_verify(self):
         """The workload's verify calls.  With both modes, the greedy call runs
@@ -512,11 +506,12 @@ def _workload_name(w):
 
 def time_steps(step, w, dev, tsd, steps: int, warmup: int, pg=None, local: int = 0,
                clocks: bool = False) -> dict:
-    """Warm-up, then `steps` timed steps: the mask build and the attention
-    call replayed from CUDA graphs, the verify calls eager; a barrier and a
-    synchronize on both sides of the timed region; CUDA events per step and
-    around the attention call.  The L2 is flushed between steps unless the
-    step already reads more than three times its size."""
+    """Warm-up (eager steps, then one replay of the timed graph), then the
+    `steps` timed steps as one replay of a CUDA graph holding them back to
+    back (Step.capture_steps), with a barrier and a synchronize on both
+    sides; CUDA events per step and around the attention call, recorded by
+    the graph on the launching stream.  The L2 is flushed between steps
+    unless the steps rotate over enough input copies to exceed it."""
     for _ in range(max(3, warmup)):
         step.run()
     torch.cuda.synchronize(dev)
@@ -527,41 +522,33 @@ def time_steps(step, w, dev, tsd, steps: int, warmup: int, pg=None, local: int =
     working = input_bytes(w)
     if nsets == 1:
         flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
-    graph_launches = step.capture()
-    for i in range(max(2, nsets)):
-        step.run_graphed((torch.cuda.Event(), torch.cuda.Event()), i)
+    ev = lambda: torch.cuda.Event(enable_timing=True, external=True)  # noqa: E731
+    att_ev = [(ev(), ev()) for _ in range(steps)]
+    st_ev = [(ev(), ev()) for _ in range(steps)]
+    graph, launches = step.capture_steps(steps, st_ev, att_ev, flush)
+    graph.replay()   # warm-up replay of the same work
     torch.cuda.synchronize(dev)
-    att_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(steps)]
-    st_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-             for _ in range(steps)]
     sampler = _clock_sampler(local) if clocks else None
     if sampler is not None:
         time.sleep(0.3)
     if pg:
         pg.barrier()
     torch.cuda.synchronize(dev)
-    launches0 = tsd.launch_count()
-    for i in range(steps):
-        if flush is not None:
-            flush.fill_(float(i))
-        st_ev[i][0].record()
-        step.run_graphed(att_ev[i], i)
-        st_ev[i][1].record()
+    graph.replay()
     torch.cuda.synchronize(dev)
-    launches = tsd.launch_count() - launches0 + graph_launches * steps
-    step.release()
     if pg:
         pg.barrier()
     clk = _clock_summary(sampler) if sampler is not None else None
     if int(tsd.device_status(dev).item()) != 0:
         raise RuntimeError(f"device status set during the timed steps ({w.name})")
-    return {"step_ms": [a.elapsed_time(b) for a, b in st_ev],
-            "att_ms": [a.elapsed_time(b) for a, b in att_ev],
-            "launches": launches, "clocks": clk,
-            "l2": "flushed between steps (2x L2 write)" if flush is not None
-            else f"inputs larger than L2: {nsets} device copies of the inputs "
-                 f"({working / 1e6:.0f} MB each), step i reads copy i mod {nsets}"}
+    res = {"step_ms": [a.elapsed_time(b) for a, b in st_ev],
+           "att_ms": [a.elapsed_time(b) for a, b in att_ev],
+           "launches": launches, "clocks": clk,
+           "l2": "flushed between steps (2x L2 write)" if flush is not None
+           else f"inputs larger than L2: {nsets} device copies of the inputs "
+                f"({working / 1e6:.0f} MB each), step i reads copy i mod {nsets}"}
+    del graph
+    return res
 
 
 def workload_record(name, w, step, t, peaks, dev, tsd, parity_budget_s: float) -> dict:
