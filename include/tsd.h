@@ -230,6 +230,12 @@ size_t tsd_tree_verify_workspace_size(int B, int Tmax, int V);
  *   n_accepted  [B] int32           out: number of accepted nodes (-1 if the
  *                                   sequence is malformed; nothing else written)
  * Entries beyond n_accepted (+1 for out_tokens) are not written.
+ * Two forms give the same result: when the batch's logits (B (Tmax+1) V
+ * floats) reach 64 MiB, one CTA per sequence walks the matched nodes level
+ * by level and reads only the root row and the matched nodes' rows;
+ * otherwise the argmax of every row with children is taken in parallel,
+ * then the path.  TSD_GREEDY_FORM = "walk" or "rows" forces one (read at
+ * every call).
  * Host errors: TSD_ERR_SHAPE (B < 0 or > 65535, Tmax, V < 1), TSD_ERR_NULL,
  * TSD_ERR_ALIGN (logits), TSD_ERR_WORKSPACE, TSD_ERR_CUDA.
  * Device: TSD_DEV_BAD_TOKEN.

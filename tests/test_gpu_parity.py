@@ -338,6 +338,41 @@ def test_verify_parity(cuda_device, case, exchange, monkeypatch):
     assert _status(cuda_device) == 0
 
 
+@pytest.mark.parametrize("form", ["walk", "rows"])
+@pytest.mark.parametrize("case", VERIFY_CASES + [(40, 6, 48, 700, "match", 1.0)],
+                         ids=[f"s{c[0]}" for c in VERIFY_CASES] + ["s40-all-match"])
+def test_verify_greedy_forms(cuda_device, case, form, monkeypatch):
+    # both greedy forms: the matched-path walk (default) and every row with
+    # children + finalize.  "match": every token is its parent row's argmax,
+    # so siblings share tokens, whole levels match and the deepest path (ties
+    # to the lowest index) decides.
+    monkeypatch.setenv("TSD_GREEDY_FORM", form)
+    seed, B, Tmax, V, mode, temp = case
+    w = gen.random_workload(seed, B=B, Tmax=Tmax, V=V, min_nodes=0, max_children=5,
+                            max_depth=10, token_mode="sample" if mode == "match" else mode,
+                            q_sigma=0.3, temperature=temp, with_attention=False)
+    if mode == "match":
+        for b in range(w.B):
+            for u in range(int(w.n_nodes[b])):
+                w.tokens[b, u] = int(np.argmax(np.asarray(w.logits[b, int(w.parent[b, u]) + 1])))
+    d = to_dev(w, cuda_device)
+    tree = run_tree(d)
+    sentinel = -7
+    out = tsd.VerifyResult(torch.full((B, Tmax + 1), sentinel, dtype=torch.int32,
+                                      device=cuda_device),
+                           torch.full((B, Tmax), sentinel, dtype=torch.int32, device=cuda_device),
+                           torch.full((B,), sentinel, dtype=torch.int32, device=cuda_device))
+    res = tsd.tree_verify_greedy(d["logits"], d["tokens"], d["parent"], d["n_nodes"], tree,
+                                 out=out)
+    ref = oracle.workload_greedy(w)
+    check_greedy(w, res, ref)
+    assert (res.out_tokens.cpu().numpy() == ref["out_tokens"]).all()   # untouched = sentinel
+    assert (res.out_path.cpu().numpy() == ref["out_path"]).all()
+    if mode == "match":   # the whole deepest path is accepted somewhere
+        assert int(res.n_accepted.max()) >= 3
+    assert _status(cuda_device) == 0
+
+
 @pytest.mark.parametrize("exchange", ["cluster", "global"])
 def test_verify_many_seeds_stochastic(cuda_device, exchange, monkeypatch):
     # many small trees with accepted paths of every length; counts excusals
@@ -359,7 +394,9 @@ def test_verify_many_seeds_stochastic(cuda_device, exchange, monkeypatch):
     assert total["excused"] <= 1e-4 * total["decisions"]
 
 
-def test_verify_malformed_inputs(cuda_device):
+@pytest.mark.parametrize("form", ["walk", "rows"])
+def test_verify_malformed_inputs(cuda_device, form, monkeypatch):
+    monkeypatch.setenv("TSD_GREEDY_FORM", form)
     w = gen.random_workload(60, B=3, Tmax=6, V=10, min_nodes=3, ragged=False,
                             with_attention=False)
     d = to_dev(w, cuda_device)

@@ -1,13 +1,20 @@
 // Tree verification from the target model's logits (SpecInfer explainer,
 // section "ツリー検証アルゴリズム").
 //
-// greedy
-//   greedy_rows_kernel      one CTA per logits row whose node has children:
-//                           argmax (lowest index on ties), float4 loads, several
-//                           in flight per thread;
-//   greedy_finalize_kernel  one CTA per sequence: the nodes whose whole root
-//                           path matches, the deepest (lowest index on ties),
-//                           and the argmax of its row (computed here for a leaf).
+// greedy (a node is matched when its token is the argmax of its parent's row;
+// the result is the deepest node whose whole root path is matched, lowest
+// index on ties, and the argmax of that node's row as the bonus token)
+//   greedy_walk_kernel      (batches whose logits exceed 64 MiB) one CTA per
+//                           sequence walks the matched nodes level by level
+//                           from the root, taking the argmax of each visited
+//                           row: it reads the root row and the rows of
+//                           matched nodes only;
+//   greedy_rows_kernel      (smaller batches) one CTA per logits row whose
+//                           node has children: argmax (lowest index on ties),
+//                           float4 loads, several in flight per thread;
+//   greedy_finalize_kernel  one CTA per sequence after it: the nodes whose
+//                           whole root path matches, the deepest, and the
+//                           argmax of its row (computed here for a leaf).
 // stochastic (multi-step speculative sampling)
 //   mss_walk_kernel         one launch.  Each sequence is walked by a team of
 //                           K CTAs, CTA k owning one contiguous chunk of the
@@ -826,6 +833,101 @@ __global__ void __launch_bounds__(kFinThreads)
     }
 }
 
+// One CTA per sequence.  Level by level from the root, for each node of the
+// level (the root, then the nodes whose whole root path matched, ascending
+// index) the block takes the argmax of the node's row and collects the
+// children whose token equals it: the next level.  The last nonempty level
+// holds the deepest fully matched nodes; its lowest index is the terminal,
+// whose row argmax (already taken) is the bonus token.  The same answer as
+// greedy_rows_kernel + greedy_finalize_kernel, from 1 + (matched nodes) rows.
+__global__ void __launch_bounds__(kFinThreads)
+    greedy_walk_kernel(const float *__restrict__ logits, const int32_t *__restrict__ tokens,
+                       const int32_t *__restrict__ parent, const int32_t *__restrict__ n_nodes,
+                       const int32_t *__restrict__ first_child, int Tmax, int V,
+                       int32_t *__restrict__ out_tokens, int32_t *__restrict__ out_path,
+                       int32_t *__restrict__ n_accepted, int32_t *dev_status)
+{
+    constexpr int NW = kFinThreads / 32;
+    __shared__ float shv[NW];
+    __shared__ int shi[NW];
+    __shared__ int s_tok[kMaxTree], s_par[kMaxTree];
+    __shared__ int s_level[2][kMaxTree + 1];   // nodes of the current / next level (-1 = root)
+    __shared__ int s_count[2];
+    const int b = blockIdx.x, u = threadIdx.x;
+    int T;
+    if (!sequence_ok(n_nodes, first_child, b, Tmax, T)) {
+        if (u == 0)
+            n_accepted[b] = -1;
+        return;
+    }
+    bool bad = false;
+    for (int i = u; i < T; i += kFinThreads) {
+        const int tok = tokens[(size_t)b * Tmax + i];
+        s_tok[i] = tok;
+        s_par[i] = parent[(size_t)b * Tmax + i];   // validated by the mask build
+        bad = bad || tok < 0 || tok >= V;
+    }
+    if (__syncthreads_or(bad)) {
+        if (u == 0) {
+            n_accepted[b] = -1;
+            flag(dev_status, TSD_DEV_BAD_TOKEN);
+        }
+        return;
+    }
+    if (u == 0) {
+        s_level[0][0] = -1;
+        s_count[0] = 1;
+    }
+    __syncthreads();
+    int cur = 0, terminal = -1, bonus = 0, depth = 0;
+    for (int level = 0; level <= T; ++level) {   // at most T + 1 levels
+        const int n = s_count[cur];
+        if (n == 0)
+            break;
+        if (u == 0)
+            s_count[cur ^ 1] = 0;
+        // the level's lowest index is the terminal if no deeper level follows
+        int lo = INT_MAX;
+        for (int k = 0; k < n; ++k)
+            lo = min(lo, s_level[cur][k]);
+        for (int k = 0; k < n; ++k) {
+            const int f = s_level[cur][k];
+            const int a = row_argmax<kFinThreads>(
+                logits + ((size_t)b * (Tmax + 1) + (f + 1)) * V, V, shv, shi);   // ends with a barrier
+            if (f == lo) {
+                terminal = f;
+                bonus = a;
+                depth = level;
+            }
+            // the children of f whose token is the argmax, one thread per node
+            // (in any order: the level's minimum is taken above)
+            for (int c = u; c < T; c += kFinThreads)
+                if (s_par[c] == f && s_tok[c] == a) {
+                    const int m = atomicAdd(&s_count[cur ^ 1], 1);
+                    if (in_bounds(m, kMaxTree + 1, dev_status))
+                        s_level[cur ^ 1][m] = c;
+                }
+        }
+        __syncthreads();   // the next level is complete
+        cur ^= 1;
+    }
+    // the terminal's root path, by parent pointers, deepest first
+    if (u == 0) {
+        int v = terminal;
+        for (int pos = depth - 1; pos >= 0 && v >= 0; --pos) {
+            if (in_bounds(pos, Tmax, dev_status)) {
+                out_path[(size_t)b * Tmax + pos] = v;
+                out_tokens[(size_t)b * (Tmax + 1) + pos] = s_tok[v];
+            }
+            v = s_par[v];
+        }
+        if (in_bounds(depth, Tmax + 1, dev_status)) {
+            out_tokens[(size_t)b * (Tmax + 1) + depth] = bonus;
+            n_accepted[b] = depth;
+        }
+    }
+}
+
 // -------------------------------------------------------------- stochastic
 
 // VEC: V % 4 == 0, so every logits / q row is 16-byte aligned (the entry
@@ -1345,6 +1447,28 @@ size_t verify_workspace(int B, int Tmax, int V)
 
 size_t verify_stochastic_scratch() { return kWalkBytes; }
 
+// The greedy form.  The all-rows scan (every row with children, then a
+// finalize pass) reads up to B (Tmax + 1) V floats at HBM speed, in time
+// that grows with the batch; the matched-path walk reads the root row and
+// the matched nodes' rows, one CTA per sequence, in time that does not (a
+// few microseconds a level).  So the walk takes batches whose scan would
+// read at least kGreedyWalkBytes, the scan the smaller ones.  Side by side
+// with the stochastic walk the scan's traffic also lengthens the latter's
+// dependent fetches, which the walk avoids.  TSD_GREEDY_FORM = "walk" or
+// "rows" forces a form (read at every launch).
+constexpr double kGreedyWalkBytes = 64.0 * 1024 * 1024;
+
+bool greedy_all_rows(int B, int Tmax, int V)
+{
+    if (const char *e = std::getenv("TSD_GREEDY_FORM")) {
+        if (std::strcmp(e, "rows") == 0)
+            return true;
+        if (std::strcmp(e, "walk") == 0)
+            return false;
+    }
+    return (double)B * (Tmax + 1) * V * sizeof(float) < kGreedyWalkBytes;
+}
+
 int launch_verify_greedy(const float *logits, const int32_t *tokens, const int32_t *parent,
                          const int32_t *n_nodes, const uint32_t *mask,
                          const int32_t *first_child, int B, int Tmax, int V,
@@ -1353,6 +1477,13 @@ int launch_verify_greedy(const float *logits, const int32_t *tokens, const int32
 {
     if (B == 0)
         return TSD_OK;
+    if (!greedy_all_rows(B, Tmax, V)) {
+        greedy_walk_kernel<<<B, kFinThreads, 0, stream>>>(logits, tokens, parent, n_nodes,
+                                                          first_child, Tmax, V, out_tokens,
+                                                          out_path, n_accepted, dev_status);
+        TSD_LAUNCH_CHECK();
+        return TSD_OK;
+    }
     const VerifyWs w = carve(ws);
     greedy_rows_kernel<<<dim3(Tmax + 1, B), kRowThreads, 0, stream>>>(logits, n_nodes,
                                                                       first_child, Tmax, V,
