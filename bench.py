@@ -99,26 +99,31 @@ def attn_bytes(w) -> int:
 
 def verify_traffic(w, step) -> dict:
     """Algorithmic bytes of the verify calls of one step: every row a
-    verifier must read, once.  Greedy: the logits row of the root and of every
-    node with children (their argmax decides the path), plus the terminal's
-    row when the path ends at a leaf (the bonus token).  Stochastic: the
-    logits rows on the accepted path and the distinct q rows of the children
-    tried there (the children before the accepted one, or all of them where
-    the walk stops); read from the step's own results."""
+    verifier must read, once.  Greedy: the logits rows of the root and of
+    every node whose whole root path matched (each row's argmax decides which
+    children match, the terminal's gives the bonus token; found level by
+    level from the root on the host copy of the inputs) -- what the
+    matched-node walk reads (the all-rows form, for small batches, reads every
+    row with children).  Stochastic: the logits rows on the accepted path and
+    the distinct q rows of the children tried there (the children before the
+    accepted one, or all of them where the walk stops); read from the step's
+    own results."""
     row = w.V * 4
     out = {}
     if "greedy" in w.verify:
-        n = step.g.n_accepted.cpu().tolist()
-        path = step.g.out_path.cpu().tolist()
         rows = 0
         for b in range(w.B):
             T = int(w.n_nodes[b])
             par = w.parent[b, :T].tolist()
-            internal = set(par)            # -1 stands for the root
-            rows += len(internal) if T else 1
-            k = n[b]
-            if k > 0 and path[b][k - 1] not in internal:
-                rows += 1                  # a leaf's row for the bonus token
+            tok = w.tokens[b, :T].tolist()
+            level = [-1]                   # -1 stands for the root
+            while level:
+                rows += len(level)
+                nxt = []
+                for f in level:
+                    a = int(np.argmax(np.asarray(w.logits[b, f + 1])))
+                    nxt += [c for c in range(T) if par[c] == f and tok[c] == a]
+                level = nxt
         out["greedy"] = rows * row
     if "stochastic" in w.verify:
         n = step.s.n_accepted.cpu().tolist()
