@@ -70,10 +70,20 @@ def test_verify_traffic_counts_rows_on_the_path():
     res = lambda n, path: types.SimpleNamespace(  # noqa: E731
         n_accepted=torch.tensor([n], dtype=torch.int32),
         out_path=torch.tensor([path + [-1] * (3 - len(path))], dtype=torch.int32))
-    # greedy: internal rows are the root's and node 0's; path ends at leaf 1
+    # greedy: the rows of the root and of every fully matched node.  Node 0
+    # matches the root row's argmax, node 1 node 0's, node 2 does not: the
+    # root's, node 0's and node 1's rows (node 1's argmax is the bonus token)
+    w.tokens[0] = torch.tensor([3, 5, 1], dtype=torch.int32)
+    w.logits[0].zero_()
+    w.logits[0, 0, 3] = 1.0
+    w.logits[0, 1, 5] = 1.0
+    w.logits[0, 2, 7] = 1.0
     st = types.SimpleNamespace(g=res(2, [0, 1]), s=res(0, []))
     vb = bench.verify_traffic(w, st)
     assert vb["greedy"] == 3 * row
+    w.tokens[0, 0] = 4   # nothing matches: the root's row alone
+    assert bench.verify_traffic(w, st)["greedy"] == 1 * row
+    w.tokens[0, 0] = 3
     # stochastic, nothing accepted: root row + the root children's q row (shared)
     assert vb["stochastic"] == 2 * row
     # stochastic, node 0 then node 1 accepted: root row + q row 0; node 0's row +
