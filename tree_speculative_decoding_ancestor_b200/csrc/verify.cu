@@ -286,8 +286,13 @@ __device__ void block_sum_last(double &s, int &last, double *shd, int *shi)
     __syncthreads();
 }
 
-// Row argmax (lowest index among the maxima); four float4 loads in flight.
-template <int NT>
+// Row argmax (lowest index among the maxima).  Each thread keeps NB float4
+// loads in flight per batch, the last batch predicated (no tail of single
+// loads).  NB = 8 (a 32000-entry row in one batch for 1024 threads) where a
+// row's latency is the cost: the greedy walk and finalize; NB = 4 where many
+// CTAs per SM keep the bytes in flight: the all-rows scan, whose occupancy
+// the extra registers would cut.
+template <int NT, int NB = 8>
 __device__ int row_argmax(const float *__restrict__ row, int V, float *shv, int *shi)
 {
     float bv = -INFINITY;
@@ -295,28 +300,22 @@ __device__ int row_argmax(const float *__restrict__ row, int V, float *shv, int 
     if ((V & 3) == 0) {
         const float4 *r4 = reinterpret_cast<const float4 *>(row);
         const int n4 = V >> 2;
-        int j = threadIdx.x;
-        for (; j + 3 * NT < n4; j += 4 * NT) {
-            float4 x[4];
+        for (int j0 = threadIdx.x; j0 < n4; j0 += NB * NT) {
+            float4 x[NB];
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-                x[k] = __ldg(r4 + j + k * NT);
+            for (int k = 0; k < NB; ++k)
+                if (j0 + k * NT < n4)
+                    x[k] = __ldg(r4 + j0 + k * NT);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int i0 = 4 * (j + k * NT);
+            for (int k = 0; k < NB; ++k) {
+                if (j0 + k * NT >= n4)
+                    break;
+                const int i0 = 4 * (j0 + k * NT);
                 if (better(x[k].x, i0, bv, bi)) { bv = x[k].x; bi = i0; }
                 if (better(x[k].y, i0 + 1, bv, bi)) { bv = x[k].y; bi = i0 + 1; }
                 if (better(x[k].z, i0 + 2, bv, bi)) { bv = x[k].z; bi = i0 + 2; }
                 if (better(x[k].w, i0 + 3, bv, bi)) { bv = x[k].w; bi = i0 + 3; }
             }
-        }
-        for (; j < n4; j += NT) {
-            const float4 x = __ldg(r4 + j);
-            const int i0 = 4 * j;
-            if (better(x.x, i0, bv, bi)) { bv = x.x; bi = i0; }
-            if (better(x.y, i0 + 1, bv, bi)) { bv = x.y; bi = i0 + 1; }
-            if (better(x.z, i0 + 2, bv, bi)) { bv = x.z; bi = i0 + 2; }
-            if (better(x.w, i0 + 3, bv, bi)) { bv = x.w; bi = i0 + 3; }
         }
     } else {
         for (int j = threadIdx.x; j < V; j += NT) {
@@ -743,7 +742,7 @@ __global__ void __launch_bounds__(kRowThreads)
     if (first_child[(size_t)b * (Tmax + 1) + r] < 0)
         return;   // leaf: its argmax is needed only if it ends the path
     const int a =
-        row_argmax<kRowThreads>(logits + ((size_t)b * (Tmax + 1) + r) * V, V, shv, shi);
+        row_argmax<kRowThreads, 4>(logits + ((size_t)b * (Tmax + 1) + r) * V, V, shv, shi);
     if (threadIdx.x == 0)
         argmax_ws[(size_t)b * (Tmax + 1) + r] = a;
 }
