@@ -53,8 +53,11 @@ def main():
                 for k in env:
                     del os.environ[k]
                 del os.environ["TSD_ATTN_SPLITS"]
-        check_greedy(w, tsd.tree_verify_greedy(d["logits"], d["tokens"], d["parent"],
-                                               d["n_nodes"], tree))
+        for form in ("walk", "rows"):   # both greedy forms
+            os.environ["TSD_GREEDY_FORM"] = form
+            check_greedy(w, tsd.tree_verify_greedy(d["logits"], d["tokens"], d["parent"],
+                                                   d["n_nodes"], tree))
+        del os.environ["TSD_GREEDY_FORM"]
         check_stochastic(w, tsd.tree_verify_stochastic(
             d["logits"], w.temperature, d["q_probs"], d["q_row"], d["tokens"], d["n_nodes"],
             tree, d["u_accept"], d["u_sample"]))
