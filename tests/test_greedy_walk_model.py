@@ -116,11 +116,3 @@ def test_the_walk_model_sees_a_wrong_tie_rule():
         n, path, _, _ = _walk(logits[b], tokens[b], parent[b], T, pick=max)
         wrong += path != [int(x) for x in ref["out_path"][b, :n]]
     assert wrong > 0
-
-
-def _root_path(parent, u):
-    out = []
-    while u >= 0:
-        out.append(u)
-        u = int(parent[u])
-    return out
