@@ -833,9 +833,9 @@ __global__ void __launch_bounds__(kFinThreads)
 }
 
 // One CTA per sequence.  Level by level from the root, for each node of the
-// level (the root, then the nodes whose whole root path matched, ascending
-// index) the block takes the argmax of the node's row and collects the
-// children whose token equals it: the next level.  The last nonempty level
+// level (the root, then the nodes whose whole root path matched, in the
+// order they were collected) the block takes the argmax of the node's row
+// and collects the children whose token equals it: the next level.  The last nonempty level
 // holds the deepest fully matched nodes; its lowest index is the terminal,
 // whose row argmax (already taken) is the bonus token.  The same answer as
 // greedy_rows_kernel + greedy_finalize_kernel, from 1 + (matched nodes) rows.
