@@ -8,7 +8,6 @@ workload choice in two spawned processes over `gloo`.
 """
 
 import datetime
-import os
 import socket
 
 import numpy as np

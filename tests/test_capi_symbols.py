@@ -1,7 +1,6 @@
 """The C ABI: every function include/tsd.h declares is exported by
 libtsd.so and bound by the Python layer (CPU only, nothing is launched)."""
 
-import ctypes
 import os
 import re
 import subprocess
