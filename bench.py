@@ -571,6 +571,7 @@ def workload_record(name, w, step, t, peaks, dev, tsd, parity_budget_s: float) -
             "roofline_step": step_roofline(w, step, ms, peaks),
             "kv_cache_gbs": kv_gbs, "kv_cache_frac_of_hbm": kv_gbs / peaks["hbm_gbs"],
             "acceptance": accepted_summary(w, step), "plan": _plan(w, dev, tsd),
+            "verify_plan": _verify_plan(w, tsd),
             "parity": parity_record(w, step, ref), "l2": t["l2"]}
 
 
@@ -579,6 +580,21 @@ def _plan(w, dev, tsd):
         w.B, w.Tmax, w.Hq, w.Hkv, w.D, int(w.k_cache.shape[2]),
         torch.bfloat16 if w.dtype == "bf16" else torch.float32,
         torch.cuda.get_device_properties(dev).multi_processor_count)
+
+
+def _verify_plan(w, tsd) -> dict:
+    """The form of each verify call the workload makes: the greedy one's
+    (walk over matched nodes, or every row with children) and the stochastic
+    walk's grid."""
+    out = {}
+    try:
+        if "greedy" in w.verify:
+            out["greedy"] = tsd.verify_greedy_plan(w.B, w.Tmax, w.V)["form"]
+        if "stochastic" in w.verify:
+            out["stochastic"] = tsd.verify_stochastic_plan(w.B, w.Tmax, w.V)
+    except tsd.TsdError as e:   # informational: never fails the measurement
+        out["error"] = str(e)
+    return out
 
 
 def acceptance_other_proposal(cfg, dev, tsd) -> dict:
@@ -710,7 +726,7 @@ def main():
             "roofline": roof,
             "roofline_step": step_roofline(w, step, statistics.mean(t["step_ms"]), peaks),
             "gpu_launches": t["launches"], "clocks": t["clocks"],
-            "acceptance": acceptance}
+            "acceptance": acceptance, "verify_plan": _verify_plan(w, tsd)}
     if gathered is not None:
         line["gathered_sequences"] = gathered
     line.update(side)

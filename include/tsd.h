@@ -304,6 +304,20 @@ int tsd_tree_verify_stochastic(const float *logits, double temperature, const fl
  */
 int tsd_tree_verify_stochastic_plan(int B, int Tmax, int V, int32_t *plan);
 
+/* Forms of greedy verification, as reported by tsd_tree_verify_greedy_plan. */
+enum tsd_greedy_form {
+    TSD_GREEDY_WALK = 0,     /* one CTA per sequence walks the matched nodes            */
+    TSD_GREEDY_ROWS = 1      /* the argmax of every row with children, then the path    */
+};
+
+/*
+ * The form tsd_tree_verify_greedy takes for these sizes (host only, nothing
+ * is launched; TSD_GREEDY_FORM is read as in the call itself): *form is a
+ * tsd_greedy_form value.
+ * Errors: TSD_ERR_NULL (form), TSD_ERR_SHAPE (B < 1, Tmax out of range, V < 1).
+ */
+int tsd_tree_verify_greedy_plan(int B, int Tmax, int V, int32_t *form);
+
 /*
  * Token-tree construction ("マルチドラフトモデルアプローチ": item 1,
  * expansion-based trees <k_1, ..., k_n> take one SSM's top-k_i tokens at

@@ -96,3 +96,21 @@ def test_forced_split_count(monkeypatch):
     assert p["splits"] == (Lmax + 63) // 64
     monkeypatch.setenv("TSD_ATTN_SPLITS", "4")        # the CUDA-core path: 128 keys at least
     assert tsd.attention_plan(*_sizes("tiny"), SMS)["splits"] == 1
+
+
+def test_greedy_form_follows_the_scan_size(monkeypatch):
+    # the walk over matched nodes for batches whose logits reach 64 MiB (the
+    # 70B-GQA workload: 32 x 65 rows x 32000), the all-rows scan below
+    # (LLaMA-7B: 8 x 21 rows); TSD_GREEDY_FORM forces either
+    monkeypatch.delenv("TSD_GREEDY_FORM", raising=False)
+    assert tsd.verify_greedy_plan(32, 64, 32000)["form"] == "walk"
+    assert tsd.verify_greedy_plan(8, 20, 32000)["form"] == "rows"
+    rows = 64 * 1024 * 1024 // (4 * 32000)          # rows of 64 MiB at V = 32000
+    assert tsd.verify_greedy_plan(1, 127, 32000)["form"] == "rows"   # 128 rows
+    assert tsd.verify_greedy_plan(rows // 128 + 1, 127, 32000)["form"] == "walk"
+    monkeypatch.setenv("TSD_GREEDY_FORM", "walk")
+    assert tsd.verify_greedy_plan(1, 6, 32)["form"] == "walk"
+    monkeypatch.setenv("TSD_GREEDY_FORM", "rows")
+    assert tsd.verify_greedy_plan(32, 64, 32000)["form"] == "rows"
+    with pytest.raises(tsd.TsdError):
+        tsd.verify_greedy_plan(0, 6, 32)

@@ -37,6 +37,7 @@ from .binding import (  # noqa: F401
     tree_verify_greedy,
     tree_verify_stochastic,
     tree_verify_stochastic_noalloc,
+    verify_greedy_plan,
     verify_stochastic_plan,
     verify_workspace_size,
 )

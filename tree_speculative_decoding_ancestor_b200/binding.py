@@ -53,6 +53,7 @@ _SIGNATURES: Dict[str, Tuple[object, list]] = {
     "tsd_tree_verify_stochastic_noalloc": (_I, [_P, ctypes.c_double, _P, _I, _P, _P, _P, _P, _P,
                                                 _P, _P, _I, _I, _I, _P, _P, _P, _P, _P]),
     "tsd_tree_verify_stochastic_plan": (_I, [_I, _I, _I, _P]),
+    "tsd_tree_verify_greedy_plan": (_I, [_I, _I, _I, _P]),
     "tsd_kv_commit": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
     "tsd_tree_attention_paged": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _I, _I, _I, _I,
                                       _I, ctypes.c_float, _I, _P, _P, _SZ, _P, _P]),
@@ -379,6 +380,19 @@ def verify_stochastic_plan(B: int, Tmax: int, V: int) -> Dict[str, int]:
     rc = load_library().tsd_tree_verify_stochastic_plan(B, Tmax, V, ctypes.addressof(plan))
     _check(rc, "tsd_tree_verify_stochastic_plan")
     return {"teams": plan[0], "ctas_per_team": plan[1], "chunk": plan[2], "ctas": plan[3]}
+
+
+GREEDY_FORMS = {0: "walk", 1: "rows"}
+
+
+def verify_greedy_plan(B: int, Tmax: int, V: int) -> Dict[str, str]:
+    """The form tree_verify_greedy takes for these sizes (host only): "walk"
+    (one CTA per sequence over the matched nodes) or "rows" (the argmax of
+    every row with children, then the path)."""
+    form = ctypes.c_int32(-1)
+    rc = load_library().tsd_tree_verify_greedy_plan(B, Tmax, V, ctypes.addressof(form))
+    _check(rc, "tsd_tree_verify_greedy_plan")
+    return {"form": GREEDY_FORMS[form.value]}
 
 
 def tree_verify_stochastic_noalloc(logits: torch.Tensor, temperature: float,

@@ -263,6 +263,16 @@ int tsd_tree_verify_stochastic_plan(int B, int Tmax, int V, int32_t *plan)
     return tsd::verify_stochastic_plan(B, V, plan);
 }
 
+int tsd_tree_verify_greedy_plan(int B, int Tmax, int V, int32_t *form)
+{
+    if (!form)
+        return TSD_ERR_NULL;
+    if (B < 1 || Tmax < 1 || Tmax > TSD_MAX_TREE || V < 1)
+        return TSD_ERR_SHAPE;
+    *form = tsd::greedy_all_rows(B, Tmax, V) ? TSD_GREEDY_ROWS : TSD_GREEDY_WALK;
+    return TSD_OK;
+}
+
 int tsd_kv_commit(void *k_cache, void *v_cache, const int32_t *prefix_len,
                   const int32_t *out_path, const int32_t *n_accepted, int B, int Tmax, int Hkv,
                   int D, int Lmax, int dtype, int32_t *new_prefix_len, int32_t *dev_status,

@@ -191,6 +191,10 @@ int launch_kv_commit(void *k_cache, void *v_cache, const int32_t *prefix_len,
                      const int32_t *out_path, const int32_t *n_accepted, int B, int Tmax, int Hkv,
                      int Lmax, int row_bytes, int32_t *new_prefix, int32_t *dev_status,
                      cudaStream_t stream);
+// true: greedy verification takes the all-rows scan for these sizes (else
+// the walk over matched nodes); reads TSD_GREEDY_FORM.
+bool greedy_all_rows(int B, int Tmax, int V);
+
 int launch_verify_greedy(const float *logits, const int32_t *tokens, const int32_t *parent,
                          const int32_t *n_nodes, const uint32_t *mask,
                          const int32_t *first_child, int B, int Tmax, int V,
