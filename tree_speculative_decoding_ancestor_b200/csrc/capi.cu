@@ -77,7 +77,7 @@ const char *tsd_status_string(int status)
     }
 }
 
-int tsd_version(void) { return 100; }
+int tsd_version(void) { return 101; }
 
 unsigned long long tsd_launch_count(void) { return tsd::g_launches.load(); }
 
